@@ -1,0 +1,437 @@
+#!/usr/bin/env python
+"""Benchmark of the KDA hot path on B200.
+
+Headline (one "step"): one chunkwise prefill call of the KDA recurrence over
+B=1, T=8192, H=32, dk=dv=128, bf16 inputs, fp32 state, 64-token chunks, with
+the per-head RMSNorm and sigmoid output gate (kda_chunk_fwd with gate).
+Reported as whole-job tokens/s (weak scaling: every rank runs its own batch),
+plus TFLOP/s against the dense BF16 tensor peak and the call's HBM roofline.
+A decode sub-measurement runs 1000 consecutive recurrent steps over 256
+sequences x 32 heads (fp32 state, 512 MiB) and reports steps/s and state GB/s
+against HBM.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+N > 1 is launched with torch.distributed.run (one rank per GPU, NCCL).  Rank 0
+prints ONE JSON line.  `--impl reference` times the fp64 CPU oracle (the only
+reference implementation that exists for this method) on rank 0.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "KDA prefill tokens/s (TFLOP/s, % peak); decode steps/s (state GB/s, % HBM)"
+D = 128
+PREFILL = dict(B=1, T=8192, H=32)
+DECODE = dict(Bd=256, H=32, steps=1000, pool=8)
+# algorithmic work per token-head (chunk 64, dk = dv = 128):
+#   bytes: q, k, v, log_alpha, gate in + y out (6 x 256 B bf16) + beta (2 B)
+#   flops: C^2 (3 dk + 2 dv) triangular intra-chunk products + 6 C dk dv state products, per chunk of C
+PREFILL_BYTES_PER_TH = 6 * 256 + 2
+PREFILL_FLOP_PER_TH = 139264
+DECODE_STATE_BYTES_PER_HEAD = 2 * D * D * 4
+DECODE_TOKEN_BYTES_PER_HEAD = 4 * 256 + 2 + 256   # q, k, v, log_alpha in; beta; o out
+WORKLOAD = ("KDA chunkwise prefill, B=1 T=8192 H=32 dk=dv=128, bf16 inputs, fp32 state, chunk 64, "
+            "fused per-head RMSNorm + sigmoid gate, zero initial state")
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return dict(hbm_gbs=float(d["hbm_gbs"]), bf16_tflops=float(d["bf16_tflops"]),
+                    bf16_tflops_sustained=float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                    source="measured")
+    return dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0, source="fallback")
+
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+# --------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples while the GPU is under load."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.proc = None
+        self.lines = []
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(gpu_index), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        rows = []
+        for ln in out.strip().splitlines():
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                rows.append(dict(sm=float(parts[0]), smax=float(parts[1]), reasons=parts[3:8]))
+            except ValueError:
+                continue
+        if not rows:
+            return None
+        smax = max(r["smax"] for r in rows)
+        loaded = [r for r in rows if r["sm"] > 0.3 * smax] or rows
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        seen = set()
+        for r in loaded:
+            for nm, val in zip(names, r["reasons"][1:]):
+                if val.lower().startswith("active"):
+                    seen.add(nm)
+        return dict(sm_mhz=statistics.median(r["sm"] for r in loaded), sm_max_mhz=smax, reasons=sorted(seen),
+                    samples=len(loaded))
+
+
+# -------------------------------------------------------------------- inputs
+
+def prefill_inputs(seed: int):
+    from linear_attention_recurrence_06_b200 import synth
+    B, T, H = PREFILL["B"], PREFILL["T"], PREFILL["H"]
+    tb = synth.tokens(seed, 0, B * T, H, D, D, bf16=True, gate=True)
+    return tb
+
+
+def to_bf16_host(a, torch, pin=True):
+    t = torch.from_numpy(np.ascontiguousarray(a)).to(torch.bfloat16)
+    return t.pin_memory() if pin else t
+
+
+# ----------------------------------------------------------------- our arm
+
+def run_ours(args, peaks):
+    import torch
+    import linear_attention_recurrence_06_b200 as kda
+
+    ws_n, rank, local = dist_env()
+    dist = None
+    if ws_n > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    stream = torch.cuda.current_stream()
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    def max_over_ranks(x: float) -> float:
+        if dist is None:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    B, T, H = PREFILL["B"], PREFILL["T"], PREFILL["H"]
+    tb = prefill_inputs(seed=rank)
+    hq = {n: to_bf16_host(getattr(tb, n).reshape(B, T, H, -1) if n != "beta" else tb.beta.reshape(B, T, H), torch)
+          for n in ("q", "k", "v", "log_alpha", "beta", "g")}
+    dq = {n: t.to(dev) for n, t in hq.items()}
+    out = torch.empty((B, T, H, D), dtype=torch.bfloat16, device=dev)
+    fs = torch.empty((B, H, D, D), dtype=torch.float32, device=dev)
+    _, ws_full = kda.workspace_size(B * T, H, B, T)
+    ws = torch.empty(ws_full, dtype=torch.uint8, device=dev)
+
+    def step():
+        kda.chunk_fwd(dq["q"], dq["k"], dq["v"], dq["log_alpha"], dq["beta"], None, gate=dq["g"], out=out,
+                      final_state=fs, workspace=ws, stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if kda.query_status(ws) != 0:
+        raise RuntimeError("device status word set during warm-up")
+
+    # per-kernel device time (events around each launch, same stream), separate pass
+    kda.profile_enable(True)
+    for _ in range(args.steps):
+        step()
+    torch.cuda.synchronize()
+    prof = kda.profile_read()
+    kda.profile_enable(False)
+    launches_per_step = sum(v[0] for v in prof.values()) / args.steps
+
+    # timed region: clocks sampled over a pre-roll plus the K timed steps
+    sampler = ClockSampler(torch.cuda.current_device()) if rank == 0 else None
+    t_end = time.time() + 1.0
+    while time.time() < t_end:
+        for _ in range(20):
+            step()
+        torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    ms_step = max_over_ranks(e0.elapsed_time(e1) / args.steps)
+
+    # decode sub-measurement: 1000 consecutive steps, state in place
+    dec = run_decode(args, torch, kda, dev, stream, rank, max_over_ranks, barrier)
+    clocks = sampler.stop() if sampler else None
+
+    # end to end through the public API: pinned host inputs -> device -> call -> host output
+    e2e = run_e2e(args, torch, kda, hq, out, fs, ws, stream, max_over_ranks, barrier)
+
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return None
+
+    tokens = ws_n * B * T
+    value = tokens / (ms_step * 1e-3)
+    th = B * T * H
+    bytes_call = PREFILL_BYTES_PER_TH * th
+    achieved_gbs = bytes_call / (ms_step * 1e-3) / 1e9
+    tflops = PREFILL_FLOP_PER_TH * th / (ms_step * 1e-3) / 1e12
+    kernels = {k: dict(launches_per_step=v[0] / args.steps, ms_per_step=v[1] / args.steps) for k, v in prof.items()}
+    tot_k = sum(v["ms_per_step"] for v in kernels.values()) or 1.0
+    for v in kernels.values():
+        v["share"] = v["ms_per_step"] / tot_k
+    dominant = max(kernels, key=lambda k: kernels[k]["ms_per_step"]) if kernels else None
+    roof = dict(bound="hbm", kernel="kda_chunk_fwd (all launches of one call)", achieved=achieved_gbs,
+                peak=peaks["hbm_gbs"], unit="GB/s", frac=achieved_gbs / peaks["hbm_gbs"],
+                traffic=recorded_traffic("kda_chunk_fwd", th), peak_source=peaks["source"],
+                algorithmic_bytes_per_launch=bytes_call, dominant_kernel=dominant)
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": ws_n, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "global_batch": ws_n * B, "seq_len": T, "heads": H,
+                   "parallelism": f"dp{ws_n} (independent sequences per rank, no collective)",
+                   "l2": "inputs larger than L2 (q,k,v,log_alpha,gate,beta = 336 MB per step)"},
+        "prefill_tflops": tflops, "prefill_tensor_frac": tflops / peaks["bf16_tflops_sustained"],
+        "roofline": roof, "kernels": kernels, "decode": dec, "e2e": e2e,
+        "gpu_launches": int(round(launches_per_step * args.steps)),
+        "clocks": clocks,
+    }
+    if ws_n == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(seconds=args.cpu_seconds)
+    return line
+
+
+def run_decode(args, torch, kda, dev, stream, rank, max_over_ranks, barrier):
+    from linear_attention_recurrence_06_b200 import synth
+    Bd, H, nsteps, pool = DECODE["Bd"], DECODE["H"], DECODE["steps"], DECODE["pool"]
+    state = torch.from_numpy(synth.states(100 + rank, Bd, H, D, D)).to(dev)
+    toks = []
+    for p in range(pool):
+        tb = synth.tokens(200 + rank, p * Bd, Bd, H, D, D, bf16=True)
+        toks.append({n: torch.from_numpy(np.ascontiguousarray(getattr(tb, n))).to(torch.bfloat16).to(dev)
+                     for n in ("q", "k", "v", "log_alpha", "beta")})
+    o = torch.empty((Bd, H, D), dtype=torch.bfloat16, device=dev)
+
+    def dstep(i):
+        t = toks[i % pool]
+        kda.decode_step(state, t["q"], t["k"], t["v"], t["log_alpha"], t["beta"], out=o, stream=stream)
+
+    for i in range(3):
+        dstep(i)
+    torch.cuda.synchronize()
+    kda.profile_enable(True)
+    for i in range(10):
+        dstep(i)
+    torch.cuda.synchronize()
+    prof = kda.profile_read()
+    kda.profile_enable(False)
+    kern_ms = prof.get("decode", (10, 0.0))[1] / 10
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for i in range(nsteps):
+        dstep(i)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    ms = max_over_ranks(e0.elapsed_time(e1))
+    steps_s = nsteps / (ms * 1e-3)
+    state_bytes = DECODE_STATE_BYTES_PER_HEAD * Bd * H
+    tok_bytes = DECODE_TOKEN_BYTES_PER_HEAD * Bd * H
+    peaks = load_peaks()
+    gbs = (state_bytes + tok_bytes) * steps_s / 1e9
+    kgbs = (state_bytes + tok_bytes) / (kern_ms * 1e-3) / 1e9 if kern_ms > 0 else None
+    return {"workload": f"KDA decode, {Bd} sequences x {H} heads, fp32 state 128x128 (512 MiB), {nsteps} "
+                        f"consecutive steps, bf16 tokens (pool of {pool} distinct steps)",
+            "value": steps_s, "unit": "steps/s", "ms_per_step": ms / nsteps, "state_gbs": gbs,
+            "hbm_frac": gbs / peaks["hbm_gbs"],
+            "roofline": {"bound": "hbm", "kernel": "decode_step_kernel", "achieved": kgbs, "peak": peaks["hbm_gbs"],
+                         "unit": "GB/s", "frac": (kgbs / peaks["hbm_gbs"]) if kgbs else None,
+                         "traffic": recorded_traffic("decode_step_kernel", Bd * H),
+                         "algorithmic_bytes_per_launch": state_bytes + tok_bytes}}
+
+
+def run_e2e(args, torch, kda, hq, out, fs, ws, stream, max_over_ranks, barrier):
+    B, T, H = PREFILL["B"], PREFILL["T"], PREFILL["H"]
+    dq = {n: torch.empty_like(t, device=out.device) for n, t in hq.items()}
+    hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in hq.values())
+    d2h = hout.numel() * hout.element_size()
+
+    def estep():
+        for n in hq:
+            dq[n].copy_(hq[n], non_blocking=True)
+        kda.chunk_fwd(dq["q"], dq["k"], dq["v"], dq["log_alpha"], dq["beta"], None, gate=dq["g"], out=out,
+                      final_state=fs, workspace=ws, stream=stream)
+        hout.copy_(out, non_blocking=True)
+
+    for _ in range(2):
+        estep()
+    torch.cuda.synchronize()
+    n = max(3, min(args.steps, 10))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(n):
+        estep()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    ms = max_over_ranks(e0.elapsed_time(e1) / n)
+    ws_n = int(os.environ.get("WORLD_SIZE", "1"))
+    return {"value": ws_n * B * T / (ms * 1e-3), "unit": "tokens/s", "ms_per_step": ms,
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+
+def recorded_traffic(kernel: str, units: int):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on
+    the current kernel sources (else None)."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    try:
+        rec = json.load(open(p)).get(kernel)
+    except Exception:
+        return None
+    if not rec or rec.get("sources_sha256") != sources_sha256():
+        return None
+    return rec["dram_bytes_per_unit"] * units
+
+
+def sources_sha256() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "linear_attention_recurrence_06_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        if f.endswith((".cu", ".cuh", ".h")):
+            h.update(open(os.path.join(csrc, f), "rb").read())
+    return h.hexdigest()
+
+
+# ------------------------------------------------------------- CPU baseline
+
+def oracle_sample_rate(n_tokens: int, heads: int, threads: int = 0):
+    """Runs the fp64 oracle (recurrence + gate-norm) on the first n_tokens of
+    the prefill workload for `heads` heads; returns (seconds, threads used)."""
+    import oracle
+    from linear_attention_recurrence_06_b200 import synth
+    H = PREFILL["H"]
+    tb = synth.tokens(0, 0, n_tokens, H, D, D, bf16=True, gate=True)
+    t0 = time.perf_counter()
+    o, _, nt = oracle.kda_recurrent(tb.q, tb.k, tb.v, tb.log_alpha, tb.beta, heads=(0, heads), n_threads=threads,
+                                    return_threads=True)
+    oracle.gate_norm(o[:, :heads], tb.g[:, :heads], None, 1e-6)
+    return time.perf_counter() - t0, nt
+
+
+def cpu_baseline(seconds: float = 10.0):
+    import oracle
+    H = PREFILL["H"]
+    cores = oracle.available_cores()
+    probe_tokens = 64
+    dt, _ = oracle_sample_rate(probe_tokens, H)
+    n_tok = int(min(PREFILL["T"], max(probe_tokens, probe_tokens * seconds / max(dt, 1e-6))))
+    dt, nt = oracle_sample_rate(n_tok, H)
+    return {"value": n_tok / dt, "unit": "tokens/s", "cores": nt, "kind": "oracle",
+            "sample": f"first {n_tok} of {PREFILL['T']} tokens, all {H} heads, fp64 recurrence + gate-norm, "
+                      f"{dt:.1f} s on {nt} threads ({cores} cores available)"}
+
+
+# -------------------------------------------------------- reference arm (oracle)
+
+def run_reference(args):
+    ws_n, rank, _ = dist_env()
+    if rank != 0:
+        return None
+    import oracle
+    H = PREFILL["H"]
+    n_tok = args.ref_tokens
+    for _ in range(args.warmup):
+        oracle_sample_rate(n_tok, H)
+    times, nt = [], 1
+    for _ in range(args.steps):
+        dt, nt = oracle_sample_rate(n_tok, H)
+        times.append(dt)
+    ms = 1e3 * sum(times) / len(times)
+    value = n_tok / (ms * 1e-3)
+    return {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": ws_n, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+            "config": {"workload": WORKLOAD, "global_batch": 1, "seq_len": PREFILL["T"], "heads": H,
+                       "parallelism": "host threads over (sequence, head)", "l2": "n/a (CPU)"},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": nt, "kind": "oracle",
+                             "sample": f"each step: first {n_tok} of {PREFILL['T']} tokens, all {H} heads"},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--ref-tokens", type=int, default=256)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    peaks = load_peaks()
+    line = run_reference(args) if args.impl == "reference" else run_ours(args, peaks)
+    if line is not None:
+        print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,192 @@
+/*
+ * kda.h -- C ABI of libkda, a B200 (sm_100a) library for the Kimi Delta
+ * Attention (KDA) gated delta-rule recurrence.
+ *
+ * The operation (sources: the K3 article summaries on the xhh.club tag page,
+ * items "KDA recurrence form", "chunkwise parallel algorithm" and "3:1
+ * hybrid"; section 6 of the nlpx.cn K3 paper walkthrough).  Each head keeps a
+ * dk x dv fp32 state S (row = key channel).  For every token t of a sequence:
+ *
+ *     l_t = max(log_alpha_t, -5)                     per key channel
+ *     S_t = (I - beta_t k_t k_t^T) Diag(exp(l_t)) S_{t-1} + beta_t k_t v_t^T
+ *     o_t = scale * S_t^T q_t
+ *
+ * optionally followed by the per-head RMSNorm and full-rank sigmoid gate
+ *     y_t = o_t / sqrt(mean_j o_tj^2 + eps) * w * sigmoid(g_t).
+ * Prefill runs the chunkwise form (64-token chunks: matrix products inside a
+ * chunk, a recurrence between chunks); decode runs the recurrent form.
+ *
+ * Conventions for every entry point:
+ *  - Pointers are DEVICE pointers owned by the caller, unless stated.  The
+ *    library never allocates, frees or keeps them past the call.
+ *  - Element layout is token-major, head-minor: [B, T, H, d] (contiguous).
+ *    beta is [B, T, H].  States are fp32 [N, H, dk, dv], row = key channel.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *    stream).  Every call is asynchronous on that stream and never
+ *    synchronises, except kda_query_status.
+ *  - Arguments are checked on the host before any launch; a rejected call
+ *    launches nothing and returns a negative kda_status.  A failed launch
+ *    returns KDA_ERR_CUDA (cudaGetLastError is cleared into the return code).
+ *    Errors detected on the device (a bounded wait that expired, cu_seqlens
+ *    that contradict T or max_seqlen) are recorded in a status word inside
+ *    the workspace and read back with kda_query_status.
+ *  - Supported shapes: dk = dv = 128.  Supported dtypes: inputs KDA_F32 or
+ *    KDA_BF16 (all of q, k, v, log_alpha, beta, gate share in_dtype);
+ *    outputs KDA_F32 or KDA_BF16.  Every pointer must be 16-byte aligned.
+ *  - Outputs must not alias inputs, except where stated (in-place states).
+ */
+#ifndef KDA_H_
+#define KDA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define KDA_API __attribute__((visibility("default")))
+#else
+#define KDA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    KDA_OK = 0,
+    KDA_ERR_INVALID_ARG = -1, /* null pointer, bad size, bad dtype */
+    KDA_ERR_UNSUPPORTED = -2, /* shape outside what the kernels implement */
+    KDA_ERR_MISALIGNED = -3,  /* a pointer is not 16-byte aligned */
+    KDA_ERR_WORKSPACE = -4,   /* workspace missing or smaller than required */
+    KDA_ERR_CUDA = -5,        /* a CUDA runtime call or launch failed */
+    KDA_ERR_TIMEOUT = -6,     /* device: a bounded wait gave up */
+    KDA_ERR_DEVICE_ARG = -7   /* device: cu_seqlens inconsistent with T / max_seqlen */
+} kda_status;
+
+typedef enum { KDA_F32 = 0, KDA_BF16 = 1 } kda_dtype;
+
+/* Human-readable name of a kda_status value (static string, never NULL). */
+KDA_API const char* kda_status_string(int status);
+
+/* Library ABI version (major * 10000 + minor * 100 + patch). */
+KDA_API int kda_version(void);
+
+/*
+ * kda_chunk_fwd_workspace_size -- bytes of device workspace kda_chunk_fwd needs.
+ *
+ *   T, H, dk, dv   as for kda_chunk_fwd (T = tokens per sequence for fixed
+ *                  length, total packed tokens for varlen)
+ *   n_seqs         number of sequences N (B for fixed length)
+ *   max_seqlen     longest sequence (T for fixed length)
+ *   bytes_min      out: the smallest workspace accepted (one 64-token chunk
+ *                  of every sequence per pass)
+ *   bytes_full     out: the workspace that lets one pass cover every chunk
+ *                  of every sequence (fewest launches)
+ * Any size in [bytes_min, inf) works; larger workspaces need fewer passes.
+ */
+KDA_API kda_status kda_chunk_fwd_workspace_size(int64_t T, int H, int dk, int dv, int n_seqs,
+                                        int64_t max_seqlen, size_t* bytes_min,
+                                        size_t* bytes_full);
+
+/*
+ * kda_chunk_fwd -- chunkwise prefill / training forward of the KDA recurrence.
+ * Defined by the "chunkwise parallel algorithm" item of the K3 article
+ * summaries (xhh.club tag page): 64-token chunks, state recurrence between
+ * chunks, matrix products inside a chunk, per-step log-decay bounded below by
+ * -5, 16-token diagonal tiles in BF16 matrix multiplies.
+ *
+ *   q, k, log_alpha  [B, T, H, dk]   in_dtype
+ *   v                [B, T, H, dv]   in_dtype
+ *   beta             [B, T, H]       in_dtype, values in [0, 1]
+ *   init_state       [N, H, dk, dv]  fp32, NULL = zero state
+ *   o                [B, T, H, dv]   out_dtype: o, or y when gate != NULL
+ *   final_state      [N, H, dk, dv]  fp32, NULL = not returned.  May alias
+ *                                    init_state (updated in place).
+ *   B, T             batch and tokens per sequence; for varlen B = 1 and T
+ *                    = total packed tokens
+ *   H, dk, dv        heads and head dims (dk = dv = 128)
+ *   cu_seqlens       device int32 [n_seqs + 1] (cu[0] = 0, non-decreasing,
+ *                    cu[n_seqs] = T), or NULL for B fixed-length sequences
+ *   n_seqs           number of sequences when cu_seqlens != NULL (else B)
+ *   max_seqlen       host upper bound on any sequence length (T when
+ *                    cu_seqlens == NULL); lengths above it are a device error
+ *   scale            output scale (1.0 for the plain recurrence)
+ *   gate             [B, T, H, dv] in_dtype, or NULL: when given, the per-head
+ *                    RMSNorm (over dv) and sigmoid gate are applied and y is
+ *                    written to o
+ *   norm_weight      [dv] fp32 RMSNorm weight shared by heads, NULL = ones
+ *   eps              RMSNorm epsilon
+ *   workspace        device buffer of workspace_bytes >=
+ *                    kda_chunk_fwd_workspace_size(...).bytes_min, 256-byte
+ *                    aligned.  Holds the per-chunk intermediates and the
+ *                    device status word; its contents on entry are ignored.
+ *   stream           cudaStream_t as void*
+ * Zero-length sequences are allowed (final state = initial state).
+ */
+KDA_API kda_status kda_chunk_fwd(const void* q, const void* k, const void* v, const void* log_alpha,
+                         const void* beta, const float* init_state, void* o,
+                         float* final_state, int B, int64_t T, int H, int dk, int dv,
+                         const int32_t* cu_seqlens, int n_seqs, int64_t max_seqlen,
+                         kda_dtype in_dtype, kda_dtype out_dtype, float scale,
+                         const void* gate, const float* norm_weight, float eps,
+                         void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * kda_decode_step -- one recurrent step for Bd independent sequences
+ * ("decode uses the recurrent form", chunkwise-algorithm item of the K3
+ * article summaries).  The state is read once and written once, in place.
+ *
+ *   state        [Bd, H, dk, dv] fp32, updated in place
+ *   q, k, log_alpha [Bd, H, dk]; v [Bd, H, dv]; beta [Bd, H]   in_dtype
+ *   o            [Bd, H, dv] out_dtype (y when gate != NULL)
+ *   gate         [Bd, H, dv] in_dtype or NULL; norm_weight [dv] fp32 or NULL
+ */
+KDA_API kda_status kda_decode_step(float* state, const void* q, const void* k, const void* v,
+                           const void* log_alpha, const void* beta, void* o, int Bd, int H,
+                           int dk, int dv, kda_dtype in_dtype, kda_dtype out_dtype,
+                           float scale, const void* gate, const float* norm_weight,
+                           float eps, void* stream);
+
+/*
+ * kda_gate_norm -- per-head RMSNorm over dv followed by the full-rank sigmoid
+ * output gate ("KDA recurrence form" and "3:1 hybrid" items of the K3
+ * article summaries):  y = o / sqrt(mean(o^2) + eps) * w * sigmoid(g).
+ *
+ *   o      [rows, dv] in_dtype (rows = B*T*H)
+ *   gate   [rows, dv] in_dtype
+ *   norm_weight [dv] fp32 or NULL (ones)
+ *   y      [rows, dv] out_dtype; may alias o exactly (in place)
+ */
+KDA_API kda_status kda_gate_norm(const void* o, const void* gate, const float* norm_weight, float eps,
+                         void* y, int64_t rows, int dv, kda_dtype in_dtype,
+                         kda_dtype out_dtype, void* stream);
+
+/*
+ * kda_query_status -- synchronises `stream`, reads the device status word of
+ * a kda_chunk_fwd workspace, clears it and returns it (KDA_OK when no device
+ * error was recorded).  This is the only call that blocks the host.
+ */
+KDA_API kda_status kda_query_status(void* workspace, void* stream);
+
+/*
+ * Per-kernel device timing (a measurement aid, off by default).
+ * kda_profile_enable(1) makes every later launch of this library bracket each
+ * of its kernels with CUDA events on the launch stream.  kda_profile_read
+ * synchronises on those events, writes one entry per kernel kind that ran
+ * (name, number of launches, summed device milliseconds) into out[0 ..
+ * max_entries), stores the count in *n_entries and resets the counters.
+ * Host-side only; not thread-safe.
+ */
+typedef struct {
+    char name[16];
+    int launches;
+    double ms;
+} kda_kernel_time;
+
+KDA_API kda_status kda_profile_enable(int on);
+KDA_API kda_status kda_profile_read(kda_kernel_time* out, int max_entries, int* n_entries);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KDA_H_ */

@@ -1,0 +1,209 @@
+// kda_decode.cu -- recurrent decode step and the per-head RMSNorm + sigmoid
+// output gate.  Both are HBM-bound: decode streams each head's fp32 state
+// once in and once out; gate-norm streams o and g once.
+//
+// Recurrent form (K3 article summaries, xhh.club tag page, items "KDA
+// recurrence form" and "chunkwise parallel algorithm": decode uses the
+// recurrence).  Per head, with S' = Diag(alpha) S:
+//     u = beta (v - S'^T k);   S_new = S' + k u^T;   o = scale * S_new^T q
+// and o = scale * (S'^T q + (k . q) u), so both dot products over the key
+// channels come from ONE pass over S' and the state is read and written once.
+#include "kda_sm100.cuh"
+
+namespace kda {
+
+// One CTA = one (sequence, head) state [128 x 128] fp32 = 64 KiB.
+// 256 threads = 8 warps; warp w owns value columns [16w, 16w + 16).
+// Lane l: row phase r0 = l / 4 (0..7) and column quad cq = l % 4, so one warp
+// load instruction covers 8 rows x 64 contiguous bytes.  Thread holds rows
+// r0 + 8i (i = 0..15) x 4 columns = 64 fp32 registers.
+template <bool IN_BF16, bool OUT_BF16, bool GATE>
+__global__ void __launch_bounds__(256, 2)
+decode_step_kernel(float* __restrict__ state, const void* __restrict__ q, const void* __restrict__ k,
+                   const void* __restrict__ v, const void* __restrict__ log_alpha,
+                   const void* __restrict__ beta, void* __restrict__ o, const void* __restrict__ gate,
+                   const float* __restrict__ norm_w, float scale, float eps) {
+    constexpr int D = 128;
+    const int bh = blockIdx.x;  // sequence * H + head
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int r0 = lane >> 2, cq = lane & 3;
+    const int col = warp * 16 + cq * 4;
+
+    __shared__ float s_k[D], s_q[D], s_alpha[D];
+    __shared__ float s_ss[8];
+
+    float* S = state + (size_t)bh * D * D;
+    float4 st[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i)
+        st[i] = __ldcs(reinterpret_cast<const float4*>(S + (size_t)(r0 + 8 * i) * D + col));
+
+    if (tid < D) {
+        const size_t idx = (size_t)bh * D + tid;
+        s_k[tid] = ld_in<IN_BF16>(k, idx);
+        s_q[tid] = ld_in<IN_BF16>(q, idx);
+        s_alpha[tid] = __expf(fmaxf(ld_in<IN_BF16>(log_alpha, idx), LOG_ALPHA_FLOOR));
+    }
+    const float b = ld_in<IN_BF16>(beta, (size_t)bh);
+    float vv[4];
+#pragma unroll
+    for (int c = 0; c < 4; ++c) vv[c] = ld_in<IN_BF16>(v, (size_t)bh * D + col + c);
+    __syncthreads();
+
+    // k . q (every warp computes it; 4 products per lane + butterfly)
+    float kq = 0.f;
+#pragma unroll
+    for (int m = 0; m < 4; ++m) kq += s_k[lane + 32 * m] * s_q[lane + 32 * m];
+#pragma unroll
+    for (int m = 16; m >= 1; m >>= 1) kq += __shfl_xor_sync(0xffffffffu, kq, m);
+
+    // decay rows, partial S'^T k and S'^T q over this thread's 16 rows
+    float sk[4] = {0.f, 0.f, 0.f, 0.f}, sq[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        const int r = r0 + 8 * i;
+        const float a = s_alpha[r], kr = s_k[r], qr = s_q[r];
+        st[i].x *= a; st[i].y *= a; st[i].z *= a; st[i].w *= a;
+        sk[0] += st[i].x * kr; sk[1] += st[i].y * kr; sk[2] += st[i].z * kr; sk[3] += st[i].w * kr;
+        sq[0] += st[i].x * qr; sq[1] += st[i].y * qr; sq[2] += st[i].z * qr; sq[3] += st[i].w * qr;
+    }
+    // reduce over the 8 row phases (lanes that share cq)
+#pragma unroll
+    for (int m = 4; m <= 16; m <<= 1) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            sk[c] += __shfl_xor_sync(0xffffffffu, sk[c], m);
+            sq[c] += __shfl_xor_sync(0xffffffffu, sq[c], m);
+        }
+    }
+    float u[4], oc[4];
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+        u[c] = b * (vv[c] - sk[c]);
+        oc[c] = scale * (sq[c] + kq * u[c]);
+    }
+    // S_new = S' + k u^T, written back once
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        const float kr = s_k[r0 + 8 * i];
+        st[i].x += kr * u[0]; st[i].y += kr * u[1]; st[i].z += kr * u[2]; st[i].w += kr * u[3];
+        __stcs(reinterpret_cast<float4*>(S + (size_t)(r0 + 8 * i) * D + col), st[i]);
+    }
+
+    if constexpr (GATE) {
+        // per-head RMSNorm over the 128 value channels, then weight and gate
+        float ss = oc[0] * oc[0] + oc[1] * oc[1] + oc[2] * oc[2] + oc[3] * oc[3];
+        ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+        ss += __shfl_xor_sync(0xffffffffu, ss, 2);
+        if (lane == 0) s_ss[warp] = ss;
+        __syncthreads();
+        float tot = 0.f;
+#pragma unroll
+        for (int w = 0; w < 8; ++w) tot += s_ss[w];
+        const float inv = rsqrtf(tot * (1.0f / D) + eps);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            const float gg = ld_in<IN_BF16>(gate, (size_t)bh * D + col + c);
+            const float wc = norm_w ? __ldg(norm_w + col + c) : 1.0f;
+            oc[c] = oc[c] * inv * wc / (1.0f + __expf(-gg));
+        }
+    }
+    if (r0 == 0) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c) st_out<OUT_BF16>(o, (size_t)bh * D + col + c, oc[c]);
+    }
+}
+
+// y = o / sqrt(mean(o^2) + eps) * w * sigmoid(g) over rows of dv = 128.
+// One warp per row, 4 consecutive channels per lane; grid-stride over rows.
+// In place (y == o) is safe: a warp reads its whole row before it writes.
+template <bool O_BF16, bool G_BF16, bool OUT_BF16>
+__global__ void __launch_bounds__(256)
+gate_norm_kernel(const void* o, const void* __restrict__ g, const float* __restrict__ norm_w, float eps,
+                 void* y, int64_t rows) {
+    constexpr int D = 128;
+    const int lane = threadIdx.x & 31;
+    const int64_t warps_total = (int64_t)gridDim.x * (blockDim.x >> 5);
+    float w4[4];
+#pragma unroll
+    for (int c = 0; c < 4; ++c) w4[c] = norm_w ? __ldg(norm_w + lane * 4 + c) : 1.0f;
+    for (int64_t row = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); row < rows;
+         row += warps_total) {
+        const size_t base = (size_t)row * D + lane * 4;
+        float ov[4], gv[4];
+        if constexpr (O_BF16) {
+            const uint2 ob = *reinterpret_cast<const uint2*>(reinterpret_cast<const uint16_t*>(o) + base);
+            ov[0] = __uint_as_float(ob.x << 16); ov[1] = __uint_as_float(ob.x & 0xFFFF0000u);
+            ov[2] = __uint_as_float(ob.y << 16); ov[3] = __uint_as_float(ob.y & 0xFFFF0000u);
+        } else {
+            const float4 of = *reinterpret_cast<const float4*>(reinterpret_cast<const float*>(o) + base);
+            ov[0] = of.x; ov[1] = of.y; ov[2] = of.z; ov[3] = of.w;
+        }
+        if constexpr (G_BF16) {
+            const uint2 gb = __ldg(reinterpret_cast<const uint2*>(reinterpret_cast<const uint16_t*>(g) + base));
+            gv[0] = __uint_as_float(gb.x << 16); gv[1] = __uint_as_float(gb.x & 0xFFFF0000u);
+            gv[2] = __uint_as_float(gb.y << 16); gv[3] = __uint_as_float(gb.y & 0xFFFF0000u);
+        } else {
+            const float4 gf = __ldg(reinterpret_cast<const float4*>(reinterpret_cast<const float*>(g) + base));
+            gv[0] = gf.x; gv[1] = gf.y; gv[2] = gf.z; gv[3] = gf.w;
+        }
+        float ss = ov[0] * ov[0] + ov[1] * ov[1] + ov[2] * ov[2] + ov[3] * ov[3];
+#pragma unroll
+        for (int m = 16; m >= 1; m >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, m);
+        const float inv = rsqrtf(ss * (1.0f / D) + eps);
+        float yv[4];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) yv[c] = ov[c] * inv * w4[c] / (1.0f + __expf(-gv[c]));
+        if constexpr (OUT_BF16) {
+            uint2 yb;
+            yb.x = pack_bf16x2(yv[0], yv[1]);
+            yb.y = pack_bf16x2(yv[2], yv[3]);
+            *reinterpret_cast<uint2*>(reinterpret_cast<uint16_t*>(y) + base) = yb;
+        } else {
+            *reinterpret_cast<float4*>(reinterpret_cast<float*>(y) + base) = make_float4(yv[0], yv[1], yv[2], yv[3]);
+        }
+    }
+}
+
+// ------------------------------------------------------------ launchers --
+
+cudaError_t launch_decode_step(float* state, const void* q, const void* k, const void* v,
+                               const void* log_alpha, const void* beta, void* o, int Bd, int H,
+                               bool in_bf16, bool out_bf16, float scale, const void* gate,
+                               const float* norm_w, float eps, cudaStream_t stream) {
+    const dim3 grid((unsigned)((int64_t)Bd * H)), block(256);
+#define KDA_DEC(IB, OB, G)                                                                              \
+    decode_step_kernel<IB, OB, G><<<grid, block, 0, stream>>>(state, q, k, v, log_alpha, beta, o, gate, \
+                                                              norm_w, scale, eps)
+    const bool g = gate != nullptr;
+    if (in_bf16) {
+        if (out_bf16) { if (g) KDA_DEC(true, true, true); else KDA_DEC(true, true, false); }
+        else          { if (g) KDA_DEC(true, false, true); else KDA_DEC(true, false, false); }
+    } else {
+        if (out_bf16) { if (g) KDA_DEC(false, true, true); else KDA_DEC(false, true, false); }
+        else          { if (g) KDA_DEC(false, false, true); else KDA_DEC(false, false, false); }
+    }
+#undef KDA_DEC
+    return cudaGetLastError();
+}
+
+cudaError_t launch_gate_norm(const void* o, const void* g, const float* norm_w, float eps, void* y,
+                             int64_t rows, bool o_bf16, bool g_bf16, bool out_bf16, int num_sms,
+                             cudaStream_t stream) {
+    const int64_t blocks_needed = (rows + 7) / 8;
+    const int64_t cap = (int64_t)num_sms * 8;
+    const dim3 grid((unsigned)(blocks_needed < cap ? blocks_needed : cap)), block(256);
+    if (rows == 0) return cudaSuccess;
+#define KDA_GN(OB, GB, YB) gate_norm_kernel<OB, GB, YB><<<grid, block, 0, stream>>>(o, g, norm_w, eps, y, rows)
+    if (o_bf16) {
+        if (g_bf16) { if (out_bf16) KDA_GN(true, true, true); else KDA_GN(true, true, false); }
+        else        { if (out_bf16) KDA_GN(true, false, true); else KDA_GN(true, false, false); }
+    } else {
+        if (g_bf16) { if (out_bf16) KDA_GN(false, true, true); else KDA_GN(false, true, false); }
+        else        { if (out_bf16) KDA_GN(false, false, true); else KDA_GN(false, false, false); }
+    }
+#undef KDA_GN
+    return cudaGetLastError();
+}
+
+}  // namespace kda

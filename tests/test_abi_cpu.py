@@ -1,0 +1,108 @@
+"""The C-ABI library loads without a GPU, exports every entry point that
+include/kda.h declares, and rejects bad arguments on the host before any
+launch (these calls never reach CUDA)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import linear_attention_recurrence_06_b200 as kda
+from linear_attention_recurrence_06_b200 import build as kbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "kda.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    kbuild.build()
+    return kda.load_library()
+
+
+def declared_symbols():
+    txt = open(HEADER).read()
+    return sorted(set(re.findall(r"KDA_API\s+[\w\s\*]+?\b(kda_\w+)\s*\(", txt)))
+
+
+def test_header_declares_the_entry_points():
+    syms = declared_symbols()
+    for s in ("kda_chunk_fwd", "kda_decode_step", "kda_gate_norm", "kda_chunk_fwd_workspace_size",
+              "kda_query_status", "kda_status_string", "kda_version"):
+        assert s in syms
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for s in declared_symbols():
+        assert hasattr(lib, s), s
+
+
+def test_status_strings(lib):
+    for st in range(0, -8, -1):
+        assert lib.kda_status_string(st).decode().startswith("KDA_")
+    assert lib.kda_version() >= 100
+
+
+def test_workspace_size(lib):
+    lo, hi = kda.workspace_size(8192, 32, 1, 8192)
+    assert 0 < lo <= hi
+    # 128 chunks of one sequence
+    per_slot = 32768 + 16384 + 32768 + 16384 + 512
+    assert hi - lo == 127 * 32 * per_slot
+    lo2, hi2 = kda.workspace_size(100, 2, 3, 50)
+    assert hi2 >= lo2
+    with pytest.raises(kda.KdaError):
+        kda.workspace_size(100, 2, 3, 50, dk=64)
+
+
+FAKE = 0x10000  # never dereferenced: every call below is rejected on the host
+
+
+def _chunk(lib, **over):
+    args = dict(q=FAKE, k=FAKE, v=FAKE, la=FAKE, beta=FAKE, s0=None, o=FAKE, fs=None, B=1, T=128, H=2, dk=128,
+                dv=128, cu=None, N=1, maxlen=128, idt=1, odt=1, scale=1.0, gate=None, w=None, eps=1e-6,
+                ws=FAKE, wsb=1 << 40, stream=None)
+    args.update(over)
+    a = args
+    return lib.kda_chunk_fwd(a["q"], a["k"], a["v"], a["la"], a["beta"], a["s0"], a["o"], a["fs"], a["B"], a["T"],
+                             a["H"], a["dk"], a["dv"], a["cu"], a["N"], a["maxlen"], a["idt"], a["odt"], a["scale"],
+                             a["gate"], a["w"], a["eps"], a["ws"], a["wsb"], a["stream"])
+
+
+def test_chunk_fwd_host_validation(lib):
+    assert _chunk(lib, q=None) == -1
+    assert _chunk(lib, o=None) == -1
+    assert _chunk(lib, H=0) == -1
+    assert _chunk(lib, idt=7) == -1
+    assert _chunk(lib, dk=64) == -2
+    assert _chunk(lib, dv=256) == -2
+    assert _chunk(lib, k=FAKE + 8) == -3
+    assert _chunk(lib, ws=FAKE + 16) == -3      # workspace needs 256-byte alignment
+    assert _chunk(lib, ws=None) == -4
+    assert _chunk(lib, wsb=1024) == -4
+    assert _chunk(lib, cu=FAKE, B=2, N=2) == -1  # varlen needs B = 1
+    assert _chunk(lib, cu=FAKE, N=0) == -1
+    assert _chunk(lib, cu=FAKE, N=2, maxlen=129) == -1  # longer than T
+    assert _chunk(lib, eps=-1.0) == -1
+
+
+def test_decode_and_gate_norm_host_validation(lib):
+    assert lib.kda_decode_step(None, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 4, 2, 128, 128, 1, 1, 1.0, None, None,
+                               1e-6, None) == -1
+    assert lib.kda_decode_step(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 4, 2, 64, 128, 1, 1, 1.0, None, None,
+                               1e-6, None) == -2
+    assert lib.kda_decode_step(FAKE, FAKE + 4, FAKE, FAKE, FAKE, FAKE, FAKE, 4, 2, 128, 128, 1, 1, 1.0, None,
+                               None, 1e-6, None) == -3
+    assert lib.kda_decode_step(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 0, 2, 128, 128, 1, 1, 1.0, None, None,
+                               1e-6, None) == 0  # nothing to do, no launch
+    assert lib.kda_gate_norm(FAKE, FAKE, None, 1e-6, FAKE, -1, 128, 1, 1, None) == -1
+    assert lib.kda_gate_norm(FAKE, FAKE, None, 1e-6, FAKE, 10, 64, 1, 1, None) == -2
+    assert lib.kda_gate_norm(FAKE, FAKE, None, 1e-6, FAKE, 10, 128, 1, 0, None) == -1  # in place, sizes differ
+    assert lib.kda_query_status(None, None) == -1
+
+
+def test_binding_refuses_cpu_tensors():
+    import torch
+    x = torch.zeros(1, 4, 1, 128)
+    with pytest.raises(ValueError):
+        kda.chunk_fwd(x, x, x, x, torch.zeros(1, 4, 1))

@@ -1,0 +1,196 @@
+"""GPU parity: the CUDA path (through the C ABI binding) against the fp64 oracle
+on the same seeded inputs, element by element, relative L2 <= 1e-2."""
+import numpy as np
+import pytest
+
+import oracle
+from kda_testutil import REL_L2_TOL, D, dev, host, make_prefill, rel_l2
+from linear_attention_recurrence_06_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+
+def _torch():
+    import torch
+    return torch
+
+
+def run_prefill(inp, H, bf16, *, varlen, gate=False, out_f32=False):
+    torch = _torch()
+    import linear_attention_recurrence_06_b200 as kda
+    dt = torch.bfloat16 if bf16 else torch.float32
+    T = inp["T"]
+    q = dev(inp["q"], dt).view(1, T, H, D)
+    k = dev(inp["k"], dt).view(1, T, H, D)
+    v = dev(inp["v"], dt).view(1, T, H, D)
+    la = dev(inp["log_alpha"], dt).view(1, T, H, D)
+    b = dev(inp["beta"], dt).view(1, T, H)
+    g = dev(inp["g"], dt).view(1, T, H, D) if gate else None
+    s0 = dev(inp["s0"], torch.float32) if inp["s0"] is not None else None
+    kw = {}
+    if varlen:
+        kw = dict(cu_seqlens=torch.from_numpy(inp["cu"].astype(np.int32)).cuda(),
+                  max_seqlen=int(np.diff(inp["cu"]).max()))
+    o, fs = kda.chunk_fwd(q, k, v, la, b, s0, gate=g, out_dtype=torch.float32 if out_f32 else None, **kw)
+    torch.cuda.synchronize()
+    return host(o).reshape(T, H, D), host(fs)
+
+
+def oracle_prefill(inp, gate=False):
+    o, fs = oracle.kda_recurrent(inp["q"], inp["k"], inp["v"], inp["log_alpha"], inp["beta"], inp["s0"], inp["cu"])
+    if gate:
+        o = oracle.gate_norm(o, inp["g"], None, 1e-6)
+    return o, fs
+
+
+def check(o, fs, ro, rfs):
+    eo, ef = rel_l2(o, ro), rel_l2(fs, rfs)
+    assert eo <= REL_L2_TOL, f"output rel-L2 {eo:.3e}"
+    assert ef <= REL_L2_TOL, f"final-state rel-L2 {ef:.3e}"
+    return eo, ef
+
+
+# ----------------------------------------------------------------- prefill
+
+
+def test_prefill_fp32_small_config():
+    """T=256, H=2, fp32 inputs and output, zero initial state, seed 0."""
+    inp = make_prefill(0, [256], 2, bf16=False)
+    o, fs = run_prefill(inp, 2, False, varlen=False)
+    ro, rfs = oracle_prefill(inp)
+    check(o, fs, ro, rfs)
+
+
+@pytest.mark.parametrize("T", [1, 15, 16, 17, 63, 64, 65, 200, 333])
+def test_prefill_ragged_lengths_bf16(T):
+    inp = make_prefill(T, [T], 3, bf16=True, init=True)
+    o, fs = run_prefill(inp, 3, True, varlen=False, out_f32=True)
+    ro, rfs = oracle_prefill(inp)
+    check(o, fs, ro, rfs)
+
+
+def test_prefill_varlen_edge_lengths():
+    lens = [1, 15, 16, 17, 63, 64, 65, 0, 130]
+    inp = make_prefill(5, lens, 2, bf16=True, init=True)
+    o, fs = run_prefill(inp, 2, True, varlen=True, out_f32=True)
+    ro, rfs = oracle_prefill(inp)
+    check(o, fs, ro, rfs)
+    # per sequence, worst case
+    for n in range(len(lens)):
+        sl = slice(inp["cu"][n], inp["cu"][n + 1])
+        if lens[n]:
+            assert rel_l2(o[sl], ro[sl]) <= REL_L2_TOL
+        assert rel_l2(fs[n], rfs[n]) <= REL_L2_TOL
+
+
+@pytest.mark.parametrize("case", ["la_floor", "la_zero", "beta_zero", "beta_one", "la_below_floor"])
+def test_prefill_degenerate_decays(case):
+    kw = {}
+    if case == "la_floor":
+        kw = dict(la_const=-5.0)
+    elif case == "la_zero":
+        kw = dict(la_const=0.0)
+    elif case == "beta_zero":
+        # nothing is written; keep the decay mild so the pure-decay state stays
+        # inside the fp32 range (e^{-0.8 * 190} would underflow)
+        kw = dict(beta_const=0.0, la_scale=0.05)
+    elif case == "beta_one":
+        kw = dict(beta_const=1.0)
+    elif case == "la_below_floor":
+        kw = dict(la_scale=8.0)   # many values far below -5: the clamp path
+    inp = make_prefill(11, [190], 2, bf16=True, init=True, **kw)
+    o, fs = run_prefill(inp, 2, True, varlen=False, out_f32=True)
+    ro, rfs = oracle_prefill(inp)
+    check(o, fs, ro, rfs)
+
+
+@pytest.mark.parametrize("out_f32", [False, True])
+def test_prefill_fused_gate_norm(out_f32):
+    inp = make_prefill(3, [300], 4, bf16=True, gate=True)
+    o, fs = run_prefill(inp, 4, True, varlen=False, gate=True, out_f32=out_f32)
+    ro, rfs = oracle_prefill(inp, gate=True)
+    check(o, fs, ro, rfs)
+
+
+def test_prefill_multi_pass_workspace():
+    """A workspace that holds one chunk per sequence forces one pass per chunk:
+    the state carried between passes must give the same result."""
+    torch = _torch()
+    import linear_attention_recurrence_06_b200 as kda
+    lens = [200, 64, 1, 129]
+    H = 2
+    inp = make_prefill(9, lens, H, bf16=True, init=True)
+    T = inp["T"]
+    dt = torch.bfloat16
+    q, k, v, la = (dev(inp[x], dt).view(1, T, H, D) for x in ("q", "k", "v", "log_alpha"))
+    b = dev(inp["beta"], dt).view(1, T, H)
+    s0 = dev(inp["s0"], torch.float32)
+    cu = torch.from_numpy(inp["cu"].astype(np.int32)).cuda()
+    lo, _ = kda.workspace_size(T, H, len(lens), max(lens))
+    ws = torch.empty(lo, dtype=torch.uint8, device="cuda")
+    o, fs = kda.chunk_fwd(q, k, v, la, b, s0, cu_seqlens=cu, max_seqlen=max(lens), workspace=ws,
+                          out_dtype=torch.float32)
+    assert kda.query_status(ws) == 0
+    ro, rfs = oracle_prefill(inp)
+    check(host(o).reshape(T, H, D), host(fs), ro, rfs)
+
+
+def test_prefill_in_place_state():
+    torch = _torch()
+    import linear_attention_recurrence_06_b200 as kda
+    H = 2
+    inp = make_prefill(13, [150], H, bf16=True, init=True)
+    T = inp["T"]
+    dt = torch.bfloat16
+    q, k, v, la = (dev(inp[x], dt).view(1, T, H, D) for x in ("q", "k", "v", "log_alpha"))
+    b = dev(inp["beta"], dt).view(1, T, H)
+    s = dev(inp["s0"], torch.float32)
+    kda.chunk_fwd(q, k, v, la, b, s, final_state=s)
+    torch.cuda.synchronize()
+    _, rfs = oracle_prefill(inp)
+    assert rel_l2(host(s), rfs) <= REL_L2_TOL
+
+
+# ------------------------------------------------------------------ decode
+
+
+@pytest.mark.parametrize("bf16", [True, False])
+@pytest.mark.parametrize("gate", [False, True])
+def test_decode_steps(bf16, gate):
+    torch = _torch()
+    import linear_attention_recurrence_06_b200 as kda
+    Bd, H, steps = 6, 3, 12
+    dt = torch.bfloat16 if bf16 else torch.float32
+    s_np = synth.states(0, Bd, H, D, D)
+    s_dev = dev(s_np, torch.float32)
+    s_ref = s_np.astype(np.float64)
+    for step in range(steps):
+        tb = synth.tokens(0, step * Bd, Bd, H, D, D, bf16=bf16, gate=gate)
+        q, k, v, la = (dev(getattr(tb, x), dt) for x in ("q", "k", "v", "log_alpha"))
+        b = dev(tb.beta, dt)
+        g = dev(tb.g, dt) if gate else None
+        o = kda.decode_step(s_dev, q, k, v, la, b, gate=g, out_dtype=torch.float32)
+        ro, s_ref = oracle.decode_steps(s_ref, tb.q, tb.k, tb.v, tb.log_alpha, tb.beta)
+        if gate:
+            ro = oracle.gate_norm(ro, tb.g, None, 1e-6)
+        torch.cuda.synchronize()
+        assert rel_l2(host(o), ro) <= REL_L2_TOL
+    assert rel_l2(host(s_dev), s_ref) <= REL_L2_TOL
+
+
+# --------------------------------------------------------------- gate norm
+
+
+@pytest.mark.parametrize("bf16", [True, False])
+def test_gate_norm(bf16):
+    torch = _torch()
+    import linear_attention_recurrence_06_b200 as kda
+    rows = 1000
+    dt = torch.bfloat16 if bf16 else torch.float32
+    o = synth.normal(1, 100, (rows, D), 1.0, bf16)
+    g = synth.normal(1, 101, (rows, D), 1.0, bf16)
+    w = synth.normal(1, 102, (D,), 0.5, False) + 1.0
+    y = kda.gate_norm(dev(o, dt), dev(g, dt), dev(w, torch.float32), out_dtype=torch.float32)
+    ref = oracle.gate_norm(o.astype(np.float64), g, w, 1e-6)
+    torch.cuda.synchronize()
+    assert rel_l2(host(y), ref) <= 1e-5 if not bf16 else rel_l2(host(y), ref) <= REL_L2_TOL
