@@ -168,6 +168,46 @@ KDA_API kda_status kda_gate_norm(const void* o, const void* gate, const float* n
 KDA_API kda_status kda_query_status(void* workspace, void* stream);
 
 /*
+ * kda_chunk_fwd_noalloc -- kda_chunk_fwd for callers that cannot allocate
+ * device memory.  (No counterpart on the pages: it is a packaging of
+ * kda_chunk_fwd, not part of the method.)
+ *
+ * Who needs it: hosts that hand a plugin its inputs and outputs but no way to
+ * get device scratch -- e.g. a framework whose memory pool already owns all
+ * free device memory, or a runtime that forbids cudaMalloc on its hot path
+ * because cudaMalloc can synchronise the device.  Here the scratch is a
+ * static array of KDA_NOALLOC_SCRATCH_BYTES inside libkda's own device
+ * memory, so there is no workspace argument and the call allocates nothing.
+ *
+ * Arguments, layouts and results are exactly those of kda_chunk_fwd minus
+ * (workspace, workspace_bytes).  The caller still owns every input and output.
+ *  - Limit: the problem must fit the static scratch, i.e.
+ *    kda_chunk_fwd_workspace_size(...).bytes_min <= KDA_NOALLOC_SCRATCH_BYTES
+ *    (roughly n_seqs * H <= 400).  Larger problems
+ *    return KDA_ERR_WORKSPACE before any CUDA call; larger scratch than the
+ *    minimum only means fewer passes.
+ *  - The array is reserved on each GPU that loads this part of the library and
+ *    is held until the process exits.  The first call on a device looks up the
+ *    array's device address (cudaGetSymbolAddress) with that device current;
+ *    make that first call before any stream capture on that device.
+ *  - Every call on a device shares the one array, which keeps the previous
+ *    call's contents (the call clears the parts that must start at zero
+ *    itself).  Calls that overlap on the GPU (different streams without
+ *    ordering, or different host threads) race on it: order them.
+ *  - kda_query_status does not apply (there is no caller-visible workspace).
+ */
+#define KDA_NOALLOC_SCRATCH_BYTES (64u * 1024u * 1024u)
+
+KDA_API kda_status kda_chunk_fwd_noalloc(const void* q, const void* k, const void* v,
+                                 const void* log_alpha, const void* beta,
+                                 const float* init_state, void* o, float* final_state,
+                                 int B, int64_t T, int H, int dk, int dv,
+                                 const int32_t* cu_seqlens, int n_seqs, int64_t max_seqlen,
+                                 kda_dtype in_dtype, kda_dtype out_dtype, float scale,
+                                 const void* gate, const float* norm_weight, float eps,
+                                 void* stream);
+
+/*
  * Per-kernel device timing (a measurement aid, off by default).
  * kda_profile_enable(1) makes every later launch of this library bracket each
  * of its kernels with CUDA events on the launch stream.  kda_profile_read
