@@ -20,17 +20,20 @@
 //   O   = Qp S0 + Ob,                          Qp = scale (Q o Gam) - P W,  Ob = P Ut
 //
 // Two kernels:
-//   intra_kernel  one CTA per (chunk, head), all chunks in parallel.  Builds
-//                 the decay-scaled operands, runs every product above on the
-//                 tensor cores (tcgen05.mma, TMEM accumulators), inverts the
-//                 64x64 unit-triangular system in fp32, and writes Mlr, Qp,
-//                 Bm, Ob and Gam_C to the workspace.
-//   chain_kernel  one CTA per (sequence, head, 32-column slice of dv); walks
-//                 the chunks in order.  Per chunk ONE round of tensor-core
-//                 products (Mlr S and Qp S, the state slice as the shared B
-//                 operand), then S <- Gam_C o S - Mlr S + Bm in fp32 registers
-//                 and o = Qp S + Ob.  Mlr/Qp tiles arrive by bulk copies
-//                 (TMA engine), double-buffered one chunk ahead.
+//   intra_kernel  persistent, one CTA per SM, loops over (chunk, head) items.
+//                 Raw q/k/v/log_alpha tiles arrive by TMA (2-D tensor maps),
+//                 prefetched one item ahead.  Builds the decay-scaled operands,
+//                 runs every product above on the tensor cores (tcgen05.mma,
+//                 fp32 accumulators in TMEM), inverts the 64x64 unit-triangular
+//                 system in fp32, and writes Mlr, Qp, Gam_C, Bm, Ob to one
+//                 workspace slot per (chunk, head).
+//   chain_kernel  one CTA per (value-column slice, head, sequence); walks the
+//                 chunks in order.  Per chunk ONE tensor-core product on the
+//                 sequential path (Mlr S, the state slice as the B operand),
+//                 then S <- Gam_C o S - Mlr S + Bm in fp32 registers; the
+//                 output product Qp S (+ Ob) runs beside it off the critical
+//                 path.  Every per-chunk operand arrives by bulk copies (TMA
+//                 engine), two chunks ahead.
 //
 // Exponent references (why the -5 bound matters): inside a 64-token chunk the
 // cumulative decay can reach e^{-320}, whose reciprocal overflows fp32/bf16.
@@ -40,6 +43,9 @@
 // column operands of earlier tiles carry e^{G_b - g_s} = e^{G_b - G_{bs+1}}
 // e^{G_{bs+1} - g_s}, a product of two factors <= 1.  Every bf16 operand is
 // finite and every product is a correctly-scaled e^{g_t - g_s}.
+#include <cudaTypedefs.h>
+#include <string.h>
+
 #include "kda_profile.h"
 #include "kda_sm100.cuh"
 
@@ -49,13 +55,19 @@ constexpr int CH = 64;    // chunk length
 constexpr int DK = 128;   // key head dim
 constexpr int DV = 128;   // value head dim
 constexpr int DVS = 32;   // value columns per chain CTA
+constexpr int NSL = DV / DVS;
 
-// Workspace bytes per (chunk, head) slot.
-constexpr size_t SLOT_M = (size_t)DK * DK * 2;   // Mlr, bf16 K-major SW128 image [128][128]
-constexpr size_t SLOT_Q = (size_t)CH * DK * 2;   // Qp,  bf16 K-major SW128 image [64][128]
-constexpr size_t SLOT_B = (size_t)DK * DV * 2;   // Bm,  bf16 row-major [128][128]
-constexpr size_t SLOT_O = (size_t)CH * DV * 2;   // Ob,  bf16 row-major [64][128]
-constexpr size_t SLOT_G = (size_t)DK * 4;        // Gam_C, fp32 [128]
+// Workspace slot per (chunk, head), all offsets 16-byte aligned:
+//   Mlr  bf16 K-major SW128 image [128 key rows][128 K]          32768 B
+//   Qp   bf16 MN-major no-swizzle image, M = 64 tokens, K = 128   16384 B
+//   GamC fp32 [128]                                                512 B
+//   Bm   bf16 [4 slices][128 key rows][32 value cols]            32768 B
+//   ObT  bf16 [4 slices][32 value cols][64 tokens]               16384 B
+constexpr size_t SO_M = 0, SO_Q = 32768, SO_G = 49152, SO_B = 49664, SO_O = 82432;
+constexpr size_t SLOT_BYTES = 98816;
+constexpr uint32_t SO_MQG = 49664;         // Mlr + Qp + GamC, one contiguous copy
+constexpr uint32_t BSL = DK * DVS * 2;     // one Bm slice, 8192 B
+constexpr uint32_t OSL = CH * DVS * 2;     // one Ob slice, 4096 B
 
 struct ChunkArgs {
     const void* q;
@@ -67,11 +79,7 @@ struct ChunkArgs {
     float* state_io;           // carry / final state [N, H, dk, dv]
     void* o;
     const int32_t* cu;         // nullable (fixed length)
-    uint8_t* ws_M;
-    uint8_t* ws_Q;
-    uint8_t* ws_B;
-    uint8_t* ws_O;
-    float* ws_G;
+    uint8_t* ws;               // slots
     uint32_t* status;
     int64_t T;                 // tokens per sequence (fixed) or total tokens (varlen)
     int H;
@@ -96,6 +104,21 @@ KDA_DEV void seq_range(const ChunkArgs& a, int n, int64_t& sb, int64_t& se) {
     }
 }
 
+// Item = workspace slot = ((n * wc) + (chunk - i0)) * H + h.  Returns false if
+// that chunk lies beyond its sequence.
+KDA_DEV bool item_info(const ChunkArgs& a, int64_t item, int& h, int64_t& t0, int& L) {
+    h = (int)(item % a.H);
+    const int64_t rest = item / a.H;
+    const int n = (int)(rest / a.wc);
+    const int ci = a.i0 + (int)(rest % a.wc);
+    int64_t sb, se;
+    seq_range(a, n, sb, se);
+    t0 = sb + (int64_t)ci * CH;
+    if (t0 >= se) return false;
+    L = (int)((se - t0) < CH ? (se - t0) : CH);
+    return true;
+}
+
 // Issues D (+)= A B^T over K (multiple of 16) for two K-major SW128 images.
 // a_rows / b_rows are the row counts of one 128-byte-wide K block of each.
 KDA_DEV void mma_run(uint32_t d, uint32_t a_addr, uint32_t a_rows, uint32_t b_addr, uint32_t b_rows, int K,
@@ -108,33 +131,76 @@ KDA_DEV void mma_run(uint32_t d, uint32_t a_addr, uint32_t a_rows, uint32_t b_ad
     }
 }
 
+// Same for two MN-major no-swizzle images (core-matrix M/N stride 128 B; K-group
+// stride a_kg / b_kg bytes): one MMA step of K = 16 spans two K groups.
+KDA_DEV void mma_run_mn(uint32_t d, uint32_t a_addr, uint32_t a_kg, uint32_t b_addr, uint32_t b_kg, int K,
+                        uint32_t idesc) {
+    for (int kk = 0; kk < K / 16; ++kk) {
+        const uint64_t ad = sdesc_interleave(a_addr + (uint32_t)kk * 2u * a_kg, a_kg, 128u);
+        const uint64_t bd = sdesc_interleave(b_addr + (uint32_t)kk * 2u * b_kg, b_kg, 128u);
+        mma_bf16(d, ad, bd, idesc, kk > 0 ? 1u : 0u);
+    }
+}
+
+KDA_DEV uint4 pack8(const float* x) {
+    return make_uint4(pack_bf16x2(x[0], x[1]), pack_bf16x2(x[2], x[3]), pack_bf16x2(x[4], x[5]),
+                      pack_bf16x2(x[6], x[7]));
+}
+
 // ---------------------------------------------------------------------------
 // intra_kernel
 // ---------------------------------------------------------------------------
 // Threads: 256.  Thread tid owns key/value channel c = tid & 127 and tokens
 // [32*half, 32*half + 32), half = tid >> 7.  Warp w reads TMEM lanes
-// 32*(w & 3) .. +31, i.e. rows c = tid & 127, and its half selects columns.
+// 32*(w & 3) .. +31, i.e. rows c = tid & 127; its half selects columns.
 //
 // Shared memory (offsets from a 1024-aligned base):
-//   X [0, 72K)      phase 1: KQr [128][128] @0, Kd [64][128] @32K,
-//                            Kb1 [16][128] @48K, Kb2 [32][128] @52K, Kb3 [48][128] @60K
-//                   phase 2: KGt [128][64] @0, Vt [128][64] @16K, Ti [64][64] @32K,
-//                            Ktt [128][64] @40K, Ph [64][64] @56K, inverse temp @64K
-//   Y [72K, 104K)   A fp32 [64][64] @0, X fp32 [64][64] @16K; later Wt [128][64] @0,
-//                   Ut [128][64] @16K
-//   misc            beta[64], G[5][128], half-0 totals[128], mbarrier, TMEM base
-constexpr uint32_t IX_KQR = 0, IX_KD = 32768, IX_KB1 = 49152, IX_KB2 = 53248, IX_KB3 = 61440;
-constexpr uint32_t IX_KGT = 0, IX_VT = 16384, IX_TI = 32768, IX_KTT = 40960, IX_PH = 57344, IX_TMP = 65536;
-constexpr uint32_t IY = 73728;
-constexpr uint32_t IY_A = IY, IY_X = IY + 16384, IY_WT = IY, IY_UT = IY + 16384;
-constexpr uint32_t IM = IY + 32768;
-constexpr uint32_t IM_BETA = IM, IM_G = IM + 256, IM_TOT = IM + 256 + 2560, IM_BAR = IM_TOT + 512,
-                   IM_TMEM = IM_BAR + 8;
-constexpr uint32_t INTRA_SMEM = IM_TMEM + 8 + 1024;  // + alignment slack
-constexpr uint32_t INTRA_TMEM_COLS = 256;
+//   RAW [0, 64K)     TMA tiles [64 tokens][128 ch] bf16: la @0, k @16K, q @32K, v @48K
+//   X   [64K, 136K)  phase 1 (MN-major, no swizzle, M/N = token): KQr 128x128 @0,
+//                             Kd 64x128 @32K, Kb1 16x128 @48K, Kb2 32x128 @52K, Kb3 48x128 @60K
+//                    phase 2: KGt [128][64] @0, Vt [128][64] @16K, Ti [64][64] @32K,
+//                             Ktt [128][64] @40K, Ph [64][64] @56K, inverse temp @64K
+//   Y   [136K, ...)  A fp32 [64][68] @0, X fp32 [64][68] @17408;
+//                    later Wt [128][64] @0, Ut [128][64] @16K
+//   misc             beta[64], G[5][128], half-0 totals[128], 2 mbarriers, TMEM base
+// TMEM (512 columns): round 1  A/P diag [0,64), off-diag [64,80) [80,112) [112,160)
+//                     round 2  Wt [160,224), Ut [224,288)
+//                     round 3  Mlr [288,416), (PW)^T [416,480), Bm [0,128), Ob^T [128,192)
+constexpr uint32_t R_LA = 0, R_K = 16384, R_Q = 32768, R_V = 49152;
+constexpr uint32_t IX = 65536;
+constexpr uint32_t IX_KQR = IX + 0, IX_KD = IX + 32768, IX_KB1 = IX + 49152, IX_KB2 = IX + 53248,
+                   IX_KB3 = IX + 61440;
+constexpr uint32_t IX_KGT = IX + 0, IX_VT = IX + 16384, IX_TI = IX + 32768, IX_KTT = IX + 40960,
+                   IX_PH = IX + 57344, IX_TMP = IX + 65536;
+constexpr uint32_t IY = IX + 73728;
+constexpr int LDA = 68;  // padded fp32 row stride of A and X (16-byte rows, spread banks)
+constexpr uint32_t IY_A = IY, IY_X = IY + 64 * LDA * 4, IY_WT = IY, IY_UT = IY + 16384;
+constexpr uint32_t IM = IY + 35840;
+constexpr uint32_t IM_BETA = IM, IM_G = IM + 256, IM_TOT = IM + 256 + 2560, IM_BAR_RAW = IM_TOT + 512,
+                   IM_BAR_MMA = IM_BAR_RAW + 8, IM_TMEM = IM_BAR_MMA + 8;
+constexpr uint32_t INTRA_SMEM = IM_TMEM + 16 + 1024;  // + alignment slack
+constexpr uint32_t INTRA_TMEM_COLS = 512;
+constexpr uint32_t TM_AD = 0, TM_B1 = 64, TM_B2 = 80, TM_B3 = 112, TM_WT = 160, TM_UT = 224, TM_M = 288,
+                   TM_PW = 416, TM_BM = 0, TM_OB = 128;
+
+struct IntraMaps {
+    CUtensorMap la, k, q, v;
+};
 
 template <bool IN_BF16>
-__global__ void __launch_bounds__(256, 2) intra_kernel(const ChunkArgs a) {
+KDA_DEV float raw_in(const uint8_t* sm, uint32_t tile, const void* gsrc, size_t ebase, size_t rowstride, int t,
+                     int c, int L) {
+    if (t >= L) return 0.f;
+    if constexpr (IN_BF16) {
+        return bf16_to_f32(*reinterpret_cast<const uint16_t*>(sm + tile + (uint32_t)(t * 128 + c) * 2u));
+    } else {
+        return __ldg(reinterpret_cast<const float*>(gsrc) + ebase + (size_t)t * rowstride);
+    }
+}
+
+template <bool IN_BF16>
+__global__ void __launch_bounds__(256, 1)
+intra_kernel(const ChunkArgs a, const __grid_constant__ IntraMaps maps, const int64_t n_items) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     const uint32_t sb = smem_u32(sm);
@@ -142,19 +208,13 @@ __global__ void __launch_bounds__(256, 2) intra_kernel(const ChunkArgs a) {
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int c = tid & 127, half = tid >> 7;
     const int qd = warp & 3;
-    const int H = a.H, h = blockIdx.y;
-    const int n = blockIdx.x / a.wc, ci = a.i0 + blockIdx.x % a.wc;
-    int64_t s_beg, s_end;
-    seq_range(a, n, s_beg, s_end);
-    const int64_t t0 = s_beg + (int64_t)ci * CH;
-    if (t0 >= s_end) return;  // chunk beyond this sequence: nothing to do
-    const int L = (int)((s_end - t0) < CH ? (s_end - t0) : CH);
-    const size_t slot = ((size_t)n * a.wc + (blockIdx.x % a.wc)) * H + h;
+    const int H = a.H;
 
     float* s_beta = reinterpret_cast<float*>(sm + IM_BETA);
     float* s_G = reinterpret_cast<float*>(sm + IM_G);      // [5][128]
     float* s_tot = reinterpret_cast<float*>(sm + IM_TOT);  // [128]
-    uint64_t* bar = reinterpret_cast<uint64_t*>(sm + IM_BAR);
+    uint64_t* bar_raw = reinterpret_cast<uint64_t*>(sm + IM_BAR_RAW);
+    uint64_t* bar_mma = reinterpret_cast<uint64_t*>(sm + IM_BAR_MMA);
     uint32_t* s_tmem = reinterpret_cast<uint32_t*>(sm + IM_TMEM);
 
     if (warp == 0) {
@@ -162,383 +222,418 @@ __global__ void __launch_bounds__(256, 2) intra_kernel(const ChunkArgs a) {
         tmem_relinquish();
     }
     if (tid == 0) {
-        mbar_init(bar, 1);
+        mbar_init(bar_raw, 1);
+        mbar_init(bar_mma, 1);
         fence_mbar_init();
     }
-    if (tid < CH) s_beta[tid] = (tid < L) ? ld_in<IN_BF16>(a.beta, (size_t)(t0 + tid) * H + h) : 0.f;
-
-    // ---- phase 1: cumulative clamped log-decay g (registers), tile references G
-    const size_t rowstride = (size_t)H * DK;
-    const size_t ebase = ((size_t)t0 * H + h) * DK + c;  // element (t0, h, c)
-    float gl[32];
-    {
-        float run = 0.f;
-#pragma unroll
-        for (int u = 0; u < 32; ++u) {
-            const int t = 32 * half + u;
-            const float l = (t < L) ? fmaxf(ld_in<IN_BF16>(a.log_alpha, ebase + (size_t)t * rowstride),
-                                            LOG_ALPHA_FLOOR)
-                                    : 0.f;
-            run += l;
-            gl[u] = run;
-        }
-        if (half == 0) s_tot[c] = run;
-    }
-    __syncthreads();
-    if (half == 1) {
-        const float off = s_tot[c];
-#pragma unroll
-        for (int u = 0; u < 32; ++u) gl[u] += off;
-    }
-    // G_0 = 0, G_1 = g_15, G_2 = g_31, G_3 = g_47, G_4 = g_63 (= g at the chunk end)
-    if (half == 0) {
-        s_G[0 * 128 + c] = 0.f;
-        s_G[1 * 128 + c] = gl[15];
-        s_G[2 * 128 + c] = gl[31];
-    } else {
-        s_G[3 * 128 + c] = gl[15];
-        s_G[4 * 128 + c] = gl[31];
-    }
-    __syncthreads();
-    float G[5];
-#pragma unroll
-    for (int b = 0; b < 5; ++b) G[b] = s_G[b * 128 + c];
-
-    // E1 = e^{g_t - G_bt} (<= 1),  E3 = e^{G_{bt+1} - g_t} (<= 1)
-    float E1[32], E3[32];
-#pragma unroll
-    for (int u = 0; u < 32; ++u) {
-        const int bt = (32 * half + u) >> 4;  // compile-time per half after unrolling
-        const float Gb = (bt == 0) ? G[0] : (bt == 1) ? G[1] : (bt == 2) ? G[2] : G[3];
-        const float Gn = (bt == 0) ? G[1] : (bt == 1) ? G[2] : (bt == 2) ? G[3] : G[4];
-        E1[u] = __expf(gl[u] - Gb);
-        E3[u] = __expf(Gn - gl[u]);
-    }
-
-    // ---- phase 1 operands: KQr = [K o E1 ; scale Q o E1], Kd = K o e^{G_bt - g}, Kb^(b)
-    {
-        const uint32_t kb = (uint32_t)c >> 6, kc = (uint32_t)c & 63u;
-        // factors e^{G_b - G_{bs+1}} for the off-diagonal column operands
-        const float f21 = __expf(G[2] - G[1]), f31 = __expf(G[3] - G[1]), f32 = __expf(G[3] - G[2]);
-#pragma unroll
-        for (int u = 0; u < 32; ++u) {
-            const int t = 32 * half + u;
-            const int bt = t >> 4;
-            const float kv = (t < L) ? ld_in<IN_BF16>(a.k, ebase + (size_t)t * rowstride) : 0.f;
-            const float qv = (t < L) ? ld_in<IN_BF16>(a.q, ebase + (size_t)t * rowstride) : 0.f;
-            const float kr = kv * E1[u];
-            *reinterpret_cast<uint16_t*>(sm + IX_KQR + kb * 16384u + sw128_off(t, kc)) = f32_to_bf16(kr);
-            *reinterpret_cast<uint16_t*>(sm + IX_KQR + kb * 16384u + sw128_off(t + 64, kc)) =
-                f32_to_bf16(qv * E1[u] * a.scale);
-            const float Gb = (bt == 0) ? G[0] : (bt == 1) ? G[1] : (bt == 2) ? G[2] : G[3];
-            *reinterpret_cast<uint16_t*>(sm + IX_KD + kb * 8192u + sw128_off(t, kc)) =
-                f32_to_bf16(kv * __expf(Gb - gl[u]));  // e^{G_bt - g_t} <= e^80
-            const float ke3 = kv * E3[u];
-            if (bt == 0) {
-                *reinterpret_cast<uint16_t*>(sm + IX_KB1 + kb * 2048u + sw128_off(t, kc)) = f32_to_bf16(ke3);
-                *reinterpret_cast<uint16_t*>(sm + IX_KB2 + kb * 4096u + sw128_off(t, kc)) =
-                    f32_to_bf16(ke3 * f21);
-                *reinterpret_cast<uint16_t*>(sm + IX_KB3 + kb * 6144u + sw128_off(t, kc)) =
-                    f32_to_bf16(ke3 * f31);
-            } else if (bt == 1) {
-                *reinterpret_cast<uint16_t*>(sm + IX_KB2 + kb * 4096u + sw128_off(t, kc)) = f32_to_bf16(ke3);
-                *reinterpret_cast<uint16_t*>(sm + IX_KB3 + kb * 6144u + sw128_off(t, kc)) =
-                    f32_to_bf16(ke3 * f32);
-            } else if (bt == 2) {
-                *reinterpret_cast<uint16_t*>(sm + IX_KB3 + kb * 6144u + sw128_off(t, kc)) = f32_to_bf16(ke3);
-            }
-        }
-    }
-    fence_async_smem();
     __syncthreads();
     tc_fence_after();
     const uint32_t tm = *s_tmem;
+    const uint32_t lane_addr = tm + ((uint32_t)(32 * qd) << 16);
+    uint32_t ph_raw = 0, ph_mma = 0;
 
-    // ---- MMA round 1: [Kr;Qr] Kd^T -> cols [0,64); [Kr;Qr] Kb(b)^T -> [64,80),[80,112),[112,160)
-    if (tid == 0) {
-        mma_run(tm + 0, sb + IX_KQR, 128, sb + IX_KD, 64, DK, idesc_bf16(128, 64));
-        mma_run(tm + 64, sb + IX_KQR, 128, sb + IX_KB1, 16, DK, idesc_bf16(128, 16));
-        mma_run(tm + 80, sb + IX_KQR, 128, sb + IX_KB2, 32, DK, idesc_bf16(128, 32));
-        mma_run(tm + 112, sb + IX_KQR, 128, sb + IX_KB3, 48, DK, idesc_bf16(128, 48));
-        mma_commit(bar);
-    }
-    uint32_t phase = 0;
-    mbar_wait(bar, phase, a.status);
-    phase ^= 1;
-    tc_fence_after();
+    // next valid item at or after `from` (stride gridDim.x), or n_items
+    auto next_valid = [&](int64_t from) -> int64_t {
+        for (int64_t it = from; it < n_items; it += gridDim.x) {
+            int hh, LL;
+            int64_t tt;
+            if (item_info(a, it, hh, tt, LL)) return it;
+        }
+        return n_items;
+    };
+    auto issue_raw = [&](int64_t it) {
+        int hh, LL;
+        int64_t tt;
+        item_info(a, it, hh, tt, LL);
+        mbar_arrive_expect_tx(bar_raw, 4u * 16384u);
+        tma_load_2d(sm + R_LA, &maps.la, hh * DK, (int)tt, bar_raw);
+        tma_load_2d(sm + R_K, &maps.k, hh * DK, (int)tt, bar_raw);
+        tma_load_2d(sm + R_Q, &maps.q, hh * DK, (int)tt, bar_raw);
+        tma_load_2d(sm + R_V, &maps.v, hh * DV, (int)tt, bar_raw);
+    };
 
-    // ---- extract A (rows 0..63) into fp32 smem and P (rows 64..127) into the bf16 image Ph
-    {
-        float* sA = reinterpret_cast<float*>(sm + IY_A);
-        const int r = 32 * qd + lane;
-        const bool isP = r >= 64;
-        const int t = r & 63, bt = t >> 4;
-        const uint32_t lane_addr = tm + ((uint32_t)(32 * qd) << 16);
-        auto put = [&](int s, float val) {
-            if (isP) {
-                *reinterpret_cast<uint16_t*>(sm + IX_PH + sw128_off(t, s)) = f32_to_bf16(val);
-            } else {
-                sA[t * 64 + s] = val;
-            }
-        };
-        if (half == 0) {
-            // diagonal tile and the zero upper part: columns s >= 16 bt
-            float d0[32], d1[32];
-            tmem_ld32(lane_addr + 0, d0);
-            tmem_ld32(lane_addr + 32, d1);
-            tmem_ld_wait();
-#pragma unroll
-            for (int s = 0; s < 64; ++s) {
-                const float val = (s < 32) ? d0[s & 31] : d1[s & 31];
-                if ((s >> 4) >= bt) {
-                    const bool keep = ((s >> 4) == bt) && (isP ? (s <= t) : (s < t));
-                    put(s, keep ? val : 0.f);
-                }
-            }
-        } else {
-            // off-diagonal tiles: columns s < 16 bt, from the operand of this row tile
-            if ((qd & 1) == 0) {  // rows t in [0, 32): tiles 0 and 1
-                float d[16];
-                tmem_ld16(lane_addr + 64, d);
-                tmem_ld_wait();
-                if (bt == 1) {
-#pragma unroll
-                    for (int s = 0; s < 16; ++s) put(s, d[s]);
-                }
-            } else {  // rows t in [32, 64): tiles 2 and 3
-                float d2[32], d3[32], d3b[16];
-                tmem_ld32(lane_addr + 80, d2);
-                tmem_ld32(lane_addr + 112, d3);
-                tmem_ld16(lane_addr + 144, d3b);
-                tmem_ld_wait();
-                if (bt == 2) {
-#pragma unroll
-                    for (int s = 0; s < 32; ++s) put(s, d2[s]);
-                } else {
-#pragma unroll
-                    for (int s = 0; s < 48; ++s) put(s, (s < 32) ? d3[s & 31] : d3b[s & 15]);
-                }
-            }
-        }
-    }
-    tc_fence_before();
-    __syncthreads();
-
-    // ---- T = (I + Diag(beta) A)^-1 Diag(beta), fp32, blocked on 16x16 tiles
-    {
-        float* sA = reinterpret_cast<float*>(sm + IY_A);  // becomes N = Diag(beta) A in place
-        float* sX = reinterpret_cast<float*>(sm + IY_X);  // X = (I + N)^-1
-        float* sY = reinterpret_cast<float*>(sm + IX_TMP);  // [3][16][16] temporaries
-        for (int e = tid; e < 64 * 64; e += 256) {
-            const int i = e >> 6;
-            sA[e] *= s_beta[i];
-        }
-        __syncthreads();
-        // diagonal blocks: thread per (block, column) does forward substitution
-        if (tid < 64) {
-            const int b = tid >> 4, j = tid & 15;
-            const float* Nb = sA + (16 * b) * 64 + 16 * b;
-            float x[16];
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                float acc = 0.f;
-#pragma unroll
-                for (int m = 0; m < i; ++m)
-                    if (m >= j) acc += Nb[i * 64 + m] * x[m];
-                x[i] = (i < j) ? 0.f : ((i == j) ? 1.f : -acc);
-            }
-#pragma unroll
-            for (int i = 0; i < 16; ++i) sX[(16 * b + i) * 64 + 16 * b + j] = x[i];
-        }
-        // zero the strictly upper blocks of X
-        for (int e = tid; e < 64 * 64; e += 256) {
-            const int i = e >> 6, j = e & 63;
-            if ((j >> 4) > (i >> 4)) sX[e] = 0.f;
-        }
-        __syncthreads();
-        // off-diagonal blocks by distance d = bi - bj:
-        //   X_ij = -X_ii * sum_{m=j}^{i-1} N_im X_mj
-        for (int d = 1; d <= 3; ++d) {
-            const int nblk = 4 - d;
-            for (int e = tid; e < nblk * 256; e += 256) {
-                const int p = e >> 8, r = (e >> 4) & 15, cc = e & 15;
-                const int bj = p, bi = p + d;
-                float acc = 0.f;
-                for (int m = bj; m < bi; ++m) {
-#pragma unroll
-                    for (int uu = 0; uu < 16; ++uu)
-                        acc += sA[(16 * bi + r) * 64 + 16 * m + uu] * sX[(16 * m + uu) * 64 + 16 * bj + cc];
-                }
-                sY[p * 256 + r * 16 + cc] = acc;
-            }
-            __syncthreads();
-            for (int e = tid; e < nblk * 256; e += 256) {
-                const int p = e >> 8, r = (e >> 4) & 15, cc = e & 15;
-                const int bj = p, bi = p + d;
-                float acc = 0.f;
-#pragma unroll
-                for (int uu = 0; uu < 16; ++uu)
-                    acc += sX[(16 * bi + r) * 64 + 16 * bi + uu] * sY[p * 256 + uu * 16 + cc];
-                sX[(16 * bi + r) * 64 + 16 * bj + cc] = -acc;
-            }
-            __syncthreads();
-        }
-        // T = X Diag(beta) -> bf16 image Ti [t][s]
-        for (int e = tid; e < 64 * 64; e += 256) {
-            const int t = e >> 6, s = e & 63;
-            *reinterpret_cast<uint16_t*>(sm + IX_TI + sw128_off(t, s)) = f32_to_bf16(sX[e] * s_beta[s]);
-        }
+    int64_t item = next_valid(blockIdx.x);
+    bool raw_in_flight = false;
+    if constexpr (IN_BF16) {
+        if (tid == 0 && item < n_items) issue_raw(item);
+        raw_in_flight = item < n_items;
     }
 
-    // ---- phase 2 operands (transposed, K = token): KGt = (K o Gam)^T, Vt = V^T, Ktt = Kt^T
-    {
-        // tiles of this half: bt = 2*half + lb, lb in {0, 1}
-        const float eG[2] = {__expf(half ? G[2] : G[0]), __expf(half ? G[3] : G[1])};
-        const float eC[2] = {__expf(G[4] - (half ? G[3] : G[1])), __expf(G[4] - (half ? G[4] : G[2]))};
+    while (item < n_items) {
+        int h, L;
+        int64_t t0;
+        item_info(a, item, h, t0, L);
+        uint8_t* wslot = a.ws + (size_t)item * SLOT_BYTES;
+        const size_t rowstride = (size_t)H * DK;
+        const size_t ebase = ((size_t)t0 * H + h) * DK + c;
         const size_t vbase = ((size_t)t0 * H + h) * DV + c;
-#pragma unroll
-        for (int m = 0; m < 4; ++m) {  // 8 consecutive tokens per 16-byte chunk
-            uint32_t pk[4], pv[4], pt[4];
-#pragma unroll
-            for (int p = 0; p < 4; ++p) {
-                float kgv[2], vvv[2], ktv[2];
-#pragma unroll
-                for (int e2 = 0; e2 < 2; ++e2) {
-                    const int u = 8 * m + 2 * p + e2;
-                    const int t = 32 * half + u;
-                    const int lb = u >> 4;  // tile within this half
-                    const float kv = (t < L) ? ld_in<IN_BF16>(a.k, ebase + (size_t)t * rowstride) : 0.f;
-                    const float vv = (t < L) ? ld_in<IN_BF16>(a.v, vbase + (size_t)t * H * DV) : 0.f;
-                    kgv[e2] = kv * E1[u] * eG[lb];
-                    ktv[e2] = kv * E3[u] * eC[lb];
-                    vvv[e2] = vv;
-                }
-                pk[p] = pack_bf16x2(kgv[0], kgv[1]);
-                pv[p] = pack_bf16x2(vvv[0], vvv[1]);
-                pt[p] = pack_bf16x2(ktv[0], ktv[1]);
-            }
-            const uint32_t s0 = (uint32_t)(32 * half + 8 * m);
-            const uint32_t off = sw128_off((uint32_t)c, s0);
-            *reinterpret_cast<uint4*>(sm + IX_KGT + off) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-            *reinterpret_cast<uint4*>(sm + IX_VT + off) = make_uint4(pv[0], pv[1], pv[2], pv[3]);
-            *reinterpret_cast<uint4*>(sm + IX_KTT + off) = make_uint4(pt[0], pt[1], pt[2], pt[3]);
-        }
-        if (half == 1) a.ws_G[slot * DK + c] = __expf(G[4]);
-    }
-    fence_async_smem();
-    __syncthreads();
-    tc_fence_after();
 
-    // ---- MMA round 2: Wt = KGt Ti^T -> cols [0,64);  Ut = Vt Ti^T -> cols [64,128)
-    if (tid == 0) {
-        mma_run(tm + 0, sb + IX_KGT, 128, sb + IX_TI, 64, CH, idesc_bf16(128, 64));
-        mma_run(tm + 64, sb + IX_VT, 128, sb + IX_TI, 64, CH, idesc_bf16(128, 64));
-        mma_commit(bar);
-    }
-    mbar_wait(bar, phase, a.status);
-    phase ^= 1;
-    tc_fence_after();
-    {
-        // half 0 extracts Wt, half 1 extracts Ut; row = channel c, 64 token columns
-        const uint32_t col0 = half ? 64u : 0u;
-        const uint32_t dst = half ? IY_UT : IY_WT;
-        float d0[32], d1[32];
-        const uint32_t lane_addr = tm + ((uint32_t)(32 * qd) << 16);
-        tmem_ld32(lane_addr + col0, d0);
-        tmem_ld32(lane_addr + col0 + 32, d1);
-        tmem_ld_wait();
-#pragma unroll
-        for (int m = 0; m < 8; ++m) {
-            const float* src = (m < 4) ? d0 : d1;
-            const int o8 = (m & 3) * 8;
-            const uint4 pk = make_uint4(pack_bf16x2(src[o8 + 0], src[o8 + 1]), pack_bf16x2(src[o8 + 2], src[o8 + 3]),
-                                        pack_bf16x2(src[o8 + 4], src[o8 + 5]), pack_bf16x2(src[o8 + 6], src[o8 + 7]));
-            *reinterpret_cast<uint4*>(sm + dst + sw128_off((uint32_t)c, (uint32_t)(8 * m))) = pk;
+        if (tid < CH) s_beta[tid] = (tid < L) ? ld_in<IN_BF16>(a.beta, (size_t)(t0 + tid) * H + h) : 0.f;
+        if constexpr (IN_BF16) {
+            mbar_wait(bar_raw, ph_raw, a.status);
+            ph_raw ^= 1;
+            raw_in_flight = false;
         }
-    }
-    fence_async_smem();
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
 
-    // ---- MMA round 3: Mlr = Ktt Wt^T -> [0,128);  (P W)^T = Wt Ph^T -> [128,192);
-    //                   Ob^T = Ut Ph^T -> [192,256)
-    if (tid == 0) {
-        mma_run(tm + 0, sb + IX_KTT, 128, sb + IY_WT, 128, CH, idesc_bf16(128, 128));
-        mma_run(tm + 128, sb + IY_WT, 128, sb + IX_PH, 64, CH, idesc_bf16(128, 64));
-        mma_run(tm + 192, sb + IY_UT, 128, sb + IX_PH, 64, CH, idesc_bf16(128, 64));
-        mma_commit(bar);
-    }
-    mbar_wait(bar, phase, a.status);
-    phase ^= 1;
-    tc_fence_after();
-    {
-        const uint32_t lane_addr = tm + ((uint32_t)(32 * qd) << 16);
-        // Mlr row c -> K-major SW128 image in the workspace (half h covers K block h)
+        // ---- a1: cumulative clamped log-decay g (registers), tile references G
+        float E1[32], E3[32];
+        uint32_t qr2[16];  // raw q of this thread's 32 tokens, bf16 pairs (kept for the Qp epilogue)
         {
-            uint8_t* dstM = a.ws_M + slot * SLOT_M + (size_t)half * (DK * 128);
-            float d0[32], d1[32];
-            tmem_ld32(lane_addr + 64 * half, d0);
-            tmem_ld32(lane_addr + 64 * half + 32, d1);
-            tmem_ld_wait();
-#pragma unroll
-            for (int m = 0; m < 8; ++m) {
-                const float* src = (m < 4) ? d0 : d1;
-                const int o8 = (m & 3) * 8;
-                const uint4 pk = make_uint4(pack_bf16x2(src[o8 + 0], src[o8 + 1]), pack_bf16x2(src[o8 + 2], src[o8 + 3]),
-                                            pack_bf16x2(src[o8 + 4], src[o8 + 5]), pack_bf16x2(src[o8 + 6], src[o8 + 7]));
-                *reinterpret_cast<uint4*>(dstM + sw128_off((uint32_t)c, (uint32_t)(8 * m))) = pk;
-            }
-        }
-        // Qp^T[c][t] = scale q_tc e^{g_tc} - (P W)^T[c][t] and Ob^T[j][t]; thread covers its 32 tokens
-        {
-            float pw[32], ob[32];
-            tmem_ld32(lane_addr + 128 + 32 * half, pw);
-            tmem_ld32(lane_addr + 192 + 32 * half, ob);
-            tmem_ld_wait();
-            const float eG[2] = {__expf(half ? G[2] : G[0]), __expf(half ? G[3] : G[1])};
-            uint8_t* dstQ = a.ws_Q + slot * SLOT_Q + (size_t)(c >> 6) * (CH * 128);
-            uint16_t* dstO = reinterpret_cast<uint16_t*>(a.ws_O + slot * SLOT_O);
+            float gl[32];
+            float run = 0.f;
 #pragma unroll
             for (int u = 0; u < 32; ++u) {
                 const int t = 32 * half + u;
-                const float qv = (t < L) ? ld_in<IN_BF16>(a.q, ebase + (size_t)t * rowstride) : 0.f;
-                const float qg = qv * E1[u] * eG[u >> 4] * a.scale;
-                *reinterpret_cast<uint16_t*>(dstQ + sw128_off((uint32_t)t, (uint32_t)(c & 63))) =
-                    f32_to_bf16(qg - pw[u]);
-                dstO[(size_t)t * DV + c] = f32_to_bf16(ob[u]);
+                const float l = raw_in<IN_BF16>(sm, R_LA, a.log_alpha, ebase, rowstride, t, c, L);
+                run += (t < L) ? fmaxf(l, LOG_ALPHA_FLOOR) : 0.f;
+                gl[u] = run;
+            }
+            if (half == 0) s_tot[c] = run;
+            __syncthreads();
+            if (half == 1) {
+                const float off = s_tot[c];
+#pragma unroll
+                for (int u = 0; u < 32; ++u) gl[u] += off;
+                s_G[3 * 128 + c] = gl[15];
+                s_G[4 * 128 + c] = gl[31];
+            } else {
+                s_G[0 * 128 + c] = 0.f;
+                s_G[1 * 128 + c] = gl[15];
+                s_G[2 * 128 + c] = gl[31];
+            }
+            __syncthreads();
+            // E1 = e^{g_t - G_bt} (<= 1),  E3 = e^{G_{bt+1} - g_t} (<= 1)
+            const float Ga = s_G[(2 * half) * 128 + c], Gb = s_G[(2 * half + 1) * 128 + c],
+                        Gc = s_G[(2 * half + 2) * 128 + c];
+#pragma unroll
+            for (int u = 0; u < 32; ++u) {
+                const float Gs = (u < 16) ? Ga : Gb, Gn = (u < 16) ? Gb : Gc;
+                E1[u] = __expf(gl[u] - Gs);
+                E3[u] = __expf(Gn - gl[u]);
             }
         }
-    }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-
-    // ---- MMA round 4: Bm = Ktt Ut^T -> cols [0,128)
-    if (tid == 0) {
-        mma_run(tm + 0, sb + IX_KTT, 128, sb + IY_UT, 128, CH, idesc_bf16(128, 128));
-        mma_commit(bar);
-    }
-    mbar_wait(bar, phase, a.status);
-    phase ^= 1;
-    tc_fence_after();
-    {
-        const uint32_t lane_addr = tm + ((uint32_t)(32 * qd) << 16);
-        float d0[32], d1[32];
-        tmem_ld32(lane_addr + 64 * half, d0);
-        tmem_ld32(lane_addr + 64 * half + 32, d1);
-        tmem_ld_wait();
-        uint8_t* dstB = a.ws_B + slot * SLOT_B + ((size_t)c * DV + 64 * half) * 2;
+        float G[5];
 #pragma unroll
-        for (int m = 0; m < 8; ++m) {
-            const float* src = (m < 4) ? d0 : d1;
-            const int o8 = (m & 3) * 8;
-            const uint4 pk = make_uint4(pack_bf16x2(src[o8 + 0], src[o8 + 1]), pack_bf16x2(src[o8 + 2], src[o8 + 3]),
-                                        pack_bf16x2(src[o8 + 4], src[o8 + 5]), pack_bf16x2(src[o8 + 6], src[o8 + 7]));
-            *reinterpret_cast<uint4*>(dstB + 16 * m) = pk;
+        for (int b = 0; b < 5; ++b) G[b] = s_G[b * 128 + c];
+
+        // ---- a2 operands (MN-major images, one 16-byte row = 8 consecutive tokens of channel c):
+        //      KQr = [K o E1 ; scale Q o E1],  Kd = K / E1,  Kb^(b) = K o E3 o e^{G_b - G_{bs+1}}
+        {
+            const float f21 = __expf(G[2] - G[1]), f31 = __expf(G[3] - G[1]), f32 = __expf(G[3] - G[2]);
+#pragma unroll
+            for (int m = 0; m < 4; ++m) {
+                const int tf = 32 * half + 8 * m;  // first token of this 8-token row
+                const int bt = tf >> 4;
+                float kr[8], qe[8], kd[8], k3[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const int u = 8 * m + e, t = tf + e;
+                    const float kv = raw_in<IN_BF16>(sm, R_K, a.k, ebase, rowstride, t, c, L);
+                    const float qv = raw_in<IN_BF16>(sm, R_Q, a.q, ebase, rowstride, t, c, L);
+                    if (e & 1) qr2[u >> 1] |= (uint32_t)f32_to_bf16(qv) << 16;
+                    else qr2[u >> 1] = (uint32_t)f32_to_bf16(qv);
+                    kr[e] = kv * E1[u];
+                    qe[e] = qv * E1[u] * a.scale;
+                    kd[e] = __fdividef(kv, E1[u]);  // k e^{G_bt - g_t}, <= e^80
+                    k3[e] = kv * E3[u];
+                }
+                *reinterpret_cast<uint4*>(sm + IX_KQR + mn_off(tf, c, 2048)) = pack8(kr);
+                *reinterpret_cast<uint4*>(sm + IX_KQR + mn_off(tf + 64, c, 2048)) = pack8(qe);
+                *reinterpret_cast<uint4*>(sm + IX_KD + mn_off(tf, c, 1024)) = pack8(kd);
+                if (bt <= 2) {
+                    float f[8];
+                    if (bt == 2) {
+                        *reinterpret_cast<uint4*>(sm + IX_KB3 + mn_off(tf, c, 768)) = pack8(k3);
+                    } else if (bt == 1) {
+                        *reinterpret_cast<uint4*>(sm + IX_KB2 + mn_off(tf, c, 512)) = pack8(k3);
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) f[e] = k3[e] * f32;
+                        *reinterpret_cast<uint4*>(sm + IX_KB3 + mn_off(tf, c, 768)) = pack8(f);
+                    } else {
+                        *reinterpret_cast<uint4*>(sm + IX_KB1 + mn_off(tf, c, 256)) = pack8(k3);
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) f[e] = k3[e] * f21;
+                        *reinterpret_cast<uint4*>(sm + IX_KB2 + mn_off(tf, c, 512)) = pack8(f);
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) f[e] = k3[e] * f31;
+                        *reinterpret_cast<uint4*>(sm + IX_KB3 + mn_off(tf, c, 768)) = pack8(f);
+                    }
+                }
+            }
         }
+        fence_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+
+        // ---- round 1: [Kr;Qr] Kd^T and [Kr;Qr] Kb(b)^T
+        if (tid == 0) {
+            mma_run_mn(tm + TM_AD, sb + IX_KQR, 2048, sb + IX_KD, 1024, DK, idesc_bf16_major(128, 64, 1, 1));
+            mma_run_mn(tm + TM_B1, sb + IX_KQR, 2048, sb + IX_KB1, 256, DK, idesc_bf16_major(128, 16, 1, 1));
+            mma_run_mn(tm + TM_B2, sb + IX_KQR, 2048, sb + IX_KB2, 512, DK, idesc_bf16_major(128, 32, 1, 1));
+            mma_run_mn(tm + TM_B3, sb + IX_KQR, 2048, sb + IX_KB3, 768, DK, idesc_bf16_major(128, 48, 1, 1));
+            mma_commit(bar_mma);
+        }
+        mbar_wait(bar_mma, ph_mma, a.status);
+        ph_mma ^= 1;
+        tc_fence_after();
+
+        // ---- A (rows 0..63) -> fp32 smem [64][68];  P (rows 64..127) -> bf16 image Ph [t][s]
+        //      16-column pieces, stored 16 bytes at a time
+        {
+            float* sA = reinterpret_cast<float*>(sm + IY_A);
+            const int r = 32 * qd + lane;
+            const bool isP = r >= 64;
+            const int t = r & 63, bt = t >> 4;
+            auto put16 = [&](int p, const float* d) {  // columns [16p, 16p + 16)
+                if (isP) {
+                    *reinterpret_cast<uint4*>(sm + IX_PH + sw128_off(t, 16 * p)) = pack8(d);
+                    *reinterpret_cast<uint4*>(sm + IX_PH + sw128_off(t, 16 * p + 8)) = pack8(d + 8);
+                } else {
+                    float4* dst = reinterpret_cast<float4*>(sA + t * LDA + 16 * p);
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) dst[i] = make_float4(d[4 * i], d[4 * i + 1], d[4 * i + 2], d[4 * i + 3]);
+                }
+            };
+            if (half == 0) {
+                // diagonal tile (masked: A strictly lower, P lower) and the zero upper part
+#pragma unroll
+                for (int p = 0; p < 4; ++p) {
+                    float d[16];
+                    tmem_ld16(lane_addr + TM_AD + 16 * p, d);
+                    tmem_ld_wait();
+                    if (p >= bt) {
+#pragma unroll
+                        for (int s16 = 0; s16 < 16; ++s16) {
+                            const int s = 16 * p + s16;
+                            const bool keep = (p == bt) && (isP ? (s <= t) : (s < t));
+                            d[s16] = keep ? d[s16] : 0.f;
+                        }
+                        put16(p, d);
+                    }
+                }
+            } else if ((qd & 1) == 0) {  // rows t in [0, 32): tiles 0 and 1
+                float d[16];
+                tmem_ld16(lane_addr + TM_B1, d);
+                tmem_ld_wait();
+                if (bt == 1) put16(0, d);
+            } else {  // rows t in [32, 64): tiles 2 and 3; off-diagonal column tiles p < bt
+#pragma unroll
+                for (int p = 0; p < 3; ++p) {
+                    float d2[16], d3[16];
+                    if (p < 2) tmem_ld16(lane_addr + TM_B2 + 16 * p, d2);
+                    tmem_ld16(lane_addr + TM_B3 + 16 * p, d3);
+                    tmem_ld_wait();
+                    if (bt == 2 && p < 2) put16(p, d2);
+                    if (bt == 3) put16(p, d3);
+                }
+            }
+        }
+        __syncthreads();
+
+        // ---- a3: T = (I + Diag(beta) A)^-1 Diag(beta), fp32, blocked on 16x16 tiles
+        {
+            float* sA = reinterpret_cast<float*>(sm + IY_A);  // becomes N = Diag(beta) A in place
+            float* sX = reinterpret_cast<float*>(sm + IY_X);  // X = (I + N)^-1
+            float* sY = reinterpret_cast<float*>(sm + IX_TMP);
+            for (int e = tid; e < 64 * 64; e += 256) {
+                const int i = e >> 6, j = e & 63;
+                sA[i * LDA + j] *= s_beta[i];
+            }
+            __syncthreads();
+            if (tid < 64) {  // diagonal blocks: one thread per (block, column)
+                const int b = tid >> 4, j = tid & 15;
+                const float* Nb = sA + (16 * b) * LDA + 16 * b;
+                float x[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    float acc = 0.f;
+#pragma unroll
+                    for (int m = 0; m < i; ++m)
+                        if (m >= j) acc += Nb[i * LDA + m] * x[m];
+                    x[i] = (i < j) ? 0.f : ((i == j) ? 1.f : -acc);
+                }
+#pragma unroll
+                for (int i = 0; i < 16; ++i) sX[(16 * b + i) * LDA + 16 * b + j] = x[i];
+            }
+            for (int e = tid; e < 64 * 64; e += 256) {
+                const int i = e >> 6, j = e & 63;
+                if ((j >> 4) > (i >> 4)) sX[i * LDA + j] = 0.f;
+            }
+            __syncthreads();
+            // off-diagonal blocks by distance d:  X_ij = -X_ii * sum_{m=j}^{i-1} N_im X_mj
+            for (int d = 1; d <= 3; ++d) {
+                const int nblk = 4 - d;
+                for (int e = tid; e < nblk * 256; e += 256) {
+                    const int p = e >> 8, r = (e >> 4) & 15, cc = e & 15;
+                    const int bj = p, bi = p + d;
+                    float acc = 0.f;
+                    for (int m = bj; m < bi; ++m) {
+#pragma unroll
+                        for (int uu = 0; uu < 16; ++uu)
+                            acc += sA[(16 * bi + r) * LDA + 16 * m + uu] * sX[(16 * m + uu) * LDA + 16 * bj + cc];
+                    }
+                    sY[p * 256 + r * 16 + cc] = acc;
+                }
+                __syncthreads();
+                for (int e = tid; e < nblk * 256; e += 256) {
+                    const int p = e >> 8, r = (e >> 4) & 15, cc = e & 15;
+                    const int bj = p, bi = p + d;
+                    float acc = 0.f;
+#pragma unroll
+                    for (int uu = 0; uu < 16; ++uu)
+                        acc += sX[(16 * bi + r) * LDA + 16 * bi + uu] * sY[p * 256 + uu * 16 + cc];
+                    sX[(16 * bi + r) * LDA + 16 * bj + cc] = -acc;
+                }
+                __syncthreads();
+            }
+            for (int e = tid; e < 64 * 8; e += 256) {  // T = X Diag(beta) -> bf16 image Ti [t][s], 8 s per store
+                const int t = e >> 3, s0 = (e & 7) * 8;
+                const float4 x0 = *reinterpret_cast<const float4*>(sX + t * LDA + s0);
+                const float4 x1 = *reinterpret_cast<const float4*>(sX + t * LDA + s0 + 4);
+                const float4 b0 = *reinterpret_cast<const float4*>(s_beta + s0);
+                const float4 b1 = *reinterpret_cast<const float4*>(s_beta + s0 + 4);
+                const float v8[8] = {x0.x * b0.x, x0.y * b0.y, x0.z * b0.z, x0.w * b0.w,
+                                     x1.x * b1.x, x1.y * b1.y, x1.z * b1.z, x1.w * b1.w};
+                *reinterpret_cast<uint4*>(sm + IX_TI + sw128_off(t, s0)) = pack8(v8);
+            }
+        }
+
+        // ---- phase 2 operands (K = token): KGt = (K o Gam)^T, Vt = V^T, Ktt = Kt^T
+        {
+            const float eG[2] = {__expf(half ? G[2] : G[0]), __expf(half ? G[3] : G[1])};
+            const float eC[2] = {__expf(G[4] - (half ? G[3] : G[1])), __expf(G[4] - (half ? G[4] : G[2]))};
+#pragma unroll
+            for (int m = 0; m < 4; ++m) {  // 8 consecutive tokens per 16-byte chunk
+                float kg[8], vv[8], kt[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const int u = 8 * m + e;
+                    const int t = 32 * half + u;
+                    const float kv = raw_in<IN_BF16>(sm, R_K, a.k, ebase, rowstride, t, c, L);
+                    vv[e] = raw_in<IN_BF16>(sm, R_V, a.v, vbase, (size_t)H * DV, t, c, L);
+                    kg[e] = kv * E1[u] * eG[u >> 4];
+                    kt[e] = kv * E3[u] * eC[u >> 4];
+                }
+                const uint32_t off = sw128_off((uint32_t)c, (uint32_t)(32 * half + 8 * m));
+                *reinterpret_cast<uint4*>(sm + IX_KGT + off) = pack8(kg);
+                *reinterpret_cast<uint4*>(sm + IX_VT + off) = pack8(vv);
+                *reinterpret_cast<uint4*>(sm + IX_KTT + off) = pack8(kt);
+            }
+            if (half == 1) *reinterpret_cast<float*>(wslot + SO_G + 4 * c) = __expf(G[4]);
+        }
+        fence_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+
+        // next item's raw tiles: every read of RAW for this item is done
+        const int64_t next = next_valid(item + gridDim.x);
+        if constexpr (IN_BF16) {
+            if (tid == 0 && next < n_items) issue_raw(next);
+            raw_in_flight = next < n_items;
+        }
+
+        // ---- round 2: Wt = KGt Ti^T, Ut = Vt Ti^T
+        if (tid == 0) {
+            mma_run(tm + TM_WT, sb + IX_KGT, 128, sb + IX_TI, 64, CH, idesc_bf16(128, 64));
+            mma_run(tm + TM_UT, sb + IX_VT, 128, sb + IX_TI, 64, CH, idesc_bf16(128, 64));
+            mma_commit(bar_mma);
+        }
+        mbar_wait(bar_mma, ph_mma, a.status);
+        ph_mma ^= 1;
+        tc_fence_after();
+        {
+            // half 0 -> Wt image, half 1 -> Ut image; row = channel c, 64 token columns
+            const uint32_t col0 = half ? TM_UT : TM_WT;
+            const uint32_t dst = half ? IY_UT : IY_WT;
+#pragma unroll
+            for (int p = 0; p < 4; ++p) {
+                float d[16];
+                tmem_ld16(lane_addr + col0 + 16 * p, d);
+                tmem_ld_wait();
+                *reinterpret_cast<uint4*>(sm + dst + sw128_off((uint32_t)c, (uint32_t)(16 * p))) = pack8(d);
+                *reinterpret_cast<uint4*>(sm + dst + sw128_off((uint32_t)c, (uint32_t)(16 * p + 8))) = pack8(d + 8);
+            }
+        }
+        fence_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+
+        // ---- round 3: Mlr = Ktt Wt^T, Bm = Ktt Ut^T, (P W)^T = Wt Ph^T, Ob^T = Ut Ph^T
+        if (tid == 0) {
+            mma_run(tm + TM_M, sb + IX_KTT, 128, sb + IY_WT, 128, CH, idesc_bf16(128, 128));
+            mma_run(tm + TM_PW, sb + IY_WT, 128, sb + IX_PH, 64, CH, idesc_bf16(128, 64));
+            mma_run(tm + TM_BM, sb + IX_KTT, 128, sb + IY_UT, 128, CH, idesc_bf16(128, 128));
+            mma_run(tm + TM_OB, sb + IY_UT, 128, sb + IX_PH, 64, CH, idesc_bf16(128, 64));
+            mma_commit(bar_mma);
+        }
+        mbar_wait(bar_mma, ph_mma, a.status);
+        ph_mma ^= 1;
+        tc_fence_after();
+        {
+            // Mlr row c -> K-major SW128 image (half h writes K block h)
+            {
+                uint8_t* dstM = wslot + SO_M + (size_t)half * (DK * 128);
+#pragma unroll
+                for (int p = 0; p < 4; ++p) {
+                    float d[16];
+                    tmem_ld16(lane_addr + TM_M + 64 * half + 16 * p, d);
+                    tmem_ld_wait();
+                    *reinterpret_cast<uint4*>(dstM + sw128_off((uint32_t)c, (uint32_t)(16 * p))) = pack8(d);
+                    *reinterpret_cast<uint4*>(dstM + sw128_off((uint32_t)c, (uint32_t)(16 * p + 8))) = pack8(d + 8);
+                }
+            }
+            // Bm row c, value columns [64 half, 64 half + 64) -> slices 2 half, 2 half + 1
+            {
+#pragma unroll
+                for (int p = 0; p < 4; ++p) {  // columns 64 half + 16 p .. +16 -> slice 2 half + p / 2
+                    float d[16];
+                    tmem_ld16(lane_addr + TM_BM + 64 * half + 16 * p, d);
+                    tmem_ld_wait();
+                    uint4* dstB = reinterpret_cast<uint4*>(wslot + SO_B + (size_t)(2 * half + (p >> 1)) * BSL +
+                                                           (size_t)c * DVS * 2) + 2 * (p & 1);
+                    dstB[0] = pack8(d);
+                    dstB[1] = pack8(d + 8);
+                }
+            }
+            // Qp^T[c][t] = scale q_tc e^{g_tc} - (P W)^T[c][t] -> MN-major image (token-contiguous rows);
+            // Ob^T[j][t] -> slice j/32, row j%32 (64 tokens).  16 bytes per store.
+            {
+                const float eG[2] = {__expf(half ? G[2] : G[0]), __expf(half ? G[3] : G[1])};
+                uint8_t* dstQ = wslot + SO_Q;
+                uint8_t* dstO = wslot + SO_O + (size_t)(c >> 5) * OSL + (size_t)(c & 31) * (CH * 2);
+#pragma unroll
+                for (int p = 0; p < 2; ++p) {
+                    float pw[16], ob[16], qq[16];
+                    tmem_ld16(lane_addr + TM_PW + 32 * half + 16 * p, pw);
+                    tmem_ld16(lane_addr + TM_OB + 32 * half + 16 * p, ob);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        const int u = 16 * p + e;
+                        const float qv =
+                            __uint_as_float((u & 1) ? (qr2[u >> 1] & 0xFFFF0000u) : (qr2[u >> 1] << 16));
+                        qq[e] = qv * E1[u] * eG[p] * a.scale - pw[e];
+                    }
+                    const int tf = 32 * half + 16 * p;
+                    *reinterpret_cast<uint4*>(dstQ + mn_off(tf, c, 1024)) = pack8(qq);
+                    *reinterpret_cast<uint4*>(dstQ + mn_off(tf + 8, c, 1024)) = pack8(qq + 8);
+                    *reinterpret_cast<uint4*>(dstO + tf * 2) = pack8(ob);
+                    *reinterpret_cast<uint4*>(dstO + tf * 2 + 16) = pack8(ob + 8);
+                }
+            }
+        }
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+        item = next;
     }
-    tc_fence_before();
+    // a prefetch can only be in flight here after a failed wait; let it land
+    if constexpr (IN_BF16) {
+        if (tid == 0 && raw_in_flight) mbar_wait(bar_raw, ph_raw, nullptr);
+    }
     __syncthreads();
     if (warp == 0) {
         tc_fence_after();
@@ -550,17 +645,18 @@ __global__ void __launch_bounds__(256, 2) intra_kernel(const ChunkArgs a) {
 // chain_kernel
 // ---------------------------------------------------------------------------
 // Threads: 128; thread c owns state row c of the 32-column slice (32 fp32
-// registers).  TMEM: 64 columns, D_S = Mlr S in [0,32) (M=128, lane = row c),
-// D_O = Qp S in [32,64) (M=64: row t lives in lane 32*(t/16) + t%16).
-// Shared memory: two buffers {Mlr image 32K, Qp image 16K}, the bf16 state
-// operand Sb [32 value cols][128 key rows] (8K), two load barriers and one
-// MMA barrier.
-constexpr uint32_t CB_M = 0, CB_Q = 32768, CB_SIZE = 49152;
-constexpr uint32_t C_SB = 2 * CB_SIZE;            // 98304
-constexpr uint32_t C_BAR = C_SB + 8192;            // 106496
-constexpr uint32_t C_TMEM = C_BAR + 24;
-constexpr uint32_t CHAIN_SMEM = C_TMEM + 8 + 1024;
-constexpr uint32_t CHAIN_TMEM_COLS = 64;
+// registers).  TMEM (128 columns): D_S = Mlr S in [0,32) (M=128, lane = row
+// c); D_O = Qp S double-buffered in [32,64) and [64,96) (M=64: row t lives in
+// lane 32*(t/16) + t%16).  Shared memory: two chunk buffers {Mlr image 32K,
+// Qp image 16K, GamC 512, Bm slice 8K, Ob slice 4K} and two bf16 state
+// operand images Sb [32 value cols][128 key rows] (8K each).
+constexpr uint32_t CB_M = 0, CB_Q = 32768, CB_G = 49152, CB_B = 49664, CB_O = 57856, CB_SIZE = 62464;
+constexpr uint32_t C_SB = 2 * CB_SIZE;        // two 8K state images
+constexpr uint32_t C_BAR = C_SB + 2 * 8192;   // bar_ld[2], bar_s, bar_o[2]
+constexpr uint32_t C_FLAG = C_BAR + 40;
+constexpr uint32_t C_TMEM = C_FLAG + 16;
+constexpr uint32_t CHAIN_SMEM = C_TMEM + 16 + 1024;
+constexpr uint32_t CHAIN_TMEM_COLS = 128;
 
 template <bool OUT_BF16>
 __global__ void __launch_bounds__(128, 1) chain_kernel(const ChunkArgs a) {
@@ -568,10 +664,15 @@ __global__ void __launch_bounds__(128, 1) chain_kernel(const ChunkArgs a) {
     uint8_t* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     const uint32_t sbase = smem_u32(sm);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int n = blockIdx.x, h = blockIdx.y, js = blockIdx.z;
+    const int js = blockIdx.x, h = blockIdx.y, n = blockIdx.z;
     const int H = a.H;
-    uint64_t* bar_ld = reinterpret_cast<uint64_t*>(sm + C_BAR);       // [2]
-    uint64_t* bar_mma = reinterpret_cast<uint64_t*>(sm + C_BAR + 16);
+    uint64_t* bar_ld = reinterpret_cast<uint64_t*>(sm + C_BAR);  // [2]
+    uint64_t* bar_s = reinterpret_cast<uint64_t*>(sm + C_BAR + 16);
+    // one output barrier per D_O buffer: the next chunk's output product is
+    // committed before this chunk's output is waited for, so a single barrier
+    // could complete two phases between waits
+    uint64_t* bar_o = reinterpret_cast<uint64_t*>(sm + C_BAR + 24);  // [2]
+    volatile int* s_fail = reinterpret_cast<volatile int*>(sm + C_FLAG);
     uint32_t* s_tmem = reinterpret_cast<uint32_t*>(sm + C_TMEM);
 
     int64_t s_beg, s_end;
@@ -581,7 +682,7 @@ __global__ void __launch_bounds__(128, 1) chain_kernel(const ChunkArgs a) {
     const int c_end = min(a.i0 + a.wc, nchunks);
     const int nit = c_end > c_beg ? c_end - c_beg : 0;
 
-    // state slice row c, columns [32 js, 32 js + 32)
+    // state slice: row tid, columns [32 js, 32 js + 32)
     const size_t st_off = (((size_t)n * H + h) * DK + tid) * DV + (size_t)DVS * js;
     float S[DVS];
     {
@@ -606,126 +707,163 @@ __global__ void __launch_bounds__(128, 1) chain_kernel(const ChunkArgs a) {
         if (tid == 0) {
             mbar_init(&bar_ld[0], 1);
             mbar_init(&bar_ld[1], 1);
-            mbar_init(bar_mma, 1);
+            mbar_init(bar_s, 1);
+            mbar_init(&bar_o[0], 1);
+            mbar_init(&bar_o[1], 1);
             fence_mbar_init();
+            *s_fail = 0;
         }
         __syncthreads();
         tc_fence_after();
         const uint32_t tm = *s_tmem;
-        auto slot_of = [&](int cidx) -> size_t { return ((size_t)n * a.wc + (cidx - a.i0)) * H + h; };
+        const uint32_t lane_addr = tm + ((uint32_t)(32 * warp) << 16);
+        const size_t slot0 = ((size_t)n * a.wc + (c_beg - a.i0)) * H + h;  // slot of iteration 0
         auto issue_load = [&](int it) {
-            const int b = it & 1;
-            const size_t sl = slot_of(c_beg + it);
-            mbar_arrive_expect_tx(&bar_ld[b], (uint32_t)(SLOT_M + SLOT_Q));
-            bulk_g2s(sm + b * CB_SIZE + CB_M, a.ws_M + sl * SLOT_M, (uint32_t)SLOT_M, &bar_ld[b]);
-            bulk_g2s(sm + b * CB_SIZE + CB_Q, a.ws_Q + sl * SLOT_Q, (uint32_t)SLOT_Q, &bar_ld[b]);
+            uint8_t* buf = sm + (it & 1) * CB_SIZE;
+            const uint8_t* src = a.ws + (slot0 + (size_t)it * H) * SLOT_BYTES;
+            mbar_arrive_expect_tx(&bar_ld[it & 1], SO_MQG + BSL + OSL);
+            bulk_g2s(buf + CB_M, src + SO_M, SO_MQG, &bar_ld[it & 1]);
+            bulk_g2s(buf + CB_B, src + SO_B + (size_t)js * BSL, BSL, &bar_ld[it & 1]);
+            bulk_g2s(buf + CB_O, src + SO_O + (size_t)js * OSL, OSL, &bar_ld[it & 1]);
         };
-        if (tid == 0) issue_load(0);
+        auto write_state_image = [&](int it) {
+            const uint32_t kb = (uint32_t)tid >> 6, kc = (uint32_t)tid & 63u;
+            uint8_t* img = sm + C_SB + (it & 1) * 8192;
+#pragma unroll
+            for (int j = 0; j < DVS; ++j)
+                *reinterpret_cast<uint16_t*>(img + kb * (DVS * 128) + sw128_off((uint32_t)j, kc)) = f32_to_bf16(S[j]);
+        };
+        // thread 0: Mlr S -> D_S (commit bar_s), then Qp S -> D_O[it&1] (commit bar_o[it&1])
+        auto issue_mma = [&](int it) -> bool {
+            const int b = it & 1;
+            if (!mbar_wait(&bar_ld[b], (uint32_t)((it >> 1) & 1), a.status)) return false;
+            tc_fence_after();
+            const uint32_t img = sbase + C_SB + (it & 1) * 8192;
+            mma_run(tm + 0, sbase + b * CB_SIZE + CB_M, 128, img, DVS, DK, idesc_bf16(128, DVS));
+            mma_commit(bar_s);
+            {  // Qp (MN-major, no swizzle) x state image (K-major SW128)
+                const uint32_t qa = sbase + b * CB_SIZE + CB_Q;
+                for (int kk = 0; kk < DK / 16; ++kk) {
+                    const uint64_t ad = sdesc_interleave(qa + (uint32_t)kk * 2048u, 1024u, 128u);
+                    const uint64_t bd = sdesc_k_sw128(img + (uint32_t)(kk >> 2) * (DVS * 128u) + (uint32_t)(kk & 3) * 32u);
+                    mma_bf16(tm + 32 + 32 * (it & 1), ad, bd, idesc_bf16_major(64, DVS, 1, 0), kk > 0 ? 1u : 0u);
+                }
+            }
+            mma_commit(&bar_o[it & 1]);
+            return true;
+        };
 
-        bool ok = true;
+        // thread-0 bookkeeping for the bounded drain after a failed wait
+        int loads_issued = 0, loads_waited = 0, mma_issued = 0;
+        if (tid == 0) {
+            issue_load(0);
+            loads_issued = 1;
+            if (nit > 1) {
+                issue_load(1);
+                loads_issued = 2;
+            }
+        }
+        write_state_image(0);
+        fence_async_smem();
+        __syncthreads();
+        tc_fence_after();
+        if (tid == 0) {
+            loads_waited = 1;
+            if (issue_mma(0)) mma_issued = 1;
+            else *s_fail = 1;
+        }
+        __syncthreads();
+
         int it = 0;
-        for (; it < nit && ok; ++it) {
-            const int cidx = c_beg + it;
-            const size_t sl = slot_of(cidx);
-            const int64_t t0 = s_beg + (int64_t)cidx * CH;
+        for (; it < nit && !*s_fail; ++it) {
+            const int b = it & 1;
+            const uint8_t* buf = sm + b * CB_SIZE;
+            const int64_t t0 = s_beg + (int64_t)(c_beg + it) * CH;
             const int L = (int)((s_end - t0) < CH ? (s_end - t0) : CH);
-            if (tid == 0 && it + 1 < nit) issue_load(it + 1);
 
-            // per-chunk inputs of this thread: Bm row slice, Gam_C, Ob row slice
-            float bm[DVS];
-            {
-                const uint4* src = reinterpret_cast<const uint4*>(a.ws_B + sl * SLOT_B + ((size_t)tid * DV + DVS * js) * 2);
+            // (1) state update: S <- GamC o S - Mlr S + Bm
+            if (mbar_wait(bar_s, (uint32_t)(it & 1), a.status)) {
+                tc_fence_after();
+                float ds[DVS];
+                tmem_ld32(lane_addr + 0, ds);
+                tmem_ld_wait();
+                const float gamC = *reinterpret_cast<const float*>(buf + CB_G + 4 * tid);
+                const uint4* bsrc = reinterpret_cast<const uint4*>(buf + CB_B + (uint32_t)tid * DVS * 2);
 #pragma unroll
                 for (int m = 0; m < DVS / 8; ++m) {
-                    const uint4 w = __ldg(src + m);
+                    const uint4 w = bsrc[m];
                     const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
                     for (int p = 0; p < 4; ++p) {
-                        bm[8 * m + 2 * p] = __uint_as_float(ww[p] << 16);
-                        bm[8 * m + 2 * p + 1] = __uint_as_float(ww[p] & 0xFFFF0000u);
+                        const int j = 8 * m + 2 * p;
+                        S[j] = gamC * S[j] - ds[j] + __uint_as_float(ww[p] << 16);
+                        S[j + 1] = gamC * S[j + 1] - ds[j + 1] + __uint_as_float(ww[p] & 0xFFFF0000u);
                     }
                 }
+            } else {
+                *s_fail = 1;
             }
-            const float gamC = __ldg(a.ws_G + sl * DK + tid);
-            const int trow = 16 * warp + (lane & 15);  // output row served by this lane (lane < 16)
-            float obv[DVS];
-            if (lane < 16) {
-                const uint4* src = reinterpret_cast<const uint4*>(a.ws_O + sl * SLOT_O + ((size_t)trow * DV + DVS * js) * 2);
-#pragma unroll
-                for (int m = 0; m < DVS / 8; ++m) {
-                    const uint4 w = __ldg(src + m);
-                    const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-                    for (int p = 0; p < 4; ++p) {
-                        obv[8 * m + 2 * p] = __uint_as_float(ww[p] << 16);
-                        obv[8 * m + 2 * p + 1] = __uint_as_float(ww[p] & 0xFFFF0000u);
-                    }
-                }
-            }
-
-            // state operand Sb[j][c] = bf16(S[c][j]) (K-major: row = value col j, K = key row c)
-            {
-                const uint32_t kb = (uint32_t)tid >> 6, kc = (uint32_t)tid & 63u;
-#pragma unroll
-                for (int j = 0; j < DVS; ++j)
-                    *reinterpret_cast<uint16_t*>(sm + C_SB + kb * (DVS * 128) + sw128_off((uint32_t)j, kc)) =
-                        f32_to_bf16(S[j]);
-            }
+            // (2) next chunk's products as early as possible
+            if (it + 1 < nit) write_state_image(it + 1);
             fence_async_smem();
             tc_fence_before();
             __syncthreads();
             tc_fence_after();
-            if (tid == 0) {
-                const int b = it & 1;
-                if (mbar_wait(&bar_ld[b], (uint32_t)((it >> 1) & 1), a.status)) {
-                    tc_fence_after();
-                    mma_run(tm + 0, sbase + b * CB_SIZE + CB_M, 128, sbase + C_SB, DVS, DK, idesc_bf16(128, DVS));
-                    mma_run(tm + 32, sbase + b * CB_SIZE + CB_Q, 64, sbase + C_SB, DVS, DK, idesc_bf16(64, DVS));
-                }
-                mma_commit(bar_mma);
+            if (*s_fail) break;
+            if (tid == 0 && it + 1 < nit) {
+                loads_waited = it + 2;
+                if (issue_mma(it + 1)) mma_issued = it + 2;
+                else *s_fail = 1;
             }
-            ok = mbar_wait(bar_mma, (uint32_t)(it & 1), a.status);
-            tc_fence_after();
-            if (!ok) {
-                // a wait gave up: let the prefetch in flight land before leaving
-                if (tid == 0 && it + 1 < nit) mbar_wait(&bar_ld[(it + 1) & 1], (uint32_t)(((it + 1) >> 1) & 1), nullptr);
-                break;
-            }
-
-            const uint32_t lane_addr = tm + ((uint32_t)(32 * warp) << 16);
-            float ds[DVS], dO[DVS];
-            tmem_ld32(lane_addr + 0, ds);
-            tmem_ld32(lane_addr + 32, dO);
-            tmem_ld_wait();
-#pragma unroll
-            for (int j = 0; j < DVS; ++j) S[j] = gamC * S[j] - ds[j] + bm[j];
-            if (lane < 16 && trow < L) {
-                const size_t obase = ((size_t)(t0 + trow) * H + h) * DV + (size_t)DVS * js;
-                if constexpr (OUT_BF16) {
-                    uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(a.o) + obase);
+            // (3) this chunk's output: o = Qp S + Ob
+            if (mbar_wait(&bar_o[it & 1], (uint32_t)((it >> 1) & 1), a.status)) {
+                tc_fence_after();
+                float dO[DVS];
+                tmem_ld32(lane_addr + 32 + 32 * (it & 1), dO);
+                tmem_ld_wait();
+                const int trow = 16 * warp + (lane & 15);
+                if (lane < 16 && trow < L) {
+                    // Ob^T slice [32 value cols][64 tokens]: column trow
+                    const uint16_t* osrc = reinterpret_cast<const uint16_t*>(buf + CB_O) + trow;
+                    const size_t obase = ((size_t)(t0 + trow) * H + h) * DV + (size_t)DVS * js;
 #pragma unroll
                     for (int m = 0; m < DVS / 8; ++m) {
-                        const int j = 8 * m;
-                        dst[m] = make_uint4(pack_bf16x2(dO[j] + obv[j], dO[j + 1] + obv[j + 1]),
-                                            pack_bf16x2(dO[j + 2] + obv[j + 2], dO[j + 3] + obv[j + 3]),
-                                            pack_bf16x2(dO[j + 4] + obv[j + 4], dO[j + 5] + obv[j + 5]),
-                                            pack_bf16x2(dO[j + 6] + obv[j + 6], dO[j + 7] + obv[j + 7]));
-                    }
-                } else {
-                    float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(a.o) + obase);
+                        float y8[8];
 #pragma unroll
-                    for (int m = 0; m < DVS / 4; ++m) {
-                        const int j = 4 * m;
-                        dst[m] = make_float4(dO[j] + obv[j], dO[j + 1] + obv[j + 1], dO[j + 2] + obv[j + 2],
-                                             dO[j + 3] + obv[j + 3]);
+                        for (int p = 0; p < 8; ++p) y8[p] = dO[8 * m + p] + bf16_to_f32(osrc[(8 * m + p) * CH]);
+                        if constexpr (OUT_BF16) {
+                            reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(a.o) + obase)[m] = pack8(y8);
+                        } else {
+                            float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(a.o) + obase) + 2 * m;
+                            dst[0] = make_float4(y8[0], y8[1], y8[2], y8[3]);
+                            dst[1] = make_float4(y8[4], y8[5], y8[6], y8[7]);
+                        }
                     }
                 }
+            } else {
+                *s_fail = 1;
             }
+            // (4) buffer b fully consumed -> refill it with chunk it + 2
             tc_fence_before();
             __syncthreads();
+            if (tid == 0 && it + 2 < nit && !*s_fail) {
+                issue_load(it + 2);
+                loads_issued = it + 3;
+            }
         }
-        tc_fence_after();
+        // after a failed wait: let copies and products still in flight finish (bounded)
+        if (tid == 0 && *s_fail) {
+            for (int j = loads_waited; j < loads_issued; ++j)
+                mbar_wait(&bar_ld[j & 1], (uint32_t)((j >> 1) & 1), nullptr);
+            if (mma_issued > 0) {
+                const int j = mma_issued - 1;
+                mbar_wait(bar_s, (uint32_t)(j & 1), nullptr);
+                mbar_wait(&bar_o[j & 1], (uint32_t)((j >> 1) & 1), nullptr);
+            }
+        }
+        tc_fence_before();
         __syncthreads();
+        tc_fence_after();
         if (warp == 0) tmem_dealloc(tm, CHAIN_TMEM_COLS);
     }
 
@@ -748,7 +886,7 @@ __global__ void check_cu_kernel(const int32_t* cu, int n_seqs, int64_t T, int64_
 
 // ------------------------------------------------------------- host side --
 
-size_t chunk_slot_bytes() { return SLOT_M + SLOT_Q + SLOT_B + SLOT_O + SLOT_G; }
+size_t chunk_slot_bytes() { return SLOT_BYTES; }
 
 // Fixed part of the workspace: status word (256 B) + state carry when the
 // caller does not ask for the final state.
@@ -758,7 +896,37 @@ size_t chunk_fixed_bytes(int n_seqs, int H, bool need_carry) {
     return b;
 }
 
-static bool g_attr_set = false;
+namespace {
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (fn == nullptr) {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    }
+    return fn;
+}
+
+// [rows, row_elems] bf16 tensor, box = 64 rows x 128 elements, no swizzle.
+bool make_tile_map(CUtensorMap* m, const void* base, int64_t rows, int64_t row_elems) {
+    auto enc = tensor_map_encoder();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)row_elems, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)row_elems * 2};
+    cuuint32_t box[2] = {128, 64};
+    cuuint32_t estr[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool g_attr_set = false;
+int g_num_sms = 0;
+
+}  // namespace
 
 cudaError_t chunk_fwd_launch(const void* q, const void* k, const void* v, const void* log_alpha, const void* beta,
                              const float* init_state, void* o, float* final_state, int B, int64_t T, int H,
@@ -774,35 +942,42 @@ cudaError_t chunk_fwd_launch(const void* q, const void* k, const void* v, const 
         if (err != cudaSuccess) return err;
         err = cudaFuncSetAttribute(chain_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, CHAIN_SMEM);
         if (err != cudaSuccess) return err;
+        int dev = 0;
+        if ((err = cudaGetDevice(&dev)) != cudaSuccess) return err;
+        if ((err = cudaDeviceGetAttribute(&g_num_sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return err;
         g_attr_set = true;
     }
     const int N = cu ? n_seqs : B;
-    const int64_t seqT = cu ? T : T;  // tokens per sequence (fixed) / total (varlen)
     const int64_t maxlen = cu ? max_seqlen : T;
+    const int64_t total_tokens = cu ? T : (int64_t)B * T;
     const int nchunks_max = (int)((maxlen + CH - 1) / CH);
     uint8_t* ws = reinterpret_cast<uint8_t*>(workspace);
     uint32_t* status = reinterpret_cast<uint32_t*>(ws);
     const bool need_carry = final_state == nullptr;
     const size_t fixed = chunk_fixed_bytes(N, H, need_carry);
     float* carry = need_carry ? reinterpret_cast<float*>(ws + 256) : final_state;
-    const size_t per_wc = (size_t)N * H * chunk_slot_bytes();
+    const size_t per_wc = (size_t)N * H * SLOT_BYTES;
     const size_t head = (fixed + 1023) & ~(size_t)1023;
     const size_t wc_fit = ws_bytes > head ? (ws_bytes - head) / per_wc : 0;
     int wc = (int)(wc_fit < (size_t)nchunks_max ? wc_fit : (size_t)nchunks_max);
     if (wc < 1) wc = 1;
-    const size_t slots = (size_t)N * wc * H;
-    uint8_t* p = ws + head;
     ChunkArgs a;
     a.q = q; a.k = k; a.v = v; a.log_alpha = log_alpha; a.beta = beta;
     a.init_state = init_state; a.state_io = carry; a.o = o; a.cu = cu;
-    a.ws_M = p; p += slots * SLOT_M;
-    a.ws_Q = p; p += slots * SLOT_Q;
-    a.ws_B = p; p += slots * SLOT_B;
-    a.ws_O = p; p += slots * SLOT_O;
-    a.ws_G = reinterpret_cast<float*>(p);
+    a.ws = ws + head;
     a.status = status;
-    a.T = cu ? T : seqT;
+    a.T = T;
     a.H = H; a.n_seqs = N; a.wc = wc; a.scale = scale;
+
+    IntraMaps maps;
+    memset(&maps, 0, sizeof(maps));
+    if (in_bf16 && total_tokens > 0) {
+        if (!make_tile_map(&maps.la, log_alpha, total_tokens, (int64_t)H * DK) ||
+            !make_tile_map(&maps.k, k, total_tokens, (int64_t)H * DK) ||
+            !make_tile_map(&maps.q, q, total_tokens, (int64_t)H * DK) ||
+            !make_tile_map(&maps.v, v, total_tokens, (int64_t)H * DV))
+            return cudaErrorInvalidValue;
+    }
 
     err = cudaMemsetAsync(status, 0, 4, stream);
     if (err != cudaSuccess) return err;
@@ -818,14 +993,15 @@ cudaError_t chunk_fwd_launch(const void* q, const void* k, const void* v, const 
         a.i0 = ps * wc;
         a.first_pass = ps == 0;
         if (nchunks_max > 0) {
-            const dim3 gi((unsigned)(N * wc), (unsigned)H);
+            const int64_t n_items = (int64_t)N * wc * H;
+            const unsigned grid = (unsigned)(n_items < g_num_sms ? n_items : g_num_sms);
             prof_begin(PROF_INTRA, stream);
-            if (in_bf16) intra_kernel<true><<<gi, 256, INTRA_SMEM, stream>>>(a);
-            else intra_kernel<false><<<gi, 256, INTRA_SMEM, stream>>>(a);
+            if (in_bf16) intra_kernel<true><<<grid, 256, INTRA_SMEM, stream>>>(a, maps, n_items);
+            else intra_kernel<false><<<grid, 256, INTRA_SMEM, stream>>>(a, maps, n_items);
             if ((err = cudaGetLastError()) != cudaSuccess) return err;
             prof_end(PROF_INTRA, stream);
         }
-        const dim3 gc((unsigned)N, (unsigned)H, (unsigned)(DV / DVS));
+        const dim3 gc((unsigned)NSL, (unsigned)H, (unsigned)N);
         prof_begin(PROF_CHAIN, stream);
         if (out_bf16) chain_kernel<true><<<gc, 128, CHAIN_SMEM, stream>>>(a);
         else chain_kernel<false><<<gc, 128, CHAIN_SMEM, stream>>>(a);

@@ -3,6 +3,7 @@
 // shared-memory matrix descriptors, bf16 helpers and bounded waits.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -85,6 +86,17 @@ KDA_DEV void bulk_g2s(void* smem_dst, const void* gmem_src, uint32_t bytes, uint
         : "memory");
 }
 
+// 2-D tiled TMA load of box (x, y) of a tensor map into shared memory,
+// completion signalled on `bar`.  x is the innermost coordinate (elements);
+// x * element size must be a multiple of 16 bytes.
+KDA_DEV void tma_load_2d(void* smem_dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
+        "[%4];" ::"r"(smem_u32(smem_dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
+        : "memory");
+}
+
 // 1-D bulk copy shared -> global (bulk async-group completion).
 KDA_DEV void bulk_s2g(void* gmem_dst, const void* smem_src, uint32_t bytes) {
     asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(gmem_dst),
@@ -160,6 +172,33 @@ KDA_DEV uint64_t sdesc_k_sw128(uint32_t addr) {
     d |= (uint64_t)1u << 46;                          // descriptor version (sm_100)
     d |= (uint64_t)2u << 61;                          // layout: SWIZZLE_128B
     return d;
+}
+
+// Shared-memory matrix descriptor for an operand in the no-swizzle
+// ("interleaved") canonical layout: core matrices of 8 rows x 16 bytes, each
+// 128 contiguous bytes.  For a K-major operand a core-matrix row runs along K;
+// for an MN-major operand it runs along M/N.  lbo = byte distance between core
+// matrices adjacent along K, sbo = between core matrices adjacent along M/N.
+KDA_DEV uint64_t sdesc_interleave(uint32_t addr, uint32_t lbo, uint32_t sbo) {
+    uint64_t d = 0;
+    d |= (uint64_t)((addr >> 4) & 0x3FFFu);
+    d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+    d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+    d |= (uint64_t)1u << 46;                          // descriptor version (sm_100)
+    return d;                                         // layout: SWIZZLE_NONE (0)
+}
+
+// Instruction descriptor for kind::f16 (bf16 in, fp32 accumulate) with the
+// operand majorness given: a_mn / b_mn = 1 for an MN-major operand.
+__host__ __device__ constexpr uint32_t idesc_bf16_major(int M, int N, int a_mn, int b_mn) {
+    return idesc_bf16(M, N) | ((uint32_t)a_mn << 15) | ((uint32_t)b_mn << 16);
+}
+
+// Byte offset of element (mn, k) of an MN-major no-swizzle image whose core
+// matrices are laid out with M/N-block stride 128 B and K-group stride
+// kgroup_bytes (= 16 * MN extent): 8 consecutive mn form one 16-byte row.
+__host__ __device__ __forceinline__ uint32_t mn_off(uint32_t mn, uint32_t k, uint32_t kgroup_bytes) {
+    return (mn >> 3) * 128u + (k >> 3) * kgroup_bytes + (k & 7u) * 16u + (mn & 7u) * 2u;
 }
 
 // Byte offset of element (row, k) inside one 128-byte-wide K block of a
