@@ -107,10 +107,12 @@ KDA_DEV void seq_range(const ChunkArgs& a, int n, int64_t& sb, int64_t& se) {
 // Item = workspace slot = ((n * wc) + (chunk - i0)) * H + h.  Returns false if
 // that chunk lies beyond its sequence.
 KDA_DEV bool item_info(const ChunkArgs& a, int64_t item, int& h, int64_t& t0, int& L) {
-    h = (int)(item % a.H);
-    const int64_t rest = item / a.H;
-    const int n = (int)(rest / a.wc);
-    const int ci = a.i0 + (int)(rest % a.wc);
+    const uint32_t it32 = (uint32_t)item;  // items per pass < 2^31
+    const uint32_t rest = it32 / (uint32_t)a.H;
+    h = (int)(it32 - rest * (uint32_t)a.H);
+    const uint32_t nn = rest / (uint32_t)a.wc;
+    const int n = (int)nn;
+    const int ci = a.i0 + (int)(rest - nn * (uint32_t)a.wc);
     int64_t sb, se;
     seq_range(a, n, sb, se);
     t0 = sb + (int64_t)ci * CH;
@@ -119,27 +121,29 @@ KDA_DEV bool item_info(const ChunkArgs& a, int64_t item, int& h, int64_t& t0, in
     return true;
 }
 
-// Issues D (+)= A B^T over K (multiple of 16) for two K-major SW128 images.
-// a_rows / b_rows are the row counts of one 128-byte-wide K block of each.
-KDA_DEV void mma_run(uint32_t d, uint32_t a_addr, uint32_t a_rows, uint32_t b_addr, uint32_t b_rows, int K,
-                     uint32_t idesc) {
-    for (int kk = 0; kk < K / 16; ++kk) {
-        const uint32_t kb = (uint32_t)kk >> 2, ks = (uint32_t)kk & 3u;
-        const uint64_t ad = sdesc_k_sw128(a_addr + kb * a_rows * 128u + ks * 32u);
-        const uint64_t bd = sdesc_k_sw128(b_addr + kb * b_rows * 128u + ks * 32u);
-        mma_bf16(d, ad, bd, idesc, kk > 0 ? 1u : 0u);
+// Issues D (+)= A B^T over K = 16 * NK for two K-major SW128 images given by
+// their base descriptors.  A_ROWS / B_ROWS are the row counts of one
+// 128-byte-wide K block of each.  A descriptor's start-address field is the
+// byte address / 16 in its low bits, so stepping K adds (byte offset / 16).
+template <int NK, int A_ROWS, int B_ROWS>
+KDA_DEV void mma_sw128(uint32_t d, uint64_t adesc, uint64_t bdesc, uint32_t idesc) {
+#pragma unroll
+    for (int kk = 0; kk < NK; ++kk) {
+        const uint32_t ao = ((uint32_t)(kk >> 2) * A_ROWS * 128u + (uint32_t)(kk & 3) * 32u) >> 4;
+        const uint32_t bo = ((uint32_t)(kk >> 2) * B_ROWS * 128u + (uint32_t)(kk & 3) * 32u) >> 4;
+        mma_bf16(d, adesc + ao, bdesc + bo, idesc, kk > 0 ? 1u : 0u);
     }
 }
 
 // Same for two MN-major no-swizzle images (core-matrix M/N stride 128 B; K-group
-// stride a_kg / b_kg bytes): one MMA step of K = 16 spans two K groups.
-KDA_DEV void mma_run_mn(uint32_t d, uint32_t a_addr, uint32_t a_kg, uint32_t b_addr, uint32_t b_kg, int K,
-                        uint32_t idesc) {
-    for (int kk = 0; kk < K / 16; ++kk) {
-        const uint64_t ad = sdesc_interleave(a_addr + (uint32_t)kk * 2u * a_kg, a_kg, 128u);
-        const uint64_t bd = sdesc_interleave(b_addr + (uint32_t)kk * 2u * b_kg, b_kg, 128u);
-        mma_bf16(d, ad, bd, idesc, kk > 0 ? 1u : 0u);
-    }
+// stride A_KG / B_KG bytes): one MMA step of K = 16 spans two K groups.
+template <int NK, int A_KG, int B_KG>
+KDA_DEV void mma_mn(uint32_t d, uint32_t a_addr, uint32_t b_addr, uint32_t idesc) {
+    const uint64_t ad0 = sdesc_interleave(a_addr, A_KG, 128u), bd0 = sdesc_interleave(b_addr, B_KG, 128u);
+#pragma unroll
+    for (int kk = 0; kk < NK; ++kk)
+        mma_bf16(d, ad0 + (uint32_t)((kk * 2 * A_KG) >> 4), bd0 + (uint32_t)((kk * 2 * B_KG) >> 4), idesc,
+                 kk > 0 ? 1u : 0u);
 }
 
 KDA_DEV uint4 pack8(const float* x) {
@@ -150,9 +154,10 @@ KDA_DEV uint4 pack8(const float* x) {
 // ---------------------------------------------------------------------------
 // intra_kernel
 // ---------------------------------------------------------------------------
-// Threads: 256.  Thread tid owns key/value channel c = tid & 127 and tokens
-// [32*half, 32*half + 32), half = tid >> 7.  Warp w reads TMEM lanes
-// 32*(w & 3) .. +31, i.e. rows c = tid & 127; its half selects columns.
+// Threads: 512.  Thread tid owns key/value channel c = tid & 127 and the
+// 16-token tile q4 = tid >> 7 (tokens [16 q4, 16 q4 + 16)).  Warp w reads TMEM
+// lanes 32*(w & 3) .. +31 (rows c = tid & 127); its group w >> 2 = q4 picks
+// the columns it extracts.
 //
 // Shared memory (offsets from a 1024-aligned base):
 //   RAW [0, 64K)     TMA tiles [64 tokens][128 ch] bf16: la @0, k @16K, q @32K, v @48K
@@ -162,10 +167,11 @@ KDA_DEV uint4 pack8(const float* x) {
 //                             Ktt [128][64] @40K, Ph [64][64] @56K, inverse temp @64K
 //   Y   [136K, ...)  A fp32 [64][68] @0, X fp32 [64][68] @17408;
 //                    later Wt [128][64] @0, Ut [128][64] @16K
-//   misc             beta[64], G[5][128], half-0 totals[128], 2 mbarriers, TMEM base
+//   misc             beta[64], G[5][128], tile totals[4][128], 2 mbarriers, TMEM base
 // TMEM (512 columns): round 1  A/P diag [0,64), off-diag [64,80) [80,112) [112,160)
 //                     round 2  Wt [160,224), Ut [224,288)
 //                     round 3  Mlr [288,416), (PW)^T [416,480), Bm [0,128), Ob^T [128,192)
+constexpr int INTRA_THREADS = 512;
 constexpr uint32_t R_LA = 0, R_K = 16384, R_Q = 32768, R_V = 49152;
 constexpr uint32_t IX = 65536;
 constexpr uint32_t IX_KQR = IX + 0, IX_KD = IX + 32768, IX_KB1 = IX + 49152, IX_KB2 = IX + 53248,
@@ -176,7 +182,7 @@ constexpr uint32_t IY = IX + 73728;
 constexpr int LDA = 68;  // padded fp32 row stride of A and X (16-byte rows, spread banks)
 constexpr uint32_t IY_A = IY, IY_X = IY + 64 * LDA * 4, IY_WT = IY, IY_UT = IY + 16384;
 constexpr uint32_t IM = IY + 35840;
-constexpr uint32_t IM_BETA = IM, IM_G = IM + 256, IM_TOT = IM + 256 + 2560, IM_BAR_RAW = IM_TOT + 512,
+constexpr uint32_t IM_BETA = IM, IM_G = IM + 256, IM_TOT = IM + 256 + 2560, IM_BAR_RAW = IM_TOT + 2048,
                    IM_BAR_MMA = IM_BAR_RAW + 8, IM_TMEM = IM_BAR_MMA + 8;
 constexpr uint32_t INTRA_SMEM = IM_TMEM + 16 + 1024;  // + alignment slack
 constexpr uint32_t INTRA_TMEM_COLS = 512;
@@ -199,20 +205,20 @@ KDA_DEV float raw_in(const uint8_t* sm, uint32_t tile, const void* gsrc, size_t 
 }
 
 template <bool IN_BF16>
-__global__ void __launch_bounds__(256, 1)
+__global__ void __launch_bounds__(INTRA_THREADS, 1)
 intra_kernel(const ChunkArgs a, const __grid_constant__ IntraMaps maps, const int64_t n_items) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     const uint32_t sb = smem_u32(sm);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int c = tid & 127, half = tid >> 7;
+    const int c = tid & 127, q4 = tid >> 7;
     const int qd = warp & 3;
     const int H = a.H;
 
     float* s_beta = reinterpret_cast<float*>(sm + IM_BETA);
     float* s_G = reinterpret_cast<float*>(sm + IM_G);      // [5][128]
-    float* s_tot = reinterpret_cast<float*>(sm + IM_TOT);  // [128]
+    float* s_tot = reinterpret_cast<float*>(sm + IM_TOT);  // [4][128]
     uint64_t* bar_raw = reinterpret_cast<uint64_t*>(sm + IM_BAR_RAW);
     uint64_t* bar_mma = reinterpret_cast<uint64_t*>(sm + IM_BAR_MMA);
     uint32_t* s_tmem = reinterpret_cast<uint32_t*>(sm + IM_TMEM);
@@ -254,6 +260,14 @@ intra_kernel(const ChunkArgs a, const __grid_constant__ IntraMaps maps, const in
 
     int64_t item = next_valid(blockIdx.x);
     bool raw_in_flight = false;
+    // beta of the next item, loaded one item ahead by threads < 64
+    float beta_next = 0.f;
+    if (item < n_items && tid < CH) {
+        int hh, LL;
+        int64_t tt;
+        item_info(a, item, hh, tt, LL);
+        beta_next = (tid < LL) ? ld_in<IN_BF16>(a.beta, (size_t)(tt + tid) * H + hh) : 0.f;
+    }
     if constexpr (IN_BF16) {
         if (tid == 0 && item < n_items) issue_raw(item);
         raw_in_flight = item < n_items;
@@ -268,62 +282,63 @@ intra_kernel(const ChunkArgs a, const __grid_constant__ IntraMaps maps, const in
         const size_t ebase = ((size_t)t0 * H + h) * DK + c;
         const size_t vbase = ((size_t)t0 * H + h) * DV + c;
 
-        if (tid < CH) s_beta[tid] = (tid < L) ? ld_in<IN_BF16>(a.beta, (size_t)(t0 + tid) * H + h) : 0.f;
+        if (tid < CH) s_beta[tid] = beta_next;
         if constexpr (IN_BF16) {
             mbar_wait(bar_raw, ph_raw, a.status);
             ph_raw ^= 1;
             raw_in_flight = false;
         }
 
-        // ---- a1: cumulative clamped log-decay g (registers), tile references G
-        float E1[32], E3[32];
-        uint32_t qr2[16];  // raw q of this thread's 32 tokens, bf16 pairs (kept for the Qp epilogue)
+        // ---- a1: cumulative clamped log-decay g of this thread's tile (registers)
+        float E1[16], E3[16];
+        float gamC = 0.f;  // e^{g at chunk end} of channel c (staged by one thread group)
+        uint32_t qr2[8];  // raw q of this thread's 16 tokens, bf16 pairs (kept for the Qp epilogue)
+        float G[5];
         {
-            float gl[32];
+            float gl[16];
             float run = 0.f;
 #pragma unroll
-            for (int u = 0; u < 32; ++u) {
-                const int t = 32 * half + u;
+            for (int u = 0; u < 16; ++u) {
+                const int t = 16 * q4 + u;
                 const float l = raw_in<IN_BF16>(sm, R_LA, a.log_alpha, ebase, rowstride, t, c, L);
                 run += (t < L) ? fmaxf(l, LOG_ALPHA_FLOOR) : 0.f;
                 gl[u] = run;
             }
-            if (half == 0) s_tot[c] = run;
+            s_tot[q4 * 128 + c] = run;
             __syncthreads();
-            if (half == 1) {
-                const float off = s_tot[c];
+            float off = 0.f;
 #pragma unroll
-                for (int u = 0; u < 32; ++u) gl[u] += off;
-                s_G[3 * 128 + c] = gl[15];
-                s_G[4 * 128 + c] = gl[31];
-            } else {
-                s_G[0 * 128 + c] = 0.f;
-                s_G[1 * 128 + c] = gl[15];
-                s_G[2 * 128 + c] = gl[31];
+            for (int qq = 0; qq < 3; ++qq)
+                if (qq < q4) off += s_tot[qq * 128 + c];
+#pragma unroll
+            for (int u = 0; u < 16; ++u) gl[u] += off;
+            // G_0 = 0, G_{b+1} = g at the last token of tile b
+            s_G[(q4 + 1) * 128 + c] = gl[15];
+            if (q4 == 0) s_G[c] = 0.f;
+            // E1 = e^{g_t - G_q4} (<= 1),  E3 = e^{G_{q4+1} - g_t} (<= 1)
+#pragma unroll
+            for (int u = 0; u < 16; ++u) {
+                E1[u] = __expf(gl[u] - off);
+                E3[u] = __expf(gl[15] - gl[u]);
             }
+            if (tid == 0) bulk_wait_read_all();  // previous item's slot copy has left X/Y
             __syncthreads();
-            // E1 = e^{g_t - G_bt} (<= 1),  E3 = e^{G_{bt+1} - g_t} (<= 1)
-            const float Ga = s_G[(2 * half) * 128 + c], Gb = s_G[(2 * half + 1) * 128 + c],
-                        Gc = s_G[(2 * half + 2) * 128 + c];
 #pragma unroll
-            for (int u = 0; u < 32; ++u) {
-                const float Gs = (u < 16) ? Ga : Gb, Gn = (u < 16) ? Gb : Gc;
-                E1[u] = __expf(gl[u] - Gs);
-                E3[u] = __expf(Gn - gl[u]);
-            }
+            for (int b = 0; b < 5; ++b) G[b] = s_G[b * 128 + c];
         }
-        float G[5];
-#pragma unroll
-        for (int b = 0; b < 5; ++b) G[b] = s_G[b * 128 + c];
+        const float Gs = (q4 == 0) ? G[0] : (q4 == 1) ? G[1] : (q4 == 2) ? G[2] : G[3];  // G_q4
+        const float Gn = (q4 == 0) ? G[1] : (q4 == 1) ? G[2] : (q4 == 2) ? G[3] : G[4];  // G_{q4+1}
 
         // ---- a2 operands (MN-major images, one 16-byte row = 8 consecutive tokens of channel c):
-        //      KQr = [K o E1 ; scale Q o E1],  Kd = K / E1,  Kb^(b) = K o E3 o e^{G_b - G_{bs+1}}
+        //      KQr = [K o E1 ; scale Q o E1],  Kd = K o e^{G_q4 - g},  Kb^(b) = K o e^{G_b - g}  (b > q4)
         {
-            const float f21 = __expf(G[2] - G[1]), f31 = __expf(G[3] - G[1]), f32 = __expf(G[3] - G[2]);
+            const float eD = __expf(Gs - Gn);  // e^{G_q4 - G_{q4+1}} in [1, e^80]
+            // factors e^{G_b - G_{q4+1}} for b = q4+1 .. 3 (the first is 1)
+            const float f2 = __expf(((q4 == 0) ? G[2] : G[3]) - Gn);  // b = q4 + 2 (q4 <= 1)
+            const float f3 = __expf(G[3] - Gn);                         // b = 3
 #pragma unroll
-            for (int m = 0; m < 4; ++m) {
-                const int tf = 32 * half + 8 * m;  // first token of this 8-token row
-                const int bt = tf >> 4;
+            for (int m = 0; m < 2; ++m) {
+                const int tf = 16 * q4 + 8 * m;  // first token of this 8-token row
                 float kr[8], qe[8], kd[8], k3[8];
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
@@ -334,30 +349,28 @@ intra_kernel(const ChunkArgs a, const __grid_constant__ IntraMaps maps, const in
                     else qr2[u >> 1] = (uint32_t)f32_to_bf16(qv);
                     kr[e] = kv * E1[u];
                     qe[e] = qv * E1[u] * a.scale;
-                    kd[e] = __fdividef(kv, E1[u]);  // k e^{G_bt - g_t}, <= e^80
                     k3[e] = kv * E3[u];
+                    kd[e] = k3[e] * eD;  // k e^{G_q4 - g_t}, <= e^80
                 }
                 *reinterpret_cast<uint4*>(sm + IX_KQR + mn_off(tf, c, 2048)) = pack8(kr);
                 *reinterpret_cast<uint4*>(sm + IX_KQR + mn_off(tf + 64, c, 2048)) = pack8(qe);
                 *reinterpret_cast<uint4*>(sm + IX_KD + mn_off(tf, c, 1024)) = pack8(kd);
-                if (bt <= 2) {
-                    float f[8];
-                    if (bt == 2) {
-                        *reinterpret_cast<uint4*>(sm + IX_KB3 + mn_off(tf, c, 768)) = pack8(k3);
-                    } else if (bt == 1) {
-                        *reinterpret_cast<uint4*>(sm + IX_KB2 + mn_off(tf, c, 512)) = pack8(k3);
+                float f[8];
+                if (q4 == 0) {
+                    *reinterpret_cast<uint4*>(sm + IX_KB1 + mn_off(tf, c, 256)) = pack8(k3);
 #pragma unroll
-                        for (int e = 0; e < 8; ++e) f[e] = k3[e] * f32;
-                        *reinterpret_cast<uint4*>(sm + IX_KB3 + mn_off(tf, c, 768)) = pack8(f);
-                    } else {
-                        *reinterpret_cast<uint4*>(sm + IX_KB1 + mn_off(tf, c, 256)) = pack8(k3);
+                    for (int e = 0; e < 8; ++e) f[e] = k3[e] * f2;
+                    *reinterpret_cast<uint4*>(sm + IX_KB2 + mn_off(tf, c, 512)) = pack8(f);
 #pragma unroll
-                        for (int e = 0; e < 8; ++e) f[e] = k3[e] * f21;
-                        *reinterpret_cast<uint4*>(sm + IX_KB2 + mn_off(tf, c, 512)) = pack8(f);
+                    for (int e = 0; e < 8; ++e) f[e] = k3[e] * f3;
+                    *reinterpret_cast<uint4*>(sm + IX_KB3 + mn_off(tf, c, 768)) = pack8(f);
+                } else if (q4 == 1) {
+                    *reinterpret_cast<uint4*>(sm + IX_KB2 + mn_off(tf, c, 512)) = pack8(k3);
 #pragma unroll
-                        for (int e = 0; e < 8; ++e) f[e] = k3[e] * f31;
-                        *reinterpret_cast<uint4*>(sm + IX_KB3 + mn_off(tf, c, 768)) = pack8(f);
-                    }
+                    for (int e = 0; e < 8; ++e) f[e] = k3[e] * f3;
+                    *reinterpret_cast<uint4*>(sm + IX_KB3 + mn_off(tf, c, 768)) = pack8(f);
+                } else if (q4 == 2) {
+                    *reinterpret_cast<uint4*>(sm + IX_KB3 + mn_off(tf, c, 768)) = pack8(k3);
                 }
             }
         }
@@ -368,24 +381,52 @@ intra_kernel(const ChunkArgs a, const __grid_constant__ IntraMaps maps, const in
 
         // ---- round 1: [Kr;Qr] Kd^T and [Kr;Qr] Kb(b)^T
         if (tid == 0) {
-            mma_run_mn(tm + TM_AD, sb + IX_KQR, 2048, sb + IX_KD, 1024, DK, idesc_bf16_major(128, 64, 1, 1));
-            mma_run_mn(tm + TM_B1, sb + IX_KQR, 2048, sb + IX_KB1, 256, DK, idesc_bf16_major(128, 16, 1, 1));
-            mma_run_mn(tm + TM_B2, sb + IX_KQR, 2048, sb + IX_KB2, 512, DK, idesc_bf16_major(128, 32, 1, 1));
-            mma_run_mn(tm + TM_B3, sb + IX_KQR, 2048, sb + IX_KB3, 768, DK, idesc_bf16_major(128, 48, 1, 1));
+            mma_mn<8, 2048, 1024>(tm + TM_AD, sb + IX_KQR, sb + IX_KD, idesc_bf16_major(128, 64, 1, 1));
+            mma_mn<8, 2048, 256>(tm + TM_B1, sb + IX_KQR, sb + IX_KB1, idesc_bf16_major(128, 16, 1, 1));
+            mma_mn<8, 2048, 512>(tm + TM_B2, sb + IX_KQR, sb + IX_KB2, idesc_bf16_major(128, 32, 1, 1));
+            mma_mn<8, 2048, 768>(tm + TM_B3, sb + IX_KQR, sb + IX_KB3, idesc_bf16_major(128, 48, 1, 1));
             mma_commit(bar_mma);
         }
         mbar_wait(bar_mma, ph_mma, a.status);
         ph_mma ^= 1;
         tc_fence_after();
 
-        // ---- A (rows 0..63) -> fp32 smem [64][68];  P (rows 64..127) -> bf16 image Ph [t][s]
-        //      16-column pieces, stored 16 bytes at a time
+        // ---- A (rows 0..63) -> fp32 smem [64][68];  P (rows 64..127) -> bf16 image Ph [t][s].
+        //      Warp (qd, p): 16-column piece p of the 32 rows of quadrant qd.
         {
             float* sA = reinterpret_cast<float*>(sm + IY_A);
+            const int p = q4;
             const int r = 32 * qd + lane;
             const bool isP = r >= 64;
             const int t = r & 63, bt = t >> 4;
-            auto put16 = [&](int p, const float* d) {  // columns [16p, 16p + 16)
+            float dA[16], dB[16], dC[16];
+            tmem_ld16(lane_addr + TM_AD + 16 * p, dA);
+            if ((qd & 1) == 0) {
+                if (p == 0) tmem_ld16(lane_addr + TM_B1, dB);  // rows of tile 1
+            } else {
+                if (p < 2) tmem_ld16(lane_addr + TM_B2 + 16 * p, dB);  // rows of tile 2
+                if (p < 3) tmem_ld16(lane_addr + TM_B3 + 16 * p, dC);  // rows of tile 3
+            }
+            tmem_ld_wait();
+            float d[16];
+            bool write = true;
+            if (p >= bt) {  // diagonal tile (A strictly lower, P lower) and the zero upper part
+#pragma unroll
+                for (int s16 = 0; s16 < 16; ++s16) {
+                    const int s = 16 * p + s16;
+                    const bool keep = (p == bt) && (isP ? (s <= t) : (s < t));
+                    d[s16] = keep ? dA[s16] : 0.f;
+                }
+            } else if (bt == 3) {
+#pragma unroll
+                for (int s16 = 0; s16 < 16; ++s16) d[s16] = dC[s16];
+            } else if (bt == 1 || bt == 2) {
+#pragma unroll
+                for (int s16 = 0; s16 < 16; ++s16) d[s16] = dB[s16];
+            } else {
+                write = false;
+            }
+            if (write) {
                 if (isP) {
                     *reinterpret_cast<uint4*>(sm + IX_PH + sw128_off(t, 16 * p)) = pack8(d);
                     *reinterpret_cast<uint4*>(sm + IX_PH + sw128_off(t, 16 * p + 8)) = pack8(d + 8);
@@ -393,39 +434,6 @@ intra_kernel(const ChunkArgs a, const __grid_constant__ IntraMaps maps, const in
                     float4* dst = reinterpret_cast<float4*>(sA + t * LDA + 16 * p);
 #pragma unroll
                     for (int i = 0; i < 4; ++i) dst[i] = make_float4(d[4 * i], d[4 * i + 1], d[4 * i + 2], d[4 * i + 3]);
-                }
-            };
-            if (half == 0) {
-                // diagonal tile (masked: A strictly lower, P lower) and the zero upper part
-#pragma unroll
-                for (int p = 0; p < 4; ++p) {
-                    float d[16];
-                    tmem_ld16(lane_addr + TM_AD + 16 * p, d);
-                    tmem_ld_wait();
-                    if (p >= bt) {
-#pragma unroll
-                        for (int s16 = 0; s16 < 16; ++s16) {
-                            const int s = 16 * p + s16;
-                            const bool keep = (p == bt) && (isP ? (s <= t) : (s < t));
-                            d[s16] = keep ? d[s16] : 0.f;
-                        }
-                        put16(p, d);
-                    }
-                }
-            } else if ((qd & 1) == 0) {  // rows t in [0, 32): tiles 0 and 1
-                float d[16];
-                tmem_ld16(lane_addr + TM_B1, d);
-                tmem_ld_wait();
-                if (bt == 1) put16(0, d);
-            } else {  // rows t in [32, 64): tiles 2 and 3; off-diagonal column tiles p < bt
-#pragma unroll
-                for (int p = 0; p < 3; ++p) {
-                    float d2[16], d3[16];
-                    if (p < 2) tmem_ld16(lane_addr + TM_B2 + 16 * p, d2);
-                    tmem_ld16(lane_addr + TM_B3 + 16 * p, d3);
-                    tmem_ld_wait();
-                    if (bt == 2 && p < 2) put16(p, d2);
-                    if (bt == 3) put16(p, d3);
                 }
             }
         }
@@ -436,59 +444,96 @@ intra_kernel(const ChunkArgs a, const __grid_constant__ IntraMaps maps, const in
             float* sA = reinterpret_cast<float*>(sm + IY_A);  // becomes N = Diag(beta) A in place
             float* sX = reinterpret_cast<float*>(sm + IY_X);  // X = (I + N)^-1
             float* sY = reinterpret_cast<float*>(sm + IX_TMP);
-            for (int e = tid; e < 64 * 64; e += 256) {
-                const int i = e >> 6, j = e & 63;
-                sA[i * LDA + j] *= s_beta[i];
+            for (int e = tid; e < 64 * 16; e += INTRA_THREADS) {  // 4 entries per step
+                const int i = e >> 4, j4 = (e & 15) * 4;
+                float4* pa = reinterpret_cast<float4*>(sA + i * LDA + j4);
+                const float b = s_beta[i];
+                float4 v4 = *pa;
+                v4.x *= b; v4.y *= b; v4.z *= b; v4.w *= b;
+                *pa = v4;
+                // zero the strictly upper blocks of X
+                if ((j4 >> 4) > (i >> 4)) *reinterpret_cast<float4*>(sX + i * LDA + j4) = make_float4(0.f, 0.f, 0.f, 0.f);
             }
             __syncthreads();
             if (tid < 64) {  // diagonal blocks: one thread per (block, column)
+                // column j of (I + N_bb)^-1: x_i = -sum_{m<i} N_im x_m, x_j = 1, x_i = 0 for i < j
+                // (entries above j are zero, so the sums need no masking)
                 const int b = tid >> 4, j = tid & 15;
                 const float* Nb = sA + (16 * b) * LDA + 16 * b;
                 float x[16];
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
-                    float acc = 0.f;
+                    float nr[16];
 #pragma unroll
-                    for (int m = 0; m < i; ++m)
-                        if (m >= j) acc += Nb[i * LDA + m] * x[m];
-                    x[i] = (i < j) ? 0.f : ((i == j) ? 1.f : -acc);
+                    for (int q = 0; q < 4; ++q) {
+                        const float4 v4 = reinterpret_cast<const float4*>(Nb + i * LDA)[q];
+                        nr[4 * q] = v4.x; nr[4 * q + 1] = v4.y; nr[4 * q + 2] = v4.z; nr[4 * q + 3] = v4.w;
+                    }
+                    float acc0 = 0.f, acc1 = 0.f;
+#pragma unroll
+                    for (int m = 0; m < i; ++m) {
+                        if (m & 1) acc1 += nr[m] * x[m];
+                        else acc0 += nr[m] * x[m];
+                    }
+                    x[i] = (i < j) ? 0.f : ((i == j) ? 1.f : -(acc0 + acc1));
                 }
 #pragma unroll
                 for (int i = 0; i < 16; ++i) sX[(16 * b + i) * LDA + 16 * b + j] = x[i];
             }
-            for (int e = tid; e < 64 * 64; e += 256) {
-                const int i = e >> 6, j = e & 63;
-                if ((j >> 4) > (i >> 4)) sX[i * LDA + j] = 0.f;
-            }
             __syncthreads();
-            // off-diagonal blocks by distance d:  X_ij = -X_ii * sum_{m=j}^{i-1} N_im X_mj
+            // off-diagonal blocks by distance d:  X_ij = -X_ii * sum_{m=j}^{i-1} N_im X_mj.
+            // One task = 1 row x 4 columns of one block pair (4 independent accumulators).
             for (int d = 1; d <= 3; ++d) {
-                const int nblk = 4 - d;
-                for (int e = tid; e < nblk * 256; e += 256) {
-                    const int p = e >> 8, r = (e >> 4) & 15, cc = e & 15;
-                    const int bj = p, bi = p + d;
-                    float acc = 0.f;
-                    for (int m = bj; m < bi; ++m) {
+                const int ntask = (4 - d) * 64;
+                if (tid < ntask) {
+                    const int pb = tid >> 6, r = (tid >> 2) & 15, cc = (tid & 3) * 4;
+                    const int bj = pb, bi = pb + d;
+                    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-                        for (int uu = 0; uu < 16; ++uu)
-                            acc += sA[(16 * bi + r) * LDA + 16 * m + uu] * sX[(16 * m + uu) * LDA + 16 * bj + cc];
+                    for (int mm = 0; mm < 3; ++mm) {
+                        if (mm < d) {
+                            const int m = bj + mm;
+                            const float* na = sA + (16 * bi + r) * LDA + 16 * m;
+                            const float* xb = sX + (16 * m) * LDA + 16 * bj + cc;
+#pragma unroll
+                            for (int u4 = 0; u4 < 4; ++u4) {
+                                const float4 nv = *reinterpret_cast<const float4*>(na + 4 * u4);
+                                const float nvs[4] = {nv.x, nv.y, nv.z, nv.w};
+#pragma unroll
+                                for (int k = 0; k < 4; ++k) {
+                                    const float4 xv = *reinterpret_cast<const float4*>(xb + (4 * u4 + k) * LDA);
+                                    acc.x += nvs[k] * xv.x; acc.y += nvs[k] * xv.y;
+                                    acc.z += nvs[k] * xv.z; acc.w += nvs[k] * xv.w;
+                                }
+                            }
+                        }
                     }
-                    sY[p * 256 + r * 16 + cc] = acc;
+                    *reinterpret_cast<float4*>(sY + pb * 256 + r * 16 + cc) = acc;
                 }
                 __syncthreads();
-                for (int e = tid; e < nblk * 256; e += 256) {
-                    const int p = e >> 8, r = (e >> 4) & 15, cc = e & 15;
-                    const int bj = p, bi = p + d;
-                    float acc = 0.f;
+                if (tid < ntask) {
+                    const int pb = tid >> 6, r = (tid >> 2) & 15, cc = (tid & 3) * 4;
+                    const int bj = pb, bi = pb + d;
+                    const float* xa = sX + (16 * bi + r) * LDA + 16 * bi;
+                    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-                    for (int uu = 0; uu < 16; ++uu)
-                        acc += sX[(16 * bi + r) * LDA + 16 * bi + uu] * sY[p * 256 + uu * 16 + cc];
-                    sX[(16 * bi + r) * LDA + 16 * bj + cc] = -acc;
+                    for (int u4 = 0; u4 < 4; ++u4) {
+                        const float4 xv4 = *reinterpret_cast<const float4*>(xa + 4 * u4);
+                        const float xs[4] = {xv4.x, xv4.y, xv4.z, xv4.w};
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) {
+                            const float4 yv = *reinterpret_cast<const float4*>(sY + pb * 256 + (4 * u4 + k) * 16 + cc);
+                            acc.x += xs[k] * yv.x; acc.y += xs[k] * yv.y;
+                            acc.z += xs[k] * yv.z; acc.w += xs[k] * yv.w;
+                        }
+                    }
+                    *reinterpret_cast<float4*>(sX + (16 * bi + r) * LDA + 16 * bj + cc) =
+                        make_float4(-acc.x, -acc.y, -acc.z, -acc.w);
                 }
                 __syncthreads();
             }
-            for (int e = tid; e < 64 * 8; e += 256) {  // T = X Diag(beta) -> bf16 image Ti [t][s], 8 s per store
-                const int t = e >> 3, s0 = (e & 7) * 8;
+            {  // T = X Diag(beta) -> bf16 image Ti [t][s], 8 s per store, one row piece per thread
+                const int t = tid >> 3, s0 = (tid & 7) * 8;
                 const float4 x0 = *reinterpret_cast<const float4*>(sX + t * LDA + s0);
                 const float4 x1 = *reinterpret_cast<const float4*>(sX + t * LDA + s0 + 4);
                 const float4 b0 = *reinterpret_cast<const float4*>(s_beta + s0);
@@ -501,60 +546,64 @@ intra_kernel(const ChunkArgs a, const __grid_constant__ IntraMaps maps, const in
 
         // ---- phase 2 operands (K = token): KGt = (K o Gam)^T, Vt = V^T, Ktt = Kt^T
         {
-            const float eG[2] = {__expf(half ? G[2] : G[0]), __expf(half ? G[3] : G[1])};
-            const float eC[2] = {__expf(G[4] - (half ? G[3] : G[1])), __expf(G[4] - (half ? G[4] : G[2]))};
+            const float eG = __expf(Gs);          // Gam_t = E1 e^{G_q4}
+            const float eC = __expf(G[4] - Gn);   // e^{g_C - g_t} = E3 e^{G_4 - G_{q4+1}}
 #pragma unroll
-            for (int m = 0; m < 4; ++m) {  // 8 consecutive tokens per 16-byte chunk
+            for (int m = 0; m < 2; ++m) {  // 8 consecutive tokens per 16-byte chunk
                 float kg[8], vv[8], kt[8];
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
                     const int u = 8 * m + e;
-                    const int t = 32 * half + u;
+                    const int t = 16 * q4 + u;
                     const float kv = raw_in<IN_BF16>(sm, R_K, a.k, ebase, rowstride, t, c, L);
                     vv[e] = raw_in<IN_BF16>(sm, R_V, a.v, vbase, (size_t)H * DV, t, c, L);
-                    kg[e] = kv * E1[u] * eG[u >> 4];
-                    kt[e] = kv * E3[u] * eC[u >> 4];
+                    kg[e] = kv * E1[u] * eG;
+                    kt[e] = kv * E3[u] * eC;
                 }
-                const uint32_t off = sw128_off((uint32_t)c, (uint32_t)(32 * half + 8 * m));
+                const uint32_t off = sw128_off((uint32_t)c, (uint32_t)(16 * q4 + 8 * m));
                 *reinterpret_cast<uint4*>(sm + IX_KGT + off) = pack8(kg);
                 *reinterpret_cast<uint4*>(sm + IX_VT + off) = pack8(vv);
                 *reinterpret_cast<uint4*>(sm + IX_KTT + off) = pack8(kt);
             }
-            if (half == 1) *reinterpret_cast<float*>(wslot + SO_G + 4 * c) = __expf(G[4]);
+            gamC = __expf(G[4]);
         }
         fence_async_smem();
         tc_fence_before();
         __syncthreads();
         tc_fence_after();
 
-        // next item's raw tiles: every read of RAW for this item is done
+        // ---- round 2: Wt = KGt Ti^T, Ut = Vt Ti^T
+        if (tid == 0) {
+            mma_sw128<4, 128, 64>(tm + TM_WT, sdesc_k_sw128(sb + IX_KGT), sdesc_k_sw128(sb + IX_TI), idesc_bf16(128, 64));
+            mma_sw128<4, 128, 64>(tm + TM_UT, sdesc_k_sw128(sb + IX_VT), sdesc_k_sw128(sb + IX_TI), idesc_bf16(128, 64));
+            mma_commit(bar_mma);
+        }
+        // next item's raw tiles (every read of RAW for this item is done) and beta
         const int64_t next = next_valid(item + gridDim.x);
         if constexpr (IN_BF16) {
             if (tid == 0 && next < n_items) issue_raw(next);
             raw_in_flight = next < n_items;
         }
-
-        // ---- round 2: Wt = KGt Ti^T, Ut = Vt Ti^T
-        if (tid == 0) {
-            mma_run(tm + TM_WT, sb + IX_KGT, 128, sb + IX_TI, 64, CH, idesc_bf16(128, 64));
-            mma_run(tm + TM_UT, sb + IX_VT, 128, sb + IX_TI, 64, CH, idesc_bf16(128, 64));
-            mma_commit(bar_mma);
+        if (tid < CH && next < n_items) {
+            int hh, LL;
+            int64_t tt;
+            item_info(a, next, hh, tt, LL);
+            beta_next = (tid < LL) ? ld_in<IN_BF16>(a.beta, (size_t)(tt + tid) * H + hh) : 0.f;
         }
         mbar_wait(bar_mma, ph_mma, a.status);
         ph_mma ^= 1;
         tc_fence_after();
         {
-            // half 0 -> Wt image, half 1 -> Ut image; row = channel c, 64 token columns
-            const uint32_t col0 = half ? TM_UT : TM_WT;
-            const uint32_t dst = half ? IY_UT : IY_WT;
+            // group 0/1 -> Wt token columns [0,32)/[32,64), group 2/3 -> Ut; row = channel c
+            const uint32_t col0 = (q4 < 2 ? TM_WT : TM_UT) + 32 * (q4 & 1);
+            const uint32_t dst = q4 < 2 ? IY_WT : IY_UT;
+            float d[32];
+            tmem_ld16(lane_addr + col0, d);
+            tmem_ld16(lane_addr + col0 + 16, d + 16);
+            tmem_ld_wait();
 #pragma unroll
-            for (int p = 0; p < 4; ++p) {
-                float d[16];
-                tmem_ld16(lane_addr + col0 + 16 * p, d);
-                tmem_ld_wait();
-                *reinterpret_cast<uint4*>(sm + dst + sw128_off((uint32_t)c, (uint32_t)(16 * p))) = pack8(d);
-                *reinterpret_cast<uint4*>(sm + dst + sw128_off((uint32_t)c, (uint32_t)(16 * p + 8))) = pack8(d + 8);
-            }
+            for (int pp = 0; pp < 4; ++pp)
+                *reinterpret_cast<uint4*>(sm + dst + sw128_off((uint32_t)c, 32 * (q4 & 1) + 8 * pp)) = pack8(d + 8 * pp);
         }
         fence_async_smem();
         tc_fence_before();
@@ -563,77 +612,87 @@ intra_kernel(const ChunkArgs a, const __grid_constant__ IntraMaps maps, const in
 
         // ---- round 3: Mlr = Ktt Wt^T, Bm = Ktt Ut^T, (P W)^T = Wt Ph^T, Ob^T = Ut Ph^T
         if (tid == 0) {
-            mma_run(tm + TM_M, sb + IX_KTT, 128, sb + IY_WT, 128, CH, idesc_bf16(128, 128));
-            mma_run(tm + TM_PW, sb + IY_WT, 128, sb + IX_PH, 64, CH, idesc_bf16(128, 64));
-            mma_run(tm + TM_BM, sb + IX_KTT, 128, sb + IY_UT, 128, CH, idesc_bf16(128, 128));
-            mma_run(tm + TM_OB, sb + IY_UT, 128, sb + IX_PH, 64, CH, idesc_bf16(128, 64));
+            const uint64_t dk = sdesc_k_sw128(sb + IX_KTT), dw = sdesc_k_sw128(sb + IY_WT),
+                           du = sdesc_k_sw128(sb + IY_UT), dp = sdesc_k_sw128(sb + IX_PH);
+            mma_sw128<4, 128, 128>(tm + TM_M, dk, dw, idesc_bf16(128, 128));
+            mma_sw128<4, 128, 64>(tm + TM_PW, dw, dp, idesc_bf16(128, 64));
+            mma_sw128<4, 128, 128>(tm + TM_BM, dk, du, idesc_bf16(128, 128));
+            mma_sw128<4, 128, 64>(tm + TM_OB, du, dp, idesc_bf16(128, 64));
             mma_commit(bar_mma);
         }
         mbar_wait(bar_mma, ph_mma, a.status);
         ph_mma ^= 1;
         tc_fence_after();
         {
-            // Mlr row c -> K-major SW128 image (half h writes K block h)
-            {
-                uint8_t* dstM = wslot + SO_M + (size_t)half * (DK * 128);
+            // The slot is assembled in shared memory (operand regions X and Y are dead
+            // once round 3 has completed) and written by one bulk copy.
+            uint8_t* st = sm + IX;
+            if (q4 < 2) {
+                // Mlr row c, K block q4 -> K-major SW128 image
+                uint8_t* dstM = st + SO_M + (size_t)q4 * (DK * 128);
 #pragma unroll
-                for (int p = 0; p < 4; ++p) {
-                    float d[16];
-                    tmem_ld16(lane_addr + TM_M + 64 * half + 16 * p, d);
+                for (int hp = 0; hp < 2; ++hp) {
+                    float d[32];
+                    tmem_ld16(lane_addr + TM_M + 64 * q4 + 32 * hp, d);
+                    tmem_ld16(lane_addr + TM_M + 64 * q4 + 32 * hp + 16, d + 16);
                     tmem_ld_wait();
-                    *reinterpret_cast<uint4*>(dstM + sw128_off((uint32_t)c, (uint32_t)(16 * p))) = pack8(d);
-                    *reinterpret_cast<uint4*>(dstM + sw128_off((uint32_t)c, (uint32_t)(16 * p + 8))) = pack8(d + 8);
-                }
-            }
-            // Bm row c, value columns [64 half, 64 half + 64) -> slices 2 half, 2 half + 1
-            {
 #pragma unroll
-                for (int p = 0; p < 4; ++p) {  // columns 64 half + 16 p .. +16 -> slice 2 half + p / 2
-                    float d[16];
-                    tmem_ld16(lane_addr + TM_BM + 64 * half + 16 * p, d);
-                    tmem_ld_wait();
-                    uint4* dstB = reinterpret_cast<uint4*>(wslot + SO_B + (size_t)(2 * half + (p >> 1)) * BSL +
-                                                           (size_t)c * DVS * 2) + 2 * (p & 1);
-                    dstB[0] = pack8(d);
-                    dstB[1] = pack8(d + 8);
+                    for (int pp = 0; pp < 4; ++pp)
+                        *reinterpret_cast<uint4*>(dstM + sw128_off((uint32_t)c, (uint32_t)(32 * hp + 8 * pp))) =
+                            pack8(d + 8 * pp);
                 }
+            } else {
+                // Bm row c, value columns [64 (q4-2), +64) -> slices 2 (q4-2) and 2 (q4-2) + 1
+                const int hh = q4 - 2;
+#pragma unroll
+                for (int hp = 0; hp < 2; ++hp) {  // one 32-column slice per half
+                    float d[32];
+                    tmem_ld16(lane_addr + TM_BM + 64 * hh + 32 * hp, d);
+                    tmem_ld16(lane_addr + TM_BM + 64 * hh + 32 * hp + 16, d + 16);
+                    tmem_ld_wait();
+                    uint4* dstB = reinterpret_cast<uint4*>(st + SO_B + (size_t)(2 * hh + hp) * BSL + (size_t)c * DVS * 2);
+#pragma unroll
+                    for (int pp = 0; pp < 4; ++pp) dstB[pp] = pack8(d + 8 * pp);
+                }
+                if (q4 == 3) *reinterpret_cast<float*>(st + SO_G + 4 * c) = gamC;
             }
             // Qp^T[c][t] = scale q_tc e^{g_tc} - (P W)^T[c][t] -> MN-major image (token-contiguous rows);
-            // Ob^T[j][t] -> slice j/32, row j%32 (64 tokens).  16 bytes per store.
+            // Ob^T[j][t] -> slice j/32, row j%32 (64 tokens).  This thread's 16 tokens.
             {
-                const float eG[2] = {__expf(half ? G[2] : G[0]), __expf(half ? G[3] : G[1])};
-                uint8_t* dstQ = wslot + SO_Q;
-                uint8_t* dstO = wslot + SO_O + (size_t)(c >> 5) * OSL + (size_t)(c & 31) * (CH * 2);
+                const float eG = __expf(Gs);
+                float pw[16], ob[16], qq[16];
+                tmem_ld16(lane_addr + TM_PW + 16 * q4, pw);
+                tmem_ld16(lane_addr + TM_OB + 16 * q4, ob);
+                tmem_ld_wait();
 #pragma unroll
-                for (int p = 0; p < 2; ++p) {
-                    float pw[16], ob[16], qq[16];
-                    tmem_ld16(lane_addr + TM_PW + 32 * half + 16 * p, pw);
-                    tmem_ld16(lane_addr + TM_OB + 32 * half + 16 * p, ob);
-                    tmem_ld_wait();
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) {
-                        const int u = 16 * p + e;
-                        const float qv =
-                            __uint_as_float((u & 1) ? (qr2[u >> 1] & 0xFFFF0000u) : (qr2[u >> 1] << 16));
-                        qq[e] = qv * E1[u] * eG[p] * a.scale - pw[e];
-                    }
-                    const int tf = 32 * half + 16 * p;
-                    *reinterpret_cast<uint4*>(dstQ + mn_off(tf, c, 1024)) = pack8(qq);
-                    *reinterpret_cast<uint4*>(dstQ + mn_off(tf + 8, c, 1024)) = pack8(qq + 8);
-                    *reinterpret_cast<uint4*>(dstO + tf * 2) = pack8(ob);
-                    *reinterpret_cast<uint4*>(dstO + tf * 2 + 16) = pack8(ob + 8);
+                for (int u = 0; u < 16; ++u) {
+                    const float qv = __uint_as_float((u & 1) ? (qr2[u >> 1] & 0xFFFF0000u) : (qr2[u >> 1] << 16));
+                    qq[u] = qv * E1[u] * eG * a.scale - pw[u];
                 }
+                const int tf = 16 * q4;
+                uint8_t* dstQ = st + SO_Q;
+                uint8_t* dstO = st + SO_O + (size_t)(c >> 5) * OSL + (size_t)(c & 31) * (CH * 2);
+                *reinterpret_cast<uint4*>(dstQ + mn_off(tf, c, 1024)) = pack8(qq);
+                *reinterpret_cast<uint4*>(dstQ + mn_off(tf + 8, c, 1024)) = pack8(qq + 8);
+                *reinterpret_cast<uint4*>(dstO + tf * 2) = pack8(ob);
+                *reinterpret_cast<uint4*>(dstO + tf * 2 + 16) = pack8(ob + 8);
             }
         }
+        fence_async_smem();
         tc_fence_before();
         __syncthreads();
         tc_fence_after();
+        if (tid == 0) {
+            bulk_s2g(wslot, sm + IX, (uint32_t)SLOT_BYTES);
+            bulk_commit();
+        }
         item = next;
     }
     // a prefetch can only be in flight here after a failed wait; let it land
     if constexpr (IN_BF16) {
         if (tid == 0 && raw_in_flight) mbar_wait(bar_raw, ph_raw, nullptr);
     }
+    if (tid == 0) bulk_wait_all();  // last slot copy complete before the CTA retires
     __syncthreads();
     if (warp == 0) {
         tc_fence_after();
@@ -647,13 +706,14 @@ intra_kernel(const ChunkArgs a, const __grid_constant__ IntraMaps maps, const in
 // Threads: 128; thread c owns state row c of the 32-column slice (32 fp32
 // registers).  TMEM (128 columns): D_S = Mlr S in [0,32) (M=128, lane = row
 // c); D_O = Qp S double-buffered in [32,64) and [64,96) (M=64: row t lives in
-// lane 32*(t/16) + t%16).  Shared memory: two chunk buffers {Mlr image 32K,
-// Qp image 16K, GamC 512, Bm slice 8K, Ob slice 4K} and two bf16 state
-// operand images Sb [32 value cols][128 key rows] (8K each).
+// lane 32*(t/16) + t%16).  Shared memory: three chunk buffers {Mlr image 32K,
+// Qp image 16K, GamC 512, Bm slice 8K, ObT slice 4K} (loads run three chunks
+// ahead) and two bf16 state operand images Sb [32 value cols][128 key rows].
 constexpr uint32_t CB_M = 0, CB_Q = 32768, CB_G = 49152, CB_B = 49664, CB_O = 57856, CB_SIZE = 62464;
-constexpr uint32_t C_SB = 2 * CB_SIZE;        // two 8K state images
-constexpr uint32_t C_BAR = C_SB + 2 * 8192;   // bar_ld[2], bar_s, bar_o[2]
-constexpr uint32_t C_FLAG = C_BAR + 40;
+constexpr int NBUF = 3;                          // chunk buffers in flight
+constexpr uint32_t C_SB = NBUF * CB_SIZE;        // two 8K state images
+constexpr uint32_t C_BAR = C_SB + 2 * 8192;      // bar_ld[3], bar_s, bar_o[2]
+constexpr uint32_t C_FLAG = C_BAR + 48;
 constexpr uint32_t C_TMEM = C_FLAG + 16;
 constexpr uint32_t CHAIN_SMEM = C_TMEM + 16 + 1024;
 constexpr uint32_t CHAIN_TMEM_COLS = 128;
@@ -666,12 +726,12 @@ __global__ void __launch_bounds__(128, 1) chain_kernel(const ChunkArgs a) {
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int js = blockIdx.x, h = blockIdx.y, n = blockIdx.z;
     const int H = a.H;
-    uint64_t* bar_ld = reinterpret_cast<uint64_t*>(sm + C_BAR);  // [2]
-    uint64_t* bar_s = reinterpret_cast<uint64_t*>(sm + C_BAR + 16);
+    uint64_t* bar_ld = reinterpret_cast<uint64_t*>(sm + C_BAR);  // [NBUF]
+    uint64_t* bar_s = reinterpret_cast<uint64_t*>(sm + C_BAR + 24);
     // one output barrier per D_O buffer: the next chunk's output product is
     // committed before this chunk's output is waited for, so a single barrier
     // could complete two phases between waits
-    uint64_t* bar_o = reinterpret_cast<uint64_t*>(sm + C_BAR + 24);  // [2]
+    uint64_t* bar_o = reinterpret_cast<uint64_t*>(sm + C_BAR + 32);  // [2]
     volatile int* s_fail = reinterpret_cast<volatile int*>(sm + C_FLAG);
     uint32_t* s_tmem = reinterpret_cast<uint32_t*>(sm + C_TMEM);
 
@@ -705,8 +765,7 @@ __global__ void __launch_bounds__(128, 1) chain_kernel(const ChunkArgs a) {
             tmem_relinquish();
         }
         if (tid == 0) {
-            mbar_init(&bar_ld[0], 1);
-            mbar_init(&bar_ld[1], 1);
+            for (int i = 0; i < NBUF; ++i) mbar_init(&bar_ld[i], 1);
             mbar_init(bar_s, 1);
             mbar_init(&bar_o[0], 1);
             mbar_init(&bar_o[1], 1);
@@ -718,13 +777,17 @@ __global__ void __launch_bounds__(128, 1) chain_kernel(const ChunkArgs a) {
         const uint32_t tm = *s_tmem;
         const uint32_t lane_addr = tm + ((uint32_t)(32 * warp) << 16);
         const size_t slot0 = ((size_t)n * a.wc + (c_beg - a.i0)) * H + h;  // slot of iteration 0
+        // chunk buffer of iteration it and its barrier phase
+        auto bidx = [](int it) { return it % NBUF; };
+        auto bpar = [](int it) { return (uint32_t)((it / NBUF) & 1); };
         auto issue_load = [&](int it) {
-            uint8_t* buf = sm + (it & 1) * CB_SIZE;
+            const int b = bidx(it);
+            uint8_t* buf = sm + b * CB_SIZE;
             const uint8_t* src = a.ws + (slot0 + (size_t)it * H) * SLOT_BYTES;
-            mbar_arrive_expect_tx(&bar_ld[it & 1], SO_MQG + BSL + OSL);
-            bulk_g2s(buf + CB_M, src + SO_M, SO_MQG, &bar_ld[it & 1]);
-            bulk_g2s(buf + CB_B, src + SO_B + (size_t)js * BSL, BSL, &bar_ld[it & 1]);
-            bulk_g2s(buf + CB_O, src + SO_O + (size_t)js * OSL, OSL, &bar_ld[it & 1]);
+            mbar_arrive_expect_tx(&bar_ld[b], SO_MQG + BSL + OSL);
+            bulk_g2s(buf + CB_M, src + SO_M, SO_MQG, &bar_ld[b]);
+            bulk_g2s(buf + CB_B, src + SO_B + (size_t)js * BSL, BSL, &bar_ld[b]);
+            bulk_g2s(buf + CB_O, src + SO_O + (size_t)js * OSL, OSL, &bar_ld[b]);
         };
         auto write_state_image = [&](int it) {
             const uint32_t kb = (uint32_t)tid >> 6, kc = (uint32_t)tid & 63u;
@@ -735,19 +798,19 @@ __global__ void __launch_bounds__(128, 1) chain_kernel(const ChunkArgs a) {
         };
         // thread 0: Mlr S -> D_S (commit bar_s), then Qp S -> D_O[it&1] (commit bar_o[it&1])
         auto issue_mma = [&](int it) -> bool {
-            const int b = it & 1;
-            if (!mbar_wait(&bar_ld[b], (uint32_t)((it >> 1) & 1), a.status)) return false;
+            const int b = bidx(it);
+            if (!mbar_wait(&bar_ld[b], bpar(it), a.status)) return false;
             tc_fence_after();
-            const uint32_t img = sbase + C_SB + (it & 1) * 8192;
-            mma_run(tm + 0, sbase + b * CB_SIZE + CB_M, 128, img, DVS, DK, idesc_bf16(128, DVS));
+            const uint64_t sdesc = sdesc_k_sw128(sbase + C_SB + (it & 1) * 8192);
+            mma_sw128<8, 128, DVS>(tm + 0, sdesc_k_sw128(sbase + b * CB_SIZE + CB_M), sdesc, idesc_bf16(128, DVS));
             mma_commit(bar_s);
             {  // Qp (MN-major, no swizzle) x state image (K-major SW128)
-                const uint32_t qa = sbase + b * CB_SIZE + CB_Q;
-                for (int kk = 0; kk < DK / 16; ++kk) {
-                    const uint64_t ad = sdesc_interleave(qa + (uint32_t)kk * 2048u, 1024u, 128u);
-                    const uint64_t bd = sdesc_k_sw128(img + (uint32_t)(kk >> 2) * (DVS * 128u) + (uint32_t)(kk & 3) * 32u);
-                    mma_bf16(tm + 32 + 32 * (it & 1), ad, bd, idesc_bf16_major(64, DVS, 1, 0), kk > 0 ? 1u : 0u);
-                }
+                const uint64_t qdesc = sdesc_interleave(sbase + b * CB_SIZE + CB_Q, 1024u, 128u);
+#pragma unroll
+                for (int kk = 0; kk < DK / 16; ++kk)
+                    mma_bf16(tm + 32 + 32 * (it & 1), qdesc + (uint32_t)((kk * 2048) >> 4),
+                             sdesc + (uint32_t)(((kk >> 2) * DVS * 128 + (kk & 3) * 32) >> 4),
+                             idesc_bf16_major(64, DVS, 1, 0), kk > 0 ? 1u : 0u);
             }
             mma_commit(&bar_o[it & 1]);
             return true;
@@ -756,11 +819,9 @@ __global__ void __launch_bounds__(128, 1) chain_kernel(const ChunkArgs a) {
         // thread-0 bookkeeping for the bounded drain after a failed wait
         int loads_issued = 0, loads_waited = 0, mma_issued = 0;
         if (tid == 0) {
-            issue_load(0);
-            loads_issued = 1;
-            if (nit > 1) {
-                issue_load(1);
-                loads_issued = 2;
+            for (int j = 0; j < NBUF && j < nit; ++j) {
+                issue_load(j);
+                loads_issued = j + 1;
             }
         }
         write_state_image(0);
@@ -776,8 +837,7 @@ __global__ void __launch_bounds__(128, 1) chain_kernel(const ChunkArgs a) {
 
         int it = 0;
         for (; it < nit && !*s_fail; ++it) {
-            const int b = it & 1;
-            const uint8_t* buf = sm + b * CB_SIZE;
+            const uint8_t* buf = sm + bidx(it) * CB_SIZE;
             const int64_t t0 = s_beg + (int64_t)(c_beg + it) * CH;
             const int L = (int)((s_end - t0) < CH ? (s_end - t0) : CH);
 
@@ -843,18 +903,17 @@ __global__ void __launch_bounds__(128, 1) chain_kernel(const ChunkArgs a) {
             } else {
                 *s_fail = 1;
             }
-            // (4) buffer b fully consumed -> refill it with chunk it + 2
+            // (4) this chunk's buffer fully consumed -> refill it with chunk it + NBUF
             tc_fence_before();
             __syncthreads();
-            if (tid == 0 && it + 2 < nit && !*s_fail) {
-                issue_load(it + 2);
-                loads_issued = it + 3;
+            if (tid == 0 && it + NBUF < nit && !*s_fail) {
+                issue_load(it + NBUF);
+                loads_issued = it + NBUF + 1;
             }
         }
         // after a failed wait: let copies and products still in flight finish (bounded)
         if (tid == 0 && *s_fail) {
-            for (int j = loads_waited; j < loads_issued; ++j)
-                mbar_wait(&bar_ld[j & 1], (uint32_t)((j >> 1) & 1), nullptr);
+            for (int j = loads_waited; j < loads_issued; ++j) mbar_wait(&bar_ld[bidx(j)], bpar(j), nullptr);
             if (mma_issued > 0) {
                 const int j = mma_issued - 1;
                 mbar_wait(bar_s, (uint32_t)(j & 1), nullptr);
@@ -996,8 +1055,8 @@ cudaError_t chunk_fwd_launch(const void* q, const void* k, const void* v, const 
             const int64_t n_items = (int64_t)N * wc * H;
             const unsigned grid = (unsigned)(n_items < g_num_sms ? n_items : g_num_sms);
             prof_begin(PROF_INTRA, stream);
-            if (in_bf16) intra_kernel<true><<<grid, 256, INTRA_SMEM, stream>>>(a, maps, n_items);
-            else intra_kernel<false><<<grid, 256, INTRA_SMEM, stream>>>(a, maps, n_items);
+            if (in_bf16) intra_kernel<true><<<grid, INTRA_THREADS, INTRA_SMEM, stream>>>(a, maps, n_items);
+            else intra_kernel<false><<<grid, INTRA_THREADS, INTRA_SMEM, stream>>>(a, maps, n_items);
             if ((err = cudaGetLastError()) != cudaSuccess) return err;
             prof_end(PROF_INTRA, stream);
         }

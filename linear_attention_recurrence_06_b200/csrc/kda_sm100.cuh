@@ -48,14 +48,17 @@ KDA_DEV void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
                  : "memory");
 }
 
-KDA_DEV bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+// Tests the phase with the given parity; while it is incomplete the thread
+// may be suspended in hardware for up to `suspend_ns` (so waiting warps do not
+// consume issue slots) before the test returns false.
+KDA_DEV bool mbar_try_wait(uint64_t* bar, uint32_t parity, uint32_t suspend_ns = 1000000u) {
     uint32_t ok;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(suspend_ns)
         : "memory");
     return ok != 0;
 }
@@ -241,8 +244,11 @@ KDA_DEV float bf16_to_f32(uint16_t b) { return __uint_as_float(((uint32_t)b) << 
 KDA_DEV uint16_t f32_to_bf16(float f) {
     return __bfloat16_as_ushort(__float2bfloat16_rn(f));
 }
+// Two floats -> one 32-bit word of two bf16 (round to nearest even), one
+// paired conversion; `lo` lands in the low half.
 KDA_DEV uint32_t pack_bf16x2(float lo, float hi) {
-    return (uint32_t)f32_to_bf16(lo) | ((uint32_t)f32_to_bf16(hi) << 16);
+    const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<const uint32_t*>(&v);
 }
 
 // Loads one element of an input tensor stored as fp32 or bf16.
