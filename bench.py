@@ -57,6 +57,22 @@ def load_peaks():
     return dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0, source="fallback")
 
 
+def max_over_ranks(x: float, dist=None, device="cpu") -> float:
+    """Largest value of x over all ranks (x itself without a process group)."""
+    if dist is None:
+        return x
+    import torch
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(n_ranks: int, units_per_rank: float, ms_max: float) -> float:
+    """Weak scaling: every rank processes its own units; the job's rate is all
+    units over the slowest rank's time."""
+    return n_ranks * units_per_rank / (ms_max * 1e-3)
+
+
 def dist_env():
     ws = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -152,12 +168,8 @@ def run_ours(args, peaks):
         if dist is not None:
             dist.barrier()
 
-    def max_over_ranks(x: float) -> float:
-        if dist is None:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+    def mor(x: float) -> float:
+        return max_over_ranks(x, dist, dev)
 
     B, T, H = PREFILL["B"], PREFILL["T"], PREFILL["H"]
     tb = prefill_inputs(seed=rank)
@@ -204,14 +216,14 @@ def run_ours(args, peaks):
     e1.record(stream)
     torch.cuda.synchronize()
     barrier()
-    ms_step = max_over_ranks(e0.elapsed_time(e1) / args.steps)
+    ms_step = mor(e0.elapsed_time(e1) / args.steps)
 
     # decode sub-measurement: 1000 consecutive steps, state in place
-    dec = run_decode(args, torch, kda, dev, stream, rank, max_over_ranks, barrier)
+    dec = run_decode(args, torch, kda, dev, stream, rank, mor, barrier)
     clocks = sampler.stop() if sampler else None
 
     # end to end through the public API: pinned host inputs -> device -> call -> host output
-    e2e = run_e2e(args, torch, kda, hq, out, fs, ws, stream, max_over_ranks, barrier)
+    e2e = run_e2e(args, torch, kda, hq, out, fs, ws, stream, mor, barrier)
 
     if dist is not None:
         dist.barrier()
@@ -219,8 +231,7 @@ def run_ours(args, peaks):
     if rank != 0:
         return None
 
-    tokens = ws_n * B * T
-    value = tokens / (ms_step * 1e-3)
+    value = whole_job_rate(ws_n, B * T, ms_step)
     th = B * T * H
     bytes_call = PREFILL_BYTES_PER_TH * th
     achieved_gbs = bytes_call / (ms_step * 1e-3) / 1e9
@@ -331,7 +342,7 @@ def run_e2e(args, torch, kda, hq, out, fs, ws, stream, max_over_ranks, barrier):
     barrier()
     ms = max_over_ranks(e0.elapsed_time(e1) / n)
     ws_n = int(os.environ.get("WORLD_SIZE", "1"))
-    return {"value": ws_n * B * T / (ms * 1e-3), "unit": "tokens/s", "ms_per_step": ms,
+    return {"value": whole_job_rate(ws_n, B * T, ms), "unit": "tokens/s", "ms_per_step": ms,
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
 
