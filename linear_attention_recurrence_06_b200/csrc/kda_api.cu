@@ -22,7 +22,8 @@ size_t chunk_fixed_bytes(int n_seqs, int H, bool need_carry);
 cudaError_t chunk_fwd_launch(const void* q, const void* k, const void* v, const void* log_alpha, const void* beta,
                              const float* init_state, void* o, float* final_state, int B, int64_t T, int H,
                              const int32_t* cu, int n_seqs, int64_t max_seqlen, bool in_bf16, bool out_bf16,
-                             float scale, void* workspace, size_t ws_bytes, cudaStream_t stream, int* n_passes);
+                             float scale, const void* gate, const float* norm_w, float eps, void* workspace,
+                             size_t ws_bytes, cudaStream_t stream, int* n_passes, bool* gate_fused);
 }  // namespace kda
 
 namespace kda {
@@ -155,11 +156,12 @@ kda_status kda_chunk_fwd(const void* q, const void* k, const void* v, const void
 
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     const bool in_bf16 = in_dtype == KDA_BF16, out_bf16 = out_dtype == KDA_BF16;
+    bool fused = false;
     cudaError_t e = kda::chunk_fwd_launch(q, k, v, log_alpha, beta, init_state, o, final_state, B, T, H, cu_seqlens,
-                                          n_seqs, max_seqlen, in_bf16, out_bf16, scale, workspace, workspace_bytes,
-                                          st, nullptr);
+                                          n_seqs, max_seqlen, in_bf16, out_bf16, scale, gate, norm_weight, eps,
+                                          workspace, workspace_bytes, st, nullptr, &fused);
     if (e != cudaSuccess) return KDA_ERR_CUDA;
-    if (gate) {
+    if (gate && !fused) {
         const int64_t rows = (int64_t)B * T * H;
         // y overwrites o in place (o already holds out_dtype values)
         kda::prof_begin(kda::PROF_GATE_NORM, st);

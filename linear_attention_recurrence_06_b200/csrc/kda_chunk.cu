@@ -183,7 +183,7 @@ constexpr int LDA = 68;  // padded fp32 row stride of A and X (16-byte rows, spr
 constexpr uint32_t IY_A = IY, IY_X = IY + 64 * LDA * 4, IY_WT = IY, IY_UT = IY + 16384;
 constexpr uint32_t IM = IY + 35840;
 constexpr uint32_t IM_BETA = IM, IM_G = IM + 256, IM_TOT = IM + 256 + 2560, IM_BAR_RAW = IM_TOT + 2048,
-                   IM_BAR_MMA = IM_BAR_RAW + 8, IM_TMEM = IM_BAR_MMA + 8;
+                   IM_BAR_MMA = IM_BAR_RAW + 8, IM_NEXT = IM_BAR_MMA + 8, IM_TMEM = IM_NEXT + 32;
 constexpr uint32_t INTRA_SMEM = IM_TMEM + 16 + 1024;  // + alignment slack
 constexpr uint32_t INTRA_TMEM_COLS = 512;
 constexpr uint32_t TM_AD = 0, TM_B1 = 64, TM_B2 = 80, TM_B3 = 112, TM_WT = 160, TM_UT = 224, TM_M = 288,
@@ -222,6 +222,9 @@ intra_kernel(const ChunkArgs a, const __grid_constant__ IntraMaps maps, const in
     uint64_t* bar_raw = reinterpret_cast<uint64_t*>(sm + IM_BAR_RAW);
     uint64_t* bar_mma = reinterpret_cast<uint64_t*>(sm + IM_BAR_MMA);
     uint32_t* s_tmem = reinterpret_cast<uint32_t*>(sm + IM_TMEM);
+    // next item of this CTA: {item, t0} as int64 and {h, L} as int
+    int64_t* s_next64 = reinterpret_cast<int64_t*>(sm + IM_NEXT);
+    int* s_next32 = reinterpret_cast<int*>(sm + IM_NEXT + 16);
 
     if (warp == 0) {
         tmem_alloc(s_tmem, INTRA_TMEM_COLS);
@@ -247,10 +250,7 @@ intra_kernel(const ChunkArgs a, const __grid_constant__ IntraMaps maps, const in
         }
         return n_items;
     };
-    auto issue_raw = [&](int64_t it) {
-        int hh, LL;
-        int64_t tt;
-        item_info(a, it, hh, tt, LL);
+    auto issue_raw = [&](int hh, int64_t tt) {
         mbar_arrive_expect_tx(bar_raw, 4u * 16384u);
         tma_load_2d(sm + R_LA, &maps.la, hh * DK, (int)tt, bar_raw);
         tma_load_2d(sm + R_K, &maps.k, hh * DK, (int)tt, bar_raw);
@@ -262,15 +262,15 @@ intra_kernel(const ChunkArgs a, const __grid_constant__ IntraMaps maps, const in
     bool raw_in_flight = false;
     // beta of the next item, loaded one item ahead by threads < 64
     float beta_next = 0.f;
-    if (item < n_items && tid < CH) {
+    if (item < n_items) {
         int hh, LL;
         int64_t tt;
         item_info(a, item, hh, tt, LL);
-        beta_next = (tid < LL) ? ld_in<IN_BF16>(a.beta, (size_t)(tt + tid) * H + hh) : 0.f;
-    }
-    if constexpr (IN_BF16) {
-        if (tid == 0 && item < n_items) issue_raw(item);
-        raw_in_flight = item < n_items;
+        if (tid < CH) beta_next = (tid < LL) ? ld_in<IN_BF16>(a.beta, (size_t)(tt + tid) * H + hh) : 0.f;
+        if constexpr (IN_BF16) {
+            if (tid == 0) issue_raw(hh, tt);
+            raw_in_flight = true;
+        }
     }
 
     while (item < n_items) {
@@ -455,6 +455,16 @@ intra_kernel(const ChunkArgs a, const __grid_constant__ IntraMaps maps, const in
                 if ((j4 >> 4) > (i >> 4)) *reinterpret_cast<float4*>(sX + i * LDA + j4) = make_float4(0.f, 0.f, 0.f, 0.f);
             }
             __syncthreads();
+            if (tid == INTRA_THREADS - 1) {  // idle in the inverse: find the next item of this CTA
+                const int64_t nx = next_valid(item + gridDim.x);
+                int hh = 0, LL = 0;
+                int64_t tt = 0;
+                if (nx < n_items) item_info(a, nx, hh, tt, LL);
+                s_next64[0] = nx;
+                s_next64[1] = tt;
+                s_next32[0] = hh;
+                s_next32[1] = LL;
+            }
             if (tid < 64) {  // diagonal blocks: one thread per (block, column)
                 // column j of (I + N_bb)^-1: x_i = -sum_{m<i} N_im x_m, x_j = 1, x_i = 0 for i < j
                 // (entries above j are zero, so the sums need no masking)
@@ -579,16 +589,15 @@ intra_kernel(const ChunkArgs a, const __grid_constant__ IntraMaps maps, const in
             mma_commit(bar_mma);
         }
         // next item's raw tiles (every read of RAW for this item is done) and beta
-        const int64_t next = next_valid(item + gridDim.x);
-        if constexpr (IN_BF16) {
-            if (tid == 0 && next < n_items) issue_raw(next);
-            raw_in_flight = next < n_items;
-        }
-        if (tid < CH && next < n_items) {
-            int hh, LL;
-            int64_t tt;
-            item_info(a, next, hh, tt, LL);
-            beta_next = (tid < LL) ? ld_in<IN_BF16>(a.beta, (size_t)(tt + tid) * H + hh) : 0.f;
+        const int64_t next = s_next64[0];
+        if (next < n_items) {
+            const int64_t tt = s_next64[1];
+            const int hh = s_next32[0], LL = s_next32[1];
+            if constexpr (IN_BF16) {
+                if (tid == 0) issue_raw(hh, tt);
+                raw_in_flight = true;
+            }
+            if (tid < CH) beta_next = (tid < LL) ? ld_in<IN_BF16>(a.beta, (size_t)(tt + tid) * H + hh) : 0.f;
         }
         mbar_wait(bar_mma, ph_mma, a.status);
         ph_mma ^= 1;
@@ -703,49 +712,90 @@ intra_kernel(const ChunkArgs a, const __grid_constant__ IntraMaps maps, const in
 // ---------------------------------------------------------------------------
 // chain_kernel
 // ---------------------------------------------------------------------------
-// Threads: 128; thread c owns state row c of the 32-column slice (32 fp32
-// registers).  TMEM (128 columns): D_S = Mlr S in [0,32) (M=128, lane = row
-// c); D_O = Qp S double-buffered in [32,64) and [64,96) (M=64: row t lives in
-// lane 32*(t/16) + t%16).  Shared memory: three chunk buffers {Mlr image 32K,
-// Qp image 16K, GamC 512, Bm slice 8K, ObT slice 4K} (loads run three chunks
-// ahead) and two bf16 state operand images Sb [32 value cols][128 key rows].
-constexpr uint32_t CB_M = 0, CB_Q = 32768, CB_G = 49152, CB_B = 49664, CB_O = 57856, CB_SIZE = 62464;
-constexpr int NBUF = 3;                          // chunk buffers in flight
-constexpr uint32_t C_SB = NBUF * CB_SIZE;        // two 8K state images
-constexpr uint32_t C_BAR = C_SB + 2 * 8192;      // bar_ld[3], bar_s, bar_o[2]
-constexpr uint32_t C_FLAG = C_BAR + 48;
-constexpr uint32_t C_TMEM = C_FLAG + 16;
-constexpr uint32_t CHAIN_SMEM = C_TMEM + 16 + 1024;
+// One CTA per (sequence, head, 32-column value slice), warp-specialised:
+//   warps 0-3 (consumers): thread c owns state row c of the slice (32 fp32
+//     registers); applies S <- GamC o S - Mlr S + Bm, writes the next bf16
+//     state operand image, then forms the chunk output o = Qp S + Ob;
+//   warp 4 (producer, one thread): bulk loads of the chunk operands (three
+//     chunks ahead) and the tensor-core products Mlr S and Qp S.
+// The two sides meet only on mbarriers, so the issue of the next products
+// overlaps the output work of the current chunk.  TMEM (128 columns): D_S =
+// Mlr S in [0,32) (M=128, lane = row c); D_O = Qp S double-buffered in [32,64)
+// and [64,96) (M=64: row t lives in lane 32*(t/16) + t%16).  Shared memory:
+// three chunk buffers {Mlr image 32K, Qp image 16K, GamC 512, Bm slice 8K, ObT
+// slice 4K[, gate tile 4K]} and two bf16 state operand images Sb [32 value
+// cols][128 key rows].
+//
+// Barriers and the order that keeps each phase from being skipped:
+//   bar_img   consumers (128) -> producer: state image of chunk i written.  The
+//             image of chunk i + 1 is written after D_S(i) is read, i.e. after
+//             the producer issued chunk i.
+//   bar_s     commit of Mlr S(i); it also covers Qp S(i - 1), so the image
+//             that product read may be rewritten once bar_s(i) is seen.
+//   bar_o[2]  commit of Qp S(i) into D_O[i & 1]; D_O[i & 1] is overwritten by
+//             chunk i + 2, issued after the image of i + 2, which consumers
+//             write after reading D_O(i).
+//   bar_ld[3] loads of a buffer; bar_free[3] consumers (128) -> producer: the
+//             buffer is no longer read and may be refilled.
+//
+// With the fused gate (GATE), the four CTAs of one (sequence, head) -- its four
+// value-column slices -- form a thread-block cluster.  The per-head RMSNorm
+// needs sum_j o_tj^2 over all 128 columns: each CTA pushes its 64 per-row
+// partial sums into every CTA's shared memory (distributed shared memory) with
+// asynchronous stores that count down a transaction barrier in the receiving
+// CTA; the normalisation of chunk i is finished during iteration i + 1.
+// Reuse of the two partial-sum slots: a peer writes row t of slot i & 1 for
+// chunk i + 2 only after it has received every CTA's chunk-(i + 1) partials,
+// and this CTA's row-t thread sends its chunk-(i + 1) partial after it has read
+// row t of the chunk-i slot.
+constexpr uint32_t CB_M = 0, CB_Q = 32768, CB_G = 49152, CB_B = 49664, CB_O = 57856, CB_GT = 61952;
+constexpr int NBUF = 3;  // chunk buffers in flight
+template <bool GATE> struct ChainLayout {
+    static constexpr uint32_t CB_SIZE = GATE ? 66560u : 62464u;  // multiples of 1024
+    static constexpr uint32_t SB = NBUF * CB_SIZE;                // two 8K state images
+    static constexpr uint32_t PART = SB + 2 * 8192;               // [2][4 slices][64 rows] fp32
+    static constexpr uint32_t BAR = PART + (GATE ? 2048u : 0u);   // barriers (128 B)
+    static constexpr uint32_t TMEMP = BAR + 128;
+    static constexpr uint32_t SMEM = TMEMP + 16 + 1024;
+};
 constexpr uint32_t CHAIN_TMEM_COLS = 128;
+constexpr int CHAIN_THREADS = 160;  // 4 consumer warps + 1 producer warp
+constexpr int CLUSTER = NSL;        // CTAs per (sequence, head) when the gate is fused
+constexpr uint32_t PART_TX = CLUSTER * 64 * 4;  // partial-sum bytes each CTA receives per chunk
 
-template <bool OUT_BF16>
-__global__ void __launch_bounds__(128, 1) chain_kernel(const ChunkArgs a) {
+template <bool OUT_BF16, bool GATE>
+__global__ void __launch_bounds__(CHAIN_THREADS, 1)
+chain_kernel(const ChunkArgs a, const __grid_constant__ CUtensorMap gate_map, const float* __restrict__ norm_w,
+             float eps) {
+    using LY = ChainLayout<GATE>;
+    constexpr uint32_t CB_SIZE = LY::CB_SIZE;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     const uint32_t sbase = smem_u32(sm);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const bool consumer = warp < 4;
     const int js = blockIdx.x, h = blockIdx.y, n = blockIdx.z;
     const int H = a.H;
-    uint64_t* bar_ld = reinterpret_cast<uint64_t*>(sm + C_BAR);  // [NBUF]
-    uint64_t* bar_s = reinterpret_cast<uint64_t*>(sm + C_BAR + 24);
-    // one output barrier per D_O buffer: the next chunk's output product is
-    // committed before this chunk's output is waited for, so a single barrier
-    // could complete two phases between waits
-    uint64_t* bar_o = reinterpret_cast<uint64_t*>(sm + C_BAR + 32);  // [2]
-    volatile int* s_fail = reinterpret_cast<volatile int*>(sm + C_FLAG);
-    uint32_t* s_tmem = reinterpret_cast<uint32_t*>(sm + C_TMEM);
+    uint64_t* bar_ld = reinterpret_cast<uint64_t*>(sm + LY::BAR);         // [NBUF]
+    uint64_t* bar_free = reinterpret_cast<uint64_t*>(sm + LY::BAR + 24);  // [NBUF]
+    uint64_t* bar_s = reinterpret_cast<uint64_t*>(sm + LY::BAR + 48);
+    uint64_t* bar_o = reinterpret_cast<uint64_t*>(sm + LY::BAR + 56);     // [2]
+    uint64_t* bar_img = reinterpret_cast<uint64_t*>(sm + LY::BAR + 72);
+    uint64_t* bar_part = reinterpret_cast<uint64_t*>(sm + LY::BAR + 80);  // [2], gate only
+    float* s_part = reinterpret_cast<float*>(sm + LY::PART);              // [2][4][64], gate only
+    uint32_t* s_tmem = reinterpret_cast<uint32_t*>(sm + LY::TMEMP);
 
     int64_t s_beg, s_end;
     seq_range(a, n, s_beg, s_end);
     const int nchunks = (int)((s_end - s_beg + CH - 1) / CH);
     const int c_beg = a.i0;
     const int c_end = min(a.i0 + a.wc, nchunks);
-    const int nit = c_end > c_beg ? c_end - c_beg : 0;
+    const int nit = c_end > c_beg ? c_end - c_beg : 0;  // the same for the whole cluster
 
     // state slice: row tid, columns [32 js, 32 js + 32)
-    const size_t st_off = (((size_t)n * H + h) * DK + tid) * DV + (size_t)DVS * js;
+    const size_t st_off = (((size_t)n * H + h) * DK + (consumer ? tid : 0)) * DV + (size_t)DVS * js;
     float S[DVS];
-    {
+    if (consumer) {
         const float* src = a.first_pass ? a.init_state : a.state_io;
         if (src) {
 #pragma unroll
@@ -765,132 +815,141 @@ __global__ void __launch_bounds__(128, 1) chain_kernel(const ChunkArgs a) {
             tmem_relinquish();
         }
         if (tid == 0) {
-            for (int i = 0; i < NBUF; ++i) mbar_init(&bar_ld[i], 1);
+            for (int i = 0; i < NBUF; ++i) {
+                mbar_init(&bar_ld[i], 1);
+                mbar_init(&bar_free[i], 128);
+            }
             mbar_init(bar_s, 1);
             mbar_init(&bar_o[0], 1);
             mbar_init(&bar_o[1], 1);
+            mbar_init(bar_img, 128);
+            if constexpr (GATE) {
+                // one local arrival (with the byte count) plus 4 B from every row of every CTA per chunk
+                mbar_init(&bar_part[0], 1);
+                mbar_init(&bar_part[1], 1);
+                mbar_arrive_expect_tx(&bar_part[0], PART_TX);
+                mbar_arrive_expect_tx(&bar_part[1], PART_TX);
+            }
             fence_mbar_init();
-            *s_fail = 0;
         }
         __syncthreads();
+        if constexpr (GATE) cluster_sync_all();  // peers' barriers exist before any remote store
         tc_fence_after();
         const uint32_t tm = *s_tmem;
-        const uint32_t lane_addr = tm + ((uint32_t)(32 * warp) << 16);
         const size_t slot0 = ((size_t)n * a.wc + (c_beg - a.i0)) * H + h;  // slot of iteration 0
         // chunk buffer of iteration it and its barrier phase
         auto bidx = [](int it) { return it % NBUF; };
         auto bpar = [](int it) { return (uint32_t)((it / NBUF) & 1); };
-        auto issue_load = [&](int it) {
-            const int b = bidx(it);
-            uint8_t* buf = sm + b * CB_SIZE;
-            const uint8_t* src = a.ws + (slot0 + (size_t)it * H) * SLOT_BYTES;
-            mbar_arrive_expect_tx(&bar_ld[b], SO_MQG + BSL + OSL);
-            bulk_g2s(buf + CB_M, src + SO_M, SO_MQG, &bar_ld[b]);
-            bulk_g2s(buf + CB_B, src + SO_B + (size_t)js * BSL, BSL, &bar_ld[b]);
-            bulk_g2s(buf + CB_O, src + SO_O + (size_t)js * OSL, OSL, &bar_ld[b]);
-        };
-        auto write_state_image = [&](int it) {
-            const uint32_t kb = (uint32_t)tid >> 6, kc = (uint32_t)tid & 63u;
-            uint8_t* img = sm + C_SB + (it & 1) * 8192;
-#pragma unroll
-            for (int j = 0; j < DVS; ++j)
-                *reinterpret_cast<uint16_t*>(img + kb * (DVS * 128) + sw128_off((uint32_t)j, kc)) = f32_to_bf16(S[j]);
-        };
-        // thread 0: Mlr S -> D_S (commit bar_s), then Qp S -> D_O[it&1] (commit bar_o[it&1])
-        auto issue_mma = [&](int it) -> bool {
-            const int b = bidx(it);
-            if (!mbar_wait(&bar_ld[b], bpar(it), a.status)) return false;
-            tc_fence_after();
-            const uint64_t sdesc = sdesc_k_sw128(sbase + C_SB + (it & 1) * 8192);
-            mma_sw128<8, 128, DVS>(tm + 0, sdesc_k_sw128(sbase + b * CB_SIZE + CB_M), sdesc, idesc_bf16(128, DVS));
-            mma_commit(bar_s);
-            {  // Qp (MN-major, no swizzle) x state image (K-major SW128)
-                const uint64_t qdesc = sdesc_interleave(sbase + b * CB_SIZE + CB_Q, 1024u, 128u);
-#pragma unroll
-                for (int kk = 0; kk < DK / 16; ++kk)
-                    mma_bf16(tm + 32 + 32 * (it & 1), qdesc + (uint32_t)((kk * 2048) >> 4),
-                             sdesc + (uint32_t)(((kk >> 2) * DVS * 128 + (kk & 3) * 32) >> 4),
-                             idesc_bf16_major(64, DVS, 1, 0), kk > 0 ? 1u : 0u);
-            }
-            mma_commit(&bar_o[it & 1]);
-            return true;
-        };
-
-        // thread-0 bookkeeping for the bounded drain after a failed wait
+        bool failed = false;
+        // producer bookkeeping for the bounded drain after a failed wait
         int loads_issued = 0, loads_waited = 0, mma_issued = 0;
-        if (tid == 0) {
-            for (int j = 0; j < NBUF && j < nit; ++j) {
-                issue_load(j);
-                loads_issued = j + 1;
-            }
-        }
-        write_state_image(0);
-        fence_async_smem();
-        __syncthreads();
-        tc_fence_after();
-        if (tid == 0) {
-            loads_waited = 1;
-            if (issue_mma(0)) mma_issued = 1;
-            else *s_fail = 1;
-        }
-        __syncthreads();
 
-        int it = 0;
-        for (; it < nit && !*s_fail; ++it) {
-            const uint8_t* buf = sm + bidx(it) * CB_SIZE;
-            const int64_t t0 = s_beg + (int64_t)(c_beg + it) * CH;
-            const int L = (int)((s_end - t0) < CH ? (s_end - t0) : CH);
-
-            // (1) state update: S <- GamC o S - Mlr S + Bm
-            if (mbar_wait(bar_s, (uint32_t)(it & 1), a.status)) {
-                tc_fence_after();
-                float ds[DVS];
-                tmem_ld32(lane_addr + 0, ds);
-                tmem_ld_wait();
-                const float gamC = *reinterpret_cast<const float*>(buf + CB_G + 4 * tid);
-                const uint4* bsrc = reinterpret_cast<const uint4*>(buf + CB_B + (uint32_t)tid * DVS * 2);
+        if (!consumer) {
+            // ------------------------------------------------------ producer
+            if (lane == 0) {
+                auto issue_load = [&](int it) {
+                    const int b = bidx(it);
+                    uint8_t* buf = sm + b * CB_SIZE;
+                    const uint8_t* src = a.ws + (slot0 + (size_t)it * H) * SLOT_BYTES;
+                    mbar_arrive_expect_tx(&bar_ld[b], SO_MQG + BSL + OSL + (GATE ? (uint32_t)(CH * DVS * 2) : 0u));
+                    bulk_g2s(buf + CB_M, src + SO_M, SO_MQG, &bar_ld[b]);
+                    bulk_g2s(buf + CB_B, src + SO_B + (size_t)js * BSL, BSL, &bar_ld[b]);
+                    bulk_g2s(buf + CB_O, src + SO_O + (size_t)js * OSL, OSL, &bar_ld[b]);
+                    if constexpr (GATE)  // gate tile [64 tokens][32 value cols] of this slice
+                        tma_load_2d(buf + CB_GT, &gate_map, h * DV + DVS * js,
+                                    (int)(s_beg + (int64_t)(c_beg + it) * CH), &bar_ld[b]);
+                };
+                for (int j = 0; j < NBUF && j < nit; ++j) {
+                    issue_load(j);
+                    loads_issued = j + 1;
+                }
+                for (int it = 0; it < nit; ++it) {
+                    const int b = bidx(it);
+                    if (!mbar_wait(bar_img, (uint32_t)(it & 1), a.status) ||
+                        !mbar_wait(&bar_ld[b], bpar(it), a.status)) {
+                        failed = true;
+                        break;
+                    }
+                    loads_waited = it + 1;
+                    tc_fence_after();
+                    // Mlr S -> D_S, then Qp S -> D_O[it & 1]
+                    const uint64_t sdesc = sdesc_k_sw128(sbase + LY::SB + (it & 1) * 8192);
+                    mma_sw128<8, 128, DVS>(tm + 0, sdesc_k_sw128(sbase + b * CB_SIZE + CB_M), sdesc,
+                                           idesc_bf16(128, DVS));
+                    mma_commit(bar_s);
+                    {  // Qp (MN-major, no swizzle) x state image (K-major SW128)
+                        const uint64_t qdesc = sdesc_interleave(sbase + b * CB_SIZE + CB_Q, 1024u, 128u);
 #pragma unroll
-                for (int m = 0; m < DVS / 8; ++m) {
-                    const uint4 w = bsrc[m];
-                    const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-                    for (int p = 0; p < 4; ++p) {
-                        const int j = 8 * m + 2 * p;
-                        S[j] = gamC * S[j] - ds[j] + __uint_as_float(ww[p] << 16);
-                        S[j + 1] = gamC * S[j + 1] - ds[j + 1] + __uint_as_float(ww[p] & 0xFFFF0000u);
+                        for (int kk = 0; kk < DK / 16; ++kk)
+                            mma_bf16(tm + 32 + 32 * (it & 1), qdesc + (uint32_t)((kk * 2048) >> 4),
+                                     sdesc + (uint32_t)(((kk >> 2) * DVS * 128 + (kk & 3) * 32) >> 4),
+                                     idesc_bf16_major(64, DVS, 1, 0), kk > 0 ? 1u : 0u);
+                    }
+                    mma_commit(&bar_o[it & 1]);
+                    mma_issued = it + 1;
+                    // refill the buffer of the previous chunk once the consumers released it
+                    const int r = it - 1 + NBUF;
+                    if (it >= 1 && r < nit) {
+                        if (!mbar_wait(&bar_free[bidx(it - 1)], bpar(it - 1), a.status)) {
+                            failed = true;
+                            break;
+                        }
+                        issue_load(r);
+                        loads_issued = r + 1;
                     }
                 }
-            } else {
-                *s_fail = 1;
             }
-            // (2) next chunk's products as early as possible
-            if (it + 1 < nit) write_state_image(it + 1);
-            fence_async_smem();
-            tc_fence_before();
-            __syncthreads();
-            tc_fence_after();
-            if (*s_fail) break;
-            if (tid == 0 && it + 1 < nit) {
-                loads_waited = it + 2;
-                if (issue_mma(it + 1)) mma_issued = it + 2;
-                else *s_fail = 1;
-            }
-            // (3) this chunk's output: o = Qp S + Ob
-            if (mbar_wait(&bar_o[it & 1], (uint32_t)((it >> 1) & 1), a.status)) {
-                tc_fence_after();
-                float dO[DVS];
-                tmem_ld32(lane_addr + 32 + 32 * (it & 1), dO);
-                tmem_ld_wait();
-                const int trow = 16 * warp + (lane & 15);
-                if (lane < 16 && trow < L) {
-                    // Ob^T slice [32 value cols][64 tokens]: column trow
-                    const uint16_t* osrc = reinterpret_cast<const uint16_t*>(buf + CB_O) + trow;
-                    const size_t obase = ((size_t)(t0 + trow) * H + h) * DV + (size_t)DVS * js;
+        } else {
+            // ----------------------------------------------------- consumers
+            const uint32_t lane_addr = tm + ((uint32_t)(32 * warp) << 16);
+            auto write_state_image = [&](int it) {
+                const uint32_t kb = (uint32_t)tid >> 6, kc = (uint32_t)tid & 63u;
+                uint8_t* img = sm + LY::SB + (it & 1) * 8192;
 #pragma unroll
-                    for (int m = 0; m < DVS / 8; ++m) {
+                for (int j = 0; j < DVS; ++j)
+                    *reinterpret_cast<uint16_t*>(img + kb * (DVS * 128) + sw128_off((uint32_t)j, kc)) =
+                        f32_to_bf16(S[j]);
+                fence_async_smem();
+                tc_fence_before();
+                mbar_arrive(bar_img);
+            };
+
+            // output row served by this lane: lanes 0-15 hold it in TMEM (M = 64
+            // layout); with the fused gate, lanes 16-31 take over its columns 16-31
+            const int trow = 16 * warp + (lane & 15);
+            const int hi = lane >> 4;
+            constexpr int HC = DVS / 2;  // columns per lane in the gate epilogue
+            float w16[GATE ? HC : 1];
+            float o_prev[GATE ? HC : 1];
+            uint32_t g_prev[GATE ? HC / 2 : 1];
+            int64_t t0_prev = 0;
+            int L_prev = 0;
+            if constexpr (GATE) {
+#pragma unroll
+                for (int j = 0; j < HC; ++j) w16[j] = norm_w ? __ldg(norm_w + DVS * js + HC * hi + j) : 1.0f;
+            }
+            // finishes y = o * rsqrt(mean o^2 + eps) * w * sigmoid(g) for chunk itp
+            auto finish_prev = [&](int itp) -> bool {
+                if (!mbar_wait_cluster(&bar_part[itp & 1], (uint32_t)((itp >> 1) & 1), a.status)) return false;
+                // arm the slot's barrier for chunk itp + 2 (its bytes may already be arriving)
+                if (tid == 0 && itp + 2 < nit) mbar_arrive_expect_tx(&bar_part[itp & 1], PART_TX);
+                if (trow < L_prev) {
+                    const float* pp = s_part + (itp & 1) * (CLUSTER * 64);
+                    float ss = 0.f;
+#pragma unroll
+                    for (int r = 0; r < CLUSTER; ++r) ss += pp[r * 64 + trow];
+                    const float inv = rsqrtf(ss * (1.0f / DV) + eps);
+                    const size_t obase = ((size_t)(t0_prev + trow) * H + h) * DV + (size_t)DVS * js + HC * hi;
+#pragma unroll
+                    for (int m = 0; m < HC / 8; ++m) {
                         float y8[8];
 #pragma unroll
-                        for (int p = 0; p < 8; ++p) y8[p] = dO[8 * m + p] + bf16_to_f32(osrc[(8 * m + p) * CH]);
+                        for (int p = 0; p < 8; ++p) {
+                            const int j = 8 * m + p;
+                            const float gj =
+                                __uint_as_float((j & 1) ? (g_prev[j >> 1] & 0xFFFF0000u) : (g_prev[j >> 1] << 16));
+                            y8[p] = o_prev[j] * inv * w16[j] * __fdividef(1.0f, 1.0f + __expf(-gj));
+                        }
                         if constexpr (OUT_BF16) {
                             reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(a.o) + obase)[m] = pack8(y8);
                         } else {
@@ -900,19 +959,119 @@ __global__ void __launch_bounds__(128, 1) chain_kernel(const ChunkArgs a) {
                         }
                     }
                 }
-            } else {
-                *s_fail = 1;
+                return true;
+            };
+
+            write_state_image(0);
+            for (int it = 0; it < nit; ++it) {
+                const int b = bidx(it);
+                const uint8_t* buf = sm + b * CB_SIZE;
+                const int64_t t0 = s_beg + (int64_t)(c_beg + it) * CH;
+                const int L = (int)((s_end - t0) < CH ? (s_end - t0) : CH);
+
+                // (1) state update: S <- GamC o S - Mlr S + Bm
+                if (!mbar_wait(bar_s, (uint32_t)(it & 1), a.status) || !mbar_wait(&bar_ld[b], bpar(it), a.status)) {
+                    failed = true;
+                    break;
+                }
+                tc_fence_after();
+                {
+                    float ds[DVS];
+                    tmem_ld32(lane_addr + 0, ds);
+                    tmem_ld_wait();
+                    const float gamC = *reinterpret_cast<const float*>(buf + CB_G + 4 * tid);
+                    const uint4* bsrc = reinterpret_cast<const uint4*>(buf + CB_B + (uint32_t)tid * DVS * 2);
+#pragma unroll
+                    for (int m = 0; m < DVS / 8; ++m) {
+                        const uint4 w = bsrc[m];
+                        const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                        for (int p = 0; p < 4; ++p) {
+                            const int j = 8 * m + 2 * p;
+                            S[j] = gamC * S[j] - ds[j] + __uint_as_float(ww[p] << 16);
+                            S[j + 1] = gamC * S[j + 1] - ds[j + 1] + __uint_as_float(ww[p] & 0xFFFF0000u);
+                        }
+                    }
+                }
+                // (2) the next chunk's state operand (D_S has been read)
+                if (it + 1 < nit) write_state_image(it + 1);
+
+                // (3) this chunk's output: o = Qp S + Ob  (then y, when the gate is fused)
+                if (!mbar_wait(&bar_o[it & 1], (uint32_t)((it >> 1) & 1), a.status)) {
+                    failed = true;
+                    break;
+                }
+                tc_fence_after();
+                float ov[DVS];
+                {
+                    float dO[DVS];
+                    tmem_ld32(lane_addr + 32 + 32 * (it & 1), dO);
+                    tmem_ld_wait();
+                    // Ob^T slice [32 value cols][64 tokens]: column trow
+                    const uint16_t* osrc = reinterpret_cast<const uint16_t*>(buf + CB_O) + trow;
+#pragma unroll
+                    for (int j = 0; j < DVS; ++j) ov[j] = dO[j] + bf16_to_f32(osrc[j * CH]);
+                }
+                if constexpr (!GATE) {
+                    if (lane < 16 && trow < L) {
+                        const size_t obase = ((size_t)(t0 + trow) * H + h) * DV + (size_t)DVS * js;
+#pragma unroll
+                        for (int m = 0; m < DVS / 8; ++m) {
+                            if constexpr (OUT_BF16) {
+                                reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(a.o) + obase)[m] = pack8(ov + 8 * m);
+                            } else {
+                                float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(a.o) + obase) + 2 * m;
+                                dst[0] = make_float4(ov[8 * m], ov[8 * m + 1], ov[8 * m + 2], ov[8 * m + 3]);
+                                dst[1] = make_float4(ov[8 * m + 4], ov[8 * m + 5], ov[8 * m + 6], ov[8 * m + 7]);
+                            }
+                        }
+                    }
+                } else {
+                    // finish the previous chunk first (its partials are read before this
+                    // chunk's partials are published, which orders the slot reuse)
+                    if (it > 0 && !finish_prev(it - 1)) {
+                        failed = true;
+                        break;
+                    }
+                    float ss = 0.f;
+#pragma unroll
+                    for (int j = 0; j < HC; ++j) {
+                        const float up = __shfl_up_sync(0xFFFFFFFFu, ov[HC + j], 16);
+                        o_prev[j] = hi ? up : ov[j];
+                        ss += o_prev[j] * o_prev[j];
+                    }
+                    ss += __shfl_down_sync(0xFFFFFFFFu, ss, 16);  // lanes 0-15: the whole 32-column row
+                    {  // this chunk's gate columns of the lane's row, kept for the next iteration
+                        const uint4* gsrc =
+                            reinterpret_cast<const uint4*>(buf + CB_GT + (uint32_t)trow * DVS * 2) + 2 * hi;
+#pragma unroll
+                        for (int m = 0; m < HC / 8; ++m) {
+                            const uint4 w = gsrc[m];
+                            g_prev[4 * m] = w.x; g_prev[4 * m + 1] = w.y; g_prev[4 * m + 2] = w.z; g_prev[4 * m + 3] = w.w;
+                        }
+                    }
+                    if (lane < 16) {
+                        const uint32_t slot = smem_u32(s_part + (it & 1) * (CLUSTER * 64) + js * 64 + trow);
+                        const uint32_t barl = smem_u32(&bar_part[it & 1]);
+#pragma unroll
+                        for (int r = 0; r < CLUSTER; ++r)
+                            st_async_f32(map_to_cta(slot, (uint32_t)r), ss, map_to_cta(barl, (uint32_t)r));
+                    }
+                    t0_prev = t0;
+                    L_prev = L;
+                }
+                // (4) this chunk's buffer and D_O[it & 1] are no longer read
+                tc_fence_before();
+                mbar_arrive(&bar_free[b]);
             }
-            // (4) this chunk's buffer fully consumed -> refill it with chunk it + NBUF
-            tc_fence_before();
-            __syncthreads();
-            if (tid == 0 && it + NBUF < nit && !*s_fail) {
-                issue_load(it + NBUF);
-                loads_issued = it + NBUF + 1;
+            if constexpr (GATE) {
+                if (!failed && !finish_prev(nit - 1)) failed = true;
             }
         }
+
         // after a failed wait: let copies and products still in flight finish (bounded)
-        if (tid == 0 && *s_fail) {
+        __syncthreads();
+        if (!consumer && lane == 0 && (failed || loads_waited < loads_issued)) {
             for (int j = loads_waited; j < loads_issued; ++j) mbar_wait(&bar_ld[bidx(j)], bpar(j), nullptr);
             if (mma_issued > 0) {
                 const int j = mma_issued - 1;
@@ -924,12 +1083,15 @@ __global__ void __launch_bounds__(128, 1) chain_kernel(const ChunkArgs a) {
         __syncthreads();
         tc_fence_after();
         if (warp == 0) tmem_dealloc(tm, CHAIN_TMEM_COLS);
+        if constexpr (GATE) cluster_sync_all();  // no CTA leaves while a peer may still write to it
     }
 
     // write the carried / final state slice
+    if (consumer) {
 #pragma unroll
-    for (int j = 0; j < DVS; j += 4)
-        *reinterpret_cast<float4*>(a.state_io + st_off + j) = make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]);
+        for (int j = 0; j < DVS; j += 4)
+            *reinterpret_cast<float4*>(a.state_io + st_off + j) = make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]);
+    }
 }
 
 // Flags cu_seqlens that contradict T, n_seqs or max_seqlen (one thread).
@@ -969,13 +1131,13 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
     return fn;
 }
 
-// [rows, row_elems] bf16 tensor, box = 64 rows x 128 elements, no swizzle.
-bool make_tile_map(CUtensorMap* m, const void* base, int64_t rows, int64_t row_elems) {
+// [rows, row_elems] bf16 tensor, box = 64 rows x box_w elements, no swizzle.
+bool make_tile_map(CUtensorMap* m, const void* base, int64_t rows, int64_t row_elems, uint32_t box_w = 128) {
     auto enc = tensor_map_encoder();
     if (!enc) return false;
     cuuint64_t dims[2] = {(cuuint64_t)row_elems, (cuuint64_t)rows};
     cuuint64_t strides[1] = {(cuuint64_t)row_elems * 2};
-    cuuint32_t box[2] = {128, 64};
+    cuuint32_t box[2] = {box_w, 64};
     cuuint32_t estr[2] = {1, 1};
     return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -990,17 +1152,24 @@ int g_num_sms = 0;
 cudaError_t chunk_fwd_launch(const void* q, const void* k, const void* v, const void* log_alpha, const void* beta,
                              const float* init_state, void* o, float* final_state, int B, int64_t T, int H,
                              const int32_t* cu, int n_seqs, int64_t max_seqlen, bool in_bf16, bool out_bf16,
-                             float scale, void* workspace, size_t ws_bytes, cudaStream_t stream, int* n_passes) {
+                             float scale, const void* gate, const float* norm_w, float eps, void* workspace,
+                             size_t ws_bytes, cudaStream_t stream, int* n_passes, bool* gate_fused) {
     cudaError_t err;
     if (!g_attr_set) {
         err = cudaFuncSetAttribute(intra_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, INTRA_SMEM);
         if (err != cudaSuccess) return err;
         err = cudaFuncSetAttribute(intra_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, INTRA_SMEM);
         if (err != cudaSuccess) return err;
-        err = cudaFuncSetAttribute(chain_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, CHAIN_SMEM);
-        if (err != cudaSuccess) return err;
-        err = cudaFuncSetAttribute(chain_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, CHAIN_SMEM);
-        if (err != cudaSuccess) return err;
+        const int plain = (int)ChainLayout<false>::SMEM, fused = (int)ChainLayout<true>::SMEM;
+        if ((err = cudaFuncSetAttribute(chain_kernel<true, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        plain)) != cudaSuccess ||
+            (err = cudaFuncSetAttribute(chain_kernel<false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        plain)) != cudaSuccess ||
+            (err = cudaFuncSetAttribute(chain_kernel<true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        fused)) != cudaSuccess ||
+            (err = cudaFuncSetAttribute(chain_kernel<false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        fused)) != cudaSuccess)
+            return err;
         int dev = 0;
         if ((err = cudaGetDevice(&dev)) != cudaSuccess) return err;
         if ((err = cudaDeviceGetAttribute(&g_num_sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return err;
@@ -1037,6 +1206,14 @@ cudaError_t chunk_fwd_launch(const void* q, const void* k, const void* v, const 
             !make_tile_map(&maps.v, v, total_tokens, (int64_t)H * DV))
             return cudaErrorInvalidValue;
     }
+    // gate + RMSNorm fused into the chain when the gate is bf16 (its tile
+    // arrives by TMA); an fp32 gate is applied by the separate row kernel
+    const bool fuse = gate != nullptr && in_bf16;
+    CUtensorMap gate_map;
+    memset(&gate_map, 0, sizeof(gate_map));
+    if (fuse && total_tokens > 0 && !make_tile_map(&gate_map, gate, total_tokens, (int64_t)H * DV, DVS))
+        return cudaErrorInvalidValue;
+    if (gate_fused) *gate_fused = fuse;
 
     err = cudaMemsetAsync(status, 0, 4, stream);
     if (err != cudaSuccess) return err;
@@ -1062,9 +1239,30 @@ cudaError_t chunk_fwd_launch(const void* q, const void* k, const void* v, const 
         }
         const dim3 gc((unsigned)NSL, (unsigned)H, (unsigned)N);
         prof_begin(PROF_CHAIN, stream);
-        if (out_bf16) chain_kernel<true><<<gc, 128, CHAIN_SMEM, stream>>>(a);
-        else chain_kernel<false><<<gc, 128, CHAIN_SMEM, stream>>>(a);
-        if ((err = cudaGetLastError()) != cudaSuccess) return err;
+        if (!fuse) {
+            const unsigned sm_bytes = ChainLayout<false>::SMEM;
+            if (out_bf16) chain_kernel<true, false><<<gc, CHAIN_THREADS, sm_bytes, stream>>>(a, gate_map, norm_w, eps);
+            else chain_kernel<false, false><<<gc, CHAIN_THREADS, sm_bytes, stream>>>(a, gate_map, norm_w, eps);
+            if ((err = cudaGetLastError()) != cudaSuccess) return err;
+        } else {
+            // the four value-column slices of one (sequence, head) form a cluster
+            cudaLaunchConfig_t cfg;
+            memset(&cfg, 0, sizeof(cfg));
+            cfg.gridDim = gc;
+            cfg.blockDim = dim3(CHAIN_THREADS, 1, 1);
+            cfg.dynamicSmemBytes = ChainLayout<true>::SMEM;
+            cfg.stream = stream;
+            cudaLaunchAttribute attr[1];
+            attr[0].id = cudaLaunchAttributeClusterDimension;
+            attr[0].val.clusterDim.x = CLUSTER;
+            attr[0].val.clusterDim.y = 1;
+            attr[0].val.clusterDim.z = 1;
+            cfg.attrs = attr;
+            cfg.numAttrs = 1;
+            err = out_bf16 ? cudaLaunchKernelEx(&cfg, chain_kernel<true, true>, a, gate_map, norm_w, eps)
+                           : cudaLaunchKernelEx(&cfg, chain_kernel<false, true>, a, gate_map, norm_w, eps);
+            if (err != cudaSuccess) return err;
+        }
         prof_end(PROF_CHAIN, stream);
         ++passes;
     }

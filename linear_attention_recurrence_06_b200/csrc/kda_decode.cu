@@ -105,7 +105,7 @@ decode_step_kernel(float* __restrict__ state, const void* __restrict__ q, const 
         for (int c = 0; c < 4; ++c) {
             const float gg = ld_in<IN_BF16>(gate, (size_t)bh * D + col + c);
             const float wc = norm_w ? __ldg(norm_w + col + c) : 1.0f;
-            oc[c] = oc[c] * inv * wc / (1.0f + __expf(-gg));
+            oc[c] = oc[c] * inv * wc * __fdividef(1.0f, 1.0f + __expf(-gg));
         }
     }
     if (r0 == 0) {
@@ -115,52 +115,69 @@ decode_step_kernel(float* __restrict__ state, const void* __restrict__ q, const 
 }
 
 // y = o / sqrt(mean(o^2) + eps) * w * sigmoid(g) over rows of dv = 128.
-// One warp per row, 4 consecutive channels per lane; grid-stride over rows.
-// In place (y == o) is safe: a warp reads its whole row before it writes.
+// Half a warp per row (8 consecutive channels = 16 bytes of bf16 per lane),
+// two rows per warp, grid-stride over row pairs (warp-uniform trip count).  In place (y == o) is safe:
+// each half-warp reads its whole row before it writes it.
+template <bool BF>
+KDA_DEV void load8(const void* base, size_t idx, float* v) {
+    if constexpr (BF) {
+        const uint4 w = *reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(base) + idx);
+        const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int p = 0; p < 4; ++p) {
+            v[2 * p] = __uint_as_float(ww[p] << 16);
+            v[2 * p + 1] = __uint_as_float(ww[p] & 0xFFFF0000u);
+        }
+    } else {
+        const float4 a = *reinterpret_cast<const float4*>(reinterpret_cast<const float*>(base) + idx);
+        const float4 b = *reinterpret_cast<const float4*>(reinterpret_cast<const float*>(base) + idx + 4);
+        v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+    }
+}
+
 template <bool O_BF16, bool G_BF16, bool OUT_BF16>
 __global__ void __launch_bounds__(256)
 gate_norm_kernel(const void* o, const void* __restrict__ g, const float* __restrict__ norm_w, float eps,
                  void* y, int64_t rows) {
     constexpr int D = 128;
-    const int lane = threadIdx.x & 31;
+    const int lane = threadIdx.x & 31, sub = lane & 15;
     const int64_t warps_total = (int64_t)gridDim.x * (blockDim.x >> 5);
-    float w4[4];
+    float w8[8];
 #pragma unroll
-    for (int c = 0; c < 4; ++c) w4[c] = norm_w ? __ldg(norm_w + lane * 4 + c) : 1.0f;
-    for (int64_t row = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); row < rows;
-         row += warps_total) {
-        const size_t base = (size_t)row * D + lane * 4;
-        float ov[4], gv[4];
-        if constexpr (O_BF16) {
-            const uint2 ob = *reinterpret_cast<const uint2*>(reinterpret_cast<const uint16_t*>(o) + base);
-            ov[0] = __uint_as_float(ob.x << 16); ov[1] = __uint_as_float(ob.x & 0xFFFF0000u);
-            ov[2] = __uint_as_float(ob.y << 16); ov[3] = __uint_as_float(ob.y & 0xFFFF0000u);
+    for (int c = 0; c < 8; ++c) w8[c] = norm_w ? __ldg(norm_w + sub * 8 + c) : 1.0f;
+    // the loop runs over row pairs so that every lane of a warp takes the same
+    // number of iterations (the shuffles below use the full mask)
+    for (int64_t pair = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); 2 * pair < rows;
+         pair += warps_total) {
+        const int64_t row = 2 * pair + (lane >> 4);
+        const bool valid = row < rows;
+        const size_t base = (size_t)row * D + sub * 8;
+        float ov[8], gv[8];
+        if (valid) {
+            load8<O_BF16>(o, base, ov);
+            load8<G_BF16>(g, base, gv);
         } else {
-            const float4 of = *reinterpret_cast<const float4*>(reinterpret_cast<const float*>(o) + base);
-            ov[0] = of.x; ov[1] = of.y; ov[2] = of.z; ov[3] = of.w;
-        }
-        if constexpr (G_BF16) {
-            const uint2 gb = __ldg(reinterpret_cast<const uint2*>(reinterpret_cast<const uint16_t*>(g) + base));
-            gv[0] = __uint_as_float(gb.x << 16); gv[1] = __uint_as_float(gb.x & 0xFFFF0000u);
-            gv[2] = __uint_as_float(gb.y << 16); gv[3] = __uint_as_float(gb.y & 0xFFFF0000u);
-        } else {
-            const float4 gf = __ldg(reinterpret_cast<const float4*>(reinterpret_cast<const float*>(g) + base));
-            gv[0] = gf.x; gv[1] = gf.y; gv[2] = gf.z; gv[3] = gf.w;
-        }
-        float ss = ov[0] * ov[0] + ov[1] * ov[1] + ov[2] * ov[2] + ov[3] * ov[3];
 #pragma unroll
-        for (int m = 16; m >= 1; m >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, m);
+            for (int c = 0; c < 8; ++c) ov[c] = gv[c] = 0.f;
+        }
+        float ss = 0.f;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) ss += ov[c] * ov[c];
+#pragma unroll
+        for (int m = 8; m >= 1; m >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, m);
         const float inv = rsqrtf(ss * (1.0f / D) + eps);
-        float yv[4];
+        float yv[8];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) yv[c] = ov[c] * inv * w4[c] / (1.0f + __expf(-gv[c]));
+        for (int c = 0; c < 8; ++c) yv[c] = ov[c] * inv * w8[c] * __fdividef(1.0f, 1.0f + __expf(-gv[c]));
+        if (!valid) continue;
         if constexpr (OUT_BF16) {
-            uint2 yb;
-            yb.x = pack_bf16x2(yv[0], yv[1]);
-            yb.y = pack_bf16x2(yv[2], yv[3]);
-            *reinterpret_cast<uint2*>(reinterpret_cast<uint16_t*>(y) + base) = yb;
+            *reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(y) + base) =
+                make_uint4(pack_bf16x2(yv[0], yv[1]), pack_bf16x2(yv[2], yv[3]), pack_bf16x2(yv[4], yv[5]),
+                           pack_bf16x2(yv[6], yv[7]));
         } else {
-            *reinterpret_cast<float4*>(reinterpret_cast<float*>(y) + base) = make_float4(yv[0], yv[1], yv[2], yv[3]);
+            float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(y) + base);
+            dst[0] = make_float4(yv[0], yv[1], yv[2], yv[3]);
+            dst[1] = make_float4(yv[4], yv[5], yv[6], yv[7]);
         }
     }
 }
@@ -190,7 +207,7 @@ cudaError_t launch_decode_step(float* state, const void* q, const void* k, const
 cudaError_t launch_gate_norm(const void* o, const void* g, const float* norm_w, float eps, void* y,
                              int64_t rows, bool o_bf16, bool g_bf16, bool out_bf16, int num_sms,
                              cudaStream_t stream) {
-    const int64_t blocks_needed = (rows + 7) / 8;
+    const int64_t blocks_needed = (rows + 15) / 16;  // 16 rows per 256-thread block
     const int64_t cap = (int64_t)num_sms * 8;
     const dim3 grid((unsigned)(blocks_needed < cap ? blocks_needed : cap)), block(256);
     if (rows == 0) return cudaSuccess;

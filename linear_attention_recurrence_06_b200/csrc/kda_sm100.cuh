@@ -48,6 +48,11 @@ KDA_DEV void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
                  : "memory");
 }
 
+// Plain arrival (count 1) on a local mbarrier, release semantics at CTA scope.
+KDA_DEV void mbar_arrive(uint64_t* bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
 // Tests the phase with the given parity; while it is incomplete the thread
 // may be suspended in hardware for up to `suspend_ns` (so waiting warps do not
 // consume issue slots) before the test returns false.
@@ -114,6 +119,49 @@ KDA_DEV void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 
 // core operand reads, bulk copies).  Call before the barrier that precedes
 // the MMA issue.
 KDA_DEV void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
+// --------------------------------------------------------------- clusters --
+KDA_DEV uint32_t cluster_ctarank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+// Address of the same shared-memory location in CTA `rank` of this cluster.
+KDA_DEV uint32_t map_to_cta(uint32_t local_smem_addr, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local_smem_addr), "r"(rank));
+    return r;
+}
+// Asynchronous 4-byte store into (possibly another CTA's) shared memory; its
+// arrival performs complete_tx(4) on the mbarrier at `cluster_bar_addr` in the
+// destination CTA, so the receiver learns of it without any fence here.
+KDA_DEV void st_async_f32(uint32_t cluster_addr, float v, uint32_t cluster_bar_addr) {
+    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.f32 [%0], %1, [%2];" ::"r"(cluster_addr),
+                 "f"(v), "r"(cluster_bar_addr)
+                 : "memory");
+}
+// Waits with acquire at cluster scope (bounded like mbar_wait).
+KDA_DEV bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, uint32_t* status) {
+    const unsigned long long t0 = globaltimer_ns();
+    while (true) {
+        uint32_t ok;
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}"
+            : "=r"(ok)
+            : "r"(smem_u32(bar)), "r"(parity), "r"(1000000u)
+            : "memory");
+        if (ok) return true;
+        if (globaltimer_ns() - t0 > WAIT_LIMIT_NS) {
+            if (status) atomicOr(status, DEV_ERR_TIMEOUT);
+            return false;
+        }
+    }
+}
+KDA_DEV void cluster_sync_all() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
 
 // ---------------------------------------------------------------- tcgen05 --
 // TMEM allocation: one warp allocates `ncols` columns (power of 2, >= 32) and

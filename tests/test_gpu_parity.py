@@ -182,10 +182,10 @@ def test_decode_steps(bf16, gate):
 
 
 @pytest.mark.parametrize("bf16", [True, False])
-def test_gate_norm(bf16):
+@pytest.mark.parametrize("rows", [1000, 999, 1, 4097])
+def test_gate_norm(bf16, rows):
     torch = _torch()
     import linear_attention_recurrence_06_b200 as kda
-    rows = 1000
     dt = torch.bfloat16 if bf16 else torch.float32
     o = synth.normal(1, 100, (rows, D), 1.0, bf16)
     g = synth.normal(1, 101, (rows, D), 1.0, bf16)
