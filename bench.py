@@ -426,6 +426,28 @@ def run_reference(args):
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
+def run_ncu_case(args):
+    """Small prefill case for profiler captures: `warmup + steps` calls of
+    kda_chunk_fwd (fused gate) on T = --ncu-tokens tokens, H = 32, no timing."""
+    import torch
+    import linear_attention_recurrence_06_b200 as kda
+    from linear_attention_recurrence_06_b200 import synth
+    T, H = args.ncu_tokens, PREFILL["H"]
+    tb = synth.tokens(0, 0, T, H, D, D, bf16=True, gate=True)
+    up = {n: torch.from_numpy(np.ascontiguousarray(getattr(tb, n))).to(torch.bfloat16).cuda()
+          for n in ("q", "k", "v", "log_alpha", "beta", "g")}
+    x = {n: t.view(1, T, H, -1) if n != "beta" else t.view(1, T, H) for n, t in up.items()}
+    out = torch.empty((1, T, H, D), dtype=torch.bfloat16, device="cuda")
+    fs = torch.empty((1, H, D, D), dtype=torch.float32, device="cuda")
+    _, full = kda.workspace_size(T, H, 1, T)
+    ws = torch.empty(full, dtype=torch.uint8, device="cuda")
+    for _ in range(args.warmup + args.steps):
+        kda.chunk_fwd(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], None, gate=x["g"], out=out,
+                      final_state=fs, workspace=ws)
+    torch.cuda.synchronize()
+    return {"ncu_case": f"prefill T={T} H={H}", "calls": args.warmup + args.steps, "status": kda.query_status(ws)}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -435,11 +457,16 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--ref-tokens", type=int, default=256)
+    ap.add_argument("--ncu-tokens", type=int, default=0,
+                    help="profiler case: only run warmup+steps prefill calls on this many tokens")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     peaks = load_peaks()
-    line = run_reference(args) if args.impl == "reference" else run_ours(args, peaks)
+    if args.ncu_tokens > 0:
+        line = run_ncu_case(args)
+    else:
+        line = run_reference(args) if args.impl == "reference" else run_ours(args, peaks)
     if line is not None:
         print(json.dumps(line), flush=True)
 

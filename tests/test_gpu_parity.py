@@ -112,6 +112,43 @@ def test_prefill_fused_gate_norm(out_f32):
     check(o, fs, ro, rfs)
 
 
+@pytest.mark.parametrize("bf16", [True, False])
+def test_prefill_gate_varlen_weights_multi_pass(bf16):
+    """Gate + RMSNorm with per-channel weights on packed sequences (an empty and
+    ragged ones included), once with the full workspace and once with one small
+    enough to force one pass per chunk.  bf16 inputs take the normalisation
+    fused into the chain (row sums exchanged inside a cluster); fp32 inputs
+    take the separate row kernel."""
+    torch = _torch()
+    import linear_attention_recurrence_06_b200 as kda
+    lens = [1, 64, 0, 200, 17, 129]
+    H = 3
+    inp = make_prefill(21, lens, H, bf16=bf16, gate=True, init=True)
+    T = inp["T"]
+    dt = torch.bfloat16 if bf16 else torch.float32
+    q, k, v, la, g = (dev(inp[x], dt).view(1, T, H, D) for x in ("q", "k", "v", "log_alpha", "g"))
+    b = dev(inp["beta"], dt).view(1, T, H)
+    s0 = dev(inp["s0"], torch.float32)
+    w = np.random.default_rng(21).uniform(0.5, 1.5, D).astype(np.float32)
+    cu = torch.from_numpy(inp["cu"].astype(np.int32)).cuda()
+    ro, rfs = oracle.kda_recurrent(inp["q"], inp["k"], inp["v"], inp["log_alpha"], inp["beta"], inp["s0"], inp["cu"])
+    ry = oracle.gate_norm(ro, inp["g"], w, 1e-6)
+    for multi in (False, True):
+        kw = {}
+        if multi:
+            lo, _ = kda.workspace_size(T, H, len(lens), max(lens))
+            kw["workspace"] = torch.empty(lo, dtype=torch.uint8, device="cuda")
+        y, fs = kda.chunk_fwd(q, k, v, la, b, s0, cu_seqlens=cu, max_seqlen=max(lens), gate=g,
+                              norm_weight=dev(w, torch.float32), out_dtype=torch.float32, **kw)
+        torch.cuda.synchronize()
+        yh = host(y).reshape(T, H, D)
+        check(yh, host(fs), ry, rfs)
+        for n in range(len(lens)):
+            sl = slice(inp["cu"][n], inp["cu"][n + 1])
+            if lens[n]:
+                assert rel_l2(yh[sl], ry[sl]) <= REL_L2_TOL
+
+
 def test_prefill_multi_pass_workspace():
     """A workspace that holds one chunk per sequence forces one pass per chunk:
     the state carried between passes must give the same result."""
