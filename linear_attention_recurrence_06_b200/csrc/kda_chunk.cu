@@ -162,36 +162,48 @@ KDA_DEV uint4 pack8(const float* x) {
 // Shared memory (offsets from a 1024-aligned base):
 //   RAW [0, 64K)     TMA tiles [64 tokens][128 ch] bf16: la @0, k @16K, q @32K, v @48K
 //   X   [64K, 136K)  phase 1 (MN-major, no swizzle, M/N = token): KQr 128x128 @0,
-//                             Kd 64x128 @32K, Kb1 16x128 @48K, Kb2 32x128 @52K, Kb3 48x128 @60K
-//                    phase 2: KGt [128][64] @0, Vt [128][64] @16K, Ti [64][64] @32K,
-//                             Ktt [128][64] @40K, Ph [64][64] @56K, inverse temp @64K
-//   Y   [136K, ...)  A fp32 [64][68] @0, X fp32 [64][68] @17408;
+//                             KC = [Kd 64 | Kb1 16 | Kb2 32 | Kb3 48] x 128 @32K
+//                    after round 1: Ti [64][64] @32K, Ph [64][64] @56K, inverse scratch @64K
+//   Y   [136K, 171K) A fp32 [64][68] @0, X fp32 [64][68] @17408;
 //                    later Wt [128][64] @0, Ut [128][64] @16K
+//   Z2  [171K, 219K) KGt, Vt, Ktt [128][64] (built while round 1 runs)
 //   misc             beta[64], G[5][128], tile totals[4][128], 2 mbarriers, TMEM base
+// The workspace slot leaves at the end of an item as two bulk copies: [Mlr | Qp | GamC]
+// assembled at X, [Bm | ObT] at Z2.
 // TMEM (512 columns): round 1  A/P diag [0,64), off-diag [64,80) [80,112) [112,160)
 //                     round 2  Wt [160,224), Ut [224,288)
-//                     round 3  Mlr [288,416), (PW)^T [416,480), Bm [0,128), Ob^T [128,192)
+//                     round 3  [Mlr | Bm] [0,256) (one N = 256 product), (PW)^T [256,320), Ob^T [320,384)
 constexpr int INTRA_THREADS = 512;
 constexpr uint32_t R_LA = 0, R_K = 16384, R_Q = 32768, R_V = 49152;
 constexpr uint32_t IX = 65536;
-constexpr uint32_t IX_KQR = IX + 0, IX_KD = IX + 32768, IX_KB1 = IX + 49152, IX_KB2 = IX + 53248,
-                   IX_KB3 = IX + 61440;
-constexpr uint32_t IX_KGT = IX + 0, IX_VT = IX + 16384, IX_TI = IX + 32768, IX_KTT = IX + 40960,
-                   IX_PH = IX + 57344, IX_TMP = IX + 65536;
+// KC stacks the column operands of round 1 as N = 160 token rows of one MN-major image:
+// rows [0,64) Kd, [64,80) Kb1, [80,112) Kb2, [112,160) Kb3 (K-group stride 160 * 16 B).
+constexpr uint32_t IX_KQR = IX + 0, IX_KC = IX + 32768;
+constexpr uint32_t KC_KG = 2560, KC_B1 = 64, KC_B2 = 80, KC_B3 = 112;
+constexpr uint32_t IX_TI = IX + 32768, IX_PH = IX + 57344, IX_TMP = IX + 65536;
 constexpr uint32_t IY = IX + 73728;
 constexpr int LDA = 68;  // padded fp32 row stride of A and X (16-byte rows, spread banks)
 constexpr uint32_t IY_A = IY, IY_X = IY + 64 * LDA * 4, IY_WT = IY, IY_UT = IY + 16384;
-constexpr uint32_t IM = IY + 35840;
+// Z2: the phase-2 operand images (built while round 1 runs), K-major SW128 [128 ch][64 tok]
+constexpr uint32_t Z2 = IY + 35840;
+constexpr uint32_t Z2_KGT = Z2, Z2_VT = Z2 + 16384, Z2_KTT = Z2 + 32768;
+constexpr uint32_t IM = Z2 + 49152;
 constexpr uint32_t IM_BETA = IM, IM_G = IM + 256, IM_TOT = IM + 256 + 2560, IM_BAR_RAW = IM_TOT + 2048,
-                   IM_BAR_MMA = IM_BAR_RAW + 8, IM_NEXT = IM_BAR_MMA + 8, IM_TMEM = IM_NEXT + 32;
+                   IM_BAR_MMA = IM_BAR_RAW + 8, IM_BAR_MMA2 = IM_BAR_MMA + 8, IM_NEXT = IM_BAR_MMA2 + 8,
+                   IM_TMEM = IM_NEXT + 32;
 constexpr uint32_t INTRA_SMEM = IM_TMEM + 16 + 1024;  // + alignment slack
 constexpr uint32_t INTRA_TMEM_COLS = 512;
-constexpr uint32_t TM_AD = 0, TM_B1 = 64, TM_B2 = 80, TM_B3 = 112, TM_WT = 160, TM_UT = 224, TM_M = 288,
-                   TM_PW = 416, TM_BM = 0, TM_OB = 128;
+constexpr uint32_t TM_AD = 0, TM_B1 = 64, TM_B2 = 80, TM_B3 = 112, TM_WT = 160, TM_UT = 224, TM_M = 0,
+                   TM_BM = 128, TM_PW = 256, TM_OB = 320;
 
 struct IntraMaps {
     CUtensorMap la, k, q, v;
 };
+
+// Raw bf16 bits of (token t, channel c) of a TMA tile, 0 past the chunk's end.
+KDA_DEV uint32_t raw_bits(const uint8_t* sm, uint32_t tile, int t, int c, int L) {
+    return (t < L) ? (uint32_t)*reinterpret_cast<const uint16_t*>(sm + tile + (uint32_t)(t * 128 + c) * 2u) : 0u;
+}
 
 template <bool IN_BF16>
 KDA_DEV float raw_in(const uint8_t* sm, uint32_t tile, const void* gsrc, size_t ebase, size_t rowstride, int t,
@@ -221,6 +233,7 @@ intra_kernel(const ChunkArgs a, const __grid_constant__ IntraMaps maps, const in
     float* s_tot = reinterpret_cast<float*>(sm + IM_TOT);  // [4][128]
     uint64_t* bar_raw = reinterpret_cast<uint64_t*>(sm + IM_BAR_RAW);
     uint64_t* bar_mma = reinterpret_cast<uint64_t*>(sm + IM_BAR_MMA);
+    uint64_t* bar_mma2 = reinterpret_cast<uint64_t*>(sm + IM_BAR_MMA2);  // second half of round 3
     uint32_t* s_tmem = reinterpret_cast<uint32_t*>(sm + IM_TMEM);
     // next item of this CTA: {item, t0} as int64 and {h, L} as int
     int64_t* s_next64 = reinterpret_cast<int64_t*>(sm + IM_NEXT);
@@ -233,13 +246,20 @@ intra_kernel(const ChunkArgs a, const __grid_constant__ IntraMaps maps, const in
     if (tid == 0) {
         mbar_init(bar_raw, 1);
         mbar_init(bar_mma, 1);
+        mbar_init(bar_mma2, 1);
         fence_mbar_init();
+        if constexpr (IN_BF16) {
+            prefetch_tmap(&maps.la);
+            prefetch_tmap(&maps.k);
+            prefetch_tmap(&maps.q);
+            prefetch_tmap(&maps.v);
+        }
     }
     __syncthreads();
     tc_fence_after();
     const uint32_t tm = *s_tmem;
     const uint32_t lane_addr = tm + ((uint32_t)(32 * qd) << 16);
-    uint32_t ph_raw = 0, ph_mma = 0;
+    uint32_t ph_raw = 0, ph_mma = 0, ph_mma2 = 0;
 
     // next valid item at or after `from` (stride gridDim.x), or n_items
     auto next_valid = [&](int64_t from) -> int64_t {
@@ -261,12 +281,22 @@ intra_kernel(const ChunkArgs a, const __grid_constant__ IntraMaps maps, const in
     int64_t item = next_valid(blockIdx.x);
     bool raw_in_flight = false;
     // beta of the next item, loaded one item ahead by threads < 64
-    float beta_next = 0.f;
+    // raw bits of the next item's beta (bf16 in the low half, or fp32), converted when
+    // used so that no instruction waits for the load before then
+    uint32_t beta_bits = 0;
+    auto load_beta = [&](int64_t tt, int hh, int LL) {
+        beta_bits = 0;
+        if (tid < LL) {
+            const size_t idx = (size_t)(tt + tid) * H + hh;
+            if constexpr (IN_BF16) beta_bits = __ldg(reinterpret_cast<const unsigned short*>(a.beta) + idx);
+            else beta_bits = __float_as_uint(__ldg(reinterpret_cast<const float*>(a.beta) + idx));
+        }
+    };
     if (item < n_items) {
         int hh, LL;
         int64_t tt;
         item_info(a, item, hh, tt, LL);
-        if (tid < CH) beta_next = (tid < LL) ? ld_in<IN_BF16>(a.beta, (size_t)(tt + tid) * H + hh) : 0.f;
+        if (tid < CH) load_beta(tt, hh, LL);
         if constexpr (IN_BF16) {
             if (tid == 0) issue_raw(hh, tt);
             raw_in_flight = true;
@@ -282,7 +312,17 @@ intra_kernel(const ChunkArgs a, const __grid_constant__ IntraMaps maps, const in
         const size_t ebase = ((size_t)t0 * H + h) * DK + c;
         const size_t vbase = ((size_t)t0 * H + h) * DV + c;
 
-        if (tid < CH) s_beta[tid] = beta_next;
+        if (tid < CH) s_beta[tid] = IN_BF16 ? __uint_as_float(beta_bits << 16) : __uint_as_float(beta_bits);
+        if (tid == INTRA_THREADS - 1) {  // the next item of this CTA (read after the round-1 issue)
+            const int64_t nx = next_valid(item + gridDim.x);
+            int hh = 0, LL = 0;
+            int64_t tt = 0;
+            if (nx < n_items) item_info(a, nx, hh, tt, LL);
+            s_next64[0] = nx;
+            s_next64[1] = tt;
+            s_next32[0] = hh;
+            s_next32[1] = LL;
+        }
         if constexpr (IN_BF16) {
             mbar_wait(bar_raw, ph_raw, a.status);
             ph_raw ^= 1;
@@ -291,37 +331,38 @@ intra_kernel(const ChunkArgs a, const __grid_constant__ IntraMaps maps, const in
 
         // ---- a1: cumulative clamped log-decay g of this thread's tile (registers)
         float E1[16], E3[16];
-        float gamC = 0.f;  // e^{g at chunk end} of channel c (staged by one thread group)
         uint32_t qr2[8];  // raw q of this thread's 16 tokens, bf16 pairs (kept for the Qp epilogue)
+        uint32_t kr2[8];  // raw k (bf16 inputs), kept from phase 1 for phase 2
         float G[5];
         {
-            float gl[16];
+            float alpha[16];
             float run = 0.f;
 #pragma unroll
             for (int u = 0; u < 16; ++u) {
                 const int t = 16 * q4 + u;
                 const float l = raw_in<IN_BF16>(sm, R_LA, a.log_alpha, ebase, rowstride, t, c, L);
-                run += (t < L) ? fmaxf(l, LOG_ALPHA_FLOOR) : 0.f;
-                gl[u] = run;
+                const float lc = (t < L) ? fmaxf(l, LOG_ALPHA_FLOOR) : 0.f;
+                run += lc;
+                alpha[u] = __expf(lc);  // per-step decay (1 past the end)
             }
             s_tot[q4 * 128 + c] = run;
+            // E1 = e^{g_t - G_q4} = prod_{r<=t} alpha_r (<= 1),  E3 = e^{G_{q4+1} - g_t} = prod_{r>t} alpha_r
+            // (products of at most 16 factors >= e^-5: no underflow in fp32)
+            E1[0] = alpha[0];
+#pragma unroll
+            for (int u = 1; u < 16; ++u) E1[u] = E1[u - 1] * alpha[u];
+            E3[15] = 1.f;
+#pragma unroll
+            for (int u = 14; u >= 0; --u) E3[u] = E3[u + 1] * alpha[u + 1];
             __syncthreads();
             float off = 0.f;
 #pragma unroll
             for (int qq = 0; qq < 3; ++qq)
                 if (qq < q4) off += s_tot[qq * 128 + c];
-#pragma unroll
-            for (int u = 0; u < 16; ++u) gl[u] += off;
             // G_0 = 0, G_{b+1} = g at the last token of tile b
-            s_G[(q4 + 1) * 128 + c] = gl[15];
+            s_G[(q4 + 1) * 128 + c] = off + run;
             if (q4 == 0) s_G[c] = 0.f;
-            // E1 = e^{g_t - G_q4} (<= 1),  E3 = e^{G_{q4+1} - g_t} (<= 1)
-#pragma unroll
-            for (int u = 0; u < 16; ++u) {
-                E1[u] = __expf(gl[u] - off);
-                E3[u] = __expf(gl[15] - gl[u]);
-            }
-            if (tid == 0) bulk_wait_read_all();  // previous item's slot copy has left X/Y
+            if (tid == 0) bulk_wait_read_all();  // previous item's slot copies have left X and Z2
             __syncthreads();
 #pragma unroll
             for (int b = 0; b < 5; ++b) G[b] = s_G[b * 128 + c];
@@ -343,10 +384,24 @@ intra_kernel(const ChunkArgs a, const __grid_constant__ IntraMaps maps, const in
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
                     const int u = 8 * m + e, t = tf + e;
-                    const float kv = raw_in<IN_BF16>(sm, R_K, a.k, ebase, rowstride, t, c, L);
-                    const float qv = raw_in<IN_BF16>(sm, R_Q, a.q, ebase, rowstride, t, c, L);
-                    if (e & 1) qr2[u >> 1] |= (uint32_t)f32_to_bf16(qv) << 16;
-                    else qr2[u >> 1] = (uint32_t)f32_to_bf16(qv);
+                    float kv, qv;
+                    if constexpr (IN_BF16) {  // keep the raw bits (exact) for later phases
+                        const uint32_t kb = raw_bits(sm, R_K, t, c, L), qb = raw_bits(sm, R_Q, t, c, L);
+                        kv = __uint_as_float(kb << 16);
+                        qv = __uint_as_float(qb << 16);
+                        if (e & 1) {
+                            kr2[u >> 1] |= kb << 16;
+                            qr2[u >> 1] |= qb << 16;
+                        } else {
+                            kr2[u >> 1] = kb;
+                            qr2[u >> 1] = qb;
+                        }
+                    } else {
+                        kv = raw_in<IN_BF16>(sm, R_K, a.k, ebase, rowstride, t, c, L);
+                        qv = raw_in<IN_BF16>(sm, R_Q, a.q, ebase, rowstride, t, c, L);
+                        if (e & 1) qr2[u >> 1] |= (uint32_t)f32_to_bf16(qv) << 16;
+                        else qr2[u >> 1] = (uint32_t)f32_to_bf16(qv);
+                    }
                     kr[e] = kv * E1[u];
                     qe[e] = qv * E1[u] * a.scale;
                     k3[e] = kv * E3[u];
@@ -354,23 +409,23 @@ intra_kernel(const ChunkArgs a, const __grid_constant__ IntraMaps maps, const in
                 }
                 *reinterpret_cast<uint4*>(sm + IX_KQR + mn_off(tf, c, 2048)) = pack8(kr);
                 *reinterpret_cast<uint4*>(sm + IX_KQR + mn_off(tf + 64, c, 2048)) = pack8(qe);
-                *reinterpret_cast<uint4*>(sm + IX_KD + mn_off(tf, c, 1024)) = pack8(kd);
+                *reinterpret_cast<uint4*>(sm + IX_KC + mn_off(tf, c, KC_KG)) = pack8(kd);
                 float f[8];
                 if (q4 == 0) {
-                    *reinterpret_cast<uint4*>(sm + IX_KB1 + mn_off(tf, c, 256)) = pack8(k3);
+                    *reinterpret_cast<uint4*>(sm + IX_KC + mn_off(KC_B1 + tf, c, KC_KG)) = pack8(k3);
 #pragma unroll
                     for (int e = 0; e < 8; ++e) f[e] = k3[e] * f2;
-                    *reinterpret_cast<uint4*>(sm + IX_KB2 + mn_off(tf, c, 512)) = pack8(f);
+                    *reinterpret_cast<uint4*>(sm + IX_KC + mn_off(KC_B2 + tf, c, KC_KG)) = pack8(f);
 #pragma unroll
                     for (int e = 0; e < 8; ++e) f[e] = k3[e] * f3;
-                    *reinterpret_cast<uint4*>(sm + IX_KB3 + mn_off(tf, c, 768)) = pack8(f);
+                    *reinterpret_cast<uint4*>(sm + IX_KC + mn_off(KC_B3 + tf, c, KC_KG)) = pack8(f);
                 } else if (q4 == 1) {
-                    *reinterpret_cast<uint4*>(sm + IX_KB2 + mn_off(tf, c, 512)) = pack8(k3);
+                    *reinterpret_cast<uint4*>(sm + IX_KC + mn_off(KC_B2 + tf, c, KC_KG)) = pack8(k3);
 #pragma unroll
                     for (int e = 0; e < 8; ++e) f[e] = k3[e] * f3;
-                    *reinterpret_cast<uint4*>(sm + IX_KB3 + mn_off(tf, c, 768)) = pack8(f);
+                    *reinterpret_cast<uint4*>(sm + IX_KC + mn_off(KC_B3 + tf, c, KC_KG)) = pack8(f);
                 } else if (q4 == 2) {
-                    *reinterpret_cast<uint4*>(sm + IX_KB3 + mn_off(tf, c, 768)) = pack8(k3);
+                    *reinterpret_cast<uint4*>(sm + IX_KC + mn_off(KC_B3 + tf, c, KC_KG)) = pack8(k3);
                 }
             }
         }
@@ -381,11 +436,49 @@ intra_kernel(const ChunkArgs a, const __grid_constant__ IntraMaps maps, const in
 
         // ---- round 1: [Kr;Qr] Kd^T and [Kr;Qr] Kb(b)^T
         if (tid == 0) {
-            mma_mn<8, 2048, 1024>(tm + TM_AD, sb + IX_KQR, sb + IX_KD, idesc_bf16_major(128, 64, 1, 1));
-            mma_mn<8, 2048, 256>(tm + TM_B1, sb + IX_KQR, sb + IX_KB1, idesc_bf16_major(128, 16, 1, 1));
-            mma_mn<8, 2048, 512>(tm + TM_B2, sb + IX_KQR, sb + IX_KB2, idesc_bf16_major(128, 32, 1, 1));
-            mma_mn<8, 2048, 768>(tm + TM_B3, sb + IX_KQR, sb + IX_KB3, idesc_bf16_major(128, 48, 1, 1));
+            // one N = 160 product: [A/P diag | tile-1 | tile-2 | tile-3 off-diagonal] columns
+            mma_mn<8, 2048, KC_KG>(tm + TM_AD, sb + IX_KQR, sb + IX_KC, idesc_bf16_major(128, 160, 1, 1));
             mma_commit(bar_mma);
+        }
+
+        // ---- phase 2 operands while round 1 runs (K = token, own region Z2):
+        //      KGt = (K o Gam)^T, Vt = V^T, Ktt = Kt^T
+        {
+            const float eG = __expf(Gs);          // Gam_t = E1 e^{G_q4}
+            const float eC = __expf(G[4] - Gn);   // e^{g_C - g_t} = E3 e^{G_4 - G_{q4+1}}
+#pragma unroll
+            for (int m = 0; m < 2; ++m) {  // 8 consecutive tokens per 16-byte chunk
+                float kg[8], vv[8], kt[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const int u = 8 * m + e;
+                    const int t = 16 * q4 + u;
+                    float kv;
+                    if constexpr (IN_BF16)
+                        kv = __uint_as_float((u & 1) ? (kr2[u >> 1] & 0xFFFF0000u) : (kr2[u >> 1] << 16));
+                    else
+                        kv = raw_in<IN_BF16>(sm, R_K, a.k, ebase, rowstride, t, c, L);
+                    vv[e] = raw_in<IN_BF16>(sm, R_V, a.v, vbase, (size_t)H * DV, t, c, L);
+                    kg[e] = kv * E1[u] * eG;
+                    kt[e] = kv * E3[u] * eC;
+                }
+                const uint32_t off = sw128_off((uint32_t)c, (uint32_t)(16 * q4 + 8 * m));
+                *reinterpret_cast<uint4*>(sm + Z2_KGT + off) = pack8(kg);
+                *reinterpret_cast<uint4*>(sm + Z2_VT + off) = pack8(vv);
+                *reinterpret_cast<uint4*>(sm + Z2_KTT + off) = pack8(kt);
+            }
+        }
+        __syncthreads();  // every read of RAW for this item is done
+        // next item's raw tiles and beta
+        const int64_t next = s_next64[0];
+        if (next < n_items) {
+            const int64_t tt = s_next64[1];
+            const int hh = s_next32[0], LL = s_next32[1];
+            if constexpr (IN_BF16) {
+                if (tid == 0) issue_raw(hh, tt);
+                raw_in_flight = true;
+            }
+            if (tid < CH) load_beta(tt, hh, LL);
         }
         mbar_wait(bar_mma, ph_mma, a.status);
         ph_mma ^= 1;
@@ -430,41 +523,28 @@ intra_kernel(const ChunkArgs a, const __grid_constant__ IntraMaps maps, const in
                 if (isP) {
                     *reinterpret_cast<uint4*>(sm + IX_PH + sw128_off(t, 16 * p)) = pack8(d);
                     *reinterpret_cast<uint4*>(sm + IX_PH + sw128_off(t, 16 * p + 8)) = pack8(d + 8);
-                } else {
+                } else {  // N = Diag(beta) A for the inverse
+                    const float bt_ = s_beta[t];
                     float4* dst = reinterpret_cast<float4*>(sA + t * LDA + 16 * p);
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) dst[i] = make_float4(d[4 * i], d[4 * i + 1], d[4 * i + 2], d[4 * i + 3]);
+                    for (int i = 0; i < 4; ++i)
+                        dst[i] = make_float4(bt_ * d[4 * i], bt_ * d[4 * i + 1], bt_ * d[4 * i + 2], bt_ * d[4 * i + 3]);
                 }
             }
         }
         __syncthreads();
 
-        // ---- a3: T = (I + Diag(beta) A)^-1 Diag(beta), fp32, blocked on 16x16 tiles
+        // ---- a3: T = (I + N)^-1 Diag(beta) with N = Diag(beta) A (scaled when A was
+        //      extracted), fp32, blocked on 16x16 tiles: X = (I + N)^-1 is built in sX from
+        //      (1) the four 16x16 diagonal blocks by forward substitution, (2) the
+        //      sub-diagonal blocks of the two 32x32 diagonal halves, X_{b+1,b} =
+        //      -X_{b+1,b+1} N_{b+1,b} X_bb (b = 0, 2), (3) the lower-left 32x32 block
+        //      X_LL = -H_1 N_LL H_0 (H_0, H_1 the halves).  Blocks above the diagonal are
+        //      never read: the sums skip them and the T image writes zeros there.
         {
-            float* sA = reinterpret_cast<float*>(sm + IY_A);  // becomes N = Diag(beta) A in place
-            float* sX = reinterpret_cast<float*>(sm + IY_X);  // X = (I + N)^-1
-            float* sY = reinterpret_cast<float*>(sm + IX_TMP);
-            for (int e = tid; e < 64 * 16; e += INTRA_THREADS) {  // 4 entries per step
-                const int i = e >> 4, j4 = (e & 15) * 4;
-                float4* pa = reinterpret_cast<float4*>(sA + i * LDA + j4);
-                const float b = s_beta[i];
-                float4 v4 = *pa;
-                v4.x *= b; v4.y *= b; v4.z *= b; v4.w *= b;
-                *pa = v4;
-                // zero the strictly upper blocks of X
-                if ((j4 >> 4) > (i >> 4)) *reinterpret_cast<float4*>(sX + i * LDA + j4) = make_float4(0.f, 0.f, 0.f, 0.f);
-            }
-            __syncthreads();
-            if (tid == INTRA_THREADS - 1) {  // idle in the inverse: find the next item of this CTA
-                const int64_t nx = next_valid(item + gridDim.x);
-                int hh = 0, LL = 0;
-                int64_t tt = 0;
-                if (nx < n_items) item_info(a, nx, hh, tt, LL);
-                s_next64[0] = nx;
-                s_next64[1] = tt;
-                s_next32[0] = hh;
-                s_next32[1] = LL;
-            }
+            const float* sA = reinterpret_cast<const float*>(sm + IY_A);
+            float* sX = reinterpret_cast<float*>(sm + IY_X);
+            float* sY = reinterpret_cast<float*>(sm + IX_TMP);  // partial products (8 KB)
             if (tid < 64) {  // diagonal blocks: one thread per (block, column)
                 // column j of (I + N_bb)^-1: x_i = -sum_{m<i} N_im x_m, x_j = 1, x_i = 0 for i < j
                 // (entries above j are zero, so the sums need no masking)
@@ -491,92 +571,101 @@ intra_kernel(const ChunkArgs a, const __grid_constant__ IntraMaps maps, const in
                 for (int i = 0; i < 16; ++i) sX[(16 * b + i) * LDA + 16 * b + j] = x[i];
             }
             __syncthreads();
-            // off-diagonal blocks by distance d:  X_ij = -X_ii * sum_{m=j}^{i-1} N_im X_mj.
-            // One task = 1 row x 4 columns of one block pair (4 independent accumulators).
-            for (int d = 1; d <= 3; ++d) {
-                const int ntask = (4 - d) * 64;
-                if (tid < ntask) {
-                    const int pb = tid >> 6, r = (tid >> 2) & 15, cc = (tid & 3) * 4;
-                    const int bj = pb, bi = pb + d;
-                    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+            // Products below use 2x4 register tiles: acc[i][j] += sum_{m < 16} R[i][m] C[m][j]
+            // (16-byte loads of 4 row entries and of 4 column entries feed 8 FMAs each);
+            // a long sum is split over warp groups into partials that the next step adds.
+            auto tile24 = [](const float* R, int ldr, const float* C, int ldc, float (&acc)[2][4]) {
+#pragma unroll 2
+                for (int m = 0; m < 16; m += 4) {
+                    float rv[2][4];
 #pragma unroll
-                    for (int mm = 0; mm < 3; ++mm) {
-                        if (mm < d) {
-                            const int m = bj + mm;
-                            const float* na = sA + (16 * bi + r) * LDA + 16 * m;
-                            const float* xb = sX + (16 * m) * LDA + 16 * bj + cc;
+                    for (int i = 0; i < 2; ++i) {
+                        const float4 v = *reinterpret_cast<const float4*>(R + i * ldr + m);
+                        rv[i][0] = v.x; rv[i][1] = v.y; rv[i][2] = v.z; rv[i][3] = v.w;
+                    }
 #pragma unroll
-                            for (int u4 = 0; u4 < 4; ++u4) {
-                                const float4 nv = *reinterpret_cast<const float4*>(na + 4 * u4);
-                                const float nvs[4] = {nv.x, nv.y, nv.z, nv.w};
+                    for (int k = 0; k < 4; ++k) {
+                        const float4 cv = *reinterpret_cast<const float4*>(C + (m + k) * ldc);
 #pragma unroll
-                                for (int k = 0; k < 4; ++k) {
-                                    const float4 xv = *reinterpret_cast<const float4*>(xb + (4 * u4 + k) * LDA);
-                                    acc.x += nvs[k] * xv.x; acc.y += nvs[k] * xv.y;
-                                    acc.z += nvs[k] * xv.z; acc.w += nvs[k] * xv.w;
-                                }
-                            }
+                        for (int i = 0; i < 2; ++i) {
+                            acc[i][0] += rv[i][k] * cv.x; acc[i][1] += rv[i][k] * cv.y;
+                            acc[i][2] += rv[i][k] * cv.z; acc[i][3] += rv[i][k] * cv.w;
                         }
                     }
-                    *reinterpret_cast<float4*>(sY + pb * 256 + r * 16 + cc) = acc;
                 }
-                __syncthreads();
-                if (tid < ntask) {
-                    const int pb = tid >> 6, r = (tid >> 2) & 15, cc = (tid & 3) * 4;
-                    const int bj = pb, bi = pb + d;
-                    const float* xa = sX + (16 * bi + r) * LDA + 16 * bi;
-                    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+            };
+            auto store24 = [](float* D, int ldd, const float (&acc)[2][4], float sg) {
 #pragma unroll
-                    for (int u4 = 0; u4 < 4; ++u4) {
-                        const float4 xv4 = *reinterpret_cast<const float4*>(xa + 4 * u4);
-                        const float xs[4] = {xv4.x, xv4.y, xv4.z, xv4.w};
-#pragma unroll
-                        for (int k = 0; k < 4; ++k) {
-                            const float4 yv = *reinterpret_cast<const float4*>(sY + pb * 256 + (4 * u4 + k) * 16 + cc);
-                            acc.x += xs[k] * yv.x; acc.y += xs[k] * yv.y;
-                            acc.z += xs[k] * yv.z; acc.w += xs[k] * yv.w;
-                        }
-                    }
-                    *reinterpret_cast<float4*>(sX + (16 * bi + r) * LDA + 16 * bj + cc) =
-                        make_float4(-acc.x, -acc.y, -acc.z, -acc.w);
-                }
-                __syncthreads();
+                for (int i = 0; i < 2; ++i)
+                    *reinterpret_cast<float4*>(D + i * ldd) =
+                        make_float4(sg * acc[i][0], sg * acc[i][1], sg * acc[i][2], sg * acc[i][3]);
+            };
+            float* sZ0 = sY;          // [32][16] partial of Z over m in block 0 (columns of block 0)
+            float* sZ1 = sY + 512;    // [32][32] partial of Z over m in block 1
+            float* sP = reinterpret_cast<float*>(sm + IY_A);  // [16][32], in the dead N region
+            // (2a) Y_b = N_{b+1,b} X_bb  (b = 0, 2; 64 tiles, warps 0-1)
+            if (tid < 64) {
+                const int b = 2 * (tid >> 5), k = tid & 31, r0 = 2 * (k >> 2), c0 = 4 * (k & 3);
+                float acc[2][4] = {};
+                tile24(sA + (16 * (b + 1) + r0) * LDA + 16 * b, LDA, sX + (16 * b) * LDA + 16 * b + c0, LDA, acc);
+                store24(sY + 1536 + (b >> 1) * 256 + r0 * 16 + c0, 16, acc, 1.f);
             }
+            __syncthreads();
+            // (2b) X_{b+1,b} = -X_{b+1,b+1} Y_b
+            if (tid < 64) {
+                const int b = 2 * (tid >> 5), k = tid & 31, r0 = 2 * (k >> 2), c0 = 4 * (k & 3);
+                float acc[2][4] = {};
+                tile24(sX + (16 * (b + 1) + r0) * LDA + 16 * (b + 1), LDA, sY + 1536 + (b >> 1) * 256 + c0, 16, acc);
+                store24(sX + (16 * (b + 1) + r0) * LDA + 16 * b + c0, LDA, acc, -1.f);
+            }
+            __syncthreads();
+            // (3a) Z = N_LL H_0 split over m: warps 0-1 m in block 0 (only the columns of block 0:
+            //      H_0 is zero above its diagonal blocks), warps 2-5 m in block 1 (all columns)
+            if (tid < 192) {
+                const int g = tid >= 64;
+                const int k = g ? tid - 64 : tid;
+                const int r0 = g ? 2 * (k >> 3) : 2 * (k >> 2), c0 = g ? 4 * (k & 7) : 4 * (k & 3);
+                float acc[2][4] = {};
+                tile24(sA + (32 + r0) * LDA + 16 * g, LDA, sX + (16 * g) * LDA + c0, LDA, acc);
+                if (g) store24(sZ1 + r0 * 32 + c0, 32, acc, 1.f);
+                else store24(sZ0 + r0 * 16 + c0, 16, acc, 1.f);
+            }
+            __syncthreads();
+            // (3b) X_LL = -H_1 Z split over m: warps 0-3 m in block 2 (every row), warps 4-5 m in
+            //      block 3 (rows of block 3 only), kept as a partial that the T image adds
+            if (tid < 192) {
+                const int g = tid >= 128;
+                const int k = g ? tid - 128 : tid;
+                const int r0 = g ? 16 + 2 * (k >> 3) : 2 * (k >> 3), c0 = 4 * (k & 7);
+                float acc[2][4] = {};
+                const float* Rp = sX + (32 + r0) * LDA + 32 + 16 * g;
+                tile24(Rp, LDA, sZ1 + (16 * g) * 32 + c0, 32, acc);
+                if (c0 < 16) tile24(Rp, LDA, sZ0 + (16 * g) * 16 + c0, 16, acc);
+                if (g) store24(sP + (r0 - 16) * 32 + c0, 32, acc, -1.f);
+                else store24(sX + (32 + r0) * LDA + c0, LDA, acc, -1.f);
+            }
+            __syncthreads();
             {  // T = X Diag(beta) -> bf16 image Ti [t][s], 8 s per store, one row piece per thread
                 const int t = tid >> 3, s0 = (tid & 7) * 8;
-                const float4 x0 = *reinterpret_cast<const float4*>(sX + t * LDA + s0);
-                const float4 x1 = *reinterpret_cast<const float4*>(sX + t * LDA + s0 + 4);
-                const float4 b0 = *reinterpret_cast<const float4*>(s_beta + s0);
-                const float4 b1 = *reinterpret_cast<const float4*>(s_beta + s0 + 4);
-                const float v8[8] = {x0.x * b0.x, x0.y * b0.y, x0.z * b0.z, x0.w * b0.w,
-                                     x1.x * b1.x, x1.y * b1.y, x1.z * b1.z, x1.w * b1.w};
+                float v8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+                if ((s0 >> 4) <= (t >> 4)) {
+                    float4 x0 = *reinterpret_cast<const float4*>(sX + t * LDA + s0);
+                    float4 x1 = *reinterpret_cast<const float4*>(sX + t * LDA + s0 + 4);
+                    if (t >= 48 && s0 < 32) {  // the second half of block 3's lower-left sums
+                        const float4 p0 = *reinterpret_cast<const float4*>(sP + (t - 48) * 32 + s0);
+                        const float4 p1 = *reinterpret_cast<const float4*>(sP + (t - 48) * 32 + s0 + 4);
+                        x0.x += p0.x; x0.y += p0.y; x0.z += p0.z; x0.w += p0.w;
+                        x1.x += p1.x; x1.y += p1.y; x1.z += p1.z; x1.w += p1.w;
+                    }
+                    const float4 b0 = *reinterpret_cast<const float4*>(s_beta + s0);
+                    const float4 b1 = *reinterpret_cast<const float4*>(s_beta + s0 + 4);
+                    v8[0] = x0.x * b0.x; v8[1] = x0.y * b0.y; v8[2] = x0.z * b0.z; v8[3] = x0.w * b0.w;
+                    v8[4] = x1.x * b1.x; v8[5] = x1.y * b1.y; v8[6] = x1.z * b1.z; v8[7] = x1.w * b1.w;
+                }
                 *reinterpret_cast<uint4*>(sm + IX_TI + sw128_off(t, s0)) = pack8(v8);
             }
         }
 
-        // ---- phase 2 operands (K = token): KGt = (K o Gam)^T, Vt = V^T, Ktt = Kt^T
-        {
-            const float eG = __expf(Gs);          // Gam_t = E1 e^{G_q4}
-            const float eC = __expf(G[4] - Gn);   // e^{g_C - g_t} = E3 e^{G_4 - G_{q4+1}}
-#pragma unroll
-            for (int m = 0; m < 2; ++m) {  // 8 consecutive tokens per 16-byte chunk
-                float kg[8], vv[8], kt[8];
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const int u = 8 * m + e;
-                    const int t = 16 * q4 + u;
-                    const float kv = raw_in<IN_BF16>(sm, R_K, a.k, ebase, rowstride, t, c, L);
-                    vv[e] = raw_in<IN_BF16>(sm, R_V, a.v, vbase, (size_t)H * DV, t, c, L);
-                    kg[e] = kv * E1[u] * eG;
-                    kt[e] = kv * E3[u] * eC;
-                }
-                const uint32_t off = sw128_off((uint32_t)c, (uint32_t)(16 * q4 + 8 * m));
-                *reinterpret_cast<uint4*>(sm + IX_KGT + off) = pack8(kg);
-                *reinterpret_cast<uint4*>(sm + IX_VT + off) = pack8(vv);
-                *reinterpret_cast<uint4*>(sm + IX_KTT + off) = pack8(kt);
-            }
-            gamC = __expf(G[4]);
-        }
         fence_async_smem();
         tc_fence_before();
         __syncthreads();
@@ -584,20 +673,9 @@ intra_kernel(const ChunkArgs a, const __grid_constant__ IntraMaps maps, const in
 
         // ---- round 2: Wt = KGt Ti^T, Ut = Vt Ti^T
         if (tid == 0) {
-            mma_sw128<4, 128, 64>(tm + TM_WT, sdesc_k_sw128(sb + IX_KGT), sdesc_k_sw128(sb + IX_TI), idesc_bf16(128, 64));
-            mma_sw128<4, 128, 64>(tm + TM_UT, sdesc_k_sw128(sb + IX_VT), sdesc_k_sw128(sb + IX_TI), idesc_bf16(128, 64));
+            mma_sw128<4, 128, 64>(tm + TM_WT, sdesc_k_sw128(sb + Z2_KGT), sdesc_k_sw128(sb + IX_TI), idesc_bf16(128, 64));
+            mma_sw128<4, 128, 64>(tm + TM_UT, sdesc_k_sw128(sb + Z2_VT), sdesc_k_sw128(sb + IX_TI), idesc_bf16(128, 64));
             mma_commit(bar_mma);
-        }
-        // next item's raw tiles (every read of RAW for this item is done) and beta
-        const int64_t next = s_next64[0];
-        if (next < n_items) {
-            const int64_t tt = s_next64[1];
-            const int hh = s_next32[0], LL = s_next32[1];
-            if constexpr (IN_BF16) {
-                if (tid == 0) issue_raw(hh, tt);
-                raw_in_flight = true;
-            }
-            if (tid < CH) beta_next = (tid < LL) ? ld_in<IN_BF16>(a.beta, (size_t)(tt + tid) * H + hh) : 0.f;
         }
         mbar_wait(bar_mma, ph_mma, a.status);
         ph_mma ^= 1;
@@ -619,26 +697,28 @@ intra_kernel(const ChunkArgs a, const __grid_constant__ IntraMaps maps, const in
         __syncthreads();
         tc_fence_after();
 
-        // ---- round 3: Mlr = Ktt Wt^T, Bm = Ktt Ut^T, (P W)^T = Wt Ph^T, Ob^T = Ut Ph^T
+        // ---- round 3: [Mlr | Bm] = Ktt [Wt ; Ut]^T (Wt and Ut are one 256-row image), then
+        //      (P W)^T = Wt Ph^T and Ob^T = Ut Ph^T under a second commit, so that staging of
+        //      Mlr and Bm overlaps the second pair of products.
         if (tid == 0) {
-            const uint64_t dk = sdesc_k_sw128(sb + IX_KTT), dw = sdesc_k_sw128(sb + IY_WT),
+            const uint64_t dk = sdesc_k_sw128(sb + Z2_KTT), dw = sdesc_k_sw128(sb + IY_WT),
                            du = sdesc_k_sw128(sb + IY_UT), dp = sdesc_k_sw128(sb + IX_PH);
-            mma_sw128<4, 128, 128>(tm + TM_M, dk, dw, idesc_bf16(128, 128));
-            mma_sw128<4, 128, 64>(tm + TM_PW, dw, dp, idesc_bf16(128, 64));
-            mma_sw128<4, 128, 128>(tm + TM_BM, dk, du, idesc_bf16(128, 128));
-            mma_sw128<4, 128, 64>(tm + TM_OB, du, dp, idesc_bf16(128, 64));
+            mma_sw128<4, 128, 256>(tm + TM_M, dk, dw, idesc_bf16(128, 256));
             mma_commit(bar_mma);
+            mma_sw128<4, 128, 64>(tm + TM_PW, dw, dp, idesc_bf16(128, 64));
+            mma_sw128<4, 128, 64>(tm + TM_OB, du, dp, idesc_bf16(128, 64));
+            mma_commit(bar_mma2);
         }
+        // The slot is assembled in two shared-memory pieces that match its layout:
+        // [Mlr | Qp | GamC] at IX (KQr/KC/Ti are dead) and [Bm | ObT] at Z2 (dead once
+        // the first product is done); each leaves by one bulk copy.
         mbar_wait(bar_mma, ph_mma, a.status);
         ph_mma ^= 1;
         tc_fence_after();
         {
-            // The slot is assembled in shared memory (operand regions X and Y are dead
-            // once round 3 has completed) and written by one bulk copy.
-            uint8_t* st = sm + IX;
             if (q4 < 2) {
                 // Mlr row c, K block q4 -> K-major SW128 image
-                uint8_t* dstM = st + SO_M + (size_t)q4 * (DK * 128);
+                uint8_t* dstM = sm + IX + SO_M + (size_t)q4 * (DK * 128);
 #pragma unroll
                 for (int hp = 0; hp < 2; ++hp) {
                     float d[32];
@@ -659,40 +739,44 @@ intra_kernel(const ChunkArgs a, const __grid_constant__ IntraMaps maps, const in
                     tmem_ld16(lane_addr + TM_BM + 64 * hh + 32 * hp, d);
                     tmem_ld16(lane_addr + TM_BM + 64 * hh + 32 * hp + 16, d + 16);
                     tmem_ld_wait();
-                    uint4* dstB = reinterpret_cast<uint4*>(st + SO_B + (size_t)(2 * hh + hp) * BSL + (size_t)c * DVS * 2);
+                    uint4* dstB = reinterpret_cast<uint4*>(sm + Z2 + (size_t)(2 * hh + hp) * BSL + (size_t)c * DVS * 2);
 #pragma unroll
                     for (int pp = 0; pp < 4; ++pp) dstB[pp] = pack8(d + 8 * pp);
                 }
-                if (q4 == 3) *reinterpret_cast<float*>(st + SO_G + 4 * c) = gamC;
+                if (q4 == 3) *reinterpret_cast<float*>(sm + IX + SO_G + 4 * c) = __expf(G[4]);  // Gam_C
             }
+        }
+        mbar_wait(bar_mma2, ph_mma2, a.status);
+        ph_mma2 ^= 1;
+        tc_fence_after();
+        {
             // Qp^T[c][t] = scale q_tc e^{g_tc} - (P W)^T[c][t] -> MN-major image (token-contiguous rows);
             // Ob^T[j][t] -> slice j/32, row j%32 (64 tokens).  This thread's 16 tokens.
-            {
-                const float eG = __expf(Gs);
-                float pw[16], ob[16], qq[16];
-                tmem_ld16(lane_addr + TM_PW + 16 * q4, pw);
-                tmem_ld16(lane_addr + TM_OB + 16 * q4, ob);
-                tmem_ld_wait();
+            const float eG = __expf(Gs);
+            float pw[16], ob[16], qq[16];
+            tmem_ld16(lane_addr + TM_PW + 16 * q4, pw);
+            tmem_ld16(lane_addr + TM_OB + 16 * q4, ob);
+            tmem_ld_wait();
 #pragma unroll
-                for (int u = 0; u < 16; ++u) {
-                    const float qv = __uint_as_float((u & 1) ? (qr2[u >> 1] & 0xFFFF0000u) : (qr2[u >> 1] << 16));
-                    qq[u] = qv * E1[u] * eG * a.scale - pw[u];
-                }
-                const int tf = 16 * q4;
-                uint8_t* dstQ = st + SO_Q;
-                uint8_t* dstO = st + SO_O + (size_t)(c >> 5) * OSL + (size_t)(c & 31) * (CH * 2);
-                *reinterpret_cast<uint4*>(dstQ + mn_off(tf, c, 1024)) = pack8(qq);
-                *reinterpret_cast<uint4*>(dstQ + mn_off(tf + 8, c, 1024)) = pack8(qq + 8);
-                *reinterpret_cast<uint4*>(dstO + tf * 2) = pack8(ob);
-                *reinterpret_cast<uint4*>(dstO + tf * 2 + 16) = pack8(ob + 8);
+            for (int u = 0; u < 16; ++u) {
+                const float qv = __uint_as_float((u & 1) ? (qr2[u >> 1] & 0xFFFF0000u) : (qr2[u >> 1] << 16));
+                qq[u] = qv * E1[u] * eG * a.scale - pw[u];
             }
+            const int tf = 16 * q4;
+            uint8_t* dstQ = sm + IX + SO_Q;
+            uint8_t* dstO = sm + Z2 + (SO_O - SO_B) + (size_t)(c >> 5) * OSL + (size_t)(c & 31) * (CH * 2);
+            *reinterpret_cast<uint4*>(dstQ + mn_off(tf, c, 1024)) = pack8(qq);
+            *reinterpret_cast<uint4*>(dstQ + mn_off(tf + 8, c, 1024)) = pack8(qq + 8);
+            *reinterpret_cast<uint4*>(dstO + tf * 2) = pack8(ob);
+            *reinterpret_cast<uint4*>(dstO + tf * 2 + 16) = pack8(ob + 8);
         }
         fence_async_smem();
         tc_fence_before();
         __syncthreads();
         tc_fence_after();
         if (tid == 0) {
-            bulk_s2g(wslot, sm + IX, (uint32_t)SLOT_BYTES);
+            bulk_s2g(wslot, sm + IX, SO_MQG);
+            bulk_s2g(wslot + SO_B, sm + Z2, (uint32_t)(SLOT_BYTES - SO_B));
             bulk_commit();
         }
         item = next;

@@ -94,6 +94,11 @@ KDA_DEV void bulk_g2s(void* smem_dst, const void* gmem_src, uint32_t bytes, uint
         : "memory");
 }
 
+// Brings a tensor map (kernel parameter or global) into the descriptor cache.
+KDA_DEV void prefetch_tmap(const CUtensorMap* map) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
 // 2-D tiled TMA load of box (x, y) of a tensor map into shared memory,
 // completion signalled on `bar`.  x is the innermost coordinate (elements);
 // x * element size must be a multiple of 16 bytes.
