@@ -62,7 +62,7 @@ constexpr int NSL = DV / DVS;
 //   Qp   bf16 MN-major no-swizzle image, M = 64 tokens, K = 128   16384 B
 //   GamC fp32 [128]                                                512 B
 //   Bm   bf16 [4 slices][128 key rows][32 value cols]            32768 B
-//   ObT  bf16 [4 slices][32 value cols][64 tokens]               16384 B
+//   Ob   bf16 [4 slices][64 tokens][32 value cols]               16384 B
 constexpr size_t SO_M = 0, SO_Q = 32768, SO_G = 49152, SO_B = 49664, SO_O = 82432;
 constexpr size_t SLOT_BYTES = 98816;
 constexpr uint32_t SO_MQG = 49664;         // Mlr + Qp + GamC, one contiguous copy
@@ -169,10 +169,11 @@ KDA_DEV uint4 pack8(const float* x) {
 //   Z2  [171K, 219K) KGt, Vt, Ktt [128][64] (built while round 1 runs)
 //   misc             beta[64], G[5][128], tile totals[4][128], 2 mbarriers, TMEM base
 // The workspace slot leaves at the end of an item as two bulk copies: [Mlr | Qp | GamC]
-// assembled at X, [Bm | ObT] at Z2.
+// assembled at X, [Bm | Ob] at Z2.
 // TMEM (512 columns): round 1  A/P diag [0,64), off-diag [64,80) [80,112) [112,160)
 //                     round 2  Wt [160,224), Ut [224,288)
-//                     round 3  [Mlr | Bm] [0,256) (one N = 256 product), (PW)^T [256,320), Ob^T [320,384)
+//                     round 3  [Mlr | Bm] [0,256) (one N = 256 product), (PW)^T [256,320),
+//                              Ob = P Ut^T [320,448) (M = 64: token t in lane 32 (t / 16) + t % 16)
 constexpr int INTRA_THREADS = 512;
 constexpr uint32_t R_LA = 0, R_K = 16384, R_Q = 32768, R_V = 49152;
 constexpr uint32_t IX = 65536;
@@ -698,7 +699,7 @@ intra_kernel(const ChunkArgs a, const __grid_constant__ IntraMaps maps, const in
         tc_fence_after();
 
         // ---- round 3: [Mlr | Bm] = Ktt [Wt ; Ut]^T (Wt and Ut are one 256-row image), then
-        //      (P W)^T = Wt Ph^T and Ob^T = Ut Ph^T under a second commit, so that staging of
+        //      (P W)^T = Wt Ph^T and Ob = Ph Ut^T (M = 64) under a second commit, so that staging of
         //      Mlr and Bm overlaps the second pair of products.
         if (tid == 0) {
             const uint64_t dk = sdesc_k_sw128(sb + Z2_KTT), dw = sdesc_k_sw128(sb + IY_WT),
@@ -706,11 +707,11 @@ intra_kernel(const ChunkArgs a, const __grid_constant__ IntraMaps maps, const in
             mma_sw128<4, 128, 256>(tm + TM_M, dk, dw, idesc_bf16(128, 256));
             mma_commit(bar_mma);
             mma_sw128<4, 128, 64>(tm + TM_PW, dw, dp, idesc_bf16(128, 64));
-            mma_sw128<4, 128, 64>(tm + TM_OB, du, dp, idesc_bf16(128, 64));
+            mma_sw128<4, 64, 128>(tm + TM_OB, dp, du, idesc_bf16(64, 128));
             mma_commit(bar_mma2);
         }
         // The slot is assembled in two shared-memory pieces that match its layout:
-        // [Mlr | Qp | GamC] at IX (KQr/KC/Ti are dead) and [Bm | ObT] at Z2 (dead once
+        // [Mlr | Qp | GamC] at IX (KQr/KC/Ti are dead) and [Bm | Ob] at Z2 (dead once
         // the first product is done); each leaves by one bulk copy.
         mbar_wait(bar_mma, ph_mma, a.status);
         ph_mma ^= 1;
@@ -750,12 +751,11 @@ intra_kernel(const ChunkArgs a, const __grid_constant__ IntraMaps maps, const in
         ph_mma2 ^= 1;
         tc_fence_after();
         {
-            // Qp^T[c][t] = scale q_tc e^{g_tc} - (P W)^T[c][t] -> MN-major image (token-contiguous rows);
-            // Ob^T[j][t] -> slice j/32, row j%32 (64 tokens).  This thread's 16 tokens.
+            // Qp^T[c][t] = scale q_tc e^{g_tc} - (P W)^T[c][t] -> MN-major image (token-contiguous
+            // rows), this thread's 16 tokens
             const float eG = __expf(Gs);
-            float pw[16], ob[16], qq[16];
+            float pw[16], qq[16];
             tmem_ld16(lane_addr + TM_PW + 16 * q4, pw);
-            tmem_ld16(lane_addr + TM_OB + 16 * q4, ob);
             tmem_ld_wait();
 #pragma unroll
             for (int u = 0; u < 16; ++u) {
@@ -764,11 +764,21 @@ intra_kernel(const ChunkArgs a, const __grid_constant__ IntraMaps maps, const in
             }
             const int tf = 16 * q4;
             uint8_t* dstQ = sm + IX + SO_Q;
-            uint8_t* dstO = sm + Z2 + (SO_O - SO_B) + (size_t)(c >> 5) * OSL + (size_t)(c & 31) * (CH * 2);
             *reinterpret_cast<uint4*>(dstQ + mn_off(tf, c, 1024)) = pack8(qq);
             *reinterpret_cast<uint4*>(dstQ + mn_off(tf + 8, c, 1024)) = pack8(qq + 8);
-            *reinterpret_cast<uint4*>(dstO + tf * 2) = pack8(ob);
-            *reinterpret_cast<uint4*>(dstO + tf * 2 + 16) = pack8(ob + 8);
+        }
+        {
+            // Ob row t = 16 qd + lane (lanes < 16 of each quadrant), value slice q4 -> [slice][t][32]
+            float ob[32];
+            tmem_ld16(lane_addr + TM_OB + 32 * q4, ob);
+            tmem_ld16(lane_addr + TM_OB + 32 * q4 + 16, ob + 16);
+            tmem_ld_wait();
+            if (lane < 16) {
+                uint4* dstO = reinterpret_cast<uint4*>(sm + Z2 + (SO_O - SO_B) + (size_t)q4 * OSL +
+                                                       (size_t)(16 * qd + lane) * (DVS * 2));
+#pragma unroll
+                for (int pp = 0; pp < 4; ++pp) dstO[pp] = pack8(ob + 8 * pp);
+            }
         }
         fence_async_smem();
         tc_fence_before();
@@ -806,9 +816,9 @@ intra_kernel(const ChunkArgs a, const __grid_constant__ IntraMaps maps, const in
 // overlaps the output work of the current chunk.  TMEM (128 columns): D_S =
 // Mlr S in [0,32) (M=128, lane = row c); D_O = Qp S double-buffered in [32,64)
 // and [64,96) (M=64: row t lives in lane 32*(t/16) + t%16).  Shared memory:
-// three chunk buffers {Mlr image 32K, Qp image 16K, GamC 512, Bm slice 8K, ObT
-// slice 4K[, gate tile 4K]} and two bf16 state operand images Sb [32 value
-// cols][128 key rows].
+// three chunk buffers {Mlr image 32K, Qp image 16K, GamC 512, Bm slice 8K, Ob
+// slice [64 tokens][32 cols] 4K[, gate tile 4K]} and two bf16 state operand
+// images (MN-major without swizzle: value columns contiguous, 8 KB each).
 //
 // Barriers and the order that keeps each phase from being skipped:
 //   bar_img   consumers (128) -> producer: state image of chunk i written.  The
@@ -843,6 +853,7 @@ template <bool GATE> struct ChainLayout {
     static constexpr uint32_t SMEM = TMEMP + 16 + 1024;
 };
 constexpr uint32_t CHAIN_TMEM_COLS = 128;
+constexpr uint32_t SB_KG = DVS * 16;  // state image K-group stride: 8 key rows x 32 columns x 2 B
 constexpr int CHAIN_THREADS = 160;  // 4 consumer warps + 1 producer warp
 constexpr int CLUSTER = NSL;        // CTAs per (sequence, head) when the gate is fused
 constexpr uint32_t PART_TX = CLUSTER * 64 * 4;  // partial-sum bytes each CTA receives per chunk
@@ -957,17 +968,24 @@ chain_kernel(const ChunkArgs a, const __grid_constant__ CUtensorMap gate_map, co
                     loads_waited = it + 1;
                     tc_fence_after();
                     // Mlr S -> D_S, then Qp S -> D_O[it & 1]
-                    const uint64_t sdesc = sdesc_k_sw128(sbase + LY::SB + (it & 1) * 8192);
-                    mma_sw128<8, 128, DVS>(tm + 0, sdesc_k_sw128(sbase + b * CB_SIZE + CB_M), sdesc,
-                                           idesc_bf16(128, DVS));
+                    // state image: MN-major, K-group (8 key rows) stride SB_KG, 8-column block stride 128
+                    const uint64_t sdesc = sdesc_interleave(sbase + LY::SB + (it & 1) * 8192, SB_KG, 128u);
+                    {  // Mlr (K-major SW128) x state image
+                        const uint64_t mdesc = sdesc_k_sw128(sbase + b * CB_SIZE + CB_M);
+#pragma unroll
+                        for (int kk = 0; kk < DK / 16; ++kk)
+                            mma_bf16(tm + 0, mdesc + (uint32_t)(((kk >> 2) * 128 * 128 + (kk & 3) * 32) >> 4),
+                                     sdesc + (uint32_t)((kk * 2 * SB_KG) >> 4), idesc_bf16_major(128, DVS, 0, 1),
+                                     kk > 0 ? 1u : 0u);
+                    }
                     mma_commit(bar_s);
-                    {  // Qp (MN-major, no swizzle) x state image (K-major SW128)
+                    {  // Qp (MN-major, no swizzle) x state image
                         const uint64_t qdesc = sdesc_interleave(sbase + b * CB_SIZE + CB_Q, 1024u, 128u);
 #pragma unroll
                         for (int kk = 0; kk < DK / 16; ++kk)
                             mma_bf16(tm + 32 + 32 * (it & 1), qdesc + (uint32_t)((kk * 2048) >> 4),
-                                     sdesc + (uint32_t)(((kk >> 2) * DVS * 128 + (kk & 3) * 32) >> 4),
-                                     idesc_bf16_major(64, DVS, 1, 0), kk > 0 ? 1u : 0u);
+                                     sdesc + (uint32_t)((kk * 2 * SB_KG) >> 4), idesc_bf16_major(64, DVS, 1, 1),
+                                     kk > 0 ? 1u : 0u);
                     }
                     mma_commit(&bar_o[it & 1]);
                     mma_issued = it + 1;
@@ -986,13 +1004,12 @@ chain_kernel(const ChunkArgs a, const __grid_constant__ CUtensorMap gate_map, co
         } else {
             // ----------------------------------------------------- consumers
             const uint32_t lane_addr = tm + ((uint32_t)(32 * warp) << 16);
+            // bf16 state operand, MN-major without swizzle (value columns contiguous): key
+            // row c's 32 columns are four 16-byte pieces, one per 8-column block
             auto write_state_image = [&](int it) {
-                const uint32_t kb = (uint32_t)tid >> 6, kc = (uint32_t)tid & 63u;
-                uint8_t* img = sm + LY::SB + (it & 1) * 8192;
+                uint8_t* img = sm + LY::SB + (it & 1) * 8192 + ((uint32_t)tid >> 3) * SB_KG + ((uint32_t)tid & 7u) * 16u;
 #pragma unroll
-                for (int j = 0; j < DVS; ++j)
-                    *reinterpret_cast<uint16_t*>(img + kb * (DVS * 128) + sw128_off((uint32_t)j, kc)) =
-                        f32_to_bf16(S[j]);
+                for (int nb = 0; nb < DVS / 8; ++nb) *reinterpret_cast<uint4*>(img + nb * 128) = pack8(S + 8 * nb);
                 fence_async_smem();
                 tc_fence_before();
                 mbar_arrive(bar_img);
@@ -1091,10 +1108,18 @@ chain_kernel(const ChunkArgs a, const __grid_constant__ CUtensorMap gate_map, co
                     float dO[DVS];
                     tmem_ld32(lane_addr + 32 + 32 * (it & 1), dO);
                     tmem_ld_wait();
-                    // Ob^T slice [32 value cols][64 tokens]: column trow
-                    const uint16_t* osrc = reinterpret_cast<const uint16_t*>(buf + CB_O) + trow;
+                    // Ob slice [64 tokens][32 value cols]: row trow
+                    const uint4* orow = reinterpret_cast<const uint4*>(buf + CB_O + (uint32_t)trow * (DVS * 2));
 #pragma unroll
-                    for (int j = 0; j < DVS; ++j) ov[j] = dO[j] + bf16_to_f32(osrc[j * CH]);
+                    for (int m = 0; m < DVS / 8; ++m) {
+                        const uint4 w = orow[m];
+                        const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                        for (int p = 0; p < 4; ++p) {
+                            ov[8 * m + 2 * p] = dO[8 * m + 2 * p] + __uint_as_float(ww[p] << 16);
+                            ov[8 * m + 2 * p + 1] = dO[8 * m + 2 * p + 1] + __uint_as_float(ww[p] & 0xFFFF0000u);
+                        }
+                    }
                 }
                 if constexpr (!GATE) {
                     if (lane < 16 && trow < L) {
