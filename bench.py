@@ -303,6 +303,31 @@ def run_decode(args, torch, kda, dev, stream, rank, max_over_ranks, barrier):
     peaks = load_peaks()
     gbs = (state_bytes + tok_bytes) * steps_s / 1e9
     kgbs = (state_bytes + tok_bytes) / (kern_ms * 1e-3) / 1e9 if kern_ms > 0 else None
+
+    # speculative verification: SPEC draft tokens per call (kda_decode_steps), state carried in place
+    SPEC = 4
+    sq = {n: torch.stack([toks[(i % pool)][n] for i in range(SPEC)]) for n in ("q", "k", "v", "log_alpha", "beta")}
+    osp = torch.empty((SPEC, Bd, H, D), dtype=torch.bfloat16, device=dev)
+
+    def vstep():
+        kda.decode_steps(state, sq["q"], sq["k"], sq["v"], sq["log_alpha"], sq["beta"], out=osp, stream=stream)
+
+    for _ in range(3):
+        vstep()
+    ncalls = nsteps // SPEC
+    barrier()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(ncalls):
+        vstep()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    ms_v = max_over_ranks(e0.elapsed_time(e1))
+    spec = {"draft_tokens_per_call": SPEC, "calls": ncalls, "ms_per_call": ms_v / ncalls,
+            "tokens_per_s": ncalls * SPEC / (ms_v * 1e-3),
+            "bytes_per_call": state_bytes + SPEC * tok_bytes,
+            "gbs": (state_bytes + SPEC * tok_bytes) * ncalls / (ms_v * 1e-3) / 1e9}
     return {"workload": f"KDA decode, {Bd} sequences x {H} heads, fp32 state 128x128 (512 MiB), {nsteps} "
                         f"consecutive steps, bf16 tokens (pool of {pool} distinct steps)",
             "value": steps_s, "unit": "steps/s", "ms_per_step": ms / nsteps, "state_gbs": gbs,
@@ -310,7 +335,8 @@ def run_decode(args, torch, kda, dev, stream, rank, max_over_ranks, barrier):
             "roofline": {"bound": "hbm", "kernel": "decode_step_kernel", "achieved": kgbs, "peak": peaks["hbm_gbs"],
                          "unit": "GB/s", "frac": (kgbs / peaks["hbm_gbs"]) if kgbs else None,
                          "traffic": recorded_traffic("decode_step_kernel", Bd * H),
-                         "algorithmic_bytes_per_launch": state_bytes + tok_bytes}}
+                         "algorithmic_bytes_per_launch": state_bytes + tok_bytes},
+            "speculative_verify": spec}
 
 
 def run_e2e(args, torch, kda, hq, out, fs, ws, stream, max_over_ranks, barrier):

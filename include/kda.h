@@ -131,6 +131,30 @@ KDA_API kda_status kda_chunk_fwd(const void* q, const void* k, const void* v, co
                          void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * kda_chunk_fwd_ckpt -- kda_chunk_fwd that also emits state checkpoints for a
+ * prefix cache (the "training and inference systems" item of the K3 article
+ * summaries: states cached at 512-token boundaries).  Arguments as
+ * kda_chunk_fwd, plus:
+ *
+ *   checkpoints  NULL (then identical to kda_chunk_fwd), or fp32
+ *                [n_seqs, n_ckpt, H, dk, dv] with n_ckpt = max_seqlen /
+ *                ckpt_tokens (fixed length: T / ckpt_tokens), 16-byte aligned.
+ *                Checkpoint j of sequence n is the state after that sequence's
+ *                first (j + 1) * ckpt_tokens tokens (initial state included);
+ *                checkpoints beyond a sequence's length are not written.
+ *   ckpt_tokens  checkpoint spacing in tokens, a positive multiple of 64
+ *                (the chunk length); KDA_ERR_INVALID_ARG otherwise.
+ */
+KDA_API kda_status kda_chunk_fwd_ckpt(const void* q, const void* k, const void* v, const void* log_alpha,
+                              const void* beta, const float* init_state, void* o,
+                              float* final_state, int B, int64_t T, int H, int dk, int dv,
+                              const int32_t* cu_seqlens, int n_seqs, int64_t max_seqlen,
+                              kda_dtype in_dtype, kda_dtype out_dtype, float scale,
+                              const void* gate, const float* norm_weight, float eps,
+                              float* checkpoints, int64_t ckpt_tokens,
+                              void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * kda_decode_step -- one recurrent step for Bd independent sequences
  * ("decode uses the recurrent form", chunkwise-algorithm item of the K3
  * article summaries).  The state is read once and written once, in place.
@@ -145,6 +169,33 @@ KDA_API kda_status kda_decode_step(float* state, const void* q, const void* k, c
                            int dk, int dv, kda_dtype in_dtype, kda_dtype out_dtype,
                            float scale, const void* gate, const float* norm_weight,
                            float eps, void* stream);
+
+/*
+ * kda_decode_steps -- n_steps consecutive recurrent steps for Bd independent
+ * sequences in one call: verification of n_steps draft tokens in speculative
+ * decoding, or plain decode of several tokens.  (Decode runs the recurrent
+ * form, chunkwise-algorithm item of the K3 article summaries; speculative
+ * decoding with state rollback is the "training and inference systems" item.)
+ * Each (sequence, head) state is read once and written once for all steps.
+ *
+ *   state        [Bd, H, dk, dv] fp32: the state before step 0; on return the
+ *                state after the last step
+ *   q, k, log_alpha, gate [n_steps, Bd, H, dk]; v [n_steps, Bd, H, dv];
+ *   beta [n_steps, Bd, H]          in_dtype (step-major)
+ *   o            [n_steps, Bd, H, dv] out_dtype (y when gate != NULL)
+ *   step_states  NULL, or [n_steps, Bd, H, dk, dv] fp32: the state after each
+ *                step (step_states[n_steps - 1] equals the final state).  To
+ *                roll back to "accepted the first a tokens" (1 <= a <= n_steps)
+ *                copy step_states[a - 1] into the state; keep a copy of the
+ *                incoming state to reject every draft token.
+ * Errors as kda_decode_step; n_steps == 0 or Bd == 0 does nothing.
+ */
+KDA_API kda_status kda_decode_steps(float* state, const void* q, const void* k, const void* v,
+                            const void* log_alpha, const void* beta, void* o, int n_steps,
+                            int Bd, int H, int dk, int dv, kda_dtype in_dtype,
+                            kda_dtype out_dtype, float scale, const void* gate,
+                            const float* norm_weight, float eps, float* step_states,
+                            void* stream);
 
 /*
  * kda_gate_norm -- per-head RMSNorm over dv followed by the full-rank sigmoid

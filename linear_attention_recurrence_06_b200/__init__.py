@@ -64,8 +64,14 @@ def load_library(path: str | None = None):
     lib.kda_chunk_fwd.restype = i32
     lib.kda_chunk_fwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i32, i64, i32, i32, i32, vp, i32, i64,
                                   i32, i32, f32, vp, vp, f32, vp, sz, vp]
+    lib.kda_chunk_fwd_ckpt.restype = i32
+    lib.kda_chunk_fwd_ckpt.argtypes = list(lib.kda_chunk_fwd.argtypes[:22]) + [vp, i64] + \
+        list(lib.kda_chunk_fwd.argtypes[22:])
     lib.kda_decode_step.restype = i32
     lib.kda_decode_step.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, f32, vp, vp, f32, vp]
+    lib.kda_decode_steps.restype = i32
+    lib.kda_decode_steps.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, f32, vp, vp, f32,
+                                     vp, vp]
     lib.kda_gate_norm.restype = i32
     lib.kda_gate_norm.argtypes = [vp, vp, vp, f32, vp, i64, i32, i32, i32, vp]
     lib.kda_query_status.restype = i32
@@ -123,7 +129,8 @@ def workspace_size(T: int, H: int, n_seqs: int, max_seqlen: int, dk: int = HEAD_
 
 def chunk_fwd(q, k, v, log_alpha, beta, initial_state=None, *, cu_seqlens=None, max_seqlen=None,
               scale: float = 1.0, gate=None, norm_weight=None, eps: float = 1e-6, out_dtype=None,
-              output_final_state: bool = True, final_state=None, out=None, workspace=None, stream=None):
+              output_final_state: bool = True, final_state=None, out=None, workspace=None, stream=None,
+              checkpoints=None, ckpt_tokens: int = 512):
     """Chunkwise KDA prefill.
 
     q, k, log_alpha: [B, T, H, 128]; v: [B, T, H, 128]; beta: [B, T, H] (bf16 or
@@ -131,6 +138,9 @@ def chunk_fwd(q, k, v, log_alpha, beta, initial_state=None, *, cu_seqlens=None, 
     device plus max_seqlen (host int).  initial_state: fp32 [N, H, 128, 128] or
     None.  gate: [B, T, H, 128] or None (then o is returned unnormalised).
     Returns (o_or_y [B, T, H, 128], final_state fp32 [N, H, 128, 128] or None).
+    checkpoints: None, True (allocate zeros) or fp32 [N, max_seqlen // ckpt_tokens, H, 128, 128]
+    receiving the state after every ckpt_tokens tokens of each sequence (ckpt_tokens a
+    multiple of 64); then the return value is (o, final_state, checkpoints).
     """
     torch = _torch()
     _check_cuda(q, k, v, log_alpha, beta, initial_state, cu_seqlens, gate, norm_weight)
@@ -157,13 +167,23 @@ def chunk_fwd(q, k, v, log_alpha, beta, initial_state=None, *, cu_seqlens=None, 
     if workspace is None:
         _, full = workspace_size(B * T if cu_seqlens is None else T, H, N, max_seqlen, dk, dv)
         workspace = torch.empty(full, dtype=torch.uint8, device=q.device)
-    st = load_library().kda_chunk_fwd(
-        _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(initial_state), _ptr(o), _ptr(fs),
-        B, T, H, dk, dv, _ptr(cu_seqlens), N, int(max_seqlen), in_dt, _dt(o), float(scale), _ptr(gate),
-        _ptr(norm_weight), float(eps), _ptr(workspace), workspace.numel(), _stream(stream))
+    args = (_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(initial_state), _ptr(o), _ptr(fs),
+            B, T, H, dk, dv, _ptr(cu_seqlens), N, int(max_seqlen), in_dt, _dt(o), float(scale), _ptr(gate),
+            _ptr(norm_weight), float(eps))
+    tail = (_ptr(workspace), workspace.numel(), _stream(stream))
+    if checkpoints is None:
+        st = load_library().kda_chunk_fwd(*args, *tail)
+        if st != KDA_OK:
+            raise KdaError(st, "kda_chunk_fwd")
+        return o, fs
+    if checkpoints is True:
+        checkpoints = torch.zeros((N, int(max_seqlen) // ckpt_tokens, H, dk, dv), dtype=torch.float32,
+                                  device=q.device)
+    _check_cuda(checkpoints)
+    st = load_library().kda_chunk_fwd_ckpt(*args, _ptr(checkpoints), int(ckpt_tokens), *tail)
     if st != KDA_OK:
-        raise KdaError(st, "kda_chunk_fwd")
-    return o, fs
+        raise KdaError(st, "kda_chunk_fwd_ckpt")
+    return o, fs, checkpoints
 
 
 def decode_step(state, q, k, v, log_alpha, beta, *, scale: float = 1.0, gate=None, norm_weight=None,
@@ -184,6 +204,34 @@ def decode_step(state, q, k, v, log_alpha, beta, *, scale: float = 1.0, gate=Non
     if st != KDA_OK:
         raise KdaError(st, "kda_decode_step")
     return o
+
+
+def decode_steps(state, q, k, v, log_alpha, beta, *, scale: float = 1.0, gate=None, norm_weight=None,
+                 eps: float = 1e-6, out_dtype=None, out=None, step_states=None, stream=None):
+    """n consecutive recurrent steps in one call (e.g. verifying n draft tokens).
+    state: fp32 [Bd, H, 128, 128], carried through the steps in place;
+    q, k, log_alpha, v: [n, Bd, H, 128]; beta: [n, Bd, H].  step_states: None,
+    True (allocate) or an fp32 [n, Bd, H, 128, 128] tensor that receives the state
+    after every step.  Returns o (or y) [n, Bd, H, 128], or (o, step_states) when
+    step_states was requested."""
+    torch = _torch()
+    want = step_states is not None
+    if step_states is True:
+        step_states = torch.empty((q.shape[0],) + tuple(state.shape), dtype=torch.float32, device=q.device)
+    _check_cuda(state, q, k, v, log_alpha, beta, gate, norm_weight, step_states if want else None)
+    if state.dtype != torch.float32:
+        raise TypeError("state must be fp32")
+    n, Bd, H, dk = q.shape
+    dv = v.shape[-1]
+    odt = out_dtype if out_dtype is not None else q.dtype
+    o = out if out is not None else torch.empty((n, Bd, H, dv), dtype=odt, device=q.device)
+    st = load_library().kda_decode_steps(_ptr(state), _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta),
+                                         _ptr(o), n, Bd, H, dk, dv, _dt(q), _dt(o), float(scale), _ptr(gate),
+                                         _ptr(norm_weight), float(eps), _ptr(step_states if want else None),
+                                         _stream(stream))
+    if st != KDA_OK:
+        raise KdaError(st, "kda_decode_steps")
+    return (o, step_states) if want else o
 
 
 def gate_norm(o, g, norm_weight=None, *, eps: float = 1e-6, out_dtype=None, out=None, stream=None):

@@ -14,7 +14,8 @@
 namespace kda {
 cudaError_t launch_decode_step(float* state, const void* q, const void* k, const void* v, const void* log_alpha,
                                const void* beta, void* o, int Bd, int H, bool in_bf16, bool out_bf16, float scale,
-                               const void* gate, const float* norm_w, float eps, cudaStream_t stream);
+                               const void* gate, const float* norm_w, float eps, int n_steps, float* step_states,
+                               cudaStream_t stream);
 cudaError_t launch_gate_norm(const void* o, const void* g, const float* norm_w, float eps, void* y, int64_t rows,
                              bool o_bf16, bool g_bf16, bool out_bf16, int num_sms, cudaStream_t stream);
 size_t chunk_slot_bytes();
@@ -22,8 +23,9 @@ size_t chunk_fixed_bytes(int n_seqs, int H, bool need_carry);
 cudaError_t chunk_fwd_launch(const void* q, const void* k, const void* v, const void* log_alpha, const void* beta,
                              const float* init_state, void* o, float* final_state, int B, int64_t T, int H,
                              const int32_t* cu, int n_seqs, int64_t max_seqlen, bool in_bf16, bool out_bf16,
-                             float scale, const void* gate, const float* norm_w, float eps, void* workspace,
-                             size_t ws_bytes, cudaStream_t stream, int* n_passes, bool* gate_fused);
+                             float scale, const void* gate, const float* norm_w, float eps, float* ckpt,
+                             int64_t ckpt_tokens, void* workspace, size_t ws_bytes, cudaStream_t stream, int* n_passes,
+                             bool* gate_fused);
 }  // namespace kda
 
 namespace kda {
@@ -126,11 +128,12 @@ kda_status kda_chunk_fwd_workspace_size(int64_t T, int H, int dk, int dv, int n_
     return KDA_OK;
 }
 
-kda_status kda_chunk_fwd(const void* q, const void* k, const void* v, const void* log_alpha, const void* beta,
-                         const float* init_state, void* o, float* final_state, int B, int64_t T, int H, int dk,
-                         int dv, const int32_t* cu_seqlens, int n_seqs, int64_t max_seqlen, kda_dtype in_dtype,
-                         kda_dtype out_dtype, float scale, const void* gate, const float* norm_weight, float eps,
-                         void* workspace, size_t workspace_bytes, void* stream) {
+kda_status kda_chunk_fwd_ckpt(const void* q, const void* k, const void* v, const void* log_alpha, const void* beta,
+                              const float* init_state, void* o, float* final_state, int B, int64_t T, int H, int dk,
+                              int dv, const int32_t* cu_seqlens, int n_seqs, int64_t max_seqlen, kda_dtype in_dtype,
+                              kda_dtype out_dtype, float scale, const void* gate, const float* norm_weight, float eps,
+                              float* checkpoints, int64_t ckpt_tokens, void* workspace, size_t workspace_bytes,
+                              void* stream) {
     if (!q || !k || !v || !log_alpha || !beta || !o) return KDA_ERR_INVALID_ARG;
     if (B <= 0 || T < 0 || H <= 0 || !dtype_ok(in_dtype) || !dtype_ok(out_dtype)) return KDA_ERR_INVALID_ARG;
     if (dk != kSupportedD || dv != kSupportedD) return KDA_ERR_UNSUPPORTED;
@@ -143,7 +146,9 @@ kda_status kda_chunk_fwd(const void* q, const void* k, const void* v, const void
     }
     if ((int64_t)B * T * H * 128 / 128 != (int64_t)B * T * H) return KDA_ERR_INVALID_ARG;
     if (eps < 0.f) return KDA_ERR_INVALID_ARG;
-    const void* ptrs[] = {q, k, v, log_alpha, beta, init_state, o, final_state, cu_seqlens, gate, norm_weight, workspace};
+    if (checkpoints && (ckpt_tokens <= 0 || ckpt_tokens % 64 != 0)) return KDA_ERR_INVALID_ARG;
+    const void* ptrs[] = {q, k, v, log_alpha, beta, init_state, o, final_state, cu_seqlens, gate, norm_weight, workspace,
+                          checkpoints};
     for (const void* p : ptrs)
         if (p && !aligned16(p)) return KDA_ERR_MISALIGNED;
     if (!workspace) return KDA_ERR_WORKSPACE;
@@ -159,7 +164,7 @@ kda_status kda_chunk_fwd(const void* q, const void* k, const void* v, const void
     bool fused = false;
     cudaError_t e = kda::chunk_fwd_launch(q, k, v, log_alpha, beta, init_state, o, final_state, B, T, H, cu_seqlens,
                                           n_seqs, max_seqlen, in_bf16, out_bf16, scale, gate, norm_weight, eps,
-                                          workspace, workspace_bytes, st, nullptr, &fused);
+                                          checkpoints, ckpt_tokens, workspace, workspace_bytes, st, nullptr, &fused);
     if (e != cudaSuccess) return KDA_ERR_CUDA;
     if (gate && !fused) {
         const int64_t rows = (int64_t)B * T * H;
@@ -173,24 +178,44 @@ kda_status kda_chunk_fwd(const void* q, const void* k, const void* v, const void
     return KDA_OK;
 }
 
+kda_status kda_chunk_fwd(const void* q, const void* k, const void* v, const void* log_alpha, const void* beta,
+                         const float* init_state, void* o, float* final_state, int B, int64_t T, int H, int dk,
+                         int dv, const int32_t* cu_seqlens, int n_seqs, int64_t max_seqlen, kda_dtype in_dtype,
+                         kda_dtype out_dtype, float scale, const void* gate, const float* norm_weight, float eps,
+                         void* workspace, size_t workspace_bytes, void* stream) {
+    return kda_chunk_fwd_ckpt(q, k, v, log_alpha, beta, init_state, o, final_state, B, T, H, dk, dv, cu_seqlens, n_seqs,
+                              max_seqlen, in_dtype, out_dtype, scale, gate, norm_weight, eps, nullptr, 0, workspace,
+                              workspace_bytes, stream);
+}
+
+kda_status kda_decode_steps(float* state, const void* q, const void* k, const void* v, const void* log_alpha,
+                            const void* beta, void* o, int n_steps, int Bd, int H, int dk, int dv,
+                            kda_dtype in_dtype, kda_dtype out_dtype, float scale, const void* gate,
+                            const float* norm_weight, float eps, float* step_states, void* stream) {
+    if (!state || !q || !k || !v || !log_alpha || !beta || !o) return KDA_ERR_INVALID_ARG;
+    if (n_steps < 0 || Bd < 0 || H <= 0 || !dtype_ok(in_dtype) || !dtype_ok(out_dtype) || eps < 0.f)
+        return KDA_ERR_INVALID_ARG;
+    if (dk != kSupportedD || dv != kSupportedD) return KDA_ERR_UNSUPPORTED;
+    if ((int64_t)Bd * H > INT32_MAX) return KDA_ERR_UNSUPPORTED;
+    const void* ptrs[] = {state, q, k, v, log_alpha, beta, o, gate, norm_weight, step_states};
+    for (const void* p : ptrs)
+        if (p && !aligned16(p)) return KDA_ERR_MISALIGNED;
+    if (Bd == 0 || n_steps == 0) return KDA_OK;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    kda::prof_begin(kda::PROF_DECODE, st);
+    const cudaError_t e = kda::launch_decode_step(state, q, k, v, log_alpha, beta, o, Bd, H, in_dtype == KDA_BF16,
+                                                  out_dtype == KDA_BF16, scale, gate, norm_weight, eps, n_steps,
+                                                  step_states, st);
+    kda::prof_end(kda::PROF_DECODE, st);
+    return from_cuda(e);
+}
+
 kda_status kda_decode_step(float* state, const void* q, const void* k, const void* v, const void* log_alpha,
                            const void* beta, void* o, int Bd, int H, int dk, int dv, kda_dtype in_dtype,
                            kda_dtype out_dtype, float scale, const void* gate, const float* norm_weight, float eps,
                            void* stream) {
-    if (!state || !q || !k || !v || !log_alpha || !beta || !o) return KDA_ERR_INVALID_ARG;
-    if (Bd < 0 || H <= 0 || !dtype_ok(in_dtype) || !dtype_ok(out_dtype) || eps < 0.f) return KDA_ERR_INVALID_ARG;
-    if (dk != kSupportedD || dv != kSupportedD) return KDA_ERR_UNSUPPORTED;
-    if ((int64_t)Bd * H > INT32_MAX) return KDA_ERR_UNSUPPORTED;
-    const void* ptrs[] = {state, q, k, v, log_alpha, beta, o, gate, norm_weight};
-    for (const void* p : ptrs)
-        if (p && !aligned16(p)) return KDA_ERR_MISALIGNED;
-    if (Bd == 0) return KDA_OK;
-    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    kda::prof_begin(kda::PROF_DECODE, st);
-    const cudaError_t e = kda::launch_decode_step(state, q, k, v, log_alpha, beta, o, Bd, H, in_dtype == KDA_BF16,
-                                                  out_dtype == KDA_BF16, scale, gate, norm_weight, eps, st);
-    kda::prof_end(kda::PROF_DECODE, st);
-    return from_cuda(e);
+    return kda_decode_steps(state, q, k, v, log_alpha, beta, o, 1, Bd, H, dk, dv, in_dtype, out_dtype, scale, gate,
+                            norm_weight, eps, nullptr, stream);
 }
 
 kda_status kda_gate_norm(const void* o, const void* gate, const float* norm_weight, float eps, void* y, int64_t rows,

@@ -88,6 +88,9 @@ struct ChunkArgs {
     int wc;                    // chunk slots per sequence in this pass
     int first_pass;
     float scale;
+    float* ckpt;               // nullable: states at every ckpt_every-th chunk boundary
+    int ckpt_every;            // in chunks
+    int n_ckpt;                // checkpoints per sequence in `ckpt`
 };
 
 // Token range [sb, se) of sequence n, clamped into [0, total tokens].
@@ -632,16 +635,24 @@ intra_kernel(const ChunkArgs a, const __grid_constant__ IntraMaps maps, const in
                 else store24(sZ0 + r0 * 16 + c0, 16, acc, 1.f);
             }
             __syncthreads();
-            // (3b) X_LL = -H_1 Z split over m: warps 0-3 m in block 2 (every row), warps 4-5 m in
+            // Z = Z^(1) + Z^(0) on the columns of block 0 (32 x 16, one float4 per thread)
+            if (tid < 128) {
+                const int r = tid >> 2, c4 = 4 * (tid & 3);
+                float4* z = reinterpret_cast<float4*>(sZ1 + r * 32 + c4);
+                const float4 z0 = *reinterpret_cast<const float4*>(sZ0 + r * 16 + c4);
+                float4 v = *z;
+                v.x += z0.x; v.y += z0.y; v.z += z0.z; v.w += z0.w;
+                *z = v;
+            }
+            __syncthreads();
+            // (3b) X_LL = -H_1 Z (Z complete in sZ1) split over m: warps 0-3 m in block 2 (every row), warps 4-5 m in
             //      block 3 (rows of block 3 only), kept as a partial that the T image adds
             if (tid < 192) {
                 const int g = tid >= 128;
                 const int k = g ? tid - 128 : tid;
                 const int r0 = g ? 16 + 2 * (k >> 3) : 2 * (k >> 3), c0 = 4 * (k & 7);
                 float acc[2][4] = {};
-                const float* Rp = sX + (32 + r0) * LDA + 32 + 16 * g;
-                tile24(Rp, LDA, sZ1 + (16 * g) * 32 + c0, 32, acc);
-                if (c0 < 16) tile24(Rp, LDA, sZ0 + (16 * g) * 16 + c0, 16, acc);
+                tile24(sX + (32 + r0) * LDA + 32 + 16 * g, LDA, sZ1 + (16 * g) * 32 + c0, 32, acc);
                 if (g) store24(sP + (r0 - 16) * 32 + c0, 32, acc, -1.f);
                 else store24(sX + (32 + r0) * LDA + c0, LDA, acc, -1.f);
             }
@@ -1096,7 +1107,6 @@ chain_kernel(const ChunkArgs a, const __grid_constant__ CUtensorMap gate_map, co
                 }
                 // (2) the next chunk's state operand (D_S has been read)
                 if (it + 1 < nit) write_state_image(it + 1);
-
                 // (3) this chunk's output: o = Qp S + Ob  (then y, when the gate is fused)
                 if (!mbar_wait(&bar_o[it & 1], (uint32_t)((it >> 1) & 1), a.status)) {
                     failed = true;
@@ -1168,6 +1178,19 @@ chain_kernel(const ChunkArgs a, const __grid_constant__ CUtensorMap gate_map, co
                     }
                     t0_prev = t0;
                     L_prev = L;
+                }
+                // checkpoint: the state after (j + 1) * ckpt_every whole chunks of the sequence
+                if (a.ckpt) {
+                    const int cdone = c_beg + it + 1;  // chunks of this sequence now folded in
+                    const int64_t t_end = s_beg + (int64_t)cdone * CH;
+                    if (cdone % a.ckpt_every == 0 && t_end <= s_end && cdone / a.ckpt_every <= a.n_ckpt) {
+                        const int j = cdone / a.ckpt_every - 1;
+                        float* dst =
+                            a.ckpt + ((((size_t)n * a.n_ckpt + j) * H + h) * DK + tid) * DV + (size_t)DVS * js;
+#pragma unroll
+                        for (int c4 = 0; c4 < DVS; c4 += 4)
+                            __stcs(reinterpret_cast<float4*>(dst + c4), make_float4(S[c4], S[c4 + 1], S[c4 + 2], S[c4 + 3]));
+                    }
                 }
                 // (4) this chunk's buffer and D_O[it & 1] are no longer read
                 tc_fence_before();
@@ -1261,8 +1284,9 @@ int g_num_sms = 0;
 cudaError_t chunk_fwd_launch(const void* q, const void* k, const void* v, const void* log_alpha, const void* beta,
                              const float* init_state, void* o, float* final_state, int B, int64_t T, int H,
                              const int32_t* cu, int n_seqs, int64_t max_seqlen, bool in_bf16, bool out_bf16,
-                             float scale, const void* gate, const float* norm_w, float eps, void* workspace,
-                             size_t ws_bytes, cudaStream_t stream, int* n_passes, bool* gate_fused) {
+                             float scale, const void* gate, const float* norm_w, float eps, float* ckpt,
+                             int64_t ckpt_tokens, void* workspace, size_t ws_bytes, cudaStream_t stream, int* n_passes,
+                             bool* gate_fused) {
     cudaError_t err;
     if (!g_attr_set) {
         err = cudaFuncSetAttribute(intra_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, INTRA_SMEM);
@@ -1305,6 +1329,9 @@ cudaError_t chunk_fwd_launch(const void* q, const void* k, const void* v, const 
     a.status = status;
     a.T = T;
     a.H = H; a.n_seqs = N; a.wc = wc; a.scale = scale;
+    a.ckpt = ckpt;
+    a.ckpt_every = ckpt ? (int)(ckpt_tokens / CH) : 1;
+    a.n_ckpt = ckpt ? (int)(maxlen / ckpt_tokens) : 0;
 
     IntraMaps maps;
     memset(&maps, 0, sizeof(maps));

@@ -12,25 +12,35 @@
 
 namespace kda {
 
-// One CTA = one (sequence, head) state [128 x 128] fp32 = 64 KiB.
+// One CTA = one (sequence, head) state [128 x 128] fp32 = 64 KiB, carried
+// through n_steps consecutive tokens (speculative-decode verification of n
+// draft tokens, or plain decode with n_steps = 1): the state is read once and
+// written once for all of them, and optionally also after every step so that
+// a caller can roll back to any accepted prefix.
 // 256 threads = 8 warps; warp w owns value columns [16w, 16w + 16).
 // Lane l: row phase r0 = l / 4 (0..7) and column quad cq = l % 4, so one warp
 // load instruction covers 8 rows x 64 contiguous bytes.  Thread holds rows
 // r0 + 8i (i = 0..15) x 4 columns = 64 fp32 registers.
+// Token tensors are step-major: element (step t, sequence-head bh, channel c)
+// at (t * BH + bh) * 128 + c (beta: t * BH + bh).
 template <bool IN_BF16, bool OUT_BF16, bool GATE>
 __global__ void __launch_bounds__(256, 2)
 decode_step_kernel(float* __restrict__ state, const void* __restrict__ q, const void* __restrict__ k,
                    const void* __restrict__ v, const void* __restrict__ log_alpha,
                    const void* __restrict__ beta, void* __restrict__ o, const void* __restrict__ gate,
-                   const float* __restrict__ norm_w, float scale, float eps) {
+                   const float* __restrict__ norm_w, float scale, float eps, int n_steps,
+                   float* __restrict__ step_states) {
     constexpr int D = 128;
     const int bh = blockIdx.x;  // sequence * H + head
+    const size_t BH = gridDim.x;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int r0 = lane >> 2, cq = lane & 3;
     const int col = warp * 16 + cq * 4;
 
-    __shared__ float s_k[D], s_q[D], s_alpha[D];
-    __shared__ float s_ss[8];
+    // per-step token vectors, double-buffered by step parity (the buffer of step
+    // t is rewritten at step t + 2, after the barrier of step t + 1)
+    __shared__ float s_k[2][D], s_q[2][D], s_alpha[2][D];
+    __shared__ float s_ss[2][8];
 
     float* S = state + (size_t)bh * D * D;
     float4 st[16];
@@ -38,79 +48,111 @@ decode_step_kernel(float* __restrict__ state, const void* __restrict__ q, const 
     for (int i = 0; i < 16; ++i)
         st[i] = __ldcs(reinterpret_cast<const float4*>(S + (size_t)(r0 + 8 * i) * D + col));
 
-    if (tid < D) {
-        const size_t idx = (size_t)bh * D + tid;
-        s_k[tid] = ld_in<IN_BF16>(k, idx);
-        s_q[tid] = ld_in<IN_BF16>(q, idx);
-        s_alpha[tid] = __expf(fmaxf(ld_in<IN_BF16>(log_alpha, idx), LOG_ALPHA_FLOOR));
-    }
-    const float b = ld_in<IN_BF16>(beta, (size_t)bh);
-    float vv[4];
-#pragma unroll
-    for (int c = 0; c < 4; ++c) vv[c] = ld_in<IN_BF16>(v, (size_t)bh * D + col + c);
-    __syncthreads();
-
-    // k . q (every warp computes it; 4 products per lane + butterfly)
-    float kq = 0.f;
-#pragma unroll
-    for (int m = 0; m < 4; ++m) kq += s_k[lane + 32 * m] * s_q[lane + 32 * m];
-#pragma unroll
-    for (int m = 16; m >= 1; m >>= 1) kq += __shfl_xor_sync(0xffffffffu, kq, m);
-
-    // decay rows, partial S'^T k and S'^T q over this thread's 16 rows
-    float sk[4] = {0.f, 0.f, 0.f, 0.f}, sq[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-        const int r = r0 + 8 * i;
-        const float a = s_alpha[r], kr = s_k[r], qr = s_q[r];
-        st[i].x *= a; st[i].y *= a; st[i].z *= a; st[i].w *= a;
-        sk[0] += st[i].x * kr; sk[1] += st[i].y * kr; sk[2] += st[i].z * kr; sk[3] += st[i].w * kr;
-        sq[0] += st[i].x * qr; sq[1] += st[i].y * qr; sq[2] += st[i].z * qr; sq[3] += st[i].w * qr;
-    }
-    // reduce over the 8 row phases (lanes that share cq)
-#pragma unroll
-    for (int m = 4; m <= 16; m <<= 1) {
+    // this step's token values, loaded one step ahead into registers
+    float nk = 0.f, nq = 0.f, nla = 0.f, nb, nv[4], ng[4];
+    auto load_step = [&](int t) {
+        const size_t tb = (size_t)t * BH + bh;
+        if (tid < D) {
+            const size_t idx = tb * D + tid;
+            nk = ld_in<IN_BF16>(k, idx);
+            nq = ld_in<IN_BF16>(q, idx);
+            nla = ld_in<IN_BF16>(log_alpha, idx);
+        }
+        nb = ld_in<IN_BF16>(beta, tb);
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
-            sk[c] += __shfl_xor_sync(0xffffffffu, sk[c], m);
-            sq[c] += __shfl_xor_sync(0xffffffffu, sq[c], m);
+            nv[c] = ld_in<IN_BF16>(v, tb * D + col + c);
+            if constexpr (GATE) ng[c] = ld_in<IN_BF16>(gate, tb * D + col + c);
         }
-    }
-    float u[4], oc[4];
-#pragma unroll
-    for (int c = 0; c < 4; ++c) {
-        u[c] = b * (vv[c] - sk[c]);
-        oc[c] = scale * (sq[c] + kq * u[c]);
-    }
-    // S_new = S' + k u^T, written back once
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-        const float kr = s_k[r0 + 8 * i];
-        st[i].x += kr * u[0]; st[i].y += kr * u[1]; st[i].z += kr * u[2]; st[i].w += kr * u[3];
-        __stcs(reinterpret_cast<float4*>(S + (size_t)(r0 + 8 * i) * D + col), st[i]);
-    }
+    };
+    load_step(0);
 
-    if constexpr (GATE) {
-        // per-head RMSNorm over the 128 value channels, then weight and gate
-        float ss = oc[0] * oc[0] + oc[1] * oc[1] + oc[2] * oc[2] + oc[3] * oc[3];
-        ss += __shfl_xor_sync(0xffffffffu, ss, 1);
-        ss += __shfl_xor_sync(0xffffffffu, ss, 2);
-        if (lane == 0) s_ss[warp] = ss;
+    for (int t = 0; t < n_steps; ++t) {
+        const int pb = t & 1;
+        const size_t tb = (size_t)t * BH + bh;  // token row of this step
+        if (tid < D) {
+            s_k[pb][tid] = nk;
+            s_q[pb][tid] = nq;
+            s_alpha[pb][tid] = __expf(fmaxf(nla, LOG_ALPHA_FLOOR));
+        }
+        const float b = nb;
+        float vv[4], gg4[4];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            vv[c] = nv[c];
+            gg4[c] = GATE ? ng[c] : 0.f;
+        }
+        if (t + 1 < n_steps) load_step(t + 1);  // in flight during this step
         __syncthreads();
-        float tot = 0.f;
+        const float* sk_ = s_k[pb];
+        const float* sq_ = s_q[pb];
+        const float* sa_ = s_alpha[pb];
+
+        // k . q (every warp computes it; 4 products per lane + butterfly)
+        float kq = 0.f;
 #pragma unroll
-        for (int w = 0; w < 8; ++w) tot += s_ss[w];
-        const float inv = rsqrtf(tot * (1.0f / D) + eps);
+        for (int m = 0; m < 4; ++m) kq += sk_[lane + 32 * m] * sq_[lane + 32 * m];
+#pragma unroll
+        for (int m = 16; m >= 1; m >>= 1) kq += __shfl_xor_sync(0xffffffffu, kq, m);
+
+        // decay rows, partial S'^T k and S'^T q over this thread's 16 rows
+        float sk[4] = {0.f, 0.f, 0.f, 0.f}, sq[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            const int r = r0 + 8 * i;
+            const float a = sa_[r], kr = sk_[r], qr = sq_[r];
+            st[i].x *= a; st[i].y *= a; st[i].z *= a; st[i].w *= a;
+            sk[0] += st[i].x * kr; sk[1] += st[i].y * kr; sk[2] += st[i].z * kr; sk[3] += st[i].w * kr;
+            sq[0] += st[i].x * qr; sq[1] += st[i].y * qr; sq[2] += st[i].z * qr; sq[3] += st[i].w * qr;
+        }
+        // reduce over the 8 row phases (lanes that share cq)
+#pragma unroll
+        for (int m = 4; m <= 16; m <<= 1) {
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                sk[c] += __shfl_xor_sync(0xffffffffu, sk[c], m);
+                sq[c] += __shfl_xor_sync(0xffffffffu, sq[c], m);
+            }
+        }
+        float u[4], oc[4];
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
-            const float gg = ld_in<IN_BF16>(gate, (size_t)bh * D + col + c);
-            const float wc = norm_w ? __ldg(norm_w + col + c) : 1.0f;
-            oc[c] = oc[c] * inv * wc * __fdividef(1.0f, 1.0f + __expf(-gg));
+            u[c] = b * (vv[c] - sk[c]);
+            oc[c] = scale * (sq[c] + kq * u[c]);
         }
-    }
-    if (r0 == 0) {
+        // S_new = S' + k u^T; this step's state when the caller keeps them, and the
+        // carried state written back once, at the last step
+        float* SS = step_states ? step_states + tb * D * D : nullptr;
+        const bool last = t + 1 == n_steps;
 #pragma unroll
-        for (int c = 0; c < 4; ++c) st_out<OUT_BF16>(o, (size_t)bh * D + col + c, oc[c]);
+        for (int i = 0; i < 16; ++i) {
+            const float kr = sk_[r0 + 8 * i];
+            st[i].x += kr * u[0]; st[i].y += kr * u[1]; st[i].z += kr * u[2]; st[i].w += kr * u[3];
+            if (SS) __stcs(reinterpret_cast<float4*>(SS + (size_t)(r0 + 8 * i) * D + col), st[i]);
+            if (last) __stcs(reinterpret_cast<float4*>(S + (size_t)(r0 + 8 * i) * D + col), st[i]);
+        }
+
+        if constexpr (GATE) {
+            // per-head RMSNorm over the 128 value channels, then weight and gate
+            float ss = oc[0] * oc[0] + oc[1] * oc[1] + oc[2] * oc[2] + oc[3] * oc[3];
+            ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+            ss += __shfl_xor_sync(0xffffffffu, ss, 2);
+            if (lane == 0) s_ss[pb][warp] = ss;
+            __syncthreads();
+            float tot = 0.f;
+#pragma unroll
+            for (int w = 0; w < 8; ++w) tot += s_ss[pb][w];
+            const float inv = rsqrtf(tot * (1.0f / D) + eps);
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                const float wc = norm_w ? __ldg(norm_w + col + c) : 1.0f;
+                oc[c] = oc[c] * inv * wc * __fdividef(1.0f, 1.0f + __expf(-gg4[c]));
+            }
+        }
+        if (r0 == 0) {
+#pragma unroll
+            for (int c = 0; c < 4; ++c) st_out<OUT_BF16>(o, tb * D + col + c, oc[c]);
+        }
     }
 }
 
@@ -187,11 +229,12 @@ gate_norm_kernel(const void* o, const void* __restrict__ g, const float* __restr
 cudaError_t launch_decode_step(float* state, const void* q, const void* k, const void* v,
                                const void* log_alpha, const void* beta, void* o, int Bd, int H,
                                bool in_bf16, bool out_bf16, float scale, const void* gate,
-                               const float* norm_w, float eps, cudaStream_t stream) {
+                               const float* norm_w, float eps, int n_steps, float* step_states,
+                               cudaStream_t stream) {
     const dim3 grid((unsigned)((int64_t)Bd * H)), block(256);
 #define KDA_DEC(IB, OB, G)                                                                              \
     decode_step_kernel<IB, OB, G><<<grid, block, 0, stream>>>(state, q, k, v, log_alpha, beta, o, gate, \
-                                                              norm_w, scale, eps)
+                                                              norm_w, scale, eps, n_steps, step_states)
     const bool g = gate != nullptr;
     if (in_bf16) {
         if (out_bf16) { if (g) KDA_DEC(true, true, true); else KDA_DEC(true, true, false); }

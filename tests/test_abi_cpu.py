@@ -27,7 +27,8 @@ def declared_symbols():
 
 def test_header_declares_the_entry_points():
     syms = declared_symbols()
-    for s in ("kda_chunk_fwd", "kda_decode_step", "kda_gate_norm", "kda_chunk_fwd_workspace_size",
+    for s in ("kda_chunk_fwd", "kda_chunk_fwd_ckpt", "kda_decode_step", "kda_decode_steps", "kda_gate_norm",
+              "kda_chunk_fwd_workspace_size",
               "kda_query_status", "kda_status_string", "kda_version"):
         assert s in syms
 
@@ -69,6 +70,23 @@ def _chunk(lib, **over):
                              a["gate"], a["w"], a["eps"], a["ws"], a["wsb"], a["stream"])
 
 
+def test_chunk_fwd_ckpt_host_validation(lib):
+    def ck(ptr, every, **over):
+        args = dict(q=FAKE, k=FAKE, v=FAKE, la=FAKE, beta=FAKE, s0=None, o=FAKE, fs=None, B=1, T=128, H=2,
+                    dk=128, dv=128, cu=None, N=1, maxlen=128, idt=1, odt=1, scale=1.0, gate=None, w=None, eps=1e-6,
+                    ws=FAKE, wsb=1 << 40, stream=None)
+        args.update(over)
+        a = args
+        return lib.kda_chunk_fwd_ckpt(a["q"], a["k"], a["v"], a["la"], a["beta"], a["s0"], a["o"], a["fs"], a["B"],
+                                      a["T"], a["H"], a["dk"], a["dv"], a["cu"], a["N"], a["maxlen"], a["idt"],
+                                      a["odt"], a["scale"], a["gate"], a["w"], a["eps"], ptr, every, a["ws"],
+                                      a["wsb"], a["stream"])
+    assert ck(FAKE, 100) == -1      # not a multiple of the chunk length
+    assert ck(FAKE, 0) == -1
+    assert ck(FAKE + 4, 64) == -3   # misaligned checkpoint buffer
+    assert ck(FAKE, 64, q=None) == -1
+
+
 def test_chunk_fwd_host_validation(lib):
     assert _chunk(lib, q=None) == -1
     assert _chunk(lib, o=None) == -1
@@ -95,6 +113,13 @@ def test_decode_and_gate_norm_host_validation(lib):
                                None, 1e-6, None) == -3
     assert lib.kda_decode_step(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 0, 2, 128, 128, 1, 1, 1.0, None, None,
                                1e-6, None) == 0  # nothing to do, no launch
+    # multi-step decode: negative step count, misaligned step_states, nothing to do
+    assert lib.kda_decode_steps(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, -1, 4, 2, 128, 128, 1, 1, 1.0, None, None,
+                                1e-6, None, None) == -1
+    assert lib.kda_decode_steps(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 3, 4, 2, 128, 128, 1, 1, 1.0, None, None,
+                                1e-6, FAKE + 8, None) == -3
+    assert lib.kda_decode_steps(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 0, 4, 2, 128, 128, 1, 1, 1.0, None, None,
+                                1e-6, None, None) == 0
     assert lib.kda_gate_norm(FAKE, FAKE, None, 1e-6, FAKE, -1, 128, 1, 1, None) == -1
     assert lib.kda_gate_norm(FAKE, FAKE, None, 1e-6, FAKE, 10, 64, 1, 1, None) == -2
     assert lib.kda_gate_norm(FAKE, FAKE, None, 1e-6, FAKE, 10, 128, 1, 0, None) == -1  # in place, sizes differ

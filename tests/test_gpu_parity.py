@@ -149,6 +149,44 @@ def test_prefill_gate_varlen_weights_multi_pass(bf16):
                 assert rel_l2(yh[sl], ry[sl]) <= REL_L2_TOL
 
 
+@pytest.mark.parametrize("multi_pass", [False, True])
+def test_prefill_state_checkpoints(multi_pass):
+    """Prefix-cache checkpoints: checkpoint j of a sequence equals the oracle's
+    final state after that sequence's first (j + 1) * 256 tokens; slots beyond a
+    sequence's length stay untouched (zero)."""
+    torch = _torch()
+    import linear_attention_recurrence_06_b200 as kda
+    lens, H, every = [700, 1100, 0, 513, 256], 2, 256
+    inp = make_prefill(31, lens, H, bf16=True, init=True)
+    T = inp["T"]
+    dt = torch.bfloat16
+    q, k, v, la = (dev(inp[x], dt).view(1, T, H, D) for x in ("q", "k", "v", "log_alpha"))
+    b = dev(inp["beta"], dt).view(1, T, H)
+    cu = inp["cu"]
+    kw = {}
+    if multi_pass:
+        lo, _ = kda.workspace_size(T, H, len(lens), max(lens))
+        kw["workspace"] = torch.empty(lo, dtype=torch.uint8, device="cuda")
+    o, fs, ck = kda.chunk_fwd(q, k, v, la, b, dev(inp["s0"], torch.float32),
+                              cu_seqlens=torch.from_numpy(cu.astype(np.int32)).cuda(), max_seqlen=max(lens),
+                              checkpoints=True, ckpt_tokens=every, **kw)
+    torch.cuda.synchronize()
+    ck = host(ck)
+    assert ck.shape == (len(lens), max(lens) // every, H, D, D)
+    for n, L in enumerate(lens):
+        for j in range(ck.shape[1]):
+            end = (j + 1) * every
+            if end > L:
+                assert not ck[n, j].any(), f"seq {n} checkpoint {j} written past the end"
+                continue
+            sl = slice(cu[n], cu[n] + end)
+            _, ref = oracle.kda_recurrent(inp["q"][sl], inp["k"][sl], inp["v"][sl], inp["log_alpha"][sl],
+                                          inp["beta"][sl], inp["s0"][n:n + 1])
+            assert rel_l2(ck[n, j], ref[0]) <= REL_L2_TOL, f"seq {n} checkpoint {j}"
+    # the last whole checkpoint of a sequence ending on a boundary is its final state
+    np.testing.assert_array_equal(ck[4, 0], host(fs)[4])
+
+
 def test_prefill_multi_pass_workspace():
     """A workspace that holds one chunk per sequence forces one pass per chunk:
     the state carried between passes must give the same result."""
@@ -213,6 +251,56 @@ def test_decode_steps(bf16, gate):
         torch.cuda.synchronize()
         assert rel_l2(host(o), ro) <= REL_L2_TOL
     assert rel_l2(host(s_dev), s_ref) <= REL_L2_TOL
+
+
+@pytest.mark.parametrize("bf16,gate,n", [(True, False, 1), (True, False, 4), (True, True, 8), (False, False, 3)])
+def test_decode_multi_step_with_step_states(bf16, gate, n):
+    """n consecutive steps in one call == n single steps of the oracle: every
+    step's output, every step's state (for rollback) and the carried state."""
+    torch = _torch()
+    import linear_attention_recurrence_06_b200 as kda
+    Bd, H = 5, 3
+    dt = torch.bfloat16 if bf16 else torch.float32
+    s0 = synth.states(7, Bd, H, D, D)
+    s_dev = dev(s0, torch.float32)
+    toks = [synth.tokens(7, step * Bd, Bd, H, D, D, bf16=bf16, gate=gate) for step in range(n)]
+    stack = lambda name: np.stack([getattr(tb, name) for tb in toks])
+    q, k, v, la = (dev(stack(x), dt) for x in ("q", "k", "v", "log_alpha"))
+    b = dev(stack("beta"), dt)
+    g = dev(stack("g"), dt) if gate else None
+    w = np.random.default_rng(7).uniform(0.5, 1.5, D).astype(np.float32) if gate else None
+    o, states = kda.decode_steps(s_dev, q, k, v, la, b, gate=g, norm_weight=dev(w, torch.float32) if gate else None,
+                                 out_dtype=torch.float32, step_states=True)
+    torch.cuda.synchronize()
+    ref = s0.astype(np.float64)
+    for step, tb in enumerate(toks):
+        ro, ref = oracle.decode_steps(ref, tb.q, tb.k, tb.v, tb.log_alpha, tb.beta)
+        if gate:
+            ro = oracle.gate_norm(ro, tb.g, w, 1e-6)
+        assert rel_l2(host(o[step]), ro) <= REL_L2_TOL, f"step {step} output"
+        assert rel_l2(host(states[step]), ref) <= REL_L2_TOL, f"step {step} state"
+    assert rel_l2(host(s_dev), ref) <= REL_L2_TOL
+    np.testing.assert_array_equal(host(s_dev), host(states[n - 1]))  # the carried state is the last step's
+
+
+def test_decode_multi_step_matches_single_steps_exactly():
+    """Carrying the state through 4 steps in registers gives the same bits as 4
+    separate one-step calls (same arithmetic, same order)."""
+    torch = _torch()
+    import linear_attention_recurrence_06_b200 as kda
+    Bd, H, n = 4, 2, 4
+    s0 = synth.states(8, Bd, H, D, D)
+    toks = [synth.tokens(8, step * Bd, Bd, H, D, D, bf16=True) for step in range(n)]
+    stack = lambda name: dev(np.stack([getattr(tb, name) for tb in toks]), torch.bfloat16)
+    q, k, v, la, b = (stack(x) for x in ("q", "k", "v", "log_alpha", "beta"))
+    s_multi = dev(s0, torch.float32)
+    o_multi = kda.decode_steps(s_multi, q, k, v, la, b, out_dtype=torch.float32)
+    s_single = dev(s0, torch.float32)
+    o_single = torch.stack([kda.decode_step(s_single, q[i], k[i], v[i], la[i], b[i], out_dtype=torch.float32)
+                            for i in range(n)])
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(host(o_multi), host(o_single))
+    np.testing.assert_array_equal(host(s_multi), host(s_single))
 
 
 # --------------------------------------------------------------- gate norm
