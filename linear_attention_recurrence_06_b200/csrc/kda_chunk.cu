@@ -63,6 +63,9 @@ constexpr int NSL = DV / DVS;
 //   GamC fp32 [128]                                                512 B
 //   Bm   bf16 [4 slices][128 key rows][32 value cols]            32768 B
 //   Ob   bf16 [4 slices][64 tokens][32 value cols]               16384 B
+// In Bm and Ob the four 16-byte pieces of each 64-byte row r are stored in the
+// order piece ^ ((r >> 1) & 3) (swz64), so that eight consecutive rows read or
+// written 16 bytes at a time touch eight different bank groups.
 constexpr size_t SO_M = 0, SO_Q = 32768, SO_G = 49152, SO_B = 49664, SO_O = 82432;
 constexpr size_t SLOT_BYTES = 98816;
 constexpr uint32_t SO_MQG = 49664;         // Mlr + Qp + GamC, one contiguous copy
@@ -148,6 +151,9 @@ KDA_DEV void mma_mn(uint32_t d, uint32_t a_addr, uint32_t b_addr, uint32_t idesc
         mma_bf16(d, ad0 + (uint32_t)((kk * 2 * A_KG) >> 4), bd0 + (uint32_t)((kk * 2 * B_KG) >> 4), idesc,
                  kk > 0 ? 1u : 0u);
 }
+
+// Position of 16-byte piece m of row r in a 64-byte-row slice (see the slot layout).
+KDA_DEV uint32_t swz64(uint32_t r, uint32_t m) { return m ^ ((r >> 1) & 3u); }
 
 KDA_DEV uint4 pack8(const float* x) {
     return make_uint4(pack_bf16x2(x[0], x[1]), pack_bf16x2(x[2], x[3]), pack_bf16x2(x[4], x[5]),
@@ -753,7 +759,7 @@ intra_kernel(const ChunkArgs a, const __grid_constant__ IntraMaps maps, const in
                     tmem_ld_wait();
                     uint4* dstB = reinterpret_cast<uint4*>(sm + Z2 + (size_t)(2 * hh + hp) * BSL + (size_t)c * DVS * 2);
 #pragma unroll
-                    for (int pp = 0; pp < 4; ++pp) dstB[pp] = pack8(d + 8 * pp);
+                    for (int pp = 0; pp < 4; ++pp) dstB[swz64(c, pp)] = pack8(d + 8 * pp);
                 }
                 if (q4 == 3) *reinterpret_cast<float*>(sm + IX + SO_G + 4 * c) = __expf(G[4]);  // Gam_C
             }
@@ -788,7 +794,7 @@ intra_kernel(const ChunkArgs a, const __grid_constant__ IntraMaps maps, const in
                 uint4* dstO = reinterpret_cast<uint4*>(sm + Z2 + (SO_O - SO_B) + (size_t)q4 * OSL +
                                                        (size_t)(16 * qd + lane) * (DVS * 2));
 #pragma unroll
-                for (int pp = 0; pp < 4; ++pp) dstO[pp] = pack8(ob + 8 * pp);
+                for (int pp = 0; pp < 4; ++pp) dstO[swz64(16 * qd + lane, pp)] = pack8(ob + 8 * pp);
             }
         }
         fence_async_smem();
@@ -1095,7 +1101,7 @@ chain_kernel(const ChunkArgs a, const __grid_constant__ CUtensorMap gate_map, co
                     const uint4* bsrc = reinterpret_cast<const uint4*>(buf + CB_B + (uint32_t)tid * DVS * 2);
 #pragma unroll
                     for (int m = 0; m < DVS / 8; ++m) {
-                        const uint4 w = bsrc[m];
+                        const uint4 w = bsrc[swz64(tid, m)];
                         const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
                         for (int p = 0; p < 4; ++p) {
@@ -1122,7 +1128,7 @@ chain_kernel(const ChunkArgs a, const __grid_constant__ CUtensorMap gate_map, co
                     const uint4* orow = reinterpret_cast<const uint4*>(buf + CB_O + (uint32_t)trow * (DVS * 2));
 #pragma unroll
                     for (int m = 0; m < DVS / 8; ++m) {
-                        const uint4 w = orow[m];
+                        const uint4 w = orow[swz64(trow, m)];
                         const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
                         for (int p = 0; p < 4; ++p) {
