@@ -302,6 +302,18 @@ intra_kernel(const ChunkArgs a, const __grid_constant__ IntraMaps maps, const in
             else beta_bits = __float_as_uint(__ldg(reinterpret_cast<const float*>(a.beta) + idx));
         }
     };
+    // the next item of this CTA after `from`, published in s_next by the last thread (it
+    // is looked up one item ahead, while that thread idles in the triangular inverse)
+    auto lookup_next = [&](int64_t from) {
+        const int64_t nx = next_valid(from);
+        int hh = 0, LL = 0;
+        int64_t tt = 0;
+        if (nx < n_items) item_info(a, nx, hh, tt, LL);
+        s_next64[0] = nx;
+        s_next64[1] = tt;
+        s_next32[0] = hh;
+        s_next32[1] = LL;
+    };
     if (item < n_items) {
         int hh, LL;
         int64_t tt;
@@ -312,6 +324,8 @@ intra_kernel(const ChunkArgs a, const __grid_constant__ IntraMaps maps, const in
             raw_in_flight = true;
         }
     }
+    if (tid == INTRA_THREADS - 1) lookup_next(item + gridDim.x);
+    __syncthreads();
 
     while (item < n_items) {
         int h, L;
@@ -323,16 +337,6 @@ intra_kernel(const ChunkArgs a, const __grid_constant__ IntraMaps maps, const in
         const size_t vbase = ((size_t)t0 * H + h) * DV + c;
 
         if (tid < CH) s_beta[tid] = IN_BF16 ? __uint_as_float(beta_bits << 16) : __uint_as_float(beta_bits);
-        if (tid == INTRA_THREADS - 1) {  // the next item of this CTA (read after the round-1 issue)
-            const int64_t nx = next_valid(item + gridDim.x);
-            int hh = 0, LL = 0;
-            int64_t tt = 0;
-            if (nx < n_items) item_info(a, nx, hh, tt, LL);
-            s_next64[0] = nx;
-            s_next64[1] = tt;
-            s_next32[0] = hh;
-            s_next32[1] = LL;
-        }
         if constexpr (IN_BF16) {
             mbar_wait(bar_raw, ph_raw, a.status);
             ph_raw ^= 1;
@@ -555,6 +559,9 @@ intra_kernel(const ChunkArgs a, const __grid_constant__ IntraMaps maps, const in
             const float* sA = reinterpret_cast<const float*>(sm + IY_A);
             float* sX = reinterpret_cast<float*>(sm + IY_X);
             float* sY = reinterpret_cast<float*>(sm + IX_TMP);  // partial products (8 KB)
+            // idle here: look up the item after the next one (every thread read s_next at the
+            // prefetch, before the extraction barrier)
+            if (tid == INTRA_THREADS - 1) lookup_next(next + gridDim.x);
             if (tid < 64) {  // diagonal blocks: one thread per (block, column)
                 // column j of (I + N_bb)^-1: x_i = -sum_{m<i} N_im x_m, x_j = 1, x_i = 0 for i < j
                 // (entries above j are zero, so the sums need no masking)
@@ -967,7 +974,7 @@ chain_kernel(const ChunkArgs a, const __grid_constant__ CUtensorMap gate_map, co
                     bulk_g2s(buf + CB_M, src + SO_M, SO_MQG, &bar_ld[b]);
                     bulk_g2s(buf + CB_B, src + SO_B + (size_t)js * BSL, BSL, &bar_ld[b]);
                     bulk_g2s(buf + CB_O, src + SO_O + (size_t)js * OSL, OSL, &bar_ld[b]);
-                    if constexpr (GATE)  // gate tile [64 tokens][32 value cols] of this slice
+                    if constexpr (GATE)  // gate tile [64 tokens][32 value cols] of this slice, 64-byte swizzled
                         tma_load_2d(buf + CB_GT, &gate_map, h * DV + DVS * js,
                                     (int)(s_beg + (int64_t)(c_beg + it) * CH), &bar_ld[b]);
                 };
@@ -1166,12 +1173,11 @@ chain_kernel(const ChunkArgs a, const __grid_constant__ CUtensorMap gate_map, co
                         ss += o_prev[j] * o_prev[j];
                     }
                     ss += __shfl_down_sync(0xFFFFFFFFu, ss, 16);  // lanes 0-15: the whole 32-column row
-                    {  // this chunk's gate columns of the lane's row, kept for the next iteration
-                        const uint4* gsrc =
-                            reinterpret_cast<const uint4*>(buf + CB_GT + (uint32_t)trow * DVS * 2) + 2 * hi;
+                    {  // this chunk's gate columns of the lane's row (64-byte swizzled tile), kept for later
+                        const uint4* gsrc = reinterpret_cast<const uint4*>(buf + CB_GT + (uint32_t)trow * DVS * 2);
 #pragma unroll
                         for (int m = 0; m < HC / 8; ++m) {
-                            const uint4 w = gsrc[m];
+                            const uint4 w = gsrc[swz64(trow, 2 * hi + m)];
                             g_prev[4 * m] = w.x; g_prev[4 * m + 1] = w.y; g_prev[4 * m + 2] = w.z; g_prev[4 * m + 3] = w.w;
                         }
                     }
@@ -1269,8 +1275,10 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
     return fn;
 }
 
-// [rows, row_elems] bf16 tensor, box = 64 rows x box_w elements, no swizzle.
-bool make_tile_map(CUtensorMap* m, const void* base, int64_t rows, int64_t row_elems, uint32_t box_w = 128) {
+// [rows, row_elems] bf16 tensor, box = 64 rows x box_w elements; no swizzle, or the
+// 64-byte pattern (16-byte piece m of row r stored at piece m ^ ((r >> 1) & 3), as swz64)
+bool make_tile_map(CUtensorMap* m, const void* base, int64_t rows, int64_t row_elems, uint32_t box_w = 128,
+                   bool swizzle64 = false) {
     auto enc = tensor_map_encoder();
     if (!enc) return false;
     cuuint64_t dims[2] = {(cuuint64_t)row_elems, (cuuint64_t)rows};
@@ -1278,7 +1286,8 @@ bool make_tile_map(CUtensorMap* m, const void* base, int64_t rows, int64_t row_e
     cuuint32_t box[2] = {box_w, 64};
     cuuint32_t estr[2] = {1, 1};
     return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
-               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_NONE,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -1353,7 +1362,7 @@ cudaError_t chunk_fwd_launch(const void* q, const void* k, const void* v, const 
     const bool fuse = gate != nullptr && in_bf16;
     CUtensorMap gate_map;
     memset(&gate_map, 0, sizeof(gate_map));
-    if (fuse && total_tokens > 0 && !make_tile_map(&gate_map, gate, total_tokens, (int64_t)H * DV, DVS))
+    if (fuse && total_tokens > 0 && !make_tile_map(&gate_map, gate, total_tokens, (int64_t)H * DV, DVS, true))
         return cudaErrorInvalidValue;
     if (gate_fused) *gate_fused = fuse;
 
