@@ -1073,7 +1073,7 @@ chain_kernel(const ChunkArgs a, const __grid_constant__ CUtensorMap gate_map, co
                             const int j = 8 * m + p;
                             const float gj =
                                 __uint_as_float((j & 1) ? (g_prev[j >> 1] & 0xFFFF0000u) : (g_prev[j >> 1] << 16));
-                            y8[p] = o_prev[j] * inv * w16[j] * __fdividef(1.0f, 1.0f + __expf(-gj));
+                            y8[p] = o_prev[j] * inv * w16[j] * sigmoid_fast(gj);
                         }
                         if constexpr (OUT_BF16) {
                             reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(a.o) + obase)[m] = pack8(y8);

@@ -168,6 +168,14 @@ KDA_DEV void cluster_sync_all() {
     asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
+// sigmoid(x) = 0.5 tanh(x / 2) + 0.5 with the hardware tanh approximation (one
+// special-function operation; relative error of tanh.approx about 2^-11).
+KDA_DEV float sigmoid_fast(float x) {
+    float t;
+    asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(0.5f * x));
+    return fmaf(0.5f, t, 0.5f);
+}
+
 // ---------------------------------------------------------------- tcgen05 --
 // TMEM allocation: one warp allocates `ncols` columns (power of 2, >= 32) and
 // the base address is written to *dst (shared memory).
