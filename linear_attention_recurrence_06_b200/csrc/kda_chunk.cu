@@ -834,10 +834,12 @@ intra_kernel(const ChunkArgs a, const __grid_constant__ IntraMaps maps, const in
 //   warps 0-3 (consumers): thread c owns state row c of the slice (32 fp32
 //     registers); applies S <- GamC o S - Mlr S + Bm, writes the next bf16
 //     state operand image, then forms the chunk output o = Qp S + Ob;
-//   warp 4 (producer, one thread): bulk loads of the chunk operands (three
-//     chunks ahead) and the tensor-core products Mlr S and Qp S.
-// The two sides meet only on mbarriers, so the issue of the next products
-// overlaps the output work of the current chunk.  TMEM (128 columns): D_S =
+//   warp 4 (one thread): the tensor-core products Mlr S and Qp S;
+//   warp 5 (one thread): bulk loads of the chunk operands, three chunks ahead,
+//     into buffers the consumers release as soon as they hold their Ob row
+//     and gate columns in registers.
+// The roles meet only on mbarriers, so the issue of the next products
+// overlaps the output work of the current chunk and never waits for a refill.  TMEM (128 columns): D_S =
 // Mlr S in [0,32) (M=128, lane = row c); D_O = Qp S double-buffered in [32,64)
 // and [64,96) (M=64: row t lives in lane 32*(t/16) + t%16).  Shared memory:
 // three chunk buffers {Mlr image 32K, Qp image 16K, GamC 512, Bm slice 8K, Ob
@@ -853,8 +855,9 @@ intra_kernel(const ChunkArgs a, const __grid_constant__ IntraMaps maps, const in
 //   bar_o[2]  commit of Qp S(i) into D_O[i & 1]; D_O[i & 1] is overwritten by
 //             chunk i + 2, issued after the image of i + 2, which consumers
 //             write after reading D_O(i).
-//   bar_ld[3] loads of a buffer; bar_free[3] consumers (128) -> producer: the
-//             buffer is no longer read and may be refilled.
+//   bar_ld[3] loads of a buffer; bar_free[3] consumers (128) -> loader: the
+//             buffer is no longer read (the products that read it completed:
+//             the consumer saw bar_o of its chunk first) and may be refilled.
 //
 // With the fused gate (GATE), the four CTAs of one (sequence, head) -- its four
 // value-column slices -- form a thread-block cluster.  The per-head RMSNorm
@@ -878,7 +881,7 @@ template <bool GATE> struct ChainLayout {
 };
 constexpr uint32_t CHAIN_TMEM_COLS = 128;
 constexpr uint32_t SB_KG = DVS * 16;  // state image K-group stride: 8 key rows x 32 columns x 2 B
-constexpr int CHAIN_THREADS = 160;  // 4 consumer warps + 1 producer warp
+constexpr int CHAIN_THREADS = 192;  // 4 consumer warps + 1 tensor-issue warp + 1 loader warp
 constexpr int CLUSTER = NSL;        // CTAs per (sequence, head) when the gate is fused
 constexpr uint32_t PART_TX = CLUSTER * 64 * 4;  // partial-sum bytes each CTA receives per chunk
 
@@ -960,11 +963,13 @@ chain_kernel(const ChunkArgs a, const __grid_constant__ CUtensorMap gate_map, co
         auto bidx = [](int it) { return it % NBUF; };
         auto bpar = [](int it) { return (uint32_t)((it / NBUF) & 1); };
         bool failed = false;
-        // producer bookkeeping for the bounded drain after a failed wait
-        int loads_issued = 0, loads_waited = 0, mma_issued = 0;
+        // loader / issuer bookkeeping for the bounded drain
+        int loads_issued = 0, mma_issued = 0;
 
-        if (!consumer) {
-            // ------------------------------------------------------ producer
+        if (warp == 5) {
+            // -------------------------------------------------------- loader
+            // (its own warp, so that waiting for a buffer to be released never holds up the
+            // tensor-core issue)
             if (lane == 0) {
                 auto issue_load = [&](int it) {
                     const int b = bidx(it);
@@ -982,6 +987,19 @@ chain_kernel(const ChunkArgs a, const __grid_constant__ CUtensorMap gate_map, co
                     issue_load(j);
                     loads_issued = j + 1;
                 }
+                // chunk r = j + NBUF goes into the buffer of chunk j once the consumers released it
+                for (int j = 0; j + NBUF < nit; ++j) {
+                    if (!mbar_wait(&bar_free[bidx(j)], bpar(j), a.status)) {
+                        failed = true;
+                        break;
+                    }
+                    issue_load(j + NBUF);
+                    loads_issued = j + NBUF + 1;
+                }
+            }
+        } else if (warp == 4) {
+            // -------------------------------------------------- tensor issue
+            if (lane == 0) {
                 for (int it = 0; it < nit; ++it) {
                     const int b = bidx(it);
                     if (!mbar_wait(bar_img, (uint32_t)(it & 1), a.status) ||
@@ -989,7 +1007,6 @@ chain_kernel(const ChunkArgs a, const __grid_constant__ CUtensorMap gate_map, co
                         failed = true;
                         break;
                     }
-                    loads_waited = it + 1;
                     tc_fence_after();
                     // Mlr S -> D_S, then Qp S -> D_O[it & 1]
                     // state image: MN-major, K-group (8 key rows) stride SB_KG, 8-column block stride 128
@@ -1013,16 +1030,6 @@ chain_kernel(const ChunkArgs a, const __grid_constant__ CUtensorMap gate_map, co
                     }
                     mma_commit(&bar_o[it & 1]);
                     mma_issued = it + 1;
-                    // refill the buffer of the previous chunk once the consumers released it
-                    const int r = it - 1 + NBUF;
-                    if (it >= 1 && r < nit) {
-                        if (!mbar_wait(&bar_free[bidx(it - 1)], bpar(it - 1), a.status)) {
-                            failed = true;
-                            break;
-                        }
-                        issue_load(r);
-                        loads_issued = r + 1;
-                    }
                 }
             }
         } else {
@@ -1144,6 +1151,16 @@ chain_kernel(const ChunkArgs a, const __grid_constant__ CUtensorMap gate_map, co
                         }
                     }
                 }
+                uint32_t g_cur[GATE ? HC / 2 : 1];
+                if constexpr (GATE) {  // this chunk's gate columns of the lane's row (64-byte swizzled tile)
+                    const uint4* gsrc = reinterpret_cast<const uint4*>(buf + CB_GT + (uint32_t)trow * DVS * 2);
+#pragma unroll
+                    for (int m = 0; m < HC / 8; ++m) {
+                        const uint4 w = gsrc[swz64(trow, 2 * hi + m)];
+                        g_cur[4 * m] = w.x; g_cur[4 * m + 1] = w.y; g_cur[4 * m + 2] = w.z; g_cur[4 * m + 3] = w.w;
+                    }
+                }
+                mbar_arrive(&bar_free[b]);  // everything this thread reads from the buffer is in registers
                 if constexpr (!GATE) {
                     if (lane < 16 && trow < L) {
                         const size_t obase = ((size_t)(t0 + trow) * H + h) * DV + (size_t)DVS * js;
@@ -1173,14 +1190,8 @@ chain_kernel(const ChunkArgs a, const __grid_constant__ CUtensorMap gate_map, co
                         ss += o_prev[j] * o_prev[j];
                     }
                     ss += __shfl_down_sync(0xFFFFFFFFu, ss, 16);  // lanes 0-15: the whole 32-column row
-                    {  // this chunk's gate columns of the lane's row (64-byte swizzled tile), kept for later
-                        const uint4* gsrc = reinterpret_cast<const uint4*>(buf + CB_GT + (uint32_t)trow * DVS * 2);
 #pragma unroll
-                        for (int m = 0; m < HC / 8; ++m) {
-                            const uint4 w = gsrc[swz64(trow, 2 * hi + m)];
-                            g_prev[4 * m] = w.x; g_prev[4 * m + 1] = w.y; g_prev[4 * m + 2] = w.z; g_prev[4 * m + 3] = w.w;
-                        }
-                    }
+                    for (int m = 0; m < HC / 2; ++m) g_prev[m] = g_cur[m];  // kept for the next iteration
                     if (lane < 16) {
                         const uint32_t slot = smem_u32(s_part + (it & 1) * (CLUSTER * 64) + js * 64 + trow);
                         const uint32_t barl = smem_u32(&bar_part[it & 1]);
@@ -1204,24 +1215,26 @@ chain_kernel(const ChunkArgs a, const __grid_constant__ CUtensorMap gate_map, co
                             __stcs(reinterpret_cast<float4*>(dst + c4), make_float4(S[c4], S[c4 + 1], S[c4 + 2], S[c4 + 3]));
                     }
                 }
-                // (4) this chunk's buffer and D_O[it & 1] are no longer read
+                // (4) D_O[it & 1] is no longer read
                 tc_fence_before();
-                mbar_arrive(&bar_free[b]);
             }
             if constexpr (GATE) {
                 if (!failed && !finish_prev(nit - 1)) failed = true;
             }
         }
 
-        // after a failed wait: let copies and products still in flight finish (bounded)
+        // copies and products still in flight finish before the CTA retires (bounded; in a
+        // normal run every one of them has been consumed and the waits return at once):
+        // the loader's last load into each buffer, the issuer's last pair of products
         __syncthreads();
-        if (!consumer && lane == 0 && (failed || loads_waited < loads_issued)) {
-            for (int j = loads_waited; j < loads_issued; ++j) mbar_wait(&bar_ld[bidx(j)], bpar(j), nullptr);
-            if (mma_issued > 0) {
-                const int j = mma_issued - 1;
-                mbar_wait(bar_s, (uint32_t)(j & 1), nullptr);
-                mbar_wait(&bar_o[j & 1], (uint32_t)((j >> 1) & 1), nullptr);
-            }
+        if (warp == 5 && lane == 0) {
+            for (int j = loads_issued - NBUF < 0 ? 0 : loads_issued - NBUF; j < loads_issued; ++j)
+                mbar_wait(&bar_ld[bidx(j)], bpar(j), nullptr);
+        }
+        if (warp == 4 && lane == 0 && failed && mma_issued > 0) {
+            const int j = mma_issued - 1;
+            mbar_wait(bar_s, (uint32_t)(j & 1), nullptr);
+            mbar_wait(&bar_o[j & 1], (uint32_t)((j >> 1) & 1), nullptr);
         }
         tc_fence_before();
         __syncthreads();
