@@ -177,8 +177,9 @@ KDA_DEV uint4 pack8(const float* x) {
 //                    later Wt [128][64] @0, Ut [128][64] @16K
 //   Z2  [171K, 219K) KGt, Vt, Ktt [128][64] (built while round 1 runs)
 //   misc             beta[64], G[5][128], tile totals[4][128], 2 mbarriers, TMEM base
-// The workspace slot leaves at the end of an item as two bulk copies: [Mlr | Qp | GamC]
-// assembled at X, [Bm | Ob] at Z2.
+// The workspace slot is assembled in two regions ([Mlr | Qp | GamC] at X, [Bm | Ob]
+// at Z2) and leaves as four bulk copies: Mlr and Bm as soon as they are staged, the
+// rest at the end of the item.
 // TMEM (512 columns): round 1  A/P diag [0,64), off-diag [64,80) [80,112) [112,160)
 //                     round 2  Wt [160,224), Ut [224,288)
 //                     round 3  [Mlr | Bm] [0,256) (one N = 256 product), (PW)^T [256,320),
@@ -771,6 +772,15 @@ intra_kernel(const ChunkArgs a, const __grid_constant__ IntraMaps maps, const in
                 if (q4 == 3) *reinterpret_cast<float*>(sm + IX + SO_G + 4 * c) = __expf(G[4]);  // Gam_C
             }
         }
+        // Mlr and Bm leave now, so that the bulk-copy engine is free earlier for the next
+        // item's tile loads; Qp, GamC and Ob follow at the end of the item
+        fence_async_smem();
+        __syncthreads();
+        if (tid == 0) {
+            bulk_s2g(wslot + SO_M, sm + IX + SO_M, (uint32_t)(SO_Q - SO_M));
+            bulk_s2g(wslot + SO_B, sm + Z2, (uint32_t)(SO_O - SO_B));
+            bulk_commit();
+        }
         mbar_wait(bar_mma2, ph_mma2, a.status);
         ph_mma2 ^= 1;
         tc_fence_after();
@@ -809,8 +819,8 @@ intra_kernel(const ChunkArgs a, const __grid_constant__ IntraMaps maps, const in
         __syncthreads();
         tc_fence_after();
         if (tid == 0) {
-            bulk_s2g(wslot, sm + IX, SO_MQG);
-            bulk_s2g(wslot + SO_B, sm + Z2, (uint32_t)(SLOT_BYTES - SO_B));
+            bulk_s2g(wslot + SO_Q, sm + IX + SO_Q, (uint32_t)(SO_MQG - SO_Q));  // Qp + GamC
+            bulk_s2g(wslot + SO_O, sm + Z2 + (SO_O - SO_B), (uint32_t)(SLOT_BYTES - SO_O));
             bulk_commit();
         }
         item = next;
