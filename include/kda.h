@@ -155,6 +155,40 @@ KDA_API kda_status kda_chunk_fwd_ckpt(const void* q, const void* k, const void* 
                               void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * kda_chunk_fwd_segmented -- kda_chunk_fwd with every sequence cut into
+ * `segments` segments of whole chunks that are walked in parallel: the
+ * segment-parallel (associative scan) form of the prefill ("training and
+ * inference systems" item of the K3 article summaries: context parallelism as a
+ * prefix scan of segment transitions; the nlpx.cn walkthrough, §6: KCP).
+ * Pass 1 computes, per (sequence, segment, head), the segment's affine state
+ * map S -> M S + B; pass 2 walks each segment from the initial state folded
+ * through the maps of the segments before it.  Useful when n_seqs * H is small
+ * next to the GPU (the plain walk has 4 * n_seqs * H independent chains).
+ * Arguments as kda_chunk_fwd plus `segments` (>= 1; 1 is kda_chunk_fwd); the
+ * workspace must hold kda_chunk_fwd_segmented_workspace_size bytes (every chunk
+ * at once plus the segment maps).  Results equal kda_chunk_fwd's up to bf16
+ * rounding of the segment maps.
+ */
+KDA_API kda_status kda_chunk_fwd_segmented(const void* q, const void* k, const void* v,
+                                   const void* log_alpha, const void* beta,
+                                   const float* init_state, void* o, float* final_state,
+                                   int B, int64_t T, int H, int dk, int dv,
+                                   const int32_t* cu_seqlens, int n_seqs, int64_t max_seqlen,
+                                   kda_dtype in_dtype, kda_dtype out_dtype, float scale,
+                                   const void* gate, const float* norm_weight, float eps,
+                                   int segments, void* workspace, size_t workspace_bytes,
+                                   void* stream);
+
+/*
+ * kda_chunk_fwd_segmented_workspace_size -- workspace bytes for
+ * kda_chunk_fwd_segmented (arguments as kda_chunk_fwd_workspace_size plus
+ * segments).
+ */
+KDA_API kda_status kda_chunk_fwd_segmented_workspace_size(int64_t T, int H, int dk, int dv, int n_seqs,
+                                                  int64_t max_seqlen, int segments,
+                                                  size_t* bytes);
+
+/*
  * kda_decode_step -- one recurrent step for Bd independent sequences
  * ("decode uses the recurrent form", chunkwise-algorithm item of the K3
  * article summaries).  The state is read once and written once, in place.

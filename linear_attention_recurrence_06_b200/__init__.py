@@ -67,6 +67,11 @@ def load_library(path: str | None = None):
     lib.kda_chunk_fwd_ckpt.restype = i32
     lib.kda_chunk_fwd_ckpt.argtypes = list(lib.kda_chunk_fwd.argtypes[:22]) + [vp, i64] + \
         list(lib.kda_chunk_fwd.argtypes[22:])
+    lib.kda_chunk_fwd_segmented.restype = i32
+    lib.kda_chunk_fwd_segmented.argtypes = list(lib.kda_chunk_fwd.argtypes[:22]) + [i32] + \
+        list(lib.kda_chunk_fwd.argtypes[22:])
+    lib.kda_chunk_fwd_segmented_workspace_size.restype = i32
+    lib.kda_chunk_fwd_segmented_workspace_size.argtypes = [i64, i32, i32, i32, i32, i64, i32, ctypes.POINTER(sz)]
     lib.kda_decode_step.restype = i32
     lib.kda_decode_step.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, f32, vp, vp, f32, vp]
     lib.kda_decode_steps.restype = i32
@@ -118,6 +123,17 @@ def _check_cuda(*ts):
                 raise ValueError("all tensors must be contiguous")
 
 
+def segmented_workspace_size(T: int, H: int, n_seqs: int, max_seqlen: int, segments: int, dk: int = HEAD_DIM,
+                             dv: int = HEAD_DIM) -> int:
+    """Workspace bytes of the segment-parallel prefill."""
+    n = ctypes.c_size_t(0)
+    st = load_library().kda_chunk_fwd_segmented_workspace_size(T, H, dk, dv, n_seqs, max_seqlen, segments,
+                                                               ctypes.byref(n))
+    if st != KDA_OK:
+        raise KdaError(st, "kda_chunk_fwd_segmented_workspace_size")
+    return n.value
+
+
 def workspace_size(T: int, H: int, n_seqs: int, max_seqlen: int, dk: int = HEAD_DIM, dv: int = HEAD_DIM):
     """(bytes_min, bytes_full) of the prefill workspace."""
     lo, hi = ctypes.c_size_t(0), ctypes.c_size_t(0)
@@ -130,7 +146,7 @@ def workspace_size(T: int, H: int, n_seqs: int, max_seqlen: int, dk: int = HEAD_
 def chunk_fwd(q, k, v, log_alpha, beta, initial_state=None, *, cu_seqlens=None, max_seqlen=None,
               scale: float = 1.0, gate=None, norm_weight=None, eps: float = 1e-6, out_dtype=None,
               output_final_state: bool = True, final_state=None, out=None, workspace=None, stream=None,
-              checkpoints=None, ckpt_tokens: int = 512):
+              checkpoints=None, ckpt_tokens: int = 512, segments: int = 1):
     """Chunkwise KDA prefill.
 
     q, k, log_alpha: [B, T, H, 128]; v: [B, T, H, 128]; beta: [B, T, H] (bf16 or
@@ -141,6 +157,8 @@ def chunk_fwd(q, k, v, log_alpha, beta, initial_state=None, *, cu_seqlens=None, 
     checkpoints: None, True (allocate zeros) or fp32 [N, max_seqlen // ckpt_tokens, H, 128, 128]
     receiving the state after every ckpt_tokens tokens of each sequence (ckpt_tokens a
     multiple of 64); then the return value is (o, final_state, checkpoints).
+    segments > 1: segment-parallel prefill (kda_chunk_fwd_segmented); not combined
+    with checkpoints.
     """
     torch = _torch()
     _check_cuda(q, k, v, log_alpha, beta, initial_state, cu_seqlens, gate, norm_weight)
@@ -165,12 +183,22 @@ def chunk_fwd(q, k, v, log_alpha, beta, initial_state=None, *, cu_seqlens=None, 
     if fs is None and output_final_state:
         fs = torch.empty((N, H, dk, dv), dtype=torch.float32, device=q.device)
     if workspace is None:
-        _, full = workspace_size(B * T if cu_seqlens is None else T, H, N, max_seqlen, dk, dv)
+        if segments > 1:
+            full = segmented_workspace_size(B * T if cu_seqlens is None else T, H, N, max_seqlen, segments, dk, dv)
+        else:
+            _, full = workspace_size(B * T if cu_seqlens is None else T, H, N, max_seqlen, dk, dv)
         workspace = torch.empty(full, dtype=torch.uint8, device=q.device)
     args = (_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(initial_state), _ptr(o), _ptr(fs),
             B, T, H, dk, dv, _ptr(cu_seqlens), N, int(max_seqlen), in_dt, _dt(o), float(scale), _ptr(gate),
             _ptr(norm_weight), float(eps))
     tail = (_ptr(workspace), workspace.numel(), _stream(stream))
+    if segments > 1:
+        if checkpoints is not None:
+            raise ValueError("segments > 1 does not take checkpoints")
+        st = load_library().kda_chunk_fwd_segmented(*args, int(segments), *tail)
+        if st != KDA_OK:
+            raise KdaError(st, "kda_chunk_fwd_segmented")
+        return o, fs
     if checkpoints is None:
         st = load_library().kda_chunk_fwd(*args, *tail)
         if st != KDA_OK:

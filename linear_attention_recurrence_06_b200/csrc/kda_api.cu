@@ -20,12 +20,13 @@ cudaError_t launch_gate_norm(const void* o, const void* g, const float* norm_w, 
                              bool o_bf16, bool g_bf16, bool out_bf16, int num_sms, cudaStream_t stream);
 size_t chunk_slot_bytes();
 size_t chunk_fixed_bytes(int n_seqs, int H, bool need_carry);
+size_t chunk_seg_bytes(int n_seqs, int H, int segs);
 cudaError_t chunk_fwd_launch(const void* q, const void* k, const void* v, const void* log_alpha, const void* beta,
                              const float* init_state, void* o, float* final_state, int B, int64_t T, int H,
                              const int32_t* cu, int n_seqs, int64_t max_seqlen, bool in_bf16, bool out_bf16,
                              float scale, const void* gate, const float* norm_w, float eps, float* ckpt,
-                             int64_t ckpt_tokens, void* workspace, size_t ws_bytes, cudaStream_t stream, int* n_passes,
-                             bool* gate_fused);
+                             int64_t ckpt_tokens, int segs, void* workspace, size_t ws_bytes, cudaStream_t stream,
+                             int* n_passes, bool* gate_fused);
 }  // namespace kda
 
 namespace kda {
@@ -128,12 +129,23 @@ kda_status kda_chunk_fwd_workspace_size(int64_t T, int H, int dk, int dv, int n_
     return KDA_OK;
 }
 
-kda_status kda_chunk_fwd_ckpt(const void* q, const void* k, const void* v, const void* log_alpha, const void* beta,
-                              const float* init_state, void* o, float* final_state, int B, int64_t T, int H, int dk,
-                              int dv, const int32_t* cu_seqlens, int n_seqs, int64_t max_seqlen, kda_dtype in_dtype,
-                              kda_dtype out_dtype, float scale, const void* gate, const float* norm_weight, float eps,
-                              float* checkpoints, int64_t ckpt_tokens, void* workspace, size_t workspace_bytes,
-                              void* stream) {
+kda_status kda_chunk_fwd_segmented_workspace_size(int64_t T, int H, int dk, int dv, int n_seqs, int64_t max_seqlen,
+                                                  int segments, size_t* bytes) {
+    if (segments < 1 || !bytes) return KDA_ERR_INVALID_ARG;
+    size_t full = 0;
+    const kda_status st = kda_chunk_fwd_workspace_size(T, H, dk, dv, n_seqs, max_seqlen, nullptr, &full);
+    if (st != KDA_OK) return st;
+    *bytes = full + (segments > 1 ? kda::chunk_seg_bytes(n_seqs, H, segments) : 0);
+    return KDA_OK;
+}
+
+static kda_status chunk_fwd_impl(const void* q, const void* k, const void* v, const void* log_alpha,
+                                 const void* beta, const float* init_state, void* o, float* final_state, int B,
+                                 int64_t T, int H, int dk, int dv, const int32_t* cu_seqlens, int n_seqs,
+                                 int64_t max_seqlen, kda_dtype in_dtype, kda_dtype out_dtype, float scale,
+                                 const void* gate, const float* norm_weight, float eps, float* checkpoints,
+                                 int64_t ckpt_tokens, int segments, void* workspace, size_t workspace_bytes,
+                                 void* stream) {
     if (!q || !k || !v || !log_alpha || !beta || !o) return KDA_ERR_INVALID_ARG;
     if (B <= 0 || T < 0 || H <= 0 || !dtype_ok(in_dtype) || !dtype_ok(out_dtype)) return KDA_ERR_INVALID_ARG;
     if (dk != kSupportedD || dv != kSupportedD) return KDA_ERR_UNSUPPORTED;
@@ -147,6 +159,7 @@ kda_status kda_chunk_fwd_ckpt(const void* q, const void* k, const void* v, const
     if ((int64_t)B * T * H * 128 / 128 != (int64_t)B * T * H) return KDA_ERR_INVALID_ARG;
     if (eps < 0.f) return KDA_ERR_INVALID_ARG;
     if (checkpoints && (ckpt_tokens <= 0 || ckpt_tokens % 64 != 0)) return KDA_ERR_INVALID_ARG;
+    if (segments < 1) return KDA_ERR_INVALID_ARG;
     const void* ptrs[] = {q, k, v, log_alpha, beta, init_state, o, final_state, cu_seqlens, gate, norm_weight, workspace,
                           checkpoints};
     for (const void* p : ptrs)
@@ -154,9 +167,12 @@ kda_status kda_chunk_fwd_ckpt(const void* q, const void* k, const void* v, const
     if (!workspace) return KDA_ERR_WORKSPACE;
     if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return KDA_ERR_MISALIGNED;
     size_t need_min = 0;
-    if (kda_chunk_fwd_workspace_size(T * (cu_seqlens ? 1 : B), H, dk, dv, n_seqs, max_seqlen, &need_min, nullptr) !=
-        KDA_OK)
-        return KDA_ERR_INVALID_ARG;
+    const kda_status wst =
+        segments > 1 ? kda_chunk_fwd_segmented_workspace_size(T * (cu_seqlens ? 1 : B), H, dk, dv, n_seqs, max_seqlen,
+                                                               segments, &need_min)
+                     : kda_chunk_fwd_workspace_size(T * (cu_seqlens ? 1 : B), H, dk, dv, n_seqs, max_seqlen,
+                                                    &need_min, nullptr);
+    if (wst != KDA_OK) return KDA_ERR_INVALID_ARG;
     if (workspace_bytes < need_min) return KDA_ERR_WORKSPACE;
 
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
@@ -164,7 +180,8 @@ kda_status kda_chunk_fwd_ckpt(const void* q, const void* k, const void* v, const
     bool fused = false;
     cudaError_t e = kda::chunk_fwd_launch(q, k, v, log_alpha, beta, init_state, o, final_state, B, T, H, cu_seqlens,
                                           n_seqs, max_seqlen, in_bf16, out_bf16, scale, gate, norm_weight, eps,
-                                          checkpoints, ckpt_tokens, workspace, workspace_bytes, st, nullptr, &fused);
+                                          checkpoints, ckpt_tokens, segments, workspace, workspace_bytes, st, nullptr,
+                                          &fused);
     if (e != cudaSuccess) return KDA_ERR_CUDA;
     if (gate && !fused) {
         const int64_t rows = (int64_t)B * T * H;
@@ -176,6 +193,28 @@ kda_status kda_chunk_fwd_ckpt(const void* q, const void* k, const void* v, const
         if (e != cudaSuccess) return KDA_ERR_CUDA;
     }
     return KDA_OK;
+}
+
+kda_status kda_chunk_fwd_ckpt(const void* q, const void* k, const void* v, const void* log_alpha, const void* beta,
+                              const float* init_state, void* o, float* final_state, int B, int64_t T, int H, int dk,
+                              int dv, const int32_t* cu_seqlens, int n_seqs, int64_t max_seqlen, kda_dtype in_dtype,
+                              kda_dtype out_dtype, float scale, const void* gate, const float* norm_weight, float eps,
+                              float* checkpoints, int64_t ckpt_tokens, void* workspace, size_t workspace_bytes,
+                              void* stream) {
+    return chunk_fwd_impl(q, k, v, log_alpha, beta, init_state, o, final_state, B, T, H, dk, dv, cu_seqlens, n_seqs,
+                          max_seqlen, in_dtype, out_dtype, scale, gate, norm_weight, eps, checkpoints, ckpt_tokens, 1,
+                          workspace, workspace_bytes, stream);
+}
+
+kda_status kda_chunk_fwd_segmented(const void* q, const void* k, const void* v, const void* log_alpha,
+                                   const void* beta, const float* init_state, void* o, float* final_state, int B,
+                                   int64_t T, int H, int dk, int dv, const int32_t* cu_seqlens, int n_seqs,
+                                   int64_t max_seqlen, kda_dtype in_dtype, kda_dtype out_dtype, float scale,
+                                   const void* gate, const float* norm_weight, float eps, int segments,
+                                   void* workspace, size_t workspace_bytes, void* stream) {
+    return chunk_fwd_impl(q, k, v, log_alpha, beta, init_state, o, final_state, B, T, H, dk, dv, cu_seqlens, n_seqs,
+                          max_seqlen, in_dtype, out_dtype, scale, gate, norm_weight, eps, nullptr, 0, segments,
+                          workspace, workspace_bytes, stream);
 }
 
 kda_status kda_chunk_fwd(const void* q, const void* k, const void* v, const void* log_alpha, const void* beta,

@@ -94,6 +94,8 @@ struct ChunkArgs {
     float* ckpt;               // nullable: states at every ckpt_every-th chunk boundary
     int ckpt_every;            // in chunks
     int n_ckpt;                // checkpoints per sequence in `ckpt`
+    int segs;                  // segments per sequence (segment-parallel prefill), else 1
+    uint8_t* seg_ws;           // segment transition slots [n_seqs][segs][H], segment-parallel only
 };
 
 // Token range [sb, se) of sequence n, clamped into [0, total tokens].
@@ -895,7 +897,16 @@ constexpr int CHAIN_THREADS = 192;  // 4 consumer warps + 1 tensor-issue warp + 
 constexpr int CLUSTER = NSL;        // CTAs per (sequence, head) when the gate is fused
 constexpr uint32_t PART_TX = CLUSTER * 64 * 4;  // partial-sum bytes each CTA receives per chunk
 
-template <bool OUT_BF16, bool GATE>
+// SEG = 0: the plain walk over this pass's chunks.  Segment-parallel prefill (each
+// sequence cut into a.segs segments of whole chunks, blockIdx.z = n * segs + g):
+// SEG = 1: per segment, the affine map S -> M_g S + B_g of its chunks; slices 0-3
+//   carry B_g (state from zero), slices 4-7 carry M_g (state from the identity,
+//   Bm dropped); the result is written as a segment slot in the chunk-slot format
+//   (Mlr = -M_g, GamC = 0, Bm = B_g), no outputs;
+// SEG = 2: segment g first folds segments 0 .. g-1 into the initial state through
+//   their slots, then walks its own chunks with outputs; the last segment writes
+//   the final state.
+template <bool OUT_BF16, bool GATE, int SEG>
 __global__ void __launch_bounds__(CHAIN_THREADS, 1)
 chain_kernel(const ChunkArgs a, const __grid_constant__ CUtensorMap gate_map, const float* __restrict__ norm_w,
              float eps) {
@@ -906,8 +917,12 @@ chain_kernel(const ChunkArgs a, const __grid_constant__ CUtensorMap gate_map, co
     const uint32_t sbase = smem_u32(sm);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const bool consumer = warp < 4;
-    const int js = blockIdx.x, h = blockIdx.y, n = blockIdx.z;
+    const int js = blockIdx.x, h = blockIdx.y;
+    const int n = SEG ? (int)blockIdx.z / a.segs : (int)blockIdx.z;
+    const int g = SEG ? (int)blockIdx.z % a.segs : 0;
     const int H = a.H;
+    const int jb = js & (NSL - 1);                // value slice of Bm / outputs
+    const bool trans = SEG == 1 && js >= NSL;     // carries M_g (identity start, no Bm)
     uint64_t* bar_ld = reinterpret_cast<uint64_t*>(sm + LY::BAR);         // [NBUF]
     uint64_t* bar_free = reinterpret_cast<uint64_t*>(sm + LY::BAR + 24);  // [NBUF]
     uint64_t* bar_s = reinterpret_cast<uint64_t*>(sm + LY::BAR + 48);
@@ -920,16 +935,29 @@ chain_kernel(const ChunkArgs a, const __grid_constant__ CUtensorMap gate_map, co
     int64_t s_beg, s_end;
     seq_range(a, n, s_beg, s_end);
     const int nchunks = (int)((s_end - s_beg + CH - 1) / CH);
-    const int c_beg = a.i0;
-    const int c_end = min(a.i0 + a.wc, nchunks);
-    const int nit = c_end > c_beg ? c_end - c_beg : 0;  // the same for the whole cluster
+    // chunk iterations [c_beg, c_end); with SEG = 2 preceded by nseg segment iterations
+    int c_beg, c_end;
+    if constexpr (SEG == 0) {
+        c_beg = a.i0;
+        c_end = min(a.i0 + a.wc, nchunks);
+    } else {
+        const int per = (nchunks + a.segs - 1) / a.segs;
+        c_beg = min(g * per, nchunks);
+        c_end = min(c_beg + per, nchunks);
+    }
+    const int nseg = SEG == 2 ? g : 0;
+    const int nck = c_end > c_beg ? c_end - c_beg : 0;
+    const int nit = nseg + nck;  // the same for the whole cluster
 
-    // state slice: row tid, columns [32 js, 32 js + 32)
-    const size_t st_off = (((size_t)n * H + h) * DK + (consumer ? tid : 0)) * DV + (size_t)DVS * js;
+    // state slice: row tid, columns [32 jb, 32 jb + 32)
+    const size_t st_off = (((size_t)n * H + h) * DK + (consumer ? tid : 0)) * DV + (size_t)DVS * jb;
     float S[DVS];
     if (consumer) {
-        const float* src = a.first_pass ? a.init_state : a.state_io;
-        if (src) {
+        const float* src = SEG == 1 ? nullptr : (a.first_pass ? a.init_state : a.state_io);
+        if (trans) {
+#pragma unroll
+            for (int j = 0; j < DVS; ++j) S[j] = (tid == DVS * jb + j) ? 1.f : 0.f;
+        } else if (src) {
 #pragma unroll
             for (int j = 0; j < DVS; j += 4) {
                 const float4 v4 = *reinterpret_cast<const float4*>(src + st_off + j);
@@ -968,7 +996,14 @@ chain_kernel(const ChunkArgs a, const __grid_constant__ CUtensorMap gate_map, co
         if constexpr (GATE) cluster_sync_all();  // peers' barriers exist before any remote store
         tc_fence_after();
         const uint32_t tm = *s_tmem;
-        const size_t slot0 = ((size_t)n * a.wc + (c_beg - a.i0)) * H + h;  // slot of iteration 0
+        const size_t slot0 = ((size_t)n * a.wc + (c_beg - a.i0)) * H + h;  // slot of the first chunk iteration
+        // iteration it: a segment iteration (it < nseg) or chunk c_beg + it - nseg;
+        // only chunk iterations of SEG != 1 form outputs (output index oi = it - nseg)
+        auto slot_of = [&](int it) -> const uint8_t* {
+            if (SEG == 2 && it < nseg) return a.seg_ws + (((size_t)n * a.segs + it) * H + h) * SLOT_BYTES;
+            return a.ws + (slot0 + (size_t)(it - nseg) * H) * SLOT_BYTES;
+        };
+        auto has_out = [&](int it) { return SEG != 1 && it >= nseg; };
         // chunk buffer of iteration it and its barrier phase
         auto bidx = [](int it) { return it % NBUF; };
         auto bpar = [](int it) { return (uint32_t)((it / NBUF) & 1); };
@@ -984,14 +1019,17 @@ chain_kernel(const ChunkArgs a, const __grid_constant__ CUtensorMap gate_map, co
                 auto issue_load = [&](int it) {
                     const int b = bidx(it);
                     uint8_t* buf = sm + b * CB_SIZE;
-                    const uint8_t* src = a.ws + (slot0 + (size_t)it * H) * SLOT_BYTES;
-                    mbar_arrive_expect_tx(&bar_ld[b], SO_MQG + BSL + OSL + (GATE ? (uint32_t)(CH * DVS * 2) : 0u));
+                    const uint8_t* src = slot_of(it);
+                    const bool out = has_out(it);
+                    mbar_arrive_expect_tx(&bar_ld[b], SO_MQG + BSL + (out ? OSL + (GATE ? (uint32_t)(CH * DVS * 2) : 0u) : 0u));
                     bulk_g2s(buf + CB_M, src + SO_M, SO_MQG, &bar_ld[b]);
-                    bulk_g2s(buf + CB_B, src + SO_B + (size_t)js * BSL, BSL, &bar_ld[b]);
-                    bulk_g2s(buf + CB_O, src + SO_O + (size_t)js * OSL, OSL, &bar_ld[b]);
-                    if constexpr (GATE)  // gate tile [64 tokens][32 value cols] of this slice, 64-byte swizzled
-                        tma_load_2d(buf + CB_GT, &gate_map, h * DV + DVS * js,
-                                    (int)(s_beg + (int64_t)(c_beg + it) * CH), &bar_ld[b]);
+                    bulk_g2s(buf + CB_B, src + SO_B + (size_t)jb * BSL, BSL, &bar_ld[b]);
+                    if (out) {
+                        bulk_g2s(buf + CB_O, src + SO_O + (size_t)jb * OSL, OSL, &bar_ld[b]);
+                        if constexpr (GATE)  // gate tile [64 tokens][32 value cols] of this slice, 64-byte swizzled
+                            tma_load_2d(buf + CB_GT, &gate_map, h * DV + DVS * jb,
+                                        (int)(s_beg + (int64_t)(c_beg + it - nseg) * CH), &bar_ld[b]);
+                    }
                 };
                 for (int j = 0; j < NBUF && j < nit; ++j) {
                     issue_load(j);
@@ -1030,15 +1068,16 @@ chain_kernel(const ChunkArgs a, const __grid_constant__ CUtensorMap gate_map, co
                                      kk > 0 ? 1u : 0u);
                     }
                     mma_commit(bar_s);
-                    {  // Qp (MN-major, no swizzle) x state image
+                    if (has_out(it)) {  // Qp (MN-major, no swizzle) x state image -> D_O[oi & 1]
+                        const int oi = it - nseg;
                         const uint64_t qdesc = sdesc_interleave(sbase + b * CB_SIZE + CB_Q, 1024u, 128u);
 #pragma unroll
                         for (int kk = 0; kk < DK / 16; ++kk)
-                            mma_bf16(tm + 32 + 32 * (it & 1), qdesc + (uint32_t)((kk * 2048) >> 4),
+                            mma_bf16(tm + 32 + 32 * (oi & 1), qdesc + (uint32_t)((kk * 2048) >> 4),
                                      sdesc + (uint32_t)((kk * 2 * SB_KG) >> 4), idesc_bf16_major(64, DVS, 1, 1),
                                      kk > 0 ? 1u : 0u);
+                        mma_commit(&bar_o[oi & 1]);
                     }
-                    mma_commit(&bar_o[it & 1]);
                     mma_issued = it + 1;
                 }
             }
@@ -1068,20 +1107,20 @@ chain_kernel(const ChunkArgs a, const __grid_constant__ CUtensorMap gate_map, co
             int L_prev = 0;
             if constexpr (GATE) {
 #pragma unroll
-                for (int j = 0; j < HC; ++j) w16[j] = norm_w ? __ldg(norm_w + DVS * js + HC * hi + j) : 1.0f;
+                for (int j = 0; j < HC; ++j) w16[j] = norm_w ? __ldg(norm_w + DVS * jb + HC * hi + j) : 1.0f;
             }
-            // finishes y = o * rsqrt(mean o^2 + eps) * w * sigmoid(g) for chunk itp
+            // finishes y = o * rsqrt(mean o^2 + eps) * w * sigmoid(g) for output chunk itp
             auto finish_prev = [&](int itp) -> bool {
                 if (!mbar_wait_cluster(&bar_part[itp & 1], (uint32_t)((itp >> 1) & 1), a.status)) return false;
                 // arm the slot's barrier for chunk itp + 2 (its bytes may already be arriving)
-                if (tid == 0 && itp + 2 < nit) mbar_arrive_expect_tx(&bar_part[itp & 1], PART_TX);
+                if (tid == 0 && itp + 2 < nck) mbar_arrive_expect_tx(&bar_part[itp & 1], PART_TX);
                 if (trow < L_prev) {
                     const float* pp = s_part + (itp & 1) * (CLUSTER * 64);
                     float ss = 0.f;
 #pragma unroll
                     for (int r = 0; r < CLUSTER; ++r) ss += pp[r * 64 + trow];
                     const float inv = rsqrtf(ss * (1.0f / DV) + eps);
-                    const size_t obase = ((size_t)(t0_prev + trow) * H + h) * DV + (size_t)DVS * js + HC * hi;
+                    const size_t obase = ((size_t)(t0_prev + trow) * H + h) * DV + (size_t)DVS * jb + HC * hi;
 #pragma unroll
                     for (int m = 0; m < HC / 8; ++m) {
                         float y8[8];
@@ -1108,7 +1147,8 @@ chain_kernel(const ChunkArgs a, const __grid_constant__ CUtensorMap gate_map, co
             for (int it = 0; it < nit; ++it) {
                 const int b = bidx(it);
                 const uint8_t* buf = sm + b * CB_SIZE;
-                const int64_t t0 = s_beg + (int64_t)(c_beg + it) * CH;
+                const int oi = it - nseg;  // output index (chunk iterations)
+                const int64_t t0 = s_beg + (int64_t)(c_beg + oi) * CH;
                 const int L = (int)((s_end - t0) < CH ? (s_end - t0) : CH);
 
                 // (1) state update: S <- GamC o S - Mlr S + Bm
@@ -1130,15 +1170,21 @@ chain_kernel(const ChunkArgs a, const __grid_constant__ CUtensorMap gate_map, co
 #pragma unroll
                         for (int p = 0; p < 4; ++p) {
                             const int j = 8 * m + 2 * p;
-                            S[j] = gamC * S[j] - ds[j] + __uint_as_float(ww[p] << 16);
-                            S[j + 1] = gamC * S[j + 1] - ds[j + 1] + __uint_as_float(ww[p] & 0xFFFF0000u);
+                            const float b0 = trans ? 0.f : __uint_as_float(ww[p] << 16);
+                            const float b1 = trans ? 0.f : __uint_as_float(ww[p] & 0xFFFF0000u);
+                            S[j] = gamC * S[j] - ds[j] + b0;
+                            S[j + 1] = gamC * S[j + 1] - ds[j + 1] + b1;
                         }
                     }
                 }
                 // (2) the next chunk's state operand (D_S has been read)
                 if (it + 1 < nit) write_state_image(it + 1);
+                if (!has_out(it)) {  // a segment iteration, or no outputs at all: the buffer is done
+                    mbar_arrive(&bar_free[b]);
+                    continue;
+                }
                 // (3) this chunk's output: o = Qp S + Ob  (then y, when the gate is fused)
-                if (!mbar_wait(&bar_o[it & 1], (uint32_t)((it >> 1) & 1), a.status)) {
+                if (!mbar_wait(&bar_o[oi & 1], (uint32_t)((oi >> 1) & 1), a.status)) {
                     failed = true;
                     break;
                 }
@@ -1146,7 +1192,7 @@ chain_kernel(const ChunkArgs a, const __grid_constant__ CUtensorMap gate_map, co
                 float ov[DVS];
                 {
                     float dO[DVS];
-                    tmem_ld32(lane_addr + 32 + 32 * (it & 1), dO);
+                    tmem_ld32(lane_addr + 32 + 32 * (oi & 1), dO);
                     tmem_ld_wait();
                     // Ob slice [64 tokens][32 value cols]: row trow
                     const uint4* orow = reinterpret_cast<const uint4*>(buf + CB_O + (uint32_t)trow * (DVS * 2));
@@ -1173,7 +1219,7 @@ chain_kernel(const ChunkArgs a, const __grid_constant__ CUtensorMap gate_map, co
                 mbar_arrive(&bar_free[b]);  // everything this thread reads from the buffer is in registers
                 if constexpr (!GATE) {
                     if (lane < 16 && trow < L) {
-                        const size_t obase = ((size_t)(t0 + trow) * H + h) * DV + (size_t)DVS * js;
+                        const size_t obase = ((size_t)(t0 + trow) * H + h) * DV + (size_t)DVS * jb;
 #pragma unroll
                         for (int m = 0; m < DVS / 8; ++m) {
                             if constexpr (OUT_BF16) {
@@ -1188,7 +1234,7 @@ chain_kernel(const ChunkArgs a, const __grid_constant__ CUtensorMap gate_map, co
                 } else {
                     // finish the previous chunk first (its partials are read before this
                     // chunk's partials are published, which orders the slot reuse)
-                    if (it > 0 && !finish_prev(it - 1)) {
+                    if (oi > 0 && !finish_prev(oi - 1)) {
                         failed = true;
                         break;
                     }
@@ -1203,8 +1249,8 @@ chain_kernel(const ChunkArgs a, const __grid_constant__ CUtensorMap gate_map, co
 #pragma unroll
                     for (int m = 0; m < HC / 2; ++m) g_prev[m] = g_cur[m];  // kept for the next iteration
                     if (lane < 16) {
-                        const uint32_t slot = smem_u32(s_part + (it & 1) * (CLUSTER * 64) + js * 64 + trow);
-                        const uint32_t barl = smem_u32(&bar_part[it & 1]);
+                        const uint32_t slot = smem_u32(s_part + (oi & 1) * (CLUSTER * 64) + jb * 64 + trow);
+                        const uint32_t barl = smem_u32(&bar_part[oi & 1]);
 #pragma unroll
                         for (int r = 0; r < CLUSTER; ++r)
                             st_async_f32(map_to_cta(slot, (uint32_t)r), ss, map_to_cta(barl, (uint32_t)r));
@@ -1214,22 +1260,22 @@ chain_kernel(const ChunkArgs a, const __grid_constant__ CUtensorMap gate_map, co
                 }
                 // checkpoint: the state after (j + 1) * ckpt_every whole chunks of the sequence
                 if (a.ckpt) {
-                    const int cdone = c_beg + it + 1;  // chunks of this sequence now folded in
+                    const int cdone = c_beg + oi + 1;  // chunks of this sequence now folded in
                     const int64_t t_end = s_beg + (int64_t)cdone * CH;
                     if (cdone % a.ckpt_every == 0 && t_end <= s_end && cdone / a.ckpt_every <= a.n_ckpt) {
                         const int j = cdone / a.ckpt_every - 1;
                         float* dst =
-                            a.ckpt + ((((size_t)n * a.n_ckpt + j) * H + h) * DK + tid) * DV + (size_t)DVS * js;
+                            a.ckpt + ((((size_t)n * a.n_ckpt + j) * H + h) * DK + tid) * DV + (size_t)DVS * jb;
 #pragma unroll
                         for (int c4 = 0; c4 < DVS; c4 += 4)
                             __stcs(reinterpret_cast<float4*>(dst + c4), make_float4(S[c4], S[c4 + 1], S[c4 + 2], S[c4 + 3]));
                     }
                 }
-                // (4) D_O[it & 1] is no longer read
+                // (4) D_O[oi & 1] is no longer read
                 tc_fence_before();
             }
             if constexpr (GATE) {
-                if (!failed && !finish_prev(nit - 1)) failed = true;
+                if (!failed && nck > 0 && !finish_prev(nck - 1)) failed = true;
             }
         }
 
@@ -1244,7 +1290,7 @@ chain_kernel(const ChunkArgs a, const __grid_constant__ CUtensorMap gate_map, co
         if (warp == 4 && lane == 0 && failed && mma_issued > 0) {
             const int j = mma_issued - 1;
             mbar_wait(bar_s, (uint32_t)(j & 1), nullptr);
-            mbar_wait(&bar_o[j & 1], (uint32_t)((j >> 1) & 1), nullptr);
+            if (has_out(j)) mbar_wait(&bar_o[(j - nseg) & 1], (uint32_t)(((j - nseg) >> 1) & 1), nullptr);
         }
         tc_fence_before();
         __syncthreads();
@@ -1253,11 +1299,34 @@ chain_kernel(const ChunkArgs a, const __grid_constant__ CUtensorMap gate_map, co
         if constexpr (GATE) cluster_sync_all();  // no CTA leaves while a peer may still write to it
     }
 
-    // write the carried / final state slice
-    if (consumer) {
+    if constexpr (SEG == 1) {
+        // this segment's slot: B_g as the Bm slice jb, -M_g as the Mlr image (rows c,
+        // K columns [32 jb, 32 jb + 32)), GamC = 0
+        if (consumer) {
+            uint8_t* slot = a.seg_ws + (((size_t)n * a.segs + g) * H + h) * SLOT_BYTES;
+            if (!trans) {
+                uint4* dst = reinterpret_cast<uint4*>(slot + SO_B + (size_t)jb * BSL + (size_t)tid * DVS * 2);
 #pragma unroll
-        for (int j = 0; j < DVS; j += 4)
-            *reinterpret_cast<float4*>(a.state_io + st_off + j) = make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]);
+                for (int m = 0; m < DVS / 8; ++m) dst[swz64(tid, m)] = pack8(S + 8 * m);
+            } else {
+                float nS[DVS];
+#pragma unroll
+                for (int j = 0; j < DVS; ++j) nS[j] = -S[j];
+                const uint32_t k0 = (uint32_t)(DVS * jb);
+                uint8_t* img = slot + SO_M + (size_t)(k0 >> 6) * (DK * 128);
+#pragma unroll
+                for (int m = 0; m < DVS / 8; ++m)
+                    *reinterpret_cast<uint4*>(img + sw128_off((uint32_t)tid, (k0 & 63u) + 8u * m)) = pack8(nS + 8 * m);
+                if (jb == 0) *reinterpret_cast<float*>(slot + SO_G + 4 * tid) = 0.f;
+            }
+        }
+    } else {
+        // the carried / final state slice (with segments: the last segment's)
+        if (consumer && (SEG == 0 || g == a.segs - 1)) {
+#pragma unroll
+            for (int j = 0; j < DVS; j += 4)
+                *reinterpret_cast<float4*>(a.state_io + st_off + j) = make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]);
+        }
     }
 }
 
@@ -1319,27 +1388,60 @@ int g_num_sms = 0;
 
 }  // namespace
 
+// The chain launch of one pass: SEG as in chain_kernel; gate fused as a 4-CTA cluster.
+template <int SEG>
+static cudaError_t launch_chain(const ChunkArgs& a, const CUtensorMap& gate_map, const float* norm_w, float eps,
+                                bool out_bf16, bool fuse, dim3 gc, cudaStream_t stream) {
+    cudaLaunchConfig_t cfg;
+    memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = gc;
+    cfg.blockDim = dim3(CHAIN_THREADS, 1, 1);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    if (!fuse) {
+        cfg.dynamicSmemBytes = ChainLayout<false>::SMEM;
+        return out_bf16 ? cudaLaunchKernelEx(&cfg, chain_kernel<true, false, SEG>, a, gate_map, norm_w, eps)
+                        : cudaLaunchKernelEx(&cfg, chain_kernel<false, false, SEG>, a, gate_map, norm_w, eps);
+    }
+    // the four value-column slices of one (sequence, head) form a cluster
+    cfg.dynamicSmemBytes = ChainLayout<true>::SMEM;
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = CLUSTER;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return out_bf16 ? cudaLaunchKernelEx(&cfg, chain_kernel<true, true, SEG>, a, gate_map, norm_w, eps)
+                    : cudaLaunchKernelEx(&cfg, chain_kernel<false, true, SEG>, a, gate_map, norm_w, eps);
+}
+
+template <bool OB, bool G, int SEG>
+static cudaError_t set_chain_smem() {
+    return cudaFuncSetAttribute(chain_kernel<OB, G, SEG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)ChainLayout<G>::SMEM);
+}
+
+// Bytes of the segment slots that follow the chunk slots in segment-parallel mode.
+size_t chunk_seg_bytes(int n_seqs, int H, int segs) { return (size_t)n_seqs * segs * H * SLOT_BYTES; }
+
 cudaError_t chunk_fwd_launch(const void* q, const void* k, const void* v, const void* log_alpha, const void* beta,
                              const float* init_state, void* o, float* final_state, int B, int64_t T, int H,
                              const int32_t* cu, int n_seqs, int64_t max_seqlen, bool in_bf16, bool out_bf16,
                              float scale, const void* gate, const float* norm_w, float eps, float* ckpt,
-                             int64_t ckpt_tokens, void* workspace, size_t ws_bytes, cudaStream_t stream, int* n_passes,
-                             bool* gate_fused) {
+                             int64_t ckpt_tokens, int segs, void* workspace, size_t ws_bytes, cudaStream_t stream,
+                             int* n_passes, bool* gate_fused) {
     cudaError_t err;
     if (!g_attr_set) {
         err = cudaFuncSetAttribute(intra_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, INTRA_SMEM);
         if (err != cudaSuccess) return err;
         err = cudaFuncSetAttribute(intra_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, INTRA_SMEM);
         if (err != cudaSuccess) return err;
-        const int plain = (int)ChainLayout<false>::SMEM, fused = (int)ChainLayout<true>::SMEM;
-        if ((err = cudaFuncSetAttribute(chain_kernel<true, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        plain)) != cudaSuccess ||
-            (err = cudaFuncSetAttribute(chain_kernel<false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        plain)) != cudaSuccess ||
-            (err = cudaFuncSetAttribute(chain_kernel<true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        fused)) != cudaSuccess ||
-            (err = cudaFuncSetAttribute(chain_kernel<false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        fused)) != cudaSuccess)
+        if ((err = set_chain_smem<true, false, 0>()) != cudaSuccess || (err = set_chain_smem<false, false, 0>()) != cudaSuccess ||
+            (err = set_chain_smem<true, true, 0>()) != cudaSuccess || (err = set_chain_smem<false, true, 0>()) != cudaSuccess ||
+            (err = set_chain_smem<true, false, 1>()) != cudaSuccess || (err = set_chain_smem<false, false, 1>()) != cudaSuccess ||
+            (err = set_chain_smem<true, true, 1>()) != cudaSuccess || (err = set_chain_smem<false, true, 1>()) != cudaSuccess ||
+            (err = set_chain_smem<true, false, 2>()) != cudaSuccess || (err = set_chain_smem<false, false, 2>()) != cudaSuccess ||
+            (err = set_chain_smem<true, true, 2>()) != cudaSuccess || (err = set_chain_smem<false, true, 2>()) != cudaSuccess)
             return err;
         int dev = 0;
         if ((err = cudaGetDevice(&dev)) != cudaSuccess) return err;
@@ -1357,9 +1459,15 @@ cudaError_t chunk_fwd_launch(const void* q, const void* k, const void* v, const 
     float* carry = need_carry ? reinterpret_cast<float*>(ws + 256) : final_state;
     const size_t per_wc = (size_t)N * H * SLOT_BYTES;
     const size_t head = (fixed + 1023) & ~(size_t)1023;
-    const size_t wc_fit = ws_bytes > head ? (ws_bytes - head) / per_wc : 0;
-    int wc = (int)(wc_fit < (size_t)nchunks_max ? wc_fit : (size_t)nchunks_max);
-    if (wc < 1) wc = 1;
+    int wc;
+    if (segs > 1) {  // segment-parallel: one pass over every chunk, segment slots after the chunk slots
+        wc = nchunks_max > 0 ? nchunks_max : 1;
+        if (ws_bytes < head + (size_t)wc * per_wc + chunk_seg_bytes(N, H, segs)) return cudaErrorInvalidValue;
+    } else {
+        const size_t wc_fit = ws_bytes > head ? (ws_bytes - head) / per_wc : 0;
+        wc = (int)(wc_fit < (size_t)nchunks_max ? wc_fit : (size_t)nchunks_max);
+        if (wc < 1) wc = 1;
+    }
     ChunkArgs a;
     a.q = q; a.k = k; a.v = v; a.log_alpha = log_alpha; a.beta = beta;
     a.init_state = init_state; a.state_io = carry; a.o = o; a.cu = cu;
@@ -1370,6 +1478,8 @@ cudaError_t chunk_fwd_launch(const void* q, const void* k, const void* v, const 
     a.ckpt = ckpt;
     a.ckpt_every = ckpt ? (int)(ckpt_tokens / CH) : 1;
     a.n_ckpt = ckpt ? (int)(maxlen / ckpt_tokens) : 0;
+    a.segs = segs > 1 ? segs : 1;
+    a.seg_ws = segs > 1 ? a.ws + (size_t)wc * per_wc : nullptr;
 
     IntraMaps maps;
     memset(&maps, 0, sizeof(maps));
@@ -1411,32 +1521,18 @@ cudaError_t chunk_fwd_launch(const void* q, const void* k, const void* v, const 
             if ((err = cudaGetLastError()) != cudaSuccess) return err;
             prof_end(PROF_INTRA, stream);
         }
-        const dim3 gc((unsigned)NSL, (unsigned)H, (unsigned)N);
         prof_begin(PROF_CHAIN, stream);
-        if (!fuse) {
-            const unsigned sm_bytes = ChainLayout<false>::SMEM;
-            if (out_bf16) chain_kernel<true, false><<<gc, CHAIN_THREADS, sm_bytes, stream>>>(a, gate_map, norm_w, eps);
-            else chain_kernel<false, false><<<gc, CHAIN_THREADS, sm_bytes, stream>>>(a, gate_map, norm_w, eps);
-            if ((err = cudaGetLastError()) != cudaSuccess) return err;
+        if (a.segs == 1) {
+            err = launch_chain<0>(a, gate_map, norm_w, eps, out_bf16, fuse, dim3(NSL, H, N), stream);
         } else {
-            // the four value-column slices of one (sequence, head) form a cluster
-            cudaLaunchConfig_t cfg;
-            memset(&cfg, 0, sizeof(cfg));
-            cfg.gridDim = gc;
-            cfg.blockDim = dim3(CHAIN_THREADS, 1, 1);
-            cfg.dynamicSmemBytes = ChainLayout<true>::SMEM;
-            cfg.stream = stream;
-            cudaLaunchAttribute attr[1];
-            attr[0].id = cudaLaunchAttributeClusterDimension;
-            attr[0].val.clusterDim.x = CLUSTER;
-            attr[0].val.clusterDim.y = 1;
-            attr[0].val.clusterDim.z = 1;
-            cfg.attrs = attr;
-            cfg.numAttrs = 1;
-            err = out_bf16 ? cudaLaunchKernelEx(&cfg, chain_kernel<true, true>, a, gate_map, norm_w, eps)
-                           : cudaLaunchKernelEx(&cfg, chain_kernel<false, true>, a, gate_map, norm_w, eps);
-            if (err != cudaSuccess) return err;
+            // segment transitions (no outputs, no gate), then the segments with outputs
+            ChunkArgs at = a;
+            at.ckpt = nullptr;
+            err = launch_chain<1>(at, gate_map, norm_w, eps, out_bf16, false, dim3(2 * NSL, H, N * a.segs), stream);
+            if (err == cudaSuccess)
+                err = launch_chain<2>(a, gate_map, norm_w, eps, out_bf16, fuse, dim3(NSL, H, N * a.segs), stream);
         }
+        if (err != cudaSuccess) return err;
         prof_end(PROF_CHAIN, stream);
         ++passes;
     }

@@ -27,7 +27,8 @@ def declared_symbols():
 
 def test_header_declares_the_entry_points():
     syms = declared_symbols()
-    for s in ("kda_chunk_fwd", "kda_chunk_fwd_ckpt", "kda_decode_step", "kda_decode_steps", "kda_gate_norm",
+    for s in ("kda_chunk_fwd", "kda_chunk_fwd_ckpt", "kda_chunk_fwd_segmented", "kda_decode_step", "kda_decode_steps",
+              "kda_gate_norm", "kda_chunk_fwd_segmented_workspace_size",
               "kda_chunk_fwd_workspace_size",
               "kda_query_status", "kda_status_string", "kda_version"):
         assert s in syms
@@ -85,6 +86,19 @@ def test_chunk_fwd_ckpt_host_validation(lib):
     assert ck(FAKE, 0) == -1
     assert ck(FAKE + 4, 64) == -3   # misaligned checkpoint buffer
     assert ck(FAKE, 64, q=None) == -1
+
+
+def test_segmented_workspace_size(lib):
+    import ctypes
+    plain_lo, plain_full = ctypes.c_size_t(0), ctypes.c_size_t(0)
+    assert lib.kda_chunk_fwd_workspace_size(4096, 4, 128, 128, 2, 2048, ctypes.byref(plain_lo),
+                                            ctypes.byref(plain_full)) == 0
+    seg = ctypes.c_size_t(0)
+    assert lib.kda_chunk_fwd_segmented_workspace_size(4096, 4, 128, 128, 2, 2048, 8, ctypes.byref(seg)) == 0
+    assert seg.value == plain_full.value + 2 * 8 * 4 * 98816  # every chunk plus one map per segment
+    assert lib.kda_chunk_fwd_segmented_workspace_size(4096, 4, 128, 128, 2, 2048, 1, ctypes.byref(seg)) == 0
+    assert seg.value == plain_full.value
+    assert lib.kda_chunk_fwd_segmented_workspace_size(4096, 4, 128, 128, 2, 2048, 0, ctypes.byref(seg)) == -1
 
 
 def test_chunk_fwd_host_validation(lib):

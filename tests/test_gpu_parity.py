@@ -187,6 +187,44 @@ def test_prefill_state_checkpoints(multi_pass):
     np.testing.assert_array_equal(ck[4, 0], host(fs)[4])
 
 
+@pytest.mark.parametrize("segments,gate,lens,memory", [
+    (2, False, [256], "short"),
+    (3, True, [300], "short"),
+    (4, False, [700, 65, 0, 1, 200, 129], "short"),
+    (8, True, [1000, 64, 450], "short"),
+    (4, False, [700, 300], "long"),      # decays x 0.01: the state carries across segments
+    (6, True, [900, 130], "none"),       # no decay at all: only the erase term forgets
+])
+def test_prefill_segment_parallel(segments, gate, lens, memory):
+    """Segment-parallel prefill (segment maps, then segments from their folded
+    initial states) against the oracle: outputs, final states, per sequence;
+    sequences shorter than `segments` chunks leave empty segments.  The long- and
+    no-decay cases make the segment maps matter (with the default decays the
+    state forgets within a chunk)."""
+    torch = _torch()
+    import linear_attention_recurrence_06_b200 as kda
+    H = 2
+    kw = {"short": {}, "long": dict(la_scale=0.01), "none": dict(la_const=0.0)}[memory]
+    inp = make_prefill(41 + segments, lens, H, bf16=True, gate=gate, init=True, **kw)
+    T = inp["T"]
+    dt = torch.bfloat16
+    q, k, v, la = (dev(inp[x], dt).view(1, T, H, D) for x in ("q", "k", "v", "log_alpha"))
+    b = dev(inp["beta"], dt).view(1, T, H)
+    g = dev(inp["g"], dt).view(1, T, H, D) if gate else None
+    cu = torch.from_numpy(inp["cu"].astype(np.int32)).cuda()
+    o, fs = kda.chunk_fwd(q, k, v, la, b, dev(inp["s0"], torch.float32), cu_seqlens=cu, max_seqlen=max(lens),
+                          gate=g, out_dtype=torch.float32, segments=segments)
+    torch.cuda.synchronize()
+    ro, rfs = oracle_prefill(inp, gate=gate)
+    oh, fh = host(o).reshape(T, H, D), host(fs)
+    check(oh, fh, ro, rfs)
+    for n, L in enumerate(lens):
+        sl = slice(inp["cu"][n], inp["cu"][n + 1])
+        if L:
+            assert rel_l2(oh[sl], ro[sl]) <= REL_L2_TOL, f"seq {n}"
+        assert rel_l2(fh[n], rfs[n]) <= REL_L2_TOL, f"seq {n} state"
+
+
 def test_prefill_multi_pass_workspace():
     """A workspace that holds one chunk per sequence forces one pass per chunk:
     the state carried between passes must give the same result."""
