@@ -225,6 +225,9 @@ def run_ours(args, peaks):
     # end to end through the public API: pinned host inputs -> device -> call -> host output
     e2e = run_e2e(args, torch, kda, hq, out, fs, ws, stream, mor, barrier)
 
+    # segment-parallel prefill on a low-parallelism shape (one sequence, one head)
+    seg = run_segmented(args, torch, kda, dev, stream, mor, barrier)
+
     if dist is not None:
         dist.barrier()
         dist.destroy_process_group()
@@ -253,7 +256,7 @@ def run_ours(args, peaks):
                    "parallelism": f"dp{ws_n} (independent sequences per rank, no collective)",
                    "l2": "inputs larger than L2 (q,k,v,log_alpha,gate,beta = 336 MB per step)"},
         "prefill_tflops": tflops, "prefill_tensor_frac": tflops / peaks["bf16_tflops_sustained"],
-        "roofline": roof, "kernels": kernels, "decode": dec, "e2e": e2e,
+        "roofline": roof, "kernels": kernels, "decode": dec, "e2e": e2e, "segment_parallel": seg,
         "gpu_launches": int(round(launches_per_step * args.steps)),
         "clocks": clocks,
     }
@@ -337,6 +340,50 @@ def run_decode(args, torch, kda, dev, stream, rank, max_over_ranks, barrier):
                          "traffic": recorded_traffic("decode_step_kernel", Bd * H),
                          "algorithmic_bytes_per_launch": state_bytes + tok_bytes},
             "speculative_verify": spec}
+
+
+SEG_SHAPE = dict(T=65536, H=1, segments=32)
+
+
+def run_segmented(args, torch, kda, dev, stream, max_over_ranks, barrier):
+    """One sequence of 65536 tokens, one head (4 chains for the plain walk): the
+    plain prefill against the segment-parallel one (32 segments), both with the
+    fused gate, decays scaled by 0.01 so that the state carries across segments."""
+    from linear_attention_recurrence_06_b200 import synth
+    T, H, G = SEG_SHAPE["T"], SEG_SHAPE["H"], SEG_SHAPE["segments"]
+    tb = synth.tokens(300, 0, T, H, D, D, bf16=True, gate=True)
+    tb.log_alpha = (tb.log_alpha * 0.01).astype(np.float32)
+    x = {n: torch.from_numpy(np.ascontiguousarray(getattr(tb, n))).to(torch.bfloat16).to(dev)
+         for n in ("q", "k", "v", "log_alpha", "beta", "g")}
+    x = {n: t.view(1, T, H, -1) if n != "beta" else t.view(1, T, H) for n, t in x.items()}
+    out = torch.empty((1, T, H, D), dtype=torch.bfloat16, device=dev)
+    fs = torch.empty((1, H, D, D), dtype=torch.float32, device=dev)
+    res = {"workload": f"KDA prefill B=1 T={T} H={H} bf16, fused gate, decays x 0.01", "segments": G}
+    for name, segs in (("plain", 1), ("segmented", G)):
+        nbytes = kda.segmented_workspace_size(T, H, 1, T, segs) if segs > 1 else kda.workspace_size(T, H, 1, T)[1]
+        ws = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+
+        def f():
+            kda.chunk_fwd(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], None, gate=x["g"], out=out,
+                          final_state=fs, workspace=ws, segments=segs, stream=stream)
+
+        for _ in range(3):
+            f()
+        n = max(5, min(args.steps, 20))
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier()
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(n):
+            f()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        ms = max_over_ranks(e0.elapsed_time(e1) / n)
+        res[name] = {"ms_per_call": ms, "tokens_per_s": T / (ms * 1e-3)}
+        del ws
+    res["speedup"] = res["plain"]["ms_per_call"] / res["segmented"]["ms_per_call"]
+    return res
 
 
 def run_e2e(args, torch, kda, hq, out, fs, ws, stream, max_over_ranks, barrier):
