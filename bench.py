@@ -228,6 +228,9 @@ def run_ours(args, peaks):
     # segment-parallel prefill on a low-parallelism shape (one sequence, one head)
     seg = run_segmented(args, torch, kda, dev, stream, mor, barrier)
 
+    # per-device steps of context parallelism across devices (ranks emulated on this GPU)
+    kcp = run_kcp(args, torch, kda, dev, stream, mor, barrier)
+
     if dist is not None:
         dist.barrier()
         dist.destroy_process_group()
@@ -257,7 +260,7 @@ def run_ours(args, peaks):
                    "l2": "inputs larger than L2 (q,k,v,log_alpha,gate,beta = 336 MB per step)"},
         "prefill_tflops": tflops, "prefill_tensor_frac": tflops / peaks["bf16_tflops_sustained"],
         "roofline": roof, "kernels": kernels, "decode": dec, "e2e": e2e, "segment_parallel": seg,
-        "gpu_launches": int(round(launches_per_step * args.steps)),
+        "kcp_per_device": kcp, "gpu_launches": int(round(launches_per_step * args.steps)),
         "clocks": clocks,
     }
     if ws_n == 1 and not args.no_cpu_baseline:
@@ -383,6 +386,65 @@ def run_segmented(args, torch, kda, dev, stream, max_over_ranks, barrier):
         res[name] = {"ms_per_call": ms, "tokens_per_s": T / (ms * 1e-3)}
         del ws
     res["speedup"] = res["plain"]["ms_per_call"] / res["segmented"]["ms_per_call"]
+    return res
+
+
+KCP_SHAPE = dict(T_rank=8192, H=32, ranks=8)
+
+
+def run_kcp(args, torch, kda, dev, stream, max_over_ranks, barrier):
+    """The work one device does when a sequence of ranks x 8192 tokens (32 heads,
+    fused gate) is split over `ranks` devices: transition (chunk-local kernel +
+    the walk that forms M and B), compose of the maps of all earlier devices
+    (the last device's case: ranks - 1 maps) and finish (the walk with outputs),
+    next to the plain prefill of the same 8192 tokens.  The all-gather between
+    transition and compose is not timed (one GPU); its size is reported."""
+    from linear_attention_recurrence_06_b200 import synth
+    T, H, R = KCP_SHAPE["T_rank"], KCP_SHAPE["H"], KCP_SHAPE["ranks"]
+    tb = synth.tokens(400, 0, T, H, D, D, bf16=True, gate=True)
+    x = {n: torch.from_numpy(np.ascontiguousarray(getattr(tb, n))).to(torch.bfloat16).to(dev)
+         for n in ("q", "k", "v", "log_alpha", "beta", "g")}
+    x = {n: t.view(1, T, H, -1) if n != "beta" else t.view(1, T, H) for n, t in x.items()}
+    out = torch.empty((1, T, H, D), dtype=torch.bfloat16, device=dev)
+    fs = torch.empty((1, H, D, D), dtype=torch.float32, device=dev)
+    ws = torch.empty(kda.kcp_workspace_size(T, H, 1, T), dtype=torch.uint8, device=dev)
+    trans = torch.empty((2, 1, H, D, D), dtype=torch.float32, device=dev)
+    s_in = torch.empty((1, H, D, D), dtype=torch.float32, device=dev)
+    s0 = torch.zeros((1, H, D, D), dtype=torch.float32, device=dev)
+    steps = {
+        "transition": lambda: kda.kcp_transition(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"],
+                                                 transition=trans, workspace=ws, stream=stream),
+        "compose": lambda: kda.kcp_compose(gathered, R - 1, s0, out=s_in, stream=stream),
+        "finish": lambda: kda.kcp_finish(s_in, ws, shape=(1, T, H, D), dtype=torch.bfloat16, gate=x["g"],
+                                         out=out, stream=stream),
+        "plain": lambda: kda.chunk_fwd(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], None, gate=x["g"],
+                                       out=out, final_state=fs, workspace=ws, stream=stream),
+    }
+    steps["transition"]()
+    torch.cuda.synchronize()
+    gathered = trans.unsqueeze(0).expand((R,) + tuple(trans.shape)).contiguous()  # stands for the all-gather
+    res = {"workload": f"one sequence of {R} x {T} tokens, H={H}, bf16, fused gate; per device",
+           "ranks": R, "tokens_per_device": T,
+           "all_gather_bytes_per_device": trans.numel() * trans.element_size()}
+    # order matters: finish reads the slots transition left in the workspace
+    for name in ("transition", "compose", "finish", "plain"):
+        f = steps[name]
+        for _ in range(3):
+            f()
+        n = max(5, min(args.steps, 20))
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier()
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(n):
+            f()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        res[name + "_ms"] = max_over_ranks(e0.elapsed_time(e1) / n)
+    res["device_ms"] = res["transition_ms"] + res["compose_ms"] + res["finish_ms"]
+    res["overhead_vs_plain"] = res["device_ms"] / res["plain_ms"]
+    res["sequence_tokens_per_s_without_gather"] = R * T / (res["device_ms"] * 1e-3)
     return res
 
 

@@ -189,6 +189,76 @@ KDA_API kda_status kda_chunk_fwd_segmented_workspace_size(int64_t T, int H, int 
                                                   size_t* bytes);
 
 /*
+ * Context parallelism across devices (KCP: the nlpx.cn K3 walkthrough, §6; the
+ * "training and inference systems" item of the K3 article summaries: context
+ * parallelism as a prefix scan of segment transitions).  Every sequence is cut
+ * into consecutive token segments, segment r on device r.  Segment r's effect
+ * on the state is affine, S -> M_r S + B_r, so each device
+ *   1. kda_kcp_transition: runs the chunk-local work over its segment, keeps it
+ *      in the workspace and writes (M_r, B_r) in fp32;
+ *   2. exchanges the maps (an all-gather in device order; the library does no
+ *      communication);
+ *   3. kda_kcp_compose: folds the maps of devices 0 .. r-1 over the sequences'
+ *      initial state into its own initial state;
+ *   4. kda_kcp_finish: walks its kept chunks from that state, with outputs.
+ * Device r's outputs then equal those of kda_chunk_fwd over the whole
+ * sequence (up to fp32 rounding of the composition and bf16 rounding of the
+ * map's state image inside the walk), and the last device's final state is
+ * the sequence's.  Arguments as kda_chunk_fwd, for this device's segment.
+ *
+ * kda_kcp_workspace_size -- bytes of the workspace that steps 1 and 4 share
+ * (every chunk's slot at once: kda_chunk_fwd_workspace_size's bytes_full).
+ */
+KDA_API kda_status kda_kcp_workspace_size(int64_t T, int H, int dk, int dv, int n_seqs, int64_t max_seqlen,
+                                          size_t* bytes);
+
+/*
+ * kda_kcp_transition -- step 1.  Inputs as kda_chunk_fwd (q and scale are used:
+ * the kept chunk work includes the output terms).
+ *
+ *   transition  [2, N, H, dk, dk] fp32, device, caller-owned: [0] = M (dk x dk),
+ *               [1] = B (dk x dv) with S_out = M S_in + B per (sequence, head);
+ *               an empty segment gives M = I, B = 0
+ *   workspace   >= kda_kcp_workspace_size bytes, 256-byte aligned; it holds the
+ *               chunk slots until kda_kcp_finish has run on the same stream
+ *
+ * Errors as kda_chunk_fwd (device-side ones land in the workspace status word).
+ */
+KDA_API kda_status kda_kcp_transition(const void* q, const void* k, const void* v, const void* log_alpha,
+                                      const void* beta, int B, int64_t T, int H, int dk, int dv,
+                                      const int32_t* cu_seqlens, int n_seqs, int64_t max_seqlen,
+                                      kda_dtype in_dtype, float scale, float* transition, void* workspace,
+                                      size_t workspace_bytes, void* stream);
+
+/*
+ * kda_kcp_compose -- step 3:  S = init_state (zero when NULL), then for
+ * j = 0 .. n_prev-1:  S = M_j S + B_j;  state_in = S.
+ *
+ *   transitions [R, 2, N, H, dk, dk] fp32, device: the gathered maps in device
+ *               order (R >= n_prev; may be NULL when n_prev == 0)
+ *   init_state  [N, H, dk, dv] fp32 or NULL; state_in [N, H, dk, dv] fp32 (output)
+ *
+ * KDA_ERR_INVALID_ARG for n_prev < 0 or missing buffers, KDA_ERR_MISALIGNED
+ * for pointers not 16-byte aligned.
+ */
+KDA_API kda_status kda_kcp_compose(const float* transitions, int n_prev, const float* init_state,
+                                   float* state_in, int n_seqs, int H, int dk, int dv, void* stream);
+
+/*
+ * kda_kcp_finish -- step 4: the walk of kda_chunk_fwd over the chunk slots
+ * that kda_kcp_transition left in `workspace` (same B, T, H, cu_seqlens,
+ * n_seqs, max_seqlen and workspace), starting from state_in (NULL = zero).
+ * o, final_state, gate, norm_weight, eps and the dtypes as kda_chunk_fwd;
+ * in_dtype is the gate's dtype.  The workspace status word carries step 1's
+ * device-side errors too.
+ */
+KDA_API kda_status kda_kcp_finish(const float* state_in, void* o, float* final_state, int B, int64_t T, int H,
+                                  int dk, int dv, const int32_t* cu_seqlens, int n_seqs, int64_t max_seqlen,
+                                  kda_dtype in_dtype, kda_dtype out_dtype, const void* gate,
+                                  const float* norm_weight, float eps, void* workspace, size_t workspace_bytes,
+                                  void* stream);
+
+/*
  * kda_decode_step -- one recurrent step for Bd independent sequences
  * ("decode uses the recurrent form", chunkwise-algorithm item of the K3
  * article summaries).  The state is read once and written once, in place.

@@ -12,6 +12,9 @@ Entry points (same names as the C ABI):
   decode_step    one recurrent step per sequence, state updated in place
   gate_norm      per-head RMSNorm over dv times sigmoid output gate
   workspace_size bytes the prefill needs
+  kcp_transition / kcp_compose / kcp_finish
+                 the per-device steps of context parallelism across devices
+                 (the exchange between them is in ``kcp.py``)
   query_status   reads and clears the device status word of a workspace
 """
 from __future__ import annotations
@@ -72,6 +75,16 @@ def load_library(path: str | None = None):
         list(lib.kda_chunk_fwd.argtypes[22:])
     lib.kda_chunk_fwd_segmented_workspace_size.restype = i32
     lib.kda_chunk_fwd_segmented_workspace_size.argtypes = [i64, i32, i32, i32, i32, i64, i32, ctypes.POINTER(sz)]
+    lib.kda_kcp_workspace_size.restype = i32
+    lib.kda_kcp_workspace_size.argtypes = [i64, i32, i32, i32, i32, i64, ctypes.POINTER(sz)]
+    lib.kda_kcp_transition.restype = i32
+    lib.kda_kcp_transition.argtypes = [vp, vp, vp, vp, vp, i32, i64, i32, i32, i32, vp, i32, i64, i32, f32, vp, vp,
+                                       sz, vp]
+    lib.kda_kcp_compose.restype = i32
+    lib.kda_kcp_compose.argtypes = [vp, i32, vp, vp, i32, i32, i32, i32, vp]
+    lib.kda_kcp_finish.restype = i32
+    lib.kda_kcp_finish.argtypes = [vp, vp, vp, i32, i64, i32, i32, i32, vp, i32, i64, i32, i32, vp, vp, f32, vp, sz,
+                                   vp]
     lib.kda_decode_step.restype = i32
     lib.kda_decode_step.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, f32, vp, vp, f32, vp]
     lib.kda_decode_steps.restype = i32
@@ -212,6 +225,96 @@ def chunk_fwd(q, k, v, log_alpha, beta, initial_state=None, *, cu_seqlens=None, 
     if st != KDA_OK:
         raise KdaError(st, "kda_chunk_fwd_ckpt")
     return o, fs, checkpoints
+
+
+def _seq_dims(q, cu_seqlens, max_seqlen):
+    torch = _torch()
+    B, T = q.shape[0], q.shape[1]
+    if cu_seqlens is not None:
+        if cu_seqlens.dtype != torch.int32:
+            raise TypeError("cu_seqlens must be int32")
+        if max_seqlen is None:
+            raise ValueError("varlen needs max_seqlen (host int)")
+        return B, T, cu_seqlens.numel() - 1, int(max_seqlen)
+    return B, T, B, T
+
+
+def kcp_workspace_size(T: int, H: int, n_seqs: int, max_seqlen: int, dk: int = HEAD_DIM, dv: int = HEAD_DIM) -> int:
+    """Workspace bytes shared by kcp_transition and kcp_finish."""
+    n = ctypes.c_size_t(0)
+    st = load_library().kda_kcp_workspace_size(T, H, dk, dv, n_seqs, max_seqlen, ctypes.byref(n))
+    if st != KDA_OK:
+        raise KdaError(st, "kda_kcp_workspace_size")
+    return n.value
+
+
+def kcp_transition(q, k, v, log_alpha, beta, *, cu_seqlens=None, max_seqlen=None, scale: float = 1.0,
+                   transition=None, workspace=None, stream=None):
+    """Step 1 of context parallelism across devices, for this device's token
+    segment (inputs as chunk_fwd).  Returns (transition fp32 [2, N, H, 128, 128]:
+    [0] = M, [1] = B with S_out = M S_in + B; workspace holding the chunk work
+    for kcp_finish)."""
+    torch = _torch()
+    _check_cuda(q, k, v, log_alpha, beta, cu_seqlens, transition, workspace)
+    B, T, N, maxlen = _seq_dims(q, cu_seqlens, max_seqlen)
+    H, dk, dv = q.shape[2], q.shape[3], v.shape[-1]
+    for t in (k, v, log_alpha, beta):
+        if t.dtype != q.dtype:
+            raise TypeError("q, k, v, log_alpha and beta must share one dtype")
+    if transition is None:
+        transition = torch.empty((2, N, H, dk, dk), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = torch.empty(kcp_workspace_size(B * T if cu_seqlens is None else T, H, N, maxlen, dk, dv),
+                                dtype=torch.uint8, device=q.device)
+    st = load_library().kda_kcp_transition(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), B, T, H, dk, dv,
+                                           _ptr(cu_seqlens), N, maxlen, _dt(q), float(scale), _ptr(transition),
+                                           _ptr(workspace), workspace.numel(), _stream(stream))
+    if st != KDA_OK:
+        raise KdaError(st, "kda_kcp_transition")
+    return transition, workspace
+
+
+def kcp_compose(transitions, n_prev: int, initial_state=None, *, out=None, stream=None):
+    """Step 3: folds maps 0 .. n_prev-1 of the gathered transitions
+    ([R, 2, N, H, 128, 128] fp32, device order) over initial_state (fp32
+    [N, H, 128, 128] or None = zero).  Returns this device's initial state."""
+    torch = _torch()
+    _check_cuda(transitions, initial_state, out)
+    _, _, N, H, dk, dv = transitions.shape
+    s_in = out if out is not None else torch.empty((N, H, dk, dv), dtype=torch.float32, device=transitions.device)
+    st = load_library().kda_kcp_compose(_ptr(transitions), int(n_prev), _ptr(initial_state), _ptr(s_in), N, H, dk,
+                                        dv, _stream(stream))
+    if st != KDA_OK:
+        raise KdaError(st, "kda_kcp_compose")
+    return s_in
+
+
+def kcp_finish(state_in, workspace, *, shape, dtype, cu_seqlens=None, max_seqlen=None, gate=None, norm_weight=None,
+               eps: float = 1e-6, out_dtype=None, output_final_state: bool = True, out=None, stream=None):
+    """Step 4: this device's outputs from its initial state and the workspace
+    kcp_transition filled.  shape = (B, T, H, 128) and dtype of the segment's
+    inputs (the gate's dtype).  Returns (o or y [B, T, H, 128], final_state)."""
+    torch = _torch()
+    _check_cuda(state_in, workspace, cu_seqlens, gate, norm_weight)
+    B, T, H, dv = shape
+    if gate is not None and gate.dtype != dtype:
+        raise TypeError("the gate must have the inputs' dtype")
+    if cu_seqlens is not None:
+        if max_seqlen is None:
+            raise ValueError("varlen needs max_seqlen (host int)")
+        N, maxlen = cu_seqlens.numel() - 1, int(max_seqlen)
+    else:
+        N, maxlen = B, T
+    in_dt = KDA_BF16 if dtype == torch.bfloat16 else KDA_F32
+    odt = out_dtype if out_dtype is not None else dtype
+    o = out if out is not None else torch.empty((B, T, H, dv), dtype=odt, device=workspace.device)
+    fs = torch.empty((N, H, HEAD_DIM, dv), dtype=torch.float32, device=workspace.device) if output_final_state else None
+    st = load_library().kda_kcp_finish(_ptr(state_in), _ptr(o), _ptr(fs), B, T, H, HEAD_DIM, dv, _ptr(cu_seqlens), N,
+                                       maxlen, in_dt, _dt(o), _ptr(gate), _ptr(norm_weight), float(eps),
+                                       _ptr(workspace), workspace.numel(), _stream(stream))
+    if st != KDA_OK:
+        raise KdaError(st, "kda_kcp_finish")
+    return o, fs
 
 
 def decode_step(state, q, k, v, log_alpha, beta, *, scale: float = 1.0, gate=None, norm_weight=None,

@@ -9,25 +9,9 @@
 #include <vector>
 
 #include "../../include/kda.h"
+#include "kda_launch.h"
 #include "kda_profile.h"
 
-namespace kda {
-cudaError_t launch_decode_step(float* state, const void* q, const void* k, const void* v, const void* log_alpha,
-                               const void* beta, void* o, int Bd, int H, bool in_bf16, bool out_bf16, float scale,
-                               const void* gate, const float* norm_w, float eps, int n_steps, float* step_states,
-                               cudaStream_t stream);
-cudaError_t launch_gate_norm(const void* o, const void* g, const float* norm_w, float eps, void* y, int64_t rows,
-                             bool o_bf16, bool g_bf16, bool out_bf16, int num_sms, cudaStream_t stream);
-size_t chunk_slot_bytes();
-size_t chunk_fixed_bytes(int n_seqs, int H, bool need_carry);
-size_t chunk_seg_bytes(int n_seqs, int H, int segs);
-cudaError_t chunk_fwd_launch(const void* q, const void* k, const void* v, const void* log_alpha, const void* beta,
-                             const float* init_state, void* o, float* final_state, int B, int64_t T, int H,
-                             const int32_t* cu, int n_seqs, int64_t max_seqlen, bool in_bf16, bool out_bf16,
-                             float scale, const void* gate, const float* norm_w, float eps, float* ckpt,
-                             int64_t ckpt_tokens, int segs, void* workspace, size_t ws_bytes, cudaStream_t stream,
-                             int* n_passes, bool* gate_fused);
-}  // namespace kda
 
 namespace kda {
 namespace {
@@ -145,10 +129,18 @@ static kda_status chunk_fwd_impl(const void* q, const void* k, const void* v, co
                                  int64_t max_seqlen, kda_dtype in_dtype, kda_dtype out_dtype, float scale,
                                  const void* gate, const float* norm_weight, float eps, float* checkpoints,
                                  int64_t ckpt_tokens, int segments, void* workspace, size_t workspace_bytes,
-                                 void* stream) {
-    if (!q || !k || !v || !log_alpha || !beta || !o) return KDA_ERR_INVALID_ARG;
+                                 void* stream, int kcp_mode = kda::KCP_NONE, float* transition = nullptr) {
+    // the finishing half of the cross-device form reads no token inputs, the
+    // transition half writes no outputs; with no tokens at all (an empty segment
+    // of a sequence split over devices) the token buffers may be NULL
+    const bool has_tokens = B > 0 && T > 0;
+    if (has_tokens && kcp_mode != kda::KCP_FINISH && (!q || !k || !v || !log_alpha || !beta))
+        return KDA_ERR_INVALID_ARG;
+    if (has_tokens && kcp_mode != kda::KCP_TRANSITION && !o) return KDA_ERR_INVALID_ARG;
+    if (kcp_mode == kda::KCP_TRANSITION && !transition) return KDA_ERR_INVALID_ARG;
     if (B <= 0 || T < 0 || H <= 0 || !dtype_ok(in_dtype) || !dtype_ok(out_dtype)) return KDA_ERR_INVALID_ARG;
     if (dk != kSupportedD || dv != kSupportedD) return KDA_ERR_UNSUPPORTED;
+    if (H > 65535 || (cu_seqlens ? n_seqs : B) > 65535) return KDA_ERR_UNSUPPORTED;  // grid y / z extents
     if (cu_seqlens) {
         if (B != 1 || n_seqs <= 0 || max_seqlen < 0 || max_seqlen > T) return KDA_ERR_INVALID_ARG;
         if (T > INT32_MAX) return KDA_ERR_UNSUPPORTED;
@@ -161,17 +153,18 @@ static kda_status chunk_fwd_impl(const void* q, const void* k, const void* v, co
     if (checkpoints && (ckpt_tokens <= 0 || ckpt_tokens % 64 != 0)) return KDA_ERR_INVALID_ARG;
     if (segments < 1) return KDA_ERR_INVALID_ARG;
     const void* ptrs[] = {q, k, v, log_alpha, beta, init_state, o, final_state, cu_seqlens, gate, norm_weight, workspace,
-                          checkpoints};
+                          checkpoints, transition};
     for (const void* p : ptrs)
         if (p && !aligned16(p)) return KDA_ERR_MISALIGNED;
     if (!workspace) return KDA_ERR_WORKSPACE;
     if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return KDA_ERR_MISALIGNED;
     size_t need_min = 0;
+    const int64_t tot = T * (cu_seqlens ? 1 : B);
     const kda_status wst =
-        segments > 1 ? kda_chunk_fwd_segmented_workspace_size(T * (cu_seqlens ? 1 : B), H, dk, dv, n_seqs, max_seqlen,
-                                                               segments, &need_min)
-                     : kda_chunk_fwd_workspace_size(T * (cu_seqlens ? 1 : B), H, dk, dv, n_seqs, max_seqlen,
-                                                    &need_min, nullptr);
+        segments > 1 ? kda_chunk_fwd_segmented_workspace_size(tot, H, dk, dv, n_seqs, max_seqlen, segments, &need_min)
+        : kcp_mode != kda::KCP_NONE
+            ? kda_chunk_fwd_workspace_size(tot, H, dk, dv, n_seqs, max_seqlen, nullptr, &need_min)
+            : kda_chunk_fwd_workspace_size(tot, H, dk, dv, n_seqs, max_seqlen, &need_min, nullptr);
     if (wst != KDA_OK) return KDA_ERR_INVALID_ARG;
     if (workspace_bytes < need_min) return KDA_ERR_WORKSPACE;
 
@@ -180,10 +173,11 @@ static kda_status chunk_fwd_impl(const void* q, const void* k, const void* v, co
     bool fused = false;
     cudaError_t e = kda::chunk_fwd_launch(q, k, v, log_alpha, beta, init_state, o, final_state, B, T, H, cu_seqlens,
                                           n_seqs, max_seqlen, in_bf16, out_bf16, scale, gate, norm_weight, eps,
-                                          checkpoints, ckpt_tokens, segments, workspace, workspace_bytes, st, nullptr,
+                                          checkpoints, ckpt_tokens, segments, kcp_mode, transition, workspace,
+                                          workspace_bytes, st, nullptr,
                                           &fused);
     if (e != cudaSuccess) return KDA_ERR_CUDA;
-    if (gate && !fused) {
+    if (gate && !fused && kcp_mode != kda::KCP_TRANSITION) {
         const int64_t rows = (int64_t)B * T * H;
         // y overwrites o in place (o already holds out_dtype values)
         kda::prof_begin(kda::PROF_GATE_NORM, st);
@@ -225,6 +219,41 @@ kda_status kda_chunk_fwd(const void* q, const void* k, const void* v, const void
     return kda_chunk_fwd_ckpt(q, k, v, log_alpha, beta, init_state, o, final_state, B, T, H, dk, dv, cu_seqlens, n_seqs,
                               max_seqlen, in_dtype, out_dtype, scale, gate, norm_weight, eps, nullptr, 0, workspace,
                               workspace_bytes, stream);
+}
+
+kda_status kda_kcp_workspace_size(int64_t T, int H, int dk, int dv, int n_seqs, int64_t max_seqlen, size_t* bytes) {
+    if (!bytes) return KDA_ERR_INVALID_ARG;
+    return kda_chunk_fwd_workspace_size(T, H, dk, dv, n_seqs, max_seqlen, nullptr, bytes);
+}
+
+kda_status kda_kcp_transition(const void* q, const void* k, const void* v, const void* log_alpha, const void* beta,
+                              int B, int64_t T, int H, int dk, int dv, const int32_t* cu_seqlens, int n_seqs,
+                              int64_t max_seqlen, kda_dtype in_dtype, float scale, float* transition,
+                              void* workspace, size_t workspace_bytes, void* stream) {
+    return chunk_fwd_impl(q, k, v, log_alpha, beta, nullptr, nullptr, nullptr, B, T, H, dk, dv, cu_seqlens, n_seqs,
+                          max_seqlen, in_dtype, in_dtype, scale, nullptr, nullptr, 0.f, nullptr, 0, 1, workspace,
+                          workspace_bytes, stream, kda::KCP_TRANSITION, transition);
+}
+
+kda_status kda_kcp_compose(const float* transitions, int n_prev, const float* init_state, float* state_in,
+                           int n_seqs, int H, int dk, int dv, void* stream) {
+    if (!state_in || n_prev < 0 || (n_prev > 0 && !transitions) || n_seqs < 0 || H <= 0) return KDA_ERR_INVALID_ARG;
+    if (dk != kSupportedD || dv != kSupportedD) return KDA_ERR_UNSUPPORTED;
+    if (H > 65535 || n_seqs > 65535) return KDA_ERR_UNSUPPORTED;
+    const void* ptrs[] = {transitions, init_state, state_in};
+    for (const void* p : ptrs)
+        if (p && !aligned16(p)) return KDA_ERR_MISALIGNED;
+    return from_cuda(kda::launch_kcp_compose(transitions, n_prev, init_state, state_in, n_seqs, H,
+                                             reinterpret_cast<cudaStream_t>(stream)));
+}
+
+kda_status kda_kcp_finish(const float* state_in, void* o, float* final_state, int B, int64_t T, int H, int dk, int dv,
+                          const int32_t* cu_seqlens, int n_seqs, int64_t max_seqlen, kda_dtype in_dtype,
+                          kda_dtype out_dtype, const void* gate, const float* norm_weight, float eps,
+                          void* workspace, size_t workspace_bytes, void* stream) {
+    return chunk_fwd_impl(nullptr, nullptr, nullptr, nullptr, nullptr, state_in, o, final_state, B, T, H, dk, dv,
+                          cu_seqlens, n_seqs, max_seqlen, in_dtype, out_dtype, 1.f, gate, norm_weight, eps, nullptr, 0,
+                          1, workspace, workspace_bytes, stream, kda::KCP_FINISH, nullptr);
 }
 
 kda_status kda_decode_steps(float* state, const void* q, const void* k, const void* v, const void* log_alpha,
@@ -280,7 +309,8 @@ kda_status kda_profile_enable(int on) {
 }
 
 kda_status kda_profile_read(kda_kernel_time* out, int max_entries, int* n_entries) {
-    static const char* names[kda::PROF_KINDS] = {"intra", "chain", "gate_norm", "decode", "check_cu"};
+    static const char* names[kda::PROF_KINDS] = {"intra",  "chain",    "gate_norm",
+                                                 "decode", "check_cu", "kcp_compose"};
     int launches[kda::PROF_KINDS] = {0};
     double ms[kda::PROF_KINDS] = {0};
     kda_status st = KDA_OK;

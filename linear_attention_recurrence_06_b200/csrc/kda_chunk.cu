@@ -46,6 +46,7 @@
 #include <cudaTypedefs.h>
 #include <string.h>
 
+#include "kda_launch.h"
 #include "kda_profile.h"
 #include "kda_sm100.cuh"
 
@@ -96,6 +97,7 @@ struct ChunkArgs {
     int n_ckpt;                // checkpoints per sequence in `ckpt`
     int segs;                  // segments per sequence (segment-parallel prefill), else 1
     uint8_t* seg_ws;           // segment transition slots [n_seqs][segs][H], segment-parallel only
+    float* trans_out;          // nullable: fp32 segment maps [2][n_seqs][H][dk][dk] (M, then B) instead of slots
 };
 
 // Token range [sb, se) of sequence n, clamped into [0, total tokens].
@@ -902,7 +904,9 @@ constexpr uint32_t PART_TX = CLUSTER * 64 * 4;  // partial-sum bytes each CTA re
 // SEG = 1: per segment, the affine map S -> M_g S + B_g of its chunks; slices 0-3
 //   carry B_g (state from zero), slices 4-7 carry M_g (state from the identity,
 //   Bm dropped); the result is written as a segment slot in the chunk-slot format
-//   (Mlr = -M_g, GamC = 0, Bm = B_g), no outputs;
+//   (Mlr = -M_g, GamC = 0, Bm = B_g), no outputs; with a.trans_out set (one
+//   segment per sequence, the per-device step of context parallelism across
+//   GPUs) M_g and B_g are written there in fp32 instead;
 // SEG = 2: segment g first folds segments 0 .. g-1 into the initial state through
 //   their slots, then walks its own chunks with outputs; the last segment writes
 //   the final state.
@@ -1300,9 +1304,15 @@ chain_kernel(const ChunkArgs a, const __grid_constant__ CUtensorMap gate_map, co
     }
 
     if constexpr (SEG == 1) {
-        // this segment's slot: B_g as the Bm slice jb, -M_g as the Mlr image (rows c,
-        // K columns [32 jb, 32 jb + 32)), GamC = 0
-        if (consumer) {
+        if (consumer && a.trans_out) {
+            // row tid, columns [32 jb, 32 jb + 32) of M_g (first half) or B_g (second half)
+            float* dst = a.trans_out + (trans ? 0 : (size_t)a.n_seqs * H * DK * DV) + st_off;
+#pragma unroll
+            for (int j = 0; j < DVS; j += 4)
+                *reinterpret_cast<float4*>(dst + j) = make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]);
+        } else if (consumer) {
+            // this segment's slot: B_g as the Bm slice jb, -M_g as the Mlr image (rows c,
+            // K columns [32 jb, 32 jb + 32)), GamC = 0
             uint8_t* slot = a.seg_ws + (((size_t)n * a.segs + g) * H + h) * SLOT_BYTES;
             if (!trans) {
                 uint4* dst = reinterpret_cast<uint4*>(slot + SO_B + (size_t)jb * BSL + (size_t)tid * DVS * 2);
@@ -1428,8 +1438,8 @@ cudaError_t chunk_fwd_launch(const void* q, const void* k, const void* v, const 
                              const float* init_state, void* o, float* final_state, int B, int64_t T, int H,
                              const int32_t* cu, int n_seqs, int64_t max_seqlen, bool in_bf16, bool out_bf16,
                              float scale, const void* gate, const float* norm_w, float eps, float* ckpt,
-                             int64_t ckpt_tokens, int segs, void* workspace, size_t ws_bytes, cudaStream_t stream,
-                             int* n_passes, bool* gate_fused) {
+                             int64_t ckpt_tokens, int segs, int kcp_mode, float* trans_out, void* workspace,
+                             size_t ws_bytes, cudaStream_t stream, int* n_passes, bool* gate_fused) {
     cudaError_t err;
     if (!g_attr_set) {
         err = cudaFuncSetAttribute(intra_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, INTRA_SMEM);
@@ -1455,14 +1465,18 @@ cudaError_t chunk_fwd_launch(const void* q, const void* k, const void* v, const 
     uint8_t* ws = reinterpret_cast<uint8_t*>(workspace);
     uint32_t* status = reinterpret_cast<uint32_t*>(ws);
     const bool need_carry = final_state == nullptr;
-    const size_t fixed = chunk_fixed_bytes(N, H, need_carry);
+    // both halves of the cross-device form place the slots after a carry-sized head
+    const size_t fixed = chunk_fixed_bytes(N, H, need_carry || kcp_mode != KCP_NONE);
     float* carry = need_carry ? reinterpret_cast<float*>(ws + 256) : final_state;
     const size_t per_wc = (size_t)N * H * SLOT_BYTES;
     const size_t head = (fixed + 1023) & ~(size_t)1023;
     int wc;
-    if (segs > 1) {  // segment-parallel: one pass over every chunk, segment slots after the chunk slots
+    if (segs > 1 || kcp_mode != KCP_NONE) {
+        // segment-parallel (segment slots after the chunk slots) and the two halves of
+        // the cross-device form: one pass over every chunk
         wc = nchunks_max > 0 ? nchunks_max : 1;
-        if (ws_bytes < head + (size_t)wc * per_wc + chunk_seg_bytes(N, H, segs)) return cudaErrorInvalidValue;
+        if (ws_bytes < head + (size_t)wc * per_wc + (segs > 1 ? chunk_seg_bytes(N, H, segs) : 0))
+            return cudaErrorInvalidValue;
     } else {
         const size_t wc_fit = ws_bytes > head ? (ws_bytes - head) / per_wc : 0;
         wc = (int)(wc_fit < (size_t)nchunks_max ? wc_fit : (size_t)nchunks_max);
@@ -1480,10 +1494,11 @@ cudaError_t chunk_fwd_launch(const void* q, const void* k, const void* v, const 
     a.n_ckpt = ckpt ? (int)(maxlen / ckpt_tokens) : 0;
     a.segs = segs > 1 ? segs : 1;
     a.seg_ws = segs > 1 ? a.ws + (size_t)wc * per_wc : nullptr;
+    a.trans_out = kcp_mode == KCP_TRANSITION ? trans_out : nullptr;
 
     IntraMaps maps;
     memset(&maps, 0, sizeof(maps));
-    if (in_bf16 && total_tokens > 0) {
+    if (in_bf16 && total_tokens > 0 && kcp_mode != KCP_FINISH) {
         if (!make_tile_map(&maps.la, log_alpha, total_tokens, (int64_t)H * DK) ||
             !make_tile_map(&maps.k, k, total_tokens, (int64_t)H * DK) ||
             !make_tile_map(&maps.q, q, total_tokens, (int64_t)H * DK) ||
@@ -1499,9 +1514,9 @@ cudaError_t chunk_fwd_launch(const void* q, const void* k, const void* v, const 
         return cudaErrorInvalidValue;
     if (gate_fused) *gate_fused = fuse;
 
-    err = cudaMemsetAsync(status, 0, 4, stream);
-    if (err != cudaSuccess) return err;
-    if (cu) {
+    // the finishing half reuses the slots (and the status word) of its transition half
+    if (kcp_mode != KCP_FINISH && (err = cudaMemsetAsync(status, 0, 4, stream)) != cudaSuccess) return err;
+    if (cu && kcp_mode != KCP_FINISH) {
         prof_begin(PROF_CHECK, stream);
         check_cu_kernel<<<1, 32, 0, stream>>>(cu, n_seqs, T, max_seqlen, status);
         if ((err = cudaGetLastError()) != cudaSuccess) return err;
@@ -1512,7 +1527,7 @@ cudaError_t chunk_fwd_launch(const void* q, const void* k, const void* v, const 
     for (int ps = 0; ps < npass; ++ps) {
         a.i0 = ps * wc;
         a.first_pass = ps == 0;
-        if (nchunks_max > 0) {
+        if (nchunks_max > 0 && kcp_mode != KCP_FINISH) {
             const int64_t n_items = (int64_t)N * wc * H;
             const unsigned grid = (unsigned)(n_items < g_num_sms ? n_items : g_num_sms);
             prof_begin(PROF_INTRA, stream);
@@ -1522,7 +1537,10 @@ cudaError_t chunk_fwd_launch(const void* q, const void* k, const void* v, const 
             prof_end(PROF_INTRA, stream);
         }
         prof_begin(PROF_CHAIN, stream);
-        if (a.segs == 1) {
+        if (kcp_mode == KCP_TRANSITION) {
+            // M_g and B_g of the whole local sequence (one segment), fp32, no outputs
+            err = launch_chain<1>(a, gate_map, norm_w, eps, out_bf16, false, dim3(2 * NSL, H, N), stream);
+        } else if (a.segs == 1) {
             err = launch_chain<0>(a, gate_map, norm_w, eps, out_bf16, fuse, dim3(NSL, H, N), stream);
         } else {
             // segment transitions (no outputs, no gate), then the segments with outputs

@@ -8,6 +8,7 @@
 //     u = beta (v - S'^T k);   S_new = S' + k u^T;   o = scale * S_new^T q
 // and o = scale * (S'^T q + (k . q) u), so both dot products over the key
 // channels come from ONE pass over S' and the state is read and written once.
+#include "kda_launch.h"
 #include "kda_sm100.cuh"
 
 namespace kda {

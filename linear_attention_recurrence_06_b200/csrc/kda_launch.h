@@ -1,0 +1,35 @@
+// kda_launch.h -- host-side launchers behind the C ABI (internal to libkda).
+#pragma once
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace kda {
+
+// The two halves of the cross-device (context-parallel) prefill of a sequence
+// split over devices.  KCP_TRANSITION runs the chunk-local kernel over every
+// chunk, keeps its slots in the workspace and writes the segment's affine state
+// map (M, B) in fp32; KCP_FINISH walks the kept slots from the initial state
+// that the maps of the earlier segments produced, with outputs.
+enum KcpMode { KCP_NONE = 0, KCP_TRANSITION = 1, KCP_FINISH = 2 };
+
+cudaError_t launch_decode_step(float* state, const void* q, const void* k, const void* v, const void* log_alpha,
+                               const void* beta, void* o, int Bd, int H, bool in_bf16, bool out_bf16, float scale,
+                               const void* gate, const float* norm_w, float eps, int n_steps, float* step_states,
+                               cudaStream_t stream);
+cudaError_t launch_gate_norm(const void* o, const void* g, const float* norm_w, float eps, void* y, int64_t rows,
+                             bool o_bf16, bool g_bf16, bool out_bf16, int num_sms, cudaStream_t stream);
+size_t chunk_slot_bytes();
+size_t chunk_fixed_bytes(int n_seqs, int H, bool need_carry);
+size_t chunk_seg_bytes(int n_seqs, int H, int segs);
+cudaError_t chunk_fwd_launch(const void* q, const void* k, const void* v, const void* log_alpha, const void* beta,
+                             const float* init_state, void* o, float* final_state, int B, int64_t T, int H,
+                             const int32_t* cu, int n_seqs, int64_t max_seqlen, bool in_bf16, bool out_bf16,
+                             float scale, const void* gate, const float* norm_w, float eps, float* ckpt,
+                             int64_t ckpt_tokens, int segs, int kcp_mode, float* trans_out, void* workspace,
+                             size_t ws_bytes, cudaStream_t stream, int* n_passes, bool* gate_fused);
+// state_in = fold of maps 0 .. n_prev-1 of `trans` over init_state (zero when null)
+cudaError_t launch_kcp_compose(const float* trans, int n_prev, const float* init_state, float* state_in, int N, int H,
+                               cudaStream_t stream);
+
+}  // namespace kda

@@ -5,7 +5,8 @@
 #include <cuda_runtime.h>
 
 namespace kda {
-enum ProfKind { PROF_INTRA = 0, PROF_CHAIN = 1, PROF_GATE_NORM = 2, PROF_DECODE = 3, PROF_CHECK = 4, PROF_KINDS = 5 };
+enum ProfKind { PROF_INTRA = 0, PROF_CHAIN = 1, PROF_GATE_NORM = 2, PROF_DECODE = 3, PROF_CHECK = 4, PROF_KCP_COMPOSE = 5,
+               PROF_KINDS = 6 };
 bool prof_enabled();
 void prof_begin(int kind, cudaStream_t stream);
 void prof_end(int kind, cudaStream_t stream);

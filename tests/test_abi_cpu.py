@@ -29,7 +29,8 @@ def test_header_declares_the_entry_points():
     syms = declared_symbols()
     for s in ("kda_chunk_fwd", "kda_chunk_fwd_ckpt", "kda_chunk_fwd_segmented", "kda_decode_step", "kda_decode_steps",
               "kda_gate_norm", "kda_chunk_fwd_segmented_workspace_size",
-              "kda_chunk_fwd_workspace_size",
+              "kda_chunk_fwd_workspace_size", "kda_kcp_workspace_size", "kda_kcp_transition", "kda_kcp_compose",
+              "kda_kcp_finish",
               "kda_query_status", "kda_status_string", "kda_version"):
         assert s in syms
 
@@ -99,6 +100,53 @@ def test_segmented_workspace_size(lib):
     assert lib.kda_chunk_fwd_segmented_workspace_size(4096, 4, 128, 128, 2, 2048, 1, ctypes.byref(seg)) == 0
     assert seg.value == plain_full.value
     assert lib.kda_chunk_fwd_segmented_workspace_size(4096, 4, 128, 128, 2, 2048, 0, ctypes.byref(seg)) == -1
+
+
+def test_kcp_workspace_and_host_validation(lib):
+    import ctypes
+    full = ctypes.c_size_t(0)
+    assert lib.kda_chunk_fwd_workspace_size(4096, 4, 128, 128, 2, 2048, None, ctypes.byref(full)) == 0
+    n = ctypes.c_size_t(0)
+    assert lib.kda_kcp_workspace_size(4096, 4, 128, 128, 2, 2048, ctypes.byref(n)) == 0
+    assert n.value == full.value  # both halves share every chunk's slot
+    assert lib.kda_kcp_workspace_size(4096, 4, 128, 128, 2, 2048, None) == -1
+
+    def tr(**over):
+        a = dict(q=FAKE, k=FAKE, v=FAKE, la=FAKE, beta=FAKE, B=1, T=128, H=2, dk=128, dv=128, cu=None, N=1,
+                 maxlen=128, idt=1, scale=1.0, trans=FAKE, ws=FAKE, wsb=1 << 40)
+        a.update(over)
+        return lib.kda_kcp_transition(a["q"], a["k"], a["v"], a["la"], a["beta"], a["B"], a["T"], a["H"], a["dk"],
+                                      a["dv"], a["cu"], a["N"], a["maxlen"], a["idt"], a["scale"], a["trans"],
+                                      a["ws"], a["wsb"], None)
+    assert tr(trans=None) == -1
+    assert tr(k=None) == -1
+    assert tr(trans=FAKE + 4) == -3
+    assert tr(dk=64) == -2
+    assert tr(H=70000) == -2
+    assert tr(wsb=1024) == -4
+    # the whole-sequence workspace is required (no multi-pass form)
+    lo, hi = ctypes.c_size_t(0), ctypes.c_size_t(0)
+    assert lib.kda_chunk_fwd_workspace_size(128, 2, 128, 128, 1, 128, ctypes.byref(lo), ctypes.byref(hi)) == 0
+    assert tr(wsb=hi.value - 1) == -4
+
+    def fin(**over):
+        a = dict(s_in=None, o=FAKE, fs=None, B=1, T=128, H=2, dk=128, dv=128, cu=None, N=1, maxlen=128, idt=1,
+                 odt=1, gate=None, w=None, eps=1e-6, ws=FAKE, wsb=1 << 40)
+        a.update(over)
+        return lib.kda_kcp_finish(a["s_in"], a["o"], a["fs"], a["B"], a["T"], a["H"], a["dk"], a["dv"], a["cu"],
+                                  a["N"], a["maxlen"], a["idt"], a["odt"], a["gate"], a["w"], a["eps"], a["ws"],
+                                  a["wsb"], None)
+    assert fin(o=None) == -1
+    assert fin(s_in=FAKE + 8) == -3
+    assert fin(ws=None) == -4
+    assert fin(eps=-1.0) == -1
+    assert fin(cu=FAKE, B=2, N=2) == -1
+    # compose: negative count, missing maps, misaligned buffers, unsupported dims
+    assert lib.kda_kcp_compose(FAKE, -1, None, FAKE, 1, 2, 128, 128, None) == -1
+    assert lib.kda_kcp_compose(None, 2, None, FAKE, 1, 2, 128, 128, None) == -1
+    assert lib.kda_kcp_compose(FAKE, 2, None, None, 1, 2, 128, 128, None) == -1
+    assert lib.kda_kcp_compose(FAKE, 2, FAKE + 4, FAKE, 1, 2, 128, 128, None) == -3
+    assert lib.kda_kcp_compose(FAKE, 2, None, FAKE, 1, 2, 64, 128, None) == -2
 
 
 def test_chunk_fwd_host_validation(lib):

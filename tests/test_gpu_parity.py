@@ -225,6 +225,127 @@ def test_prefill_segment_parallel(segments, gate, lens, memory):
         assert rel_l2(fh[n], rfs[n]) <= REL_L2_TOL, f"seq {n} state"
 
 
+# --------------------------------------- context parallelism across devices
+# One process per device in production (linear_attention_recurrence_06_b200.kcp,
+# exchange over NCCL); here the devices are emulated one after another on one
+# GPU: every "rank" runs its transition, the stacked maps stand for the
+# all-gather, then every rank composes its initial state and finishes.  No
+# kernel waits on another.
+
+
+def _kcp_pieces(L, R, ragged):
+    """Cut points of a length-L sequence into R consecutive pieces."""
+    if ragged:  # token boundaries off the chunk grid, one piece empty when R > 2
+        cuts = [0] + [min(L, (L * (2 * r + 1)) // (2 * R) + 7 * r) for r in range(1, R)] + [L]
+        if R > 2:
+            cuts[2] = cuts[1]
+    else:
+        cuts = [(L * r) // R // 64 * 64 for r in range(R)] + [L]
+    return [cuts[r + 1] - cuts[r] for r in range(R)]
+
+
+@pytest.mark.parametrize("R,gate,lens,memory,ragged", [
+    (2, False, [300], "short", False),
+    (3, True, [700, 130], "long", True),
+    (4, False, [1000, 64, 0, 257], "none", True),
+    (8, True, [2048], "long", False),
+])
+def test_kcp_emulated_ranks(R, gate, lens, memory, ragged):
+    """Each sequence cut into R consecutive pieces, piece r on rank r: per-rank
+    transition, stacked maps, compose, finish.  The ranks' outputs, put back in
+    order, and the last rank's final states equal the oracle over the whole
+    sequences; a middle rank's state equals the oracle's state after its piece."""
+    torch = _torch()
+    import linear_attention_recurrence_06_b200 as kda
+    H = 2
+    kw = {"short": {}, "long": dict(la_scale=0.01), "none": dict(la_const=0.0)}[memory]
+    inp = make_prefill(61 + R, lens, H, bf16=True, gate=gate, init=True, **kw)
+    dt = torch.bfloat16
+    pieces = [_kcp_pieces(L, R, ragged) for L in lens]
+    ranks = []
+    for r in range(R):
+        idx, cu = [], [0]
+        for n, L in enumerate(lens):
+            a = int(inp["cu"][n]) + sum(pieces[n][:r])
+            idx.extend(range(a, a + pieces[n][r]))
+            cu.append(cu[-1] + pieces[n][r])
+        idx = np.asarray(idx, dtype=np.int64)
+        Tl = len(idx)
+        loc = lambda x, last: dev(np.ascontiguousarray(inp[x][idx]), dt).view((1, Tl, H) + last)
+        ranks.append(dict(idx=idx, T=Tl, cu=torch.tensor(cu, dtype=torch.int32, device="cuda"),
+                          maxlen=max(int(np.diff(cu).max()), 0),
+                          q=loc("q", (D,)), k=loc("k", (D,)), v=loc("v", (D,)), la=loc("log_alpha", (D,)),
+                          b=loc("beta", ()), g=loc("g", (D,)) if gate else None))
+    for rk in ranks:
+        rk["trans"], rk["ws"] = kda.kcp_transition(rk["q"], rk["k"], rk["v"], rk["la"], rk["b"],
+                                                   cu_seqlens=rk["cu"], max_seqlen=rk["maxlen"])
+    gathered = torch.stack([rk["trans"] for rk in ranks])
+    s0 = dev(inp["s0"], torch.float32)
+    o_all = np.zeros((inp["T"], H, D))
+    for r, rk in enumerate(ranks):
+        s_in = kda.kcp_compose(gathered, r, s0)
+        o, fs = kda.kcp_finish(s_in, rk["ws"], shape=(1, rk["T"], H, D), dtype=dt, cu_seqlens=rk["cu"],
+                               max_seqlen=rk["maxlen"], gate=rk["g"], out_dtype=torch.float32)
+        torch.cuda.synchronize()
+        assert kda.query_status(rk["ws"]) == 0
+        o_all[rk["idx"]] = host(o).reshape(rk["T"], H, D)
+        rk["fs"] = host(fs)
+    ro, rfs = oracle_prefill(inp, gate=gate)
+    check(o_all, ranks[-1]["fs"], ro, rfs)
+    for n, L in enumerate(lens):
+        sl = slice(inp["cu"][n], inp["cu"][n + 1])
+        if L:
+            assert rel_l2(o_all[sl], ro[sl]) <= REL_L2_TOL, f"seq {n}"
+    # rank R//2's state: the oracle's state after pieces 0 .. R//2 of each sequence
+    m = R // 2
+    for n, L in enumerate(lens):
+        end = int(inp["cu"][n]) + sum(pieces[n][:m + 1])
+        sl = slice(int(inp["cu"][n]), end)
+        _, ref = oracle.kda_recurrent(inp["q"][sl], inp["k"][sl], inp["v"][sl], inp["log_alpha"][sl],
+                                      inp["beta"][sl], inp["s0"][n:n + 1])
+        assert rel_l2(ranks[m]["fs"][n], ref[0]) <= REL_L2_TOL, f"seq {n} state after rank {m}"
+
+
+def test_kcp_transition_is_the_oracle_segment_map():
+    """(M, B) of kcp_transition against the oracle's segment transition, per
+    head, on a ragged segment with long memory (M far from zero: the erase term
+    shrinks it as the segment grows)."""
+    torch = _torch()
+    import linear_attention_recurrence_06_b200 as kda
+    H, L = 2, 150
+    inp = make_prefill(71, [L], H, bf16=True, la_scale=0.01)
+    dt = torch.bfloat16
+    q, k, v, la = (dev(inp[x], dt).view(1, L, H, D) for x in ("q", "k", "v", "log_alpha"))
+    b = dev(inp["beta"], dt).view(1, L, H)
+    trans, _ = kda.kcp_transition(q, k, v, la, b)
+    torch.cuda.synchronize()
+    t = host(trans)
+    for h in range(H):
+        M, B = oracle.segment_transition(inp["k"][:, h], inp["v"][:, h], inp["log_alpha"][:, h], inp["beta"][:, h])
+        assert rel_l2(t[0, 0, h], M) <= REL_L2_TOL, f"M head {h}"
+        assert rel_l2(t[1, 0, h], B) <= REL_L2_TOL, f"B head {h}"
+        assert np.abs(M).max() > 0.1  # the segment map carries the state
+
+
+def test_kcp_compose_is_the_fold():
+    """kcp_compose against the fp64 fold S <- M_j S + B_j of the same fp32 maps."""
+    torch = _torch()
+    import linear_attention_recurrence_06_b200 as kda
+    R, N, H = 5, 2, 3
+    rng = np.random.default_rng(5)
+    trans = rng.standard_normal((R, 2, N, H, D, D)).astype(np.float32)
+    trans[:, 0] /= np.sqrt(D)  # spectral radius about 1
+    s0 = rng.standard_normal((N, H, D, D)).astype(np.float32)
+    g = torch.from_numpy(trans).cuda()
+    for n_prev in (0, 1, 4):
+        for init in (None, s0):
+            out = host(kda.kcp_compose(g, n_prev, None if init is None else torch.from_numpy(init).cuda()))
+            ref = np.zeros((N, H, D, D)) if init is None else init.astype(np.float64)
+            for j in range(n_prev):
+                ref = np.einsum("nhik,nhkc->nhic", trans[j, 0].astype(np.float64), ref) + trans[j, 1]
+            assert rel_l2(out, ref) <= 1e-5 if n_prev else np.array_equal(out, ref)
+
+
 def test_prefill_multi_pass_workspace():
     """A workspace that holds one chunk per sequence forces one pass per chunk:
     the state carried between passes must give the same result."""
