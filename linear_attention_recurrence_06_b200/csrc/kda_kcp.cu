@@ -22,8 +22,10 @@ constexpr int CS = 32;        // state columns per CTA
 constexpr int CP_THREADS = 256;
 
 // gathered maps: trans[r][0][n][h] = M_r (dk x dk), trans[r][1][n][h] = B_r (dk x dv), fp32 row-major.
-// One CTA = columns [32 js, 32 js + 32) of one (sequence, head) state; thread t
-// owns row t / 2, columns 16 (t % 2) .. + 16 of that slice.
+// One CTA = columns [32 js, 32 js + 32) of one (sequence, head) state.  Thread t
+// owns rows 4 (t / 8) .. + 4 and columns 4 (t % 8) .. + 4 of that slice: per key
+// index k one 16-byte shared load of S[k] feeds 16 FMAs, and the four M rows
+// stream from global memory (L1-resident across the 8 threads that share them).
 __global__ void __launch_bounds__(CP_THREADS)
 kcp_compose_kernel(const float* __restrict__ trans, int n_prev, const float* __restrict__ init_state,
                    float* __restrict__ state_in, int N, int H) {
@@ -38,40 +40,40 @@ kcp_compose_kernel(const float* __restrict__ trans, int n_prev, const float* __r
                                   : make_float4(0.f, 0.f, 0.f, 0.f);
     }
     __syncthreads();
-    const int i = t >> 1, ch = t & 1;
+    const int i0 = 4 * (t >> 3), cq = t & 7;
     int cur = 0;
     for (int j = 0; j < n_prev; ++j) {
         const float* M = trans + (size_t)j * 2 * half + mat;
         const float* Bj = M + half;
-        float acc[16];
-        const float4* b4 = reinterpret_cast<const float4*>(Bj + (size_t)i * D + col0 + 16 * ch);
+        float acc[4][4];
 #pragma unroll
-        for (int c4 = 0; c4 < 4; ++c4) {
-            const float4 b = b4[c4];
-            acc[4 * c4] = b.x; acc[4 * c4 + 1] = b.y; acc[4 * c4 + 2] = b.z; acc[4 * c4 + 3] = b.w;
+        for (int r = 0; r < 4; ++r) {
+            const float4 b = *reinterpret_cast<const float4*>(Bj + (size_t)(i0 + r) * D + col0 + 4 * cq);
+            acc[r][0] = b.x; acc[r][1] = b.y; acc[r][2] = b.z; acc[r][3] = b.w;
         }
-        const float4* m4 = reinterpret_cast<const float4*>(M + (size_t)i * D);
-#pragma unroll 4
+#pragma unroll 2
         for (int kk = 0; kk < D / 4; ++kk) {
-            const float4 m = m4[kk];
-            const float mv[4] = {m.x, m.y, m.z, m.w};
+            float m[4][4];  // M[i0 + r][4 kk + u]
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
+                const float4 v = *reinterpret_cast<const float4*>(M + (size_t)(i0 + r) * D + 4 * kk);
+                m[r][0] = v.x; m[r][1] = v.y; m[r][2] = v.z; m[r][3] = v.w;
+            }
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
-                const float4* srow = sS[cur][4 * kk + u] + 4 * ch;
+                const float4 s = sS[cur][4 * kk + u][cq];
 #pragma unroll
-                for (int c4 = 0; c4 < 4; ++c4) {
-                    const float4 s = srow[c4];
-                    acc[4 * c4] = fmaf(mv[u], s.x, acc[4 * c4]);
-                    acc[4 * c4 + 1] = fmaf(mv[u], s.y, acc[4 * c4 + 1]);
-                    acc[4 * c4 + 2] = fmaf(mv[u], s.z, acc[4 * c4 + 2]);
-                    acc[4 * c4 + 3] = fmaf(mv[u], s.w, acc[4 * c4 + 3]);
+                for (int r = 0; r < 4; ++r) {
+                    acc[r][0] = fmaf(m[r][u], s.x, acc[r][0]);
+                    acc[r][1] = fmaf(m[r][u], s.y, acc[r][1]);
+                    acc[r][2] = fmaf(m[r][u], s.z, acc[r][2]);
+                    acc[r][3] = fmaf(m[r][u], s.w, acc[r][3]);
                 }
             }
         }
         // the other buffer was last read before the previous step's barrier
 #pragma unroll
-        for (int c4 = 0; c4 < 4; ++c4)
-            sS[cur ^ 1][i][4 * ch + c4] = make_float4(acc[4 * c4], acc[4 * c4 + 1], acc[4 * c4 + 2], acc[4 * c4 + 3]);
+        for (int r = 0; r < 4; ++r) sS[cur ^ 1][i0 + r][cq] = make_float4(acc[r][0], acc[r][1], acc[r][2], acc[r][3]);
         __syncthreads();
         cur ^= 1;
     }
