@@ -519,17 +519,26 @@ def recorded_traffic(kernel: str, units: int):
         rec = json.load(open(p)).get(kernel)
     except Exception:
         return None
-    if not rec or rec.get("sources_sha256") != sources_sha256():
+    if not rec or rec.get("sources_sha256") != sources_sha256(kernel):
         return None
     return rec["dram_bytes_per_unit"] * units
 
 
-def sources_sha256() -> str:
+# the source files each recorded kernel is built from (a change to any of them
+# voids its recorded traffic)
+KERNEL_SOURCES = {
+    "kda_chunk_fwd": ("kda_chunk.cu", "kda_sm100.cuh"),
+    "intra_kernel": ("kda_chunk.cu", "kda_sm100.cuh"),
+    "chain_kernel": ("kda_chunk.cu", "kda_sm100.cuh"),
+    "decode_step_kernel": ("kda_decode.cu", "kda_sm100.cuh"),
+}
+
+
+def sources_sha256(kernel: str) -> str:
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "linear_attention_recurrence_06_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
-        if f.endswith((".cu", ".cuh", ".h")):
-            h.update(open(os.path.join(csrc, f), "rb").read())
+    for f in KERNEL_SOURCES[kernel]:
+        h.update(open(os.path.join(csrc, f), "rb").read())
     return h.hexdigest()
 
 
