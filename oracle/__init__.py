@@ -54,6 +54,9 @@ def _setup(lib):
     lib.oracle_kda_segment_transition.argtypes = [f32p, f32p, f32p, f32p, ci, ci, ci, cd,
                                                   f64p, f64p]
     lib.oracle_kda_segment_transition.restype = ci
+    lib.oracle_kda_recurrent_bwd.argtypes = [f32p, f32p, f32p, f32p, f32p, f64p, i64p, f64p, f64p,
+                                             ci, ci, ci, ci, cd, cd, f64p, f64p, f64p, f64p, f64p, f64p, ci]
+    lib.oracle_kda_recurrent_bwd.restype = ci
     lib.oracle_gate_norm.argtypes = [f64p, f32p, f32p, cd, ctypes.c_int64, ci, f64p]
     lib.oracle_gate_norm.restype = ci
     return lib
@@ -119,6 +122,43 @@ def kda_recurrent(q, k, v, log_alpha, beta, init_state=None, cu_seqlens=None, *,
     if return_threads:
         return o, fs, nt
     return o, fs
+
+
+def kda_recurrent_bwd(q, k, v, log_alpha, beta, d_o, init_state=None, d_final=None, cu_seqlens=None, *,
+                      scale: float = 1.0, la_floor: float = LOG_ALPHA_FLOOR, n_threads: int = 0):
+    """Exact gradients of kda_recurrent (fp64, reverse sweep over the tokens).
+
+    d_o: [T, H, dv] (dL/do); d_final: [N, H, dk, dv] or None (dL/d final state).
+    Returns dict with dq, dk [T,H,dk], dv [T,H,dv], dbeta [T,H], dlog_alpha
+    [T,H,dk] and d_init [N,H,dk,dv] (all fp64).  The clamp passes the gradient
+    where log_alpha >= la_floor.
+    """
+    T, H, dk = q.shape
+    dv = v.shape[-1]
+    cu = _cu(cu_seqlens, T)
+    N = len(cu) - 1
+    q, qp = _f32(q); k, kp = _f32(k); v, vp = _f32(v)
+    la, lp = _f32(log_alpha); b, bp = _f32(beta)
+    do, dop = _f64(d_o)
+    P = lambda a: a.ctypes.data_as(ctypes.POINTER(ctypes.c_double))
+    null = ctypes.POINTER(ctypes.c_double)()
+    if init_state is not None:
+        s0, s0p = _f64(init_state)
+    else:
+        s0, s0p = None, null
+    if d_final is not None:
+        dfin, dfp = _f64(d_final)
+    else:
+        dfin, dfp = None, null
+    out = dict(dq=np.zeros((T, H, dk)), dk=np.zeros((T, H, dk)), dv=np.zeros((T, H, dv)),
+               dbeta=np.zeros((T, H)), dlog_alpha=np.zeros((T, H, dk)), d_init=np.zeros((N, H, dk, dv)))
+    nt = _L().oracle_kda_recurrent_bwd(qp, kp, vp, lp, bp, s0p, cu.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)),
+                                       dop, dfp, N, H, dk, dv, scale, la_floor, P(out["dq"]), P(out["dk"]),
+                                       P(out["dv"]), P(out["dbeta"]), P(out["dlog_alpha"]), P(out["d_init"]),
+                                       n_threads)
+    if nt < 0:
+        raise ValueError("oracle_kda_recurrent_bwd: bad arguments")
+    return out
 
 
 def kda_chunkwise(q, k, v, log_alpha, beta, init_state=None, cu_seqlens=None, *, chunk: int = 64,

@@ -198,6 +198,157 @@ OR_API int oracle_kda_recurrent(const float* q, const float* k, const float* v,
 }
 
 /* ------------------------------------------------------------------------ */
+/* backward of the token-by-token recurrence (reverse-mode, fp64)            */
+/* ------------------------------------------------------------------------ */
+/*
+ * The pages give no backward pass.  This is the exact gradient of the forward
+ * definition above, taken step by step in reverse: given dL/do_t and dL/dS_T
+ * it returns dL/dq, dL/dk, dL/dv, dL/dbeta, dL/dlog_alpha and dL/dS_0.  The
+ * clamp l = max(log_alpha, floor) passes the gradient where log_alpha >= floor
+ * (equality included) and blocks it below.  Per token, with r = v - S'^T k,
+ * u = beta r and G = dL/dS_t (accumulated from later tokens):
+ *     G     += scale q do^T                      dq  = scale S_t do
+ *     dk     = G u                               du  = G^T k
+ *     dbeta  = du . r                            dr  = beta du,  dv = dr
+ *     dS'    = G - k dr^T                        dk -= S' dr
+ *     dl     = alpha o rowsum(dS' o S_{t-1})     G  <- Diag(alpha) dS'
+ * The forward states S_{t-1} are kept for the whole sequence (test sizes only).
+ * Pinned by central finite differences of the forward (test_oracle_pins.py).
+ */
+typedef struct {
+    const float *q, *k, *v, *log_alpha, *beta;
+    const double* init_state;
+    const double *d_o, *d_final;
+    const int64_t* cu;
+    int N, H, dk, dv;
+    double scale, la_floor;
+    double *dq, *dk_out, *dv_out, *dbeta, *dla, *d_init;
+} bwd_ctx;
+
+static void bwd_unit(void* vctx, int64_t unit) {
+    const bwd_ctx* c = (const bwd_ctx*)vctx;
+    const int n = (int)(unit / c->H), h = (int)(unit % c->H);
+    const int dk = c->dk, dv = c->dv, H = c->H;
+    const int64_t t0 = c->cu[n], L = c->cu[n + 1] - c->cu[n];
+    const size_t SZ = (size_t)dk * dv;
+    const size_t st_off = ((size_t)n * H + h) * SZ;
+    /* forward: the state before every token, u and r of every token */
+    double* Sb = malloc(sizeof(double) * SZ * (size_t)(L + 1));
+    double* R = malloc(sizeof(double) * (size_t)dv * (size_t)(L > 0 ? L : 1));
+    double* alpha = malloc(sizeof(double) * (size_t)dk * (size_t)(L > 0 ? L : 1));
+    if (c->init_state) memcpy(Sb, c->init_state + st_off, sizeof(double) * SZ);
+    else memset(Sb, 0, sizeof(double) * SZ);
+    for (int64_t tt = 0; tt < L; ++tt) {
+        const int64_t t = t0 + tt;
+        const float* kt = c->k + ((size_t)t * H + h) * dk;
+        const float* vt = c->v + ((size_t)t * H + h) * dv;
+        const float* lt = c->log_alpha + ((size_t)t * H + h) * dk;
+        const double bt = (double)c->beta[(size_t)t * H + h];
+        const double* Sp = Sb + SZ * (size_t)tt;
+        double* Sn = Sb + SZ * (size_t)(tt + 1);
+        double* al = alpha + (size_t)dk * tt;
+        double* r = R + (size_t)dv * tt;
+        for (int i = 0; i < dk; ++i) {
+            double l = (double)lt[i];
+            if (l < c->la_floor) l = c->la_floor;
+            al[i] = exp(l);
+        }
+        for (int i = 0; i < dk; ++i)
+            for (int j = 0; j < dv; ++j) Sn[(size_t)i * dv + j] = al[i] * Sp[(size_t)i * dv + j];
+        for (int j = 0; j < dv; ++j) {
+            double sk = 0.0;
+            for (int i = 0; i < dk; ++i) sk += Sn[(size_t)i * dv + j] * (double)kt[i];
+            r[j] = (double)vt[j] - sk;
+        }
+        for (int i = 0; i < dk; ++i)
+            for (int j = 0; j < dv; ++j) Sn[(size_t)i * dv + j] += (double)kt[i] * bt * r[j];
+    }
+    /* reverse sweep */
+    double* G = malloc(sizeof(double) * SZ);
+    double* dSp = malloc(sizeof(double) * SZ);
+    double* du = malloc(sizeof(double) * (size_t)dv);
+    double* dr = malloc(sizeof(double) * (size_t)dv);
+    if (c->d_final) memcpy(G, c->d_final + st_off, sizeof(double) * SZ);
+    else memset(G, 0, sizeof(double) * SZ);
+    for (int64_t tt = L - 1; tt >= 0; --tt) {
+        const int64_t t = t0 + tt;
+        const size_t ti = (size_t)t * H + h;
+        const float* qt = c->q + ti * dk;
+        const float* kt = c->k + ti * dk;
+        const float* lt = c->log_alpha + ti * dk;
+        const double bt = (double)c->beta[ti];
+        const double* dot = c->d_o + ti * dv;
+        const double* Sprev = Sb + SZ * (size_t)tt;      /* S_{t-1} */
+        const double* St = Sb + SZ * (size_t)(tt + 1);   /* S_t */
+        const double* al = alpha + (size_t)dk * tt;
+        const double* r = R + (size_t)dv * tt;
+        /* o_t = scale S_t^T q_t */
+        for (int i = 0; i < dk; ++i) {
+            double acc = 0.0;
+            for (int j = 0; j < dv; ++j) acc += St[(size_t)i * dv + j] * dot[j];
+            c->dq[ti * dk + i] = c->scale * acc;
+            for (int j = 0; j < dv; ++j) G[(size_t)i * dv + j] += c->scale * (double)qt[i] * dot[j];
+        }
+        /* S_t = S' + k u^T */
+        for (int j = 0; j < dv; ++j) {
+            double acc = 0.0;
+            for (int i = 0; i < dk; ++i) acc += G[(size_t)i * dv + j] * (double)kt[i];
+            du[j] = acc;
+        }
+        double db = 0.0;
+        for (int j = 0; j < dv; ++j) {
+            db += du[j] * r[j];
+            dr[j] = bt * du[j];
+            c->dv_out[ti * dv + j] = dr[j];
+        }
+        c->dbeta[ti] = db;
+        for (int i = 0; i < dk; ++i) {
+            double acc_u = 0.0, acc_r = 0.0;
+            for (int j = 0; j < dv; ++j) {
+                const double sp = al[i] * Sprev[(size_t)i * dv + j];   /* S' */
+                acc_u += G[(size_t)i * dv + j] * bt * r[j];
+                acc_r += sp * dr[j];
+            }
+            c->dk_out[ti * dk + i] = acc_u - acc_r;
+        }
+        /* S' = Diag(alpha) S_{t-1};  dS' = G - k dr^T */
+        for (int i = 0; i < dk; ++i) {
+            double da = 0.0;
+            for (int j = 0; j < dv; ++j) {
+                const double g = G[(size_t)i * dv + j] - (double)kt[i] * dr[j];
+                dSp[(size_t)i * dv + j] = g;
+                da += g * Sprev[(size_t)i * dv + j];
+            }
+            const double pass = ((double)lt[i] >= c->la_floor) ? 1.0 : 0.0;
+            c->dla[ti * dk + i] = pass * al[i] * da;
+        }
+        for (int i = 0; i < dk; ++i)
+            for (int j = 0; j < dv; ++j) G[(size_t)i * dv + j] = al[i] * dSp[(size_t)i * dv + j];
+    }
+    if (c->d_init) memcpy(c->d_init + st_off, G, sizeof(double) * SZ);
+    free(Sb); free(R); free(alpha); free(G); free(dSp); free(du); free(dr);
+}
+
+/* Backward of oracle_kda_recurrent (erase form) over N packed sequences.
+ * d_o [T,H,dv]; d_final [N,H,dk,dv] or NULL (zero).  Outputs (fp64): dq, dk
+ * [T,H,dk], dv [T,H,dv], dbeta [T,H], dlog_alpha [T,H,dk], d_init [N,H,dk,dv]
+ * or NULL.  Returns the number of threads used, or -1 on bad arguments. */
+OR_API int oracle_kda_recurrent_bwd(const float* q, const float* k, const float* v,
+                                    const float* log_alpha, const float* beta,
+                                    const double* init_state, const int64_t* cu_seqlens,
+                                    const double* d_o, const double* d_final,
+                                    int N, int H, int dk, int dv, double scale, double la_floor,
+                                    double* dq, double* dk_out, double* dv_out, double* dbeta,
+                                    double* dlog_alpha, double* d_init, int n_threads) {
+    if (N < 0 || H <= 0 || dk <= 0 || dv <= 0) return -1;
+    for (int n = 0; n < N; ++n)
+        if (cu_seqlens[n + 1] < cu_seqlens[n]) return -1;
+    bwd_ctx c = {q, k, v, log_alpha, beta, init_state, d_o, d_final, cu_seqlens, N, H, dk, dv,
+                 scale, la_floor, dq, dk_out, dv_out, dbeta, dlog_alpha, d_init};
+    return run_units(bwd_unit, &c, (int64_t)N * H, n_threads);
+}
+
+/* ------------------------------------------------------------------------ */
 /* naive chunkwise form (fp64), the same result reached by matrix products   */
 /* inside each chunk and a recurrence between chunks ([chunk]).              */
 /* ------------------------------------------------------------------------ */

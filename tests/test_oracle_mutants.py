@@ -58,3 +58,46 @@ def test_pins_catch_mutant(tmp_path, name, old, new):
     finally:
         oracle._lib = saved
     assert caught >= 1, f"no pin caught mutant {name}"
+
+
+# mistakes in the backward sweep, caught by the finite-difference and closed-form pins
+BWD_MUTANTS = [
+    ("dbeta_scaled_by_beta", "db += du[j] * r[j];", "db += du[j] * r[j] * bt;"),
+    ("state_gradient_not_decayed", "G[(size_t)i * dv + j] = al[i] * dSp[(size_t)i * dv + j];",
+     "G[(size_t)i * dv + j] = dSp[(size_t)i * dv + j];"),
+    ("erase_term_dropped_from_dk", "c->dk_out[ti * dk + i] = acc_u - acc_r;", "c->dk_out[ti * dk + i] = acc_u;"),
+    ("clamp_passes_everything", "((double)lt[i] >= c->la_floor) ? 1.0 : 0.0", "1.0"),
+    ("dq_from_decayed_previous_state", "for (int j = 0; j < dv; ++j) acc += St[(size_t)i * dv + j] * dot[j];",
+     "for (int j = 0; j < dv; ++j) acc += al[i] * Sprev[(size_t)i * dv + j] * dot[j];"),
+    ("erase_gradient_sign", "const double g = G[(size_t)i * dv + j] - (double)kt[i] * dr[j];",
+     "const double g = G[(size_t)i * dv + j] + (double)kt[i] * dr[j];"),
+]
+
+BWD_CHECKS = [
+    lambda: pins.test_backward_matches_finite_differences(),
+    lambda: pins.test_backward_clamp_blocks_gradient(),
+    lambda: pins.test_backward_of_one_token_closed_form(),
+]
+
+
+@pytest.mark.parametrize("name,old,new", BWD_MUTANTS, ids=[m[0] for m in BWD_MUTANTS])
+def test_backward_pins_catch_mutant(tmp_path, name, old, new):
+    src = open(SRC).read()
+    assert src.count(old) == 1, f"mutation anchor not found: {name}"
+    c_path = tmp_path / "mut.c"
+    so_path = tmp_path / "libmut.so"
+    c_path.write_text(src.replace(old, new, 1))
+    subprocess.run(["gcc", "-O1", "-std=c11", "-fPIC", "-shared", "-o", str(so_path), str(c_path),
+                    "-lm", "-lpthread"], check=True)
+    saved = oracle._lib
+    oracle._lib = oracle._setup(ctypes.CDLL(str(so_path)))
+    caught = 0
+    try:
+        for chk in BWD_CHECKS:
+            try:
+                chk()
+            except AssertionError:
+                caught += 1
+    finally:
+        oracle._lib = saved
+    assert caught >= 1, f"no pin caught mutant {name}"

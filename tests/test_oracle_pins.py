@@ -397,3 +397,95 @@ def test_heads_subset_matches_full():
     np.testing.assert_array_equal(o2[:, 1:3], o[:, 1:3])
     np.testing.assert_array_equal(fs2[:, 1:3], fs[:, 1:3])
     assert np.all(o2[:, 0] == 0) and np.all(o2[:, 3] == 0)
+
+
+# ------------------------------------------- backward (exact gradients, I11)
+# The pages give no backward; the oracle's is the exact gradient of its forward.
+# Pinned by central finite differences of the fp64 forward: a scalar loss
+#   L = sum(d_o * o) + sum(d_final * S_final)
+# is perturbed in every element of every input; the difference quotient uses
+# the perturbation actually representable in float32.
+
+BWD_LENS = [5, 4]
+BWD_SCALE = 0.7
+
+
+def _bwd_case(seed=31, la_lo=-1.5):
+    rng = np.random.default_rng(seed)
+    T, H, dk, dv = sum(BWD_LENS), 2, 4, 3
+    q, k, v, la, b = rand_inputs(T, H, dk, dv, rng, unit_k=False, la_lo=la_lo)
+    s0 = rng.standard_normal((len(BWD_LENS), H, dk, dv))
+    d_o = rng.standard_normal((T, H, dv))
+    d_fin = rng.standard_normal((len(BWD_LENS), H, dk, dv))
+    cu = np.cumsum([0] + BWD_LENS)
+    return dict(q=q, k=k, v=v, log_alpha=la, beta=b), s0, d_o, d_fin, cu
+
+
+def _loss(x, s0, d_o, d_fin, cu):
+    o, fs = oracle.kda_recurrent(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], s0, cu, scale=BWD_SCALE,
+                                 n_threads=1)
+    return float((o * d_o).sum() + (fs * d_fin).sum())
+
+
+def _fd(x, name, idx, s0, d_o, d_fin, cu, h=1e-3):
+    base = x[name][idx]
+    hi, lo = np.float32(base + h), np.float32(base - h)
+    xp = {kk: vv.copy() for kk, vv in x.items()}
+    xp[name][idx] = hi
+    lp = _loss(xp, s0, d_o, d_fin, cu)
+    xp[name][idx] = lo
+    lm = _loss(xp, s0, d_o, d_fin, cu)
+    return (lp - lm) / (float(hi) - float(lo))
+
+
+def test_backward_matches_finite_differences():
+    x, s0, d_o, d_fin, cu = _bwd_case()
+    g = oracle.kda_recurrent_bwd(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], d_o, s0, d_fin, cu,
+                                 scale=BWD_SCALE, n_threads=1)
+    names = dict(q="dq", k="dk", v="dv", log_alpha="dlog_alpha", beta="dbeta")
+    for name, gname in names.items():
+        for idx in np.ndindex(*x[name].shape):
+            fd = _fd(x, name, idx, s0, d_o, d_fin, cu)
+            an = g[gname][idx]
+            assert abs(fd - an) <= 2e-5 * max(1.0, abs(an)), f"{gname}{idx}: fd {fd} analytic {an}"
+    # initial state (fp64 input): plain central differences
+    for idx in np.ndindex(*s0.shape):
+        sp, sm = s0.copy(), s0.copy()
+        sp[idx] += 1e-4
+        sm[idx] -= 1e-4
+        fd = (_loss(x, sp, d_o, d_fin, cu) - _loss(x, sm, d_o, d_fin, cu)) / 2e-4
+        assert abs(fd - g["d_init"][idx]) <= 1e-6 * max(1.0, abs(fd)), f"d_init{idx}"
+
+
+def test_backward_clamp_blocks_gradient():
+    """Log-decays below the floor get no gradient (the clamp is flat there);
+    above it the gradient matches finite differences."""
+    x, s0, d_o, d_fin, cu = _bwd_case(seed=32, la_lo=-8.0)
+    g = oracle.kda_recurrent_bwd(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], d_o, s0, d_fin, cu,
+                                 scale=BWD_SCALE, n_threads=1)
+    below = x["log_alpha"] < -5.0 - 1e-3
+    above = x["log_alpha"] > -5.0 + 1e-3
+    assert below.any() and above.any()
+    assert np.all(g["dlog_alpha"][below] == 0.0)
+    for idx in zip(*np.nonzero(above)):
+        fd = _fd(x, "log_alpha", idx, s0, d_o, d_fin, cu)
+        assert abs(fd - g["dlog_alpha"][idx]) <= 2e-5 * max(1.0, abs(fd))
+    assert np.abs(g["dlog_alpha"][above]).max() > 1e-4  # the comparison is not vacuous
+
+
+def test_backward_of_one_token_closed_form():
+    """One token from a zero state: o = scale (q.k) beta v, so dv = scale beta (q.k) d_o,
+    dbeta = scale (q.k) (v.d_o), dq = scale beta (v.d_o) k; the decay does not act
+    (zero state), so dlog_alpha = 0."""
+    rng = np.random.default_rng(33)
+    q, k, v, la, b = rand_inputs(1, 1, 5, 3, rng, unit_k=False)
+    d_o = rng.standard_normal((1, 1, 3))
+    g = oracle.kda_recurrent_bwd(q, k, v, la, b, d_o, scale=0.5, n_threads=1)
+    qk = float(np.dot(q[0, 0].astype(np.float64), k[0, 0]))
+    vd = float(np.dot(v[0, 0].astype(np.float64), d_o[0, 0]))
+    bb = float(b[0, 0])
+    np.testing.assert_allclose(g["dv"][0, 0], 0.5 * bb * qk * d_o[0, 0], rtol=1e-12)
+    np.testing.assert_allclose(g["dbeta"][0, 0], 0.5 * qk * vd, rtol=1e-12)
+    np.testing.assert_allclose(g["dq"][0, 0], 0.5 * bb * vd * k[0, 0].astype(np.float64), rtol=1e-12)
+    np.testing.assert_allclose(g["dk"][0, 0], 0.5 * bb * vd * q[0, 0].astype(np.float64), rtol=1e-12)
+    assert np.all(g["dlog_alpha"] == 0.0)
