@@ -259,6 +259,43 @@ KDA_API kda_status kda_kcp_finish(const float* state_in, void* o, float* final_s
                                   void* stream);
 
 /*
+ * kda_chunk_bwd -- gradients of kda_chunk_fwd (without the gate) with respect
+ * to q, k, v, log_alpha, beta and the initial state, given dL/do and dL/d(final
+ * state).  The pages give no backward pass; this is the exact gradient of the
+ * forward definition, computed chunkwise: the forward walk is recomputed (chunk
+ * slots and chunk-boundary states kept in the workspace), a reverse walk forms
+ * dL/d(state) at every chunk end, and a chunk-local kernel forms the token
+ * gradients.  The clamp l = max(log_alpha, -5) passes the gradient where
+ * log_alpha >= -5 and blocks it below.
+ *
+ *   q, k, v, log_alpha, beta, init_state, B, T, H, cu_seqlens, n_seqs,
+ *   max_seqlen, in_dtype, scale   as kda_chunk_fwd
+ *   d_o           [B, T, H, dv] in_dtype: dL/do (device)
+ *   d_final_state [N, H, dk, dv] fp32 or NULL (zero)
+ *   dq, dk, dlog_alpha [B, T, H, dk] fp32; dv [B, T, H, dv] fp32; dbeta [B, T, H]
+ *                 fp32 (outputs, caller-owned device memory)
+ *   d_init_state  [N, H, dk, dv] fp32 or NULL: dL/d(initial state)
+ *   workspace     >= kda_chunk_bwd_workspace_size bytes, 256-byte aligned
+ *
+ * Errors as kda_chunk_fwd; device-side ones land in the workspace status word.
+ */
+KDA_API kda_status kda_chunk_bwd(const void* q, const void* k, const void* v, const void* log_alpha,
+                                 const void* beta, const float* init_state, const void* d_o,
+                                 const float* d_final_state, float* dq, float* dk, float* dv,
+                                 float* dlog_alpha, float* dbeta, float* d_init_state, int B, int64_t T,
+                                 int H, int dk_dim, int dv_dim, const int32_t* cu_seqlens, int n_seqs,
+                                 int64_t max_seqlen, kda_dtype in_dtype, float scale, void* workspace,
+                                 size_t workspace_bytes, void* stream);
+
+/*
+ * kda_chunk_bwd_workspace_size -- workspace bytes of kda_chunk_bwd: the
+ * forward's whole-sequence workspace plus one fp32 state per chunk boundary and
+ * per chunk (arguments as kda_chunk_fwd_workspace_size).
+ */
+KDA_API kda_status kda_chunk_bwd_workspace_size(int64_t T, int H, int dk, int dv, int n_seqs, int64_t max_seqlen,
+                                                size_t* bytes);
+
+/*
  * kda_decode_step -- one recurrent step for Bd independent sequences
  * ("decode uses the recurrent form", chunkwise-algorithm item of the K3
  * article summaries).  The state is read once and written once, in place.

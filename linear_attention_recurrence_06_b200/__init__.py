@@ -12,6 +12,7 @@ Entry points (same names as the C ABI):
   decode_step    one recurrent step per sequence, state updated in place
   gate_norm      per-head RMSNorm over dv times sigmoid output gate
   workspace_size bytes the prefill needs
+  chunk_bwd      gradients of the prefill (without the gate)
   kcp_transition / kcp_compose / kcp_finish
                  the per-device steps of context parallelism across devices
                  (the exchange between them is in ``kcp.py``)
@@ -85,6 +86,11 @@ def load_library(path: str | None = None):
     lib.kda_kcp_finish.restype = i32
     lib.kda_kcp_finish.argtypes = [vp, vp, vp, i32, i64, i32, i32, i32, vp, i32, i64, i32, i32, vp, vp, f32, vp, sz,
                                    vp]
+    lib.kda_chunk_bwd_workspace_size.restype = i32
+    lib.kda_chunk_bwd_workspace_size.argtypes = [i64, i32, i32, i32, i32, i64, ctypes.POINTER(sz)]
+    lib.kda_chunk_bwd.restype = i32
+    lib.kda_chunk_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, i64, i32, i32, i32,
+                                  vp, i32, i64, i32, f32, vp, sz, vp]
     lib.kda_decode_step.restype = i32
     lib.kda_decode_step.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, f32, vp, vp, f32, vp]
     lib.kda_decode_steps.restype = i32
@@ -225,6 +231,46 @@ def chunk_fwd(q, k, v, log_alpha, beta, initial_state=None, *, cu_seqlens=None, 
     if st != KDA_OK:
         raise KdaError(st, "kda_chunk_fwd_ckpt")
     return o, fs, checkpoints
+
+
+def bwd_workspace_size(T: int, H: int, n_seqs: int, max_seqlen: int, dk: int = HEAD_DIM, dv: int = HEAD_DIM) -> int:
+    """Workspace bytes of chunk_bwd."""
+    n = ctypes.c_size_t(0)
+    st = load_library().kda_chunk_bwd_workspace_size(T, H, dk, dv, n_seqs, max_seqlen, ctypes.byref(n))
+    if st != KDA_OK:
+        raise KdaError(st, "kda_chunk_bwd_workspace_size")
+    return n.value
+
+
+def chunk_bwd(q, k, v, log_alpha, beta, d_o, initial_state=None, d_final_state=None, *, cu_seqlens=None,
+              max_seqlen=None, scale: float = 1.0, want_d_initial_state: bool = True, workspace=None, stream=None):
+    """Gradients of chunk_fwd (no gate): inputs as chunk_fwd, d_o = dL/do [B, T, H, 128]
+    (the inputs' dtype), d_final_state = dL/d(final state) fp32 [N, H, 128, 128] or None.
+    Returns a dict of fp32 tensors: dq, dk, dv, dlog_alpha [B, T, H, 128], dbeta [B, T, H]
+    and d_initial_state [N, H, 128, 128] (None when not wanted)."""
+    torch = _torch()
+    _check_cuda(q, k, v, log_alpha, beta, d_o, initial_state, d_final_state, cu_seqlens, workspace)
+    B, T, N, maxlen = _seq_dims(q, cu_seqlens, max_seqlen)
+    H, dk, dv = q.shape[2], q.shape[3], v.shape[-1]
+    for t in (k, v, log_alpha, beta, d_o):
+        if t.dtype != q.dtype:
+            raise TypeError("q, k, v, log_alpha, beta and d_o must share one dtype")
+    f32 = dict(dtype=torch.float32, device=q.device)
+    g = dict(dq=torch.empty((B, T, H, dk), **f32), dk=torch.empty((B, T, H, dk), **f32),
+             dv=torch.empty((B, T, H, dv), **f32), dlog_alpha=torch.empty((B, T, H, dk), **f32),
+             dbeta=torch.empty((B, T, H), **f32),
+             d_initial_state=torch.empty((N, H, dk, dv), **f32) if want_d_initial_state else None)
+    if workspace is None:
+        workspace = torch.empty(bwd_workspace_size(B * T if cu_seqlens is None else T, H, N, maxlen, dk, dv),
+                                dtype=torch.uint8, device=q.device)
+    st = load_library().kda_chunk_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(initial_state),
+                                      _ptr(d_o), _ptr(d_final_state), _ptr(g["dq"]), _ptr(g["dk"]), _ptr(g["dv"]),
+                                      _ptr(g["dlog_alpha"]), _ptr(g["dbeta"]), _ptr(g["d_initial_state"]), B, T, H,
+                                      dk, dv, _ptr(cu_seqlens), N, maxlen, _dt(q), float(scale), _ptr(workspace),
+                                      workspace.numel(), _stream(stream))
+    if st != KDA_OK:
+        raise KdaError(st, "kda_chunk_bwd")
+    return g
 
 
 def _seq_dims(q, cu_seqlens, max_seqlen):

@@ -256,6 +256,53 @@ kda_status kda_kcp_finish(const float* state_in, void* o, float* final_state, in
                           1, workspace, workspace_bytes, stream, kda::KCP_FINISH, nullptr);
 }
 
+kda_status kda_chunk_bwd_workspace_size(int64_t T, int H, int dk, int dv, int n_seqs, int64_t max_seqlen,
+                                       size_t* bytes) {
+    if (!bytes) return KDA_ERR_INVALID_ARG;
+    size_t full = 0;
+    const kda_status st = kda_chunk_fwd_workspace_size(T, H, dk, dv, n_seqs, max_seqlen, nullptr, &full);
+    if (st != KDA_OK) return st;
+    *bytes = full + kda::chunk_bwd_extra_bytes(n_seqs, H, max_seqlen);
+    return KDA_OK;
+}
+
+kda_status kda_chunk_bwd(const void* q, const void* k, const void* v, const void* log_alpha, const void* beta,
+                         const float* init_state, const void* d_o, const float* d_final_state, float* dq, float* dk,
+                         float* dv, float* dlog_alpha, float* dbeta, float* d_init_state, int B, int64_t T, int H,
+                         int dk_dim, int dv_dim, const int32_t* cu_seqlens, int n_seqs, int64_t max_seqlen,
+                         kda_dtype in_dtype, float scale, void* workspace, size_t workspace_bytes, void* stream) {
+    if (B <= 0 || T < 0 || H <= 0 || !dtype_ok(in_dtype)) return KDA_ERR_INVALID_ARG;
+    if (dk_dim != kSupportedD || dv_dim != kSupportedD) return KDA_ERR_UNSUPPORTED;
+    if (H > 65535 || (cu_seqlens ? n_seqs : B) > 65535) return KDA_ERR_UNSUPPORTED;
+    const bool has_tokens = T > 0;
+    if (has_tokens && (!q || !k || !v || !log_alpha || !beta || !d_o || !dq || !dk || !dv || !dlog_alpha || !dbeta))
+        return KDA_ERR_INVALID_ARG;
+    if (cu_seqlens) {
+        if (B != 1 || n_seqs <= 0 || max_seqlen < 0 || max_seqlen > T) return KDA_ERR_INVALID_ARG;
+        if (T > INT32_MAX) return KDA_ERR_UNSUPPORTED;
+    } else {
+        n_seqs = B;
+        max_seqlen = T;
+    }
+    const void* ptrs[] = {q,  k,  v,  log_alpha, beta,  init_state, d_o,          d_final_state, dq,
+                          dk, dv, dlog_alpha, dbeta, d_init_state, cu_seqlens, workspace};
+    for (const void* p : ptrs)
+        if (p && !aligned16(p)) return KDA_ERR_MISALIGNED;
+    if (!workspace) return KDA_ERR_WORKSPACE;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return KDA_ERR_MISALIGNED;
+    const int64_t tot = T * (cu_seqlens ? 1 : B);
+    size_t fwd_full = 0, need = 0;
+    if (kda_chunk_fwd_workspace_size(tot, H, dk_dim, dv_dim, n_seqs, max_seqlen, nullptr, &fwd_full) != KDA_OK ||
+        kda_chunk_bwd_workspace_size(tot, H, dk_dim, dv_dim, n_seqs, max_seqlen, &need) != KDA_OK)
+        return KDA_ERR_INVALID_ARG;
+    if (workspace_bytes < need) return KDA_ERR_WORKSPACE;
+    const cudaError_t e = kda::chunk_bwd_launch(q, k, v, log_alpha, beta, init_state, d_o, d_final_state, dq, dk, dv,
+                                                dlog_alpha, dbeta, d_init_state, B, T, H, cu_seqlens, n_seqs,
+                                                max_seqlen, in_dtype == KDA_BF16, scale, workspace, fwd_full,
+                                                reinterpret_cast<cudaStream_t>(stream));
+    return from_cuda(e);
+}
+
 kda_status kda_decode_steps(float* state, const void* q, const void* k, const void* v, const void* log_alpha,
                             const void* beta, void* o, int n_steps, int Bd, int H, int dk, int dv,
                             kda_dtype in_dtype, kda_dtype out_dtype, float scale, const void* gate,
@@ -309,8 +356,9 @@ kda_status kda_profile_enable(int on) {
 }
 
 kda_status kda_profile_read(kda_kernel_time* out, int max_entries, int* n_entries) {
-    static const char* names[kda::PROF_KINDS] = {"intra",  "chain",    "gate_norm",
-                                                 "decode", "check_cu", "kcp_compose"};
+    static const char* names[kda::PROF_KINDS] = {"intra",      "chain",    "gate_norm",
+                                                 "decode",     "check_cu", "kcp_compose",
+                                                 "chain_bwd",  "intra_bwd"};
     int launches[kda::PROF_KINDS] = {0};
     double ms[kda::PROF_KINDS] = {0};
     kda_status st = KDA_OK;

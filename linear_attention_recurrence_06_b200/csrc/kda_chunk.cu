@@ -49,29 +49,11 @@
 #include "kda_launch.h"
 #include "kda_profile.h"
 #include "kda_sm100.cuh"
+#include "kda_slots.h"
 
 namespace kda {
 
-constexpr int CH = 64;    // chunk length
-constexpr int DK = 128;   // key head dim
-constexpr int DV = 128;   // value head dim
-constexpr int DVS = 32;   // value columns per chain CTA
-constexpr int NSL = DV / DVS;
-
-// Workspace slot per (chunk, head), all offsets 16-byte aligned:
-//   Mlr  bf16 K-major SW128 image [128 key rows][128 K]          32768 B
-//   Qp   bf16 MN-major no-swizzle image, M = 64 tokens, K = 128   16384 B
-//   GamC fp32 [128]                                                512 B
-//   Bm   bf16 [4 slices][128 key rows][32 value cols]            32768 B
-//   Ob   bf16 [4 slices][64 tokens][32 value cols]               16384 B
-// In Bm and Ob the four 16-byte pieces of each 64-byte row r are stored in the
-// order piece ^ ((r >> 1) & 3) (swz64), so that eight consecutive rows read or
-// written 16 bytes at a time touch eight different bank groups.
-constexpr size_t SO_M = 0, SO_Q = 32768, SO_G = 49152, SO_B = 49664, SO_O = 82432;
-constexpr size_t SLOT_BYTES = 98816;
-constexpr uint32_t SO_MQG = 49664;         // Mlr + Qp + GamC, one contiguous copy
-constexpr uint32_t BSL = DK * DVS * 2;     // one Bm slice, 8192 B
-constexpr uint32_t OSL = CH * DVS * 2;     // one Ob slice, 4096 B
+// chunk length, head dims and the workspace slot layout: kda_slots.h
 
 struct ChunkArgs {
     const void* q;
@@ -1007,7 +989,9 @@ chain_kernel(const ChunkArgs a, const __grid_constant__ CUtensorMap gate_map, co
             if (SEG == 2 && it < nseg) return a.seg_ws + (((size_t)n * a.segs + it) * H + h) * SLOT_BYTES;
             return a.ws + (slot0 + (size_t)(it - nseg) * H) * SLOT_BYTES;
         };
-        auto has_out = [&](int it) { return SEG != 1 && it >= nseg; };
+        // (a.o == NULL: the walk only produces states, e.g. the chunk-start states a
+        // backward pass recomputes)
+        auto has_out = [&](int it) { return SEG != 1 && it >= nseg && a.o != nullptr; };
         // chunk buffer of iteration it and its barrier phase
         auto bidx = [](int it) { return it % NBUF; };
         auto bpar = [](int it) { return (uint32_t)((it / NBUF) & 1); };
@@ -1147,6 +1131,20 @@ chain_kernel(const ChunkArgs a, const __grid_constant__ CUtensorMap gate_map, co
                 return true;
             };
 
+            // checkpoint: the state after (j + 1) * ckpt_every whole chunks of the sequence
+            auto store_ckpt = [&](int oi) {
+                if (!a.ckpt) return;
+                const int cdone = c_beg + oi + 1;  // chunks of this sequence now folded in
+                const int64_t t_end = s_beg + (int64_t)cdone * CH;
+                if (cdone % a.ckpt_every == 0 && t_end <= s_end && cdone / a.ckpt_every <= a.n_ckpt) {
+                    const int j = cdone / a.ckpt_every - 1;
+                    float* dst = a.ckpt + ((((size_t)n * a.n_ckpt + j) * H + h) * DK + tid) * DV + (size_t)DVS * jb;
+#pragma unroll
+                    for (int c4 = 0; c4 < DVS; c4 += 4)
+                        __stcs(reinterpret_cast<float4*>(dst + c4), make_float4(S[c4], S[c4 + 1], S[c4 + 2], S[c4 + 3]));
+                }
+            };
+
             write_state_image(0);
             for (int it = 0; it < nit; ++it) {
                 const int b = bidx(it);
@@ -1185,6 +1183,7 @@ chain_kernel(const ChunkArgs a, const __grid_constant__ CUtensorMap gate_map, co
                 if (it + 1 < nit) write_state_image(it + 1);
                 if (!has_out(it)) {  // a segment iteration, or no outputs at all: the buffer is done
                     mbar_arrive(&bar_free[b]);
+                    if (SEG != 1 && it >= nseg) store_ckpt(oi);
                     continue;
                 }
                 // (3) this chunk's output: o = Qp S + Ob  (then y, when the gate is fused)
@@ -1262,19 +1261,7 @@ chain_kernel(const ChunkArgs a, const __grid_constant__ CUtensorMap gate_map, co
                     t0_prev = t0;
                     L_prev = L;
                 }
-                // checkpoint: the state after (j + 1) * ckpt_every whole chunks of the sequence
-                if (a.ckpt) {
-                    const int cdone = c_beg + oi + 1;  // chunks of this sequence now folded in
-                    const int64_t t_end = s_beg + (int64_t)cdone * CH;
-                    if (cdone % a.ckpt_every == 0 && t_end <= s_end && cdone / a.ckpt_every <= a.n_ckpt) {
-                        const int j = cdone / a.ckpt_every - 1;
-                        float* dst =
-                            a.ckpt + ((((size_t)n * a.n_ckpt + j) * H + h) * DK + tid) * DV + (size_t)DVS * jb;
-#pragma unroll
-                        for (int c4 = 0; c4 < DVS; c4 += 4)
-                            __stcs(reinterpret_cast<float4*>(dst + c4), make_float4(S[c4], S[c4 + 1], S[c4 + 2], S[c4 + 3]));
-                    }
-                }
+                store_ckpt(oi);
                 // (4) D_O[oi & 1] is no longer read
                 tc_fence_before();
             }

@@ -32,4 +32,14 @@ cudaError_t chunk_fwd_launch(const void* q, const void* k, const void* v, const 
 cudaError_t launch_kcp_compose(const float* trans, int n_prev, const float* init_state, float* state_in, int N, int H,
                                cudaStream_t stream);
 
+// Backward of the chunkwise prefill.  The workspace holds the forward's whole-
+// sequence workspace (fwd_bytes: kda_chunk_fwd_workspace_size's bytes_full),
+// then chunk_bwd_extra_bytes of chunk-boundary states and state gradients.
+size_t chunk_bwd_extra_bytes(int n_seqs, int H, int64_t max_seqlen);
+cudaError_t chunk_bwd_launch(const void* q, const void* k, const void* v, const void* log_alpha, const void* beta,
+                             const float* init_state, const void* d_o, const float* d_final, float* dq, float* dk,
+                             float* dv, float* dlog_alpha, float* dbeta, float* d_init, int B, int64_t T, int H,
+                             const int32_t* cu, int n_seqs, int64_t max_seqlen, bool in_bf16, float scale,
+                             void* workspace, size_t fwd_bytes, cudaStream_t stream);
+
 }  // namespace kda

@@ -30,7 +30,7 @@ def test_header_declares_the_entry_points():
     for s in ("kda_chunk_fwd", "kda_chunk_fwd_ckpt", "kda_chunk_fwd_segmented", "kda_decode_step", "kda_decode_steps",
               "kda_gate_norm", "kda_chunk_fwd_segmented_workspace_size",
               "kda_chunk_fwd_workspace_size", "kda_kcp_workspace_size", "kda_kcp_transition", "kda_kcp_compose",
-              "kda_kcp_finish",
+              "kda_kcp_finish", "kda_chunk_bwd", "kda_chunk_bwd_workspace_size",
               "kda_query_status", "kda_status_string", "kda_version"):
         assert s in syms
 
@@ -147,6 +147,38 @@ def test_kcp_workspace_and_host_validation(lib):
     assert lib.kda_kcp_compose(FAKE, 2, None, None, 1, 2, 128, 128, None) == -1
     assert lib.kda_kcp_compose(FAKE, 2, FAKE + 4, FAKE, 1, 2, 128, 128, None) == -3
     assert lib.kda_kcp_compose(FAKE, 2, None, FAKE, 1, 2, 64, 128, None) == -2
+
+
+def test_chunk_bwd_workspace_and_host_validation(lib):
+    import ctypes
+    full = ctypes.c_size_t(0)
+    assert lib.kda_chunk_fwd_workspace_size(300, 2, 128, 128, 1, 300, None, ctypes.byref(full)) == 0
+    n = ctypes.c_size_t(0)
+    assert lib.kda_chunk_bwd_workspace_size(300, 2, 128, 128, 1, 300, ctypes.byref(n)) == 0
+    # the forward's whole-sequence workspace + 5 chunk-end gradients + 4 chunk-boundary states
+    assert n.value == full.value + (5 + 4) * 2 * 128 * 128 * 4
+
+    def bw(**over):
+        a = dict(q=FAKE, k=FAKE, v=FAKE, la=FAKE, beta=FAKE, s0=None, do=FAKE, dfin=None, dq=FAKE, dk=FAKE,
+                 dv=FAKE, dla=FAKE, db=FAKE, dinit=None, B=1, T=128, H=2, dk_=128, dv_=128, cu=None, N=1,
+                 maxlen=128, idt=1, scale=1.0, ws=FAKE, wsb=1 << 40)
+        a.update(over)
+        return lib.kda_chunk_bwd(a["q"], a["k"], a["v"], a["la"], a["beta"], a["s0"], a["do"], a["dfin"], a["dq"],
+                                 a["dk"], a["dv"], a["dla"], a["db"], a["dinit"], a["B"], a["T"], a["H"], a["dk_"],
+                                 a["dv_"], a["cu"], a["N"], a["maxlen"], a["idt"], a["scale"], a["ws"], a["wsb"],
+                                 None)
+    assert bw(do=None) == -1
+    assert bw(dla=None) == -1
+    assert bw(db=None) == -1
+    assert bw(idt=5) == -1
+    assert bw(dk_=64) == -2
+    assert bw(H=70000) == -2
+    assert bw(dq=FAKE + 4) == -3
+    assert bw(dinit=FAKE + 8) == -3
+    assert bw(ws=FAKE + 16) == -3
+    assert bw(ws=None) == -4
+    assert bw(wsb=1024) == -4
+    assert bw(cu=FAKE, B=2, N=2) == -1
 
 
 def test_chunk_fwd_host_validation(lib):
