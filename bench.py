@@ -231,6 +231,9 @@ def run_ours(args, peaks):
     # per-device steps of context parallelism across devices (ranks emulated on this GPU)
     kcp = run_kcp(args, torch, kda, dev, stream, mor, barrier)
 
+    # backward of the prefill on the same shape
+    bwd = run_backward(args, torch, kda, dev, stream, mor, barrier)
+
     if dist is not None:
         dist.barrier()
         dist.destroy_process_group()
@@ -260,7 +263,7 @@ def run_ours(args, peaks):
                    "l2": "inputs larger than L2 (q,k,v,log_alpha,gate,beta = 336 MB per step)"},
         "prefill_tflops": tflops, "prefill_tensor_frac": tflops / peaks["bf16_tflops_sustained"],
         "roofline": roof, "kernels": kernels, "decode": dec, "e2e": e2e, "segment_parallel": seg,
-        "kcp_per_device": kcp, "gpu_launches": int(round(launches_per_step * args.steps)),
+        "kcp_per_device": kcp, "backward": bwd, "gpu_launches": int(round(launches_per_step * args.steps)),
         "clocks": clocks,
     }
     if ws_n == 1 and not args.no_cpu_baseline:
@@ -390,6 +393,53 @@ def run_segmented(args, torch, kda, dev, stream, max_over_ranks, barrier):
 
 
 KCP_SHAPE = dict(T_rank=8192, H=32, ranks=8)
+
+
+def run_backward(args, torch, kda, dev, stream, max_over_ranks, barrier):
+    """kda_chunk_bwd on the prefill shape (B=1, T=8192, H=32, bf16 inputs and dL/do,
+    an initial state and dL/d(final state)): one call = the forward walk recomputed
+    without outputs + the reverse walk + the chunk-local gradient kernel."""
+    from linear_attention_recurrence_06_b200 import synth
+    B, T, H = PREFILL["B"], PREFILL["T"], PREFILL["H"]
+    tb = synth.tokens(500, 0, T, H, D, D, bf16=True)
+    x = {n: torch.from_numpy(np.ascontiguousarray(getattr(tb, n))).to(torch.bfloat16).to(dev)
+         for n in ("q", "k", "v", "log_alpha", "beta")}
+    x = {n: t.view(1, T, H, -1) if n != "beta" else t.view(1, T, H) for n, t in x.items()}
+    d_o = torch.from_numpy(synth.normal(501, synth.TAG_V, (T, H, D), 1.0, True)).to(torch.bfloat16).to(dev)
+    d_o = d_o.view(1, T, H, D)
+    s0 = torch.from_numpy(synth.states(502, 1, H, D, D)).to(dev)
+    dfin = torch.from_numpy(synth.states(503, 1, H, D, D)).to(dev)
+    ws = torch.empty(kda.bwd_workspace_size(T, H, 1, T), dtype=torch.uint8, device=dev)
+
+    def f():
+        kda.chunk_bwd(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], d_o, s0, dfin, scale=D ** -0.5,
+                      workspace=ws, stream=stream)
+
+    for _ in range(3):
+        f()
+    n = max(3, min(args.steps, 10))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(n):
+        f()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    ms = max_over_ranks(e0.elapsed_time(e1) / n)
+    # per-kernel split from a separate, profiled set of calls
+    kda.profile_enable(True)
+    kda.profile_read()
+    for _ in range(n):
+        f()
+    torch.cuda.synchronize()
+    prof = kda.profile_read()
+    kda.profile_enable(False)
+    kernels = {k: dict(launches_per_call=v[0] / n, ms_per_call=v[1] / n) for k, v in prof.items()}
+    return {"workload": f"KDA backward B={B} T={T} H={H} bf16 inputs and dL/do, fp32 gradients, initial state "
+                        "and final-state gradient", "ms_per_call": ms, "tokens_per_s": B * T / (ms * 1e-3),
+            "kernels": kernels}
 
 
 def run_kcp(args, torch, kda, dev, stream, max_over_ranks, barrier):

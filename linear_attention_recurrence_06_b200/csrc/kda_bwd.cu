@@ -121,6 +121,16 @@ __global__ void __launch_bounds__(CB_THREADS, 1) chain_bwd_kernel(const BwdArgs 
     __syncthreads();
     int issued = nck < 2 ? nck : 2, waited = 0;
     bool failed = false;
+    // this thread's 4 values of a chunk's dO slice: token tid / 8, columns 4 (tid % 8) ..
+    auto load_dO = [&](int c) {
+        const int t = tid >> 3, c4 = (tid & 7) * 4;
+        const int64_t tc = s_beg + (int64_t)c * CH + t;
+        if (c < 0 || tc >= s_end) return make_float4(0.f, 0.f, 0.f, 0.f);
+        const size_t base = ((size_t)tc * H + h) * DV + DVS * js + c4;
+        return make_float4(ld_in(a.d_o, base, a.in_bf16), ld_in(a.d_o, base + 1, a.in_bf16),
+                           ld_in(a.d_o, base + 2, a.in_bf16), ld_in(a.d_o, base + 3, a.in_bf16));
+    };
+    float4 dO_next = load_dO(nck - 1);
     for (int r = 0; r < nck; ++r) {
         const int c = nck - 1 - r, b = r & 1;
         const int64_t t0 = s_beg + (int64_t)c * CH;
@@ -131,16 +141,8 @@ __global__ void __launch_bounds__(CB_THREADS, 1) chain_bwd_kernel(const BwdArgs 
         reinterpret_cast<float4*>(dst)[1] = make_float4(dS[4], dS[5], dS[6], dS[7]);
         reinterpret_cast<float4*>(sdS + i * DVS + 8 * cq)[0] = make_float4(dS[0], dS[1], dS[2], dS[3]);
         reinterpret_cast<float4*>(sdS + i * DVS + 8 * cq)[1] = make_float4(dS[4], dS[5], dS[6], dS[7]);
-        {  // dO slice of chunk c: [64 tokens][32 columns]
-            const int t = tid >> 3, c4 = (tid & 7) * 4;
-            float4 v4 = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (t < L) {
-                const size_t base = ((size_t)(t0 + t) * H + h) * DV + DVS * js + c4;
-                v4 = make_float4(ld_in(a.d_o, base, a.in_bf16), ld_in(a.d_o, base + 1, a.in_bf16),
-                                 ld_in(a.d_o, base + 2, a.in_bf16), ld_in(a.d_o, base + 3, a.in_bf16));
-            }
-            *reinterpret_cast<float4*>(sdO + t * DVS + c4) = v4;
-        }
+        // dO slice of chunk c ([64 tokens][32 columns]), loaded during the previous iteration
+        *reinterpret_cast<float4*>(sdO + (tid >> 3) * DVS + (tid & 7) * 4) = dO_next;
         const bool ok = mbar_wait(&bar[b], (uint32_t)((r >> 1) & 1), a.status);
         if (!__syncthreads_and(ok)) {
             failed = true;
@@ -173,6 +175,7 @@ __global__ void __launch_bounds__(CB_THREADS, 1) chain_bwd_kernel(const BwdArgs 
             acc[0] += qv * o0.x; acc[1] += qv * o0.y; acc[2] += qv * o0.z; acc[3] += qv * o0.w;
             acc[4] += qv * o1.x; acc[5] += qv * o1.y; acc[6] += qv * o1.z; acc[7] += qv * o1.w;
         }
+        dO_next = load_dO(c - 1);
         __syncthreads();  // buffer b, dS and dO are no longer read
         if (tid == 0 && r + 2 < nck) {
             mbar_arrive_expect_tx(&bar[b], CB_SLOT);
@@ -222,30 +225,68 @@ constexpr uint32_t BI_SMEM = BI_DGC + 512;
 KDA_DEV void build_factors(const BwdArgs& a, float* sF, const float* sG, int bt, int64_t t0, int L, int h,
                            int tid) {
     const int r = 16 * bt, ns = 16 * bt + 16;
-    for (int e = tid; e < (ns + 32) * DK; e += BI_THREADS) {
-        const int row = e >> 7, i = e & (DK - 1);
-        const float gr = sG[r * DK + i];
-        if (row < ns) {
-            const int s = row;
-            float kv = 0.f;
-            if (s < L) kv = ld_in(a.k, ((size_t)(t0 + s) * a.H + h) * DK + i, a.in_bf16);
-            sF[s * FP + i] = kv * __expf(gr - sG[s * DK + i]);
-        } else {
-            const int tt = row - ns;            // 0..31
-            const int t = r + (tt & 15);
-            float x = 0.f;
+    const int n_el = (ns + 32) * DK;  // a multiple of 4 * BI_THREADS
+    for (int e0 = tid; e0 < n_el; e0 += 4 * BI_THREADS) {
+        float x[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {  // loads first, all four in flight
+            const int e = e0 + u * BI_THREADS, row = e >> 7, i = e & (DK - 1);
+            const int t = row < ns ? row : r + ((row - ns) & 15);
+            x[u] = 0.f;
             if (t < L) {
                 const size_t idx = ((size_t)(t0 + t) * a.H + h) * DK + i;
-                x = (tt < 16) ? ld_in(a.k, idx, a.in_bf16) : a.scale * ld_in(a.q, idx, a.in_bf16);
-                x *= __expf(sG[t * DK + i] - gr);
+                x[u] = (row < ns + 16) ? ld_in(a.k, idx, a.in_bf16) : a.scale * ld_in(a.q, idx, a.in_bf16);
             }
-            sF[(64 + tt) * FP + i] = x;
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int e = e0 + u * BI_THREADS, row = e >> 7, i = e & (DK - 1);
+            const float gr = sG[r * DK + i];
+            if (row < ns) {
+                sF[row * FP + i] = x[u] * __expf(gr - sG[row * DK + i]);
+            } else {
+                const int tt = row - ns;  // 0..31: Kin rows, then Qin rows
+                const int t = r + (tt & 15);
+                sF[(64 + tt) * FP + i] = x[u] * __expf(sG[t * DK + i] - gr);
+            }
         }
     }
 }
 
+// Pulls an item's token rows (q, k, v, log_alpha, dO: 64 rows each), its
+// chunk-start state and its end-of-chunk state gradient into L2 ahead of use.
+KDA_DEV void prefetch_item(const BwdArgs& a, int64_t item, int64_t n_items, int tid) {
+    if (item >= n_items) return;
+    const int H = a.H;
+    const int h = (int)(item % H);
+    const int c = (int)((item / H) % a.wc);
+    const int n = (int)(item / ((int64_t)H * a.wc));
+    int64_t s_beg, s_end;
+    bwd_seq_range(a, n, s_beg, s_end);
+    const int64_t t0 = s_beg + (int64_t)c * CH;
+    if (t0 >= s_end) return;
+    const int L = (int)((s_end - t0) < CH ? (s_end - t0) : CH);
+    const size_t esz = a.in_bf16 ? 2 : 4, row = DK * esz;  // bytes of one head row
+    const int lines_row = (int)(row / 128);
+    const void* tens[5] = {a.q, a.k, a.v, a.log_alpha, a.d_o};
+    for (int e = tid; e < 5 * CH * lines_row; e += BI_THREADS) {
+        const int tsr = e / (CH * lines_row), rem = e % (CH * lines_row), t = rem / lines_row, ln = rem % lines_row;
+        if (t >= L) continue;
+        const char* p = reinterpret_cast<const char*>(tens[tsr]) + ((size_t)(t0 + t) * H + h) * row + ln * 128;
+        asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+    }
+    const float* S0 = c == 0 ? (a.init_state ? a.init_state + ((size_t)n * H + h) * STATE : nullptr)
+                             : a.ckpt + (((size_t)n * a.n_ckpt + (c - 1)) * H + h) * STATE;
+    const float* dSC = a.ds_end + (((size_t)n * a.wc + c) * H + h) * STATE;
+    for (int e = tid; e < 2 * STATE * 4 / 128; e += BI_THREADS) {
+        const int which = e / (STATE * 4 / 128), ln = e % (STATE * 4 / 128);
+        const float* base = which ? dSC : S0;
+        if (base) asm volatile("prefetch.global.L2 [%0];" ::"l"(reinterpret_cast<const char*>(base) + (size_t)ln * 128));
+    }
+}
+
 __global__ void __launch_bounds__(BI_THREADS, 1) bwd_intra_kernel(const BwdArgs a, int64_t n_items) {
-    extern __shared__ __align__(16) uint8_t sm[];
+    extern __shared__ __align__(128) uint8_t sm[];
     float* sG = reinterpret_cast<float*>(sm + BI_G);
     float* sA = reinterpret_cast<float*>(sm + BI_A);
     float* sP = reinterpret_cast<float*>(sm + BI_P);
@@ -278,6 +319,7 @@ __global__ void __launch_bounds__(BI_THREADS, 1) bwd_intra_kernel(const BwdArgs 
         const float* S0 = c == 0 ? (a.init_state ? a.init_state + ((size_t)n * H + h) * STATE : nullptr)
                                  : a.ckpt + (((size_t)n * a.n_ckpt + (c - 1)) * H + h) * STATE;
         const float* dSC = a.ds_end + (((size_t)n * a.wc + c) * H + h) * STATE;
+        prefetch_item(a, item + gridDim.x, n_items, tid);  // the next item's inputs into L2
 
         // ---- P0: beta, g (cumulative clamped log-decay), zeroed accumulators
         if (tid < CH) {
@@ -285,9 +327,14 @@ __global__ void __launch_bounds__(BI_THREADS, 1) bwd_intra_kernel(const BwdArgs 
             sDb[tid] = 0.f;
         }
         if (tid < DK) {
+            float lv[CH];  // all loads in flight at once
+#pragma unroll
+            for (int t = 0; t < CH; ++t)
+                lv[t] = t < L ? fmaxf(ld_in(a.log_alpha, ((size_t)(t0 + t) * H + h) * DK + tid, a.in_bf16), -5.f) : 0.f;
             float g = 0.f;
+#pragma unroll
             for (int t = 0; t < CH; ++t) {
-                if (t < L) g += fmaxf(ld_in(a.log_alpha, ((size_t)(t0 + t) * H + h) * DK + tid, a.in_bf16), -5.f);
+                g += lv[t];
                 sG[t * DK + tid] = g;
             }
             sGC[tid] = g;
@@ -345,13 +392,20 @@ __global__ void __launch_bounds__(BI_THREADS, 1) bwd_intra_kernel(const BwdArgs 
             }
         }
         // factors K o Gam (rows 0-63) and K^C = K o e^{g_C - g} (rows 64-127)
-        for (int e = tid; e < CH * DK; e += BI_THREADS) {
-            const int t = e >> 7, i = e & (DK - 1);
-            float kv = 0.f;
-            if (t < L) kv = ld_in(a.k, ((size_t)(t0 + t) * H + h) * DK + i, a.in_bf16);
-            const float g = sG[t * DK + i];
-            sF[t * FP + i] = kv * __expf(g);
-            sF[(64 + t) * FP + i] = kv * __expf(sGC[i] - g);
+        for (int e0 = tid; e0 < CH * DK; e0 += 4 * BI_THREADS) {
+            float kv[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int e = e0 + u * BI_THREADS, t = e >> 7, i = e & (DK - 1);
+                kv[u] = t < L ? ld_in(a.k, ((size_t)(t0 + t) * H + h) * DK + i, a.in_bf16) : 0.f;
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int e = e0 + u * BI_THREADS, t = e >> 7, i = e & (DK - 1);
+                const float g = sG[t * DK + i];
+                sF[t * FP + i] = kv[u] * __expf(g);
+                sF[(64 + t) * FP + i] = kv[u] * __expf(sGC[i] - g);
+            }
         }
         __syncthreads();
 
@@ -379,7 +433,7 @@ __global__ void __launch_bounds__(BI_THREADS, 1) bwd_intra_kernel(const BwdArgs 
                     }
                     if (S0) {
                         const float* kg = sF + t * FP;
-#pragma unroll 4
+#pragma unroll 8
                         for (int i = 0; i < DK; ++i) {
                             const float4 s4 = __ldg(reinterpret_cast<const float4*>(S0 + (size_t)i * DV + j0 + jq));
                             const float w = kg[i];
@@ -409,7 +463,7 @@ __global__ void __launch_bounds__(BI_THREADS, 1) bwd_intra_kernel(const BwdArgs 
                     for (int x = 0; x < 4; ++x) d4[x] += w * sDO[tt * QP + jq + x];
                 }
                 const float* kc = sF + (64 + t) * FP;
-#pragma unroll 4
+#pragma unroll 8
                 for (int i = 0; i < DK; ++i) {
                     const float4 s4 = __ldg(reinterpret_cast<const float4*>(dSC + (size_t)i * DV + j0 + jq));
                     const float w = kc[i];
@@ -548,29 +602,43 @@ __global__ void __launch_bounds__(BI_THREADS, 1) bwd_intra_kernel(const BwdArgs 
         __syncthreads();
 
         // ---- P5: the A / P contractions, block row by block row
+        float* sC = sR;  // [3][16][128] contributions of the block's tokens (the quarter buffers are free)
         for (int bt = 0; bt < nb; ++bt) {
             build_factors(a, sF, sG, bt, t0, L, h, tid);
             __syncthreads();
             const int r = 16 * bt;
+            {  // tokens t of the block, all threads: dKin_t = sum_s dA_ts Kout_s, dQin_t = sum_s dP_ts Kout_s
+                const int tl = tid >> 5, i4 = (tid & 31) * 4, t = r + tl;
+                if (t < L) {
+                    float dki[4] = {0.f, 0.f, 0.f, 0.f}, dqi[4] = {0.f, 0.f, 0.f, 0.f};
+                    for (int s = 0; s <= t; ++s) {
+                        const float wm = s < t ? sdM[t * LP + s] : 0.f, wp = sdP[t * LP + s];
+                        const float4 ko = *reinterpret_cast<const float4*>(sF + s * FP + i4);
+                        dki[0] += wm * ko.x; dki[1] += wm * ko.y; dki[2] += wm * ko.z; dki[3] += wm * ko.w;
+                        dqi[0] += wp * ko.x; dqi[1] += wp * ko.y; dqi[2] += wp * ko.z; dqi[3] += wp * ko.w;
+                    }
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const int i = i4 + u;
+                        const float e = __expf(sG[t * DK + i] - sG[r * DK + i]);
+                        sC[(0 * 16 + tl) * DK + i] = e * dki[u];
+                        sC[(1 * 16 + tl) * DK + i] = e * dqi[u];
+                        sC[(2 * 16 + tl) * DK + i] = sF[(64 + tl) * FP + i] * dki[u] + sF[(80 + tl) * FP + i] * dqi[u];
+                    }
+                }
+            }
+            __syncthreads();
 #pragma unroll
             for (int x = 0; x < 4; ++x) {
                 const int t = 4 * tg + x;
-                if ((t >> 4) == bt && t < L) {  // t in the block: dKin_t, dQin_t
+                if ((t >> 4) == bt && t < L) {  // owner of a block token: take its contributions
                     const int tl = t - r;
 #pragma unroll
                     for (int y = 0; y < 4; ++y) {
                         const int i = 4 * ig + y;
-                        float dki = 0.f, dqi = 0.f;
-                        for (int s = 0; s <= t; ++s) {
-                            const float ko = sF[s * FP + i];
-                            if (s < t) dki += sdM[t * LP + s] * ko;
-                            dqi += sdP[t * LP + s] * ko;
-                        }
-                        const float kin = sF[(64 + tl) * FP + i], qin = sF[(80 + tl) * FP + i];
-                        const float e = __expf(sG[t * DK + i] - sG[r * DK + i]);
-                        dkk[x][y] += e * dki;
-                        dqb[x][y] += e * dqi;
-                        dg[x][y] += kin * dki + qin * dqi;
+                        dkk[x][y] += sC[(0 * 16 + tl) * DK + i];
+                        dqb[x][y] += sC[(1 * 16 + tl) * DK + i];
+                        dg[x][y] += sC[(2 * 16 + tl) * DK + i];
                     }
                 }
                 if (t < r + 16 && t < L) {  // t as an earlier token s: dKout_t
@@ -609,12 +677,17 @@ __global__ void __launch_bounds__(BI_THREADS, 1) bwd_intra_kernel(const BwdArgs 
         __syncthreads();
         if (tid < DK) {
             const int i = tid;
+            float lv[CH];
+#pragma unroll
+            for (int t = 0; t < CH; ++t)
+                lv[t] = t < L ? ld_in(a.log_alpha, ((size_t)(t0 + t) * H + h) * DK + i, a.in_bf16) : 0.f;
             float run = sDgC[i];  // g_C is g of the last token
-            for (int t = L - 1; t >= 0; --t) {
-                run += sF[t * FP + i];
-                const size_t idx = ((size_t)(t0 + t) * H + h) * DK + i;
-                const float la = ld_in(a.log_alpha, idx, a.in_bf16);
-                a.dla[idx] = la >= -5.f ? run : 0.f;
+#pragma unroll
+            for (int t = CH - 1; t >= 0; --t) {
+                if (t < L) {
+                    run += sF[t * FP + i];
+                    a.dla[((size_t)(t0 + t) * H + h) * DK + i] = lv[t] >= -5.f ? run : 0.f;
+                }
             }
         }
         __syncthreads();  // shared memory is reused by the next item

@@ -891,7 +891,9 @@ constexpr uint32_t PART_TX = CLUSTER * 64 * 4;  // partial-sum bytes each CTA re
 //   GPUs) M_g and B_g are written there in fp32 instead;
 // SEG = 2: segment g first folds segments 0 .. g-1 into the initial state through
 //   their slots, then walks its own chunks with outputs; the last segment writes
-//   the final state.
+//   the final state;
+// SEG = 3: the plain walk without outputs, keeping only the states (checkpoints
+//   and the final state): the forward recomputation of the backward pass.
 template <bool OUT_BF16, bool GATE, int SEG>
 __global__ void __launch_bounds__(CHAIN_THREADS, 1)
 chain_kernel(const ChunkArgs a, const __grid_constant__ CUtensorMap gate_map, const float* __restrict__ norm_w,
@@ -904,8 +906,8 @@ chain_kernel(const ChunkArgs a, const __grid_constant__ CUtensorMap gate_map, co
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const bool consumer = warp < 4;
     const int js = blockIdx.x, h = blockIdx.y;
-    const int n = SEG ? (int)blockIdx.z / a.segs : (int)blockIdx.z;
-    const int g = SEG ? (int)blockIdx.z % a.segs : 0;
+    const int n = (SEG == 1 || SEG == 2) ? (int)blockIdx.z / a.segs : (int)blockIdx.z;
+    const int g = (SEG == 1 || SEG == 2) ? (int)blockIdx.z % a.segs : 0;
     const int H = a.H;
     const int jb = js & (NSL - 1);                // value slice of Bm / outputs
     const bool trans = SEG == 1 && js >= NSL;     // carries M_g (identity start, no Bm)
@@ -923,7 +925,7 @@ chain_kernel(const ChunkArgs a, const __grid_constant__ CUtensorMap gate_map, co
     const int nchunks = (int)((s_end - s_beg + CH - 1) / CH);
     // chunk iterations [c_beg, c_end); with SEG = 2 preceded by nseg segment iterations
     int c_beg, c_end;
-    if constexpr (SEG == 0) {
+    if constexpr (SEG == 0 || SEG == 3) {
         c_beg = a.i0;
         c_end = min(a.i0 + a.wc, nchunks);
     } else {
@@ -989,9 +991,7 @@ chain_kernel(const ChunkArgs a, const __grid_constant__ CUtensorMap gate_map, co
             if (SEG == 2 && it < nseg) return a.seg_ws + (((size_t)n * a.segs + it) * H + h) * SLOT_BYTES;
             return a.ws + (slot0 + (size_t)(it - nseg) * H) * SLOT_BYTES;
         };
-        // (a.o == NULL: the walk only produces states, e.g. the chunk-start states a
-        // backward pass recomputes)
-        auto has_out = [&](int it) { return SEG != 1 && it >= nseg && a.o != nullptr; };
+        auto has_out = [&](int it) { return SEG != 1 && SEG != 3 && it >= nseg; };
         // chunk buffer of iteration it and its barrier phase
         auto bidx = [](int it) { return it % NBUF; };
         auto bpar = [](int it) { return (uint32_t)((it / NBUF) & 1); };
@@ -1183,7 +1183,7 @@ chain_kernel(const ChunkArgs a, const __grid_constant__ CUtensorMap gate_map, co
                 if (it + 1 < nit) write_state_image(it + 1);
                 if (!has_out(it)) {  // a segment iteration, or no outputs at all: the buffer is done
                     mbar_arrive(&bar_free[b]);
-                    if (SEG != 1 && it >= nseg) store_ckpt(oi);
+                    if constexpr (SEG == 3) store_ckpt(oi);
                     continue;
                 }
                 // (3) this chunk's output: o = Qp S + Ob  (then y, when the gate is fused)
@@ -1319,7 +1319,7 @@ chain_kernel(const ChunkArgs a, const __grid_constant__ CUtensorMap gate_map, co
         }
     } else {
         // the carried / final state slice (with segments: the last segment's)
-        if (consumer && (SEG == 0 || g == a.segs - 1)) {
+        if (consumer && (SEG != 2 || g == a.segs - 1)) {
 #pragma unroll
             for (int j = 0; j < DVS; j += 4)
                 *reinterpret_cast<float4*>(a.state_io + st_off + j) = make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]);
@@ -1395,7 +1395,7 @@ static cudaError_t launch_chain(const ChunkArgs& a, const CUtensorMap& gate_map,
     cfg.blockDim = dim3(CHAIN_THREADS, 1, 1);
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
-    if (!fuse) {
+    if (SEG == 3 || !fuse) {
         cfg.dynamicSmemBytes = ChainLayout<false>::SMEM;
         return out_bf16 ? cudaLaunchKernelEx(&cfg, chain_kernel<true, false, SEG>, a, gate_map, norm_w, eps)
                         : cudaLaunchKernelEx(&cfg, chain_kernel<false, false, SEG>, a, gate_map, norm_w, eps);
@@ -1408,8 +1408,10 @@ static cudaError_t launch_chain(const ChunkArgs& a, const CUtensorMap& gate_map,
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return out_bf16 ? cudaLaunchKernelEx(&cfg, chain_kernel<true, true, SEG>, a, gate_map, norm_w, eps)
-                    : cudaLaunchKernelEx(&cfg, chain_kernel<false, true, SEG>, a, gate_map, norm_w, eps);
+    if constexpr (SEG == 3) return cudaErrorInvalidValue;  // no outputs, nothing to gate
+    else
+        return out_bf16 ? cudaLaunchKernelEx(&cfg, chain_kernel<true, true, SEG>, a, gate_map, norm_w, eps)
+                        : cudaLaunchKernelEx(&cfg, chain_kernel<false, true, SEG>, a, gate_map, norm_w, eps);
 }
 
 template <bool OB, bool G, int SEG>
@@ -1438,7 +1440,8 @@ cudaError_t chunk_fwd_launch(const void* q, const void* k, const void* v, const 
             (err = set_chain_smem<true, false, 1>()) != cudaSuccess || (err = set_chain_smem<false, false, 1>()) != cudaSuccess ||
             (err = set_chain_smem<true, true, 1>()) != cudaSuccess || (err = set_chain_smem<false, true, 1>()) != cudaSuccess ||
             (err = set_chain_smem<true, false, 2>()) != cudaSuccess || (err = set_chain_smem<false, false, 2>()) != cudaSuccess ||
-            (err = set_chain_smem<true, true, 2>()) != cudaSuccess || (err = set_chain_smem<false, true, 2>()) != cudaSuccess)
+            (err = set_chain_smem<true, true, 2>()) != cudaSuccess || (err = set_chain_smem<false, true, 2>()) != cudaSuccess ||
+            (err = set_chain_smem<false, false, 3>()) != cudaSuccess)
             return err;
         int dev = 0;
         if ((err = cudaGetDevice(&dev)) != cudaSuccess) return err;
@@ -1524,7 +1527,10 @@ cudaError_t chunk_fwd_launch(const void* q, const void* k, const void* v, const 
             prof_end(PROF_INTRA, stream);
         }
         prof_begin(PROF_CHAIN, stream);
-        if (kcp_mode == KCP_TRANSITION) {
+        if (o == nullptr && kcp_mode == KCP_NONE && a.segs == 1) {
+            // states only (checkpoints, final state): the backward pass's recomputation
+            err = launch_chain<3>(a, gate_map, norm_w, eps, false, false, dim3(NSL, H, N), stream);
+        } else if (kcp_mode == KCP_TRANSITION) {
             // M_g and B_g of the whole local sequence (one segment), fp32, no outputs
             err = launch_chain<1>(a, gate_map, norm_w, eps, out_bf16, false, dim3(2 * NSL, H, N), stream);
         } else if (a.segs == 1) {
