@@ -577,9 +577,9 @@ def recorded_traffic(kernel: str, units: int):
 # the source files each recorded kernel is built from (a change to any of them
 # voids its recorded traffic)
 KERNEL_SOURCES = {
-    "kda_chunk_fwd": ("kda_chunk.cu", "kda_sm100.cuh"),
-    "intra_kernel": ("kda_chunk.cu", "kda_sm100.cuh"),
-    "chain_kernel": ("kda_chunk.cu", "kda_sm100.cuh"),
+    "kda_chunk_fwd": ("kda_chunk.cu", "kda_sm100.cuh", "kda_slots.h"),
+    "intra_kernel": ("kda_chunk.cu", "kda_sm100.cuh", "kda_slots.h"),
+    "chain_kernel": ("kda_chunk.cu", "kda_sm100.cuh", "kda_slots.h"),
     "decode_step_kernel": ("kda_decode.cu", "kda_sm100.cuh"),
 }
 
