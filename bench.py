@@ -395,6 +395,18 @@ def run_segmented(args, torch, kda, dev, stream, max_over_ranks, barrier):
 KCP_SHAPE = dict(T_rank=8192, H=32, ranks=8)
 
 
+# Algorithmic work of the backward per (64-token chunk, head), counted from its products
+# (2 FLOP per multiply-add): A and P 4,096 dot products of 128; M^-1 43.7 k; R = V - (K o Gam) S0
+# 64x128x128; U, P^T dO, Y (triangular) 3 x 266 k; K^C dS_C 64x128x128; dP, dM 524 k; the three
+# (token, channel) accumulations 3 x 64x128x128; the A/P contractions 2 x 524 k.  The reverse
+# chain per chunk step and head: M_lr^T dS 128x128x128 and Q'^T dO 128x64x128.
+BWD_INTRA_FLOP_PER_ITEM = 2 * (524288 + 43690 + 1048576 + 3 * 266240 + 1048576 + 524288 + 3 * 1048576 + 2 * 524288)
+BWD_CHAIN_FLOP_PER_ITEM = 2 * (128 * 128 * 128 + 128 * 64 * 128)
+# fp32 FMA peak of the CUDA cores: 148 SMs x 128 lanes x 2 FLOP x 1.965 GHz (unit counts and
+# the maximum SM clock; no measured figure exists for this unit)
+FP32_FMA_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+
+
 def run_backward(args, torch, kda, dev, stream, max_over_ranks, barrier):
     """kda_chunk_bwd on the prefill shape (B=1, T=8192, H=32, bf16 inputs and dL/do,
     an initial state and dL/d(final state)): one call = the forward walk recomputed
@@ -437,9 +449,17 @@ def run_backward(args, torch, kda, dev, stream, max_over_ranks, barrier):
     prof = kda.profile_read()
     kda.profile_enable(False)
     kernels = {k: dict(launches_per_call=v[0] / n, ms_per_call=v[1] / n) for k, v in prof.items()}
+    # the two backward kernels run fp32 FMA on the CUDA cores: roofline against that ALU peak
+    items = B * (T // 64) * H
+    alu = {}
+    for name, flop in (("intra_bwd", BWD_INTRA_FLOP_PER_ITEM), ("chain_bwd", BWD_CHAIN_FLOP_PER_ITEM)):
+        if name in kernels and kernels[name]["ms_per_call"] > 0:
+            tf = flop * items / (kernels[name]["ms_per_call"] * 1e-3) / 1e12
+            alu[name] = dict(bound="alu", achieved=tf, peak=FP32_FMA_TFLOPS, unit="TFLOP/s",
+                             frac=tf / FP32_FMA_TFLOPS, flop_per_launch=flop * items)
     return {"workload": f"KDA backward B={B} T={T} H={H} bf16 inputs and dL/do, fp32 gradients, initial state "
                         "and final-state gradient", "ms_per_call": ms, "tokens_per_s": B * T / (ms * 1e-3),
-            "kernels": kernels}
+            "kernels": kernels, "roofline": alu}
 
 
 def run_kcp(args, torch, kda, dev, stream, max_over_ranks, barrier):
