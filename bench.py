@@ -230,6 +230,8 @@ def run_ours(args, peaks):
 
     # per-device steps of context parallelism across devices (ranks emulated on this GPU)
     kcp = run_kcp(args, torch, kda, dev, stream, mor, barrier)
+    if ws_n > 1:  # and across the ranks of this job: one sequence split over all of them
+        kcp["across_ranks"] = run_kcp_ranks(args, torch, kda, dev, stream, rank, ws_n, mor, barrier)
 
     # backward of the prefill on the same shape
     bwd = run_backward(args, torch, kda, dev, stream, mor, barrier)
@@ -516,6 +518,39 @@ def run_kcp(args, torch, kda, dev, stream, max_over_ranks, barrier):
     res["overhead_vs_plain"] = res["device_ms"] / res["plain_ms"]
     res["sequence_tokens_per_s_without_gather"] = R * T / (res["device_ms"] * 1e-3)
     return res
+
+
+def run_kcp_ranks(args, torch, kda, dev, stream, rank, world, max_over_ranks, barrier):
+    """One sequence of world x 8192 tokens (32 heads, fused gate) split over the ranks of
+    this job: every rank runs kcp.kcp_prefill on its segment (transition, NCCL all-gather
+    of the 4 MiB of segment maps, compose, finish).  Time = max over ranks."""
+    from linear_attention_recurrence_06_b200 import kcp, synth
+    T, H = KCP_SHAPE["T_rank"], KCP_SHAPE["H"]
+    tb = synth.tokens(400, rank * T, T, H, D, D, bf16=True, gate=True)
+    x = {n: torch.from_numpy(np.ascontiguousarray(getattr(tb, n))).to(torch.bfloat16).to(dev)
+         for n in ("q", "k", "v", "log_alpha", "beta", "g")}
+    x = {n: t.view(1, T, H, -1) if n != "beta" else t.view(1, T, H) for n, t in x.items()}
+
+    def f():
+        return kcp.kcp_prefill(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], None, gate=x["g"],
+                               stream=stream)
+
+    for _ in range(3):
+        f()
+    n = max(3, min(args.steps, 10))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(n):
+        f()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    ms = max_over_ranks(e0.elapsed_time(e1) / n)
+    return {"ranks": world, "tokens_per_rank": T, "ms_per_call": ms,
+            "sequence_tokens_per_s": world * T / (ms * 1e-3),
+            "all_gather_bytes_per_rank": 2 * H * D * D * 4}
 
 
 def run_e2e(args, torch, kda, hq, out, fs, ws, stream, max_over_ranks, barrier):
