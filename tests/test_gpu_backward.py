@@ -86,3 +86,25 @@ def test_backward_per_sequence_and_token_tail():
         tail = slice(inp["cu"][n] + (L - 1) // 64 * 64, inp["cu"][n + 1])
         assert rel_l2(mine["dk"][tail], ref["dk"][tail]) <= REL_L2_TOL, f"seq {n} tail dk"
         assert rel_l2(mine["d_init"][n], ref["d_init"][n]) <= REL_L2_TOL, f"seq {n} d_init"
+
+
+def test_backward_fixed_length_batch():
+    """B = 2 sequences of 100 tokens without cu_seqlens ([B, T, H, 128] layout)."""
+    torch = _torch()
+    import linear_attention_recurrence_06_b200 as kda
+    B, T, H = 2, 100, 2
+    inp = make_prefill(99, [T] * B, H, bf16=True, init=True)
+    dt = torch.bfloat16
+    d_o = synth.normal(1099, synth.TAG_V, (B * T, H, D), 1.0, True)
+    d_fin = synth.states(2099, B, H, D, D, std=0.5)
+    q, k, v, la = (dev(inp[x], dt).view(B, T, H, D) for x in ("q", "k", "v", "log_alpha"))
+    b = dev(inp["beta"], dt).view(B, T, H)
+    g = kda.chunk_bwd(q, k, v, la, b, dev(d_o, dt).view(B, T, H, D), dev(inp["s0"], torch.float32),
+                      dev(d_fin, torch.float32), scale=0.2)
+    torch.cuda.synchronize()
+    ref = oracle.kda_recurrent_bwd(inp["q"], inp["k"], inp["v"], inp["log_alpha"], inp["beta"], d_o, inp["s0"],
+                                   d_fin, inp["cu"], scale=0.2)
+    mine = {"dq": host(g["dq"]).reshape(B * T, H, D), "dk": host(g["dk"]).reshape(B * T, H, D),
+            "dv": host(g["dv"]).reshape(B * T, H, D), "dlog_alpha": host(g["dlog_alpha"]).reshape(B * T, H, D),
+            "dbeta": host(g["dbeta"]).reshape(B * T, H), "d_init": host(g["d_initial_state"])}
+    _check(mine, ref, "B=2 fixed length")
