@@ -371,24 +371,21 @@ __global__ void __launch_bounds__(BI_THREADS, 1) bwd_intra_kernel(const BwdArgs 
             __syncthreads();
         }
 
-        // ---- P2: M^-1, M = I + Diag(beta) A (unit lower triangular), one column per thread
-        if (tid < CH) {
-            const int cc = tid;
+        // ---- P2: M^-1, M = I + Diag(beta) A (unit lower triangular): column cc by the
+        // 8 lanes tid / 8 == cc, forward substitution down the rows, the sum over earlier
+        // rows split over the lanes and reduced by shuffles (all lanes take part in every
+        // shuffle; loop trip counts differ, the warp reconverges before them)
+        {
+            const int cc = tid >> 3, part = tid & 7;
             for (int t = 0; t < CH; ++t) {
-                float x;
-                if (t < cc) x = 0.f;
-                else if (t == cc) x = 1.f;
-                else {
-                    float s0 = 0.f, s1 = 0.f;
-                    int s = cc;
-                    for (; s + 1 < t; s += 2) {
-                        s0 += sA[t * LP + s] * sMi[s * LP + cc];
-                        s1 += sA[t * LP + s + 1] * sMi[(s + 1) * LP + cc];
-                    }
-                    if (s < t) s0 += sA[t * LP + s] * sMi[s * LP + cc];
-                    x = -sBeta[t] * (s0 + s1);
-                }
-                sMi[t * LP + cc] = x;
+                float p = 0.f;
+                for (int s = cc + part; s < t; s += 8) p += sA[t * LP + s] * sMi[s * LP + cc];
+                p += __shfl_xor_sync(0xFFFFFFFFu, p, 1);
+                p += __shfl_xor_sync(0xFFFFFFFFu, p, 2);
+                p += __shfl_xor_sync(0xFFFFFFFFu, p, 4);
+                const float x = t < cc ? 0.f : (t == cc ? 1.f : -sBeta[t] * p);
+                if (part == 0) sMi[t * LP + cc] = x;
+                __syncwarp();
             }
         }
         // factors K o Gam (rows 0-63) and K^C = K o e^{g_C - g} (rows 64-127)
