@@ -725,6 +725,26 @@ def run_ncu_case(args):
     return {"ncu_case": f"prefill T={T} H={H}", "calls": args.warmup + args.steps, "status": kda.query_status(ws)}
 
 
+def run_ncu_bwd_case(args):
+    """Small backward case for profiler captures: `warmup + steps` calls of kda_chunk_bwd
+    on T = --ncu-bwd-tokens tokens, H = 32, bf16 inputs and dL/do, no timing."""
+    import torch
+    import linear_attention_recurrence_06_b200 as kda
+    from linear_attention_recurrence_06_b200 import synth
+    T, H = args.ncu_bwd_tokens, PREFILL["H"]
+    tb = synth.tokens(500, 0, T, H, D, D, bf16=True)
+    up = {n: torch.from_numpy(np.ascontiguousarray(getattr(tb, n))).to(torch.bfloat16).cuda()
+          for n in ("q", "k", "v", "log_alpha", "beta")}
+    x = {n: t.view(1, T, H, -1) if n != "beta" else t.view(1, T, H) for n, t in up.items()}
+    d_o = torch.from_numpy(synth.normal(501, synth.TAG_V, (T, H, D), 1.0, True)).to(torch.bfloat16).cuda()
+    ws = torch.empty(kda.bwd_workspace_size(T, H, 1, T), dtype=torch.uint8, device="cuda")
+    for _ in range(args.warmup + args.steps):
+        kda.chunk_bwd(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], d_o.view(1, T, H, D), None, None,
+                      scale=D ** -0.5, workspace=ws)
+    torch.cuda.synchronize()
+    return {"ncu_case": f"backward T={T} H={H}", "calls": args.warmup + args.steps, "status": kda.query_status(ws)}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -736,12 +756,16 @@ def main():
     ap.add_argument("--ref-tokens", type=int, default=256)
     ap.add_argument("--ncu-tokens", type=int, default=0,
                     help="profiler case: only run warmup+steps prefill calls on this many tokens")
+    ap.add_argument("--ncu-bwd-tokens", type=int, default=0,
+                    help="profiler case: only run warmup+steps backward calls on this many tokens")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     peaks = load_peaks()
     if args.ncu_tokens > 0:
         line = run_ncu_case(args)
+    elif args.ncu_bwd_tokens > 0:
+        line = run_ncu_bwd_case(args)
     else:
         line = run_reference(args) if args.impl == "reference" else run_ours(args, peaks)
     if line is not None:
