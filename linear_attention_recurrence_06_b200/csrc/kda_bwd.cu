@@ -303,7 +303,8 @@ __global__ void __launch_bounds__(BI_THREADS, 1) bwd_intra_kernel(const BwdArgs 
     float* sGC = reinterpret_cast<float*>(sm + BI_GC);
     float* sDgC = reinterpret_cast<float*>(sm + BI_DGC);
     const int tid = threadIdx.x, H = a.H;
-    // register-owned elements: tokens 4 tg .. 4 tg + 3, key channels 4 ig .. 4 ig + 3
+    // register-owned elements: tokens 4 tg .. 4 tg + 3, key channels ig + 32 y (y = 0..3;
+    // interleaved so that a warp's 32 lanes touch 32 consecutive channels)
     const int tg = tid >> 5, ig = tid & 31;
 
     for (int64_t item = blockIdx.x; item < n_items; item += gridDim.x) {
@@ -498,7 +499,8 @@ __global__ void __launch_bounds__(BI_THREADS, 1) bwd_intra_kernel(const BwdArgs 
             __syncthreads();
             // (d) dP += dO U^T (s <= t);  dM -= Y U^T (s < t)
             {
-                const int t = tid >> 3, s0 = (tid & 7) * 8;
+                // rows s = sl + 8 x: the 8 lanes sharing t read 8 consecutive rows of U
+                const int t = tid >> 3, sl = tid & 7;
                 float dp[8], dm[8];
 #pragma unroll
                 for (int x = 0; x < 8; ++x) dp[x] = dm[x] = 0.f;
@@ -506,14 +508,14 @@ __global__ void __launch_bounds__(BI_THREADS, 1) bwd_intra_kernel(const BwdArgs 
                     const float o = sDO[t * QP + j], y = sDU[t * QP + j];
 #pragma unroll
                     for (int x = 0; x < 8; ++x) {
-                        const float u = sU[(s0 + x) * QP + j];
+                        const float u = sU[(sl + 8 * x) * QP + j];
                         dp[x] += o * u;
                         dm[x] -= y * u;
                     }
                 }
 #pragma unroll
                 for (int x = 0; x < 8; ++x) {
-                    const int s = s0 + x;
+                    const int s = sl + 8 * x;
                     if (s <= t) sdP[t * LP + s] += dp[x];
                     if (s < t) sdM[t * LP + s] += dm[x];
                 }
@@ -525,7 +527,7 @@ __global__ void __launch_bounds__(BI_THREADS, 1) bwd_intra_kernel(const BwdArgs 
                     float4 s0v[4], dsv[4];
 #pragma unroll
                     for (int y = 0; y < 4; ++y) {
-                        const int i = 4 * ig + y;
+                        const int i = ig + 32 * y;
                         s0v[y] = S0 ? __ldg(reinterpret_cast<const float4*>(S0 + (size_t)i * DV + j0 + j))
                                     : make_float4(0.f, 0.f, 0.f, 0.f);
                         dsv[y] = __ldg(reinterpret_cast<const float4*>(dSC + (size_t)i * DV + j0 + j));
@@ -577,7 +579,7 @@ __global__ void __launch_bounds__(BI_THREADS, 1) bwd_intra_kernel(const BwdArgs 
             const int t = 4 * tg + x;
 #pragma unroll
             for (int y = 0; y < 4; ++y) {
-                const int i = 4 * ig + y;
+                const int i = ig + 32 * y;
                 float kv = 0.f, qv = 0.f;
                 if (t < L) {
                     const size_t idx = ((size_t)(t0 + t) * H + h) * DK + i;
@@ -594,7 +596,7 @@ __global__ void __launch_bounds__(BI_THREADS, 1) bwd_intra_kernel(const BwdArgs 
         }
         if (tg == 0) {
 #pragma unroll
-            for (int y = 0; y < 4; ++y) atomicAdd(&sDgC[4 * ig + y], __expf(sGC[4 * ig + y]) * rowS[y]);
+            for (int y = 0; y < 4; ++y) atomicAdd(&sDgC[ig + 32 * y], __expf(sGC[ig + 32 * y]) * rowS[y]);
         }
         __syncthreads();
 
@@ -632,7 +634,7 @@ __global__ void __launch_bounds__(BI_THREADS, 1) bwd_intra_kernel(const BwdArgs 
                     const int tl = t - r;
 #pragma unroll
                     for (int y = 0; y < 4; ++y) {
-                        const int i = 4 * ig + y;
+                        const int i = ig + 32 * y;
                         dkk[x][y] += sC[(0 * 16 + tl) * DK + i];
                         dqb[x][y] += sC[(1 * 16 + tl) * DK + i];
                         dg[x][y] += sC[(2 * 16 + tl) * DK + i];
@@ -641,7 +643,7 @@ __global__ void __launch_bounds__(BI_THREADS, 1) bwd_intra_kernel(const BwdArgs 
                 if (t < r + 16 && t < L) {  // t as an earlier token s: dKout_t
 #pragma unroll
                     for (int y = 0; y < 4; ++y) {
-                        const int i = 4 * ig + y;
+                        const int i = ig + 32 * y;
                         float dko = 0.f;
                         for (int tl = (t > r ? t - r : 0); tl < 16; ++tl) {
                             const int tt = r + tl;
@@ -663,13 +665,15 @@ __global__ void __launch_bounds__(BI_THREADS, 1) bwd_intra_kernel(const BwdArgs 
         for (int x = 0; x < 4; ++x) {
             const int t = 4 * tg + x;
             if (t < L) {
-                const size_t base = ((size_t)(t0 + t) * H + h) * DK + 4 * ig;
-                *reinterpret_cast<float4*>(a.dq + base) =
-                    make_float4(a.scale * dqb[x][0], a.scale * dqb[x][1], a.scale * dqb[x][2], a.scale * dqb[x][3]);
-                *reinterpret_cast<float4*>(a.dk + base) = make_float4(dkk[x][0], dkk[x][1], dkk[x][2], dkk[x][3]);
+                const size_t base = ((size_t)(t0 + t) * H + h) * DK + ig;
+#pragma unroll
+                for (int y = 0; y < 4; ++y) {
+                    a.dq[base + 32 * y] = a.scale * dqb[x][y];
+                    a.dk[base + 32 * y] = dkk[x][y];
+                }
             }
 #pragma unroll
-            for (int y = 0; y < 4; ++y) sF[t * FP + 4 * ig + y] = dg[x][y];
+            for (int y = 0; y < 4; ++y) sF[t * FP + ig + 32 * y] = dg[x][y];
         }
         __syncthreads();
         if (tid < DK) {
