@@ -131,6 +131,9 @@ __global__ void __launch_bounds__(CB_THREADS, 1) chain_bwd_kernel(const BwdArgs 
                            ld_in(a.d_o, base + 2, a.in_bf16), ld_in(a.d_o, base + 3, a.in_bf16));
     };
     float4 dO_next = load_dO(nck - 1);
+    uint32_t m_off[8];  // sw128_off(mm, i & 63) for mm = 0..7
+#pragma unroll
+    for (int mm = 0; mm < 8; ++mm) m_off[mm] = sw128_off((uint32_t)mm, (uint32_t)(i & 63));
     for (int r = 0; r < nck; ++r) {
         const int c = nck - 1 - r, b = r & 1;
         const int64_t t0 = s_beg + (int64_t)c * CH;
@@ -154,16 +157,22 @@ __global__ void __launch_bounds__(CB_THREADS, 1) chain_bwd_kernel(const BwdArgs 
         float acc[8];
 #pragma unroll
         for (int j = 0; j < 8; ++j) acc[j] = gam * dS[j];
-        // - M_lr^T dS: column i of M_lr against every row of dS
+        // - M_lr^T dS: column i of M_lr against every row of dS.  Element (m, i) of the
+        // K-major SW128 image sits at (i >> 6) * 16384 + sw128_off(m, i & 63); for
+        // m = 8 m8 + mm that is m8 * 1024 + off[mm], with off[] fixed per thread.
         const uint8_t* mcol = buf + SO_M + (size_t)(i >> 6) * 16384;
-#pragma unroll 4
-        for (int m = 0; m < DK; ++m) {
-            const uint16_t bits = *reinterpret_cast<const uint16_t*>(mcol + sw128_off((uint32_t)m, (uint32_t)(i & 63)));
-            const float mv = __uint_as_float((uint32_t)bits << 16);
-            const float4 d0 = reinterpret_cast<const float4*>(sdS + m * DVS + 8 * cq)[0];
-            const float4 d1 = reinterpret_cast<const float4*>(sdS + m * DVS + 8 * cq)[1];
-            acc[0] -= mv * d0.x; acc[1] -= mv * d0.y; acc[2] -= mv * d0.z; acc[3] -= mv * d0.w;
-            acc[4] -= mv * d1.x; acc[5] -= mv * d1.y; acc[6] -= mv * d1.z; acc[7] -= mv * d1.w;
+        for (int m8 = 0; m8 < DK / 8; ++m8) {
+            const uint8_t* mrow = mcol + m8 * 1024;
+            const float* drow = sdS + m8 * 8 * DVS + 8 * cq;
+#pragma unroll
+            for (int mm = 0; mm < 8; ++mm) {
+                const uint16_t bits = *reinterpret_cast<const uint16_t*>(mrow + m_off[mm]);
+                const float mv = __uint_as_float((uint32_t)bits << 16);
+                const float4 d0 = reinterpret_cast<const float4*>(drow + mm * DVS)[0];
+                const float4 d1 = reinterpret_cast<const float4*>(drow + mm * DVS)[1];
+                acc[0] -= mv * d0.x; acc[1] -= mv * d0.y; acc[2] -= mv * d0.z; acc[3] -= mv * d0.w;
+                acc[4] -= mv * d1.x; acc[5] -= mv * d1.y; acc[6] -= mv * d1.z; acc[7] -= mv * d1.w;
+            }
         }
         // + Q'^T dO: column i of Q' against every token row of dO
         const uint8_t* qcol = buf + SO_Q + (size_t)(i >> 3) * 1024 + (i & 7) * 16;
