@@ -12,8 +12,9 @@ against HBM.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
-N > 1 is launched with torch.distributed.run (one rank per GPU, NCCL).  Rank 0
-prints ONE JSON line.  `--impl reference` times the fp64 CPU oracle (the only
+N > 1: one rank per GPU over NCCL.  Launched under torch.distributed.run the
+script uses its RANK / WORLD_SIZE; launched plainly with --gpus N it starts the
+N ranks itself through torch.distributed.run.  Rank 0 prints ONE JSON line.  `--impl reference` times the fp64 CPU oracle (the only
 reference implementation that exists for this method) on rank 0.
 """
 from __future__ import annotations
@@ -156,6 +157,9 @@ def run_ours(args, peaks):
     if ws_n > 1:
         import datetime
         import torch.distributed as dist
+        # NCCL prints its communicator set-up, so the number of ranks that formed is on record
+        os.environ.setdefault("NCCL_DEBUG", "INFO")
+        os.environ.setdefault("NCCL_DEBUG_SUBSYS", "INIT")
         torch.cuda.set_device(local)
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local))
@@ -236,6 +240,12 @@ def run_ours(args, peaks):
     # backward of the prefill on the same shape
     bwd = run_backward(args, torch, kda, dev, stream, mor, barrier)
 
+    # the packed varlen and the long-context workloads
+    torch.cuda.empty_cache()
+    varlen = run_varlen(args, torch, kda, dev, stream, mor, barrier)
+    torch.cuda.empty_cache()
+    long_ctx = run_long(args, torch, kda, dev, stream, mor, barrier)
+
     if dist is not None:
         dist.barrier()
         dist.destroy_process_group()
@@ -265,7 +275,8 @@ def run_ours(args, peaks):
                    "l2": "inputs larger than L2 (q,k,v,log_alpha,gate,beta = 336 MB per step)"},
         "prefill_tflops": tflops, "prefill_tensor_frac": tflops / peaks["bf16_tflops_sustained"],
         "roofline": roof, "kernels": kernels, "decode": dec, "e2e": e2e, "segment_parallel": seg,
-        "kcp_per_device": kcp, "backward": bwd, "gpu_launches": int(round(launches_per_step * args.steps)),
+        "kcp_per_device": kcp, "backward": bwd, "varlen": varlen, "long_context": long_ctx,
+        "gpu_launches": int(round(launches_per_step * args.steps)),
         "clocks": clocks,
     }
     if ws_n == 1 and not args.no_cpu_baseline:
@@ -391,6 +402,106 @@ def run_segmented(args, torch, kda, dev, stream, max_over_ranks, barrier):
         res[name] = {"ms_per_call": ms, "tokens_per_s": T / (ms * 1e-3)}
         del ws
     res["speedup"] = res["plain"]["ms_per_call"] / res["segmented"]["ms_per_call"]
+    return res
+
+
+VARLEN = dict(n_seqs=16, lo=512, hi=16384, H=32)
+LONG = dict(T=1 << 20, H=32, pool=65536)
+# algorithmic bytes per token-head without the gate: q, k, v, log_alpha in + o out (bf16) + beta
+PREFILL_NOGATE_BYTES_PER_TH = 5 * 256 + 2
+
+
+def _time_calls(torch, f, n, stream, max_over_ranks, barrier):
+    for _ in range(3):
+        f()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(n):
+        f()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    return max_over_ranks(e0.elapsed_time(e1) / n)
+
+
+def _pool_tokens(torch, dev, seed, n, H):
+    """n tokens of every input (bf16, the workload's distributions) on the device."""
+    from linear_attention_recurrence_06_b200 import synth
+    tb = synth.tokens(seed, 0, n, H, D, D, bf16=True)
+    return {k: torch.from_numpy(np.ascontiguousarray(getattr(tb, k))).to(torch.bfloat16).to(dev)
+            for k in ("q", "k", "v", "log_alpha", "beta")}
+
+
+def run_varlen(args, torch, kda, dev, stream, max_over_ranks, barrier):
+    """Packed varlen prefill: 16 sequences with lengths uniform on [512, 16384]
+    (seeded), H=32, bf16, random fp32 initial states N(0, 0.02^2), final states
+    returned.  Token values come from one 16,384-token pool of the same
+    distributions (sequence n takes its first L_n tokens): the kernels' time does
+    not depend on the values."""
+    from linear_attention_recurrence_06_b200 import synth
+    n, H = VARLEN["n_seqs"], VARLEN["H"]
+    lengths = synth.varlen_lengths(0, n, VARLEN["lo"], VARLEN["hi"])
+    cu = synth.cu_from_lengths(lengths)
+    T = int(cu[-1])
+    pool = _pool_tokens(torch, dev, 500, VARLEN["hi"], H)
+    x = {}
+    for k, t in pool.items():
+        x[k] = torch.cat([t[:int(L)] for L in lengths]).view((1, T, H) + tuple(t.shape[2:]))
+    s0 = torch.from_numpy(synth.states(501, n, H, D, D)).to(dev)
+    cu_d = torch.from_numpy(cu.astype(np.int32)).to(dev)
+    out = torch.empty((1, T, H, D), dtype=torch.bfloat16, device=dev)
+    fs = torch.empty((n, H, D, D), dtype=torch.float32, device=dev)
+    _, full = kda.workspace_size(T, H, n, int(lengths.max()))
+    ws = torch.empty(full, dtype=torch.uint8, device=dev)
+
+    def f():
+        kda.chunk_fwd(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], s0, cu_seqlens=cu_d,
+                      max_seqlen=int(lengths.max()), out=out, final_state=fs, workspace=ws, stream=stream)
+
+    ms = _time_calls(torch, f, max(5, min(args.steps, 20)), stream, max_over_ranks, barrier)
+    th = T * H
+    nbytes = PREFILL_NOGATE_BYTES_PER_TH * th + 2 * n * H * D * D * 4
+    peaks = load_peaks()
+    return {"workload": f"KDA varlen prefill, {n} sequences, lengths uniform on [{VARLEN['lo']}, {VARLEN['hi']}] "
+                        f"(seed 0: {T} tokens), H={H}, bf16, fp32 initial and final states",
+            "tokens": T, "ms_per_call": ms, "tokens_per_s": T / (ms * 1e-3),
+            "algorithmic_bytes": nbytes, "hbm_bound_ms": nbytes / (peaks["hbm_gbs"] * 1e9) * 1e3,
+            "hbm_frac": nbytes / (ms * 1e-3) / (peaks["hbm_gbs"] * 1e9),
+            "tflops": PREFILL_FLOP_PER_TH * th / (ms * 1e-3) / 1e12, "passes": 1}
+
+
+def run_long(args, torch, kda, dev, stream, max_over_ranks, barrier):
+    """Long-context prefill: B=1, T=2^20, H=32, bf16, zero initial state, one pass
+    (the whole-sequence workspace).  Token values: a 65,536-token pool of the
+    workload's distributions repeated 16 times (timing does not depend on the
+    values; the parity test runs fresh tokens throughout)."""
+    T, H, P = LONG["T"], LONG["H"], LONG["pool"]
+    pool = _pool_tokens(torch, dev, 600, P, H)
+    x = {k: t.repeat((T // P,) + (1,) * (t.dim() - 1)).view((1, T, H) + tuple(t.shape[2:])) for k, t in pool.items()}
+    del pool
+    out = torch.empty((1, T, H, D), dtype=torch.bfloat16, device=dev)
+    fs = torch.empty((1, H, D, D), dtype=torch.float32, device=dev)
+    _, full = kda.workspace_size(T, H, 1, T)
+    ws = torch.empty(full, dtype=torch.uint8, device=dev)
+
+    def f():
+        kda.chunk_fwd(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], None, out=out, final_state=fs,
+                      workspace=ws, stream=stream)
+
+    ms = _time_calls(torch, f, 3, stream, max_over_ranks, barrier)
+    th = T * H
+    nbytes = PREFILL_NOGATE_BYTES_PER_TH * th
+    peaks = load_peaks()
+    res = {"workload": f"KDA long-context prefill B=1 T={T} H={H} bf16, zero initial state",
+           "tokens": T, "ms_per_call": ms, "tokens_per_s": T / (ms * 1e-3),
+           "algorithmic_bytes": nbytes, "hbm_bound_ms": nbytes / (peaks["hbm_gbs"] * 1e9) * 1e3,
+           "hbm_frac": nbytes / (ms * 1e-3) / (peaks["hbm_gbs"] * 1e9),
+           "workspace_bytes": full, "passes": 1,
+           "sequential_chunk_steps": T // 64}
+    del x, out, ws
+    torch.cuda.empty_cache()
     return res
 
 
@@ -703,6 +814,24 @@ def run_reference(args):
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
+def run_ncu_decode_case(args):
+    """Decode case for profiler captures: `warmup + steps` single decode steps on
+    the 256 x 32 workload (512 MiB fp32 state), no timing."""
+    import torch
+    import linear_attention_recurrence_06_b200 as kda
+    from linear_attention_recurrence_06_b200 import synth
+    Bd, H = DECODE["Bd"], DECODE["H"]
+    state = torch.from_numpy(synth.states(100, Bd, H, D, D)).cuda()
+    tb = synth.tokens(200, 0, Bd, H, D, D, bf16=True)
+    t = {n: torch.from_numpy(np.ascontiguousarray(getattr(tb, n))).to(torch.bfloat16).cuda()
+         for n in ("q", "k", "v", "log_alpha", "beta")}
+    o = torch.empty((Bd, H, D), dtype=torch.bfloat16, device="cuda")
+    for _ in range(args.warmup + args.steps):
+        kda.decode_step(state, t["q"], t["k"], t["v"], t["log_alpha"], t["beta"], out=o)
+    torch.cuda.synchronize()
+    return {"ncu_case": f"decode Bd={Bd} H={H}", "calls": args.warmup + args.steps}
+
+
 def run_ncu_case(args):
     """Small prefill case for profiler captures: `warmup + steps` calls of
     kda_chunk_fwd (fused gate) on T = --ncu-tokens tokens, H = 32, no timing."""
@@ -745,6 +874,50 @@ def run_ncu_bwd_case(args):
     return {"ncu_case": f"backward T={T} H={H}", "calls": args.warmup + args.steps, "status": kda.query_status(ws)}
 
 
+def free_port() -> int:
+    import socket
+    with socket.socket(socket.AF_INET, socket.SOCK_STREAM) as so:
+        so.bind(("127.0.0.1", 0))
+        return so.getsockname()[1]
+
+
+def launch_ranks(n: int, argv) -> int:
+    """Re-runs this script as n ranks of one node (torch.distributed.run, one
+    process per GPU, rendezvous on 127.0.0.1).  The ranks' output passes through;
+    rank 0 prints the JSON line.  Returns the launcher's exit code."""
+    env = dict(os.environ)
+    # NCCL prints its communicator set-up (ranks, transport) so the rank count is on record
+    env.setdefault("NCCL_DEBUG", "INFO")
+    env.setdefault("NCCL_DEBUG_SUBSYS", "INIT")
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes", "1", "--nproc-per-node", str(n),
+           "--master-addr", "127.0.0.1", "--master-port", str(free_port()), os.path.abspath(__file__), *argv]
+    return subprocess.run(cmd, env=env).returncode
+
+
+def run_dry(args):
+    """The multi-rank plumbing without a GPU: every rank joins a gloo process
+    group, reports its rank and takes part in the max-over-ranks reduction that
+    the timed runs use; rank 0 prints what it saw."""
+    import datetime
+    import torch
+    import torch.distributed as dist
+    ws_n, rank, _ = dist_env()
+    if ws_n > 1:
+        dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=60))
+    ranks = torch.zeros(ws_n, dtype=torch.float64)
+    ranks[rank] = 1.0
+    if ws_n > 1:
+        dist.all_reduce(ranks)
+    ms = max_over_ranks(float(rank + 1), dist if ws_n > 1 else None)
+    if ws_n > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return None
+    return {"dry_run": True, "n_gpus": ws_n, "ranks_reported": int(ranks.sum().item()), "max_over_ranks": ms,
+            "value": whole_job_rate(ws_n, 1.0, ms)}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -758,11 +931,28 @@ def main():
                     help="profiler case: only run warmup+steps prefill calls on this many tokens")
     ap.add_argument("--ncu-bwd-tokens", type=int, default=0,
                     help="profiler case: only run warmup+steps backward calls on this many tokens")
+    ap.add_argument("--ncu-decode", action="store_true",
+                    help="profiler case: only run warmup+steps decode steps on the 256 x 32 workload")
+    ap.add_argument("--dry-run", action="store_true",
+                    help="no GPU work: ranks join a gloo group and report (tests the multi-rank launch)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    ws_env = os.environ.get("WORLD_SIZE")
+    if args.gpus > 1 and ws_env is None:
+        # not launched by torch.distributed.run: start one rank per GPU here
+        sys.exit(launch_ranks(args.gpus, sys.argv[1:]))
+    if ws_env is not None and int(ws_env) != args.gpus:
+        ap.error(f"--gpus {args.gpus} but WORLD_SIZE={ws_env}: launch one rank per GPU")
+    if args.dry_run:
+        line = run_dry(args)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return
     peaks = load_peaks()
-    if args.ncu_tokens > 0:
+    if args.ncu_decode:
+        line = run_ncu_decode_case(args)
+    elif args.ncu_tokens > 0:
         line = run_ncu_case(args)
     elif args.ncu_bwd_tokens > 0:
         line = run_ncu_bwd_case(args)

@@ -360,6 +360,20 @@ KDA_API kda_status kda_gate_norm(const void* o, const void* gate, const float* n
 KDA_API kda_status kda_query_status(void* workspace, void* stream);
 
 /*
+ * kda_test_drop_tile_load -- test hook for the device-side failure path (no
+ * counterpart on the pages).  The next kda_chunk_fwd-family call with bf16
+ * inputs in this process runs its chunk-local kernel with one change: CTA 0
+ * does not issue one of the four tile loads of its first item, and its wait
+ * for them gives up after wait_limit_ns (1e3 .. 1e9 ns) instead of the usual
+ * second.  That CTA then stops; the call returns KDA_OK, its outputs are
+ * undefined, and kda_query_status on its workspace returns KDA_ERR_TIMEOUT.
+ * The process and the GPU context stay usable: the next call is normal.
+ * wait_limit_ns = 0 cancels a pending drop.  Host-side only; not
+ * thread-safe.  KDA_ERR_INVALID_ARG for any other limit outside the range.
+ */
+KDA_API kda_status kda_test_drop_tile_load(unsigned long long wait_limit_ns);
+
+/*
  * kda_chunk_fwd_noalloc -- kda_chunk_fwd for callers that cannot allocate
  * device memory.  (No counterpart on the pages: it is a packaging of
  * kda_chunk_fwd, not part of the method.)
@@ -386,7 +400,15 @@ KDA_API kda_status kda_query_status(void* workspace, void* stream);
  *    call's contents (the call clears the parts that must start at zero
  *    itself).  Calls that overlap on the GPU (different streams without
  *    ordering, or different host threads) race on it: order them.
- *  - kda_query_status does not apply (there is no caller-visible workspace).
+ *  - Errors the kernels detect on the device (a bounded wait that gave up,
+ *    cu_seqlens that contradict T or max_seqlen) are recorded in a status word
+ *    at the start of the static array; read them with
+ *    kda_chunk_fwd_noalloc_query_status (kda_query_status takes a workspace,
+ *    and this entry point has none).  Each call clears the word first, so it
+ *    describes the last call on the device.
+ *  - The array's device address is cached per device; after a cudaDeviceReset
+ *    the module is unloaded and the cached address is stale, so do not call
+ *    this entry point again in that process after a reset.
  */
 #define KDA_NOALLOC_SCRATCH_BYTES (64u * 1024u * 1024u)
 
@@ -398,6 +420,15 @@ KDA_API kda_status kda_chunk_fwd_noalloc(const void* q, const void* k, const voi
                                  kda_dtype in_dtype, kda_dtype out_dtype, float scale,
                                  const void* gate, const float* norm_weight, float eps,
                                  void* stream);
+
+/*
+ * kda_chunk_fwd_noalloc_query_status -- synchronises `stream` and returns the
+ * device status word of the last kda_chunk_fwd_noalloc call on the current
+ * device (then clears it): KDA_OK, KDA_ERR_TIMEOUT or KDA_ERR_DEVICE_ARG, as
+ * kda_query_status does for a workspace.  Allocates nothing.  Returns
+ * KDA_ERR_CUDA if the array's address cannot be looked up.
+ */
+KDA_API kda_status kda_chunk_fwd_noalloc_query_status(void* stream);
 
 /*
  * Per-kernel device timing (a measurement aid, off by default).

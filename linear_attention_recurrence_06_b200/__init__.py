@@ -100,6 +100,12 @@ def load_library(path: str | None = None):
     lib.kda_gate_norm.argtypes = [vp, vp, vp, f32, vp, i64, i32, i32, i32, vp]
     lib.kda_query_status.restype = i32
     lib.kda_query_status.argtypes = [vp, vp]
+    lib.kda_chunk_fwd_noalloc.restype = i32
+    lib.kda_chunk_fwd_noalloc.argtypes = list(lib.kda_chunk_fwd.argtypes[:22]) + [vp]
+    lib.kda_chunk_fwd_noalloc_query_status.restype = i32
+    lib.kda_chunk_fwd_noalloc_query_status.argtypes = [vp]
+    lib.kda_test_drop_tile_load.restype = i32
+    lib.kda_test_drop_tile_load.argtypes = [ctypes.c_ulonglong]
     lib.kda_profile_enable.restype = i32
     lib.kda_profile_enable.argtypes = [i32]
     lib.kda_profile_read.restype = i32

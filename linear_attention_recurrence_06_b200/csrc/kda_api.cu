@@ -387,6 +387,12 @@ kda_status kda_profile_read(kda_kernel_time* out, int max_entries, int* n_entrie
     return st;
 }
 
+kda_status kda_test_drop_tile_load(unsigned long long wait_limit_ns) {
+    if (wait_limit_ns != 0 && (wait_limit_ns < 1000ull || wait_limit_ns > 1000000000ull)) return KDA_ERR_INVALID_ARG;
+    kda::set_test_tile_drop(wait_limit_ns);
+    return KDA_OK;
+}
+
 kda_status kda_query_status(void* workspace, void* stream) {
     if (!workspace) return KDA_ERR_INVALID_ARG;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);

@@ -80,6 +80,8 @@ struct ChunkArgs {
     int segs;                  // segments per sequence (segment-parallel prefill), else 1
     uint8_t* seg_ws;           // segment transition slots [n_seqs][segs][H], segment-parallel only
     float* trans_out;          // nullable: fp32 segment maps [2][n_seqs][H][dk][dk] (M, then B) instead of slots
+    unsigned long long wait_ns;  // limit of the intra kernel's tile-load wait (WAIT_LIMIT_NS unless a test shortens it)
+    int drop_tile;             // test hook: CTA 0 does not issue one tile load of its first item (its wait runs out)
 };
 
 // Token range [sb, se) of sequence n, clamped into [0, total tokens].
@@ -158,22 +160,22 @@ KDA_DEV uint4 pack8(const float* x) {
 //   RAW [0, 64K)     TMA tiles [64 tokens][128 ch] bf16: la @0, k @16K, q @32K, v @48K
 //   X   [64K, 136K)  phase 1 (MN-major, no swizzle, M/N = token): KQr 128x128 @0,
 //                             KC = [Kd 64 | Kb1 16 | Kb2 32 | Kb3 48] x 128 @32K
-//                    after round 1: Ti [64][64] @32K, Ph [64][64] @56K, inverse scratch @64K
+//                    after stage 1: Ti [64][64] @32K, Ph [64][64] @56K, inverse scratch @64K
 //   Y   [136K, 171K) A fp32 [64][68] @0, X fp32 [64][68] @17408;
 //                    later Wt [128][64] @0, Ut [128][64] @16K
-//   Z2  [171K, 219K) KGt, Vt, Ktt [128][64] (built while round 1 runs)
+//   Z2  [171K, 219K) KGt, Vt, Ktt [128][64] (built while stage 1 runs)
 //   misc             beta[64], G[5][128], tile totals[4][128], 2 mbarriers, TMEM base
 // The workspace slot is assembled in two regions ([Mlr | Qp | GamC] at X, [Bm | Ob]
 // at Z2) and leaves as four bulk copies: Mlr and Bm as soon as they are staged, the
 // rest at the end of the item.
-// TMEM (512 columns): round 1  A/P diag [0,64), off-diag [64,80) [80,112) [112,160)
-//                     round 2  Wt [160,224), Ut [224,288)
-//                     round 3  [Mlr | Bm] [0,256) (one N = 256 product), (PW)^T [256,320),
+// TMEM (512 columns): stage 1  A/P diag [0,64), off-diag [64,80) [80,112) [112,160)
+//                     stage 2  Wt [160,224), Ut [224,288)
+//                     stage 3  [Mlr | Bm] [0,256) (one N = 256 product), (PW)^T [256,320),
 //                              Ob = P Ut^T [320,448) (M = 64: token t in lane 32 (t / 16) + t % 16)
 constexpr int INTRA_THREADS = 512;
 constexpr uint32_t R_LA = 0, R_K = 16384, R_Q = 32768, R_V = 49152;
 constexpr uint32_t IX = 65536;
-// KC stacks the column operands of round 1 as N = 160 token rows of one MN-major image:
+// KC stacks the column operands of stage 1 as N = 160 token rows of one MN-major image:
 // rows [0,64) Kd, [64,80) Kb1, [80,112) Kb2, [112,160) Kb3 (K-group stride 160 * 16 B).
 constexpr uint32_t IX_KQR = IX + 0, IX_KC = IX + 32768;
 constexpr uint32_t KC_KG = 2560, KC_B1 = 64, KC_B2 = 80, KC_B3 = 112;
@@ -181,7 +183,7 @@ constexpr uint32_t IX_TI = IX + 32768, IX_PH = IX + 57344, IX_TMP = IX + 65536;
 constexpr uint32_t IY = IX + 73728;
 constexpr int LDA = 68;  // padded fp32 row stride of A and X (16-byte rows, spread banks)
 constexpr uint32_t IY_A = IY, IY_X = IY + 64 * LDA * 4, IY_WT = IY, IY_UT = IY + 16384;
-// Z2: the phase-2 operand images (built while round 1 runs), K-major SW128 [128 ch][64 tok]
+// Z2: the phase-2 operand images (built while stage 1 runs), K-major SW128 [128 ch][64 tok]
 constexpr uint32_t Z2 = IY + 35840;
 constexpr uint32_t Z2_KGT = Z2, Z2_VT = Z2 + 16384, Z2_KTT = Z2 + 32768;
 constexpr uint32_t IM = Z2 + 49152;
@@ -230,7 +232,7 @@ intra_kernel(const ChunkArgs a, const __grid_constant__ IntraMaps maps, const in
     float* s_tot = reinterpret_cast<float*>(sm + IM_TOT);  // [4][128]
     uint64_t* bar_raw = reinterpret_cast<uint64_t*>(sm + IM_BAR_RAW);
     uint64_t* bar_mma = reinterpret_cast<uint64_t*>(sm + IM_BAR_MMA);
-    uint64_t* bar_mma2 = reinterpret_cast<uint64_t*>(sm + IM_BAR_MMA2);  // second half of round 3
+    uint64_t* bar_mma2 = reinterpret_cast<uint64_t*>(sm + IM_BAR_MMA2);  // second half of stage 3
     uint32_t* s_tmem = reinterpret_cast<uint32_t*>(sm + IM_TMEM);
     // next item of this CTA: {item, t0} as int64 and {h, L} as int
     int64_t* s_next64 = reinterpret_cast<int64_t*>(sm + IM_NEXT);
@@ -267,12 +269,13 @@ intra_kernel(const ChunkArgs a, const __grid_constant__ IntraMaps maps, const in
         }
         return n_items;
     };
-    auto issue_raw = [&](int hh, int64_t tt) {
+    // drop: the test hook's missing tile (the barrier still expects its bytes)
+    auto issue_raw = [&](int hh, int64_t tt, bool drop) {
         mbar_arrive_expect_tx(bar_raw, 4u * 16384u);
         tma_load_2d(sm + R_LA, &maps.la, hh * DK, (int)tt, bar_raw);
         tma_load_2d(sm + R_K, &maps.k, hh * DK, (int)tt, bar_raw);
         tma_load_2d(sm + R_Q, &maps.q, hh * DK, (int)tt, bar_raw);
-        tma_load_2d(sm + R_V, &maps.v, hh * DV, (int)tt, bar_raw);
+        if (!drop) tma_load_2d(sm + R_V, &maps.v, hh * DV, (int)tt, bar_raw);
     };
 
     int64_t item = next_valid(blockIdx.x);
@@ -307,7 +310,7 @@ intra_kernel(const ChunkArgs a, const __grid_constant__ IntraMaps maps, const in
         item_info(a, item, hh, tt, LL);
         if (tid < CH) load_beta(tt, hh, LL);
         if constexpr (IN_BF16) {
-            if (tid == 0) issue_raw(hh, tt);
+            if (tid == 0) issue_raw(hh, tt, a.drop_tile && blockIdx.x == 0);
             raw_in_flight = true;
         }
     }
@@ -325,7 +328,9 @@ intra_kernel(const ChunkArgs a, const __grid_constant__ IntraMaps maps, const in
 
         if (tid < CH) s_beta[tid] = IN_BF16 ? __uint_as_float(beta_bits << 16) : __uint_as_float(beta_bits);
         if constexpr (IN_BF16) {
-            mbar_wait(bar_raw, ph_raw, a.status);
+            // a tile load that never completes ends the CTA's work, on every thread at once
+            const bool ok = mbar_wait(bar_raw, ph_raw, a.status, a.wait_ns);
+            if (__syncthreads_or(!ok)) break;
             ph_raw ^= 1;
             raw_in_flight = false;
         }
@@ -435,14 +440,14 @@ intra_kernel(const ChunkArgs a, const __grid_constant__ IntraMaps maps, const in
         __syncthreads();
         tc_fence_after();
 
-        // ---- round 1: [Kr;Qr] Kd^T and [Kr;Qr] Kb(b)^T
+        // ---- stage 1: [Kr;Qr] Kd^T and [Kr;Qr] Kb(b)^T
         if (tid == 0) {
             // one N = 160 product: [A/P diag | tile-1 | tile-2 | tile-3 off-diagonal] columns
             mma_mn<8, 2048, KC_KG>(tm + TM_AD, sb + IX_KQR, sb + IX_KC, idesc_bf16_major(128, 160, 1, 1));
             mma_commit(bar_mma);
         }
 
-        // ---- phase 2 operands while round 1 runs (K = token, own region Z2):
+        // ---- phase 2 operands while stage 1 runs (K = token, own region Z2):
         //      KGt = (K o Gam)^T, Vt = V^T, Ktt = Kt^T
         {
             const float eG = __expf(Gs);          // Gam_t = E1 e^{G_q4}
@@ -476,7 +481,7 @@ intra_kernel(const ChunkArgs a, const __grid_constant__ IntraMaps maps, const in
             const int64_t tt = s_next64[1];
             const int hh = s_next32[0], LL = s_next32[1];
             if constexpr (IN_BF16) {
-                if (tid == 0) issue_raw(hh, tt);
+                if (tid == 0) issue_raw(hh, tt, false);
                 raw_in_flight = true;
             }
             if (tid < CH) load_beta(tt, hh, LL);
@@ -683,7 +688,7 @@ intra_kernel(const ChunkArgs a, const __grid_constant__ IntraMaps maps, const in
         __syncthreads();
         tc_fence_after();
 
-        // ---- round 2: Wt = KGt Ti^T, Ut = Vt Ti^T
+        // ---- stage 2: Wt = KGt Ti^T, Ut = Vt Ti^T
         if (tid == 0) {
             mma_sw128<4, 128, 64>(tm + TM_WT, sdesc_k_sw128(sb + Z2_KGT), sdesc_k_sw128(sb + IX_TI), idesc_bf16(128, 64));
             mma_sw128<4, 128, 64>(tm + TM_UT, sdesc_k_sw128(sb + Z2_VT), sdesc_k_sw128(sb + IX_TI), idesc_bf16(128, 64));
@@ -709,7 +714,7 @@ intra_kernel(const ChunkArgs a, const __grid_constant__ IntraMaps maps, const in
         __syncthreads();
         tc_fence_after();
 
-        // ---- round 3: [Mlr | Bm] = Ktt [Wt ; Ut]^T (Wt and Ut are one 256-row image), then
+        // ---- stage 3: [Mlr | Bm] = Ktt [Wt ; Ut]^T (Wt and Ut are one 256-row image), then
         //      (P W)^T = Wt Ph^T and Ob = Ph Ut^T (M = 64) under a second commit, so that staging of
         //      Mlr and Bm overlaps the second pair of products.
         if (tid == 0) {
@@ -811,9 +816,9 @@ intra_kernel(const ChunkArgs a, const __grid_constant__ IntraMaps maps, const in
         }
         item = next;
     }
-    // a prefetch can only be in flight here after a failed wait; let it land
+    // tile loads can only be in flight here after a failed wait; let them land (bounded)
     if constexpr (IN_BF16) {
-        if (tid == 0 && raw_in_flight) mbar_wait(bar_raw, ph_raw, nullptr);
+        if (tid == 0 && raw_in_flight) mbar_wait(bar_raw, ph_raw, nullptr, a.wait_ns);
     }
     if (tid == 0) bulk_wait_all();  // last slot copy complete before the CTA retires
     __syncthreads();
@@ -1382,8 +1387,16 @@ bool make_tile_map(CUtensorMap* m, const void* base, int64_t rows, int64_t row_e
 
 bool g_attr_set = false;
 int g_num_sms = 0;
+// test hook (set_test_tile_drop): consumed by the next chunk-local launch
+bool g_drop_tile = false;
+unsigned long long g_drop_wait_ns = WAIT_LIMIT_NS;
 
 }  // namespace
+
+void set_test_tile_drop(unsigned long long wait_ns) {
+    g_drop_tile = wait_ns != 0;
+    g_drop_wait_ns = wait_ns != 0 ? wait_ns : WAIT_LIMIT_NS;
+}
 
 // The chain launch of one pass: SEG as in chain_kernel; gate fused as a 4-CTA cluster.
 template <int SEG>
@@ -1485,6 +1498,8 @@ cudaError_t chunk_fwd_launch(const void* q, const void* k, const void* v, const 
     a.segs = segs > 1 ? segs : 1;
     a.seg_ws = segs > 1 ? a.ws + (size_t)wc * per_wc : nullptr;
     a.trans_out = kcp_mode == KCP_TRANSITION ? trans_out : nullptr;
+    a.wait_ns = WAIT_LIMIT_NS;
+    a.drop_tile = 0;
 
     IntraMaps maps;
     memset(&maps, 0, sizeof(maps));
@@ -1521,10 +1536,17 @@ cudaError_t chunk_fwd_launch(const void* q, const void* k, const void* v, const 
             const int64_t n_items = (int64_t)N * wc * H;
             const unsigned grid = (unsigned)(n_items < g_num_sms ? n_items : g_num_sms);
             prof_begin(PROF_INTRA, stream);
+            if (g_drop_tile && in_bf16) {  // the test hook applies to one launch
+                a.drop_tile = 1;
+                a.wait_ns = g_drop_wait_ns;
+                g_drop_tile = false;
+            }
             if (in_bf16) intra_kernel<true><<<grid, INTRA_THREADS, INTRA_SMEM, stream>>>(a, maps, n_items);
             else intra_kernel<false><<<grid, INTRA_THREADS, INTRA_SMEM, stream>>>(a, maps, n_items);
             if ((err = cudaGetLastError()) != cudaSuccess) return err;
             prof_end(PROF_INTRA, stream);
+            a.drop_tile = 0;
+            a.wait_ns = WAIT_LIMIT_NS;
         }
         prof_begin(PROF_CHAIN, stream);
         if (o == nullptr && kcp_mode == KCP_NONE && a.segs == 1) {

@@ -28,6 +28,10 @@ cudaError_t chunk_fwd_launch(const void* q, const void* k, const void* v, const 
                              float scale, const void* gate, const float* norm_w, float eps, float* ckpt,
                              int64_t ckpt_tokens, int segs, int kcp_mode, float* trans_out, void* workspace,
                              size_t ws_bytes, cudaStream_t stream, int* n_passes, bool* gate_fused);
+// Test hook: the next chunk-local launch with bf16 inputs has CTA 0 skip one of
+// its first item's four tile loads and give up waiting after wait_ns (0 cancels).
+void set_test_tile_drop(unsigned long long wait_ns);
+
 // state_in = fold of maps 0 .. n_prev-1 of `trans` over init_state (zero when null)
 cudaError_t launch_kcp_compose(const float* trans, int n_prev, const float* init_state, float* state_in, int N, int H,
                                cudaStream_t stream);

@@ -17,6 +17,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+
 #include "../../include/kda.h"
 
 namespace {
@@ -24,19 +26,23 @@ namespace {
 static __device__ __align__(256) uint8_t g_kda_noalloc_scratch[KDA_NOALLOC_SCRATCH_BYTES];
 
 constexpr int kMaxDevices = 64;
-void* g_scratch_dev_ptr[kMaxDevices] = {};
+// Device address of the array per device.  Host threads may call concurrently:
+// each entry is an atomic, and two threads that look up the same device at once
+// both store the same address.  A cudaDeviceReset unloads the module, so a cached
+// address is stale afterwards (documented in kda.h).
+std::atomic<void*> g_scratch_dev_ptr[kMaxDevices];
 
 // Device address of the scratch array on the current device (looked up once
-// per device).  Returns nullptr on failure.
+// per device, with that device current).  Returns nullptr on failure.
 void* scratch_on_current_device() {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
-    if (g_scratch_dev_ptr[dev] == nullptr) {
-        void* p = nullptr;
+    void* p = g_scratch_dev_ptr[dev].load(std::memory_order_acquire);
+    if (p == nullptr) {
         if (cudaGetSymbolAddress(&p, g_kda_noalloc_scratch) != cudaSuccess) return nullptr;
-        g_scratch_dev_ptr[dev] = p;
+        g_scratch_dev_ptr[dev].store(p, std::memory_order_release);
     }
-    return g_scratch_dev_ptr[dev];
+    return p;
 }
 
 }  // namespace
@@ -60,4 +66,13 @@ extern "C" kda_status kda_chunk_fwd_noalloc(const void* q, const void* k, const 
     return kda_chunk_fwd(q, k, v, log_alpha, beta, init_state, o, final_state, B, T, H, dk, dv, cu_seqlens, n_seqs,
                          max_seqlen, in_dtype, out_dtype, scale, gate, norm_weight, eps, scratch,
                          (size_t)KDA_NOALLOC_SCRATCH_BYTES, stream);
+}
+
+// The device status word of the last kda_chunk_fwd_noalloc call on the current
+// device sits at the start of the static array (the layout every prefill
+// workspace has); kda_query_status reads and clears it.
+extern "C" kda_status kda_chunk_fwd_noalloc_query_status(void* stream) {
+    void* scratch = scratch_on_current_device();
+    if (scratch == nullptr) return KDA_ERR_CUDA;
+    return kda_query_status(scratch, stream);
 }

@@ -69,14 +69,15 @@ KDA_DEV bool mbar_try_wait(uint64_t* bar, uint32_t parity, uint32_t suspend_ns =
 }
 
 // Waits for the phase with the given parity to complete.  Gives up after about
-// WAIT_LIMIT_NS, ORs DEV_ERR_TIMEOUT into *status (if non-null) and returns
-// false; never spins forever.
-KDA_DEV bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t* status) {
+// limit_ns (WAIT_LIMIT_NS by default), ORs DEV_ERR_TIMEOUT into *status (if
+// non-null) and returns false; never spins forever.
+KDA_DEV bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t* status,
+                       unsigned long long limit_ns = WAIT_LIMIT_NS) {
     if (mbar_try_wait(bar, parity)) return true;
     const unsigned long long t0 = globaltimer_ns();
     while (true) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if (globaltimer_ns() - t0 > WAIT_LIMIT_NS) {
+        if (mbar_try_wait(bar, parity, 100000u)) return true;
+        if (globaltimer_ns() - t0 > limit_ns) {
             if (status) atomicOr(status, DEV_ERR_TIMEOUT);
             return false;
         }

@@ -54,3 +54,45 @@ def make_prefill(seed, lengths, H, bf16=True, gate=False, init=False, la_const=N
     s0 = synth.states(seed, len(lengths), H, D, D) if init else None
     cu = synth.cu_from_lengths(lengths)
     return dict(q=tb.q, k=tb.k, v=tb.v, log_alpha=la, beta=beta, g=tb.g, s0=s0, cu=cu, T=T)
+
+
+# Achieved errors of every parity comparison, printed at the end of the
+# session (tests/conftest.py) so the margin to the tolerance is on record.
+MARGINS = []
+
+
+def assert_rel_l2(x, ref, what: str, tol: float = REL_L2_TOL) -> float:
+    """Relative L2 error of x against ref, recorded with the running test's id,
+    and asserted to be within tol."""
+    import os
+    e = rel_l2(x, ref)
+    test = os.environ.get("PYTEST_CURRENT_TEST", "?").split(" ")[0]
+    MARGINS.append((test, what, e, tol))
+    assert e <= tol, f"{what}: rel-L2 {e:.3e} above {tol:g}"
+    return e
+
+
+# Canary guard regions: an output buffer is allocated with GUARD extra elements
+# on each side, all set to a fixed NaN bit pattern; after the call the guards
+# must still hold it (a cheap stand-in for an out-of-bounds write checker).
+GUARD = 1024
+_CANARY = {"float32": (0x7FC0DEAD, "int32"), "bfloat16": (0x7FDE, "int16")}
+
+
+def guarded_empty(shape, dtype):
+    """(tensor of `shape` on the GPU, check()) where check() asserts that
+    nothing was written into the guard regions around it."""
+    import torch
+    n = int(np.prod(shape))
+    pat, ity = _CANARY[str(dtype).split(".")[-1]]
+    ity = getattr(torch, ity)
+    buf = torch.empty(n + 2 * GUARD, dtype=dtype, device="cuda")
+    buf.view(ity).fill_(pat)
+    inner = buf[GUARD:GUARD + n].view(shape)
+
+    def check(what="output"):
+        torch.cuda.synchronize()
+        for side, part in (("before", buf[:GUARD]), ("after", buf[GUARD + n:])):
+            bad = (part.view(ity) != pat).nonzero()
+            assert bad.numel() == 0, f"{what}: {bad.numel()} guard elements {side} the buffer were overwritten"
+    return inner, check

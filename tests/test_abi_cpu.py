@@ -31,7 +31,8 @@ def test_header_declares_the_entry_points():
               "kda_gate_norm", "kda_chunk_fwd_segmented_workspace_size",
               "kda_chunk_fwd_workspace_size", "kda_kcp_workspace_size", "kda_kcp_transition", "kda_kcp_compose",
               "kda_kcp_finish", "kda_chunk_bwd", "kda_chunk_bwd_workspace_size",
-              "kda_query_status", "kda_status_string", "kda_version"):
+              "kda_query_status", "kda_status_string", "kda_version", "kda_chunk_fwd_noalloc",
+              "kda_chunk_fwd_noalloc_query_status", "kda_test_drop_tile_load"):
         assert s in syms
 
 
@@ -225,3 +226,32 @@ def test_binding_refuses_cpu_tensors():
     x = torch.zeros(1, 4, 1, 128)
     with pytest.raises(ValueError):
         kda.chunk_fwd(x, x, x, x, torch.zeros(1, 4, 1))
+
+
+def test_failure_hooks_host_side(lib):
+    """The test hook that makes one tile load go missing takes a wait limit in
+    [1 us, 1 s] (0 cancels a pending drop); other values are rejected on the
+    host.  Setting and cancelling it touch no device."""
+    assert lib.kda_test_drop_tile_load(5) == -1
+    assert lib.kda_test_drop_tile_load(2_000_000_000) == -1
+    assert lib.kda_test_drop_tile_load(2_000_000) == 0
+    assert lib.kda_test_drop_tile_load(0) == 0  # cancelled again
+
+
+def test_build_tracks_every_header(tmp_path):
+    """An edit to any header the CUDA sources include (the slot layout among
+    them) makes the library out of date, so it is rebuilt before use."""
+    hs = [os.path.basename(h) for h in kbuild.headers()]
+    for name in ("kda_slots.h", "kda_launch.h", "kda_profile.h", "kda_sm100.cuh", "kda.h"):
+        assert name in hs, name
+    kbuild.build()
+    assert kbuild.up_to_date()
+    slots = os.path.join(kbuild.CSRC, "kda_slots.h")
+    st = os.stat(slots)
+    lib_t = os.path.getmtime(kbuild.LIB)
+    try:
+        os.utime(slots, (st.st_atime, lib_t + 10))
+        assert not kbuild.up_to_date()
+    finally:
+        os.utime(slots, (st.st_atime, st.st_mtime))
+    assert kbuild.up_to_date()

@@ -9,6 +9,7 @@ reduced (max over ranks).  These tests run two gloo ranks on the host:
 """
 import os
 import socket
+import sys
 
 import numpy as np
 import pytest
@@ -205,3 +206,31 @@ def test_kcp_three_ranks_match_the_whole_sequence():
     np.testing.assert_allclose(results[-1][3], fs_ref, rtol=0, atol=1e-10)
     # a middle rank's state is the state after the first two segments, not the final one
     assert np.abs(results[1][3] - fs_ref).max() > 1e-3
+
+
+def test_bench_launches_its_own_ranks():
+    """`python bench.py --gpus 2` without a launcher starts two ranks itself
+    (torch.distributed.run on 127.0.0.1); in dry mode they join a gloo group and
+    rank 0 reports that both formed and took part in the max-over-ranks timing."""
+    import json
+    import subprocess
+    env = {k: v for k, v in os.environ.items() if k not in ("WORLD_SIZE", "RANK", "LOCAL_RANK", "MASTER_ADDR",
+                                                           "MASTER_PORT")}
+    env["NCCL_DEBUG"] = "WARN"
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--gpus", "2", "--dry-run", "--steps", "3",
+                        "--warmup", "3"], env=env, capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [json.loads(ln) for ln in r.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1, r.stdout
+    line = lines[0]
+    assert line["n_gpus"] == 2 and line["ranks_reported"] == 2
+    assert line["max_over_ranks"] == 2.0          # the slower (larger) of the two ranks' values
+    assert line["value"] == 2 * 1.0 / 2.0e-3      # whole-job rate over the slowest rank
+
+
+def test_bench_refuses_a_world_size_that_contradicts_gpus():
+    import subprocess
+    env = dict(os.environ, WORLD_SIZE="3", RANK="0", LOCAL_RANK="0")
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--gpus", "2", "--dry-run"], env=env,
+                       capture_output=True, text=True, timeout=120)
+    assert r.returncode != 0 and "WORLD_SIZE" in r.stderr

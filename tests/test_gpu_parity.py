@@ -4,7 +4,7 @@ import numpy as np
 import pytest
 
 import oracle
-from kda_testutil import REL_L2_TOL, D, dev, host, make_prefill, rel_l2
+from kda_testutil import REL_L2_TOL, D, assert_rel_l2, dev, guarded_empty, host, make_prefill, rel_l2
 from linear_attention_recurrence_06_b200 import synth
 
 pytestmark = pytest.mark.gpu
@@ -15,7 +15,7 @@ def _torch():
     return torch
 
 
-def run_prefill(inp, H, bf16, *, varlen, gate=False, out_f32=False):
+def run_prefill(inp, H, bf16, *, varlen, gate=False, out_f32=False, scale=1.0):
     torch = _torch()
     import linear_attention_recurrence_06_b200 as kda
     dt = torch.bfloat16 if bf16 else torch.float32
@@ -31,22 +31,27 @@ def run_prefill(inp, H, bf16, *, varlen, gate=False, out_f32=False):
     if varlen:
         kw = dict(cu_seqlens=torch.from_numpy(inp["cu"].astype(np.int32)).cuda(),
                   max_seqlen=int(np.diff(inp["cu"]).max()))
-    o, fs = kda.chunk_fwd(q, k, v, la, b, s0, gate=g, out_dtype=torch.float32 if out_f32 else None, **kw)
-    torch.cuda.synchronize()
+    # outputs inside canary guard regions (checked after the call)
+    N = len(inp["cu"]) - 1 if varlen else 1
+    o, o_check = guarded_empty((1, T, H, D), torch.float32 if out_f32 else dt)
+    fs, fs_check = guarded_empty((N, H, D, D), torch.float32)
+    kda.chunk_fwd(q, k, v, la, b, s0, gate=g, scale=scale, out=o, final_state=fs, **kw)
+    o_check("o")
+    fs_check("final state")
     return host(o).reshape(T, H, D), host(fs)
 
 
-def oracle_prefill(inp, gate=False):
-    o, fs = oracle.kda_recurrent(inp["q"], inp["k"], inp["v"], inp["log_alpha"], inp["beta"], inp["s0"], inp["cu"])
+def oracle_prefill(inp, gate=False, scale=1.0):
+    o, fs = oracle.kda_recurrent(inp["q"], inp["k"], inp["v"], inp["log_alpha"], inp["beta"], inp["s0"], inp["cu"],
+                                 scale=scale)
     if gate:
         o = oracle.gate_norm(o, inp["g"], None, 1e-6)
     return o, fs
 
 
-def check(o, fs, ro, rfs):
-    eo, ef = rel_l2(o, ro), rel_l2(fs, rfs)
-    assert eo <= REL_L2_TOL, f"output rel-L2 {eo:.3e}"
-    assert ef <= REL_L2_TOL, f"final-state rel-L2 {ef:.3e}"
+def check(o, fs, ro, rfs, what=""):
+    eo = assert_rel_l2(o, ro, f"{what} output".strip())
+    ef = assert_rel_l2(fs, rfs, f"{what} final state".strip())
     return eo, ef
 
 
@@ -79,8 +84,40 @@ def test_prefill_varlen_edge_lengths():
     for n in range(len(lens)):
         sl = slice(inp["cu"][n], inp["cu"][n + 1])
         if lens[n]:
-            assert rel_l2(o[sl], ro[sl]) <= REL_L2_TOL
-        assert rel_l2(fs[n], rfs[n]) <= REL_L2_TOL
+            assert_rel_l2(o[sl], ro[sl], f"seq {n} o")
+        assert_rel_l2(fs[n], rfs[n], f"seq {n} final state")
+
+
+# Output scales other than 1 (the usual dk^-1/2 among them).  The scale enters
+# the chunk's P and Q' terms and the decode output; the gate's RMSNorm is
+# invariant to it, so the ungated cases are the ones that see a misplaced factor.
+SCALES = (0.125, 128 ** -0.5)
+
+
+@pytest.mark.parametrize("scale", SCALES)
+@pytest.mark.parametrize("bf16,gate,varlen", [
+    (True, False, False), (True, True, False), (False, False, False), (False, True, False),
+    (True, False, True), (True, True, True), (False, False, True),
+])
+def test_prefill_scale(scale, bf16, gate, varlen):
+    """Prefill with scale != 1 against the oracle with the same scale: bf16
+    and fp32 inputs, with and without the gate, one sequence or packed
+    sequences (an empty and ragged ones) with initial states."""
+    lens = [200, 64, 0, 77] if varlen else [300]
+    H = 3
+    inp = make_prefill(17 + int(1000 * scale), lens, H, bf16=bf16, gate=gate, init=True)
+    o, fs = run_prefill(inp, H, bf16, varlen=varlen, gate=gate, out_f32=True, scale=scale)
+    ro, rfs = oracle_prefill(inp, gate=gate, scale=scale)
+    check(o, fs, ro, rfs, f"scale={scale:.4f}")
+    if not gate:
+        # o is linear in the scale: the unscaled oracle times the scale is the same answer
+        ro1, _ = oracle_prefill(inp, gate=False, scale=1.0)
+        assert_rel_l2(o, scale * ro1, "o against scale x unscaled oracle")
+    if varlen:
+        for n, L in enumerate(lens):
+            sl = slice(inp["cu"][n], inp["cu"][n + 1])
+            if L:
+                assert_rel_l2(o[sl], ro[sl], f"seq {n} output")
 
 
 @pytest.mark.parametrize("case", ["la_floor", "la_zero", "beta_zero", "beta_one", "la_below_floor"])
@@ -146,7 +183,7 @@ def test_prefill_gate_varlen_weights_multi_pass(bf16):
         for n in range(len(lens)):
             sl = slice(inp["cu"][n], inp["cu"][n + 1])
             if lens[n]:
-                assert rel_l2(yh[sl], ry[sl]) <= REL_L2_TOL
+                assert_rel_l2(yh[sl], ry[sl], f"multi_pass={multi} seq {n} y")
 
 
 @pytest.mark.parametrize("multi_pass", [False, True])
@@ -167,10 +204,12 @@ def test_prefill_state_checkpoints(multi_pass):
     if multi_pass:
         lo, _ = kda.workspace_size(T, H, len(lens), max(lens))
         kw["workspace"] = torch.empty(lo, dtype=torch.uint8, device="cuda")
+    ck_buf, ck_check = guarded_empty((len(lens), max(lens) // every, H, D, D), torch.float32)
+    ck_buf.zero_()
     o, fs, ck = kda.chunk_fwd(q, k, v, la, b, dev(inp["s0"], torch.float32),
                               cu_seqlens=torch.from_numpy(cu.astype(np.int32)).cuda(), max_seqlen=max(lens),
-                              checkpoints=True, ckpt_tokens=every, **kw)
-    torch.cuda.synchronize()
+                              checkpoints=ck_buf, ckpt_tokens=every, **kw)
+    ck_check("checkpoints")
     ck = host(ck)
     assert ck.shape == (len(lens), max(lens) // every, H, D, D)
     for n, L in enumerate(lens):
@@ -182,7 +221,7 @@ def test_prefill_state_checkpoints(multi_pass):
             sl = slice(cu[n], cu[n] + end)
             _, ref = oracle.kda_recurrent(inp["q"][sl], inp["k"][sl], inp["v"][sl], inp["log_alpha"][sl],
                                           inp["beta"][sl], inp["s0"][n:n + 1])
-            assert rel_l2(ck[n, j], ref[0]) <= REL_L2_TOL, f"seq {n} checkpoint {j}"
+            assert_rel_l2(ck[n, j], ref[0], f"seq {n} checkpoint {j}")
     # the last whole checkpoint of a sequence ending on a boundary is its final state
     np.testing.assert_array_equal(ck[4, 0], host(fs)[4])
 
@@ -221,8 +260,8 @@ def test_prefill_segment_parallel(segments, gate, lens, memory):
     for n, L in enumerate(lens):
         sl = slice(inp["cu"][n], inp["cu"][n + 1])
         if L:
-            assert rel_l2(oh[sl], ro[sl]) <= REL_L2_TOL, f"seq {n}"
-        assert rel_l2(fh[n], rfs[n]) <= REL_L2_TOL, f"seq {n} state"
+            assert_rel_l2(oh[sl], ro[sl], f"seq {n}")
+        assert_rel_l2(fh[n], rfs[n], f"seq {n} state")
 
 
 # --------------------------------------- context parallelism across devices
@@ -295,7 +334,7 @@ def test_kcp_emulated_ranks(R, gate, lens, memory, ragged):
     for n, L in enumerate(lens):
         sl = slice(inp["cu"][n], inp["cu"][n + 1])
         if L:
-            assert rel_l2(o_all[sl], ro[sl]) <= REL_L2_TOL, f"seq {n}"
+            assert_rel_l2(o_all[sl], ro[sl], f"seq {n}")
     # rank R//2's state: the oracle's state after pieces 0 .. R//2 of each sequence
     m = R // 2
     for n, L in enumerate(lens):
@@ -303,7 +342,7 @@ def test_kcp_emulated_ranks(R, gate, lens, memory, ragged):
         sl = slice(int(inp["cu"][n]), end)
         _, ref = oracle.kda_recurrent(inp["q"][sl], inp["k"][sl], inp["v"][sl], inp["log_alpha"][sl],
                                       inp["beta"][sl], inp["s0"][n:n + 1])
-        assert rel_l2(ranks[m]["fs"][n], ref[0]) <= REL_L2_TOL, f"seq {n} state after rank {m}"
+        assert_rel_l2(ranks[m]["fs"][n], ref[0], f"seq {n} state after rank {m}")
 
 
 def test_kcp_transition_is_the_oracle_segment_map():
@@ -322,8 +361,8 @@ def test_kcp_transition_is_the_oracle_segment_map():
     t = host(trans)
     for h in range(H):
         M, B = oracle.segment_transition(inp["k"][:, h], inp["v"][:, h], inp["log_alpha"][:, h], inp["beta"][:, h])
-        assert rel_l2(t[0, 0, h], M) <= REL_L2_TOL, f"M head {h}"
-        assert rel_l2(t[1, 0, h], B) <= REL_L2_TOL, f"B head {h}"
+        assert_rel_l2(t[0, 0, h], M, f"M head {h}")
+        assert_rel_l2(t[1, 0, h], B, f"B head {h}")
         assert np.abs(M).max() > 0.1  # the segment map carries the state
 
 
@@ -382,15 +421,16 @@ def test_prefill_in_place_state():
     kda.chunk_fwd(q, k, v, la, b, s, final_state=s)
     torch.cuda.synchronize()
     _, rfs = oracle_prefill(inp)
-    assert rel_l2(host(s), rfs) <= REL_L2_TOL
+    assert_rel_l2(host(s), rfs, "in-place final state")
 
 
 # ------------------------------------------------------------------ decode
 
 
+@pytest.mark.parametrize("scale", [1.0, 128 ** -0.5])
 @pytest.mark.parametrize("bf16", [True, False])
 @pytest.mark.parametrize("gate", [False, True])
-def test_decode_steps(bf16, gate):
+def test_decode_steps(bf16, gate, scale):
     torch = _torch()
     import linear_attention_recurrence_06_b200 as kda
     Bd, H, steps = 6, 3, 12
@@ -403,17 +443,19 @@ def test_decode_steps(bf16, gate):
         q, k, v, la = (dev(getattr(tb, x), dt) for x in ("q", "k", "v", "log_alpha"))
         b = dev(tb.beta, dt)
         g = dev(tb.g, dt) if gate else None
-        o = kda.decode_step(s_dev, q, k, v, la, b, gate=g, out_dtype=torch.float32)
-        ro, s_ref = oracle.decode_steps(s_ref, tb.q, tb.k, tb.v, tb.log_alpha, tb.beta)
+        o = kda.decode_step(s_dev, q, k, v, la, b, gate=g, out_dtype=torch.float32, scale=scale)
+        ro, s_ref = oracle.decode_steps(s_ref, tb.q, tb.k, tb.v, tb.log_alpha, tb.beta, scale=scale)
         if gate:
             ro = oracle.gate_norm(ro, tb.g, None, 1e-6)
         torch.cuda.synchronize()
-        assert rel_l2(host(o), ro) <= REL_L2_TOL
-    assert rel_l2(host(s_dev), s_ref) <= REL_L2_TOL
+        assert_rel_l2(host(o), ro, f"step {step} o")
+    assert_rel_l2(host(s_dev), s_ref, "state after the steps")
 
 
-@pytest.mark.parametrize("bf16,gate,n", [(True, False, 1), (True, False, 4), (True, True, 8), (False, False, 3)])
-def test_decode_multi_step_with_step_states(bf16, gate, n):
+@pytest.mark.parametrize("bf16,gate,n,scale", [(True, False, 1, 1.0), (True, False, 4, 1.0), (True, True, 8, 1.0),
+                                               (False, False, 3, 1.0), (True, False, 4, 128 ** -0.5),
+                                               (False, True, 3, 0.125)])
+def test_decode_multi_step_with_step_states(bf16, gate, n, scale):
     """n consecutive steps in one call == n single steps of the oracle: every
     step's output, every step's state (for rollback) and the carried state."""
     torch = _torch()
@@ -428,17 +470,20 @@ def test_decode_multi_step_with_step_states(bf16, gate, n):
     b = dev(stack("beta"), dt)
     g = dev(stack("g"), dt) if gate else None
     w = np.random.default_rng(7).uniform(0.5, 1.5, D).astype(np.float32) if gate else None
+    o_buf, o_check = guarded_empty((n, Bd, H, D), torch.float32)
+    st_buf, st_check = guarded_empty((n, Bd, H, D, D), torch.float32)
     o, states = kda.decode_steps(s_dev, q, k, v, la, b, gate=g, norm_weight=dev(w, torch.float32) if gate else None,
-                                 out_dtype=torch.float32, step_states=True)
-    torch.cuda.synchronize()
+                                 out=o_buf, step_states=st_buf, scale=scale)
+    o_check("o")
+    st_check("step states")
     ref = s0.astype(np.float64)
     for step, tb in enumerate(toks):
-        ro, ref = oracle.decode_steps(ref, tb.q, tb.k, tb.v, tb.log_alpha, tb.beta)
+        ro, ref = oracle.decode_steps(ref, tb.q, tb.k, tb.v, tb.log_alpha, tb.beta, scale=scale)
         if gate:
             ro = oracle.gate_norm(ro, tb.g, w, 1e-6)
-        assert rel_l2(host(o[step]), ro) <= REL_L2_TOL, f"step {step} output"
-        assert rel_l2(host(states[step]), ref) <= REL_L2_TOL, f"step {step} state"
-    assert rel_l2(host(s_dev), ref) <= REL_L2_TOL
+        assert_rel_l2(host(o[step]), ro, f"step {step} output")
+        assert_rel_l2(host(states[step]), ref, f"step {step} state")
+    assert_rel_l2(host(s_dev), ref, "carried state")
     np.testing.assert_array_equal(host(s_dev), host(states[n - 1]))  # the carried state is the last step's
 
 
@@ -477,4 +522,4 @@ def test_gate_norm(bf16, rows):
     y = kda.gate_norm(dev(o, dt), dev(g, dt), dev(w, torch.float32), out_dtype=torch.float32)
     ref = oracle.gate_norm(o.astype(np.float64), g, w, 1e-6)
     torch.cuda.synchronize()
-    assert rel_l2(host(y), ref) <= 1e-5 if not bf16 else rel_l2(host(y), ref) <= REL_L2_TOL
+    assert_rel_l2(host(y), ref, "y", tol=1e-5 if not bf16 else REL_L2_TOL)
