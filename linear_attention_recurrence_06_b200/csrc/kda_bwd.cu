@@ -11,9 +11,9 @@
 //      dS = dL/d(state at the end of chunk c):
 //          dS_end[c] = dS,    dS <- Diag(Gamma_C) dS - M_lr^T dS + Q'^T dO_c
 //      starting from dL/dS_final and ending with dL/dS_0;
-//   3. bwd_intra_kernel takes one (chunk, head) at a time, with the chunk-start
+//   3. bwd_tc_kernel takes one (chunk, head) at a time, with the chunk-start
 //      state S0 and dS_C = dS_end[c], and forms dq, dk, dv, dbeta, dlog_alpha of
-//      the chunk's tokens.
+//      the chunk's tokens; its products run on the tensor cores.
 // Per chunk (L <= 64 tokens; g = in-chunk cumulative sum of the clamped
 // log-decays, Gam = e^g, g_C = g of the last token, qb = scale q,
 // K^C = K o e^{g_C - g}):
@@ -27,14 +27,15 @@
 //   contractions (-> q, k, g); dlog_alpha = reverse cumulative sum of dg over the
 //   chunk, zero where log_alpha < -5 (the clamp passes the gradient where
 //   log_alpha >= -5).
-// The A / P terms use per-16-token-block reference points r (the block's first
-// token): e^{g_t - g_s} = e^{g_t - g_r} e^{g_r - g_s}, so each exponential is
-// formed once per (token, channel, block) and never overflows.
-// Everything is fp32 on the CUDA cores.
+// The A / P terms use the forward's per-16-token-tile exponent references G_b (g
+// just before tile b): e^{g_t - g_s} = e^{g_t - G_b} e^{G_b - g_s}, so no operand
+// overflows.  Products run on the tensor cores with bf16 operands and fp32
+// accumulators; M^-1, the exponentials and the gradient assembly are fp32.
 #include "kda_launch.h"
 #include "kda_profile.h"
 #include "kda_slots.h"
 #include "kda_sm100.cuh"
+#include "kda_tri.cuh"
 
 namespace kda {
 
@@ -205,62 +206,7 @@ __global__ void __launch_bounds__(CB_THREADS, 1) chain_bwd_kernel(const BwdArgs 
     }
 }
 
-// -------------------------------------------------------- chunk-local part
-constexpr int BI_THREADS = 512;
-constexpr int LP = 65;    // padded row of the 64 x 64 matrices
-constexpr int FP = 132;   // padded row of the factor buffer
-constexpr int QP = 33;    // padded row of the 64 x 32 quarter buffers
-constexpr int NQ = 32;    // value columns per quarter
-constexpr uint32_t BI_G = 0;                                  // g [64][128]
-constexpr uint32_t BI_A = BI_G + CH * DK * 4;                  // A [64][65]
-constexpr uint32_t BI_P = BI_A + CH * LP * 4;                  // P
-constexpr uint32_t BI_MI = BI_P + CH * LP * 4;                 // M^-1
-constexpr uint32_t BI_DP = BI_MI + CH * LP * 4;                // dP (accumulated)
-constexpr uint32_t BI_DM = BI_DP + CH * LP * 4;                // dM (accumulated), then dA
-constexpr uint32_t BI_F = BI_DM + CH * LP * 4;                 // factors [128][132]
-constexpr uint32_t BI_R = BI_F + 128 * FP * 4;                 // R quarter [64][33]
-constexpr uint32_t BI_U = BI_R + CH * QP * 4;                  // U quarter
-constexpr uint32_t BI_DU = BI_U + CH * QP * 4;                 // dU quarter, then Y
-constexpr uint32_t BI_DO = BI_DU + CH * QP * 4;                // dO quarter
-constexpr uint32_t BI_BETA = BI_DO + CH * QP * 4;              // beta [64]
-constexpr uint32_t BI_DB = BI_BETA + 256;                      // rowsum(Y o R) [64]
-constexpr uint32_t BI_GC = BI_DB + 256;                        // g_C [128]
-constexpr uint32_t BI_DGC = BI_GC + 512;                       // dL/dg_C [128]
-constexpr uint32_t BI_SMEM = BI_DGC + 512;
-
-// Factor rows of block bt (reference token r = 16 bt) in the factor buffer:
-// rows [0, 16 bt + 16): Kout_s = k_s o e^{g_r - g_s};  rows [64, 80): Kin_t = k_t o
-// e^{g_t - g_r};  rows [80, 96): Qin_t = qb_t o e^{g_t - g_r}  (t in the block).
-KDA_DEV void build_factors(const BwdArgs& a, float* sF, const float* sG, int bt, int64_t t0, int L, int h,
-                           int tid) {
-    const int r = 16 * bt, ns = 16 * bt + 16;
-    const int n_el = (ns + 32) * DK;  // a multiple of 4 * BI_THREADS
-    for (int e0 = tid; e0 < n_el; e0 += 4 * BI_THREADS) {
-        float x[4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {  // loads first, all four in flight
-            const int e = e0 + u * BI_THREADS, row = e >> 7, i = e & (DK - 1);
-            const int t = row < ns ? row : r + ((row - ns) & 15);
-            x[u] = 0.f;
-            if (t < L) {
-                const size_t idx = ((size_t)(t0 + t) * a.H + h) * DK + i;
-                x[u] = (row < ns + 16) ? ld_in(a.k, idx, a.in_bf16) : a.scale * ld_in(a.q, idx, a.in_bf16);
-            }
-        }
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            const int e = e0 + u * BI_THREADS, row = e >> 7, i = e & (DK - 1);
-            const float gr = sG[r * DK + i];
-            if (row < ns) {
-                sF[row * FP + i] = x[u] * __expf(gr - sG[row * DK + i]);
-            } else {
-                const int tt = row - ns;  // 0..31: Kin rows, then Qin rows
-                const int t = r + (tt & 15);
-                sF[(64 + tt) * FP + i] = x[u] * __expf(sG[t * DK + i] - gr);
-            }
-        }
-    }
-}
+constexpr int BT_THREADS = 512;  // threads of the chunk-local kernel
 
 // Pulls an item's token rows (q, k, v, log_alpha, dO: 64 rows each), its
 // chunk-start state and its end-of-chunk state gradient into L2 ahead of use.
@@ -278,7 +224,7 @@ KDA_DEV void prefetch_item(const BwdArgs& a, int64_t item, int64_t n_items, int 
     const size_t esz = a.in_bf16 ? 2 : 4, row = DK * esz;  // bytes of one head row
     const int lines_row = (int)(row / 128);
     const void* tens[5] = {a.q, a.k, a.v, a.log_alpha, a.d_o};
-    for (int e = tid; e < 5 * CH * lines_row; e += BI_THREADS) {
+    for (int e = tid; e < 5 * CH * lines_row; e += BT_THREADS) {
         const int tsr = e / (CH * lines_row), rem = e % (CH * lines_row), t = rem / lines_row, ln = rem % lines_row;
         if (t >= L) continue;
         const char* p = reinterpret_cast<const char*>(tens[tsr]) + ((size_t)(t0 + t) * H + h) * row + ln * 128;
@@ -287,420 +233,841 @@ KDA_DEV void prefetch_item(const BwdArgs& a, int64_t item, int64_t n_items, int 
     const float* S0 = c == 0 ? (a.init_state ? a.init_state + ((size_t)n * H + h) * STATE : nullptr)
                              : a.ckpt + (((size_t)n * a.n_ckpt + (c - 1)) * H + h) * STATE;
     const float* dSC = a.ds_end + (((size_t)n * a.wc + c) * H + h) * STATE;
-    for (int e = tid; e < 2 * STATE * 4 / 128; e += BI_THREADS) {
+    for (int e = tid; e < 2 * STATE * 4 / 128; e += BT_THREADS) {
         const int which = e / (STATE * 4 / 128), ln = e % (STATE * 4 / 128);
         const float* base = which ? dSC : S0;
         if (base) asm volatile("prefetch.global.L2 [%0];" ::"l"(reinterpret_cast<const char*>(base) + (size_t)ln * 128));
     }
 }
 
-__global__ void __launch_bounds__(BI_THREADS, 1) bwd_intra_kernel(const BwdArgs a, int64_t n_items) {
-    extern __shared__ __align__(128) uint8_t sm[];
-    float* sG = reinterpret_cast<float*>(sm + BI_G);
-    float* sA = reinterpret_cast<float*>(sm + BI_A);
-    float* sP = reinterpret_cast<float*>(sm + BI_P);
-    float* sMi = reinterpret_cast<float*>(sm + BI_MI);
-    float* sdP = reinterpret_cast<float*>(sm + BI_DP);
-    float* sdM = reinterpret_cast<float*>(sm + BI_DM);
-    float* sF = reinterpret_cast<float*>(sm + BI_F);
-    float* sR = reinterpret_cast<float*>(sm + BI_R);
-    float* sU = reinterpret_cast<float*>(sm + BI_U);
-    float* sDU = reinterpret_cast<float*>(sm + BI_DU);
-    float* sDO = reinterpret_cast<float*>(sm + BI_DO);
-    float* sBeta = reinterpret_cast<float*>(sm + BI_BETA);
-    float* sDb = reinterpret_cast<float*>(sm + BI_DB);
-    float* sGC = reinterpret_cast<float*>(sm + BI_GC);
-    float* sDgC = reinterpret_cast<float*>(sm + BI_DGC);
-    const int tid = threadIdx.x, H = a.H;
-    // register-owned elements: tokens 4 tg .. 4 tg + 3, key channels ig + 32 y (y = 0..3;
-    // interleaved so that a warp's 32 lanes touch 32 consecutive channels)
-    const int tg = tid >> 5, ig = tid & 31;
+// ------------------------------------------------ chunk-local part (tensor cores)
+// One item = (chunk, head); 512 threads, thread (c = tid % 128, q4 = tid / 128) owns
+// channel c (key channel i, or value column j) and the 16-token tile q4.  Every product
+// of the item runs on the tensor cores (tcgen05.mma kind::f16: bf16 operand images in
+// shared memory, fp32 accumulators in TMEM); the SIMT phases between them build the
+// operand images, invert M in fp32 and assemble the gradients.
+//
+// Operand images: row-major with 16-byte pieces along the columns, no swizzle:
+// element (r, c) of an image with nc columns at il_off(r, c, nc).  The same image is a
+// K-major operand (columns = K) or an MN-major one (columns = M or N), which is how each
+// image below serves two products.  Transposed products keep a channel (i or j) in the
+// 128 TMEM lanes, so thread (c, q4) reads its own channel's row.
+//   I1 KQr  [i][t']  t' < 64: k_t e^{g_t - G_b},  t' >= 64: scale q_t e^{g_t - G_b}  (b = tile of t)
+//   I2 KC   [i][sv]  the 160 column versions of the keys (forward stage 1): sv < 64:
+//                    k_s e^{G_b(s) - g_s}; Kb1/Kb2/Kb3: tiles before b w.r.t. G_b
+//   I3 KG   [i][t]   k_t e^{g_t};   I4 KCe [i][t]  k_t e^{g_C - g_t}
+//   I5 S0   [i][j];  I6 dSC [i][j]  (chunk-start state, gradient at the chunk end)
+//   I7 [Y|dO] [j][t'] t' < 64: Y_t, t' >= 64: dO_t
+//   I8 P    [t][s];  I9 Minv [t][s];  I10 beta R^T [j][s];  I11 dU^T [j][s];  I12 U^T [j][t]
+//   I13 [A'|P'] [t'][sv]  dA (rows < 64) and dP (rows >= 64) placed at the column version
+//                    their row's tile uses, zero elsewhere
+// Products (M x N x K, D in TMEM with lane = M row):
+//   stage 1  A/P raw = I1^T-rows x I2            128 x 160 x 128   (as the forward)
+//            X1^T = S0^T (K o Gam)^T              128 x  64 x 128   (R = V - (K o Gam) S0)
+//            dU^T = dSC^T K^C^T                   128 x  64 x 128
+//   stage 2  U^T = (beta R)^T Minv^T              128 x  64 x  64
+//            dU^T += dO^T P                       128 x  64 x  64
+//   stage 3  Y^T = dU^T Minv                      128 x  64 x  64
+//            aKC = dSC U^T  [i][t]                128 x  64 x 128
+//   stage 4  [-dM ; dP] = [Y ; dO] U^T            128 x  64 x 128
+//            [S0 Y^T | S0 dO^T]  [i][t']          128 x 128 x 128
+//   stage 5  [RowA | RowP]^T = KC^T-cols x [A';P'] 128 x 128 x 160
+//            Col^T = KQr x [A';P']                128 x 160 x 128
+// shared memory (offsets from a 1024-aligned base)
+constexpr uint32_t BT_I5 = 0, BT_I6 = 32768, BT_I7 = 65536;
+constexpr uint32_t BT_I1 = 98304, BT_I2 = 131072;                       // stage-1 copies
+constexpr uint32_t BT_N = 98304, BT_X = BT_N + 17408, BT_TMP = BT_X + 17408;  // inverse (fp32)
+constexpr uint32_t BT_I8 = BT_TMP + 8192, BT_I9 = BT_I8 + 8192, BT_I10 = BT_I9 + 8192, BT_I11 = BT_I10;
+constexpr uint32_t BT_I12 = 98304;
+constexpr uint32_t BT_I3 = BT_I10 + 16384, BT_I4 = BT_I3 + 16384;
+constexpr uint32_t BT_I13 = 0, BT_I1B = 40960, BT_I2B = 73728;          // stage-5 images
+constexpr uint32_t BT_I2L = 114688, BT_I1L = 155648;                    // their low parts
+constexpr uint32_t BT_MISC = BT_I4 + 16384;
+constexpr uint32_t BT_BETA = BT_MISC, BT_G = BT_BETA + 256, BT_TOT = BT_G + 2560, BT_RS = BT_TOT + 2048,
+                   BT_DGC = BT_RS + 2048, BT_DB = BT_DGC + 2048, BT_BAR = BT_DB + 256, BT_TPTR = BT_BAR + 64;
+constexpr uint32_t BT_SMEM = BT_TPTR + 16 + 1024;
+constexpr int BT_LDA = TRI_LDA;
+// TMEM columns
+constexpr uint32_t TB_AP = 0, TB_X1 = 160, TB_DU = 224, TB_U = 288, TB_Y = 352, TB_KC = 416;
+constexpr uint32_t TB_S4A = 288, TB_S4B = 160, TB_S5A = 288, TB_S5B = 0;
+// column versions of the keys (forward stage 1): Kd [0,64), Kb1 [64,80), Kb2 [80,112), Kb3 [112,160)
+constexpr uint32_t SV_B1 = 64, SV_B2 = 80, SV_B3 = 112, NSV = 160;
 
-    for (int64_t item = blockIdx.x; item < n_items; item += gridDim.x) {
+static_assert(BT_I10 + 16384 <= BT_I3, "I10 overlaps I3");
+static_assert(BT_I2 + 40960 <= BT_I3, "stage-1 KC image overlaps KG");
+static_assert(BT_TMP + 8192 <= BT_I8, "inverse scratch overlaps P");
+static_assert(BT_SMEM <= 227 * 1024, "shared memory");
+static_assert(BT_I1L + 32768 <= BT_MISC, "stage-5 low parts overlap the scalars");
+
+KDA_DEV uint32_t il_off(uint32_t r, uint32_t c, uint32_t nc) {
+    return (r >> 3) * (16u * nc) + (c >> 3) * 128u + (r & 7u) * 16u + (c & 7u) * 2u;
+}
+// descriptor of an image with nc columns read with its columns as the MN dimension
+// (rows = K) or as the K dimension (rows = M/N); `col0` selects a first column (multiple of 8)
+KDA_DEV uint64_t desc_mn(uint32_t addr, uint32_t nc, uint32_t col0 = 0) {
+    return sdesc_interleave(addr + (col0 >> 3) * 128u, 16u * nc, 128u);
+}
+KDA_DEV uint64_t desc_k(uint32_t addr, uint32_t nc, uint32_t col0 = 0) {
+    return sdesc_interleave(addr + (col0 >> 3) * 128u, 128u, 16u * nc);
+}
+// K-step (16) advance of the two views, in bytes
+KDA_DEV constexpr uint32_t step_mn(uint32_t nc) { return 32u * nc; }
+constexpr uint32_t STEP_K = 256u;
+
+// D (+)= A B^T over nk steps of K = 16
+KDA_DEV void mma_run(uint32_t d, uint64_t ad, uint32_t astep, uint64_t bd, uint32_t bstep, uint32_t idesc, int nk,
+                     bool acc) {
+    for (int kk = 0; kk < nk; ++kk)
+        mma_bf16(d, ad + ((uint32_t)kk * astep >> 4), bd + ((uint32_t)kk * bstep >> 4), idesc,
+                 (acc || kk > 0) ? 1u : 0u);
+}
+
+KDA_DEV void tmem_ld8(uint32_t taddr, float* r) {
+    uint32_t* u = reinterpret_cast<uint32_t*>(r);
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                 : "=r"(u[0]), "=r"(u[1]), "=r"(u[2]), "=r"(u[3]), "=r"(u[4]), "=r"(u[5]), "=r"(u[6]), "=r"(u[7])
+                 : "r"(taddr));
+}
+
+KDA_DEV uint4 pack8f(const float* x) {
+    return make_uint4(pack_bf16x2(x[0], x[1]), pack_bf16x2(x[2], x[3]), pack_bf16x2(x[4], x[5]),
+                      pack_bf16x2(x[6], x[7]));
+}
+KDA_DEV void st16(uint8_t* p, const float* x) { *reinterpret_cast<uint4*>(p) = pack8f(x); }
+// x as the sum of two bf16 images, hi = bf16(x) and lo = bf16(x - hi): a product with
+// both (two MMAs into one accumulator) carries about 16 bits of x instead of 8
+KDA_DEV void st16_hilo(uint8_t* hi, uint8_t* lo, const float* x) {
+    float h[8], l[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+        h[e] = __bfloat162float(__float2bfloat16_rn(x[e]));
+        l[e] = x[e] - h[e];
+    }
+    *reinterpret_cast<uint4*>(hi) = pack8f(h);
+    *reinterpret_cast<uint4*>(lo) = pack8f(l);
+}
+KDA_DEV void st16z(uint8_t* p) { *reinterpret_cast<uint4*>(p) = make_uint4(0u, 0u, 0u, 0u); }
+KDA_DEV float lo_bf(uint32_t w) { return __uint_as_float(w << 16); }
+KDA_DEV float hi_bf(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+// Sum over the 32 lanes of v[u] for each u < 16; lane l ends with the sum for token
+// u = l >> 1 (both lanes of a pair hold it).  16 shuffles.
+KDA_DEV float lane_sum16(float (&v)[16], int lane) {
+    float w8[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+        const bool up = lane & 16;
+        const float send = up ? v[k] : v[k + 8], keep = up ? v[k + 8] : v[k];
+        w8[k] = keep + __shfl_xor_sync(0xFFFFFFFFu, send, 16);
+    }
+    float w4[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        const bool up = lane & 8;
+        const float send = up ? w8[k] : w8[k + 4], keep = up ? w8[k + 4] : w8[k];
+        w4[k] = keep + __shfl_xor_sync(0xFFFFFFFFu, send, 8);
+    }
+    float w2[2];
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+        const bool up = lane & 4;
+        const float send = up ? w4[k] : w4[k + 2], keep = up ? w4[k + 2] : w4[k];
+        w2[k] = keep + __shfl_xor_sync(0xFFFFFFFFu, send, 4);
+    }
+    const bool up = lane & 2;
+    float w1 = (up ? w2[1] : w2[0]) + __shfl_xor_sync(0xFFFFFFFFu, up ? w2[0] : w2[1], 2);
+    w1 += __shfl_xor_sync(0xFFFFFFFFu, w1, 1);
+    return w1;  // token index: 8 (lane>>4 & 1) + 4 (lane>>3 & 1) + 2 (lane>>2 & 1) + (lane>>1 & 1)
+}
+KDA_DEV int lane_sum16_token(int lane) { return (lane >> 1) & 15; }
+
+// log-decays of the 16 tokens of tile q4 at channel c: per-step decays and the in-tile
+// prefix / suffix products E1 = e^{g_t - G_q4}, E3 = e^{G_{q4+1} - g_t}; returns the tile total
+template <bool IN_BF16>
+KDA_DEV float tile_decays(const BwdArgs& a, size_t base_c, size_t rowk, int q4, int L, float (&E1)[16],
+                          float (&E3)[16], uint32_t* keep_mask) {
+    float alpha[16];
+    float run = 0.f;
+    uint32_t keep = 0;
+#pragma unroll
+    for (int u = 0; u < 16; ++u) {
+        const int t = 16 * q4 + u;
+        float l = 0.f;
+        if (t < L) {
+            l = ld_in(a.log_alpha, base_c + (size_t)t * rowk, IN_BF16 ? 1 : 0);
+            if (l >= -5.f) keep |= 1u << u;
+            l = fmaxf(l, -5.f);
+        }
+        run += l;
+        alpha[u] = __expf(l);
+    }
+    E1[0] = alpha[0];
+#pragma unroll
+    for (int u = 1; u < 16; ++u) E1[u] = E1[u - 1] * alpha[u];
+    E3[15] = 1.f;
+#pragma unroll
+    for (int u = 14; u >= 0; --u) E3[u] = E3[u + 1] * alpha[u + 1];
+    if (keep_mask) *keep_mask = keep;
+    return run;
+}
+
+template <bool IN_BF16>
+__global__ void __launch_bounds__(BT_THREADS, 1) bwd_tc_kernel(const BwdArgs a, int64_t n_items) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    const uint32_t sb = smem_u32(sm);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int c = tid & 127, q4 = tid >> 7, qd = warp & 3;
+    const int H = a.H;
+    float* s_beta = reinterpret_cast<float*>(sm + BT_BETA);
+    float* s_G = reinterpret_cast<float*>(sm + BT_G);       // [5][128]
+    float* s_tot = reinterpret_cast<float*>(sm + BT_TOT);   // [4][128]
+    float* s_rs = reinterpret_cast<float*>(sm + BT_RS);     // [4][128] rowsum(S0 o dSC) partials
+    float* s_dgc = reinterpret_cast<float*>(sm + BT_DGC);   // [4][128] dL/dg_C partials
+    float* s_db = reinterpret_cast<float*>(sm + BT_DB);     // [64] dL/dbeta
+    uint64_t* bar = reinterpret_cast<uint64_t*>(sm + BT_BAR);  // [6]
+    uint32_t* s_tmem = reinterpret_cast<uint32_t*>(sm + BT_TPTR);
+    if (warp == 0) {
+        tmem_alloc(s_tmem, 512);
+        tmem_relinquish();
+    }
+    if (tid == 0) {
+        for (int i = 0; i < 6; ++i) mbar_init(&bar[i], 1);
+        fence_mbar_init();
+    }
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tm = *s_tmem;
+    const uint32_t lane_addr = tm + ((uint32_t)(32 * qd) << 16);
+    uint32_t par = 0;
+    bool failed = false;
+    int committed = 0;  // barriers committed in the current item (for the bounded drain)
+
+    // waits for the tensor-core products of barrier i; a wait that gives up ends the
+    // kernel's work on every thread at once
+    auto wait_mma = [&](int i) -> bool {
+        const bool ok = mbar_wait(&bar[i], par, a.status);
+        const bool any_fail = __syncthreads_or(!ok);
+        tc_fence_after();
+        return !any_fail;
+    };
+    auto images_ready = [&]() {
+        fence_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+    };
+
+    for (int64_t item = blockIdx.x; item < n_items && !failed; item += gridDim.x) {
         const int h = (int)(item % H);
-        const int c = (int)((item / H) % a.wc);
+        const int cidx = (int)((item / H) % a.wc);
         const int n = (int)(item / ((int64_t)H * a.wc));
         int64_t s_beg, s_end;
         bwd_seq_range(a, n, s_beg, s_end);
-        const int64_t t0 = s_beg + (int64_t)c * CH;
+        const int64_t t0 = s_beg + (int64_t)cidx * CH;
         if (t0 >= s_end) continue;  // uniform over the CTA
         const int L = (int)((s_end - t0) < CH ? (s_end - t0) : CH);
-        const int nb = (L + 15) >> 4;
-        const float* S0 = c == 0 ? (a.init_state ? a.init_state + ((size_t)n * H + h) * STATE : nullptr)
-                                 : a.ckpt + (((size_t)n * a.n_ckpt + (c - 1)) * H + h) * STATE;
-        const float* dSC = a.ds_end + (((size_t)n * a.wc + c) * H + h) * STATE;
-        prefetch_item(a, item + gridDim.x, n_items, tid);  // the next item's inputs into L2
+        const float* S0 = cidx == 0 ? (a.init_state ? a.init_state + ((size_t)n * H + h) * STATE : nullptr)
+                                    : a.ckpt + (((size_t)n * a.n_ckpt + (cidx - 1)) * H + h) * STATE;
+        const float* dSC = a.ds_end + (((size_t)n * a.wc + cidx) * H + h) * STATE;
+        prefetch_item(a, item + gridDim.x, n_items, tid);
+        const size_t rowk = (size_t)H * DK;
+        const size_t base_c = ((size_t)t0 * H + h) * DK + c;  // (token t0, head h, channel c)
+        const int ib = IN_BF16 ? 1 : 0;
 
-        // ---- P0: beta, g (cumulative clamped log-decay), zeroed accumulators
+        // ================================================================ phase A
+        float E1[16], E3[16];
+        const float run = tile_decays<IN_BF16>(a, base_c, rowk, q4, L, E1, E3, nullptr);
+        s_tot[q4 * 128 + c] = run;
         if (tid < CH) {
-            sBeta[tid] = tid < L ? ld_in(a.beta, (size_t)(t0 + tid) * H + h, a.in_bf16) : 0.f;
-            sDb[tid] = 0.f;
-        }
-        if (tid < DK) {
-            float lv[CH];  // all loads in flight at once
-#pragma unroll
-            for (int t = 0; t < CH; ++t)
-                lv[t] = t < L ? fmaxf(ld_in(a.log_alpha, ((size_t)(t0 + t) * H + h) * DK + tid, a.in_bf16), -5.f) : 0.f;
-            float g = 0.f;
-#pragma unroll
-            for (int t = 0; t < CH; ++t) {
-                g += lv[t];
-                sG[t * DK + tid] = g;
-            }
-            sGC[tid] = g;
-            sDgC[tid] = 0.f;
-        }
-        for (int e = tid; e < CH * LP; e += BI_THREADS) {
-            sA[e] = 0.f; sP[e] = 0.f; sdP[e] = 0.f; sdM[e] = 0.f;
+            s_beta[tid] = tid < L ? ld_in(a.beta, (size_t)(t0 + tid) * H + h, ib) : 0.f;
+            s_db[tid] = 0.f;
         }
         __syncthreads();
-
-        // ---- P1: A (s < t) and P (s <= t), block row by block row
-        for (int bt = 0; bt < nb; ++bt) {
-            build_factors(a, sF, sG, bt, t0, L, h, tid);
-            __syncthreads();
-            const int ns = 16 * bt + 16;
-            for (int e = tid; e < 16 * ns; e += BI_THREADS) {
-                const int tl = e & 15, s = e >> 4, t = 16 * bt + tl;
-                if (t >= L || s > t) continue;
-                const float* kin = sF + (64 + tl) * FP;
-                const float* qin = sF + (80 + tl) * FP;
-                const float* ko = sF + s * FP;
-                float da = 0.f, dp = 0.f;
-#pragma unroll 8
-                for (int i4 = 0; i4 < DK; i4 += 4) {
-                    const float4 kv = *reinterpret_cast<const float4*>(ko + i4);
-                    const float4 x = *reinterpret_cast<const float4*>(kin + i4);
-                    const float4 y = *reinterpret_cast<const float4*>(qin + i4);
-                    da += x.x * kv.x + x.y * kv.y + x.z * kv.z + x.w * kv.w;
-                    dp += y.x * kv.x + y.y * kv.y + y.z * kv.z + y.w * kv.w;
-                }
-                if (s < t) sA[t * LP + s] = da;
-                sP[t * LP + s] = dp;
-            }
-            __syncthreads();
-        }
-
-        // ---- P2: M^-1, M = I + Diag(beta) A (unit lower triangular): column cc by the
-        // 8 lanes tid / 8 == cc, forward substitution down the rows, the sum over earlier
-        // rows split over the lanes and reduced by shuffles (all lanes take part in every
-        // shuffle; loop trip counts differ, the warp reconverges before them)
         {
-            const int cc = tid >> 3, part = tid & 7;
-            for (int t = 0; t < CH; ++t) {
-                float p = 0.f;
-                for (int s = cc + part; s < t; s += 8) p += sA[t * LP + s] * sMi[s * LP + cc];
-                p += __shfl_xor_sync(0xFFFFFFFFu, p, 1);
-                p += __shfl_xor_sync(0xFFFFFFFFu, p, 2);
-                p += __shfl_xor_sync(0xFFFFFFFFu, p, 4);
-                const float x = t < cc ? 0.f : (t == cc ? 1.f : -sBeta[t] * p);
-                if (part == 0) sMi[t * LP + cc] = x;
-                __syncwarp();
-            }
-        }
-        // factors K o Gam (rows 0-63) and K^C = K o e^{g_C - g} (rows 64-127)
-        for (int e0 = tid; e0 < CH * DK; e0 += 4 * BI_THREADS) {
-            float kv[4];
+            float off = 0.f;
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const int e = e0 + u * BI_THREADS, t = e >> 7, i = e & (DK - 1);
-                kv[u] = t < L ? ld_in(a.k, ((size_t)(t0 + t) * H + h) * DK + i, a.in_bf16) : 0.f;
-            }
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const int e = e0 + u * BI_THREADS, t = e >> 7, i = e & (DK - 1);
-                const float g = sG[t * DK + i];
-                sF[t * FP + i] = kv[u] * __expf(g);
-                sF[(64 + t) * FP + i] = kv[u] * __expf(sGC[i] - g);
-            }
+            for (int qq = 0; qq < 3; ++qq)
+                if (qq < q4) off += s_tot[qq * 128 + c];
+            s_G[(q4 + 1) * 128 + c] = off + run;
+            if (q4 == 0) s_G[c] = 0.f;
         }
         __syncthreads();
-
-        float aQG[4][4], aKG[4][4], aKC[4][4], rowS[4];
+        float G[5];
 #pragma unroll
-        for (int x = 0; x < 4; ++x) {
-            rowS[x] = 0.f;
+        for (int b = 0; b < 5; ++b) G[b] = s_G[b * 128 + c];
+        const float Gs = (q4 == 0) ? G[0] : (q4 == 1) ? G[1] : (q4 == 2) ? G[2] : G[3];
+        const float Gn = (q4 == 0) ? G[1] : (q4 == 1) ? G[2] : (q4 == 2) ? G[3] : G[4];
+        // raw k, q, v of this thread's 16 tokens (bf16 bit pairs; exact for bf16 inputs)
+        uint32_t kr2[8], qr2[8], vr2[8];
+        {
+            const float eD = __expf(Gs - Gn);
+            const float f2 = __expf(((q4 == 0) ? G[2] : G[3]) - Gn);
+            const float f3 = __expf(G[3] - Gn);
+            const float eG = __expf(Gs), eC = __expf(G[4] - Gn);
 #pragma unroll
-            for (int y = 0; y < 4; ++y) aQG[x][y] = aKG[x][y] = aKC[x][y] = 0.f;
+            for (int m = 0; m < 2; ++m) {
+                const int tf = 16 * q4 + 8 * m;
+                float kv[8], qv[8], vv[8], dov[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const int t = tf + e;
+                    const bool in = t < L;
+                    const size_t idx = base_c + (size_t)t * rowk;
+                    kv[e] = in ? ld_in(a.k, idx, ib) : 0.f;
+                    qv[e] = in ? ld_in(a.q, idx, ib) : 0.f;
+                    vv[e] = in ? ld_in(a.v, idx, ib) : 0.f;
+                    dov[e] = in ? ld_in(a.d_o, idx, ib) : 0.f;
+                }
+#pragma unroll
+                for (int e = 0; e < 8; e += 2) {
+                    kr2[(8 * m + e) >> 1] = pack_bf16x2(kv[e], kv[e + 1]);
+                    qr2[(8 * m + e) >> 1] = pack_bf16x2(qv[e], qv[e + 1]);
+                    vr2[(8 * m + e) >> 1] = pack_bf16x2(vv[e], vv[e + 1]);
+                }
+                float x[8], y[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    x[e] = kv[e] * E1[8 * m + e];
+                    y[e] = qv[e] * E1[8 * m + e] * a.scale;
+                }
+                st16(sm + BT_I1 + il_off(c, tf, 128), x);
+                st16(sm + BT_I1 + il_off(c, 64 + tf, 128), y);
+                float k3[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    k3[e] = kv[e] * E3[8 * m + e];
+                    x[e] = k3[e] * eD;
+                }
+                st16(sm + BT_I2 + il_off(c, tf, NSV), x);
+                if (q4 == 0) {
+                    st16(sm + BT_I2 + il_off(c, SV_B1 + tf, NSV), k3);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) x[e] = k3[e] * f2;
+                    st16(sm + BT_I2 + il_off(c, SV_B2 + tf, NSV), x);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) x[e] = k3[e] * f3;
+                    st16(sm + BT_I2 + il_off(c, SV_B3 + tf, NSV), x);
+                } else if (q4 == 1) {
+                    st16(sm + BT_I2 + il_off(c, SV_B2 + tf, NSV), k3);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) x[e] = k3[e] * f3;
+                    st16(sm + BT_I2 + il_off(c, SV_B3 + tf, NSV), x);
+                } else if (q4 == 2) {
+                    st16(sm + BT_I2 + il_off(c, SV_B3 + tf, NSV), k3);
+                }
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    x[e] = kv[e] * E1[8 * m + e] * eG;  // k e^{g}
+                    y[e] = k3[e] * eC;                  // k e^{g_C - g}
+                }
+                st16(sm + BT_I3 + il_off(c, tf, 64), x);
+                st16(sm + BT_I4 + il_off(c, tf, 64), y);
+                st16(sm + BT_I7 + il_off(c, 64 + tf, 128), dov);  // dO^T: row j = c
+            }
+            // S0 and dSC row c, columns [32 q4, 32 q4 + 32)
+            float rs = 0.f;
+#pragma unroll
+            for (int m = 0; m < 4; ++m) {
+                const int j = 32 * q4 + 8 * m;
+                float s8[8], d8[8];
+                if (S0) {
+                    const float4 u0 = __ldg(reinterpret_cast<const float4*>(S0 + (size_t)c * DV + j));
+                    const float4 u1 = __ldg(reinterpret_cast<const float4*>(S0 + (size_t)c * DV + j + 4));
+                    s8[0] = u0.x; s8[1] = u0.y; s8[2] = u0.z; s8[3] = u0.w;
+                    s8[4] = u1.x; s8[5] = u1.y; s8[6] = u1.z; s8[7] = u1.w;
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) s8[e] = 0.f;
+                }
+                const float4 w0 = __ldg(reinterpret_cast<const float4*>(dSC + (size_t)c * DV + j));
+                const float4 w1 = __ldg(reinterpret_cast<const float4*>(dSC + (size_t)c * DV + j + 4));
+                d8[0] = w0.x; d8[1] = w0.y; d8[2] = w0.z; d8[3] = w0.w;
+                d8[4] = w1.x; d8[5] = w1.y; d8[6] = w1.z; d8[7] = w1.w;
+#pragma unroll
+                for (int e = 0; e < 8; ++e) rs += s8[e] * d8[e];
+                st16(sm + BT_I5 + il_off(c, j, 128), s8);
+                st16(sm + BT_I6 + il_off(c, j, 128), d8);
+            }
+            s_rs[q4 * 128 + c] = rs;
         }
+        images_ready();
 
-        // ---- P3: value columns in quarters of 32
-        for (int qd = 0; qd < DV / NQ; ++qd) {
-            const int j0 = NQ * qd;
-            // (a) dO quarter and R = V - (K o Gam) S0
-            {
-                const int t = tid >> 3, jq = (tid & 7) * 4;
-                float r4[4] = {0.f, 0.f, 0.f, 0.f}, o4[4] = {0.f, 0.f, 0.f, 0.f};
-                if (t < L) {
-                    const size_t base = ((size_t)(t0 + t) * H + h) * DV + j0 + jq;
+        // ------------------------------------------------------------- stage 1
+        if (tid == 0) {
+            mma_run(tm + TB_AP, desc_mn(sb + BT_I1, 128), step_mn(128), desc_mn(sb + BT_I2, NSV), step_mn(NSV),
+                    idesc_bf16_major(128, 160, 1, 1), 8, false);
+            mma_commit(&bar[0]);
+            mma_run(tm + TB_X1, desc_mn(sb + BT_I5, 128), step_mn(128), desc_mn(sb + BT_I3, 64), step_mn(64),
+                    idesc_bf16_major(128, 64, 1, 1), 8, false);
+            mma_run(tm + TB_DU, desc_mn(sb + BT_I6, 128), step_mn(128), desc_mn(sb + BT_I4, 64), step_mn(64),
+                    idesc_bf16_major(128, 64, 1, 1), 8, false);
+            mma_commit(&bar[1]);
+        }
+        committed = 2;
+
+        // ================================================================ phase B
+        if (!wait_mma(0)) { failed = true; break; }
+        {   // A (rows 0..63) -> N = Diag(beta) A fp32;  P (rows 64..127) -> image I8 [t][s]
+            float* sN = reinterpret_cast<float*>(sm + BT_N);
+            const int p = q4, r = 32 * qd + lane;
+            const bool isP = r >= 64;
+            const int t = r & 63, bt = t >> 4;
+            float dA[16], dB[16], dC[16];
+            tmem_ld16(lane_addr + TB_AP + 16 * p, dA);
+            if ((qd & 1) == 0) {
+                if (p == 0) tmem_ld16(lane_addr + TB_AP + SV_B1, dB);
+            } else {
+                if (p < 2) tmem_ld16(lane_addr + TB_AP + SV_B2 + 16 * p, dB);
+                if (p < 3) tmem_ld16(lane_addr + TB_AP + SV_B3 + 16 * p, dC);
+            }
+            tmem_ld_wait();
+            float d[16];
+            if (p >= bt) {
 #pragma unroll
-                    for (int x = 0; x < 4; ++x) {
-                        r4[x] = ld_in(a.v, base + x, a.in_bf16);
-                        o4[x] = ld_in(a.d_o, base + x, a.in_bf16);
+                for (int s16 = 0; s16 < 16; ++s16) {
+                    const int s = 16 * p + s16;
+                    const bool keep = (p == bt) && (isP ? (s <= t) : (s < t));
+                    d[s16] = keep ? dA[s16] : 0.f;
+                }
+            } else if (bt == 3) {
+#pragma unroll
+                for (int s16 = 0; s16 < 16; ++s16) d[s16] = dC[s16];
+            } else {
+#pragma unroll
+                for (int s16 = 0; s16 < 16; ++s16) d[s16] = dB[s16];
+            }
+            if (isP) {
+                st16(sm + BT_I8 + il_off(t, 16 * p, 64), d);
+                st16(sm + BT_I8 + il_off(t, 16 * p + 8, 64), d + 8);
+            } else {
+                const float bt_ = s_beta[t];
+                float4* dst = reinterpret_cast<float4*>(sN + t * BT_LDA + 16 * p);
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                    dst[i] = make_float4(bt_ * d[4 * i], bt_ * d[4 * i + 1], bt_ * d[4 * i + 2], bt_ * d[4 * i + 3]);
+            }
+        }
+        if (!wait_mma(1)) { failed = true; break; }
+        float R[16];
+        {   // R = V - (K o Gam) S0 for this thread's value column j = c and 16 tokens
+            float x1[16];
+            tmem_ld16(lane_addr + TB_X1 + 16 * q4, x1);
+            tmem_ld_wait();
+            float br[16];
+#pragma unroll
+            for (int u = 0; u < 16; ++u) {
+                const float vv = IN_BF16 ? ((u & 1) ? hi_bf(vr2[u >> 1]) : lo_bf(vr2[u >> 1]))
+                                         : (16 * q4 + u < L ? ld_in(a.v, base_c + (size_t)(16 * q4 + u) * rowk, 0) : 0.f);
+                R[u] = vv - x1[u];
+                br[u] = s_beta[16 * q4 + u] * R[u];
+            }
+            st16(sm + BT_I10 + il_off(c, 16 * q4, 64), br);
+            st16(sm + BT_I10 + il_off(c, 16 * q4 + 8, 64), br + 8);
+        }
+        __syncthreads();
+        tri_inverse64(reinterpret_cast<const float*>(sm + BT_N), reinterpret_cast<float*>(sm + BT_X),
+                      reinterpret_cast<float*>(sm + BT_TMP), reinterpret_cast<float*>(sm + BT_N), tid);
+        {   // Minv image I9 [t][s] (blocks above the diagonal are zero)
+            const float* sX = reinterpret_cast<const float*>(sm + BT_X);
+            const float* sP = reinterpret_cast<const float*>(sm + BT_N);  // second half of the lower-left sums
+            const int t = tid >> 3, s0 = (tid & 7) * 8;
+            float v8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+            if ((s0 >> 4) <= (t >> 4)) {
+                float4 x0 = *reinterpret_cast<const float4*>(sX + t * BT_LDA + s0);
+                float4 x1 = *reinterpret_cast<const float4*>(sX + t * BT_LDA + s0 + 4);
+                if (t >= 48 && s0 < 32) {
+                    const float4 p0 = *reinterpret_cast<const float4*>(sP + (t - 48) * 32 + s0);
+                    const float4 p1 = *reinterpret_cast<const float4*>(sP + (t - 48) * 32 + s0 + 4);
+                    x0.x += p0.x; x0.y += p0.y; x0.z += p0.z; x0.w += p0.w;
+                    x1.x += p1.x; x1.y += p1.y; x1.z += p1.z; x1.w += p1.w;
+                }
+                v8[0] = x0.x; v8[1] = x0.y; v8[2] = x0.z; v8[3] = x0.w;
+                v8[4] = x1.x; v8[5] = x1.y; v8[6] = x1.z; v8[7] = x1.w;
+            }
+            st16(sm + BT_I9 + il_off(t, s0, 64), v8);
+        }
+        images_ready();
+
+        // ------------------------------------------------------------- stage 2
+        if (tid == 0) {
+            mma_run(tm + TB_U, desc_k(sb + BT_I10, 64), STEP_K, desc_k(sb + BT_I9, 64), STEP_K,
+                    idesc_bf16_major(128, 64, 0, 0), 4, false);
+            mma_run(tm + TB_DU, desc_k(sb + BT_I7, 128, 64), STEP_K, desc_mn(sb + BT_I8, 64), step_mn(64),
+                    idesc_bf16_major(128, 64, 0, 1), 4, true);
+            mma_commit(&bar[2]);
+        }
+        committed = 3;
+
+        // ================================================================ phase C
+        if (!wait_mma(2)) { failed = true; break; }
+        {
+            float x[16];
+            tmem_ld16(lane_addr + TB_U + 16 * q4, x);
+            tmem_ld_wait();
+            st16(sm + BT_I12 + il_off(c, 16 * q4, 64), x);
+            st16(sm + BT_I12 + il_off(c, 16 * q4 + 8, 64), x + 8);
+            tmem_ld16(lane_addr + TB_DU + 16 * q4, x);
+            tmem_ld_wait();
+            st16(sm + BT_I11 + il_off(c, 16 * q4, 64), x);
+            st16(sm + BT_I11 + il_off(c, 16 * q4 + 8, 64), x + 8);
+        }
+        images_ready();
+
+        // ------------------------------------------------------------- stage 3
+        if (tid == 0) {
+            mma_run(tm + TB_Y, desc_k(sb + BT_I11, 64), STEP_K, desc_mn(sb + BT_I9, 64), step_mn(64),
+                    idesc_bf16_major(128, 64, 0, 1), 4, false);
+            mma_run(tm + TB_KC, desc_k(sb + BT_I6, 128), STEP_K, desc_mn(sb + BT_I12, 64), step_mn(64),
+                    idesc_bf16_major(128, 64, 0, 1), 8, false);
+            mma_commit(&bar[3]);
+        }
+        committed = 4;
+
+        // ================================================================ phase D
+        if (!wait_mma(3)) { failed = true; break; }
+        {
+            float y[16];
+            tmem_ld16(lane_addr + TB_Y + 16 * q4, y);
+            tmem_ld_wait();
+            float pr[16];
+#pragma unroll
+            for (int u = 0; u < 16; ++u) {
+                const int t = 16 * q4 + u;
+                pr[u] = y[u] * R[u];
+                if (t < L) a.dv[((size_t)(t0 + t) * H + h) * DV + c] = s_beta[t] * y[u];
+            }
+            st16(sm + BT_I7 + il_off(c, 16 * q4, 128), y);
+            st16(sm + BT_I7 + il_off(c, 16 * q4 + 8, 128), y + 8);
+            const float sum = lane_sum16(pr, lane);
+            if ((lane & 1) == 0) atomicAdd(&s_db[16 * q4 + lane_sum16_token(lane)], sum);
+        }
+        images_ready();
+
+        // ------------------------------------------------------------- stage 4
+        if (tid == 0) {
+            mma_run(tm + TB_S4A, desc_mn(sb + BT_I7, 128), step_mn(128), desc_mn(sb + BT_I12, 64), step_mn(64),
+                    idesc_bf16_major(128, 64, 1, 1), 8, false);
+            mma_run(tm + TB_S4B, desc_k(sb + BT_I5, 128), STEP_K, desc_mn(sb + BT_I7, 128), step_mn(128),
+                    idesc_bf16_major(128, 128, 0, 1), 8, false);
+            mma_commit(&bar[4]);
+        }
+        committed = 5;
+
+        // ================================================================ phase E
+        if (!wait_mma(4)) { failed = true; break; }
+        uint32_t keep_la = 0;  // tokens whose log-decay is at or above the floor (the clamp passes them)
+        {   // [-dM ; dP] rows -> [A' ; P'] image at their column versions, dbeta's dM o A part
+            const int p = q4, r = 32 * qd + lane;
+            const bool isP = r >= 64;
+            const int t = r & 63, bt = t >> 4;
+            float val[16], dmv[16];
+            {
+                float dd[16];
+                tmem_ld16(lane_addr + TB_S4A + 16 * p, dd);
+                tmem_ld_wait();
+                const float bt_ = s_beta[t];
+#pragma unroll
+                for (int s16 = 0; s16 < 16; ++s16) {
+                    const int s = 16 * p + s16;
+                    dmv[s16] = (!isP && s < t) ? -dd[s16] : 0.f;
+                    val[s16] = isP ? ((s <= t) ? dd[s16] : 0.f) : bt_ * dmv[s16];
+                }
+            }
+            if (!isP) {
+                // dbeta += sum_s dM_ts A_ts over this piece: the unscaled A row piece from the
+                // stage-1 accumulator, selected per lane from warp-uniform loads (tcgen05.ld
+                // is warp-collective), as in the extraction
+                float db2 = 0.f, aa[16];
+                tmem_ld16(lane_addr + TB_AP + 16 * p, aa);
+                tmem_ld_wait();
+                if (p == bt) {
+#pragma unroll
+                    for (int s16 = 0; s16 < 16; ++s16) db2 += dmv[s16] * aa[s16];
+                }
+                if (qd == 0 && p == 0) {
+                    tmem_ld16(lane_addr + TB_AP + SV_B1, aa);
+                    tmem_ld_wait();
+                    if (bt == 1) {
+#pragma unroll
+                        for (int s16 = 0; s16 < 16; ++s16) db2 += dmv[s16] * aa[s16];
                     }
-                    if (S0) {
-                        const float* kg = sF + t * FP;
-#pragma unroll 8
-                        for (int i = 0; i < DK; ++i) {
-                            const float4 s4 = __ldg(reinterpret_cast<const float4*>(S0 + (size_t)i * DV + j0 + jq));
-                            const float w = kg[i];
-                            r4[0] -= w * s4.x; r4[1] -= w * s4.y; r4[2] -= w * s4.z; r4[3] -= w * s4.w;
-                        }
+                }
+                if (qd == 1 && p < 2) {
+                    tmem_ld16(lane_addr + TB_AP + SV_B2 + 16 * p, aa);
+                    tmem_ld_wait();
+                    if (bt == 2) {
+#pragma unroll
+                        for (int s16 = 0; s16 < 16; ++s16) db2 += dmv[s16] * aa[s16];
                     }
                 }
+                if (qd == 1 && p < 3) {
+                    tmem_ld16(lane_addr + TB_AP + SV_B3 + 16 * p, aa);
+                    tmem_ld_wait();
+                    if (bt == 3) {
 #pragma unroll
-                for (int x = 0; x < 4; ++x) {
-                    sR[t * QP + jq + x] = r4[x];
-                    sDO[t * QP + jq + x] = o4[x];
-                }
-            }
-            __syncthreads();
-            // (b) U = M^-1 Diag(beta) R;  dU = P^T dO + K^C dS_C
-            {
-                const int t = tid >> 3, jq = (tid & 7) * 4;
-                float u4[4] = {0.f, 0.f, 0.f, 0.f}, d4[4] = {0.f, 0.f, 0.f, 0.f};
-                for (int s = 0; s <= t; ++s) {
-                    const float w = sMi[t * LP + s] * sBeta[s];
-#pragma unroll
-                    for (int x = 0; x < 4; ++x) u4[x] += w * sR[s * QP + jq + x];
-                }
-                for (int tt = t; tt < CH; ++tt) {
-                    const float w = sP[tt * LP + t];
-#pragma unroll
-                    for (int x = 0; x < 4; ++x) d4[x] += w * sDO[tt * QP + jq + x];
-                }
-                const float* kc = sF + (64 + t) * FP;
-#pragma unroll 8
-                for (int i = 0; i < DK; ++i) {
-                    const float4 s4 = __ldg(reinterpret_cast<const float4*>(dSC + (size_t)i * DV + j0 + jq));
-                    const float w = kc[i];
-                    d4[0] += w * s4.x; d4[1] += w * s4.y; d4[2] += w * s4.z; d4[3] += w * s4.w;
-                }
-#pragma unroll
-                for (int x = 0; x < 4; ++x) {
-                    sU[t * QP + jq + x] = u4[x];
-                    sDU[t * QP + jq + x] = d4[x];
-                }
-            }
-            __syncthreads();
-            // (c) Y = M^-T dU; dv = beta Y; rowsum(Y o R)
-            {
-                const int t = tid >> 3, jq = (tid & 7) * 4;
-                float y4[4] = {0.f, 0.f, 0.f, 0.f};
-                for (int s = t; s < CH; ++s) {
-                    const float w = sMi[s * LP + t];
-#pragma unroll
-                    for (int x = 0; x < 4; ++x) y4[x] += w * sDU[s * QP + jq + x];
-                }
-                float yr = 0.f;
-#pragma unroll
-                for (int x = 0; x < 4; ++x) yr += y4[x] * sR[t * QP + jq + x];
-                atomicAdd(&sDb[t], yr);
-                if (t < L) {
-                    const float b = sBeta[t];
-                    float4* dst = reinterpret_cast<float4*>(a.dv + ((size_t)(t0 + t) * H + h) * DV + j0 + jq);
-                    *dst = make_float4(b * y4[0], b * y4[1], b * y4[2], b * y4[3]);
-                }
-                __syncthreads();  // every read of dU is done
-#pragma unroll
-                for (int x = 0; x < 4; ++x) sDU[t * QP + jq + x] = y4[x];  // sDU now holds Y
-            }
-            __syncthreads();
-            // (d) dP += dO U^T (s <= t);  dM -= Y U^T (s < t)
-            {
-                // rows s = sl + 8 x: the 8 lanes sharing t read 8 consecutive rows of U
-                const int t = tid >> 3, sl = tid & 7;
-                float dp[8], dm[8];
-#pragma unroll
-                for (int x = 0; x < 8; ++x) dp[x] = dm[x] = 0.f;
-                for (int j = 0; j < NQ; ++j) {
-                    const float o = sDO[t * QP + j], y = sDU[t * QP + j];
-#pragma unroll
-                    for (int x = 0; x < 8; ++x) {
-                        const float u = sU[(sl + 8 * x) * QP + j];
-                        dp[x] += o * u;
-                        dm[x] -= y * u;
+                        for (int s16 = 0; s16 < 16; ++s16) db2 += dmv[s16] * aa[s16];
                     }
                 }
+                if (p <= bt) atomicAdd(&s_db[t], db2);
+            }
+            uint8_t* row = sm + BT_I13;
+            // Kd columns of tile p: the value on the diagonal block, zero elsewhere
+            if (p == bt) {
+                st16(row + il_off(r, 16 * p, NSV), val);
+                st16(row + il_off(r, 16 * p + 8, NSV), val + 8);
+            } else {
+                st16z(row + il_off(r, 16 * p, NSV));
+                st16z(row + il_off(r, 16 * p + 8, NSV));
+            }
+            // Kb pieces (6 of 16 columns): piece kb(bt) + p holds tile p < bt; the rest zero
+            const int kb = bt == 1 ? 0 : bt == 2 ? 1 : 3;  // first value piece of this row's tile
+            const int nval = bt;                           // value pieces: kb .. kb + bt - 1
+            if (p < bt) {
+                const uint32_t col = SV_B1 + 16u * (uint32_t)(kb + p);
+                st16(row + il_off(r, col, NSV), val);
+                st16(row + il_off(r, col + 8, NSV), val + 8);
+            }
 #pragma unroll
-                for (int x = 0; x < 8; ++x) {
-                    const int s = sl + 8 * x;
-                    if (s <= t) sdP[t * LP + s] += dp[x];
-                    if (s < t) sdM[t * LP + s] += dm[x];
+            for (int z = 0; z < 2; ++z) {
+                const int piece = p + 4 * z;
+                if (piece < 6 && !(bt > 0 && piece >= kb && piece < kb + nval)) {
+                    const uint32_t col = SV_B1 + 16u * (uint32_t)piece;
+                    st16z(row + il_off(r, col, NSV));
+                    st16z(row + il_off(r, col + 8, NSV));
                 }
             }
-            // (e) owned (t, i): dO S0^T, -(beta Y) S0^T, U dS_C^T over this quarter's columns
-            {
+        }
+        {   // KQr and KC again (their stage-1 copies were overwritten), now each as a high and a
+            // low bf16 part: the row (KC) and column (KQr) forms of every A and P term must round
+            // alike, or their contributions to dg, which cancel in dlog_alpha's chunk sums, stop
+            // cancelling
+            const float eD = __expf(Gs - Gn);
+            const float f2 = __expf(((q4 == 0) ? G[2] : G[3]) - Gn);
+            const float f3 = __expf(G[3] - Gn);
+            float (&E1b)[16] = E1;
+            float (&E3b)[16] = E3;
+            tile_decays<IN_BF16>(a, base_c, rowk, q4, L, E1b, E3b, &keep_la);
+#pragma unroll
+            for (int m = 0; m < 2; ++m) {
+                const int tf = 16 * q4 + 8 * m;
+                float x[8], y[8], k3[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const int u = 8 * m + e;
+                    float kv, qv;
+                    if (IN_BF16) {
+                        kv = (u & 1) ? hi_bf(kr2[u >> 1]) : lo_bf(kr2[u >> 1]);
+                        qv = (u & 1) ? hi_bf(qr2[u >> 1]) : lo_bf(qr2[u >> 1]);
+                    } else {
+                        const int t = tf + e;
+                        kv = t < L ? ld_in(a.k, base_c + (size_t)t * rowk, 0) : 0.f;
+                        qv = t < L ? ld_in(a.q, base_c + (size_t)t * rowk, 0) : 0.f;
+                    }
+                    x[e] = kv * E1b[u];
+                    y[e] = qv * E1b[u] * a.scale;
+                    k3[e] = kv * E3b[u];
+                }
+                st16_hilo(sm + BT_I1B + il_off(c, tf, 128), sm + BT_I1L + il_off(c, tf, 128), x);
+                st16_hilo(sm + BT_I1B + il_off(c, 64 + tf, 128), sm + BT_I1L + il_off(c, 64 + tf, 128), y);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) x[e] = k3[e] * eD;
+                st16_hilo(sm + BT_I2B + il_off(c, tf, NSV), sm + BT_I2L + il_off(c, tf, NSV), x);
+                if (q4 == 0) {
+                    st16_hilo(sm + BT_I2B + il_off(c, SV_B1 + tf, NSV), sm + BT_I2L + il_off(c, SV_B1 + tf, NSV), k3);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) x[e] = k3[e] * f2;
+                    st16_hilo(sm + BT_I2B + il_off(c, SV_B2 + tf, NSV), sm + BT_I2L + il_off(c, SV_B2 + tf, NSV), x);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) x[e] = k3[e] * f3;
+                    st16_hilo(sm + BT_I2B + il_off(c, SV_B3 + tf, NSV), sm + BT_I2L + il_off(c, SV_B3 + tf, NSV), x);
+                } else if (q4 == 1) {
+                    st16_hilo(sm + BT_I2B + il_off(c, SV_B2 + tf, NSV), sm + BT_I2L + il_off(c, SV_B2 + tf, NSV), k3);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) x[e] = k3[e] * f3;
+                    st16_hilo(sm + BT_I2B + il_off(c, SV_B3 + tf, NSV), sm + BT_I2L + il_off(c, SV_B3 + tf, NSV), x);
+                } else if (q4 == 2) {
+                    st16_hilo(sm + BT_I2B + il_off(c, SV_B3 + tf, NSV), sm + BT_I2L + il_off(c, SV_B3 + tf, NSV), k3);
+                }
+            }
+        }
+        images_ready();
+
+        // ------------------------------------------------------------- stage 5
+        if (tid == 0) {
+            mma_run(tm + TB_S5A, desc_k(sb + BT_I2B, NSV), STEP_K, desc_k(sb + BT_I13, NSV), STEP_K,
+                    idesc_bf16_major(128, 128, 0, 0), NSV / 16, false);
+            mma_run(tm + TB_S5A, desc_k(sb + BT_I2L, NSV), STEP_K, desc_k(sb + BT_I13, NSV), STEP_K,
+                    idesc_bf16_major(128, 128, 0, 0), NSV / 16, true);
+            mma_run(tm + TB_S5B, desc_k(sb + BT_I1B, 128), STEP_K, desc_mn(sb + BT_I13, NSV), step_mn(NSV),
+                    idesc_bf16_major(128, 160, 0, 1), 8, false);
+            mma_run(tm + TB_S5B, desc_k(sb + BT_I1L, 128), STEP_K, desc_mn(sb + BT_I13, NSV), step_mn(NSV),
+                    idesc_bf16_major(128, 160, 0, 1), 8, true);
+            mma_commit(&bar[5]);
+        }
+        committed = 6;
+
+        // ================================================================ phase F
+        if (!wait_mma(5)) { failed = true; break; }
+        {
+            const float eG = __expf(Gs), eC = __expf(G[4] - Gn), eD = __expf(Gs - Gn);
+            const float f2 = __expf(((q4 == 0) ? G[2] : G[3]) - Gn);
+            const float f3 = __expf(G[3] - Gn);
+            float* s_dg = reinterpret_cast<float*>(sm);  // [64 t][128 c]: every image is dead now
+            float dgc = 0.f, tot = 0.f;
 #pragma unroll 1
-                for (int j = 0; j < NQ; j += 4) {
-                    float4 s0v[4], dsv[4];
-#pragma unroll
-                    for (int y = 0; y < 4; ++y) {
-                        const int i = ig + 32 * y;
-                        s0v[y] = S0 ? __ldg(reinterpret_cast<const float4*>(S0 + (size_t)i * DV + j0 + j))
-                                    : make_float4(0.f, 0.f, 0.f, 0.f);
-                        dsv[y] = __ldg(reinterpret_cast<const float4*>(dSC + (size_t)i * DV + j0 + j));
+            for (int m = 0; m < 2; ++m) {
+                const uint32_t cu = 16u * q4 + 8u * m;
+                // this half's raw k, scale * q and decay factors (selected, not indexed, so that
+                // they stay in registers)
+                auto kv = [&](int e) -> float {
+                    const int u = 8 * m + e, t = 16 * q4 + u;
+                    if (IN_BF16) {
+                        const uint32_t w = m ? kr2[4 + (e >> 1)] : kr2[e >> 1];
+                        return (e & 1) ? hi_bf(w) : lo_bf(w);
                     }
-                    if (tg == 0) {
-#pragma unroll
-                        for (int y = 0; y < 4; ++y)
-                            rowS[y] += s0v[y].x * dsv[y].x + s0v[y].y * dsv[y].y + s0v[y].z * dsv[y].z +
-                                       s0v[y].w * dsv[y].w;
+                    return t < L ? ld_in(a.k, base_c + (size_t)t * rowk, 0) : 0.f;
+                };
+                auto qb = [&](int e) -> float {
+                    const int u = 8 * m + e, t = 16 * q4 + u;
+                    if (IN_BF16) {
+                        const uint32_t w = m ? qr2[4 + (e >> 1)] : qr2[e >> 1];
+                        return a.scale * ((e & 1) ? hi_bf(w) : lo_bf(w));
                     }
+                    return t < L ? a.scale * ld_in(a.q, base_c + (size_t)t * rowk, 0) : 0.f;
+                };
+                auto e1 = [&](int e) -> float { return m ? E1[8 + e] : E1[e]; };
+                auto e3 = [&](int e) -> float { return m ? E3[8 + e] : E3[e]; };
+                float dq8[8], dk8[8], dg8[8], x[8];
+                // q: through the state, dO S0^T scaled by Gam; through P's rows
+                tmem_ld8(lane_addr + TB_S4B + 64 + cu, x);
+                tmem_ld_wait();
 #pragma unroll
-                    for (int x = 0; x < 4; ++x) {
-                        const int t = 4 * tg + x;
-                        const float bt = sBeta[t];
-                        const float o[4] = {sDO[t * QP + j], sDO[t * QP + j + 1], sDO[t * QP + j + 2], sDO[t * QP + j + 3]};
-                        const float yy[4] = {bt * sDU[t * QP + j], bt * sDU[t * QP + j + 1], bt * sDU[t * QP + j + 2],
-                                             bt * sDU[t * QP + j + 3]};
-                        const float u[4] = {sU[t * QP + j], sU[t * QP + j + 1], sU[t * QP + j + 2], sU[t * QP + j + 3]};
+                for (int e = 0; e < 8; ++e) {
+                    const float w = e1(e) * eG * x[e];
+                    dq8[e] = w;
+                    dg8[e] = qb(e) * w;
+                }
+                tmem_ld8(lane_addr + TB_S5A + 64 + cu, x);
+                tmem_ld_wait();
 #pragma unroll
-                        for (int y = 0; y < 4; ++y) {
-                            const float sv[4] = {s0v[y].x, s0v[y].y, s0v[y].z, s0v[y].w};
-                            const float dv4[4] = {dsv[y].x, dsv[y].y, dsv[y].z, dsv[y].w};
+                for (int e = 0; e < 8; ++e) {
+                    const float w = e1(e) * x[e];
+                    dq8[e] += w;
+                    dg8[e] += qb(e) * w;
+                    const int t = (int)cu + e;
+                    if (t < L) a.dq[base_c + (size_t)t * rowk] = a.scale * dq8[e];
+                }
+                // k: through R, -(beta Y) S0^T scaled by Gam
+                tmem_ld8(lane_addr + TB_S4B + cu, x);
+                tmem_ld_wait();
 #pragma unroll
-                            for (int z = 0; z < 4; ++z) {
-                                aQG[x][y] += o[z] * sv[z];
-                                aKG[x][y] -= yy[z] * sv[z];
-                                aKC[x][y] += u[z] * dv4[z];
-                            }
-                        }
+                for (int e = 0; e < 8; ++e) {
+                    const float w = -s_beta[cu + e] * x[e] * e1(e) * eG;
+                    dk8[e] = w;
+                    dg8[e] += kv(e) * w;
+                }
+                // k: through the chunk-end state, U dS_C^T scaled by e^{g_C - g}
+                tmem_ld8(lane_addr + TB_KC + cu, x);
+                tmem_ld_wait();
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const float w = x[e] * e3(e) * eC;
+                    dk8[e] += w;
+                    dg8[e] -= kv(e) * w;
+                    dgc += kv(e) * w;
+                }
+                // k: A's rows (t as the row token)
+                tmem_ld8(lane_addr + TB_S5A + cu, x);
+                tmem_ld_wait();
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const float w = e1(e) * x[e];
+                    dk8[e] += w;
+                    dg8[e] += kv(e) * w;
+                }
+                // k: A's and P's columns (t as the column token): its versions, each with its factor
+                tmem_ld8(lane_addr + TB_S5B + cu, x);
+                tmem_ld_wait();
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const float w = e3(e) * eD * x[e];
+                    dk8[e] += w;
+                    dg8[e] -= kv(e) * w;
+                }
+                if (q4 <= 2) {  // the version of tile q4 + 1: factor e^{G_{q4+1} - g} = E3
+                    const uint32_t base = q4 == 0 ? SV_B1 : q4 == 1 ? SV_B2 + 16 : SV_B3 + 32;
+                    tmem_ld8(lane_addr + TB_S5B + base + 8u * m, x);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const float w = e3(e) * x[e];
+                        dk8[e] += w;
+                        dg8[e] -= kv(e) * w;
                     }
                 }
-            }
-            __syncthreads();  // the quarter buffers are rewritten next
-        }
-
-        // ---- P4: dbeta and dA = Diag(beta) dM
-        if (tid < CH) {
-            const int t = tid;
-            float acc = sDb[t];
-            for (int s = 0; s < t; ++s) acc += sdM[t * LP + s] * sA[t * LP + s];
-            if (t < L) a.dbeta[(size_t)(t0 + t) * H + h] = acc;
-            const float b = sBeta[t];
-            for (int s = 0; s < t; ++s) sdM[t * LP + s] *= b;
-        }
-        // owned accumulators -> gradients of qb, k, g
-        float dqb[4][4], dkk[4][4], dg[4][4];
+                if (q4 <= 1) {  // tile q4 + 2
+                    const uint32_t base = q4 == 0 ? SV_B2 : SV_B3 + 16;
+                    tmem_ld8(lane_addr + TB_S5B + base + 8u * m, x);
+                    tmem_ld_wait();
 #pragma unroll
-        for (int x = 0; x < 4; ++x) {
-            const int t = 4 * tg + x;
-#pragma unroll
-            for (int y = 0; y < 4; ++y) {
-                const int i = ig + 32 * y;
-                float kv = 0.f, qv = 0.f;
-                if (t < L) {
-                    const size_t idx = ((size_t)(t0 + t) * H + h) * DK + i;
-                    kv = ld_in(a.k, idx, a.in_bf16);
-                    qv = a.scale * ld_in(a.q, idx, a.in_bf16);
+                    for (int e = 0; e < 8; ++e) {
+                        const float w = e3(e) * f2 * x[e];
+                        dk8[e] += w;
+                        dg8[e] -= kv(e) * w;
+                    }
                 }
-                const float g = sG[t * DK + i];
-                const float gam = __expf(g), ec = __expf(sGC[i] - g);
-                dqb[x][y] = gam * aQG[x][y];
-                dkk[x][y] = gam * aKG[x][y] + ec * aKC[x][y];
-                dg[x][y] = qv * gam * aQG[x][y] + kv * gam * aKG[x][y] - kv * ec * aKC[x][y];
-                atomicAdd(&sDgC[i], kv * ec * aKC[x][y]);
-            }
-        }
-        if (tg == 0) {
+                if (q4 == 0) {  // tile 3
+                    tmem_ld8(lane_addr + TB_S5B + SV_B3 + 8u * m, x);
+                    tmem_ld_wait();
 #pragma unroll
-            for (int y = 0; y < 4; ++y) atomicAdd(&sDgC[ig + 32 * y], __expf(sGC[ig + 32 * y]) * rowS[y]);
-        }
-        __syncthreads();
-
-        // ---- P5: the A / P contractions, block row by block row
-        float* sC = sR;  // [3][16][128] contributions of the block's tokens (the quarter buffers are free)
-        for (int bt = 0; bt < nb; ++bt) {
-            build_factors(a, sF, sG, bt, t0, L, h, tid);
+                    for (int e = 0; e < 8; ++e) {
+                        const float w = e3(e) * f3 * x[e];
+                        dk8[e] += w;
+                        dg8[e] -= kv(e) * w;
+                    }
+                }
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const int t = (int)cu + e;
+                    tot += dg8[e];
+                    s_dg[t * 128 + c] = dg8[e];
+                    if (t < L) a.dk[base_c + (size_t)t * rowk] = dk8[e];
+                }
+            }
+            // dlog_alpha: reverse cumulative sum of dg over the chunk plus dL/dg_C
+            s_tot[q4 * 128 + c] = tot;
+            s_dgc[q4 * 128 + c] = dgc;
             __syncthreads();
-            const int r = 16 * bt;
-            {  // tokens t of the block, all threads: dKin_t = sum_s dA_ts Kout_s, dQin_t = sum_s dP_ts Kout_s
-                const int tl = tid >> 5, i4 = (tid & 31) * 4, t = r + tl;
-                if (t < L) {
-                    float dki[4] = {0.f, 0.f, 0.f, 0.f}, dqi[4] = {0.f, 0.f, 0.f, 0.f};
-                    for (int s = 0; s <= t; ++s) {
-                        const float wm = s < t ? sdM[t * LP + s] : 0.f, wp = sdP[t * LP + s];
-                        const float4 ko = *reinterpret_cast<const float4*>(sF + s * FP + i4);
-                        dki[0] += wm * ko.x; dki[1] += wm * ko.y; dki[2] += wm * ko.z; dki[3] += wm * ko.w;
-                        dqi[0] += wp * ko.x; dqi[1] += wp * ko.y; dqi[2] += wp * ko.z; dqi[3] += wp * ko.w;
-                    }
+            float run = 0.f;
 #pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        const int i = i4 + u;
-                        const float e = __expf(sG[t * DK + i] - sG[r * DK + i]);
-                        sC[(0 * 16 + tl) * DK + i] = e * dki[u];
-                        sC[(1 * 16 + tl) * DK + i] = e * dqi[u];
-                        sC[(2 * 16 + tl) * DK + i] = sF[(64 + tl) * FP + i] * dki[u] + sF[(80 + tl) * FP + i] * dqi[u];
-                    }
-                }
+            for (int qq = 0; qq < 4; ++qq) {
+                run += s_dgc[qq * 128 + c] + __expf(G[4]) * s_rs[qq * 128 + c];
+                if (qq > q4) run += s_tot[qq * 128 + c];
             }
-            __syncthreads();
 #pragma unroll
-            for (int x = 0; x < 4; ++x) {
-                const int t = 4 * tg + x;
-                if ((t >> 4) == bt && t < L) {  // owner of a block token: take its contributions
-                    const int tl = t - r;
-#pragma unroll
-                    for (int y = 0; y < 4; ++y) {
-                        const int i = ig + 32 * y;
-                        dkk[x][y] += sC[(0 * 16 + tl) * DK + i];
-                        dqb[x][y] += sC[(1 * 16 + tl) * DK + i];
-                        dg[x][y] += sC[(2 * 16 + tl) * DK + i];
-                    }
-                }
-                if (t < r + 16 && t < L) {  // t as an earlier token s: dKout_t
-#pragma unroll
-                    for (int y = 0; y < 4; ++y) {
-                        const int i = ig + 32 * y;
-                        float dko = 0.f;
-                        for (int tl = (t > r ? t - r : 0); tl < 16; ++tl) {
-                            const int tt = r + tl;
-                            if (tt >= L) break;
-                            if (tt > t) dko += sdM[tt * LP + t] * sF[(64 + tl) * FP + i];
-                            dko += sdP[tt * LP + t] * sF[(80 + tl) * FP + i];
-                        }
-                        const float e = __expf(sG[r * DK + i] - sG[t * DK + i]);
-                        dkk[x][y] += e * dko;
-                        dg[x][y] -= sF[t * FP + i] * dko;
-                    }
-                }
+            for (int u = 15; u >= 0; --u) {
+                const int t = 16 * q4 + u;
+                run += s_dg[t * 128 + c];
+                if (t < L) a.dla[base_c + (size_t)t * rowk] = (keep_la >> u) & 1u ? run : 0.f;
             }
-            __syncthreads();
+            if (tid < CH && tid < L) a.dbeta[(size_t)(t0 + tid) * H + h] = s_db[tid];
         }
-
-        // ---- P6: dq, dk out; dg -> dlog_alpha (reverse cumulative sum over the chunk)
-#pragma unroll
-        for (int x = 0; x < 4; ++x) {
-            const int t = 4 * tg + x;
-            if (t < L) {
-                const size_t base = ((size_t)(t0 + t) * H + h) * DK + ig;
-#pragma unroll
-                for (int y = 0; y < 4; ++y) {
-                    a.dq[base + 32 * y] = a.scale * dqb[x][y];
-                    a.dk[base + 32 * y] = dkk[x][y];
-                }
-            }
-#pragma unroll
-            for (int y = 0; y < 4; ++y) sF[t * FP + ig + 32 * y] = dg[x][y];
-        }
-        __syncthreads();
-        if (tid < DK) {
-            const int i = tid;
-            float lv[CH];
-#pragma unroll
-            for (int t = 0; t < CH; ++t)
-                lv[t] = t < L ? ld_in(a.log_alpha, ((size_t)(t0 + t) * H + h) * DK + i, a.in_bf16) : 0.f;
-            float run = sDgC[i];  // g_C is g of the last token
-#pragma unroll
-            for (int t = CH - 1; t >= 0; --t) {
-                if (t < L) {
-                    run += sF[t * FP + i];
-                    a.dla[((size_t)(t0 + t) * H + h) * DK + i] = lv[t] >= -5.f ? run : 0.f;
-                }
-            }
-        }
-        __syncthreads();  // shared memory is reused by the next item
+        tc_fence_before();
+        __syncthreads();  // shared memory and TMEM are reused by the next item
+        tc_fence_after();
+        par ^= 1u;
+        committed = 0;
+    }
+    if (failed && tid == 0) {
+        // products still in flight complete before the TMEM is released (bounded)
+        for (int i = 0; i < committed; ++i) mbar_wait(&bar[i], par, nullptr);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tm, 512);
     }
 }
 
@@ -723,8 +1090,10 @@ cudaError_t chunk_bwd_launch(const void* q, const void* k, const void* v, const 
     if (!attr) {
         if ((err = cudaFuncSetAttribute(chain_bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)CB_SMEM)) !=
                 cudaSuccess ||
-            (err = cudaFuncSetAttribute(bwd_intra_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)BI_SMEM)) !=
-                cudaSuccess)
+            (err = cudaFuncSetAttribute(bwd_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        (int)BT_SMEM)) != cudaSuccess ||
+            (err = cudaFuncSetAttribute(bwd_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        (int)BT_SMEM)) != cudaSuccess)
             return err;
         int dev = 0;
         if ((err = cudaGetDevice(&dev)) != cudaSuccess) return err;
@@ -767,7 +1136,8 @@ cudaError_t chunk_bwd_launch(const void* q, const void* k, const void* v, const 
     if (nck > 0 && n_items > 0) {
         const unsigned grid = (unsigned)(n_items < sms ? n_items : sms);
         prof_begin(PROF_INTRA_BWD, stream);
-        bwd_intra_kernel<<<grid, BI_THREADS, BI_SMEM, stream>>>(a, n_items);
+        if (in_bf16) bwd_tc_kernel<true><<<grid, BT_THREADS, BT_SMEM, stream>>>(a, n_items);
+        else bwd_tc_kernel<false><<<grid, BT_THREADS, BT_SMEM, stream>>>(a, n_items);
         if ((err = cudaGetLastError()) != cudaSuccess) return err;
         prof_end(PROF_INTRA_BWD, stream);
     }
