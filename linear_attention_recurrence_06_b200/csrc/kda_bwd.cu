@@ -7,7 +7,7 @@
 //   1. the forward walk is recomputed without outputs; it leaves every chunk's
 //      slot (M_lr, Q', Gamma_C) in the workspace and the state at every chunk
 //      boundary in a checkpoint buffer;
-//   2. chain_bwd_kernel walks the chunks of a sequence in reverse with
+//   2. chain_bwd_tc_kernel walks the chunks of a sequence in reverse with
 //      dS = dL/d(state at the end of chunk c):
 //          dS_end[c] = dS,    dS <- Diag(Gamma_C) dS - M_lr^T dS + Q'^T dO_c
 //      starting from dL/dS_final and ending with dL/dS_0;
@@ -85,125 +85,6 @@ KDA_DEV void bwd_seq_range(const BwdArgs& a, int n, int64_t& sb, int64_t& se) {
 KDA_DEV float ld_in(const void* p, size_t idx, int bf16) {
     if (bf16) return __uint_as_float((uint32_t)__ldg(reinterpret_cast<const unsigned short*>(p) + idx) << 16);
     return __ldg(reinterpret_cast<const float*>(p) + idx);
-}
-
-// ------------------------------------------------------------ reverse chain
-constexpr int CB_THREADS = 512;  // thread = (key row i = tid % 128, 8-column group tid / 128)
-constexpr uint32_t CB_SLOT = SO_MQG;                 // M_lr + Q' + Gamma_C of one chunk
-constexpr uint32_t CB_DS = 2 * CB_SLOT;              // dS [128][32] fp32
-constexpr uint32_t CB_DO = CB_DS + DK * DVS * 4;     // dO [64][32] fp32
-constexpr uint32_t CB_BAR = CB_DO + CH * DVS * 4;    // two mbarriers
-constexpr uint32_t CB_SMEM = CB_BAR + 16 + 128;
-
-__global__ void __launch_bounds__(CB_THREADS, 1) chain_bwd_kernel(const BwdArgs a) {
-    extern __shared__ __align__(128) uint8_t sm[];
-    const int js = blockIdx.x, h = blockIdx.y, n = blockIdx.z, H = a.H;
-    const int tid = threadIdx.x, i = tid & (DK - 1), cq = tid >> 7;
-    uint64_t* bar = reinterpret_cast<uint64_t*>(sm + CB_BAR);
-    float* sdS = reinterpret_cast<float*>(sm + CB_DS);
-    float* sdO = reinterpret_cast<float*>(sm + CB_DO);
-    int64_t s_beg, s_end;
-    bwd_seq_range(a, n, s_beg, s_end);
-    const int nck = (int)((s_end - s_beg + CH - 1) / CH);
-    const size_t st = ((size_t)n * H + h) * STATE + (size_t)i * DV + DVS * js + 8 * cq;  // this thread's 8 values
-    float dS[8];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) dS[j] = a.d_final ? a.d_final[st + j] : 0.f;
-    auto slot = [&](int c) { return a.slots + (((size_t)n * a.wc + c) * H + h) * SLOT_BYTES; };
-    if (tid == 0) {
-        mbar_init(&bar[0], 1);
-        mbar_init(&bar[1], 1);
-        fence_mbar_init();
-        for (int r = 0; r < 2 && r < nck; ++r) {
-            mbar_arrive_expect_tx(&bar[r], CB_SLOT);
-            bulk_g2s(sm + r * CB_SLOT, slot(nck - 1 - r), CB_SLOT, &bar[r]);
-        }
-    }
-    __syncthreads();
-    int issued = nck < 2 ? nck : 2, waited = 0;
-    bool failed = false;
-    // this thread's 4 values of a chunk's dO slice: token tid / 8, columns 4 (tid % 8) ..
-    auto load_dO = [&](int c) {
-        const int t = tid >> 3, c4 = (tid & 7) * 4;
-        const int64_t tc = s_beg + (int64_t)c * CH + t;
-        if (c < 0 || tc >= s_end) return make_float4(0.f, 0.f, 0.f, 0.f);
-        const size_t base = ((size_t)tc * H + h) * DV + DVS * js + c4;
-        return make_float4(ld_in(a.d_o, base, a.in_bf16), ld_in(a.d_o, base + 1, a.in_bf16),
-                           ld_in(a.d_o, base + 2, a.in_bf16), ld_in(a.d_o, base + 3, a.in_bf16));
-    };
-    float4 dO_next = load_dO(nck - 1);
-    uint32_t m_off[8];  // sw128_off(mm, i & 63) for mm = 0..7
-#pragma unroll
-    for (int mm = 0; mm < 8; ++mm) m_off[mm] = sw128_off((uint32_t)mm, (uint32_t)(i & 63));
-    for (int r = 0; r < nck; ++r) {
-        const int c = nck - 1 - r, b = r & 1;
-        const int64_t t0 = s_beg + (int64_t)c * CH;
-        const int L = (int)((s_end - t0) < CH ? (s_end - t0) : CH);
-        // dS at the end of chunk c
-        float* dst = a.ds_end + (((size_t)n * a.wc + c) * H + h) * STATE + (size_t)i * DV + DVS * js + 8 * cq;
-        reinterpret_cast<float4*>(dst)[0] = make_float4(dS[0], dS[1], dS[2], dS[3]);
-        reinterpret_cast<float4*>(dst)[1] = make_float4(dS[4], dS[5], dS[6], dS[7]);
-        reinterpret_cast<float4*>(sdS + i * DVS + 8 * cq)[0] = make_float4(dS[0], dS[1], dS[2], dS[3]);
-        reinterpret_cast<float4*>(sdS + i * DVS + 8 * cq)[1] = make_float4(dS[4], dS[5], dS[6], dS[7]);
-        // dO slice of chunk c ([64 tokens][32 columns]), loaded during the previous iteration
-        *reinterpret_cast<float4*>(sdO + (tid >> 3) * DVS + (tid & 7) * 4) = dO_next;
-        const bool ok = mbar_wait(&bar[b], (uint32_t)((r >> 1) & 1), a.status);
-        if (!__syncthreads_and(ok)) {
-            failed = true;
-            break;
-        }
-        waited = r + 1;
-        const uint8_t* buf = sm + b * CB_SLOT;
-        const float gam = *reinterpret_cast<const float*>(buf + SO_G + 4 * i);
-        float acc[8];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) acc[j] = gam * dS[j];
-        // - M_lr^T dS: column i of M_lr against every row of dS.  Element (m, i) of the
-        // K-major SW128 image sits at (i >> 6) * 16384 + sw128_off(m, i & 63); for
-        // m = 8 m8 + mm that is m8 * 1024 + off[mm], with off[] fixed per thread.
-        const uint8_t* mcol = buf + SO_M + (size_t)(i >> 6) * 16384;
-        for (int m8 = 0; m8 < DK / 8; ++m8) {
-            const uint8_t* mrow = mcol + m8 * 1024;
-            const float* drow = sdS + m8 * 8 * DVS + 8 * cq;
-#pragma unroll
-            for (int mm = 0; mm < 8; ++mm) {
-                const uint16_t bits = *reinterpret_cast<const uint16_t*>(mrow + m_off[mm]);
-                const float mv = __uint_as_float((uint32_t)bits << 16);
-                const float4 d0 = reinterpret_cast<const float4*>(drow + mm * DVS)[0];
-                const float4 d1 = reinterpret_cast<const float4*>(drow + mm * DVS)[1];
-                acc[0] -= mv * d0.x; acc[1] -= mv * d0.y; acc[2] -= mv * d0.z; acc[3] -= mv * d0.w;
-                acc[4] -= mv * d1.x; acc[5] -= mv * d1.y; acc[6] -= mv * d1.z; acc[7] -= mv * d1.w;
-            }
-        }
-        // + Q'^T dO: column i of Q' against every token row of dO
-        const uint8_t* qcol = buf + SO_Q + (size_t)(i >> 3) * 1024 + (i & 7) * 16;
-        for (int t = 0; t < L; ++t) {
-            const uint16_t bits = *reinterpret_cast<const uint16_t*>(qcol + (t >> 3) * 128 + (t & 7) * 2);
-            const float qv = __uint_as_float((uint32_t)bits << 16);
-            const float4 o0 = reinterpret_cast<const float4*>(sdO + t * DVS + 8 * cq)[0];
-            const float4 o1 = reinterpret_cast<const float4*>(sdO + t * DVS + 8 * cq)[1];
-            acc[0] += qv * o0.x; acc[1] += qv * o0.y; acc[2] += qv * o0.z; acc[3] += qv * o0.w;
-            acc[4] += qv * o1.x; acc[5] += qv * o1.y; acc[6] += qv * o1.z; acc[7] += qv * o1.w;
-        }
-        dO_next = load_dO(c - 1);
-        __syncthreads();  // buffer b, dS and dO are no longer read
-        if (tid == 0 && r + 2 < nck) {
-            mbar_arrive_expect_tx(&bar[b], CB_SLOT);
-            bulk_g2s(sm + b * CB_SLOT, slot(nck - 1 - (r + 2)), CB_SLOT, &bar[b]);
-            issued = r + 3;
-        }
-#pragma unroll
-        for (int j = 0; j < 8; ++j) dS[j] = acc[j];
-    }
-    if (failed && tid == 0) {
-        // copies still in flight land before the CTA retires (bounded)
-        for (int r = waited; r < issued; ++r) mbar_wait(&bar[r & 1], (uint32_t)((r >> 1) & 1), nullptr);
-    }
-    if (!failed && a.d_init) {
-        float* dst = a.d_init + st;
-        reinterpret_cast<float4*>(dst)[0] = make_float4(dS[0], dS[1], dS[2], dS[3]);
-        reinterpret_cast<float4*>(dst)[1] = make_float4(dS[4], dS[5], dS[6], dS[7]);
-    }
 }
 
 constexpr int BT_THREADS = 512;  // threads of the chunk-local kernel
@@ -1071,6 +952,270 @@ __global__ void __launch_bounds__(BT_THREADS, 1) bwd_tc_kernel(const BwdArgs a, 
     }
 }
 
+// ------------------------------------------------ reverse chain (tensor cores)
+// One CTA per (sequence, head, 32-column slice js of dS), warp-specialised like the
+// forward chain: warps 0-3 own one row i of the dS slice each (32 fp32 registers),
+// warp 4 (one thread) issues the tensor-core products, warp 5 (one thread) bulk-loads
+// each chunk's M_lr, Q' and Gamma_C from the forward's workspace slot, three chunks ahead.
+// Per chunk c, in reverse:
+//     dS_end[c] = dS;   dS <- Gamma_C o dS + D,   D = Q'^T dO_c - M_lr^T dS
+// D (M = 128 rows i, N = 32 columns) accumulates in TMEM: Q'^T dO_c first (it does not
+// depend on dS, so it is issued one chunk ahead, off the sequential path), then M_lr^T
+// (-dS) on top.  M_lr^T is the slot's K-major 128-byte-swizzle M_lr image read as an
+// MN-major operand; Q'^T is the slot's token-contiguous Q' image read as a K-major one.
+// dO_c enters as a bf16 image [32 j][64 t] written by the consumers from registers
+// loaded one chunk ahead; -dS as a bf16 image [128 m][32 j].
+constexpr int RB_THREADS = 192;
+constexpr int RB_NBUF = 3;
+constexpr uint32_t RB_SLOT = 50176;                    // M_lr + Q' + Gamma_C (49,664 B), 1024-aligned stride
+constexpr uint32_t RB_DS = RB_NBUF * RB_SLOT;          // -dS image [128 m][32 j] bf16
+constexpr uint32_t RB_DO = RB_DS + 8192;               // dO images [2][32 j][64 t] bf16
+constexpr uint32_t RB_BAR = RB_DO + 8192;
+constexpr uint32_t RB_TPTR = RB_BAR + 128;
+constexpr uint32_t RB_SMEM = RB_TPTR + 16 + 1024;
+static_assert(RB_SLOT >= SO_MQG && RB_SLOT % 1024 == 0, "slot buffer stride");
+
+// M_lr^T from the K-major 128-byte-swizzle M_lr image: MN-major operand, 64-element MN
+// blocks 16,384 B apart, 8-row K groups 1,024 B apart
+KDA_DEV uint64_t sdesc_mn_sw128(uint32_t addr) {
+    uint64_t d = 0;
+    d |= (uint64_t)((addr >> 4) & 0x3FFFu);
+    d |= (uint64_t)(16384u >> 4) << 16;
+    d |= (uint64_t)(1024u >> 4) << 32;
+    d |= (uint64_t)1u << 46;
+    d |= (uint64_t)2u << 61;
+    return d;
+}
+// element (t, j) of a dO image: 8-column blocks 1,024 B apart, token rows 16 B apart
+KDA_DEV uint32_t do_off(uint32_t t, uint32_t j) { return (j >> 3) * 1024u + t * 16u + (j & 7u) * 2u; }
+
+template <bool IN_BF16>
+__global__ void __launch_bounds__(RB_THREADS, 1) chain_bwd_tc_kernel(const BwdArgs a) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    const uint32_t sbase = smem_u32(sm);
+    const int js = blockIdx.x, h = blockIdx.y, n = blockIdx.z, H = a.H;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const bool consumer = warp < 4;
+    uint64_t* bar_ld = reinterpret_cast<uint64_t*>(sm + RB_BAR);          // [3]
+    uint64_t* bar_free = reinterpret_cast<uint64_t*>(sm + RB_BAR + 24);   // [3]
+    uint64_t* bar_img = reinterpret_cast<uint64_t*>(sm + RB_BAR + 48);
+    uint64_t* bar_d = reinterpret_cast<uint64_t*>(sm + RB_BAR + 56);      // [2]
+    uint32_t* s_tmem = reinterpret_cast<uint32_t*>(sm + RB_TPTR);
+    int64_t s_beg, s_end;
+    bwd_seq_range(a, n, s_beg, s_end);
+    const int nck = (int)((s_end - s_beg + CH - 1) / CH);
+    // this consumer's row i = tid, columns [32 js, 32 js + 32)
+    const size_t st = ((size_t)n * H + h) * STATE + (size_t)(consumer ? tid : 0) * DV + (size_t)DVS * js;
+    float dS[DVS];
+    if (consumer) {
+#pragma unroll
+        for (int j = 0; j < DVS; j += 4) {
+            float4 v4 = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (a.d_final) v4 = *reinterpret_cast<const float4*>(a.d_final + st + j);
+            dS[j] = v4.x; dS[j + 1] = v4.y; dS[j + 2] = v4.z; dS[j + 3] = v4.w;
+        }
+    }
+    if (nck > 0) {
+        if (warp == 0) {
+            tmem_alloc(s_tmem, 64);
+            tmem_relinquish();
+        }
+        if (tid == 0) {
+            for (int i = 0; i < RB_NBUF; ++i) {
+                mbar_init(&bar_ld[i], 1);
+                mbar_init(&bar_free[i], 128);
+            }
+            mbar_init(bar_img, 128);
+            mbar_init(&bar_d[0], 1);
+            mbar_init(&bar_d[1], 1);
+            fence_mbar_init();
+        }
+        __syncthreads();
+        tc_fence_after();
+        const uint32_t tm = *s_tmem;
+        // iteration it handles chunk c = nck - 1 - it
+        auto slot_of = [&](int it) {
+            return a.slots + (((size_t)n * a.wc + (nck - 1 - it)) * H + h) * SLOT_BYTES;
+        };
+        auto bidx = [](int it) { return it % RB_NBUF; };
+        auto bpar = [](int it) { return (uint32_t)((it / RB_NBUF) & 1); };
+        bool failed = false;
+        int loads_issued = 0, mma_issued = 0;
+
+        if (warp == 5) {
+            // ------------------------------------------------------------ loader
+            if (lane == 0) {
+                auto issue_load = [&](int it) {
+                    const int b = bidx(it);
+                    mbar_arrive_expect_tx(&bar_ld[b], SO_MQG);
+                    bulk_g2s(sm + b * RB_SLOT, slot_of(it) + SO_M, SO_MQG, &bar_ld[b]);
+                };
+                for (int j = 0; j < RB_NBUF && j < nck; ++j) {
+                    issue_load(j);
+                    loads_issued = j + 1;
+                }
+                for (int j = 0; j + RB_NBUF < nck; ++j) {
+                    if (!mbar_wait(&bar_free[bidx(j)], bpar(j), a.status)) {
+                        failed = true;
+                        break;
+                    }
+                    issue_load(j + RB_NBUF);
+                    loads_issued = j + RB_NBUF + 1;
+                }
+            }
+        } else if (warp == 4) {
+            // ------------------------------------------------------ tensor issue
+            if (lane == 0) {
+                const uint32_t id1 = idesc_bf16_major(128, DVS, 1, 1), id2 = idesc_bf16_major(128, DVS, 0, 1);
+                // Q'^T dO of iteration it into accumulator it & 1 (overwrites)
+                auto issue_qdo = [&](int it) {
+                    const uint32_t buf = sbase + bidx(it) * RB_SLOT;
+                    const uint64_t ad = sdesc_interleave(buf + SO_Q, 128u, 1024u);
+                    const uint64_t bd = sdesc_interleave(sbase + RB_DO + (it & 1) * 4096, 128u, 1024u);
+#pragma unroll
+                    for (int kk = 0; kk < CH / 16; ++kk)
+                        mma_bf16(tm + 32 * (it & 1), ad + (uint32_t)((kk * 256) >> 4), bd + (uint32_t)((kk * 256) >> 4), id2,
+                                 kk > 0 ? 1u : 0u);
+                };
+                // the first chunk's dO image (announced on bar_img's phase 0) and slot
+                if (!mbar_wait(bar_img, 0u, a.status) || !mbar_wait(&bar_ld[bidx(0)], bpar(0), a.status)) {
+                    failed = true;
+                } else {
+                    tc_fence_after();
+                    issue_qdo(0);
+                    for (int it = 0; it < nck; ++it) {
+                        // the -dS image of this chunk (and the dO image of the next one)
+                        if (!mbar_wait(bar_img, (uint32_t)((it + 1) & 1), a.status)) {
+                            failed = true;
+                            break;
+                        }
+                        tc_fence_after();
+                        const uint64_t md = sdesc_mn_sw128(sbase + bidx(it) * RB_SLOT + SO_M);
+                        const uint64_t sd = sdesc_interleave(sbase + RB_DS, 512u, 128u);
+#pragma unroll
+                        for (int kk = 0; kk < DK / 16; ++kk)
+                            mma_bf16(tm + 32 * (it & 1), md + (uint32_t)((kk * 2048) >> 4),
+                                     sd + (uint32_t)((kk * 1024) >> 4), id1, 1u);
+                        mma_commit(&bar_d[it & 1]);
+                        mma_issued = it + 1;
+                        if (it + 1 < nck) {
+                            if (!mbar_wait(&bar_ld[bidx(it + 1)], bpar(it + 1), a.status)) {
+                                failed = true;
+                                break;
+                            }
+                            tc_fence_after();
+                            issue_qdo(it + 1);
+                        }
+                    }
+                }
+            }
+        } else {
+            // --------------------------------------------------------- consumers
+            const int i = tid;
+            const uint32_t lane_addr = tm + ((uint32_t)(32 * warp) << 16);
+            // dO of iteration it: token t = i / 2, 16 columns from 16 (i % 2), bf16 bits in registers
+            uint32_t dw[8];
+            auto load_do = [&](int it) {
+#pragma unroll
+                for (int e = 0; e < 8; ++e) dw[e] = 0u;
+                if (it >= nck) return;
+                const int c = nck - 1 - it;
+                const int t = i >> 1;
+                const int64_t tok = s_beg + (int64_t)c * CH + t;
+                if (tok >= s_end) return;
+                const size_t base = ((size_t)tok * H + h) * DV + (size_t)DVS * js + 16 * (i & 1);
+                if constexpr (IN_BF16) {
+                    const uint4 u0 = __ldg(reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(a.d_o) + base));
+                    const uint4 u1 = __ldg(reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(a.d_o) + base + 8));
+                    dw[0] = u0.x; dw[1] = u0.y; dw[2] = u0.z; dw[3] = u0.w;
+                    dw[4] = u1.x; dw[5] = u1.y; dw[6] = u1.z; dw[7] = u1.w;
+                } else {
+                    const float* src = reinterpret_cast<const float*>(a.d_o) + base;
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float4 f = __ldg(reinterpret_cast<const float4*>(src) + e);
+                        dw[2 * e] = pack_bf16x2(f.x, f.y);
+                        dw[2 * e + 1] = pack_bf16x2(f.z, f.w);
+                    }
+                }
+            };
+            auto write_do = [&](int it) {
+                uint8_t* img = sm + RB_DO + (it & 1) * 4096;
+                const int t = i >> 1, jb = 2 * (i & 1);
+                *reinterpret_cast<uint4*>(img + do_off((uint32_t)t, 8u * jb)) = make_uint4(dw[0], dw[1], dw[2], dw[3]);
+                *reinterpret_cast<uint4*>(img + do_off((uint32_t)t, 8u * (jb + 1))) = make_uint4(dw[4], dw[5], dw[6], dw[7]);
+            };
+            load_do(0);
+            write_do(0);
+            load_do(1);
+            fence_async_smem();
+            tc_fence_before();
+            mbar_arrive(bar_img);
+            for (int it = 0; it < nck; ++it) {
+                const int c = nck - 1 - it, b = bidx(it);
+                // dL/d(state at the end of chunk c)
+                float* dst = a.ds_end + (((size_t)n * a.wc + c) * H + h) * STATE + (size_t)i * DV + (size_t)DVS * js;
+#pragma unroll
+                for (int j = 0; j < DVS; j += 4)
+                    *reinterpret_cast<float4*>(dst + j) = make_float4(dS[j], dS[j + 1], dS[j + 2], dS[j + 3]);
+                // -dS image (row m = i) and the next chunk's dO image
+                {
+                    uint8_t* img = sm + RB_DS + (uint32_t)(i >> 3) * 512u + (uint32_t)(i & 7) * 16u;
+                    float ng[8];
+#pragma unroll
+                    for (int jb = 0; jb < DVS / 8; ++jb) {
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) ng[e] = -dS[8 * jb + e];
+                        *reinterpret_cast<uint4*>(img + jb * 128) = pack8f(ng);
+                    }
+                }
+                if (it + 1 < nck) {
+                    write_do(it + 1);
+                    load_do(it + 2);
+                }
+                fence_async_smem();
+                tc_fence_before();
+                mbar_arrive(bar_img);
+                if (!mbar_wait(&bar_d[it & 1], (uint32_t)((it >> 1) & 1), a.status) ||
+                    !mbar_wait(&bar_ld[b], bpar(it), a.status)) {
+                    failed = true;
+                    break;
+                }
+                tc_fence_after();
+                float d[DVS];
+                tmem_ld32(lane_addr + 32 * (it & 1), d);
+                tmem_ld_wait();
+                const float gam = *reinterpret_cast<const float*>(sm + b * RB_SLOT + SO_G + 4 * i);
+#pragma unroll
+                for (int j = 0; j < DVS; ++j) dS[j] = gam * dS[j] + d[j];
+                tc_fence_before();
+                mbar_arrive(&bar_free[b]);
+            }
+        }
+        // copies and products in flight finish before the CTA retires (bounded)
+        __syncthreads();
+        if (warp == 5 && lane == 0) {
+            for (int j = loads_issued - RB_NBUF < 0 ? 0 : loads_issued - RB_NBUF; j < loads_issued; ++j)
+                mbar_wait(&bar_ld[bidx(j)], bpar(j), nullptr);
+        }
+        if (warp == 4 && lane == 0 && failed && mma_issued > 0) {
+            const int j = mma_issued - 1;
+            mbar_wait(&bar_d[j & 1], (uint32_t)((j >> 1) & 1), nullptr);
+        }
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+        if (warp == 0) tmem_dealloc(tm, 64);
+        if (failed) return;
+    }
+    if (consumer && a.d_init) {
+#pragma unroll
+        for (int j = 0; j < DVS; j += 4)
+            *reinterpret_cast<float4*>(a.d_init + st + j) = make_float4(dS[j], dS[j + 1], dS[j + 2], dS[j + 3]);
+    }
+}
+
 }  // namespace
 
 size_t chunk_bwd_extra_bytes(int n_seqs, int H, int64_t max_seqlen) {
@@ -1088,8 +1233,10 @@ cudaError_t chunk_bwd_launch(const void* q, const void* k, const void* v, const 
     static int sms = 0;
     cudaError_t err;
     if (!attr) {
-        if ((err = cudaFuncSetAttribute(chain_bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)CB_SMEM)) !=
-                cudaSuccess ||
+        if ((err = cudaFuncSetAttribute(chain_bwd_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        (int)RB_SMEM)) != cudaSuccess ||
+            (err = cudaFuncSetAttribute(chain_bwd_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        (int)RB_SMEM)) != cudaSuccess ||
             (err = cudaFuncSetAttribute(bwd_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                         (int)BT_SMEM)) != cudaSuccess ||
             (err = cudaFuncSetAttribute(bwd_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -1128,7 +1275,8 @@ cudaError_t chunk_bwd_launch(const void* q, const void* k, const void* v, const 
     a.in_bf16 = in_bf16 ? 1 : 0;
     // 2. the reverse walk: dL/d(state) at every chunk end, dL/dS_0
     prof_begin(PROF_CHAIN_BWD, stream);
-    chain_bwd_kernel<<<dim3(NSL, H, N), CB_THREADS, CB_SMEM, stream>>>(a);
+    if (in_bf16) chain_bwd_tc_kernel<true><<<dim3(NSL, H, N), RB_THREADS, RB_SMEM, stream>>>(a);
+    else chain_bwd_tc_kernel<false><<<dim3(NSL, H, N), RB_THREADS, RB_SMEM, stream>>>(a);
     if ((err = cudaGetLastError()) != cudaSuccess) return err;
     prof_end(PROF_CHAIN_BWD, stream);
     // 3. the chunk-local gradients
