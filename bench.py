@@ -515,9 +515,13 @@ KCP_SHAPE = dict(T_rank=8192, H=32, ranks=8)
 # chain per chunk step and head: M_lr^T dS 128x128x128 and Q'^T dO 128x64x128.
 BWD_INTRA_FLOP_PER_ITEM = 2 * (524288 + 43690 + 1048576 + 3 * 266240 + 1048576 + 524288 + 3 * 1048576 + 2 * 524288)
 BWD_CHAIN_FLOP_PER_ITEM = 2 * (128 * 128 * 128 + 128 * 64 * 128)
-# fp32 FMA peak of the CUDA cores: 148 SMs x 128 lanes x 2 FLOP x 1.965 GHz (unit counts and
-# the maximum SM clock; no measured figure exists for this unit)
-FP32_FMA_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+# Tensor-core work the backward kernels issue per (chunk, head) (dense tiles, 2 FLOP per
+# multiply-add): the chunk-local kernel's 12 products (stage 1: 128x160x128 + 2 x 128x64x128;
+# stage 2: 2 x 128x64x64; stage 3: 128x64x64 + 128x64x128; stage 4: 128x64x128 + 128x128x128;
+# stage 5, high and low parts: 2 x 128x128x160 + 2 x 128x160x128); the reverse chain's
+# M_lr^T dS and Q'^T dO (as counted above).
+BWD_INTRA_ISSUED_FLOP_PER_ITEM = 2 * (128 * 160 * 128 + 2 * 128 * 64 * 128 + 2 * 128 * 64 * 64 + 128 * 64 * 64
+                                      + 128 * 64 * 128 + 128 * 64 * 128 + 128 * 128 * 128 + 4 * 128 * 128 * 160)
 
 
 def run_backward(args, torch, kda, dev, stream, max_over_ranks, barrier):
@@ -562,17 +566,21 @@ def run_backward(args, torch, kda, dev, stream, max_over_ranks, barrier):
     prof = kda.profile_read()
     kda.profile_enable(False)
     kernels = {k: dict(launches_per_call=v[0] / n, ms_per_call=v[1] / n) for k, v in prof.items()}
-    # the two backward kernels run fp32 FMA on the CUDA cores: roofline against that ALU peak
+    # both backward kernels run their products on the tensor cores: roofline against the bf16
+    # tensor peak (the sustained figure: the kernels run inside a loop of calls)
+    peaks = load_peaks()
     items = B * (T // 64) * H
-    alu = {}
-    for name, flop in (("intra_bwd", BWD_INTRA_FLOP_PER_ITEM), ("chain_bwd", BWD_CHAIN_FLOP_PER_ITEM)):
+    roof = {}
+    for name, flop, issued in (("intra_bwd", BWD_INTRA_FLOP_PER_ITEM, BWD_INTRA_ISSUED_FLOP_PER_ITEM),
+                               ("chain_bwd", BWD_CHAIN_FLOP_PER_ITEM, BWD_CHAIN_FLOP_PER_ITEM)):
         if name in kernels and kernels[name]["ms_per_call"] > 0:
             tf = flop * items / (kernels[name]["ms_per_call"] * 1e-3) / 1e12
-            alu[name] = dict(bound="alu", achieved=tf, peak=FP32_FMA_TFLOPS, unit="TFLOP/s",
-                             frac=tf / FP32_FMA_TFLOPS, flop_per_launch=flop * items)
+            roof[name] = dict(bound="tensor", achieved=tf, peak=peaks["bf16_tflops_sustained"], unit="TFLOP/s",
+                              frac=tf / peaks["bf16_tflops_sustained"], flop_per_launch=flop * items,
+                              issued_flop_per_launch=issued * items, peak_source=peaks["source"])
     return {"workload": f"KDA backward B={B} T={T} H={H} bf16 inputs and dL/do, fp32 gradients, initial state "
                         "and final-state gradient", "ms_per_call": ms, "tokens_per_s": B * T / (ms * 1e-3),
-            "kernels": kernels, "roofline": alu}
+            "kernels": kernels, "roofline": roof}
 
 
 def run_kcp(args, torch, kda, dev, stream, max_over_ranks, barrier):

@@ -157,6 +157,142 @@ decode_step_kernel(float* __restrict__ state, const void* __restrict__ q, const 
     }
 }
 
+// Ungated steps, one or several per call: the head's columns are split over two CTAs of
+// 128 threads (the columns evolve independently given the token's k, q, alpha, beta),
+// so twice as many, half-size CTAs are in flight per SM and the loads, steps and stores
+// of different CTAs overlap when a call runs several steps.  Warp w of slice sl owns
+// columns [64 sl + 16 w, +16); lane l: row block rb = l / 8 (rows 32 rb .. 32 rb + 31,
+// contiguous) and column pair cp = l % 8 (columns 2 cp, 2 cp + 1 of the warp's 16): a
+// thread holds 32 rows x 2 columns (64 fp32 registers), reads the rows' decay, k and q
+// four at a time (16-byte shared loads), and the column sums need one 4-lane reduction.
+// Per step and column: S' = alpha o S;  u = beta (v - S'^T k);  o = scale (S'^T q + (k.q) u);
+// S = S' + k u^T, the same arithmetic whatever the number of steps per call.
+template <bool IN_BF16, bool OUT_BF16>
+__global__ void __launch_bounds__(128, 4)
+decode_multi_kernel(float* __restrict__ state, const void* __restrict__ q, const void* __restrict__ k,
+                    const void* __restrict__ v, const void* __restrict__ log_alpha, const void* __restrict__ beta,
+                    void* __restrict__ o, float scale, int n_steps, float* __restrict__ step_states) {
+    constexpr int D = 128;
+    const int bh = blockIdx.x >> 1, sl = blockIdx.x & 1;  // (sequence * H + head, column half)
+    const size_t BH = gridDim.x >> 1;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int rb = lane >> 3, cp = lane & 7;
+    const int col = 64 * sl + 16 * warp + 2 * cp;
+    const int row0 = 32 * rb;
+    // per-row token values, rows of block rb at offset 36 rb (4 floats of padding per block):
+    // the four row blocks a warp reads at once fall into different banks
+    constexpr int DP = D + 12;
+    __shared__ __align__(16) float s_k[2][DP], s_q[2][DP], s_alpha[2][DP];
+    const int pr = tid + 4 * (tid >> 5);   // padded slot of row tid
+    const int prow0 = row0 + 4 * rb;       // padded slot of this thread's first row
+
+    float* S = state + (size_t)bh * D * D;
+    float2 st[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) st[i] = __ldcs(reinterpret_cast<const float2*>(S + (size_t)(row0 + i) * D + col));
+
+    // this step's token values, loaded one step ahead into registers
+    float nk, nq, nla, nb, nv[2];
+    auto load_step = [&](int t) {
+        const size_t tb = (size_t)t * BH + bh;
+        const size_t idx = tb * D + tid;
+        nk = ld_in<IN_BF16>(k, idx);
+        nq = ld_in<IN_BF16>(q, idx);
+        nla = ld_in<IN_BF16>(log_alpha, idx);
+        nb = ld_in<IN_BF16>(beta, tb);
+        nv[0] = ld_in<IN_BF16>(v, tb * D + col);
+        nv[1] = ld_in<IN_BF16>(v, tb * D + col + 1);
+    };
+    load_step(0);
+
+    for (int t = 0; t < n_steps; ++t) {
+        const int pb = t & 1;
+        const size_t tb = (size_t)t * BH + bh;
+        s_k[pb][pr] = nk;
+        s_q[pb][pr] = nq;
+        s_alpha[pb][pr] = __expf(fmaxf(nla, LOG_ALPHA_FLOOR));
+        const float b = nb, v0 = nv[0], v1 = nv[1];
+        if (t + 1 < n_steps) load_step(t + 1);  // in flight during this step
+        __syncthreads();
+        const float* sk_ = s_k[pb];
+        const float* sq_ = s_q[pb];
+        const float* sa_ = s_alpha[pb];
+
+        float kq = 0.f;
+#pragma unroll
+        for (int m = 0; m < 4; ++m) kq += sk_[lane + 36 * m] * sq_[lane + 36 * m];
+#pragma unroll
+        for (int m = 16; m >= 1; m >>= 1) kq += __shfl_xor_sync(0xffffffffu, kq, m);
+
+        // decay the rows, partial S'^T k and S'^T q over this thread's 32 rows; the two
+        // columns of a row go through the paired fp32 instructions (each half rounds as
+        // the scalar one would)
+        // (two partial sums per dot product: even and odd row groups, half the dependent chain)
+        float2 skv = make_float2(0.f, 0.f), sqv = make_float2(0.f, 0.f);
+        float2 skw = make_float2(0.f, 0.f), sqw = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int i4 = 0; i4 < 8; ++i4) {
+            const float4 a4 = *reinterpret_cast<const float4*>(sa_ + prow0 + 4 * i4);
+            const float4 k4 = *reinterpret_cast<const float4*>(sk_ + prow0 + 4 * i4);
+            const float4 q4 = *reinterpret_cast<const float4*>(sq_ + prow0 + 4 * i4);
+            const float av[4] = {a4.x, a4.y, a4.z, a4.w}, kv[4] = {k4.x, k4.y, k4.z, k4.w},
+                        qv[4] = {q4.x, q4.y, q4.z, q4.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                float2& x = st[4 * i4 + e];
+                x = __fmul2_rn(x, make_float2(av[e], av[e]));
+                if (e & 1) {
+                    skw = __ffma2_rn(x, make_float2(kv[e], kv[e]), skw);
+                    sqw = __ffma2_rn(x, make_float2(qv[e], qv[e]), sqw);
+                } else {
+                    skv = __ffma2_rn(x, make_float2(kv[e], kv[e]), skv);
+                    sqv = __ffma2_rn(x, make_float2(qv[e], qv[e]), sqv);
+                }
+            }
+        }
+        float sk0 = skv.x + skw.x, sk1 = skv.y + skw.y, sq0 = sqv.x + sqw.x, sq1 = sqv.y + sqw.y;
+        // reduce over the 4 row blocks (lanes that share cp)
+#pragma unroll
+        for (int m = 8; m <= 16; m <<= 1) {
+            sk0 += __shfl_xor_sync(0xffffffffu, sk0, m);
+            sk1 += __shfl_xor_sync(0xffffffffu, sk1, m);
+            sq0 += __shfl_xor_sync(0xffffffffu, sq0, m);
+            sq1 += __shfl_xor_sync(0xffffffffu, sq1, m);
+        }
+        const float u0 = b * (v0 - sk0), u1 = b * (v1 - sk1);
+        const float o0 = scale * (sq0 + kq * u0), o1 = scale * (sq1 + kq * u1);
+        const float2 u2 = make_float2(u0, u1);
+        // S = S' + k u^T; this step's state when the caller keeps them, and the carried
+        // state written back once, at the last step
+        float* SS = step_states ? step_states + tb * D * D : nullptr;
+        const bool last = t + 1 == n_steps;
+#pragma unroll
+        for (int i4 = 0; i4 < 8; ++i4) {
+            const float4 k4 = *reinterpret_cast<const float4*>(sk_ + prow0 + 4 * i4);
+            const float kv[4] = {k4.x, k4.y, k4.z, k4.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) st[4 * i4 + e] = __ffma2_rn(make_float2(kv[e], kv[e]), u2, st[4 * i4 + e]);
+        }
+        if (SS || last) {
+            float* dst = (SS ? SS : S) + (size_t)row0 * D + col;
+#pragma unroll
+            for (int i = 0; i < 32; ++i) __stcs(reinterpret_cast<float2*>(dst + (size_t)i * D), st[i]);
+            if (SS && last) {
+#pragma unroll
+                for (int i = 0; i < 32; ++i)
+                    __stcs(reinterpret_cast<float2*>(S + (size_t)(row0 + i) * D + col), st[i]);
+            }
+        }
+        if (rb == 0) {
+            if constexpr (OUT_BF16) {
+                *reinterpret_cast<uint32_t*>(reinterpret_cast<uint16_t*>(o) + tb * D + col) = pack_bf16x2(o0, o1);
+            } else {
+                *reinterpret_cast<float2*>(reinterpret_cast<float*>(o) + tb * D + col) = make_float2(o0, o1);
+            }
+        }
+    }
+}
+
 // y = o / sqrt(mean(o^2) + eps) * w * sigmoid(g) over rows of dv = 128.
 // Half a warp per row (8 consecutive channels = 16 bytes of bf16 per lane),
 // two rows per warp, grid-stride over row pairs (warp-uniform trip count).  In place (y == o) is safe:
@@ -232,20 +368,33 @@ cudaError_t launch_decode_step(float* state, const void* q, const void* k, const
                                bool in_bf16, bool out_bf16, float scale, const void* gate,
                                const float* norm_w, float eps, int n_steps, float* step_states,
                                cudaStream_t stream) {
-    const dim3 grid((unsigned)((int64_t)Bd * H)), block(256);
-#define KDA_DEC(IB, OB, G)                                                                              \
-    decode_step_kernel<IB, OB, G><<<grid, block, 0, stream>>>(state, q, k, v, log_alpha, beta, o, gate, \
-                                                              norm_w, scale, eps, n_steps, step_states)
     const bool g = gate != nullptr;
-    if (in_bf16) {
-        if (out_bf16) { if (g) KDA_DEC(true, true, true); else KDA_DEC(true, true, false); }
-        else          { if (g) KDA_DEC(true, false, true); else KDA_DEC(true, false, false); }
-    } else {
-        if (out_bf16) { if (g) KDA_DEC(false, true, true); else KDA_DEC(false, true, false); }
-        else          { if (g) KDA_DEC(false, false, true); else KDA_DEC(false, false, false); }
-    }
+    if (g && n_steps == 1) {  // one step with the gate fused: one CTA per (sequence, head)
+        const dim3 grid((unsigned)((int64_t)Bd * H)), block(256);
+#define KDA_DEC(IB, OB)                                                                                    \
+    decode_step_kernel<IB, OB, true><<<grid, block, 0, stream>>>(state, q, k, v, log_alpha, beta, o, gate, \
+                                                                 norm_w, scale, eps, n_steps, step_states)
+        if (in_bf16) { if (out_bf16) KDA_DEC(true, true); else KDA_DEC(true, false); }
+        else         { if (out_bf16) KDA_DEC(false, true); else KDA_DEC(false, false); }
 #undef KDA_DEC
-    return cudaGetLastError();
+        return cudaGetLastError();
+    }
+    // two half-head CTAs per (sequence, head); with a gate, the per-head RMSNorm and gate
+    // then run over the n_steps output rows in place
+    const dim3 grid((unsigned)((int64_t)Bd * H * 2)), block(128);
+#define KDA_DECM(IB, OB)                                                                               \
+    decode_multi_kernel<IB, OB><<<grid, block, 0, stream>>>(state, q, k, v, log_alpha, beta, o, scale, \
+                                                            n_steps, step_states)
+    if (in_bf16) { if (out_bf16) KDA_DECM(true, true); else KDA_DECM(true, false); }
+    else         { if (out_bf16) KDA_DECM(false, true); else KDA_DECM(false, false); }
+#undef KDA_DECM
+    cudaError_t err = cudaGetLastError();
+    if (err != cudaSuccess || !g) return err;
+    int dev = 0, sms = 0;
+    if ((err = cudaGetDevice(&dev)) != cudaSuccess) return err;
+    if ((err = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return err;
+    return launch_gate_norm(o, gate, norm_w, eps, o, (int64_t)n_steps * Bd * H, out_bf16, in_bf16, out_bf16, sms,
+                            stream);
 }
 
 cudaError_t launch_gate_norm(const void* o, const void* g, const float* norm_w, float eps, void* y,
