@@ -289,8 +289,9 @@ KDA_API kda_status kda_chunk_bwd(const void* q, const void* k, const void* v, co
 
 /*
  * kda_chunk_bwd_workspace_size -- workspace bytes of kda_chunk_bwd: the
- * forward's whole-sequence workspace plus one fp32 state per chunk boundary and
- * per chunk (arguments as kda_chunk_fwd_workspace_size).
+ * forward's whole-sequence workspace plus, per chunk and head, the state at the
+ * chunk's start and the state gradient at its end, each kept as a bf16 128 x 128
+ * operand image (arguments as kda_chunk_fwd_workspace_size).
  */
 KDA_API kda_status kda_chunk_bwd_workspace_size(int64_t T, int H, int dk, int dv, int n_seqs, int64_t max_seqlen,
                                                 size_t* bytes);

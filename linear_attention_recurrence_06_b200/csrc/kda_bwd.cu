@@ -31,6 +31,8 @@
 // just before tile b): e^{g_t - g_s} = e^{g_t - G_b} e^{G_b - g_s}, so no operand
 // overflows.  Products run on the tensor cores with bf16 operands and fp32
 // accumulators; M^-1, the exponentials and the gradient assembly are fp32.
+#include <string.h>
+
 #include "kda_launch.h"
 #include "kda_profile.h"
 #include "kda_slots.h"
@@ -56,8 +58,8 @@ struct BwdArgs {
     float* dbeta;
     const int32_t* cu;         // nullable (fixed length)
     const uint8_t* slots;      // forward chunk slots [n_seqs][wc][H]
-    const float* ckpt;         // states after every whole chunk [n_seqs][n_ckpt][H][dk][dv]
-    float* ds_end;             // dL/d(state at chunk end) [n_seqs][wc][H][dk][dv]
+    const uint8_t* ckpt;       // states after every whole chunk, bf16 images [n_seqs][n_ckpt][H]
+    uint8_t* ds_end;           // dL/d(state at chunk end), bf16 images [n_seqs][wc][H]
     uint32_t* status;
     int64_t T;
     int H, n_seqs, wc, n_ckpt;
@@ -111,13 +113,15 @@ KDA_DEV void prefetch_item(const BwdArgs& a, int64_t item, int64_t n_items, int 
         const char* p = reinterpret_cast<const char*>(tens[tsr]) + ((size_t)(t0 + t) * H + h) * row + ln * 128;
         asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
     }
-    const float* S0 = c == 0 ? (a.init_state ? a.init_state + ((size_t)n * H + h) * STATE : nullptr)
-                             : a.ckpt + (((size_t)n * a.n_ckpt + (c - 1)) * H + h) * STATE;
-    const float* dSC = a.ds_end + (((size_t)n * a.wc + c) * H + h) * STATE;
-    for (int e = tid; e < 2 * STATE * 4 / 128; e += BT_THREADS) {
-        const int which = e / (STATE * 4 / 128), ln = e % (STATE * 4 / 128);
-        const float* base = which ? dSC : S0;
-        if (base) asm volatile("prefetch.global.L2 [%0];" ::"l"(reinterpret_cast<const char*>(base) + (size_t)ln * 128));
+    const char* S0 = c == 0 ? reinterpret_cast<const char*>(a.init_state ? a.init_state + ((size_t)n * H + h) * STATE
+                                                                            : nullptr)
+                            : reinterpret_cast<const char*>(a.ckpt + (((size_t)n * a.n_ckpt + (c - 1)) * H + h) *
+                                                                         STATE_IMG_BYTES);
+    const uint32_t s0_bytes = c == 0 ? STATE * 4 : STATE_IMG_BYTES;
+    const char* dSC = reinterpret_cast<const char*>(a.ds_end + (((size_t)n * a.wc + c) * H + h) * STATE_IMG_BYTES);
+    for (uint32_t e = tid; e < (s0_bytes + STATE_IMG_BYTES) / 128; e += BT_THREADS) {
+        const char* p = e < s0_bytes / 128 ? (S0 ? S0 + (size_t)e * 128 : nullptr) : dSC + (size_t)(e - s0_bytes / 128) * 128;
+        if (p) asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
     }
 }
 
@@ -166,6 +170,7 @@ constexpr uint32_t BT_I2L = 114688, BT_I1L = 155648;                    // their
 constexpr uint32_t BT_MISC = BT_I4 + 16384;
 constexpr uint32_t BT_BETA = BT_MISC, BT_G = BT_BETA + 256, BT_TOT = BT_G + 2560, BT_RS = BT_TOT + 2048,
                    BT_DGC = BT_RS + 2048, BT_DB = BT_DGC + 2048, BT_BAR = BT_DB + 256, BT_TPTR = BT_BAR + 64;
+static_assert(8 * 8 <= 64, "barriers");
 constexpr uint32_t BT_SMEM = BT_TPTR + 16 + 1024;
 constexpr int BT_LDA = TRI_LDA;
 // TMEM columns
@@ -292,8 +297,22 @@ KDA_DEV float tile_decays(const BwdArgs& a, size_t base_c, size_t rowk, int q4, 
     return run;
 }
 
+// the item's raw tiles (bf16 inputs): [64 tokens][128 channels] each, by TMA, at the start
+// of the item into the region of the state images (written after the tiles are read)
+struct BwdMaps {
+    CUtensorMap la, k, q, v, d_o;
+};
+constexpr uint32_t BT_RLA = 0, BT_RK = 16384, BT_RQ = 32768, BT_RV = 49152, BT_RDO = 65536;
+
+KDA_DEV float raw_bf16(const uint8_t* sm, uint32_t tile, int t, int c, int L) {
+    return t < L ? __uint_as_float((uint32_t)*reinterpret_cast<const uint16_t*>(sm + tile + (uint32_t)(t * 128 + c) * 2u)
+                                   << 16)
+                 : 0.f;
+}
+
 template <bool IN_BF16>
-__global__ void __launch_bounds__(BT_THREADS, 1) bwd_tc_kernel(const BwdArgs a, int64_t n_items) {
+__global__ void __launch_bounds__(BT_THREADS, 1) bwd_tc_kernel(const BwdArgs a, const __grid_constant__ BwdMaps maps,
+                                                            int64_t n_items) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     const uint32_t sb = smem_u32(sm);
@@ -313,8 +332,15 @@ __global__ void __launch_bounds__(BT_THREADS, 1) bwd_tc_kernel(const BwdArgs a, 
         tmem_relinquish();
     }
     if (tid == 0) {
-        for (int i = 0; i < 6; ++i) mbar_init(&bar[i], 1);
+        for (int i = 0; i < 8; ++i) mbar_init(&bar[i], 1);  // 0-5: the stages' products, 6: raw tiles, 7: states
         fence_mbar_init();
+        if constexpr (IN_BF16) {
+            prefetch_tmap(&maps.la);
+            prefetch_tmap(&maps.k);
+            prefetch_tmap(&maps.q);
+            prefetch_tmap(&maps.v);
+            prefetch_tmap(&maps.d_o);
+        }
     }
     __syncthreads();
     tc_fence_after();
@@ -348,17 +374,52 @@ __global__ void __launch_bounds__(BT_THREADS, 1) bwd_tc_kernel(const BwdArgs a, 
         const int64_t t0 = s_beg + (int64_t)cidx * CH;
         if (t0 >= s_end) continue;  // uniform over the CTA
         const int L = (int)((s_end - t0) < CH ? (s_end - t0) : CH);
-        const float* S0 = cidx == 0 ? (a.init_state ? a.init_state + ((size_t)n * H + h) * STATE : nullptr)
-                                    : a.ckpt + (((size_t)n * a.n_ckpt + (cidx - 1)) * H + h) * STATE;
-        const float* dSC = a.ds_end + (((size_t)n * a.wc + cidx) * H + h) * STATE;
+        // the chunk-start state: the initial state (fp32, or none) for the first chunk, else the
+        // forward walk's bf16 image; the chunk-end state gradient: the reverse walk's bf16 image
+        const float* S0f = (cidx == 0 && a.init_state) ? a.init_state + ((size_t)n * H + h) * STATE : nullptr;
+        const uint8_t* S0img = cidx == 0 ? nullptr : a.ckpt + (((size_t)n * a.n_ckpt + (cidx - 1)) * H + h) * STATE_IMG_BYTES;
+        const uint8_t* dSCimg = a.ds_end + (((size_t)n * a.wc + cidx) * H + h) * STATE_IMG_BYTES;
         prefetch_item(a, item + gridDim.x, n_items, tid);
         const size_t rowk = (size_t)H * DK;
         const size_t base_c = ((size_t)t0 * H + h) * DK + c;  // (token t0, head h, channel c)
         const int ib = IN_BF16 ? 1 : 0;
 
         // ================================================================ phase A
+        if constexpr (IN_BF16) {
+            if (tid == 0) {
+                fence_async_smem();  // the previous item's generic reads of this region are done
+                mbar_arrive_expect_tx(&bar[6], 5u * 16384u);
+                tma_load_2d(sm + BT_RLA, &maps.la, h * DK, (int)t0, &bar[6]);
+                tma_load_2d(sm + BT_RK, &maps.k, h * DK, (int)t0, &bar[6]);
+                tma_load_2d(sm + BT_RQ, &maps.q, h * DK, (int)t0, &bar[6]);
+                tma_load_2d(sm + BT_RV, &maps.v, h * DV, (int)t0, &bar[6]);
+                tma_load_2d(sm + BT_RDO, &maps.d_o, h * DV, (int)t0, &bar[6]);
+            }
+            committed = 7;  // for the drain: the tile loads are in flight
+            if (!wait_mma(6)) { failed = true; break; }
+            committed = 0;
+        }
         float E1[16], E3[16];
-        const float run = tile_decays<IN_BF16>(a, base_c, rowk, q4, L, E1, E3, nullptr);
+        float run;
+        if constexpr (IN_BF16) {
+            float alpha[16];
+            run = 0.f;
+#pragma unroll
+            for (int u = 0; u < 16; ++u) {
+                const int t = 16 * q4 + u;
+                const float l = t < L ? fmaxf(raw_bf16(sm, BT_RLA, t, c, L), -5.f) : 0.f;
+                run += l;
+                alpha[u] = __expf(l);
+            }
+            E1[0] = alpha[0];
+#pragma unroll
+            for (int u = 1; u < 16; ++u) E1[u] = E1[u - 1] * alpha[u];
+            E3[15] = 1.f;
+#pragma unroll
+            for (int u = 14; u >= 0; --u) E3[u] = E3[u + 1] * alpha[u + 1];
+        } else {
+            run = tile_decays<IN_BF16>(a, base_c, rowk, q4, L, E1, E3, nullptr);
+        }
         s_tot[q4 * 128 + c] = run;
         if (tid < CH) {
             s_beta[tid] = tid < L ? ld_in(a.beta, (size_t)(t0 + tid) * H + h, ib) : 0.f;
@@ -380,7 +441,7 @@ __global__ void __launch_bounds__(BT_THREADS, 1) bwd_tc_kernel(const BwdArgs a, 
         const float Gs = (q4 == 0) ? G[0] : (q4 == 1) ? G[1] : (q4 == 2) ? G[2] : G[3];
         const float Gn = (q4 == 0) ? G[1] : (q4 == 1) ? G[2] : (q4 == 2) ? G[3] : G[4];
         // raw k, q, v of this thread's 16 tokens (bf16 bit pairs; exact for bf16 inputs)
-        uint32_t kr2[8], qr2[8], vr2[8];
+        uint32_t kr2[8], qr2[8], vr2[8], dor2[8];
         {
             const float eD = __expf(Gs - Gn);
             const float f2 = __expf(((q4 == 0) ? G[2] : G[3]) - Gn);
@@ -393,18 +454,26 @@ __global__ void __launch_bounds__(BT_THREADS, 1) bwd_tc_kernel(const BwdArgs a, 
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
                     const int t = tf + e;
-                    const bool in = t < L;
-                    const size_t idx = base_c + (size_t)t * rowk;
-                    kv[e] = in ? ld_in(a.k, idx, ib) : 0.f;
-                    qv[e] = in ? ld_in(a.q, idx, ib) : 0.f;
-                    vv[e] = in ? ld_in(a.v, idx, ib) : 0.f;
-                    dov[e] = in ? ld_in(a.d_o, idx, ib) : 0.f;
+                    if constexpr (IN_BF16) {
+                        kv[e] = raw_bf16(sm, BT_RK, t, c, L);
+                        qv[e] = raw_bf16(sm, BT_RQ, t, c, L);
+                        vv[e] = raw_bf16(sm, BT_RV, t, c, L);
+                        dov[e] = raw_bf16(sm, BT_RDO, t, c, L);
+                    } else {
+                        const bool in = t < L;
+                        const size_t idx = base_c + (size_t)t * rowk;
+                        kv[e] = in ? ld_in(a.k, idx, ib) : 0.f;
+                        qv[e] = in ? ld_in(a.q, idx, ib) : 0.f;
+                        vv[e] = in ? ld_in(a.v, idx, ib) : 0.f;
+                        dov[e] = in ? ld_in(a.d_o, idx, ib) : 0.f;
+                    }
                 }
 #pragma unroll
                 for (int e = 0; e < 8; e += 2) {
                     kr2[(8 * m + e) >> 1] = pack_bf16x2(kv[e], kv[e + 1]);
                     qr2[(8 * m + e) >> 1] = pack_bf16x2(qv[e], qv[e + 1]);
                     vr2[(8 * m + e) >> 1] = pack_bf16x2(vv[e], vv[e + 1]);
+                    dor2[(8 * m + e) >> 1] = pack_bf16x2(dov[e], dov[e + 1]);
                 }
                 float x[8], y[8];
 #pragma unroll
@@ -444,31 +513,50 @@ __global__ void __launch_bounds__(BT_THREADS, 1) bwd_tc_kernel(const BwdArgs a, 
                 }
                 st16(sm + BT_I3 + il_off(c, tf, 64), x);
                 st16(sm + BT_I4 + il_off(c, tf, 64), y);
-                st16(sm + BT_I7 + il_off(c, 64 + tf, 128), dov);  // dO^T: row j = c
             }
-            // S0 and dSC row c, columns [32 q4, 32 q4 + 32)
+            __syncthreads();  // every read of the raw tiles is done: their region takes S0, dSC, dO^T
+#pragma unroll
+            for (int m = 0; m < 2; ++m)  // dO^T: row j = c
+                *reinterpret_cast<uint4*>(sm + BT_I7 + il_off(c, 64 + 16 * q4 + 8 * m, 128)) =
+                    make_uint4(dor2[4 * m], dor2[4 * m + 1], dor2[4 * m + 2], dor2[4 * m + 3]);
+            // S0 and dSC: the images arrive by bulk copies into the region the raw tiles just left
+            // (the first chunk's S0 comes from the fp32 initial state, converted here)
+            if (tid == 0) {
+                fence_async_smem();
+                mbar_arrive_expect_tx(&bar[7], S0img ? 2u * STATE_IMG_BYTES : STATE_IMG_BYTES);
+                if (S0img) bulk_g2s(sm + BT_I5, S0img, STATE_IMG_BYTES, &bar[7]);
+                bulk_g2s(sm + BT_I6, dSCimg, STATE_IMG_BYTES, &bar[7]);
+            }
+            if (!S0img) {
+#pragma unroll
+                for (int m = 0; m < 4; ++m) {
+                    const int j = 32 * q4 + 8 * m;
+                    float s8[8];
+                    if (S0f) {
+                        const float4 u0 = __ldg(reinterpret_cast<const float4*>(S0f + (size_t)c * DV + j));
+                        const float4 u1 = __ldg(reinterpret_cast<const float4*>(S0f + (size_t)c * DV + j + 4));
+                        s8[0] = u0.x; s8[1] = u0.y; s8[2] = u0.z; s8[3] = u0.w;
+                        s8[4] = u1.x; s8[5] = u1.y; s8[6] = u1.z; s8[7] = u1.w;
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) s8[e] = 0.f;
+                    }
+                    st16(sm + BT_I5 + il_off(c, j, 128), s8);
+                }
+            }
+            committed = 8;  // for the drain: the state copies are in flight
+            if (!wait_mma(7)) { failed = true; break; }
+            committed = 0;
+            // rowsum(S0 o dSC) of row c over columns [32 q4, 32 q4 + 32), from the images
             float rs = 0.f;
 #pragma unroll
             for (int m = 0; m < 4; ++m) {
-                const int j = 32 * q4 + 8 * m;
-                float s8[8], d8[8];
-                if (S0) {
-                    const float4 u0 = __ldg(reinterpret_cast<const float4*>(S0 + (size_t)c * DV + j));
-                    const float4 u1 = __ldg(reinterpret_cast<const float4*>(S0 + (size_t)c * DV + j + 4));
-                    s8[0] = u0.x; s8[1] = u0.y; s8[2] = u0.z; s8[3] = u0.w;
-                    s8[4] = u1.x; s8[5] = u1.y; s8[6] = u1.z; s8[7] = u1.w;
-                } else {
+                const uint32_t off = il_off(c, 32 * q4 + 8 * m, 128);
+                const uint4 x = *reinterpret_cast<const uint4*>(sm + BT_I5 + off);
+                const uint4 y = *reinterpret_cast<const uint4*>(sm + BT_I6 + off);
+                const uint32_t xs[4] = {x.x, x.y, x.z, x.w}, ys[4] = {y.x, y.y, y.z, y.w};
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) s8[e] = 0.f;
-                }
-                const float4 w0 = __ldg(reinterpret_cast<const float4*>(dSC + (size_t)c * DV + j));
-                const float4 w1 = __ldg(reinterpret_cast<const float4*>(dSC + (size_t)c * DV + j + 4));
-                d8[0] = w0.x; d8[1] = w0.y; d8[2] = w0.z; d8[3] = w0.w;
-                d8[4] = w1.x; d8[5] = w1.y; d8[6] = w1.z; d8[7] = w1.w;
-#pragma unroll
-                for (int e = 0; e < 8; ++e) rs += s8[e] * d8[e];
-                st16(sm + BT_I5 + il_off(c, j, 128), s8);
-                st16(sm + BT_I6 + il_off(c, j, 128), d8);
+                for (int e = 0; e < 4; ++e) rs += lo_bf(xs[e]) * lo_bf(ys[e]) + hi_bf(xs[e]) * hi_bf(ys[e]);
             }
             s_rs[q4 * 128 + c] = rs;
         }
@@ -941,8 +1029,11 @@ __global__ void __launch_bounds__(BT_THREADS, 1) bwd_tc_kernel(const BwdArgs a, 
         committed = 0;
     }
     if (failed && tid == 0) {
-        // products still in flight complete before the TMEM is released (bounded)
-        for (int i = 0; i < committed; ++i) mbar_wait(&bar[i], par, nullptr);
+        // tile loads and products still in flight complete before the CTA retires (bounded)
+        if (committed == 7) mbar_wait(&bar[6], par, nullptr);
+        else if (committed == 8) mbar_wait(&bar[7], par, nullptr);
+        else
+            for (int i = 0; i < committed; ++i) mbar_wait(&bar[i], par, nullptr);
     }
     tc_fence_before();
     __syncthreads();
@@ -1154,11 +1245,12 @@ __global__ void __launch_bounds__(RB_THREADS, 1) chain_bwd_tc_kernel(const BwdAr
             mbar_arrive(bar_img);
             for (int it = 0; it < nck; ++it) {
                 const int c = nck - 1 - it, b = bidx(it);
-                // dL/d(state at the end of chunk c)
-                float* dst = a.ds_end + (((size_t)n * a.wc + c) * H + h) * STATE + (size_t)i * DV + (size_t)DVS * js;
+                // dL/d(state at the end of chunk c), as a bf16 operand image (row i, this slice's columns)
+                uint8_t* dimg = a.ds_end + (((size_t)n * a.wc + c) * H + h) * STATE_IMG_BYTES;
 #pragma unroll
-                for (int j = 0; j < DVS; j += 4)
-                    *reinterpret_cast<float4*>(dst + j) = make_float4(dS[j], dS[j + 1], dS[j + 2], dS[j + 3]);
+                for (int m = 0; m < DVS / 8; ++m)
+                    *reinterpret_cast<uint4*>(dimg + state_img_off((uint32_t)i, (uint32_t)(DVS * js + 8 * m))) =
+                        pack8f(dS + 8 * m);
                 // -dS image (row m = i) and the next chunk's dO image
                 {
                     uint8_t* img = sm + RB_DS + (uint32_t)(i >> 3) * 512u + (uint32_t)(i & 7) * 16u;
@@ -1221,7 +1313,7 @@ __global__ void __launch_bounds__(RB_THREADS, 1) chain_bwd_tc_kernel(const BwdAr
 size_t chunk_bwd_extra_bytes(int n_seqs, int H, int64_t max_seqlen) {
     const int64_t nck = (max_seqlen + CH - 1) / CH;
     const int64_t n_ckpt = max_seqlen / CH;
-    return (size_t)n_seqs * H * STATE * sizeof(float) * (size_t)(nck + n_ckpt);
+    return (size_t)n_seqs * H * STATE_IMG_BYTES * (size_t)(nck + n_ckpt);
 }
 
 cudaError_t chunk_bwd_launch(const void* q, const void* k, const void* v, const void* log_alpha, const void* beta,
@@ -1252,11 +1344,11 @@ cudaError_t chunk_bwd_launch(const void* q, const void* k, const void* v, const 
     const int nck = (int)((maxlen + CH - 1) / CH);
     const int n_ckpt = (int)(maxlen / CH);
     uint8_t* ws = reinterpret_cast<uint8_t*>(workspace);
-    float* ckpt = reinterpret_cast<float*>(ws + fwd_bytes);
-    float* ds_end = ckpt + (size_t)N * n_ckpt * H * STATE;
+    uint8_t* ckpt = ws + fwd_bytes;  // chunk-boundary states, bf16 images
+    uint8_t* ds_end = ckpt + (size_t)N * n_ckpt * H * STATE_IMG_BYTES;
     // 1. the forward walk again, without outputs: chunk slots and chunk-boundary states
     err = chunk_fwd_launch(q, k, v, log_alpha, beta, init_state, nullptr, nullptr, B, T, H, cu, n_seqs, max_seqlen,
-                           in_bf16, false, scale, nullptr, nullptr, 0.f, n_ckpt > 0 ? ckpt : nullptr, CH, 1, KCP_NONE,
+                           in_bf16, false, scale, nullptr, nullptr, 0.f, n_ckpt > 0 ? reinterpret_cast<float*>(ckpt) : nullptr, CH, 1, KCP_NONE,
                            nullptr, workspace, fwd_bytes, stream, nullptr, nullptr);
     if (err != cudaSuccess) return err;
     // the forward's slot region (whole-sequence workspace: one pass)
@@ -1283,9 +1375,18 @@ cudaError_t chunk_bwd_launch(const void* q, const void* k, const void* v, const 
     const int64_t n_items = (int64_t)N * a.wc * H;
     if (nck > 0 && n_items > 0) {
         const unsigned grid = (unsigned)(n_items < sms ? n_items : sms);
+        BwdMaps maps;
+        memset(&maps, 0, sizeof(maps));
+        const int64_t total_tokens = cu ? T : (int64_t)B * T;
+        if (in_bf16 && (!make_bf16_tile_map(&maps.la, log_alpha, total_tokens, (int64_t)H * DK) ||
+                        !make_bf16_tile_map(&maps.k, k, total_tokens, (int64_t)H * DK) ||
+                        !make_bf16_tile_map(&maps.q, q, total_tokens, (int64_t)H * DK) ||
+                        !make_bf16_tile_map(&maps.v, v, total_tokens, (int64_t)H * DV) ||
+                        !make_bf16_tile_map(&maps.d_o, d_o, total_tokens, (int64_t)H * DV)))
+            return cudaErrorInvalidValue;
         prof_begin(PROF_INTRA_BWD, stream);
-        if (in_bf16) bwd_tc_kernel<true><<<grid, BT_THREADS, BT_SMEM, stream>>>(a, n_items);
-        else bwd_tc_kernel<false><<<grid, BT_THREADS, BT_SMEM, stream>>>(a, n_items);
+        if (in_bf16) bwd_tc_kernel<true><<<grid, BT_THREADS, BT_SMEM, stream>>>(a, maps, n_items);
+        else bwd_tc_kernel<false><<<grid, BT_THREADS, BT_SMEM, stream>>>(a, maps, n_items);
         if ((err = cudaGetLastError()) != cudaSuccess) return err;
         prof_end(PROF_INTRA_BWD, stream);
     }

@@ -1038,10 +1038,22 @@ chain_kernel(const ChunkArgs a, const __grid_constant__ CUtensorMap gate_map, co
                 const int64_t t_end = s_beg + (int64_t)cdone * CH;
                 if (cdone % a.ckpt_every == 0 && t_end <= s_end && cdone / a.ckpt_every <= a.n_ckpt) {
                     const int j = cdone / a.ckpt_every - 1;
-                    float* dst = a.ckpt + ((((size_t)n * a.n_ckpt + j) * H + h) * DK + tid) * DV + (size_t)DVS * jb;
+                    if constexpr (SEG == 3) {
+                        // the backward's chunk-boundary states: bf16 operand images (row tid, columns
+                        // [32 jb, 32 jb + 32)), bulk-copied by its chunk-local kernel
+                        uint8_t* img = reinterpret_cast<uint8_t*>(a.ckpt) +
+                                       (((size_t)n * a.n_ckpt + j) * H + h) * STATE_IMG_BYTES;
 #pragma unroll
-                    for (int c4 = 0; c4 < DVS; c4 += 4)
-                        __stcs(reinterpret_cast<float4*>(dst + c4), make_float4(S[c4], S[c4 + 1], S[c4 + 2], S[c4 + 3]));
+                        for (int m = 0; m < DVS / 8; ++m)
+                            *reinterpret_cast<uint4*>(img + state_img_off((uint32_t)tid, (uint32_t)(DVS * jb + 8 * m))) =
+                                pack8(S + 8 * m);
+                    } else {
+                        float* dst = a.ckpt + ((((size_t)n * a.n_ckpt + j) * H + h) * DK + tid) * DV + (size_t)DVS * jb;
+#pragma unroll
+                        for (int c4 = 0; c4 < DVS; c4 += 4)
+                            __stcs(reinterpret_cast<float4*>(dst + c4),
+                                   make_float4(S[c4], S[c4 + 1], S[c4 + 2], S[c4 + 3]));
+                    }
                 }
             };
 
@@ -1287,6 +1299,10 @@ bool g_drop_tile = false;
 unsigned long long g_drop_wait_ns = WAIT_LIMIT_NS;
 
 }  // namespace
+
+bool make_bf16_tile_map(CUtensorMap* m, const void* base, int64_t rows, int64_t row_elems) {
+    return make_tile_map(m, base, rows, row_elems);
+}
 
 void set_test_tile_drop(unsigned long long wait_ns) {
     g_drop_tile = wait_ns != 0;

@@ -1,5 +1,6 @@
 // kda_launch.h -- host-side launchers behind the C ABI (internal to libkda).
 #pragma once
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -28,6 +29,10 @@ cudaError_t chunk_fwd_launch(const void* q, const void* k, const void* v, const 
                              float scale, const void* gate, const float* norm_w, float eps, float* ckpt,
                              int64_t ckpt_tokens, int segs, int kcp_mode, float* trans_out, void* workspace,
                              size_t ws_bytes, cudaStream_t stream, int* n_passes, bool* gate_fused);
+// 2-D tensor map of a [rows, row_elems] bf16 tensor with a box of 64 rows x 128
+// elements, no swizzle (the chunk-local kernels' tile loads).  False on failure.
+bool make_bf16_tile_map(CUtensorMap* m, const void* base, int64_t rows, int64_t row_elems);
+
 // Test hook: the next chunk-local launch with bf16 inputs has CTA 0 skip one of
 // its first item's four tile loads and give up waiting after wait_ns (0 cancels).
 void set_test_tile_drop(unsigned long long wait_ns);

@@ -30,4 +30,13 @@ constexpr uint32_t SO_MQG = 49664;         // Mlr + Qp + GamC, one contiguous co
 constexpr uint32_t BSL = DK * DVS * 2;     // one Bm slice, 8192 B
 constexpr uint32_t OSL = CH * DVS * 2;     // one Ob slice, 4096 B
 
+// A 128 x 128 state as a bf16 tensor-core operand image (the backward pass keeps its
+// chunk-boundary states and chunk-end state gradients this way): element (row i,
+// column j) at state_img_off(i, j), rows in 16-byte pieces of 8 columns, 8-row core
+// matrices of 128 bytes, column pieces 128 bytes apart, row groups 2,048 bytes apart.
+constexpr uint32_t STATE_IMG_BYTES = DK * DV * 2;
+__host__ __device__ inline uint32_t state_img_off(uint32_t i, uint32_t j) {
+    return (i >> 3) * 2048u + (j >> 3) * 128u + (i & 7u) * 16u + (j & 7u) * 2u;
+}
+
 }  // namespace kda

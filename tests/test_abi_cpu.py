@@ -156,8 +156,9 @@ def test_chunk_bwd_workspace_and_host_validation(lib):
     assert lib.kda_chunk_fwd_workspace_size(300, 2, 128, 128, 1, 300, None, ctypes.byref(full)) == 0
     n = ctypes.c_size_t(0)
     assert lib.kda_chunk_bwd_workspace_size(300, 2, 128, 128, 1, 300, ctypes.byref(n)) == 0
-    # the forward's whole-sequence workspace + 5 chunk-end gradients + 4 chunk-boundary states
-    assert n.value == full.value + (5 + 4) * 2 * 128 * 128 * 4
+    # the forward's whole-sequence workspace + 5 chunk-end gradients + 4 chunk-boundary states,
+    # each a bf16 128 x 128 image per head
+    assert n.value == full.value + (5 + 4) * 2 * 128 * 128 * 2
 
     def bw(**over):
         a = dict(q=FAKE, k=FAKE, v=FAKE, la=FAKE, beta=FAKE, s0=None, do=FAKE, dfin=None, dq=FAKE, dk=FAKE,
