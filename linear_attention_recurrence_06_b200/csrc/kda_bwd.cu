@@ -93,19 +93,28 @@ constexpr int BT_THREADS = 512;  // threads of the chunk-local kernel
 
 // Pulls an item's token rows (q, k, v, log_alpha, dO: 64 rows each), its
 // chunk-start state and its end-of-chunk state gradient into L2 ahead of use.
+// (sequence, chunk, head) of an item: item = (n * wc + chunk) * H + h (items < 2^31)
+KDA_DEV void bwd_item(const BwdArgs& a, int64_t item, int& n, int& c, int& h) {
+    const uint32_t it = (uint32_t)item, rest = it / (uint32_t)a.H;
+    h = (int)(it - rest * (uint32_t)a.H);
+    const uint32_t nn = rest / (uint32_t)a.wc;
+    c = (int)(rest - nn * (uint32_t)a.wc);
+    n = (int)nn;
+}
+
+template <bool IN_BF16>
 KDA_DEV void prefetch_item(const BwdArgs& a, int64_t item, int64_t n_items, int tid) {
     if (item >= n_items) return;
     const int H = a.H;
-    const int h = (int)(item % H);
-    const int c = (int)((item / H) % a.wc);
-    const int n = (int)(item / ((int64_t)H * a.wc));
+    int n, c, h;
+    bwd_item(a, item, n, c, h);
     int64_t s_beg, s_end;
     bwd_seq_range(a, n, s_beg, s_end);
     const int64_t t0 = s_beg + (int64_t)c * CH;
     if (t0 >= s_end) return;
     const int L = (int)((s_end - t0) < CH ? (s_end - t0) : CH);
-    const size_t esz = a.in_bf16 ? 2 : 4, row = DK * esz;  // bytes of one head row
-    const int lines_row = (int)(row / 128);
+    constexpr size_t row = DK * (IN_BF16 ? 2 : 4);  // bytes of one head row
+    constexpr int lines_row = (int)(row / 128);
     const void* tens[5] = {a.q, a.k, a.v, a.log_alpha, a.d_o};
     for (int e = tid; e < 5 * CH * lines_row; e += BT_THREADS) {
         const int tsr = e / (CH * lines_row), rem = e % (CH * lines_row), t = rem / lines_row, ln = rem % lines_row;
@@ -219,22 +228,22 @@ KDA_DEV uint4 pack8f(const float* x) {
     return make_uint4(pack_bf16x2(x[0], x[1]), pack_bf16x2(x[2], x[3]), pack_bf16x2(x[4], x[5]),
                       pack_bf16x2(x[6], x[7]));
 }
+KDA_DEV float lo_bf(uint32_t w) { return __uint_as_float(w << 16); }
+KDA_DEV float hi_bf(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 KDA_DEV void st16(uint8_t* p, const float* x) { *reinterpret_cast<uint4*>(p) = pack8f(x); }
 // x as the sum of two bf16 images, hi = bf16(x) and lo = bf16(x - hi): a product with
 // both (two MMAs into one accumulator) carries about 16 bits of x instead of 8
 KDA_DEV void st16_hilo(uint8_t* hi, uint8_t* lo, const float* x) {
-    float h[8], l[8];
+    uint32_t hw[4], lw[4];
 #pragma unroll
-    for (int e = 0; e < 8; ++e) {
-        h[e] = __bfloat162float(__float2bfloat16_rn(x[e]));
-        l[e] = x[e] - h[e];
+    for (int e = 0; e < 4; ++e) {
+        hw[e] = pack_bf16x2(x[2 * e], x[2 * e + 1]);  // the high parts, rounded to nearest
+        lw[e] = pack_bf16x2(x[2 * e] - lo_bf(hw[e]), x[2 * e + 1] - hi_bf(hw[e]));
     }
-    *reinterpret_cast<uint4*>(hi) = pack8f(h);
-    *reinterpret_cast<uint4*>(lo) = pack8f(l);
+    *reinterpret_cast<uint4*>(hi) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+    *reinterpret_cast<uint4*>(lo) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
 }
 KDA_DEV void st16z(uint8_t* p) { *reinterpret_cast<uint4*>(p) = make_uint4(0u, 0u, 0u, 0u); }
-KDA_DEV float lo_bf(uint32_t w) { return __uint_as_float(w << 16); }
-KDA_DEV float hi_bf(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
 // Sum over the 32 lanes of v[u] for each u < 16; lane l ends with the sum for token
 // u = l >> 1 (both lanes of a pair hold it).  16 shuffles.
@@ -366,9 +375,8 @@ __global__ void __launch_bounds__(BT_THREADS, 1) bwd_tc_kernel(const BwdArgs a, 
     };
 
     for (int64_t item = blockIdx.x; item < n_items && !failed; item += gridDim.x) {
-        const int h = (int)(item % H);
-        const int cidx = (int)((item / H) % a.wc);
-        const int n = (int)(item / ((int64_t)H * a.wc));
+        int n, cidx, h;
+        bwd_item(a, item, n, cidx, h);
         int64_t s_beg, s_end;
         bwd_seq_range(a, n, s_beg, s_end);
         const int64_t t0 = s_beg + (int64_t)cidx * CH;
@@ -379,7 +387,7 @@ __global__ void __launch_bounds__(BT_THREADS, 1) bwd_tc_kernel(const BwdArgs a, 
         const float* S0f = (cidx == 0 && a.init_state) ? a.init_state + ((size_t)n * H + h) * STATE : nullptr;
         const uint8_t* S0img = cidx == 0 ? nullptr : a.ckpt + (((size_t)n * a.n_ckpt + (cidx - 1)) * H + h) * STATE_IMG_BYTES;
         const uint8_t* dSCimg = a.ds_end + (((size_t)n * a.wc + cidx) * H + h) * STATE_IMG_BYTES;
-        prefetch_item(a, item + gridDim.x, n_items, tid);
+        prefetch_item<IN_BF16>(a, item + gridDim.x, n_items, tid);
         const size_t rowk = (size_t)H * DK;
         const size_t base_c = ((size_t)t0 * H + h) * DK + c;  // (token t0, head h, channel c)
         const int ib = IN_BF16 ? 1 : 0;
@@ -401,13 +409,19 @@ __global__ void __launch_bounds__(BT_THREADS, 1) bwd_tc_kernel(const BwdArgs a, 
         }
         float E1[16], E3[16];
         float run;
+        uint32_t lar2[8];      // raw log-decays of this thread's tokens (bf16 pairs), for phases E and F
+        uint32_t keep_la = 0;  // tokens whose log-decay is at or above the floor (the clamp passes them)
         if constexpr (IN_BF16) {
             float alpha[16];
             run = 0.f;
 #pragma unroll
             for (int u = 0; u < 16; ++u) {
                 const int t = 16 * q4 + u;
-                const float l = t < L ? fmaxf(raw_bf16(sm, BT_RLA, t, c, L), -5.f) : 0.f;
+                const float raw = raw_bf16(sm, BT_RLA, t, c, L);
+                if (u & 1) lar2[u >> 1] |= __float_as_uint(raw) & 0xFFFF0000u;
+                else lar2[u >> 1] = __float_as_uint(raw) >> 16;
+                if (t < L && raw >= -5.f) keep_la |= 1u << u;
+                const float l = t < L ? fmaxf(raw, -5.f) : 0.f;
                 run += l;
                 alpha[u] = __expf(l);
             }
@@ -725,7 +739,6 @@ __global__ void __launch_bounds__(BT_THREADS, 1) bwd_tc_kernel(const BwdArgs a, 
 
         // ================================================================ phase E
         if (!wait_mma(4)) { failed = true; break; }
-        uint32_t keep_la = 0;  // tokens whose log-decay is at or above the floor (the clamp passes them)
         {   // [-dM ; dP] rows -> [A' ; P'] image at their column versions, dbeta's dM o A part
             const int p = q4, r = 32 * qd + lane;
             const bool isP = r >= 64;
@@ -816,7 +829,23 @@ __global__ void __launch_bounds__(BT_THREADS, 1) bwd_tc_kernel(const BwdArgs a, 
             const float f3 = __expf(G[3] - Gn);
             float (&E1b)[16] = E1;
             float (&E3b)[16] = E3;
-            tile_decays<IN_BF16>(a, base_c, rowk, q4, L, E1b, E3b, &keep_la);
+            if constexpr (IN_BF16) {  // from the log-decays kept since phase A
+                float alpha[16];
+#pragma unroll
+                for (int u = 0; u < 16; ++u) {
+                    const int t = 16 * q4 + u;
+                    const float raw = (u & 1) ? hi_bf(lar2[u >> 1]) : lo_bf(lar2[u >> 1]);
+                    alpha[u] = __expf(t < L ? fmaxf(raw, -5.f) : 0.f);
+                }
+                E1b[0] = alpha[0];
+#pragma unroll
+                for (int u = 1; u < 16; ++u) E1b[u] = E1b[u - 1] * alpha[u];
+                E3b[15] = 1.f;
+#pragma unroll
+                for (int u = 14; u >= 0; --u) E3b[u] = E3b[u + 1] * alpha[u + 1];
+            } else {
+                tile_decays<IN_BF16>(a, base_c, rowk, q4, L, E1b, E3b, &keep_la);
+            }
 #pragma unroll
             for (int m = 0; m < 2; ++m) {
                 const int tf = 16 * q4 + 8 * m;
