@@ -354,9 +354,9 @@ def run_decode(args, torch, kda, dev, stream, rank, max_over_ranks, barrier):
                         f"consecutive steps, bf16 tokens (pool of {pool} distinct steps)",
             "value": steps_s, "unit": "steps/s", "ms_per_step": ms / nsteps, "state_gbs": gbs,
             "hbm_frac": gbs / peaks["hbm_gbs"],
-            "roofline": {"bound": "hbm", "kernel": "decode_step_kernel", "achieved": kgbs, "peak": peaks["hbm_gbs"],
+            "roofline": {"bound": "hbm", "kernel": "decode_multi_kernel", "achieved": kgbs, "peak": peaks["hbm_gbs"],
                          "unit": "GB/s", "frac": (kgbs / peaks["hbm_gbs"]) if kgbs else None,
-                         "traffic": recorded_traffic("decode_step_kernel", Bd * H),
+                         "traffic": recorded_traffic("decode_multi_kernel", Bd * H),
                          "algorithmic_bytes_per_launch": state_bytes + tok_bytes},
             "speculative_verify": spec}
 
@@ -751,10 +751,12 @@ def recorded_traffic(kernel: str, units: int):
 # the source files each recorded kernel is built from (a change to any of them
 # voids its recorded traffic)
 KERNEL_SOURCES = {
-    "kda_chunk_fwd": ("kda_chunk.cu", "kda_sm100.cuh", "kda_slots.h"),
-    "intra_kernel": ("kda_chunk.cu", "kda_sm100.cuh", "kda_slots.h"),
+    "kda_chunk_fwd": ("kda_chunk.cu", "kda_sm100.cuh", "kda_slots.h", "kda_tri.cuh"),
+    "intra_kernel": ("kda_chunk.cu", "kda_sm100.cuh", "kda_slots.h", "kda_tri.cuh"),
     "chain_kernel": ("kda_chunk.cu", "kda_sm100.cuh", "kda_slots.h"),
-    "decode_step_kernel": ("kda_decode.cu", "kda_sm100.cuh"),
+    "decode_multi_kernel": ("kda_decode.cu", "kda_sm100.cuh"),
+    "bwd_tc_kernel": ("kda_bwd.cu", "kda_sm100.cuh", "kda_slots.h", "kda_tri.cuh"),
+    "chain_bwd_tc_kernel": ("kda_bwd.cu", "kda_sm100.cuh", "kda_slots.h"),
 }
 
 
