@@ -265,7 +265,8 @@ def run_ours(args, peaks):
     roof = dict(bound="hbm", kernel="kda_chunk_fwd (all launches of one call)", achieved=achieved_gbs,
                 peak=peaks["hbm_gbs"], unit="GB/s", frac=achieved_gbs / peaks["hbm_gbs"],
                 traffic=recorded_traffic("kda_chunk_fwd", th), peak_source=peaks["source"],
-                algorithmic_bytes_per_launch=bytes_call, dominant_kernel=dominant)
+                algorithmic_bytes_per_launch=bytes_call, dominant_kernel=dominant,
+                intra_tensor_pipe=recorded_tensor_pipe("intra_kernel"))
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": ws_n, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
@@ -731,6 +732,24 @@ def run_e2e(args, torch, kda, hq, out, fs, ws, stream, max_over_ranks, barrier):
     return {"value": whole_job_rate(ws_n, B * T, ms), "unit": "tokens/s", "ms_per_step": ms,
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
             "pipelined": "two buffer sets; copy-in, compute and read-back of consecutive steps overlap"}
+
+
+def recorded_tensor_pipe(kernel: str):
+    """Tensor-pipe activity of a kernel from the committed ncu summary (fraction of its
+    elapsed cycles, and over its tensor-core product stages), if taken on the current
+    sources (else None)."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    try:
+        rec = json.load(open(p)).get(kernel)
+    except Exception:
+        return None
+    if not rec or rec.get("sources_sha256") != sources_sha256(kernel) or "tensor_pipe_active_frac" not in rec:
+        return None
+    return {"active_frac": rec["tensor_pipe_active_frac"],
+            "active_frac_over_product_stages": rec.get("tensor_pipe_active_frac_over_product_stages"),
+            "source": "ncu sm__pipe_tensor_cycles_active, profiles/kda_intra_T4096_H32_ncu_full.md"}
 
 
 def recorded_traffic(kernel: str, units: int):

@@ -256,3 +256,44 @@ def test_build_tracks_every_header(tmp_path):
     finally:
         os.utime(slots, (st.st_atime, st.st_mtime))
     assert kbuild.up_to_date()
+
+
+# The boundary's entry points as declared in include/kda.h.  Against the planned boundary
+# (the scope table's list: kda_chunk_fwd(q, k, v, log_alpha, beta, init_state -> o,
+# final_state; B, T, H, dk, dv, cu_seqlens ...), kda_decode_step, kda_gate_norm,
+# kda_query_status, kda_chunk_fwd_workspace_size, kda_status_string) the differences are
+# deliberate: kda_chunk_fwd takes max_seqlen (the host never reads cu_seqlens), the
+# workspace query returns a minimum and a full size (multi-pass workspaces), kda_decode_step
+# takes the optional fused gate, kda_status_string takes an int (callable from any
+# language), and streams pass as void*.  Pinning the declarations here makes any further
+# change to them a visible, reviewed edit.
+BOUNDARY = {
+    "kda_chunk_fwd": ("kda_status", [
+        "const void* q", "const void* k", "const void* v", "const void* log_alpha", "const void* beta",
+        "const float* init_state", "void* o", "float* final_state", "int B", "int64_t T", "int H", "int dk",
+        "int dv", "const int32_t* cu_seqlens", "int n_seqs", "int64_t max_seqlen", "kda_dtype in_dtype",
+        "kda_dtype out_dtype", "float scale", "const void* gate", "const float* norm_weight", "float eps",
+        "void* workspace", "size_t workspace_bytes", "void* stream"]),
+    "kda_decode_step": ("kda_status", [
+        "float* state", "const void* q", "const void* k", "const void* v", "const void* log_alpha",
+        "const void* beta", "void* o", "int Bd", "int H", "int dk", "int dv", "kda_dtype in_dtype",
+        "kda_dtype out_dtype", "float scale", "const void* gate", "const float* norm_weight", "float eps",
+        "void* stream"]),
+    "kda_gate_norm": ("kda_status", [
+        "const void* o", "const void* gate", "const float* norm_weight", "float eps", "void* y", "int64_t rows",
+        "int dv", "kda_dtype in_dtype", "kda_dtype out_dtype", "void* stream"]),
+    "kda_query_status": ("kda_status", ["void* workspace", "void* stream"]),
+    "kda_chunk_fwd_workspace_size": ("kda_status", [
+        "int64_t T", "int H", "int dk", "int dv", "int n_seqs", "int64_t max_seqlen", "size_t* bytes_min",
+        "size_t* bytes_full"]),
+    "kda_status_string": ("const char*", ["int status"]),
+}
+
+
+def test_boundary_declarations_are_pinned():
+    txt = open(HEADER).read()
+    for name, (ret, params) in BOUNDARY.items():
+        m = re.search(r"KDA_API\s+([\w\s\*]+?)\b" + name + r"\s*\(([^;]*?)\);", txt, re.S)
+        assert m, name
+        assert " ".join(m.group(1).split()) == ret, name
+        assert [" ".join(p.split()) for p in m.group(2).split(",")] == params, name
