@@ -783,12 +783,7 @@ constexpr uint32_t PART_TX = CLUSTER * 64 * 4;  // partial-sum bytes each CTA re
 
 // SEG = 0: the plain walk over this pass's chunks.  Segment-parallel prefill (each
 // sequence cut into a.segs segments of whole chunks, blockIdx.z = n * segs + g):
-// SEG = 1: per segment, the affine map S -> M_g S + B_g of its chunks; slices 0-3
-//   carry B_g (state from zero), slices 4-7 carry M_g (state from the identity,
-//   Bm dropped); the result is written as a segment slot in the chunk-slot format
-//   (Mlr = -M_g, GamC = 0, Bm = B_g), no outputs; with a.trans_out set (one
-//   segment per sequence, the per-device step of context parallelism across
-//   GPUs) M_g and B_g are written there in fp32 instead;
+//   (pass 1, each segment's affine map, is map_walk_kernel's)
 // SEG = 2: segment g first folds segments 0 .. g-1 into the initial state through
 //   their slots, then walks its own chunks with outputs; the last segment writes
 //   the final state;
@@ -806,11 +801,10 @@ chain_kernel(const ChunkArgs a, const __grid_constant__ CUtensorMap gate_map, co
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const bool consumer = warp < 4;
     const int js = blockIdx.x, h = blockIdx.y;
-    const int n = (SEG == 1 || SEG == 2) ? (int)blockIdx.z / a.segs : (int)blockIdx.z;
-    const int g = (SEG == 1 || SEG == 2) ? (int)blockIdx.z % a.segs : 0;
+    const int n = SEG == 2 ? (int)blockIdx.z / a.segs : (int)blockIdx.z;
+    const int g = SEG == 2 ? (int)blockIdx.z % a.segs : 0;
     const int H = a.H;
     const int jb = js & (NSL - 1);                // value slice of Bm / outputs
-    const bool trans = SEG == 1 && js >= NSL;     // carries M_g (identity start, no Bm)
     uint64_t* bar_ld = reinterpret_cast<uint64_t*>(sm + LY::BAR);         // [NBUF]
     uint64_t* bar_free = reinterpret_cast<uint64_t*>(sm + LY::BAR + 24);  // [NBUF]
     uint64_t* bar_s = reinterpret_cast<uint64_t*>(sm + LY::BAR + 48);
@@ -841,11 +835,8 @@ chain_kernel(const ChunkArgs a, const __grid_constant__ CUtensorMap gate_map, co
     const size_t st_off = (((size_t)n * H + h) * DK + (consumer ? tid : 0)) * DV + (size_t)DVS * jb;
     float S[DVS];
     if (consumer) {
-        const float* src = SEG == 1 ? nullptr : (a.first_pass ? a.init_state : a.state_io);
-        if (trans) {
-#pragma unroll
-            for (int j = 0; j < DVS; ++j) S[j] = (tid == DVS * jb + j) ? 1.f : 0.f;
-        } else if (src) {
+        const float* src = a.first_pass ? a.init_state : a.state_io;
+        if (src) {
 #pragma unroll
             for (int j = 0; j < DVS; j += 4) {
                 const float4 v4 = *reinterpret_cast<const float4*>(src + st_off + j);
@@ -1084,8 +1075,8 @@ chain_kernel(const ChunkArgs a, const __grid_constant__ CUtensorMap gate_map, co
 #pragma unroll
                         for (int p = 0; p < 4; ++p) {
                             const int j = 8 * m + 2 * p;
-                            const float b0 = trans ? 0.f : __uint_as_float(ww[p] << 16);
-                            const float b1 = trans ? 0.f : __uint_as_float(ww[p] & 0xFFFF0000u);
+                            const float b0 = __uint_as_float(ww[p] << 16);
+                            const float b1 = __uint_as_float(ww[p] & 0xFFFF0000u);
                             S[j] = gamC * S[j] - ds[j] + b0;
                             S[j + 1] = gamC * S[j + 1] - ds[j + 1] + b1;
                         }
@@ -1202,40 +1193,217 @@ chain_kernel(const ChunkArgs a, const __grid_constant__ CUtensorMap gate_map, co
         if constexpr (GATE) cluster_sync_all();  // no CTA leaves while a peer may still write to it
     }
 
-    if constexpr (SEG == 1) {
-        if (consumer && a.trans_out) {
-            // row tid, columns [32 jb, 32 jb + 32) of M_g (first half) or B_g (second half)
-            float* dst = a.trans_out + (trans ? 0 : (size_t)a.n_seqs * H * DK * DV) + st_off;
+    // the carried / final state slice (with segments: the last segment's)
+    if (consumer && (SEG != 2 || g == a.segs - 1)) {
 #pragma unroll
-            for (int j = 0; j < DVS; j += 4)
-                *reinterpret_cast<float4*>(dst + j) = make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]);
-        } else if (consumer) {
-            // this segment's slot: B_g as the Bm slice jb, -M_g as the Mlr image (rows c,
-            // K columns [32 jb, 32 jb + 32)), GamC = 0
-            uint8_t* slot = a.seg_ws + (((size_t)n * a.segs + g) * H + h) * SLOT_BYTES;
-            if (!trans) {
-                uint4* dst = reinterpret_cast<uint4*>(slot + SO_B + (size_t)jb * BSL + (size_t)tid * DVS * 2);
+        for (int j = 0; j < DVS; j += 4)
+            *reinterpret_cast<float4*>(a.state_io + st_off + j) = make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// map_walk_kernel
+// ---------------------------------------------------------------------------
+// The affine map S -> M_g S + B_g of a segment of whole chunks (segment-parallel
+// prefill, pass 1; the per-device step of context parallelism across devices): one CTA
+// per (sequence and segment, head, 32-column slice jb) carries both the slice of B_g
+// (the state walked from zero, with B_m) and the slice of M_g (the identity walked
+// without B_m), so the chunk's one tensor-core product M_lr [S_B | S_M] has N = 64 and a
+// head needs four CTAs.  Roles as in chain_kernel: warps 0-3 own one row each of both
+// slices (64 fp32 registers), warp 4 issues the products, warp 5 bulk-loads each chunk's
+// M_lr image, Gamma_C and B_m slice three chunks ahead.
+constexpr uint32_t MW_M = 0, MW_G = 32768, MW_B = 33280;         // one chunk buffer
+constexpr uint32_t MW_BUF = 41984;                               // 1024-aligned stride
+constexpr uint32_t MW_IMG = NBUF * MW_BUF;                       // [S_B | S_M] bf16 image, 16 KB
+constexpr uint32_t MW_BAR = MW_IMG + 16384;
+constexpr uint32_t MW_TMEMP = MW_BAR + 128;
+constexpr uint32_t MW_SMEM = MW_TMEMP + 16 + 1024;
+constexpr uint32_t MW_KG = 2 * DVS * 16;  // image K-group (8 key rows) stride: 64 columns x 2 B x 8 rows
+
+__global__ void __launch_bounds__(CHAIN_THREADS, 1) map_walk_kernel(const ChunkArgs a) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    const uint32_t sbase = smem_u32(sm);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const bool consumer = warp < 4;
+    const int jb = blockIdx.x, h = blockIdx.y;
+    const int n = (int)blockIdx.z / a.segs, g = (int)blockIdx.z % a.segs;
+    const int H = a.H;
+    uint64_t* bar_ld = reinterpret_cast<uint64_t*>(sm + MW_BAR);         // [NBUF]
+    uint64_t* bar_free = reinterpret_cast<uint64_t*>(sm + MW_BAR + 24);  // [NBUF]
+    uint64_t* bar_s = reinterpret_cast<uint64_t*>(sm + MW_BAR + 48);
+    uint64_t* bar_img = reinterpret_cast<uint64_t*>(sm + MW_BAR + 56);
+    uint32_t* s_tmem = reinterpret_cast<uint32_t*>(sm + MW_TMEMP);
+
+    int64_t s_beg, s_end;
+    seq_range(a, n, s_beg, s_end);
+    const int nchunks = (int)((s_end - s_beg + CH - 1) / CH);
+    const int per = (nchunks + a.segs - 1) / a.segs;
+    const int c_beg = min(g * per, nchunks), c_end = min(c_beg + per, nchunks);
+    const int nit = c_end > c_beg ? c_end - c_beg : 0;
+
+    // row tid: SB = columns [32 jb, +32) of B_g (from zero), SM = the same columns of M_g (from I)
+    float SB[DVS], SM[DVS];
 #pragma unroll
-                for (int m = 0; m < DVS / 8; ++m) dst[swz64(tid, m)] = pack8(S + 8 * m);
-            } else {
-                float nS[DVS];
+    for (int j = 0; j < DVS; ++j) {
+        SB[j] = 0.f;
+        SM[j] = (consumer && tid == DVS * jb + j) ? 1.f : 0.f;
+    }
+    if (nit > 0) {
+        if (warp == 0) {
+            tmem_alloc(s_tmem, 64);
+            tmem_relinquish();
+        }
+        if (tid == 0) {
+            for (int i = 0; i < NBUF; ++i) {
+                mbar_init(&bar_ld[i], 1);
+                mbar_init(&bar_free[i], 128);
+            }
+            mbar_init(bar_s, 1);
+            mbar_init(bar_img, 128);
+            fence_mbar_init();
+        }
+        __syncthreads();
+        tc_fence_after();
+        const uint32_t tm = *s_tmem;
+        const size_t slot0 = ((size_t)n * a.wc + (c_beg - a.i0)) * H + h;
+        auto slot_of = [&](int it) -> const uint8_t* { return a.ws + (slot0 + (size_t)it * H) * SLOT_BYTES; };
+        auto bidx = [](int it) { return it % NBUF; };
+        auto bpar = [](int it) { return (uint32_t)((it / NBUF) & 1); };
+        bool failed = false;
+        int loads_issued = 0, mma_issued = 0;
+
+        if (warp == 5) {
+            if (lane == 0) {
+                auto issue_load = [&](int it) {
+                    const int b = bidx(it);
+                    uint8_t* buf = sm + b * MW_BUF;
+                    const uint8_t* src = slot_of(it);
+                    mbar_arrive_expect_tx(&bar_ld[b], 32768u + 512u + BSL);
+                    bulk_g2s(buf + MW_M, src + SO_M, 32768u, &bar_ld[b]);
+                    bulk_g2s(buf + MW_G, src + SO_G, 512u, &bar_ld[b]);
+                    bulk_g2s(buf + MW_B, src + SO_B + (size_t)jb * BSL, BSL, &bar_ld[b]);
+                };
+                for (int j = 0; j < NBUF && j < nit; ++j) {
+                    issue_load(j);
+                    loads_issued = j + 1;
+                }
+                for (int j = 0; j + NBUF < nit; ++j) {
+                    if (!mbar_wait(&bar_free[bidx(j)], bpar(j), a.status)) {
+                        failed = true;
+                        break;
+                    }
+                    issue_load(j + NBUF);
+                    loads_issued = j + NBUF + 1;
+                }
+            }
+        } else if (warp == 4) {
+            if (lane == 0) {
+                const uint32_t idesc = idesc_bf16_major(128, 2 * DVS, 0, 1);
+                for (int it = 0; it < nit; ++it) {
+                    const int b = bidx(it);
+                    if (!mbar_wait(bar_img, (uint32_t)(it & 1), a.status) ||
+                        !mbar_wait(&bar_ld[b], bpar(it), a.status)) {
+                        failed = true;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint64_t sdesc = sdesc_interleave(sbase + MW_IMG, MW_KG, 128u);
+                    const uint64_t mdesc = sdesc_k_sw128(sbase + b * MW_BUF + MW_M);
 #pragma unroll
-                for (int j = 0; j < DVS; ++j) nS[j] = -S[j];
-                const uint32_t k0 = (uint32_t)(DVS * jb);
-                uint8_t* img = slot + SO_M + (size_t)(k0 >> 6) * (DK * 128);
+                    for (int kk = 0; kk < DK / 16; ++kk)
+                        mma_bf16(tm, mdesc + (uint32_t)(((kk >> 2) * 128 * 128 + (kk & 3) * 32) >> 4),
+                                 sdesc + (uint32_t)((kk * 2 * MW_KG) >> 4), idesc, kk > 0 ? 1u : 0u);
+                    mma_commit(bar_s);
+                    mma_issued = it + 1;
+                }
+            }
+        } else {
+            const uint32_t lane_addr = tm + ((uint32_t)(32 * warp) << 16);
+            // [S_B | S_M] as the bf16 B operand: MN-major without swizzle, key row tid's 64
+            // columns as eight 16-byte pieces, one per 8-column block
+            auto write_image = [&]() {
+                uint8_t* img = sm + MW_IMG + ((uint32_t)tid >> 3) * MW_KG + ((uint32_t)tid & 7u) * 16u;
 #pragma unroll
-                for (int m = 0; m < DVS / 8; ++m)
-                    *reinterpret_cast<uint4*>(img + sw128_off((uint32_t)tid, (k0 & 63u) + 8u * m)) = pack8(nS + 8 * m);
-                if (jb == 0) *reinterpret_cast<float*>(slot + SO_G + 4 * tid) = 0.f;
+                for (int nb = 0; nb < DVS / 8; ++nb) {
+                    *reinterpret_cast<uint4*>(img + nb * 128) = pack8(SB + 8 * nb);
+                    *reinterpret_cast<uint4*>(img + (DVS / 8 + nb) * 128) = pack8(SM + 8 * nb);
+                }
+                fence_async_smem();
+                tc_fence_before();
+                mbar_arrive(bar_img);
+            };
+            write_image();
+            for (int it = 0; it < nit; ++it) {
+                const int b = bidx(it);
+                const uint8_t* buf = sm + b * MW_BUF;
+                if (!mbar_wait(bar_s, (uint32_t)(it & 1), a.status) || !mbar_wait(&bar_ld[b], bpar(it), a.status)) {
+                    failed = true;
+                    break;
+                }
+                tc_fence_after();
+                float d[DVS];
+                const float gamC = *reinterpret_cast<const float*>(buf + MW_G + 4 * tid);
+                tmem_ld32(lane_addr + 0, d);
+                tmem_ld_wait();
+                const uint4* bsrc = reinterpret_cast<const uint4*>(buf + MW_B + (uint32_t)tid * DVS * 2);
+#pragma unroll
+                for (int m = 0; m < DVS / 8; ++m) {
+                    const uint4 w = bsrc[swz64(tid, m)];
+                    const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                    for (int p = 0; p < 4; ++p) {
+                        const int j = 8 * m + 2 * p;
+                        SB[j] = gamC * SB[j] - d[j] + __uint_as_float(ww[p] << 16);
+                        SB[j + 1] = gamC * SB[j + 1] - d[j + 1] + __uint_as_float(ww[p] & 0xFFFF0000u);
+                    }
+                }
+                tmem_ld32(lane_addr + DVS, d);
+                tmem_ld_wait();
+#pragma unroll
+                for (int j = 0; j < DVS; ++j) SM[j] = gamC * SM[j] - d[j];
+                mbar_arrive(&bar_free[b]);
+                if (it + 1 < nit) write_image();
             }
         }
-    } else {
-        // the carried / final state slice (with segments: the last segment's)
-        if (consumer && (SEG != 2 || g == a.segs - 1)) {
-#pragma unroll
-            for (int j = 0; j < DVS; j += 4)
-                *reinterpret_cast<float4*>(a.state_io + st_off + j) = make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]);
+        __syncthreads();
+        if (warp == 5 && lane == 0) {
+            for (int j = loads_issued - NBUF < 0 ? 0 : loads_issued - NBUF; j < loads_issued; ++j)
+                mbar_wait(&bar_ld[bidx(j)], bpar(j), nullptr);
         }
+        if (warp == 4 && lane == 0 && failed && mma_issued > 0) mbar_wait(bar_s, (uint32_t)((mma_issued - 1) & 1), nullptr);
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+        if (warp == 0) tmem_dealloc(tm, 64);
+    }
+    if (!consumer) return;
+    const size_t st_off = (((size_t)n * H + h) * DK + tid) * DV + (size_t)DVS * jb;
+    if (a.trans_out) {
+        // row tid, columns [32 jb, 32 jb + 32) of M_g (first half of the output) and B_g
+        float* dm = a.trans_out + st_off;
+        float* db = a.trans_out + (size_t)a.n_seqs * H * DK * DV + st_off;
+#pragma unroll
+        for (int j = 0; j < DVS; j += 4) {
+            *reinterpret_cast<float4*>(dm + j) = make_float4(SM[j], SM[j + 1], SM[j + 2], SM[j + 3]);
+            *reinterpret_cast<float4*>(db + j) = make_float4(SB[j], SB[j + 1], SB[j + 2], SB[j + 3]);
+        }
+    } else {
+        // this segment's slot: B_g as the Bm slice jb, -M_g as the Mlr image (rows tid, K columns
+        // [32 jb, 32 jb + 32)), GamC = 0
+        uint8_t* slot = a.seg_ws + (((size_t)n * a.segs + g) * H + h) * SLOT_BYTES;
+        uint4* dst = reinterpret_cast<uint4*>(slot + SO_B + (size_t)jb * BSL + (size_t)tid * DVS * 2);
+#pragma unroll
+        for (int m = 0; m < DVS / 8; ++m) dst[swz64(tid, m)] = pack8(SB + 8 * m);
+        float nS[DVS];
+#pragma unroll
+        for (int j = 0; j < DVS; ++j) nS[j] = -SM[j];
+        const uint32_t k0 = (uint32_t)(DVS * jb);
+        uint8_t* img = slot + SO_M + (size_t)(k0 >> 6) * (DK * 128);
+#pragma unroll
+        for (int m = 0; m < DVS / 8; ++m)
+            *reinterpret_cast<uint4*>(img + sw128_off((uint32_t)tid, (k0 & 63u) + 8u * m)) = pack8(nS + 8 * m);
+        if (jb == 0) *reinterpret_cast<float*>(slot + SO_G + 4 * tid) = 0.f;
     }
 }
 
@@ -1361,11 +1529,11 @@ cudaError_t chunk_fwd_launch(const void* q, const void* k, const void* v, const 
         if (err != cudaSuccess) return err;
         if ((err = set_chain_smem<true, false, 0>()) != cudaSuccess || (err = set_chain_smem<false, false, 0>()) != cudaSuccess ||
             (err = set_chain_smem<true, true, 0>()) != cudaSuccess || (err = set_chain_smem<false, true, 0>()) != cudaSuccess ||
-            (err = set_chain_smem<true, false, 1>()) != cudaSuccess || (err = set_chain_smem<false, false, 1>()) != cudaSuccess ||
-            (err = set_chain_smem<true, true, 1>()) != cudaSuccess || (err = set_chain_smem<false, true, 1>()) != cudaSuccess ||
             (err = set_chain_smem<true, false, 2>()) != cudaSuccess || (err = set_chain_smem<false, false, 2>()) != cudaSuccess ||
             (err = set_chain_smem<true, true, 2>()) != cudaSuccess || (err = set_chain_smem<false, true, 2>()) != cudaSuccess ||
-            (err = set_chain_smem<false, false, 3>()) != cudaSuccess)
+            (err = set_chain_smem<false, false, 3>()) != cudaSuccess ||
+            (err = cudaFuncSetAttribute(map_walk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)MW_SMEM)) !=
+                cudaSuccess)
             return err;
         int dev = 0;
         if ((err = cudaGetDevice(&dev)) != cudaSuccess) return err;
@@ -1465,14 +1633,16 @@ cudaError_t chunk_fwd_launch(const void* q, const void* k, const void* v, const 
             err = launch_chain<3>(a, gate_map, norm_w, eps, false, false, dim3(NSL, H, N), stream);
         } else if (kcp_mode == KCP_TRANSITION) {
             // M_g and B_g of the whole local sequence (one segment), fp32, no outputs
-            err = launch_chain<1>(a, gate_map, norm_w, eps, out_bf16, false, dim3(2 * NSL, H, N), stream);
+            map_walk_kernel<<<dim3(NSL, H, N), CHAIN_THREADS, MW_SMEM, stream>>>(a);
+            err = cudaGetLastError();
         } else if (a.segs == 1) {
             err = launch_chain<0>(a, gate_map, norm_w, eps, out_bf16, fuse, dim3(NSL, H, N), stream);
         } else {
             // segment transitions (no outputs, no gate), then the segments with outputs
             ChunkArgs at = a;
             at.ckpt = nullptr;
-            err = launch_chain<1>(at, gate_map, norm_w, eps, out_bf16, false, dim3(2 * NSL, H, N * a.segs), stream);
+            map_walk_kernel<<<dim3(NSL, H, N * a.segs), CHAIN_THREADS, MW_SMEM, stream>>>(at);
+            err = cudaGetLastError();
             if (err == cudaSuccess)
                 err = launch_chain<2>(a, gate_map, norm_w, eps, out_bf16, fuse, dim3(NSL, H, N * a.segs), stream);
         }
