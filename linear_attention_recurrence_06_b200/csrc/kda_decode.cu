@@ -167,6 +167,18 @@ decode_step_kernel(float* __restrict__ state, const void* __restrict__ q, const 
 // four at a time (16-byte shared loads), and the column sums need one 4-lane reduction.
 // Per step and column: S' = alpha o S;  u = beta (v - S'^T k);  o = scale (S'^T q + (k.q) u);
 // S = S' + k u^T, the same arithmetic whatever the number of steps per call.
+// The token rows of up to DECODE_BLOCK steps (k, q, log_alpha and the CTA's half of v)
+// arrive together by asynchronous copies into shared memory, the first block's in the
+// shadow of the state load: a step then waits for no global load (a step is shorter than
+// the latency of one under a full HBM load).
+constexpr int DECODE_BLOCK = 8;
+
+KDA_DEV void cp_async16(void* smem_dst, const void* gmem_src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)), "l"(gmem_src) : "memory");
+}
+KDA_DEV void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+KDA_DEV void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+
 template <bool IN_BF16, bool OUT_BF16>
 __global__ void __launch_bounds__(128, 4)
 decode_multi_kernel(float* __restrict__ state, const void* __restrict__ q, const void* __restrict__ k,
@@ -185,34 +197,60 @@ decode_multi_kernel(float* __restrict__ state, const void* __restrict__ q, const
     __shared__ __align__(16) float s_k[2][DP], s_q[2][DP], s_alpha[2][DP];
     const int pr = tid + 4 * (tid >> 5);   // padded slot of row tid
     const int prow0 = row0 + 4 * rb;       // padded slot of this thread's first row
+    // a block of steps' raw token rows: per step [k | q | log_alpha] rows of 128 elements and
+    // this CTA's 64 elements of v, then beta per step
+    constexpr int ES = IN_BF16 ? 2 : 4;
+    constexpr int ROWB = D * ES, VB = 64 * ES, STEPB = 3 * ROWB + VB;
+    __shared__ __align__(16) uint8_t s_tok[DECODE_BLOCK * STEPB];
+    __shared__ float s_beta[DECODE_BLOCK];
+    auto tok = [&](int s_, int part, int e) -> float {  // element e of part (0 k, 1 q, 2 log_alpha, 3 v)
+        const uint8_t* p = s_tok + s_ * STEPB + part * ROWB + e * ES;
+        if constexpr (IN_BF16) return __uint_as_float((uint32_t)*reinterpret_cast<const uint16_t*>(p) << 16);
+        else return *reinterpret_cast<const float*>(p);
+    };
+    // copies of steps [t0, t0 + nb): 16-byte pieces, CHUNK_ROW per row, CHUNK_V for v
+    auto fetch_block = [&](int t0) {
+        const int nb = n_steps - t0 < DECODE_BLOCK ? n_steps - t0 : DECODE_BLOCK;
+        constexpr int CR = ROWB / 16, CV = VB / 16, CS = 3 * CR + CV;
+        for (int ci = tid; ci < nb * CS; ci += 128) {
+            const int s_ = ci / CS, r = ci - s_ * CS;
+            const size_t tb = (size_t)(t0 + s_) * BH + bh;
+            const uint8_t* src;
+            if (r < 3 * CR) {
+                const int part = r / CR;
+                const void* base = part == 0 ? k : (part == 1 ? q : log_alpha);
+                src = reinterpret_cast<const uint8_t*>(base) + tb * ROWB + (size_t)(r - part * CR) * 16;
+            } else {
+                src = reinterpret_cast<const uint8_t*>(v) + tb * ROWB + (size_t)sl * VB + (size_t)(r - 3 * CR) * 16;
+            }
+            cp_async16(s_tok + s_ * STEPB + r * 16, src);
+        }
+        cp_async_commit();
+        // beta of step t0 + tid: kept in a register until the block's wait
+        return tid < nb ? ld_in<IN_BF16>(beta, (size_t)(t0 + tid) * BH + bh) : 0.f;
+    };
+    float beta_next = fetch_block(0);  // in flight with the state load
 
     float* S = state + (size_t)bh * D * D;
     float2 st[32];
 #pragma unroll
     for (int i = 0; i < 32; ++i) st[i] = __ldcs(reinterpret_cast<const float2*>(S + (size_t)(row0 + i) * D + col));
 
-    // this step's token values, loaded one step ahead into registers
-    float nk, nq, nla, nb, nv[2];
-    auto load_step = [&](int t) {
-        const size_t tb = (size_t)t * BH + bh;
-        const size_t idx = tb * D + tid;
-        nk = ld_in<IN_BF16>(k, idx);
-        nq = ld_in<IN_BF16>(q, idx);
-        nla = ld_in<IN_BF16>(log_alpha, idx);
-        nb = ld_in<IN_BF16>(beta, tb);
-        nv[0] = ld_in<IN_BF16>(v, tb * D + col);
-        nv[1] = ld_in<IN_BF16>(v, tb * D + col + 1);
-    };
-    load_step(0);
-
+    const int vc = col - 64 * sl;  // this thread's v columns within the CTA's half
     for (int t = 0; t < n_steps; ++t) {
         const int pb = t & 1;
         const size_t tb = (size_t)t * BH + bh;
-        s_k[pb][pr] = nk;
-        s_q[pb][pr] = nq;
-        s_alpha[pb][pr] = __expf(fmaxf(nla, LOG_ALPHA_FLOOR));
-        const float b = nb, v0 = nv[0], v1 = nv[1];
-        if (t + 1 < n_steps) load_step(t + 1);  // in flight during this step
+        const int s_ = t % DECODE_BLOCK;
+        if (s_ == 0) {
+            if (t > 0) beta_next = fetch_block(t);  // every thread is past the last step's barrier: s_tok is free
+            if (tid < DECODE_BLOCK) s_beta[tid] = beta_next;
+            cp_async_wait_all();
+            __syncthreads();
+        }
+        s_k[pb][pr] = tok(s_, 0, tid);
+        s_q[pb][pr] = tok(s_, 1, tid);
+        s_alpha[pb][pr] = __expf(fmaxf(tok(s_, 2, tid), LOG_ALPHA_FLOOR));
+        const float b = s_beta[s_], v0 = tok(s_, 3, vc), v1 = tok(s_, 3, vc + 1);
         __syncthreads();
         const float* sk_ = s_k[pb];
         const float* sq_ = s_q[pb];
