@@ -454,10 +454,12 @@ def test_decode_steps(bf16, gate, scale):
 
 @pytest.mark.parametrize("bf16,gate,n,scale", [(True, False, 1, 1.0), (True, False, 4, 1.0), (True, True, 8, 1.0),
                                                (False, False, 3, 1.0), (True, False, 4, 128 ** -0.5),
-                                               (False, True, 3, 0.125)])
+                                               (False, True, 3, 0.125), (True, False, 17, 1.0),
+                                               (False, False, 11, 128 ** -0.5)])
 def test_decode_multi_step_with_step_states(bf16, gate, n, scale):
     """n consecutive steps in one call == n single steps of the oracle: every
-    step's output, every step's state (for rollback) and the carried state."""
+    step's output, every step's state (for rollback) and the carried state.
+    n = 11 and 17 cross the kernel's blocks of 8 staged token steps."""
     torch = _torch()
     import linear_attention_recurrence_06_b200 as kda
     Bd, H = 5, 3
@@ -487,12 +489,14 @@ def test_decode_multi_step_with_step_states(bf16, gate, n, scale):
     np.testing.assert_array_equal(host(s_dev), host(states[n - 1]))  # the carried state is the last step's
 
 
-def test_decode_multi_step_matches_single_steps_exactly():
-    """Carrying the state through 4 steps in registers gives the same bits as 4
-    separate one-step calls (same arithmetic, same order)."""
+@pytest.mark.parametrize("n", [4, 10])
+def test_decode_multi_step_matches_single_steps_exactly(n):
+    """Carrying the state through n steps in registers gives the same bits as n
+    separate one-step calls (same arithmetic, same order; n = 10 crosses a block
+    of 8 staged token steps)."""
     torch = _torch()
     import linear_attention_recurrence_06_b200 as kda
-    Bd, H, n = 4, 2, 4
+    Bd, H = 4, 2
     s0 = synth.states(8, Bd, H, D, D)
     toks = [synth.tokens(8, step * Bd, Bd, H, D, D, bf16=True) for step in range(n)]
     stack = lambda name: dev(np.stack([getattr(tb, name) for tb in toks]), torch.bfloat16)
