@@ -14,10 +14,11 @@
 namespace kda {
 
 // One CTA = one (sequence, head) state [128 x 128] fp32 = 64 KiB, carried
-// through n_steps consecutive tokens (speculative-decode verification of n
-// draft tokens, or plain decode with n_steps = 1): the state is read once and
-// written once for all of them, and optionally also after every step so that
-// a caller can roll back to any accepted prefix.
+// through n_steps consecutive tokens; the state is read once and written once
+// for all of them, and optionally also after every step.  The launcher uses it
+// for single steps with the output gate fused (GATE: the per-head RMSNorm needs
+// all 128 value columns of the head in one CTA); ungated steps and several steps
+// per call go to decode_multi_kernel below.
 // 256 threads = 8 warps; warp w owns value columns [16w, 16w + 16).
 // Lane l: row phase r0 = l / 4 (0..7) and column quad cq = l % 4, so one warp
 // load instruction covers 8 rows x 64 contiguous bytes.  Thread holds rows
