@@ -487,7 +487,7 @@ intra_kernel(const ChunkArgs a, const __grid_constant__ IntraMaps maps, const in
             }
             if (tid < CH) load_beta(tt, hh, LL);
         }
-        mbar_wait(bar_mma, ph_mma, a.status);
+        mbar_wait_spin(bar_mma, ph_mma, a.status);
         ph_mma ^= 1;
         tc_fence_after();
 
@@ -589,7 +589,7 @@ intra_kernel(const ChunkArgs a, const __grid_constant__ IntraMaps maps, const in
             mma_sw128<4, 128, 64>(tm + TM_UT, sdesc_k_sw128(sb + Z2_VT), sdesc_k_sw128(sb + IX_TI), idesc_bf16(128, 64));
             mma_commit(bar_mma);
         }
-        mbar_wait(bar_mma, ph_mma, a.status);
+        mbar_wait_spin(bar_mma, ph_mma, a.status);
         ph_mma ^= 1;
         tc_fence_after();
         {
@@ -624,7 +624,7 @@ intra_kernel(const ChunkArgs a, const __grid_constant__ IntraMaps maps, const in
         // The slot is assembled in two shared-memory pieces that match its layout:
         // [Mlr | Qp | GamC] at IX (KQr/KC/Ti are dead) and [Bm | Ob] at Z2 (dead once
         // the first product is done); each leaves by one bulk copy.
-        mbar_wait(bar_mma, ph_mma, a.status);
+        mbar_wait_spin(bar_mma, ph_mma, a.status);
         ph_mma ^= 1;
         tc_fence_after();
         {
@@ -667,7 +667,7 @@ intra_kernel(const ChunkArgs a, const __grid_constant__ IntraMaps maps, const in
             bulk_s2g(wslot + SO_B, sm + Z2, (uint32_t)(SO_O - SO_B));
             bulk_commit();
         }
-        mbar_wait(bar_mma2, ph_mma2, a.status);
+        mbar_wait_spin(bar_mma2, ph_mma2, a.status);
         ph_mma2 ^= 1;
         tc_fence_after();
         {
@@ -929,8 +929,8 @@ chain_kernel(const ChunkArgs a, const __grid_constant__ CUtensorMap gate_map, co
             if (lane == 0) {
                 for (int it = 0; it < nit; ++it) {
                     const int b = bidx(it);
-                    if (!mbar_wait(bar_img, (uint32_t)(it & 1), a.status) ||
-                        !mbar_wait(&bar_ld[b], bpar(it), a.status)) {
+                    if (!mbar_wait_spin(bar_img, (uint32_t)(it & 1), a.status) ||
+                        !mbar_wait_spin(&bar_ld[b], bpar(it), a.status)) {
                         failed = true;
                         break;
                     }
@@ -1057,7 +1057,7 @@ chain_kernel(const ChunkArgs a, const __grid_constant__ CUtensorMap gate_map, co
                 const int L = (int)((s_end - t0) < CH ? (s_end - t0) : CH);
 
                 // (1) state update: S <- GamC o S - Mlr S + Bm
-                if (!mbar_wait(bar_s, (uint32_t)(it & 1), a.status) || !mbar_wait(&bar_ld[b], bpar(it), a.status)) {
+                if (!mbar_wait_spin(bar_s, (uint32_t)(it & 1), a.status) || !mbar_wait_spin(&bar_ld[b], bpar(it), a.status)) {
                     failed = true;
                     break;
                 }
@@ -1090,7 +1090,7 @@ chain_kernel(const ChunkArgs a, const __grid_constant__ CUtensorMap gate_map, co
                     continue;
                 }
                 // (3) this chunk's output: o = Qp S + Ob  (then y, when the gate is fused)
-                if (!mbar_wait(&bar_o[oi & 1], (uint32_t)((oi >> 1) & 1), a.status)) {
+                if (!mbar_wait_spin(&bar_o[oi & 1], (uint32_t)((oi >> 1) & 1), a.status)) {
                     failed = true;
                     break;
                 }
@@ -1302,8 +1302,8 @@ __global__ void __launch_bounds__(CHAIN_THREADS, 1) map_walk_kernel(const ChunkA
                 const uint32_t idesc = idesc_bf16_major(128, 2 * DVS, 0, 1);
                 for (int it = 0; it < nit; ++it) {
                     const int b = bidx(it);
-                    if (!mbar_wait(bar_img, (uint32_t)(it & 1), a.status) ||
-                        !mbar_wait(&bar_ld[b], bpar(it), a.status)) {
+                    if (!mbar_wait_spin(bar_img, (uint32_t)(it & 1), a.status) ||
+                        !mbar_wait_spin(&bar_ld[b], bpar(it), a.status)) {
                         failed = true;
                         break;
                     }
@@ -1337,7 +1337,7 @@ __global__ void __launch_bounds__(CHAIN_THREADS, 1) map_walk_kernel(const ChunkA
             for (int it = 0; it < nit; ++it) {
                 const int b = bidx(it);
                 const uint8_t* buf = sm + b * MW_BUF;
-                if (!mbar_wait(bar_s, (uint32_t)(it & 1), a.status) || !mbar_wait(&bar_ld[b], bpar(it), a.status)) {
+                if (!mbar_wait_spin(bar_s, (uint32_t)(it & 1), a.status) || !mbar_wait_spin(&bar_ld[b], bpar(it), a.status)) {
                     failed = true;
                     break;
                 }

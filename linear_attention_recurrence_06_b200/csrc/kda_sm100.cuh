@@ -84,6 +84,34 @@ KDA_DEV bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t* status,
     }
 }
 
+// Same bound, but polling with mbarrier.test_wait instead of letting the hardware
+// suspend the thread: a suspended waiter resumes some 100-200 cycles after the
+// phase completes, which matters on a critical path of short waits (a CTA's own
+// tensor-core products); use it where the waiting warps have nothing else to issue.
+KDA_DEV bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+KDA_DEV bool mbar_wait_spin(uint64_t* bar, uint32_t parity, uint32_t* status,
+                            unsigned long long limit_ns = WAIT_LIMIT_NS) {
+    if (mbar_test_wait(bar, parity)) return true;
+    const unsigned long long t0 = globaltimer_ns();
+    for (uint32_t n = 1;; ++n) {
+        if (mbar_test_wait(bar, parity)) return true;
+        if ((n & 255u) == 0 && globaltimer_ns() - t0 > limit_ns) {
+            if (status) atomicOr(status, DEV_ERR_TIMEOUT);
+            return false;
+        }
+    }
+}
+
 // ------------------------------------------------- bulk copies (TMA engine) --
 // 1-D bulk copy global -> shared, completion signalled on `bar` (tx bytes).
 // Both addresses 16-byte aligned, bytes a multiple of 16.
