@@ -174,17 +174,18 @@ KDA_DEV void st_async_f32(uint32_t cluster_addr, float v, uint32_t cluster_bar_a
                  "f"(v), "r"(cluster_bar_addr)
                  : "memory");
 }
-// Waits with acquire at cluster scope (bounded like mbar_wait).
+// Waits with acquire at cluster scope, polling (test_wait: the peers' partial sums are
+// on the chain's critical path), bounded like mbar_wait.
 KDA_DEV bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, uint32_t* status) {
     const unsigned long long t0 = globaltimer_ns();
     while (true) {
         uint32_t ok;
         asm volatile(
             "{\n\t.reg .pred p;\n\t"
-            "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3;\n\t"
+            "mbarrier.test_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
             "selp.u32 %0, 1, 0, p;\n\t}"
             : "=r"(ok)
-            : "r"(smem_u32(bar)), "r"(parity), "r"(1000000u)
+            : "r"(smem_u32(bar)), "r"(parity)
             : "memory");
         if (ok) return true;
         if (globaltimer_ns() - t0 > WAIT_LIMIT_NS) {
