@@ -170,8 +170,10 @@ decode_step_kernel(float* __restrict__ state, const void* __restrict__ q, const 
 // S = S' + k u^T, the same arithmetic whatever the number of steps per call.
 // The token rows of up to DECODE_BLOCK steps (k, q, log_alpha and the CTA's half of v)
 // arrive together by asynchronous copies into shared memory, the first block's in the
-// shadow of the state load: a step then waits for no global load (a step is shorter than
-// the latency of one under a full HBM load).
+// shadow of the state load, and are converted once per block into fp32 per-row vectors
+// (k, q, alpha = e^l) and v columns: the steps of a block then wait for no global load
+// (a step is shorter than the latency of one under a full HBM load) and for no barrier,
+// so the warps of a CTA run through them independently.
 constexpr int DECODE_BLOCK = 8;
 
 KDA_DEV void cp_async16(void* smem_dst, const void* gmem_src) {
@@ -195,7 +197,8 @@ decode_multi_kernel(float* __restrict__ state, const void* __restrict__ q, const
     // per-row token values, rows of block rb at offset 36 rb (4 floats of padding per block):
     // the four row blocks a warp reads at once fall into different banks
     constexpr int DP = D + 12;
-    __shared__ __align__(16) float s_k[2][DP], s_q[2][DP], s_alpha[2][DP];
+    __shared__ __align__(16) float s_k[DECODE_BLOCK][DP], s_q[DECODE_BLOCK][DP], s_alpha[DECODE_BLOCK][DP];
+    __shared__ float s_v[DECODE_BLOCK][64];
     const int pr = tid + 4 * (tid >> 5);   // padded slot of row tid
     const int prow0 = row0 + 4 * rb;       // padded slot of this thread's first row
     // a block of steps' raw token rows: per step [k | q | log_alpha] rows of 128 elements and
@@ -239,23 +242,28 @@ decode_multi_kernel(float* __restrict__ state, const void* __restrict__ q, const
 
     const int vc = col - 64 * sl;  // this thread's v columns within the CTA's half
     for (int t = 0; t < n_steps; ++t) {
-        const int pb = t & 1;
         const size_t tb = (size_t)t * BH + bh;
         const int s_ = t % DECODE_BLOCK;
         if (s_ == 0) {
-            if (t > 0) beta_next = fetch_block(t);  // every thread is past the last step's barrier: s_tok is free
-            if (tid < DECODE_BLOCK) s_beta[tid] = beta_next;
+            // s_tok was last read by the previous block's conversion, which every thread
+            // finished before that block's second barrier
+            if (t > 0) beta_next = fetch_block(t);
             cp_async_wait_all();
+            __syncthreads();  // the copies have landed; every thread is done with the last block's vectors
+            const int nb = n_steps - t < DECODE_BLOCK ? n_steps - t : DECODE_BLOCK;
+            for (int j = 0; j < nb; ++j) {
+                s_k[j][pr] = tok(j, 0, tid);
+                s_q[j][pr] = tok(j, 1, tid);
+                s_alpha[j][pr] = __expf(fmaxf(tok(j, 2, tid), LOG_ALPHA_FLOOR));
+                if (tid < 64) s_v[j][tid] = tok(j, 3, tid);
+            }
+            if (tid < DECODE_BLOCK) s_beta[tid] = beta_next;
             __syncthreads();
         }
-        s_k[pb][pr] = tok(s_, 0, tid);
-        s_q[pb][pr] = tok(s_, 1, tid);
-        s_alpha[pb][pr] = __expf(fmaxf(tok(s_, 2, tid), LOG_ALPHA_FLOOR));
-        const float b = s_beta[s_], v0 = tok(s_, 3, vc), v1 = tok(s_, 3, vc + 1);
-        __syncthreads();
-        const float* sk_ = s_k[pb];
-        const float* sq_ = s_q[pb];
-        const float* sa_ = s_alpha[pb];
+        const float b = s_beta[s_], v0 = s_v[s_][vc], v1 = s_v[s_][vc + 1];
+        const float* sk_ = s_k[s_];
+        const float* sq_ = s_q[s_];
+        const float* sa_ = s_alpha[s_];
 
         float kq = 0.f;
 #pragma unroll
