@@ -83,6 +83,8 @@ struct ChunkArgs {
     float* trans_out;          // nullable: fp32 segment maps [2][n_seqs][H][dk][dk] (M, then B) instead of slots
     unsigned long long wait_ns;  // limit of the intra kernel's tile-load wait (WAIT_LIMIT_NS unless a test shortens it)
     int drop_tile;             // test hook: CTA 0 does not issue one tile load of its first item (its wait runs out)
+    int state_from_prev;       // the initial state is written by the kernel ahead of the chain (the cross-device
+                               // fold): the chain waits for that kernel before reading it
 };
 
 // Token range [sb, se) of sequence n, clamped into [0, total tokens].
@@ -257,6 +259,9 @@ intra_kernel(const ChunkArgs a, const __grid_constant__ IntraMaps maps, const in
     }
     __syncthreads();
     tc_fence_after();
+    // the chain launch that follows may be scheduled now: its CTAs take SMs as this
+    // kernel's CTAs retire and wait (pdl_wait) for the whole of this kernel
+    pdl_trigger();
     const uint32_t tm = *s_tmem;
     const uint32_t lane_addr = tm + ((uint32_t)(32 * qd) << 16);
     uint32_t ph_raw = 0, ph_mma = 0, ph_mma2 = 0;
@@ -834,6 +839,7 @@ chain_kernel(const ChunkArgs a, const __grid_constant__ CUtensorMap gate_map, co
     // state slice: row tid, columns [32 jb, 32 jb + 32)
     const size_t st_off = (((size_t)n * H + h) * DK + (consumer ? tid : 0)) * DV + (size_t)DVS * jb;
     float S[DVS];
+    if (a.state_from_prev) pdl_wait();
     if (consumer) {
         const float* src = a.first_pass ? a.init_state : a.state_io;
         if (src) {
@@ -874,6 +880,7 @@ chain_kernel(const ChunkArgs a, const __grid_constant__ CUtensorMap gate_map, co
         __syncthreads();
         if constexpr (GATE) cluster_sync_all();  // peers' barriers exist before any remote store
         tc_fence_after();
+        pdl_wait();  // the slots (and segment slots) written by the kernel ahead of this one
         const uint32_t tm = *s_tmem;
         const size_t slot0 = ((size_t)n * a.wc + (c_beg - a.i0)) * H + h;  // slot of the first chunk iteration
         // iteration it: a segment iteration (it < nseg) or chunk c_beg + it - nseg;
@@ -1486,7 +1493,13 @@ static cudaError_t launch_chain(const ChunkArgs& a, const CUtensorMap& gate_map,
     cfg.gridDim = gc;
     cfg.blockDim = dim3(CHAIN_THREADS, 1, 1);
     cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
+    // programmatic serialisation: scheduled while the kernel ahead of it (the chunk-local
+    // kernel, or the segment-map walk) still runs; it waits for it before reading slots
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
     if (SEG == 3 || !fuse) {
         cfg.dynamicSmemBytes = ChainLayout<false>::SMEM;
         return out_bf16 ? cudaLaunchKernelEx(&cfg, chain_kernel<true, false, SEG>, a, gate_map, norm_w, eps)
@@ -1494,12 +1507,11 @@ static cudaError_t launch_chain(const ChunkArgs& a, const CUtensorMap& gate_map,
     }
     // the four value-column slices of one (sequence, head) form a cluster
     cfg.dynamicSmemBytes = ChainLayout<true>::SMEM;
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = CLUSTER;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = CLUSTER;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    cfg.numAttrs = 2;
     if constexpr (SEG == 3) return cudaErrorInvalidValue;  // no outputs, nothing to gate
     else
         return out_bf16 ? cudaLaunchKernelEx(&cfg, chain_kernel<true, true, SEG>, a, gate_map, norm_w, eps)
@@ -1579,6 +1591,7 @@ cudaError_t chunk_fwd_launch(const void* q, const void* k, const void* v, const 
     a.trans_out = kcp_mode == KCP_TRANSITION ? trans_out : nullptr;
     a.wait_ns = WAIT_LIMIT_NS;
     a.drop_tile = 0;
+    a.state_from_prev = kcp_mode == KCP_FINISH ? 1 : 0;
 
     IntraMaps maps;
     memset(&maps, 0, sizeof(maps));

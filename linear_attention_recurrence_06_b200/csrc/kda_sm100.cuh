@@ -112,6 +112,16 @@ KDA_DEV bool mbar_wait_spin(uint64_t* bar, uint32_t parity, uint32_t* status,
     }
 }
 
+// ------------------------------------------- programmatic dependent launch --
+// A kernel launched with programmatic stream serialisation may be scheduled before
+// the kernel ahead of it in the stream has finished; pdl_wait() returns once that
+// kernel has completed and its memory operations are visible, and must come before
+// anything that reads what it writes.  pdl_trigger() in the earlier kernel lets the
+// later one be scheduled as soon as every CTA has issued it (or exited).  Both are
+// no-ops when the launches are not paired this way.
+KDA_DEV void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+KDA_DEV void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ------------------------------------------------- bulk copies (TMA engine) --
 // 1-D bulk copy global -> shared, completion signalled on `bar` (tx bytes).
 // Both addresses 16-byte aligned, bytes a multiple of 16.
