@@ -83,8 +83,9 @@ struct ChunkArgs {
     float* trans_out;          // nullable: fp32 segment maps [2][n_seqs][H][dk][dk] (M, then B) instead of slots
     unsigned long long wait_ns;  // limit of the intra kernel's tile-load wait (WAIT_LIMIT_NS unless a test shortens it)
     int drop_tile;             // test hook: CTA 0 does not issue one tile load of its first item (its wait runs out)
-    int state_from_prev;       // the initial state is written by the kernel ahead of the chain (the cross-device
-                               // fold): the chain waits for that kernel before reading it
+    int wait_first;            // the kernel ahead of the chain may be the caller's (the cross-device finish,
+                               // whose initial state the fold wrote): the chain waits for it before reading
+                               // anything, not only before the slots
 };
 
 // Token range [sb, se) of sequence n, clamped into [0, total tokens].
@@ -800,6 +801,7 @@ chain_kernel(const ChunkArgs a, const __grid_constant__ CUtensorMap gate_map, co
              float eps) {
     using LY = ChainLayout<GATE>;
     constexpr uint32_t CB_SIZE = LY::CB_SIZE;
+    if (a.wait_first) pdl_wait();
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     const uint32_t sbase = smem_u32(sm);
@@ -839,7 +841,6 @@ chain_kernel(const ChunkArgs a, const __grid_constant__ CUtensorMap gate_map, co
     // state slice: row tid, columns [32 jb, 32 jb + 32)
     const size_t st_off = (((size_t)n * H + h) * DK + (consumer ? tid : 0)) * DV + (size_t)DVS * jb;
     float S[DVS];
-    if (a.state_from_prev) pdl_wait();
     if (consumer) {
         const float* src = a.first_pass ? a.init_state : a.state_io;
         if (src) {
@@ -1591,7 +1592,7 @@ cudaError_t chunk_fwd_launch(const void* q, const void* k, const void* v, const 
     a.trans_out = kcp_mode == KCP_TRANSITION ? trans_out : nullptr;
     a.wait_ns = WAIT_LIMIT_NS;
     a.drop_tile = 0;
-    a.state_from_prev = kcp_mode == KCP_FINISH ? 1 : 0;
+    a.wait_first = kcp_mode == KCP_FINISH ? 1 : 0;
 
     IntraMaps maps;
     memset(&maps, 0, sizeof(maps));
